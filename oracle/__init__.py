@@ -1,0 +1,194 @@
+"""CPU oracle of the Hybrid Linear Temporal Attention operator (fp64, plain definitions).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's
+``cpu_baseline`` / reference leg may import this package; the product package never does.
+The arithmetic lives in ``hlta_oracle.c`` (explicit masked softmax, token-by-token gated
+delta recurrence); this file only marshals numpy arrays and composes the branches.
+
+Branch composition (Kairos abstract, chatpaper.ai page, item (2); researchpapers.dev summary,
+"How hybrid linear temporal attention suppresses drift"): the heads are split into three
+groups, SWA | DSWA | GDN, each group runs its own branch, and the outputs are concatenated
+back on the head axis in the same order.
+
+Streaming (zhichai.net blog, section 2.3, the "streaming token" design: generate
+incrementally without waiting for the whole sequence): the oracle does not keep caches; the
+output of a step that appends frame f is, by definition, the last frame of the hybrid output
+over frames 0..f.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hlta_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (OpenMP, no fast-math) into oracle/liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", _LIB, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f32 = ctypes.POINTER(ctypes.c_float)
+        f64 = ctypes.POINTER(ctypes.c_double)
+        i64 = ctypes.POINTER(ctypes.c_long)
+        L_, I_, D_ = ctypes.c_long, ctypes.c_int, ctypes.c_double
+        lib.oracle_swa.argtypes = [f32, f32, f32, f64, L_, I_, I_, I_, I_, D_, i64, L_]
+        lib.oracle_dswa.argtypes = [f32, f32, f32, f64, L_, I_, I_, I_, I_, I_, D_, i64, L_]
+        lib.oracle_gdn.argtypes = [f32, f32, f32, f32, f32, f64, f64, f64, f64, L_, L_, I_]
+        for fn in (lib.oracle_swa, lib.oracle_dswa, lib.oracle_gdn):
+            fn.restype = ctypes.c_int
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f32(x) -> np.ndarray:
+    """Host float32 contiguous copy of a numpy array or torch tensor (bf16 is exact in f32)."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu", torch.float32).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _ptr(arr, ctype):
+    if arr is None:
+        return None
+    return arr.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _window(q, k, v, T, N, w, r, dilated, scale, rows):
+    qf, kf, vf = _f32(q), _f32(k), _f32(v)
+    d = qf.shape[-1]
+    L = T * N
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    assert qf.shape[-2] == L, "q must hold T*N rows"
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    lib = _load()
+    if rows is None:
+        o = np.empty(qf.shape, dtype=np.float64)
+        rp, nr = None, 0
+    else:
+        rr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        o = np.empty((rr.size, d), dtype=np.float64)
+        rp, nr = _ptr(rr, ctypes.c_long), rr.size
+    if dilated:
+        rc = lib.oracle_dswa(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                             _ptr(vf, ctypes.c_float), _ptr(o, ctypes.c_double),
+                             BH, T, N, d, w, r, float(scale), rp, nr)
+    else:
+        rc = lib.oracle_swa(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                            _ptr(vf, ctypes.c_float), _ptr(o, ctypes.c_double),
+                            BH, T, N, d, w, float(scale), rp, nr)
+    if rc != 0:
+        raise RuntimeError(f"oracle window attention failed ({rc})")
+    return o
+
+
+def swa(q, k, v, T: int, N: int, w: int, scale=None, rows=None) -> np.ndarray:
+    """Block-causal sliding-window attention over frames max(0,f-w+1)..f.
+
+    q, k, v: [..., L, d]. ``rows``: optional flat indices (head-major, bh*L + l) to compute
+    only those query rows; the result is then [len(rows), d]."""
+    return _window(q, k, v, T, N, w, 1, False, scale, rows)
+
+
+def dswa(q, k, v, T: int, N: int, w: int, r: int, scale=None, rows=None) -> np.ndarray:
+    """Dilated sliding-window attention over frames f, f-r, ..., f-r(w-1) (>= 0)."""
+    return _window(q, k, v, T, N, w, r, True, scale, rows)
+
+
+def gdn(q, k, v, a, b, S0=None, history: bool = False):
+    """Gated delta rule, token by token. q,k,v: [..., L, d]; a,b: [..., L].
+
+    Returns (o, S_final) and, with ``history``, also every S_t as [..., L, d, d]."""
+    qf, kf, vf, af, bf = _f32(q), _f32(k), _f32(v), _f32(a), _f32(b)
+    d = qf.shape[-1]
+    L = qf.shape[-2]
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    S0d = None
+    if S0 is not None:
+        if hasattr(S0, "detach"):
+            S0 = S0.detach().cpu().double().numpy()
+        S0d = np.ascontiguousarray(np.asarray(S0, dtype=np.float64)).reshape(BH, d, d)
+    o = np.empty(qf.shape, dtype=np.float64)
+    S_out = np.empty(lead + (d, d), dtype=np.float64)
+    hist = np.empty(lead + (L, d, d), dtype=np.float64) if history else None
+    rc = _load().oracle_gdn(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                            _ptr(vf, ctypes.c_float), _ptr(af, ctypes.c_float),
+                            _ptr(bf, ctypes.c_float), _ptr(S0d, ctypes.c_double),
+                            _ptr(o, ctypes.c_double), _ptr(S_out, ctypes.c_double),
+                            _ptr(hist, ctypes.c_double), BH, L, d)
+    if rc != 0:
+        raise RuntimeError(f"oracle gdn failed ({rc})")
+    return (o, S_out, hist) if history else (o, S_out)
+
+
+def hybrid(q, k, v, a, b, Hs: int, Hd: int, Hg: int, T: int, N: int,
+           w_swa: int, w_dswa: int, r: int, S0=None, scale=None):
+    """All three branches on their head groups of [B, H, L, d]; concat on the head axis.
+
+    Returns (o [B,H,L,d] float64, S_final [B,Hg,d,d] float64)."""
+    qf, kf, vf = _f32(q), _f32(k), _f32(v)
+    B, H, L, d = qf.shape
+    assert H == Hs + Hd + Hg
+    o = np.empty(qf.shape, dtype=np.float64)
+    if Hs:
+        o[:, :Hs] = swa(qf[:, :Hs], kf[:, :Hs], vf[:, :Hs], T, N, w_swa, scale)
+    if Hd:
+        s = slice(Hs, Hs + Hd)
+        o[:, s] = dswa(qf[:, s], kf[:, s], vf[:, s], T, N, w_dswa, r, scale)
+    S_fin = np.zeros((B, Hg, d, d))
+    if Hg:
+        s = slice(Hs + Hd, H)
+        og, S_fin = gdn(qf[:, s], kf[:, s], vf[:, s], a, b, S0)
+        o[:, s] = og
+    return o, S_fin
+
+
+def hybrid_rows(q, k, v, a, b, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, rows, scale=None):
+    """Softmax branches on sampled query rows only, GDN in full.
+
+    ``rows``: query positions l (shared by every head). Returns
+    (o_sw [B,Hs,len(rows),d], o_dsw [B,Hd,len(rows),d], o_gdn [B,Hg,L,d], S_final)."""
+    qf, kf, vf = _f32(q), _f32(k), _f32(v)
+    B, H, L, d = qf.shape
+    rows = np.asarray(rows, dtype=np.int64)
+
+    def flat(nh):
+        return (np.arange(B * nh)[:, None] * L + rows[None, :]).reshape(-1)
+
+    o_s = o_d = None
+    if Hs:
+        o_s = swa(qf[:, :Hs], kf[:, :Hs], vf[:, :Hs], T, N, w_swa, scale,
+                  rows=flat(Hs)).reshape(B, Hs, rows.size, d)
+    if Hd:
+        s = slice(Hs, Hs + Hd)
+        o_d = dswa(qf[:, s], kf[:, s], vf[:, s], T, N, w_dswa, r, scale,
+                   rows=flat(Hd)).reshape(B, Hd, rows.size, d)
+    o_g, S_fin = (None, None)
+    if Hg:
+        s = slice(Hs + Hd, H)
+        o_g, S_fin = gdn(qf[:, s], kf[:, s], vf[:, s], a, b)
+    return o_s, o_d, o_g, S_fin

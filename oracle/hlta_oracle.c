@@ -1,0 +1,221 @@
+/*
+ * CPU oracle for the Hybrid Linear Temporal Attention operator.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path may link, load or call this
+ * file: only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+ * use it. It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes, straight from the definitions and nothing cleverer:
+ *
+ *   Sliding-window attention (SWA) and dilated sliding-window attention (DSWA): the
+ *   Kairos abstract (chatpaper.ai page, item (2)) and the zhichai.net blog (section 2.2,
+ *   "Maintain the world") name the three branches: sliding windows capture local
+ *   dynamics, dilated sliding windows mid-range dependencies. Here a query token in
+ *   frame f attends with an explicit, max-subtracted softmax to every token of its key
+ *   frames; SWA's key frames are max(0, f-w+1) .. f, DSWA's are f, f-r, ..., f-r(w-1)
+ *   (taps below frame 0 are dropped). The softmax is the plain definition (llm-atlas
+ *   long-context explainer, section 03 "Flash Attention": exact attention is softmax
+ *   over all valid query-key pairs, whatever the tiling).
+ *
+ *   Gated delta rule (GDN): the persistent global memory of the same abstract. The
+ *   related-papers analysis (zhaifeiyue.github.io, row A and the Kimi K2 paragraph)
+ *   writes its decay term S_t = alpha_t S_{t-1} + ...; the long-context explainer
+ *   (section 06 "Finite-state memory") describes the delta rule as "erase the old
+ *   association aligned with the key, then write the true value", with a gate that
+ *   forgets first. The full update used here is the Gated DeltaNet form
+ *       S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,     o_t = S_t q_t,
+ *   token by token in sequence order, S a d x d matrix (rows: value dimension, columns:
+ *   key dimension), the output read after the update.
+ *
+ * Precision: inputs are float32 arrays (bf16 inputs are exactly representable); every
+ * sum, product, exponential and state element is double precision.
+ *
+ * Parity status: every function here is pinned by tests that do not re-type its
+ * formula (brute-force full attention, closed forms, contraction and retrieval
+ * invariants); see tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Key frames of a query in frame f, in increasing order. Returns the count. */
+static int swa_key_frames(int f, int w, int *out)
+{
+    int lo = f - w + 1;
+    if (lo < 0) lo = 0;
+    int n = 0;
+    for (int fk = lo; fk <= f; ++fk) out[n++] = fk;
+    return n;
+}
+
+static int dswa_key_frames(int f, int w, int r, int *out)
+{
+    /* taps f - r*i, i = w-1 .. 0, kept only when >= 0; listed in increasing order */
+    int n = 0;
+    for (int i = w - 1; i >= 0; --i) {
+        long fk = (long)f - (long)r * i;
+        if (fk >= 0) out[n++] = (int)fk;
+    }
+    return n;
+}
+
+/* Explicit softmax attention of one query row over the tokens of the listed frames. */
+static void softmax_row(const float *qrow, const float *K, const float *V, int N, int d,
+                        const int *frames, int nf, double scale, double *z, double *out)
+{
+    int nk = nf * N;
+    double m = -INFINITY;
+    for (int i = 0; i < nf; ++i) {
+        for (int n = 0; n < N; ++n) {
+            const float *krow = K + ((long)frames[i] * N + n) * d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += (double)qrow[c] * (double)krow[c];
+            s *= scale;
+            z[(long)i * N + n] = s;
+            if (s > m) m = s;
+        }
+    }
+    double den = 0.0;
+    for (int j = 0; j < nk; ++j) {
+        z[j] = exp(z[j] - m);
+        den += z[j];
+    }
+    for (int c = 0; c < d; ++c) out[c] = 0.0;
+    for (int i = 0; i < nf; ++i) {
+        for (int n = 0; n < N; ++n) {
+            const float *vrow = V + ((long)frames[i] * N + n) * d;
+            double p = z[(long)i * N + n];
+            for (int c = 0; c < d; ++c) out[c] += p * (double)vrow[c];
+        }
+    }
+    for (int c = 0; c < d; ++c) out[c] /= den;
+}
+
+/*
+ * Shared driver of the two windowed branches.
+ * q, k, v: [BH][L][d] float32, L = T*N. Output o: double.
+ * rows == NULL: every row, o is [BH][L][d].
+ * rows != NULL: nrows flat indices bh*L + l, o is [nrows][d].
+ */
+static int window_attention(const float *q, const float *k, const float *v, double *o,
+                            long BH, int T, int N, int d, int w, int r, int dilated,
+                            double scale, const long *rows, long nrows)
+{
+    if (BH <= 0 || T <= 0 || N <= 0 || d <= 0 || w <= 0 || r <= 0) return 1;
+    long L = (long)T * N;
+    long total = rows ? nrows : BH * L;
+    int err = 0;
+#pragma omp parallel
+    {
+        int *frames = (int *)malloc(sizeof(int) * (size_t)w);
+        double *z = (double *)malloc(sizeof(double) * (size_t)w * (size_t)N);
+        if (!frames || !z) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long it = 0; it < total; ++it) {
+                long flat = rows ? rows[it] : it;
+                long bh = flat / L, l = flat % L;
+                if (bh < 0 || bh >= BH) continue;
+                int f = (int)(l / N);
+                int nf = dilated ? dswa_key_frames(f, w, r, frames) : swa_key_frames(f, w, frames);
+                const float *K = k + bh * L * d;
+                const float *V = v + bh * L * d;
+                softmax_row(q + flat * d, K, V, N, d, frames, nf, scale, z, o + it * d);
+            }
+        }
+        free(frames);
+        free(z);
+    }
+    return err;
+}
+
+int oracle_swa(const float *q, const float *k, const float *v, double *o,
+               long BH, int T, int N, int d, int w, double scale,
+               const long *rows, long nrows)
+{
+    return window_attention(q, k, v, o, BH, T, N, d, w, 1, 0, scale, rows, nrows);
+}
+
+int oracle_dswa(const float *q, const float *k, const float *v, double *o,
+                long BH, int T, int N, int d, int w, int r, double scale,
+                const long *rows, long nrows)
+{
+    return window_attention(q, k, v, o, BH, T, N, d, w, r, 1, scale, rows, nrows);
+}
+
+/*
+ * Gated delta rule, token by token.
+ * q, k, v: [BH][L][d] float32; a, b: [BH][L] float32 gates.
+ * S0: [BH][d][d] double or NULL (zero state). o: [BH][L][d] double.
+ * S_out: [BH][d][d] double or NULL. S_hist: [BH][L][d][d] double or NULL (every S_t,
+ * for small invariant checks).
+ */
+int oracle_gdn(const float *q, const float *k, const float *v, const float *a,
+               const float *b, const double *S0, double *o, double *S_out,
+               double *S_hist, long BH, long L, int d)
+{
+    if (BH <= 0 || L < 0 || d <= 0) return 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+        double *Sk = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!S || !Sk) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                if (S0) memcpy(S, S0 + bh * d * d, sizeof(double) * (size_t)d * d);
+                else memset(S, 0, sizeof(double) * (size_t)d * d);
+                for (long t = 0; t < L; ++t) {
+                    const float *kt = k + (bh * L + t) * d;
+                    const float *vt = v + (bh * L + t) * d;
+                    const float *qt = q + (bh * L + t) * d;
+                    double at = a[bh * L + t], bt = b[bh * L + t];
+                    /* S k_t */
+                    for (int i = 0; i < d; ++i) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += S[(long)i * d + j] * (double)kt[j];
+                        Sk[i] = s;
+                    }
+                    /* S <- a S (I - b k k^T) + b v k^T = a (S - b (S k) k^T) + b v k^T */
+                    for (int i = 0; i < d; ++i) {
+                        for (int j = 0; j < d; ++j) {
+                            double kj = (double)kt[j];
+                            S[(long)i * d + j] = at * (S[(long)i * d + j] - bt * Sk[i] * kj)
+                                                 + bt * (double)vt[i] * kj;
+                        }
+                    }
+                    /* o_t = S_t q_t */
+                    double *ot = o + (bh * L + t) * d;
+                    for (int i = 0; i < d; ++i) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += S[(long)i * d + j] * (double)qt[j];
+                        ot[i] = s;
+                    }
+                    if (S_hist)
+                        memcpy(S_hist + (bh * L + t) * d * d, S, sizeof(double) * (size_t)d * d);
+                }
+                if (S_out) memcpy(S_out + bh * d * d, S, sizeof(double) * (size_t)d * d);
+            }
+        }
+        free(S);
+        free(Sk);
+    }
+    return err;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
