@@ -1,0 +1,178 @@
+/*
+ * hlta.h - C ABI of the B200 (sm_100a) Hybrid Linear Temporal Attention library.
+ *
+ * The operator (Kairos abstract, chatpaper.ai page, item (2); zhichai.net blog, section 2.2
+ * "Maintain the world"; researchpapers.dev summary, "How hybrid linear temporal attention
+ * suppresses drift") runs three branches over a frame-major video token sequence:
+ *   - SWA:  block-causal sliding-window softmax attention over the last w latent frames
+ *           ("sliding-window attention captures local dynamics");
+ *   - DSWA: dilated sliding-window softmax attention over frames f, f-r, ..., f-r(w-1)
+ *           ("dilated sliding windows capture mid-range dependencies");
+ *   - GDN:  gated linear attention with the delta rule, the persistent global memory
+ *           ("gated linear attention maintains persistent global memory"; decay term
+ *           S_t = alpha_t S_{t-1} + ... in the zhaifeiyue.github.io related-papers analysis,
+ *           erase-then-write in the llm-atlas long-context explainer, section 06), here
+ *           S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,  o_t = S_t q_t.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Token l of a clip is l = f*N + n: frame f, token n of that frame (patch raster order).
+ * Tensors are dense row-major. q, k, v, o: [B, H, L, d] with L = T*N. Gates a, b: [B, H, L]
+ * float32 (GDN heads only). State S: [B, H, d, d] float32, S[i][j] with i the value index
+ * and j the key index, so o = S q.
+ * Pointers passed to compute calls are DEVICE pointers (cudaMalloc / torch tensors on the
+ * GPU), owned by the caller, 16-byte aligned; the library never frees them. Element type:
+ * HLTA_BF16 (bf16 in/out, fp32 accumulation and fp32 state) or HLTA_FP32 (fp32 in/out,
+ * fp32 arithmetic throughout, no tensor-core rounding).
+ * `stream` is a cudaStream_t (NULL: the legacy default stream). Calls are asynchronous:
+ * they validate arguments on the host, enqueue kernels on `stream` and return; they never
+ * synchronize the stream.
+ * Softmax scale: `scale <= 0` selects 1/sqrt(d).
+ *
+ * Errors: every call returns hlta_status. Argument errors are detected before any launch
+ * (nothing is enqueued). HLTA_ERR_CUDA reports a launch or runtime failure (asynchronous
+ * faults from earlier work surface at a later call). HLTA_ERR_TIMEOUT is reported by
+ * hlta_device_status() when a kernel's bounded wait expired and the kernel stopped early.
+ * hlta_last_error() returns a thread-local description of the last non-OK status.
+ * No C++ exception crosses this interface.
+ *
+ * Supported shapes: d = 128 for HLTA_BF16; 1 <= d <= 128 for HLTA_FP32. N >= 1, T >= 1,
+ * w >= 1, r >= 1, chunk = 64 (the GDN chunk length; results do not depend on it beyond
+ * rounding).
+ */
+#ifndef HLTA_H
+#define HLTA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HLTA_OK = 0,
+    HLTA_ERR_INVALID_ARG = 1,
+    HLTA_ERR_UNSUPPORTED = 2,
+    HLTA_ERR_CUDA = 3,
+    HLTA_ERR_TIMEOUT = 4
+} hlta_status;
+
+typedef enum { HLTA_BF16 = 0, HLTA_FP32 = 1 } hlta_dtype;
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int hlta_version(void);
+
+/* Thread-local message describing the last non-OK status returned on this thread. */
+const char *hlta_last_error(void);
+
+/*
+ * Block-causal sliding-window attention (SWA).
+ * For every query token in frame f: softmax over the scaled dot products with every token
+ * of frames max(0, f-w+1) .. f (all N tokens of each, including later tokens of frame f),
+ * then the weighted sum of their values. Defined by the Kairos abstract's "sliding-window
+ * attention captures local dynamics" read as: window = the last w latent frames, the
+ * current one included; bidirectional inside a frame, causal across frames.
+ * q, k, v, o: [B, H, T*N, d] device, element type `dt`. o is written in full.
+ */
+hlta_status hlta_swa_fwd(const void *q, const void *k, const void *v, void *o,
+                         int B, int H, int T, int N, int d, int w, float scale,
+                         hlta_dtype dt, void *stream);
+
+/*
+ * Dilated sliding-window attention (DSWA). As hlta_swa_fwd, but the key frames of a query
+ * in frame f are f - r*i for i = 0 .. w-1, dropping taps below frame 0 (Kairos abstract:
+ * "dilated sliding windows capture mid-range dependencies"). r = 1 gives SWA.
+ */
+hlta_status hlta_dswa_fwd(const void *q, const void *k, const void *v, void *o,
+                          int B, int H, int T, int N, int d, int w, int r, float scale,
+                          hlta_dtype dt, void *stream);
+
+/*
+ * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens.
+ */
+size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt);
+
+/*
+ * Gated delta rule in chunkwise form (UT transform within 64-token chunks, state passed
+ * between chunks; llm-atlas long-context explainer, sections 06 and 09: "parallel within a
+ * block, recurrent across blocks"). Result equals the token recurrence
+ *   S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S_t q_t
+ * in sequence order l = 0 .. L-1 for each (batch, head), up to rounding.
+ * q, k, v, o: [B, H, L, d] device (type `dt`); a, b: [B, H, L] float32 device, with
+ * a in (0, 1] and b in [0, 1] (values outside are not rejected; the result is then the
+ * same algebra without the contraction guarantee).
+ * S0: [B, H, d, d] float32 initial state, or NULL for zero. S_out: final state or NULL;
+ * S_out may equal S0 (in-place update).
+ * workspace: device scratch of at least hlta_gdn_workspace_bytes(...) bytes, 256-byte
+ * aligned, owned by the caller; its contents on entry are ignored.
+ */
+hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                               const float *a, const float *b, void *o,
+                               const float *S0, float *S_out,
+                               int B, int H, long L, int d, int chunk,
+                               void *workspace, size_t ws_bytes,
+                               hlta_dtype dt, void *stream);
+
+/* Workspace size in bytes for hlta_hybrid_fwd. */
+size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk,
+                                   hlta_dtype dt);
+
+/*
+ * The hybrid operator: heads [0, Hs) run SWA(w_swa), heads [Hs, Hs+Hd) run DSWA(w_dswa, r),
+ * heads [Hs+Hd, H) run the gated delta rule; outputs are concatenated on the head axis
+ * (each branch writes its own head range of o, in place).
+ * q, k, v, o: [B, H, T*N, d] with H = Hs + Hd + Hg; a, b: [B, Hg, T*N] float32.
+ * S0 / S_out: [B, Hg, d, d] float32 or NULL (as hlta_gdn_chunk_fwd).
+ * The GDN branch runs on a library-owned second stream ordered after `stream` by events,
+ * so it overlaps the softmax branches; the call still completes, in stream order, on
+ * `stream` (later work on `stream` sees every output).
+ */
+hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v,
+                            const float *a, const float *b, void *o,
+                            const float *S0, float *S_out,
+                            int B, int Hs, int Hd, int Hg, int T, int N, int d,
+                            int w_swa, int w_dswa, int r, int chunk, float scale,
+                            void *workspace, size_t ws_bytes,
+                            hlta_dtype dt, void *stream);
+
+/*
+ * Streaming rollout (zhichai.net blog, section 2.3: the "streaming token" design generates
+ * incrementally without waiting for the whole sequence). A cache holds, for B independent
+ * rollouts advancing in lockstep, the K/V of the last w_swa frames of the SWA heads, of the
+ * last r*(w_dswa-1)+1 frames of the DSWA heads, and the fp32 state of the GDN heads.
+ * Each step appends one frame of N tokens per rollout; its output equals the last frame of
+ * hlta_hybrid_fwd over all frames appended so far (up to rounding).
+ */
+typedef struct hlta_stream *hlta_stream_t;
+
+/* Allocates the cache on the current CUDA device (the only call that allocates). S0:
+ * [B, Hg, d, d] float32 device initial state or NULL for zero. Starts at frame 0. */
+hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N,
+                               int d, int w_swa, int w_dswa, int r, int chunk, float scale,
+                               hlta_dtype dt, const float *S0);
+
+/* One step. q_new, k_new, v_new, o_new: [B, H, N, d] device; a_new, b_new: [B, Hg, N]
+ * float32 device. Appends the new K/V to the rings, advances the frame counter. */
+hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_new,
+                             const void *v_new, const float *a_new, const float *b_new,
+                             void *o_new, void *stream);
+
+/* Device pointer to the carried GDN state [B, Hg, d, d] (owned by the cache) and the
+ * number of frames appended so far. */
+hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done);
+
+/* Frees the cache. Synchronizes the device first. */
+hlta_status hlta_stream_destroy(hlta_stream_t c);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device error word.
+ * *code receives the raw word (0: no kernel stopped early). Returns HLTA_ERR_TIMEOUT if a
+ * bounded wait expired in any kernel since the last call, HLTA_ERR_CUDA on a CUDA error.
+ */
+hlta_status hlta_device_status(void *stream, unsigned int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HLTA_H */

@@ -1,0 +1,240 @@
+"""Python binding of the B200 Hybrid Linear Temporal Attention library (libhlta.so).
+
+Argument marshalling only: every function passes device pointers, sizes and the current
+CUDA stream to the C ABI declared in include/hlta.h, and raises ``HltaError`` on a non-OK
+status. Tensors are torch tensors on a CUDA device (torch provides memory and streams);
+no computation happens here, and there is no fallback: if the compiled library is missing,
+importing this package fails.
+
+Function names match the C entry points (``hlta_swa_fwd`` ...). The convenience wrappers
+at the end (``swa``, ``dswa``, ``gdn``, ``hybrid``, ``Stream``) allocate outputs and
+workspaces with torch and then call those same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhlta.so")
+
+HLTA_OK, HLTA_ERR_INVALID_ARG, HLTA_ERR_UNSUPPORTED, HLTA_ERR_CUDA, HLTA_ERR_TIMEOUT = range(5)
+HLTA_BF16, HLTA_FP32 = 0, 1
+_STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
+
+
+class HltaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"HLTA_ERR_{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m linear_video_world_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, L, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "hlta_version": (I, []),
+        "hlta_last_error": (ctypes.c_char_p, []),
+        "hlta_swa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, F, I, P]),
+        "hlta_dswa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, F, I, P]),
+        "hlta_gdn_workspace_bytes": (Z, [I, I, L, I, I, I]),
+        "hlta_gdn_chunk_fwd": (I, [P, P, P, P, P, P, P, P, I, I, L, I, I, P, Z, I, P]),
+        "hlta_hybrid_workspace_bytes": (Z, [I, I, I, I, I, I, I]),
+        "hlta_hybrid_fwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F,
+                                P, Z, I, P]),
+        "hlta_stream_create": (I, [ctypes.POINTER(P), I, I, I, I, I, I, I, I, I, I, F, I, P]),
+        "hlta_stream_step": (I, [P, P, P, P, P, P, P, P]),
+        "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
+        "hlta_stream_destroy": (I, [P]),
+        "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != HLTA_OK:
+        raise HltaError(status, (_lib.hlta_last_error() or b"").decode(errors="replace"))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dt(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return HLTA_BF16
+    if t.dtype == torch.float32:
+        return HLTA_FP32
+    raise HltaError(HLTA_ERR_INVALID_ARG, f"unsupported dtype {t.dtype}")
+
+
+def _need(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise HltaError(HLTA_ERR_INVALID_ARG, f"{name} must be a contiguous CUDA tensor")
+
+
+# ---- entry points (same names as the C ABI) -----------------------------------------
+
+def hlta_version() -> int:
+    return int(_lib.hlta_version())
+
+
+def hlta_swa_fwd(q, k, v, o, B, H, T, N, d, w, scale=0.0, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n)
+    _check(_lib.hlta_swa_fwd(_p(q), _p(k), _p(v), _p(o), B, H, T, N, d, w, float(scale),
+                             _dt(q), _stream(stream)))
+
+
+def hlta_dswa_fwd(q, k, v, o, B, H, T, N, d, w, r, scale=0.0, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n)
+    _check(_lib.hlta_dswa_fwd(_p(q), _p(k), _p(v), _p(o), B, H, T, N, d, w, r, float(scale),
+                              _dt(q), _stream(stream)))
+
+
+def hlta_gdn_workspace_bytes(B, H, L, d, chunk=64, dt=HLTA_BF16) -> int:
+    return int(_lib.hlta_gdn_workspace_bytes(B, H, L, d, chunk, dt))
+
+
+def hlta_gdn_chunk_fwd(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, workspace,
+                       stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (a, "a"), (b, "b"), (o, "o"), (workspace, "workspace")):
+        _need(t, n)
+    _check(_lib.hlta_gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(o), _p(S0), _p(S_out),
+                                   B, H, L, d, chunk, _p(workspace), workspace.numel() * workspace.element_size(),
+                                   _dt(q), _stream(stream)))
+
+
+def hlta_hybrid_workspace_bytes(B, Hg, T, N, d, chunk=64, dt=HLTA_BF16) -> int:
+    return int(_lib.hlta_hybrid_workspace_bytes(B, Hg, T, N, d, chunk, dt))
+
+
+def hlta_hybrid_fwd(q, k, v, a, b, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa, r,
+                    chunk, scale, workspace, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel() * workspace.element_size())
+    _check(_lib.hlta_hybrid_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(o), _p(S0), _p(S_out),
+                                B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa, r, chunk, float(scale),
+                                ws_ptr, ws_bytes, _dt(q), _stream(stream)))
+
+
+def hlta_device_status(stream=None) -> int:
+    code = ctypes.c_uint(0)
+    _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
+    return int(code.value)
+
+
+# ---- convenience wrappers (allocate with torch, then call the entry points) ----------
+
+def _workspace(nbytes, device):
+    import torch
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def swa(q, k, v, T, N, w, scale=0.0, out=None, stream=None):
+    import torch
+    B, H, _, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    hlta_swa_fwd(q, k, v, o, B, H, T, N, d, w, scale, stream)
+    return o
+
+
+def dswa(q, k, v, T, N, w, r, scale=0.0, out=None, stream=None):
+    import torch
+    B, H, _, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    hlta_dswa_fwd(q, k, v, o, B, H, T, N, d, w, r, scale, stream)
+    return o
+
+
+def gdn(q, k, v, a, b, S0=None, chunk=64, out=None, S_out=None, workspace=None, stream=None):
+    import torch
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    if S_out is None:
+        S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(hlta_gdn_workspace_bytes(B, H, L, d, chunk, _dt(q)), q.device)
+    hlta_gdn_chunk_fwd(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, workspace, stream)
+    return o, S_out
+
+
+def hybrid(q, k, v, a, b, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, S0=None, chunk=64, scale=0.0,
+           out=None, S_out=None, workspace=None, stream=None):
+    import torch
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    if Hg and S_out is None:
+        S_out = torch.empty((B, Hg, d, d), dtype=torch.float32, device=q.device)
+    if Hg and workspace is None:
+        workspace = _workspace(hlta_hybrid_workspace_bytes(B, Hg, T, N, d, chunk, _dt(q)), q.device)
+    hlta_hybrid_fwd(q, k, v, a, b, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa, r,
+                    chunk, scale, workspace, stream)
+    return o, S_out
+
+
+class Stream:
+    """Streaming cache (hlta_stream_create / _step / _state / _destroy)."""
+
+    def __init__(self, B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk=64, scale=0.0,
+                 dtype=None, S0=None):
+        import torch
+        dt = HLTA_BF16 if dtype in (None, torch.bfloat16) else HLTA_FP32
+        self._h = ctypes.c_void_p()
+        _check(_lib.hlta_stream_create(ctypes.byref(self._h), B, Hs, Hd, Hg, N, d, w_swa,
+                                       w_dswa, r, chunk, float(scale), dt, _p(S0)))
+        self.B, self.H, self.Hg, self.N, self.d = B, Hs + Hd + Hg, Hg, N, d
+
+    def step(self, q, k, v, a, b, out=None, stream=None):
+        import torch
+        o = torch.empty_like(q) if out is None else out
+        _check(_lib.hlta_stream_step(self._h, _p(q), _p(k), _p(v), _p(a), _p(b), _p(o),
+                                     _stream(stream)))
+        return o
+
+    def state(self):
+        """(device address of the [B,Hg,d,d] fp32 state, frames appended so far)."""
+        ptr, n = ctypes.c_void_p(), ctypes.c_int()
+        _check(_lib.hlta_stream_state(self._h, ctypes.byref(ptr), ctypes.byref(n)))
+        return ptr.value, n.value
+
+    def state_tensor(self):
+        """A torch copy of the carried state [B, Hg, d, d] fp32 (ordered on the current stream)."""
+        import torch
+        ptr, _ = self.state()
+
+        class _View:   # exposes the cache's device buffer to torch without copying
+            __cuda_array_interface__ = {"shape": (self.B, self.Hg, self.d, self.d),
+                                        "typestr": "<f4", "data": (ptr, False), "version": 2}
+        return torch.as_tensor(_View(), device="cuda").clone()
+
+    def close(self):
+        if self._h:
+            _check(_lib.hlta_stream_destroy(self._h))
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,597 @@
+// Windowed softmax attention (SWA / DSWA / streaming step) on the sm_100a tensor cores.
+// bf16 q/k/v/o, head dim 128, fp32 accumulation in tensor memory.
+//
+// Exact attention by tiles with a running max and normaliser (llm-atlas long-context
+// explainer, section 03 "Flash Attention": the score matrix never leaves the chip and the
+// result equals the full softmax). The key set of a query tile is the union of the key
+// frames of its rows' frames (sliding window: frames f-w+1..f; dilated: f, f-r, ...,
+// f-r(w-1); Kairos abstract, item (2)); each key frame is walked in 128-token tiles and a
+// per-element mask (row frame vs. key frame, ragged frame end) removes what a row must not
+// see.
+//
+// One CTA = one 128-row query tile of one head; 6 warps:
+//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring (128B swizzle)
+//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers,
+//               O += P_j V_j into the TMEM O accumulator (tcgen05.mma kind::f16)
+//   warps 2..5  softmax: one thread per query row; reads S from TMEM, updates the running
+//               max (rescaling O in TMEM only when the max grows by more than 2^8), writes
+//               P (bf16) to shared memory for the PV product, and finally normalises O.
+// Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in the
+// device error word, every role stops, and the TMEM allocation is released.
+#include "hlta_internal.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+
+namespace hlta {
+namespace {
+
+constexpr int BM = 128;                 // query rows per tile
+constexpr int BN = 128;                 // keys per tile
+constexpr int D = 128;                  // head dim
+constexpr int NS = 2;                   // K/V ring stages
+constexpr int THREADS = 192;
+constexpr uint32_t HALF = 16384;        // one [128 rows][64 cols] bf16 half tile
+constexpr uint32_t TILE = 2 * HALF;     // [128][128] bf16
+constexpr uint32_t TMEM_COLS = 512;     // S0 @0, S1 @128, O @256
+constexpr uint32_t TM_S = 0, TM_O = 256;
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t SM_Q = 0;
+constexpr uint32_t SM_K0 = TILE;                        // K[s] = SM_K0 + s * 2 * TILE
+constexpr uint32_t SM_P = TILE + NS * 2 * TILE;
+constexpr uint32_t SM_BAR = SM_P + TILE;
+// barriers (8 bytes each)
+enum {
+    B_QFULL = 0,
+    B_KFULL = 1,                // + s
+    B_VFULL = B_KFULL + NS,
+    B_KEMPTY = B_VFULL + NS,
+    B_VEMPTY = B_KEMPTY + NS,
+    B_SFULL = B_VEMPTY + NS,    // + buffer (2)
+    B_SFREE = B_SFULL + 2,
+    B_PFULL = B_SFREE + 2,
+    B_PVDONE = B_PFULL + 1,
+    NBARS = B_PVDONE + 1
+};
+constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
+constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
+constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
+constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;          // slack for the 1024-byte alignment
+
+struct TcParams {
+    int Hbr, q_Htot, q_h0, kv_Htot, kv_h0, kv_slots;
+    long q_rows, kv_rows;
+    int N, w, r, fq0;
+    float sl2;                  // softmax scale * log2(e)
+    __nv_bfloat16 *o;
+    unsigned int *err;
+};
+
+// ---------------------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after ~2^32 SM cycles (about two seconds), or at once when another
+// role already gave up; records the expiry in the device error word.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       unsigned int *err)
+{
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > (1LL << 32)) {
+            *abort_flag = 1;
+            atomicOr(err, (unsigned)DEVERR_ATTN_WAIT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version bit.
+// lbo / sbo in bytes: K-major operands use sbo = 1024 (8 rows of 128 B) and an unused lbo;
+// MN-major operands use lbo = distance between 64-element column blocks, sbo = 1024.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16: bf16 A and B, fp32 accumulator, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+#define TMEM_REGS32(x)                                                                      \
+    "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]),     \
+        "=r"(x[7]), "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]),          \
+        "=r"(x[13]), "=r"(x[14]), "=r"(x[15]), "=r"(x[16]), "=r"(x[17]), "=r"(x[18]),       \
+        "=r"(x[19]), "=r"(x[20]), "=r"(x[21]), "=r"(x[22]), "=r"(x[23]), "=r"(x[24]),       \
+        "=r"(x[25]), "=r"(x[26]), "=r"(x[27]), "=r"(x[28]), "=r"(x[29]), "=r"(x[30]),       \
+        "=r"(x[31])
+#define TMEM_SRC32(x)                                                                        \
+    "r"(x[0]), "r"(x[1]), "r"(x[2]), "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7]), \
+        "r"(x[8]), "r"(x[9]), "r"(x[10]), "r"(x[11]), "r"(x[12]), "r"(x[13]), "r"(x[14]),    \
+        "r"(x[15]), "r"(x[16]), "r"(x[17]), "r"(x[18]), "r"(x[19]), "r"(x[20]), "r"(x[21]),  \
+        "r"(x[22]), "r"(x[23]), "r"(x[24]), "r"(x[25]), "r"(x[26]), "r"(x[27]), "r"(x[28]),  \
+        "r"(x[29]), "r"(x[30]), "r"(x[31])
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32*(w%4)..).
+// The load and its wait sit in one asm statement, so no use of the registers can be
+// scheduled between them.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&x)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : TMEM_REGS32(x)
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&x)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31, %32};" ::"r"(taddr),
+        TMEM_SRC32(x)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ---------------------------------------------------------------------------------------
+// key-tile walk shared by every role (all roles must visit the same sequence)
+// ---------------------------------------------------------------------------------------
+struct Walk {
+    int fa, fb, w, r, tpf;
+    // frame fk is a key frame of some query frame in [fa, fb]
+    __device__ __forceinline__ bool needed(int fk) const
+    {
+        int i0 = fa > fk ? (fa - fk + r - 1) / r : 0;
+        return i0 < w && fk + r * i0 <= fb;
+    }
+    // advance (fk, jt) to the next tile; false when done
+    __device__ __forceinline__ bool next(int &fk, int &jt) const
+    {
+        if (++jt < tpf) return true;
+        for (++fk; fk <= fb; ++fk)
+            if (needed(fk)) {
+                jt = 0;
+                return true;
+            }
+        return false;
+    }
+};
+
+__device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
+{
+    int dist = fq - fk;
+    return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+               const __grid_constant__ CUtensorMap tv, const TcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + SM_BAR;
+    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    volatile int *abort_flag = (volatile int *)(smem + SM_ABORT);
+    uint32_t *tmem_slot = (uint32_t *)(smem + SM_TMEMSLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int b = bh / p.Hbr, h = bh % p.Hbr;
+    const long l0 = (long)blockIdx.x * BM;
+    const long q_head = (long)(b * p.q_Htot + p.q_h0 + h) * p.q_rows;
+    const long kv_head = (long)(b * p.kv_Htot + p.kv_h0 + h) * p.kv_rows;
+    const int nrows = (int)min((long)BM, p.q_rows - l0);
+    Walk wk;
+    wk.fa = p.fq0 + (int)(l0 / p.N);
+    wk.fb = p.fq0 + (int)((l0 + nrows - 1) / p.N);
+    wk.w = p.w;
+    wk.r = p.r;
+    wk.tpf = (p.N + BN - 1) / BN;
+    const int fstart = max(0, wk.fa - p.r * (p.w - 1));
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QFULL), 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(BAR(B_KFULL + s), 1);
+            mbar_init(BAR(B_VFULL + s), 1);
+            mbar_init(BAR(B_KEMPTY + s), 1);
+            mbar_init(BAR(B_VEMPTY + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(B_SFULL + i), 1);
+            mbar_init(BAR(B_SFREE + i), 128);
+        }
+        mbar_init(BAR(B_PFULL), 128);
+        mbar_init(BAR(B_PVDONE), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------- TMA producer -----------------------------------
+        if (lane == 0) {
+            const int qrow = (int)(q_head + l0);
+            mbar_expect_tx(BAR(B_QFULL), TILE);
+            tma_load_2d(sbase + SM_Q, &tq, 0, qrow, BAR(B_QFULL));
+            tma_load_2d(sbase + SM_Q + HALF, &tq, 64, qrow, BAR(B_QFULL));
+            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
+            while (wk.next(fk, jt)) {
+                const int s = j % NS;
+                const uint32_t ph = (uint32_t)((j / NS) + 1) & 1u;
+                const int krow = (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
+                const uint32_t kdst = sbase + SM_K0 + (uint32_t)s * 2 * TILE;
+                const uint32_t vdst = kdst + TILE;
+                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, p.err)) break;
+                mbar_expect_tx(BAR(B_KFULL + s), TILE);
+                tma_load_2d(kdst, &tk, 0, krow, BAR(B_KFULL + s));
+                tma_load_2d(kdst + HALF, &tk, 64, krow, BAR(B_KFULL + s));
+                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, p.err)) break;
+                mbar_expect_tx(BAR(B_VFULL + s), TILE);
+                tma_load_2d(vdst, &tv, 0, krow, BAR(B_VFULL + s));
+                tma_load_2d(vdst + HALF, &tv, 64, krow, BAR(B_VFULL + s));
+                ++j;
+            }
+            if (*abort_flag) {
+                // let this CTA's copies in flight land before the CTA may exit
+                const long long t0 = clock64();
+                for (int s = 0; s < NS; ++s) {
+                    for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj) {
+                        if (jj % NS != s) continue;
+                        const uint32_t ph = (uint32_t)(jj / NS) & 1u;
+                        while (!mbar_try(BAR(B_KFULL + s), ph) && clock64() - t0 < (1LL << 31)) {}
+                        while (!mbar_try(BAR(B_VFULL + s), ph) && clock64() - t0 < (1LL << 31)) {}
+                    }
+                }
+                while (!mbar_try(BAR(B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer -------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
+            constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P K-major, V MN-major
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err);
+            auto issue_pv = [&](int t) -> bool {
+                const int s = t % NS;
+                if (!mbar_wait(BAR(B_PFULL), (uint32_t)t & 1u, abort_flag, p.err)) return false;
+                if (!mbar_wait(BAR(B_VFULL + s), (uint32_t)(t / NS) & 1u, abort_flag, p.err)) return false;
+                fence_after_sync();
+                const uint32_t vaddr = sbase + SM_K0 + (uint32_t)s * 2 * TILE + TILE;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(sbase + SM_P + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(vaddr + kk * 2048, HALF, 1024);
+                    umma_bf16(tmem + TM_O, ad, bd, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(BAR(B_VEMPTY + s));
+                umma_commit(BAR(B_PVDONE));
+                return true;
+            };
+            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
+            while (ok && wk.next(fk, jt)) {
+                const int s = j % NS, sb = j & 1;
+                if (!mbar_wait(BAR(B_KFULL + s), (uint32_t)(j / NS) & 1u, abort_flag, p.err)) { ok = false; break; }
+                if (j >= 2 && !mbar_wait(BAR(B_SFREE + sb), (uint32_t)((j / 2) + 1) & 1u, abort_flag, p.err)) { ok = false; break; }
+                fence_after_sync();
+                const uint32_t kaddr = sbase + SM_K0 + (uint32_t)s * 2 * TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+                    umma_bf16(tmem + TM_S + (uint32_t)sb * BN, sw128_desc(sbase + SM_Q + off, 16, 1024),
+                              sw128_desc(kaddr + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(BAR(B_KEMPTY + s));
+                umma_commit(BAR(B_SFULL + sb));
+                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+                ++j;
+            }
+            if (ok && j >= 1) issue_pv(j - 1);
+        }
+    } else {
+        // ------------------------------- softmax ----------------------------------------
+        const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+        const int row = quad * 32 + lane;
+        const long lrow = l0 + row;
+        const bool row_valid = lrow < p.q_rows;
+        const int fq = p.fq0 + (int)(lrow / p.N);
+        const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+        uint8_t *prow = smem + SM_P + row * 128;
+        const int sw = row & 7;
+        float m = -INFINITY, lsum = 0.f;
+        bool ok = true;
+        int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
+        while (wk.next(fk, jt)) {
+            const int sb = j & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (uint32_t)(j / 2) & 1u, abort_flag, p.err))) { ok = false; break; }
+            fence_after_sync();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tlane + TM_S + (uint32_t)sb * BN + c * 32, sr[c]);
+            fence_before_sync();
+            mbar_arrive(BAR(B_SFREE + sb));
+
+            const int nv = min(BN, p.N - jt * BN);
+            const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
+            float mt = -INFINITY;
+            if (rok) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float sv = __uint_as_float(sr[c][i]);
+                        mt = fmaxf(mt, (c * 32 + i < nv) ? sv : -INFINITY);
+                    }
+            }
+            // P buffer and O are in use by the previous tile's PV product until it completes
+            if (j >= 1) {
+                if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (uint32_t)(j - 1) & 1u, abort_flag, p.err))) { ok = false; break; }
+                fence_after_sync();
+            }
+            float mnew = m;
+            if (rok) mnew = fmaxf(m, mt * p.sl2);
+            // grow the reference max only when it rose by more than 2^8; the TMEM traffic of
+            // the O rescale is warp-collective, so the whole warp takes that branch together
+            const bool need = rok && mnew > m + 8.f;
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
+                if (j >= 1) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t orow[32];
+                        tmem_ld32(tlane + TM_O + c * 32, orow);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                        tmem_st32(tlane + TM_O + c * 32, orow);
+                    }
+                    tmem_wait_st();
+                }
+                if (need) {
+                    lsum *= alpha;
+                    m = mnew;
+                }
+            }
+            float part = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int col = c * 32 + 2 * i;
+                    float p0 = 0.f, p1 = 0.f;
+                    if (rok) {
+                        p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[c][2 * i]), p.sl2, -m)) : 0.f;
+                        p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), p.sl2, -m)) : 0.f;
+                    }
+                    part += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+                // 32 keys = 4 chunks of 16 B; chunk index within the 64-key half is XOR-swizzled
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int chunk = c * 4 + q4;               // 0..15 over 128 keys
+                    const int half = chunk >> 3, cc = chunk & 7;
+                    uint8_t *dst = prow + half * HALF + ((cc ^ sw) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)),
+                                 "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]),
+                                 "r"(pk[4 * q4 + 3])
+                                 : "memory");
+                }
+            }
+            lsum += part;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_before_sync();
+            mbar_arrive(BAR(B_PFULL));
+            ++j;
+        }
+        if (ok && j >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (uint32_t)(j - 1) & 1u, abort_flag, p.err))) {
+            fence_after_sync();
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(tlane + TM_O + c * 32, ov);
+                if (row_valid) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk[i] = pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                }
+            }
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t get_encoder()
+{
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    });
+    return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// 2-D view [rows][128] bf16 of a row-major tensor; box = 128 rows x 64 columns, 128B swizzle
+cudaError_t make_map(CUtensorMap *map, const void *base, long rows)
+{
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)BM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
+{
+    if (a.d != D) return cudaErrorNotSupported;
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    const long q_total = (long)a.B * a.q_Htot * a.q_rows;
+    const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
+    if (q_total + BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if ((e = make_map(&mq, a.q, q_total)) != cudaSuccess) return e;
+    if ((e = make_map(&mk, a.k, kv_total)) != cudaSuccess) return e;
+    if ((e = make_map(&mv, a.v, kv_total)) != cudaSuccess) return e;
+    TcParams p;
+    p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
+    p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
+    p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0;
+    p.sl2 = a.scale * 1.4426950408889634f;
+    p.o = (__nv_bfloat16 *)a.o;
+    p.err = a.err;
+    e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((a.q_rows + BM - 1) / BM), (unsigned)(a.B * a.Hbr));
+    attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace hlta

@@ -1,0 +1,458 @@
+// C ABI of the library: argument validation, dispatch to the kernels, the hybrid operator's
+// branch fork/join, the streaming cache and the device error word. Declarations and the
+// contract of every entry point are in include/hlta.h.
+#include "hlta.h"
+#include "hlta_internal.cuh"
+
+#include <math.h>
+#include <mutex>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+namespace hlta {
+
+__device__ unsigned int g_device_error;
+
+namespace {
+
+thread_local char t_msg[512] = "";
+
+hlta_status fail(hlta_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_msg, sizeof t_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+hlta_status cuda_fail(cudaError_t e, const char *where)
+{
+    return fail(HLTA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Per-device helpers: the device error word's address and an auxiliary stream plus two
+// events for the hybrid operator's fork/join. Created once per device, kept until exit.
+struct DeviceCtx {
+    bool ready = false;
+    unsigned int *err = nullptr;
+    cudaStream_t aux = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+DeviceCtx g_ctx[kMaxDevices];
+std::mutex g_ctx_mu;
+std::mutex g_fork_mu;   // the per-device fork/join events are shared by all host threads
+
+hlta_status device_ctx(DeviceCtx **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(HLTA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(g_ctx_mu);
+    DeviceCtx &c = g_ctx[dev];
+    if (!c.ready) {
+        if ((e = cudaGetSymbolAddress((void **)&c.err, g_device_error)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+        if ((e = cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreate");
+        if ((e = cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventCreate");
+        if ((e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventCreate");
+        c.ready = true;
+    }
+    *out = &c;
+    return HLTA_OK;
+}
+
+hlta_status check_dtype_d(hlta_dtype dt, int d)
+{
+    if (dt == HLTA_BF16) {
+        if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "bf16 path supports d = 128 only (got %d)", d);
+    } else if (dt == HLTA_FP32) {
+        if (d < 1 || d > 128) return fail(HLTA_ERR_UNSUPPORTED, "fp32 path supports 1 <= d <= 128 (got %d)", d);
+    } else {
+        return fail(HLTA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    }
+    return HLTA_OK;
+}
+
+hlta_status check_window(int w, int r)
+{
+    if (w < 1) return fail(HLTA_ERR_INVALID_ARG, "window w must be >= 1 (got %d)", w);
+    if (r < 1) return fail(HLTA_ERR_INVALID_ARG, "dilation r must be >= 1 (got %d)", r);
+    if ((long)r * (w - 1) > (1L << 24)) return fail(HLTA_ERR_INVALID_ARG, "r*(w-1) too large");
+    return HLTA_OK;
+}
+
+hlta_status run_attn(const AttnArgs &a, hlta_dtype dt, cudaStream_t s)
+{
+    if (a.B * a.Hbr == 0 || a.q_rows == 0) return HLTA_OK;
+    cudaError_t e = dt == HLTA_FP32 ? launch_attn_f32(a, s) : launch_attn_bf16_tc(a, s);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "window attention: unsupported shape");
+    if (e != cudaSuccess) return cuda_fail(e, "window attention launch");
+    return HLTA_OK;
+}
+
+hlta_status run_gdn(const GdnArgs &g, hlta_dtype dt, cudaStream_t s)
+{
+    if (g.B * g.Hg == 0) return HLTA_OK;
+    cudaError_t e = dt == HLTA_FP32 ? launch_gdn_f32(g, s) : launch_gdn_bf16(g, s);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "gated delta rule: unsupported shape");
+    if (e != cudaSuccess) return cuda_fail(e, "gated delta rule launch");
+    return HLTA_OK;
+}
+
+AttnArgs clip_attn_args(const void *q, const void *k, const void *v, void *o, int B, int Htot,
+                        int h0, int Hbr, int T, int N, int d, int w, int r, float scale,
+                        unsigned int *err)
+{
+    AttnArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o;
+    a.B = B; a.Hbr = Hbr;
+    a.q_Htot = Htot; a.q_h0 = h0; a.q_rows = (long)T * N;
+    a.kv_Htot = Htot; a.kv_h0 = h0; a.kv_rows = (long)T * N; a.kv_slots = T;
+    a.N = N; a.d = d; a.w = w; a.r = r; a.fq0 = 0;
+    a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+    a.err = err;
+    return a;
+}
+
+hlta_status window_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                       int T, int N, int d, int w, int r, float scale, hlta_dtype dt,
+                       void *stream)
+{
+    hlta_status st;
+    if (!q || !k || !v || !o) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 0 || H < 0 || T < 1 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d T=%d N=%d", B, H, T, N);
+    if ((long)T * N > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "T*N too large");
+    if ((st = check_dtype_d(dt, d)) != HLTA_OK) return st;
+    if ((st = check_window(w, r)) != HLTA_OK) return st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    AttnArgs a = clip_attn_args(q, k, v, o, B, H, 0, H, T, N, d, w, r, scale, ctx->err);
+    return run_attn(a, dt, (cudaStream_t)stream);
+}
+
+hlta_status check_gdn_common(const void *q, const void *k, const void *v, const float *a,
+                             const float *b, const void *o, const float *S0, const float *S_out,
+                             int d, int chunk, hlta_dtype dt)
+{
+    hlta_status st;
+    if (!q || !k || !v || !a || !b || !o) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(a) ||
+        !aligned16(b) || (S0 && !aligned16(S0)) || (S_out && !aligned16(S_out)))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64 (got %d)", chunk);
+    if ((st = check_dtype_d(dt, d)) != HLTA_OK) return st;
+    return HLTA_OK;
+}
+
+}  // namespace
+
+size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
+{
+    const size_t el = bf16 ? 2 : 4;
+    const size_t nch = (size_t)gdn_num_chunks(L, C);
+    const size_t arr = ((size_t)BH * nch * C * d * el + 255) & ~(size_t)255;
+    return 5 * arr + (((size_t)BH * nch * sizeof(float) + 255) & ~(size_t)255);
+}
+
+GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16)
+{
+    const size_t el = bf16 ? 2 : 4;
+    const size_t nch = (size_t)gdn_num_chunks(L, C);
+    const size_t arr = ((size_t)BH * nch * C * d * el + 255) & ~(size_t)255;
+    char *p = (char *)base;
+    GdnWorkspace w;
+    w.W = p; w.Up = p + arr; w.Op = p + 2 * arr; w.Qt = p + 3 * arr; w.Kt = p + 4 * arr;
+    w.gam = (float *)(p + 5 * arr);
+    return w;
+}
+
+unsigned int *device_error_word()
+{
+    DeviceCtx *c;
+    return device_ctx(&c) == HLTA_OK ? c->err : nullptr;
+}
+
+}  // namespace hlta
+
+using namespace hlta;
+
+// ------------------------------------------------------------------------------------
+// Streaming cache
+// ------------------------------------------------------------------------------------
+struct hlta_stream {
+    int device;
+    int B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk;
+    float scale;
+    hlta_dtype dt;
+    int slots_s, slots_d;     // ring slots: SWA w_swa frames, DSWA r*(w_dswa-1)+1 frames
+    void *ks, *vs, *kd, *vd;  // rings [B][Hs][slots_s][N][d], [B][Hd][slots_d][N][d]
+    float *S;                 // [B][Hg][d][d]
+    void *ws;                 // GDN workspace for N tokens
+    size_t ws_bytes;
+    int frames;
+};
+
+extern "C" {
+
+int hlta_version(void) { return 100; }
+
+const char *hlta_last_error(void) { return t_msg; }
+
+hlta_status hlta_swa_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                         int T, int N, int d, int w, float scale, hlta_dtype dt, void *stream)
+{
+    return window_fwd(q, k, v, o, B, H, T, N, d, w, 1, scale, dt, stream);
+}
+
+hlta_status hlta_dswa_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                          int T, int N, int d, int w, int r, float scale, hlta_dtype dt,
+                          void *stream)
+{
+    return window_fwd(q, k, v, o, B, H, T, N, d, w, r, scale, dt, stream);
+}
+
+size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt)
+{
+    if (B < 0 || H < 0 || L < 0 || d < 1 || chunk != 64) return 0;
+    return gdn_workspace_bytes((long)B * H, L, d, chunk, dt == HLTA_BF16);
+}
+
+hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *a,
+                               const float *b, void *o, const float *S0, float *S_out, int B,
+                               int H, long L, int d, int chunk, void *workspace,
+                               size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    hlta_status st = check_gdn_common(q, k, v, a, b, o, S0, S_out, d, chunk, dt);
+    if (st != HLTA_OK) return st;
+    if (B < 0 || H < 0 || L < 1 || L > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld", B, H, L);
+    size_t need = gdn_workspace_bytes((long)B * H, L, d, chunk, dt == HLTA_BF16);
+    if (!workspace || ws_bytes < need)
+        return fail(HLTA_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, ws_bytes);
+    if (((uintptr_t)workspace & 255u) != 0) return fail(HLTA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    GdnArgs g;
+    g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o;
+    g.B = B; g.Hg = H; g.Htot = H; g.h0 = 0; g.L = L; g.d = d; g.chunk = chunk;
+    g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
+    return run_gdn(g, dt, (cudaStream_t)stream);
+}
+
+size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk, hlta_dtype dt)
+{
+    if (B < 0 || Hg < 0 || T < 1 || N < 1 || d < 1 || chunk != 64) return 0;
+    return gdn_workspace_bytes((long)B * Hg, (long)T * N, d, chunk, dt == HLTA_BF16);
+}
+
+hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const float *a,
+                            const float *b, void *o, const float *S0, float *S_out, int B,
+                            int Hs, int Hd, int Hg, int T, int N, int d, int w_swa,
+                            int w_dswa, int r, int chunk, float scale, void *workspace,
+                            size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    hlta_status st;
+    if (B < 0 || Hs < 0 || Hd < 0 || Hg < 0 || T < 1 || N < 1)
+        return fail(HLTA_ERR_INVALID_ARG, "bad shape");
+    if ((long)T * N > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "T*N too large");
+    const int H = Hs + Hd + Hg;
+    if (!q || !k || !v || !o) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if ((st = check_dtype_d(dt, d)) != HLTA_OK) return st;
+    if (Hs && (st = check_window(w_swa, 1)) != HLTA_OK) return st;
+    if (Hd && (st = check_window(w_dswa, r)) != HLTA_OK) return st;
+    const long L = (long)T * N;
+    if (Hg) {
+        if ((st = check_gdn_common(q, k, v, a, b, o, S0, S_out, d, chunk, dt)) != HLTA_OK) return st;
+        size_t need = gdn_workspace_bytes((long)B * Hg, L, d, chunk, dt == HLTA_BF16);
+        if (!workspace || ws_bytes < need)
+            return fail(HLTA_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, ws_bytes);
+        if (((uintptr_t)workspace & 255u) != 0) return fail(HLTA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    }
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    // GDN heads on the auxiliary stream, ordered after everything already on `s`
+    if (Hg) {
+        std::lock_guard<std::mutex> lk(g_fork_mu);
+        if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        GdnArgs g;
+        g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o;
+        g.B = B; g.Hg = Hg; g.Htot = H; g.h0 = Hs + Hd; g.L = L; g.d = d; g.chunk = chunk;
+        g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
+        st = run_gdn(g, dt, ctx->aux);
+        // join even on failure so `s` never runs ahead of work that was enqueued
+        cudaEventRecord(ctx->join, ctx->aux);
+        cudaStreamWaitEvent(s, ctx->join, 0);
+        if (st != HLTA_OK) return st;
+    }
+    if (Hs) {
+        AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
+        if ((st = run_attn(a1, dt, s)) != HLTA_OK) return st;
+    }
+    if (Hd) {
+        AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
+        if ((st = run_attn(a2, dt, s)) != HLTA_OK) return st;
+    }
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N, int d,
+                               int w_swa, int w_dswa, int r, int chunk, float scale,
+                               hlta_dtype dt, const float *S0)
+{
+    hlta_status st;
+    if (!out) return fail(HLTA_ERR_INVALID_ARG, "null output handle");
+    *out = nullptr;
+    if (B < 1 || Hs < 0 || Hd < 0 || Hg < 0 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape");
+    if ((st = check_dtype_d(dt, d)) != HLTA_OK) return st;
+    if (Hs && (st = check_window(w_swa, 1)) != HLTA_OK) return st;
+    if (Hd && (st = check_window(w_dswa, r)) != HLTA_OK) return st;
+    if (Hg && chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
+    if (S0 && !aligned16(S0)) return fail(HLTA_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    hlta_stream *c = new (std::nothrow) hlta_stream();
+    if (!c) return fail(HLTA_ERR_CUDA, "host allocation failed");
+    cudaGetDevice(&c->device);
+    c->B = B; c->Hs = Hs; c->Hd = Hd; c->Hg = Hg; c->N = N; c->d = d;
+    c->w_swa = w_swa; c->w_dswa = w_dswa; c->r = r; c->chunk = chunk; c->dt = dt;
+    c->scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+    c->slots_s = Hs ? w_swa : 0;
+    c->slots_d = Hd ? r * (w_dswa - 1) + 1 : 0;
+    const size_t el = dt == HLTA_BF16 ? 2 : 4;
+    const size_t frame = (size_t)N * d * el;
+    size_t bs = (size_t)B * Hs * c->slots_s * frame, bd = (size_t)B * Hd * c->slots_d * frame;
+    c->ws_bytes = Hg ? gdn_workspace_bytes((long)B * Hg, N, d, chunk, dt == HLTA_BF16) : 0;
+    cudaError_t e = cudaSuccess;
+    if (bs && e == cudaSuccess) e = cudaMalloc(&c->ks, bs);
+    if (bs && e == cudaSuccess) e = cudaMalloc(&c->vs, bs);
+    if (bd && e == cudaSuccess) e = cudaMalloc(&c->kd, bd);
+    if (bd && e == cudaSuccess) e = cudaMalloc(&c->vd, bd);
+    if (Hg && e == cudaSuccess) e = cudaMalloc((void **)&c->S, (size_t)B * Hg * d * d * sizeof(float));
+    if (Hg && e == cudaSuccess) e = cudaMalloc(&c->ws, c->ws_bytes);
+    if (e == cudaSuccess && Hg) {
+        if (S0) e = cudaMemcpy(c->S, S0, (size_t)B * Hg * d * d * sizeof(float), cudaMemcpyDeviceToDevice);
+        else e = cudaMemset(c->S, 0, (size_t)B * Hg * d * d * sizeof(float));
+    }
+    if (e != cudaSuccess) {
+        hlta_stream_destroy(c);
+        return cuda_fail(e, "stream cache allocation");
+    }
+    c->frames = 0;
+    *out = c;
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_new,
+                             const void *v_new, const float *a_new, const float *b_new,
+                             void *o_new, void *stream)
+{
+    if (!c) return fail(HLTA_ERR_INVALID_ARG, "null cache");
+    if (!q_new || !k_new || !v_new || !o_new) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (c->Hg && (!a_new || !b_new)) return fail(HLTA_ERR_INVALID_ARG, "null gate pointer");
+    if (!aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(o_new) ||
+        (c->Hg && (!aligned16(a_new) || !aligned16(b_new))))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != c->device) return fail(HLTA_ERR_INVALID_ARG, "cache lives on device %d, current device is %d", c->device, dev);
+    hlta_status st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    const int H = c->Hs + c->Hd + c->Hg;
+    const int f = c->frames;
+    const size_t el = c->dt == HLTA_BF16 ? 2 : 4;
+    if (c->Hg) {
+        std::lock_guard<std::mutex> lk(g_fork_mu);
+        if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        GdnArgs g;
+        g.q = q_new; g.k = k_new; g.v = v_new; g.a = a_new; g.b = b_new; g.o = o_new;
+        g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = c->N; g.d = c->d;
+        g.chunk = c->chunk; g.S0 = c->S; g.S_out = c->S; g.ws = c->ws; g.ws_bytes = c->ws_bytes;
+        g.err = ctx->err;
+        st = run_gdn(g, c->dt, ctx->aux);
+        cudaEventRecord(ctx->join, ctx->aux);
+        cudaStreamWaitEvent(s, ctx->join, 0);
+        if (st != HLTA_OK) return st;
+    }
+    struct Branch { int h0, Hbr, slots, w, r; void *rk, *rv; } br[2] = {
+        {0, c->Hs, c->slots_s, c->w_swa, 1, c->ks, c->vs},
+        {c->Hs, c->Hd, c->slots_d, c->w_dswa, c->r, c->kd, c->vd}};
+    for (const Branch &x : br) {
+        if (!x.Hbr) continue;
+        const int slot = f % x.slots;
+        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rk, x.slots, slot, s)) != cudaSuccess)
+            return cuda_fail(e, "ring append");
+        if ((e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rv, x.slots, slot, s)) != cudaSuccess)
+            return cuda_fail(e, "ring append");
+        AttnArgs a;
+        a.q = q_new; a.k = x.rk; a.v = x.rv; a.o = o_new;
+        a.B = c->B; a.Hbr = x.Hbr;
+        a.q_Htot = H; a.q_h0 = x.h0; a.q_rows = c->N;
+        a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
+        a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.scale = c->scale;
+        a.err = ctx->err;
+        if ((st = run_attn(a, c->dt, s)) != HLTA_OK) return st;
+    }
+    c->frames = f + 1;
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done)
+{
+    if (!c) return fail(HLTA_ERR_INVALID_ARG, "null cache");
+    if (S_dev) *S_dev = c->S;
+    if (frames_done) *frames_done = c->frames;
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_destroy(hlta_stream_t c)
+{
+    if (!c) return HLTA_OK;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    cudaSetDevice(c->device);
+    cudaDeviceSynchronize();
+    void *bufs[] = {c->ks, c->vs, c->kd, c->vd, c->S, c->ws};
+    for (void *p : bufs)
+        if (p) cudaFree(p);
+    if (prev >= 0) cudaSetDevice(prev);
+    delete c;
+    return HLTA_OK;
+}
+
+hlta_status hlta_device_status(void *stream, unsigned int *code)
+{
+    hlta_status st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int word = 0, zero = 0;
+    if ((e = cudaMemcpy(&word, ctx->err, sizeof word, cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "read device error word");
+    if ((e = cudaMemcpy(ctx->err, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+        return cuda_fail(e, "clear device error word");
+    if (code) *code = word;
+    if (word) return fail(HLTA_ERR_TIMEOUT, "a kernel's bounded wait expired (device error word 0x%x)", word);
+    return HLTA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Internal declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace hlta {
+
+// Windowed softmax attention over frames. One description covers SWA (r = 1), DSWA and the
+// streaming step: queries are rows of a [B][q_Htot][q_rows][d] tensor (this branch's heads
+// start at q_h0); query row n lies in frame fq0 + n / N. Keys and values are rows of a
+// [B][kv_Htot][kv_rows][d] tensor; key frame fk occupies rows (fk % kv_slots) * N ...
+// (a clip when kv_slots covers every frame, a ring of frame slots when streaming).
+// The key frames of query frame f are f - r*i for i in [0, w), kept when >= 0.
+struct AttnArgs {
+    const void *q, *k, *v;
+    void *o;
+    int B, Hbr;
+    int q_Htot, q_h0;
+    long q_rows;
+    int kv_Htot, kv_h0;
+    long kv_rows;
+    int kv_slots;
+    int N, d, w, r;
+    int fq0;
+    float scale;
+    unsigned int *err;   // device error word (bounded waits that expired)
+};
+
+// Gated delta rule over [B][Htot][L][d] tensors, this branch's heads at h0 .. h0 + Hg.
+// Gates a, b: [B][Hg][L]. State: [B][Hg][d][d] (S[i][j], i value index, j key index).
+struct GdnArgs {
+    const void *q, *k, *v;
+    const float *a, *b;
+    void *o;
+    int B, Hg, Htot, h0;
+    long L;
+    int d, chunk;
+    const float *S0;
+    float *S_out;
+    void *ws;
+    size_t ws_bytes;
+    unsigned int *err;
+};
+
+// Chunk workspace (per GDN head, per chunk of C tokens; elements of type E):
+//   W  = T diag(b e^g) K,   Up = T diag(b) V,   Op = P Up,
+//   Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K        each [C][d]
+//   gam = e^{g_C}                                             one float per chunk
+// laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks].
+struct GdnWorkspace {
+    void *W, *Up, *Op, *Qt, *Kt;
+    float *gam;
+};
+
+__host__ __device__ inline long gdn_num_chunks(long L, int C) { return (L + C - 1) / C; }
+size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16);
+GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16);
+
+// Launchers. Return cudaGetLastError() of their launches.
+cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
+cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
+cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N,
+                               int d, size_t elem, void *ring, int slots, int slot,
+                               cudaStream_t s);
+
+// Device error word: kernels OR a code into it when a bounded wait expires.
+enum : unsigned int {
+    DEVERR_ATTN_WAIT = 1u << 0,
+    DEVERR_GDN_WAIT = 1u << 1,
+};
+unsigned int *device_error_word();  // device address of the word (current device)
+
+}  // namespace hlta

@@ -1,0 +1,82 @@
+"""CPU-only checks of the C ABI: the library loads, exports every entry point that
+include/hlta.h declares, and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hlta.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hlta_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import linear_video_world_b200 as h
+    return h._lib
+
+
+def test_header_declares_the_documented_calls():
+    names = _declared()
+    for n in ("hlta_swa_fwd", "hlta_dswa_fwd", "hlta_gdn_chunk_fwd", "hlta_hybrid_fwd",
+              "hlta_stream_create", "hlta_stream_step", "hlta_stream_destroy", "hlta_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version(lib):
+    assert lib.hlta_version() >= 100
+
+
+def test_null_pointers_rejected_on_host(lib):
+    import linear_video_world_b200 as h
+    st = lib.hlta_swa_fwd(None, None, None, None, 1, 1, 2, 16, 128, 2, 0.0, h.HLTA_BF16, None)
+    assert st == h.HLTA_ERR_INVALID_ARG
+    assert b"null" in lib.hlta_last_error()
+
+
+def test_bad_shapes_rejected_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    assert lib.hlta_swa_fwd(p, p, p, p, 1, 1, 0, 16, 128, 2, 0.0, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_swa_fwd(p, p, p, p, 1, 1, 2, 16, 64, 2, 0.0, h.HLTA_BF16, None) == h.HLTA_ERR_UNSUPPORTED
+    assert lib.hlta_dswa_fwd(p, p, p, p, 1, 1, 2, 16, 128, 2, 0, 0.0, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_dswa_fwd(p, p, p, p, 1, 1, 2, 16, 128, 0, 2, 0.0, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_swa_fwd(p, p, p, ctypes.c_void_p(264), 1, 1, 2, 16, 128, 2, 0.0, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_swa_fwd(p, p, p, p, 1, 1, 2, 16, 129, 2, 0.0, h.HLTA_FP32, None) == h.HLTA_ERR_UNSUPPORTED
+    # gated delta rule: chunk other than 64 and a short workspace
+    assert lib.hlta_gdn_chunk_fwd(p, p, p, p, p, p, None, None, 1, 1, 100, 128, 32, p, 1 << 30,
+                                  h.HLTA_BF16, None) == h.HLTA_ERR_UNSUPPORTED
+    assert lib.hlta_gdn_chunk_fwd(p, p, p, p, p, p, None, None, 1, 1, 100, 128, 64, p, 16,
+                                  h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert b"workspace" in lib.hlta_last_error()
+
+
+def test_workspace_sizes(lib):
+    import linear_video_world_b200 as h
+    # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16 plus one float per chunk
+    n = h.hlta_gdn_workspace_bytes(1, 8, 32760, 128, 64, h.HLTA_BF16)
+    nch = (32760 + 63) // 64
+    arr = 8 * nch * 64 * 128 * 2
+    assert n == 5 * arr + ((8 * nch * 4 + 255) // 256) * 256
+    assert h.hlta_hybrid_workspace_bytes(1, 8, 21, 1560, 128, 64, h.HLTA_BF16) == n
+    assert h.hlta_gdn_workspace_bytes(1, 1, 10, 64, 64, h.HLTA_FP32) > 5 * 64 * 64 * 4 - 1
+
+
+def test_stream_create_validates_before_allocating(lib):
+    import linear_video_world_b200 as h
+    out = ctypes.c_void_p()
+    assert lib.hlta_stream_create(ctypes.byref(out), 0, 1, 1, 1, 16, 128, 3, 4, 6, 64, 0.0,
+                                  h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_stream_create(ctypes.byref(out), 1, 1, 1, 1, 16, 128, 3, 4, 6, 32, 0.0,
+                                  h.HLTA_BF16, None) == h.HLTA_ERR_UNSUPPORTED
+    assert out.value is None
