@@ -1,0 +1,380 @@
+#!/usr/bin/env python
+"""Benchmark: hybrid linear temporal attention forward on B200, 480P workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one call of hlta_hybrid_fwd over one 480P clip (B=1, 24 heads split 8 SWA / 8 DSWA
+/ 8 GDN, d=128, T=21 frames of N=1560 tokens, L=32760), i.e. every branch of the operator on
+one batch of seeded synthetic inputs already resident in HBM. `value` is tokens/s (B*L per
+step, summed over ranks). The q/k/v inputs (603 MB) are larger than the 126 MB L2, so no L2
+flush is done between steps.
+
+Under torchrun with N > 1 ranks every rank runs an independent replica on its own GPU with
+its own inputs (the operator has no exchange step between GPUs); the timing is taken on the
+device, bracketed by barriers, and reduced as the max over ranks.
+
+`--impl reference` times the CPU oracle (oracle/, fp64 plain definitions) on the host cores,
+on bounded samples of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hybrid temporal attention fwd tokens/s @480P; % of bf16 tensor / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="480p")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------
+# work accounting (algorithmic: valid query-key pairs at 4*d FLOP, GDN q/k/v/o + gate bytes)
+# ------------------------------------------------------------------------------------------
+def window_pairs(T: int, N: int, w: int, r: int) -> int:
+    frames = 0
+    for f in range(T):
+        frames += sum(1 for i in range(w) if f - r * i >= 0)
+    return frames * N * N
+
+
+def work(wl):
+    ps = window_pairs(wl.T, wl.N, wl.w_swa, 1) * wl.B * wl.Hs
+    pd = window_pairs(wl.T, wl.N, wl.w_dswa, wl.r) * wl.B * wl.Hd
+    gdn_bytes = wl.B * wl.Hg * wl.L * (4 * wl.d * 2 + 2 * 4)
+    return {"swa_flop": 4 * wl.d * ps, "dswa_flop": 4 * wl.d * pd, "gdn_bytes": gdn_bytes}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_record(kernel_src: str):
+    """DRAM bytes per launch from a committed ncu summary, valid only for the same source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "linear_video_world_b200", "csrc", kernel_src), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        r = rec.get(kernel_src)
+        if r and r.get("src_sha") == sha:
+            return r
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu_index],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ------------------------------------------------------------------------------------------
+def oracle_sample(x, wl, rows: int, seed: int):
+    """Time the oracle on `rows` query positions of every softmax head plus `rows`
+    consecutive tokens of every GDN head; returns (tokens, seconds)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    g = torch.Generator().manual_seed(seed)
+    pos = torch.randint(0, wl.L, (rows,), generator=g).numpy()
+    q, k, v = (x[n][0] for n in "qkv")          # [H, L, d], batch 0
+    Hs, Hd, Hg = wl.Hs, wl.Hd, wl.Hg
+    t0 = time.perf_counter()
+    if Hs:
+        flat = (np.arange(Hs)[:, None] * wl.L + pos[None, :]).reshape(-1)
+        oracle.swa(q[:Hs], k[:Hs], v[:Hs], wl.T, wl.N, wl.w_swa, rows=flat)
+    if Hd:
+        flat = (np.arange(Hd)[:, None] * wl.L + pos[None, :]).reshape(-1)
+        s = slice(Hs, Hs + Hd)
+        oracle.dswa(q[s], k[s], v[s], wl.T, wl.N, wl.w_dswa, wl.r, rows=flat)
+    if Hg:
+        s = slice(Hs + Hd, Hs + Hd + Hg)
+        oracle.gdn(q[s, :rows], k[s, :rows], v[s, :rows], x["a"][0, :, :rows], x["b"][0, :, :rows])
+    return rows, time.perf_counter() - t0
+
+
+def calibrated_rows(x, wl, seconds: float, seed: int) -> int:
+    n0 = 16
+    _, t = oracle_sample(x, wl, n0, seed)
+    return max(n0, int(n0 * seconds / max(t, 1e-3)))
+
+
+def cpu_baseline(x, wl, seconds: float):
+    import oracle
+    oracle.build()
+    rows = calibrated_rows(x, wl, seconds, seed=123)
+    tokens, sec = oracle_sample(x, wl, rows, seed=124)
+    return {"value": tokens * wl.B / sec, "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"{rows} random query positions of the 480P clip on all {wl.Hs + wl.Hd} "
+                       f"softmax heads (explicit fp64 softmax) plus {rows} consecutive tokens of "
+                       f"all {wl.Hg} GDN heads (fp64 token recurrence); {sec:.1f} s")}
+
+
+def run_reference(args, wl):
+    import hlta_inputs as hi
+    import oracle
+    oracle.build()
+    x = hi.make_inputs(wl, seed=0)
+    budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))   # CPU seconds per step
+    rows = calibrated_rows(x, wl, max(0.5, budget), seed=7)
+    for i in range(args.warmup):
+        oracle_sample(x, wl, rows, seed=1000 + i)
+    times = []
+    for i in range(args.steps):
+        _, sec = oracle_sample(x, wl, rows, seed=2000 + i)
+        times.append(sec)
+    total = sum(times)
+    value = rows * wl.B * args.steps / total
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: {rows} random query positions on every softmax "
+                                   f"head plus {rows} GDN tokens on every GDN head"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl):
+    return {"workload": f"{wl.name}: B={wl.B} heads {wl.Hs}/{wl.Hd}/{wl.Hg} (SWA/DSWA/GDN) d={wl.d} "
+                        f"T={wl.T} N={wl.N} L={wl.L} SWA w={wl.w_swa} DSWA w={wl.w_dswa} r={wl.r} "
+                        f"GDN chunk {wl.chunk}",
+            "global_batch": wl.B, "seq_len": wl.L, "parallelism": "replicas",
+            "l2": "inputs larger than L2 (q,k,v 603 MB vs 126 MB); no flush between steps"}
+
+
+# ------------------------------------------------------------------------------------------
+def main():
+    args = parse_args()
+    import hlta_inputs as hi
+    wl = hi.WORKLOADS[args.workload]
+    assert not wl.streaming, "bench workloads: 480p, 480p_long, 720p_long, tiny_fp32"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import linear_video_world_b200 as h
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def allmax(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    x = hi.make_inputs(wl, seed=rank)
+    q, k, v, a, b = (x[n].to(dev) for n in "qkvab")
+    o = torch.empty_like(q)
+    S_out = torch.empty((wl.B, wl.Hg, wl.d, wl.d), device=dev, dtype=torch.float32)
+    ws = torch.empty(h.hlta_hybrid_workspace_bytes(wl.B, wl.Hg, wl.T, wl.N, wl.d, wl.chunk,
+                                                   h.HLTA_BF16 if wl.dtype == "bf16" else h.HLTA_FP32),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        h.hlta_hybrid_fwd(q, k, v, a, b, o, None, S_out, wl.B, wl.Hs, wl.Hd, wl.Hg, wl.T, wl.N,
+                          wl.d, wl.w_swa, wl.w_dswa, wl.r, wl.chunk, 0.0, ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+
+    # ---- device-resident timed region -----------------------------------------------------
+    K = args.steps
+    prof = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    gpu_index = vis.split(",")[local_rank] if vis else str(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(gpu_index)
+    time.sleep(0.3)
+    ev0.record()
+    for i in range(K):
+        h.hlta_set_profile_events(prof[i])
+        step()
+    ev1.record()
+    torch.cuda.synchronize()
+    h.hlta_set_profile_events(None)
+    barrier()
+    clocks = clk.stop()
+    total_ms = allmax(ev0.elapsed_time(ev1))
+    ms = total_ms / K
+    swa_ms = statistics.mean(p[0].elapsed_time(p[1]) for p in prof)
+    dswa_ms = statistics.mean(p[1].elapsed_time(p[2]) for p in prof)
+    gdn_ms = statistics.mean(p[3].elapsed_time(p[4]) for p in prof)
+    assert h.hlta_device_status() == 0
+    tokens = wl.B * wl.L
+    value = tokens * world / (ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers -----------------------------------
+    pin = {n: x[n].pin_memory() for n in "qkvab"}
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    S_host = torch.empty(S_out.shape, dtype=S_out.dtype, pin_memory=True)
+    dev_in = {"q": q, "k": k, "v": v, "a": a, "b": b}
+
+    def e2e_step():
+        for n in "qkvab":
+            dev_in[n].copy_(pin[n], non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S_out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(K):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = allmax(e0.elapsed_time(e1)) / K
+    h2d = sum(pin[n].numel() * pin[n].element_size() for n in "qkvab")
+    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
+
+    # ---- roofline of the dominant kernel (windowed attention, both launches) --------------
+    wk = work(wl)
+    pk, pk_kind = peaks()
+    attn_flop = wk["swa_flop"] + wk["dswa_flop"]
+    attn_ms = swa_ms + dswa_ms
+    achieved = attn_flop / (attn_ms / 1e3) / 1e12
+    peak = float(pk.get("bf16_tflops_sustained", pk.get("bf16_tflops")))
+    tr = traffic_record("attn_tc.cu")
+    roofline = {"bound": "tensor", "kernel": "attn_tc_kernel (SWA + DSWA launches)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": f"{pk_kind} bf16 dense, sustained (kernel timed inside a long step)",
+                "traffic": (tr["swa_bytes"] + tr["dswa_bytes"]) if tr else None}
+    hbm = float(pk.get("hbm_gbs"))
+    gdn_gbs = wk["gdn_bytes"] / (gdn_ms / 1e3) / 1e9
+    detail = {
+        "swa_ms": swa_ms, "dswa_ms": dswa_ms, "gdn_ms": gdn_ms,
+        "swa_tflops": wk["swa_flop"] / (swa_ms / 1e3) / 1e12,
+        "dswa_tflops": wk["dswa_flop"] / (dswa_ms / 1e3) / 1e12,
+        "gdn_gbs": gdn_gbs, "gdn_hbm_frac": gdn_gbs / hbm,
+        "hbm_peak_gbs": hbm, "hbm_peak_kind": pk_kind,
+        "note": "GDN runs on a second stream concurrently with SWA/DSWA; its HBM fraction "
+                "uses the algorithmic q/k/v/o + gate bytes of the 8 GDN heads",
+    }
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, per-rank seed)",
+        "config": config_of(wl), "clocks": clocks,
+        "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * K, "roofline": roofline, "detail": detail,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x, wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -165,6 +165,16 @@ hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done);
 hlta_status hlta_stream_destroy(hlta_stream_t c);
 
 /*
+ * Profiling hook for hlta_hybrid_fwd (measurement, not needed for results). `events` is NULL
+ * (off) or an array of 5 cudaEvent_t created by the caller on the current device. While set,
+ * each hlta_hybrid_fwd call records events[0] before its SWA kernel, events[1] between the
+ * SWA and DSWA kernels and events[2] after the DSWA kernel (all on the caller's stream),
+ * events[3] before and events[4] after the GDN kernels (on the GDN stream). The array is
+ * copied; the setting is process-wide and stays until changed.
+ */
+hlta_status hlta_set_profile_events(void *const *events);
+
+/*
  * Synchronizes `stream`, then reads and clears the library's device error word.
  * *code receives the raw word (0: no kernel stopped early). Returns HLTA_ERR_TIMEOUT if a
  * bounded wait expired in any kernel since the last call, HLTA_ERR_CUDA on a CUDA error.

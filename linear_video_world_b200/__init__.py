@@ -32,7 +32,7 @@ class HltaError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m linear_video_world_b200.build` (nvcc, sm_100a)")
+                          "`python linear_video_world_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, L, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_float, ctypes.c_size_t
     sig = {
@@ -50,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
+        "hlta_set_profile_events": (I, [ctypes.POINTER(P)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -142,6 +143,15 @@ def hlta_device_status(stream=None) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
     return int(code.value)
+
+
+def hlta_set_profile_events(events):
+    """events: None, or 5 torch.cuda.Event objects (already created on the device)."""
+    if events is None:
+        _check(_lib.hlta_set_profile_events(None))
+        return
+    arr = (ctypes.c_void_p * 5)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _check(_lib.hlta_set_profile_events(arr))
 
 
 # ---- convenience wrappers (allocate with torch, then call the entry points) ----------

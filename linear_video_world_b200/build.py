@@ -1,6 +1,7 @@
 """Build the CUDA library in-tree: linear_video_world_b200/libhlta.so (sm_100a only).
 
-Usage: python -m linear_video_world_b200.build [--force] [--verbose-ptxas]
+Usage: python linear_video_world_b200/build.py [--force] [--verbose-ptxas]
+(run by path: importing the package first would load the library being rebuilt)
 """
 from __future__ import annotations
 

@@ -1,4 +1,526 @@
+// Gated delta rule, chunkwise form, bf16 in / bf16 out, fp32 accumulation and fp32 state.
+//
+// Chunk algebra (derived from S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T; the
+// chunkwise split is the "parallel within a block, recurrent across blocks" form of the
+// llm-atlas long-context explainer, sections 06 and 09). For a chunk of n <= 64 tokens with
+// incoming state S0 and g_t = sum_{s<=t} log a_s within the chunk:
+//   A_ti = b_t e^{g_t-g_i} k_t.k_i (i < t),    T = (I + A)^{-1}          (UT transform)
+//   W  = T diag(b e^g) K,  Up = T diag(b) V,   P_ti = e^{g_t-g_i} q_t.k_i (i <= t)
+//   Op = P Up,  Qt = diag(e^g) Q - P W,  Kt = diag(e^{g_n-g}) K,  gam = e^{g_n}
+//   U = Up - W S0^T,   O = Op + Qt S0^T,   S_n = gam S0 + U^T Kt.
+// Only decays e^{g_t-g_i} with t >= i are formed, so nothing overflows.
+//
+// Two kernels:
+//   prep   one CTA per (chunk, head), every chunk in parallel: KK^T, QK^T, the forward
+//          substitution for T (fp32), then W, Up, Op, Qt on mma.sync bf16 tensor cores;
+//          writes W, Up, Op, Qt, Kt (bf16) and gam (fp32) to the workspace.
+//   state  serial over the chunks of a head; the 128 state rows are split over 8 CTAs of
+//          16 rows (rows of S evolve independently). The state slice lives in registers as
+//          the accumulator fragments of the S update; each chunk does two dependent small
+//          GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync, with the next chunk's operands
+//          prefetched by cp.async.
+// The serial chain is latency-bound (two dependent 64x16x128-class products per chunk), so
+// it uses register-resident warp MMAs rather than a TMEM round trip per dependent step.
 #include "hlta_internal.cuh"
+
+#include <math.h>
+
 namespace hlta {
-cudaError_t launch_gdn_bf16(const GdnArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int C = 64;             // chunk length
+constexpr int D = 128;            // head dim
+constexpr int SD = D + 8;         // padded smem row stride (elements) of [.][128] bf16 tiles
+constexpr int SC = C + 8;         // padded smem row stride of [.][64] bf16 tiles
+constexpr int FP = C + 1;         // fp32 [64][65] tiles
+constexpr int THREADS = 128;
+constexpr int RB = 16;            // state rows per CTA in the state pass
+constexpr int SR = RB + 8;        // padded stride of [64][16] slices
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
 }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += a * b (m16n8k16, bf16 operands, fp32 accumulate)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// A fragment (16x16) of a row-major [M][K] bf16 tile with row stride `ld` (elements)
+__device__ __forceinline__ void frag_a(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld, int m0,
+                                       int k0, int lane)
+{
+    const int q = lane >> 3, rr = lane & 7;
+    ldsm_x4(r, smem_u32(base + (m0 + (q & 1) * 8 + rr) * ld + k0 + (q >> 1) * 8));
+}
+
+// A fragment (16x16, rows m, cols k) taken from a [K][M] row-major tile (transposed load)
+__device__ __forceinline__ void frag_a_t(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
+                                         int m0, int k0, int lane)
+{
+    const int q = lane >> 3, rr = lane & 7;
+    ldsm_x4_t(r, smem_u32(base + (k0 + (q >> 1) * 8 + rr) * ld + m0 + (q & 1) * 8));
+}
+
+// B fragments of two adjacent n-tiles (k16 x n16) from a [N][K] row-major tile:
+// r[0], r[1] = n-tile n0, r[2], r[3] = n-tile n0 + 8
+__device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
+                                          int n0, int k0, int lane)
+{
+    ldsm_x4(r, smem_u32(base + (n0 + (lane >> 4) * 8 + (lane & 7)) * ld + k0 + ((lane >> 3) & 1) * 8));
+}
+
+// B fragments of two adjacent n-tiles from a [K][N] row-major tile (transposed load)
+__device__ __forceinline__ void frag_b_kn(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
+                                          int k0, int n0, int lane)
+{
+    ldsm_x4_t(r, smem_u32(base + (k0 + ((lane >> 3) & 1) * 8 + (lane & 7)) * ld + n0 + (lane >> 4) * 8));
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void st_pair(__nv_bfloat16 *p, float lo, float hi)
+{
+    *reinterpret_cast<uint32_t *>(p) = pack2(lo, hi);
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// -----------------------------------------------------------------------------------------
+// prep
+// -----------------------------------------------------------------------------------------
+struct PrepSmem {
+    __nv_bfloat16 Q[C * SD], K[C * SD], V[C * SD], W[C * SD], U[C * SD];
+    __nv_bfloat16 P[C * SC], T1[C * SC], T2[C * SC];
+    float A[C * FP], T[C * FP];
+    float g[C], bb[C];
+};
+
+// One warp's 16 rows x (2*npairs*8) columns of X = Amat (row-major [64][ldA]) * Bmat ([K][N]
+// row-major, transposed fragment loads), k-steps 0..ksteps-1.
+template <int NT>
+__device__ __forceinline__ void gemm_rows_kn(float (&acc)[NT][4], const __nv_bfloat16 *Am, int lda,
+                                             const __nv_bfloat16 *Bm, int ldb, int m0, int ksteps,
+                                             int lane)
+{
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    for (int kk = 0; kk < ksteps; ++kk) {
+        uint32_t a[4];
+        frag_a(a, Am, lda, m0, kk * 16, lane);
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+            uint32_t b[4];
+            frag_b_kn(b, Bm, ldb, kk * 16, np * 16, lane);
+            mma16816(acc[2 * np], a, b[0], b[1]);
+            mma16816(acc[2 * np + 1], a, b[2], b[3]);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace ws)
+{
+    extern __shared__ uint8_t smem_raw[];
+    PrepSmem &s = *reinterpret_cast<PrepSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / p.Hg, h = bh % p.Hg;
+    const long nch = gdn_num_chunks(p.L, C);
+    const long t0 = (long)chunk * C;
+    const int n = (int)min((long)C, p.L - t0);
+    const long head = (long)(b * p.Htot + p.h0 + h) * p.L;
+    const uint4 *gq = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.q + (head + t0) * D);
+    const uint4 *gk = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.k + (head + t0) * D);
+    const uint4 *gv = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.v + (head + t0) * D);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, tg = lane & 3;
+
+    // ---- load the chunk (rows >= n are zero) and the gates
+    for (int e = tid; e < C * (D / 8); e += THREADS) {
+        const int t = e / (D / 8), c8 = e % (D / 8);
+        uint4 zq = make_uint4(0, 0, 0, 0), zk = zq, zv = zq;
+        if (t < n) {
+            zq = gq[(long)t * (D / 8) + c8];
+            zk = gk[(long)t * (D / 8) + c8];
+            zv = gv[(long)t * (D / 8) + c8];
+        }
+        *reinterpret_cast<uint4 *>(&s.Q[t * SD + c8 * 8]) = zq;
+        *reinterpret_cast<uint4 *>(&s.K[t * SD + c8 * 8]) = zk;
+        *reinterpret_cast<uint4 *>(&s.V[t * SD + c8 * 8]) = zv;
+    }
+    if (tid < C) {
+        const float av = tid < n ? p.a[(long)bh * p.L + t0 + tid] : 1.f;
+        s.g[tid] = tid < n ? logf(av) : 0.f;
+        s.bb[tid] = tid < n ? p.b[(long)bh * p.L + t0 + tid] : 0.f;
+    }
+    __syncthreads();
+    // inclusive prefix sum of log a (Hillis-Steele over 64 entries)
+    for (int off = 1; off < C; off <<= 1) {
+        float v = 0.f;
+        if (tid < C && tid >= off) v = s.g[tid - off];
+        __syncthreads();
+        if (tid < C) s.g[tid] += v;
+        __syncthreads();
+    }
+
+    // ---- KK^T and QK^T for this warp's 16 rows; only columns i <= t are needed
+    {
+        const int m0 = warp * 16;
+        const int ntiles = 2 * warp + 2;      // column tiles 0 .. 2w+1 cover i <= 16w+15
+        float kk[8][4], qk[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) kk[nt][e] = qk[nt][e] = 0.f;
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t ak[4], aq[4];
+            frag_a(ak, s.K, SD, m0, ks * 16, lane);
+            frag_a(aq, s.Q, SD, m0, ks * 16, lane);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                if (2 * np < ntiles) {
+                    uint32_t bk[4];
+                    frag_b_nk(bk, s.K, SD, np * 16, ks * 16, lane);
+                    mma16816(kk[2 * np], ak, bk[0], bk[1]);
+                    mma16816(kk[2 * np + 1], ak, bk[2], bk[3]);
+                    mma16816(qk[2 * np], aq, bk[0], bk[1]);
+                    mma16816(qk[2 * np + 1], aq, bk[2], bk[3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = m0 + g8 + (e >> 1) * 8;
+                const int i = nt * 8 + 2 * tg + (e & 1);
+                const bool lower = i <= t && t < n;
+                const float dec = lower ? expf(s.g[t] - s.g[i]) : 0.f;
+                s.A[t * FP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
+                s.P[t * SC + i] = __float2bfloat16_rn(lower ? dec * qk[nt][e] : 0.f);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^{-1}: forward substitution, one thread per column (fp32)
+    if (tid < C) {
+        const int j = tid;
+        for (int t = 0; t <= j; ++t) s.T[t * FP + j] = t == j ? 1.f : 0.f;
+        for (int t = j + 1; t < C; ++t) {
+            float a0 = 0.f, a1 = 0.f;
+            int i = j;
+            for (; i + 1 < t; i += 2) {
+                a0 = fmaf(s.A[t * FP + i], s.T[i * FP + j], a0);
+                a1 = fmaf(s.A[t * FP + i + 1], s.T[(i + 1) * FP + j], a1);
+            }
+            if (i < t) a0 = fmaf(s.A[t * FP + i], s.T[i * FP + j], a0);
+            s.T[t * FP + j] = -(a0 + a1);
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += THREADS) {
+        const int t = e / C, i = e % C;
+        const float tv = s.T[t * FP + i];
+        s.T1[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i] * expf(s.g[i]));
+        s.T2[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i]);
+    }
+    __syncthreads();
+
+    const int m0 = warp * 16;
+    const int ksteps = warp + 1;              // T1, T2, P are lower triangular
+    // ---- W = T1 K, Up = T2 V  (kept in smem as bf16)
+    {
+        float acc[16][4];
+        gemm_rows_kn<16>(acc, s.T1, SC, s.K, SD, m0, ksteps, lane);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = nt * 8 + 2 * tg;
+            st_pair(&s.W[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
+            st_pair(&s.W[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
+        }
+        gemm_rows_kn<16>(acc, s.T2, SC, s.V, SD, m0, ksteps, lane);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = nt * 8 + 2 * tg;
+            st_pair(&s.U[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
+            st_pair(&s.U[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
+        }
+    }
+    __syncthreads();
+    // ---- Op = P Up (into the V buffer), Qt = e^g Q - P W (in place over Q)
+    {
+        float acc[16][4];
+        gemm_rows_kn<16>(acc, s.P, SC, s.U, SD, m0, ksteps, lane);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = nt * 8 + 2 * tg;
+            st_pair(&s.V[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
+            st_pair(&s.V[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
+        }
+        gemm_rows_kn<16>(acc, s.P, SC, s.W, SD, m0, ksteps, lane);
+        const int ta = m0 + g8, tb = ta + 8;
+        const float ea = ta < n ? expf(s.g[ta]) : 0.f, eb = tb < n ? expf(s.g[tb]) : 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = nt * 8 + 2 * tg;
+            __nv_bfloat16 *qa = &s.Q[ta * SD + c], *qb = &s.Q[tb * SD + c];
+            const float qa0 = __bfloat162float(qa[0]), qa1 = __bfloat162float(qa[1]);
+            const float qb0 = __bfloat162float(qb[0]), qb1 = __bfloat162float(qb[1]);
+            st_pair(qa, ta < n ? ea * qa0 - acc[nt][0] : 0.f, ta < n ? ea * qa1 - acc[nt][1] : 0.f);
+            st_pair(qb, tb < n ? eb * qb0 - acc[nt][2] : 0.f, tb < n ? eb * qb1 - acc[nt][3] : 0.f);
+        }
+    }
+    __syncthreads();
+
+    // ---- write W, Up, Op, Qt, Kt and gam
+    const long base = ((long)bh * nch + chunk) * C * D;
+    uint4 *oW = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.W + base);
+    uint4 *oU = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Up + base);
+    uint4 *oO = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Op + base);
+    uint4 *oQ = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Qt + base);
+    uint4 *oK = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Kt + base);
+    const float gn = s.g[n - 1];
+    for (int e = tid; e < C * (D / 8); e += THREADS) {
+        const int t = e / (D / 8), c8 = e % (D / 8);
+        const int so = t * SD + c8 * 8;
+        oW[e] = *reinterpret_cast<const uint4 *>(&s.W[so]);
+        oU[e] = *reinterpret_cast<const uint4 *>(&s.U[so]);
+        oO[e] = *reinterpret_cast<const uint4 *>(&s.V[so]);
+        oQ[e] = *reinterpret_cast<const uint4 *>(&s.Q[so]);
+        const float dk = t < n ? expf(gn - s.g[t]) : 0.f;
+        uint4 kv = *reinterpret_cast<const uint4 *>(&s.K[so]);
+        __nv_bfloat162 *k2 = reinterpret_cast<__nv_bfloat162 *>(&kv);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float2 f = __bfloat1622float2(k2[u]);
+            k2[u] = __floats2bfloat162_rn(f.x * dk, f.y * dk);
+        }
+        oK[e] = kv;
+    }
+    if (tid == 0) ws.gam[(long)bh * nch + chunk] = expf(gn);
+}
+
+// -----------------------------------------------------------------------------------------
+// state pass
+// -----------------------------------------------------------------------------------------
+struct StateBuf {
+    __nv_bfloat16 W[C * SD], Q[C * SD], K[C * SD];   // W, Qt, Kt of one chunk
+    __nv_bfloat16 U[C * SR], O[C * SR];              // this CTA's 16 columns of Up, Op
+};
+struct StateSmem {
+    StateBuf buf[2];
+    __nv_bfloat16 Sb[RB * SD];                       // state slice as bf16 [i][j]
+    __nv_bfloat16 Ut[RB * SC];                       // U^T slice [i][t]
+    __nv_bfloat16 Os[C * SR];                        // output staging [t][i]
+    float gam[2];
+};
+
+__device__ __forceinline__ void load_chunk(StateBuf &bf, const GdnWorkspace &ws, int bh, long nch,
+                                           long c, int i0, int tid)
+{
+    const long base = ((long)bh * nch + c) * C * D;
+    const __nv_bfloat16 *W = (const __nv_bfloat16 *)ws.W + base;
+    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)ws.Qt + base;
+    const __nv_bfloat16 *K = (const __nv_bfloat16 *)ws.Kt + base;
+    const __nv_bfloat16 *U = (const __nv_bfloat16 *)ws.Up + base;
+    const __nv_bfloat16 *O = (const __nv_bfloat16 *)ws.Op + base;
+    for (int e = tid; e < C * (D / 8); e += THREADS) {
+        const int t = e / (D / 8), c8 = e % (D / 8);
+        cp_async16(&bf.W[t * SD + c8 * 8], W + (long)t * D + c8 * 8);
+        cp_async16(&bf.Q[t * SD + c8 * 8], Q + (long)t * D + c8 * 8);
+        cp_async16(&bf.K[t * SD + c8 * 8], K + (long)t * D + c8 * 8);
+    }
+    for (int e = tid; e < C * 2; e += THREADS) {
+        const int t = e >> 1, hlf = e & 1;
+        cp_async16(&bf.U[t * SR + hlf * 8], U + (long)t * D + i0 + hlf * 8);
+        cp_async16(&bf.O[t * SR + hlf * 8], O + (long)t * D + i0 + hlf * 8);
+    }
+}
+
+__global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspace ws)
+{
+    extern __shared__ uint8_t smem_raw[];
+    StateSmem &s = *reinterpret_cast<StateSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    const int i0 = blockIdx.x * RB, bh = blockIdx.y;
+    const int b = bh / p.Hg, h = bh % p.Hg;
+    const long nch = gdn_num_chunks(p.L, C);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, tg = lane & 3;
+    __nv_bfloat16 *o = (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D;
+
+    // state fragments: this warp owns key columns j in [32w, 32w+32) of S^T = D[m=j][n=i]
+    float st[2][2][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
+                const int i = nt * 8 + 2 * tg + (e & 1);
+                st[mt][nt][e] = p.S0 ? p.S0[((long)bh * D + i0 + i) * D + j] : 0.f;
+                s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
+            }
+
+    load_chunk(s.buf[0], ws, bh, nch, 0, i0, tid);
+    cp_async_commit();
+    for (long c = 0; c < nch; ++c) {
+        StateBuf &cur = s.buf[c & 1];
+        cp_async_wait<0>();
+        __syncthreads();                       // chunk c landed; Sb holds the incoming state
+        if (c + 1 < nch) load_chunk(s.buf[(c + 1) & 1], ws, bh, nch, c + 1, i0, tid);
+        cp_async_commit();
+        const float gam = ws.gam[(long)bh * nch + c];
+
+        // GEMM 1: rows [W; Qt] (warps 0-1: W rows, warps 2-3: Qt rows) times S^T
+        {
+            const __nv_bfloat16 *Am = warp < 2 ? cur.W : cur.Q;
+            const int mb = (warp & 1) * 32;
+            float acc[2][2][4];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t bsf[4];
+                frag_b_nk(bsf, s.Sb, SD, 0, ks * 16, lane);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    uint32_t a[4];
+                    frag_a(a, Am, SD, mb + mt * 16, ks * 16, lane);
+                    mma16816(acc[mt][0], a, bsf[0], bsf[1]);
+                    mma16816(acc[mt][1], a, bsf[2], bsf[3]);
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = mb + mt * 16 + g8 + (e >> 1) * 8;
+                        const int i = nt * 8 + 2 * tg + (e & 1);
+                        if (warp < 2) {
+                            const float u = __bfloat162float(cur.U[t * SR + i]) - acc[mt][nt][e];
+                            s.Ut[i * SC + t] = __float2bfloat16_rn(u);
+                        } else {
+                            const float ov = __bfloat162float(cur.O[t * SR + i]) + acc[mt][nt][e];
+                            s.Os[t * SR + i] = __float2bfloat16_rn(ov);
+                        }
+                    }
+        }
+        __syncthreads();                       // Ut and Os complete
+
+        // outputs of this chunk: 64 rows x 16 columns
+        {
+            const long t0 = c * C;
+            const int t = tid >> 1, hlf = tid & 1;
+            if (t0 + t < p.L)
+                *reinterpret_cast<uint4 *>(o + (t0 + t) * D + i0 + hlf * 8) =
+                    *reinterpret_cast<const uint4 *>(&s.Os[t * SR + hlf * 8]);
+        }
+        // GEMM 2: S^T <- gam S^T + Kt^T U   (D[m=j][n=i] = sum_t Kt[t][j] U[t][i])
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) st[mt][nt][e] *= gam;
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+            uint32_t bu[4];
+            frag_b_nk(bu, s.Ut, SC, 0, ks * 16, lane);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                uint32_t a[4];
+                frag_a_t(a, cur.K, SD, warp * 32 + mt * 16, ks * 16, lane);
+                mma16816(st[mt][0], a, bu[0], bu[1]);
+                mma16816(st[mt][1], a, bu[2], bu[3]);
+            }
+        }
+        // bf16 copy of the new state for the next chunk's GEMM 1 (made visible by the
+        // barrier at the top of the loop)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
+                    const int i = nt * 8 + 2 * tg + (e & 1);
+                    s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
+                }
+    }
+    cp_async_wait<0>();
+    if (p.S_out) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
+                    const int i = nt * 8 + 2 * tg + (e & 1);
+                    p.S_out[((long)bh * D + i0 + i) * D + j] = st[mt][nt][e];
+                }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
+{
+    if (g.d != D) return cudaErrorNotSupported;
+    const long nch = gdn_num_chunks(g.L, C);
+    if (nch > 0x7fffffffL) return cudaErrorNotSupported;
+    GdnWorkspace ws = gdn_workspace_carve(g.ws, (long)g.B * g.Hg, g.L, D, C, true);
+    const size_t smem_prep = sizeof(PrepSmem) + 128;
+    const size_t smem_state = sizeof(StateSmem) + 128;
+    cudaError_t e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_prep);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_state);
+    if (e != cudaSuccess) return e;
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), THREADS, smem_prep, s>>>(g, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gdn_state_bf16<<<dim3(D / RB, (unsigned)(g.B * g.Hg)), THREADS, smem_state, s>>>(g, ws);
+    return cudaGetLastError();
+}
+
+}  // namespace hlta

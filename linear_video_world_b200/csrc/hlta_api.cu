@@ -46,6 +46,13 @@ constexpr int kMaxDevices = 64;
 DeviceCtx g_ctx[kMaxDevices];
 std::mutex g_ctx_mu;
 std::mutex g_fork_mu;   // the per-device fork/join events are shared by all host threads
+cudaEvent_t g_prof[5];  // profiling events of hlta_set_profile_events (guarded by g_fork_mu)
+bool g_prof_on = false;
+
+void prof_record(int i, cudaStream_t s)
+{
+    if (g_prof_on && g_prof[i]) cudaEventRecord(g_prof[i], s);
+}
 
 hlta_status device_ctx(DeviceCtx **out)
 {
@@ -284,29 +291,34 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const f
     if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
+    std::lock_guard<std::mutex> lk(g_fork_mu);
     // GDN heads on the auxiliary stream, ordered after everything already on `s`
     if (Hg) {
-        std::lock_guard<std::mutex> lk(g_fork_mu);
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         GdnArgs g;
         g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o;
         g.B = B; g.Hg = Hg; g.Htot = H; g.h0 = Hs + Hd; g.L = L; g.d = d; g.chunk = chunk;
         g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
+        prof_record(3, ctx->aux);
         st = run_gdn(g, dt, ctx->aux);
+        prof_record(4, ctx->aux);
         // join even on failure so `s` never runs ahead of work that was enqueued
         cudaEventRecord(ctx->join, ctx->aux);
         cudaStreamWaitEvent(s, ctx->join, 0);
         if (st != HLTA_OK) return st;
     }
+    prof_record(0, s);
     if (Hs) {
         AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
         if ((st = run_attn(a1, dt, s)) != HLTA_OK) return st;
     }
+    prof_record(1, s);
     if (Hd) {
         AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
         if ((st = run_attn(a2, dt, s)) != HLTA_OK) return st;
     }
+    prof_record(2, s);
     return HLTA_OK;
 }
 
@@ -435,6 +447,14 @@ hlta_status hlta_stream_destroy(hlta_stream_t c)
         if (p) cudaFree(p);
     if (prev >= 0) cudaSetDevice(prev);
     delete c;
+    return HLTA_OK;
+}
+
+hlta_status hlta_set_profile_events(void *const *events)
+{
+    std::lock_guard<std::mutex> lk(g_fork_mu);
+    g_prof_on = events != nullptr;
+    for (int i = 0; i < 5; ++i) g_prof[i] = events ? (cudaEvent_t)events[i] : nullptr;
     return HLTA_OK;
 }
 
