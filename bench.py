@@ -282,6 +282,9 @@ def main():
     # ---- device-resident timed region -----------------------------------------------------
     K = args.steps
     prof = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for evs in prof:            # torch creates the CUDA event at its first record
+        for e in evs:
+            e.record()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     gpu_index = vis.split(",")[local_rank] if vis else str(local_rank)

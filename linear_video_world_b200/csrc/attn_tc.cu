@@ -211,6 +211,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&x)[32])
         : "memory");
 }
 
+// 128 consecutive fp32 columns of this thread's TMEM lane, one instruction plus its wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[128])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
+        "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+        "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
+        "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
+        "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, "
+        "[%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : TMEM_REGS32(x), TMEM_REGS32((x + 32)), TMEM_REGS32((x + 64)), TMEM_REGS32((x + 96))
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&x)[32])
 {
     asm volatile(
@@ -420,37 +440,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const int sb = j & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (uint32_t)(j / 2) & 1u, abort_flag, p.err))) { ok = false; break; }
             fence_after_sync();
-            uint32_t sr[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tlane + TM_S + (uint32_t)sb * BN + c * 32, sr[c]);
+            uint32_t sr[128];
+            tmem_ld128(tlane + TM_S + (uint32_t)sb * BN, sr);
             fence_before_sync();
             mbar_arrive(BAR(B_SFREE + sb));
 
             const int nv = min(BN, p.N - jt * BN);
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
-            float mt = -INFINITY;
-            if (rok) {
+            const bool full = rok && nv == BN;
+            // row max of this tile (four independent chains)
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (full) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+            } else if (rok) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float sv = __uint_as_float(sr[c][i]);
-                        mt = fmaxf(mt, (c * 32 + i < nv) ? sv : -INFINITY);
-                    }
+                for (int i = 0; i < 128; ++i)
+                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
             }
-            // P buffer and O are in use by the previous tile's PV product until it completes
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
+            // grow the reference max only when it rose by more than 2^8 (lazy rescale)
+            const bool need = rok && mnew > m + 8.f;
+            const float muse = need ? mnew : m;
+            const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
+            // exponentials into registers before waiting for the previous PV product
+            uint32_t pk[64];
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            if (full) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse));
+                    const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse));
+                    ps[i & 3] += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (rok) {
+                        p0 = 2 * i < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
+                        p1 = 2 * i + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
+                    }
+                    ps[i & 3] += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+            }
+            // the P buffer and O belong to the previous tile's PV product until it completes
             if (j >= 1) {
                 if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (uint32_t)(j - 1) & 1u, abort_flag, p.err))) { ok = false; break; }
                 fence_after_sync();
-            }
-            float mnew = m;
-            if (rok) mnew = fmaxf(m, mt * p.sl2);
-            // grow the reference max only when it rose by more than 2^8; the TMEM traffic of
-            // the O rescale is warp-collective, so the whole warp takes that branch together
-            const bool need = rok && mnew > m + 8.f;
-            if (__any_sync(0xffffffffu, need)) {
-                const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-                if (j >= 1) {
+                // the O rescale is warp-collective TMEM traffic: the whole warp takes it together
+                if (__any_sync(0xffffffffu, need && m != -INFINITY)) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t orow[32];
@@ -462,39 +504,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     }
                     tmem_wait_st();
                 }
-                if (need) {
-                    lsum *= alpha;
-                    m = mnew;
-                }
             }
-            float part = 0.f;
+            lsum = lsum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            m = muse;
+            // 128 keys = 16 chunks of 16 B; the chunk index within each 64-key half is
+            // XOR-swizzled with the row (128-byte swizzle, as the MMA descriptor expects)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int col = c * 32 + 2 * i;
-                    float p0 = 0.f, p1 = 0.f;
-                    if (rok) {
-                        p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[c][2 * i]), p.sl2, -m)) : 0.f;
-                        p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), p.sl2, -m)) : 0.f;
-                    }
-                    part += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
-                }
-                // 32 keys = 4 chunks of 16 B; chunk index within the 64-key half is XOR-swizzled
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int chunk = c * 4 + q4;               // 0..15 over 128 keys
-                    const int half = chunk >> 3, cc = chunk & 7;
-                    uint8_t *dst = prow + half * HALF + ((cc ^ sw) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)),
-                                 "r"(pk[4 * q4]), "r"(pk[4 * q4 + 1]), "r"(pk[4 * q4 + 2]),
-                                 "r"(pk[4 * q4 + 3])
-                                 : "memory");
-                }
+            for (int chunk = 0; chunk < 16; ++chunk) {
+                const int half = chunk >> 3, cc = chunk & 7;
+                uint8_t *dst = prow + half * HALF + ((cc ^ sw) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)),
+                             "r"(pk[4 * chunk]), "r"(pk[4 * chunk + 1]), "r"(pk[4 * chunk + 2]),
+                             "r"(pk[4 * chunk + 3])
+                             : "memory");
             }
-            lsum += part;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             fence_before_sync();
             mbar_arrive(BAR(B_PFULL));

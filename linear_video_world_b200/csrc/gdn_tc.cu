@@ -120,19 +120,33 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // -----------------------------------------------------------------------------------------
 // prep
 // -----------------------------------------------------------------------------------------
-struct PrepSmem {
-    __nv_bfloat16 Q[C * SD], K[C * SD], V[C * SD], W[C * SD], U[C * SD];
-    __nv_bfloat16 P[C * SC], T1[C * SC], T2[C * SC];
-    float A[C * FP], T[C * FP];
-    float g[C], bb[C];
-};
+constexpr int PREP_THREADS = 256;
+constexpr int TP = C + 4;         // fp32 stride of T (17408 bytes = one [64][136] bf16 tile)
 
-// One warp's 16 rows x (2*npairs*8) columns of X = Amat (row-major [64][ldA]) * Bmat ([K][N]
-// row-major, transposed fragment loads), k-steps 0..ksteps-1.
+// Shared memory of the prep kernel (about 99 KB, two CTAs per SM). Regions are reused once
+// their contents are dead:
+//   R1: A (fp32 [64][65]) -> T1, T2 (bf16 [64][72] each) -> Op (bf16 [64][136])
+//   R2: T (fp32 [64][68]) -> W (bf16 [64][136])
+//   V:  V -> Up
+//   Q:  Q -> Qt
+struct PrepSmem {
+    __nv_bfloat16 Q[C * SD], K[C * SD], V[C * SD];
+    __nv_bfloat16 P[C * SC];
+    alignas(16) uint8_t R1[2 * C * SC * 2];
+    alignas(16) uint8_t R2[C * SD * 2];
+    float X[3 * 256];             // off-diagonal block products of the blocked inversion
+    float g[C], eg[C], ek[C], bb[C];
+};
+static_assert(sizeof(float) * C * (C + 1) <= 2 * C * SC * 2, "A must fit in R1");
+static_assert(sizeof(float) * C * TP <= C * SD * 2, "T must fit in R2");
+static_assert(C * SD * 2 <= 2 * C * SC * 2 + 1024, "Op must fit in R1");
+
+// One warp's 16 rows x (NT*8) columns of X = Am ([64][lda] row-major) * Bm ([K][N] row-major,
+// transposed fragment loads), k-steps 0 .. ksteps-1, columns n0 ...
 template <int NT>
 __device__ __forceinline__ void gemm_rows_kn(float (&acc)[NT][4], const __nv_bfloat16 *Am, int lda,
-                                             const __nv_bfloat16 *Bm, int ldb, int m0, int ksteps,
-                                             int lane)
+                                             const __nv_bfloat16 *Bm, int ldb, int m0, int n0,
+                                             int ksteps, int lane)
 {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -143,17 +157,37 @@ __device__ __forceinline__ void gemm_rows_kn(float (&acc)[NT][4], const __nv_bfl
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
             uint32_t b[4];
-            frag_b_kn(b, Bm, ldb, kk * 16, np * 16, lane);
+            frag_b_kn(b, Bm, ldb, kk * 16, n0 + np * 16, lane);
             mma16816(acc[2 * np], a, b[0], b[1]);
             mma16816(acc[2 * np + 1], a, b[2], b[3]);
         }
     }
 }
 
-__global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace ws)
+template <int NT>
+__device__ __forceinline__ void store_acc_bf16(__nv_bfloat16 *dst, int ld, const float (&acc)[NT][4],
+                                               int m0, int n0, int lane)
+{
+    const int g8 = lane >> 2, tg = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int c = n0 + nt * 8 + 2 * tg;
+        st_pair(&dst[(m0 + g8) * ld + c], acc[nt][0], acc[nt][1]);
+        st_pair(&dst[(m0 + g8 + 8) * ld + c], acc[nt][2], acc[nt][3]);
+    }
+}
+
+__global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnWorkspace ws)
 {
     extern __shared__ uint8_t smem_raw[];
     PrepSmem &s = *reinterpret_cast<PrepSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    float *A = reinterpret_cast<float *>(s.R1);            // [64][65]
+    __nv_bfloat16 *T1 = reinterpret_cast<__nv_bfloat16 *>(s.R1);
+    __nv_bfloat16 *T2 = T1 + C * SC;
+    __nv_bfloat16 *Op = reinterpret_cast<__nv_bfloat16 *>(s.R1);
+    float *T = reinterpret_cast<float *>(s.R2);            // [64][68]
+    __nv_bfloat16 *W = reinterpret_cast<__nv_bfloat16 *>(s.R2);
+
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long nch = gdn_num_chunks(p.L, C);
@@ -165,9 +199,11 @@ __global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace
     const uint4 *gv = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.v + (head + t0) * D);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g8 = lane >> 2, tg = lane & 3;
+    const int rb = warp & 3, ch = warp >> 2;               // 16-row block, column half
+    const int m0 = rb * 16;
 
     // ---- load the chunk (rows >= n are zero) and the gates
-    for (int e = tid; e < C * (D / 8); e += THREADS) {
+    for (int e = tid; e < C * (D / 8); e += PREP_THREADS) {
         const int t = e / (D / 8), c8 = e % (D / 8);
         uint4 zq = make_uint4(0, 0, 0, 0), zk = zq, zv = zq;
         if (t < n) {
@@ -179,39 +215,49 @@ __global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace
         *reinterpret_cast<uint4 *>(&s.K[t * SD + c8 * 8]) = zk;
         *reinterpret_cast<uint4 *>(&s.V[t * SD + c8 * 8]) = zv;
     }
-    if (tid < C) {
-        const float av = tid < n ? p.a[(long)bh * p.L + t0 + tid] : 1.f;
-        s.g[tid] = tid < n ? logf(av) : 0.f;
-        s.bb[tid] = tid < n ? p.b[(long)bh * p.L + t0 + tid] : 0.f;
+    if (warp == 0) {
+        // inclusive prefix sum of log a over 64 entries: two per lane, then a warp scan
+        const int t = 2 * lane;
+        const float l0 = t < n ? logf(p.a[(long)bh * p.L + t0 + t]) : 0.f;
+        const float l1 = t + 1 < n ? logf(p.a[(long)bh * p.L + t0 + t + 1]) : 0.f;
+        float pair = l0 + l1, x = pair;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        const float excl = x - pair;
+        s.g[t] = excl + l0;
+        s.g[t + 1] = x;
+        s.bb[t] = t < n ? p.b[(long)bh * p.L + t0 + t] : 0.f;
+        s.bb[t + 1] = t + 1 < n ? p.b[(long)bh * p.L + t0 + t + 1] : 0.f;
     }
     __syncthreads();
-    // inclusive prefix sum of log a (Hillis-Steele over 64 entries)
-    for (int off = 1; off < C; off <<= 1) {
-        float v = 0.f;
-        if (tid < C && tid >= off) v = s.g[tid - off];
-        __syncthreads();
-        if (tid < C) s.g[tid] += v;
-        __syncthreads();
+    if (tid < C) {
+        const float gn = s.g[n - 1];
+        s.eg[tid] = tid < n ? expf(s.g[tid]) : 0.f;
+        s.ek[tid] = tid < n ? expf(gn - s.g[tid]) : 0.f;
     }
 
-    // ---- KK^T and QK^T for this warp's 16 rows; only columns i <= t are needed
+    // ---- KK^T and QK^T: this warp's 16 rows, 32 columns; columns above the diagonal block
+    //      are zero and not computed
     {
-        const int m0 = warp * 16;
-        const int ntiles = 2 * warp + 2;      // column tiles 0 .. 2w+1 cover i <= 16w+15
-        float kk[8][4], qk[8][4];
+        const int n0 = ch * 32;
+        const bool live = n0 <= m0 + 15;
+        float kk[4][4], qk[4][4];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) kk[nt][e] = qk[nt][e] = 0.f;
-        for (int ks = 0; ks < D / 16; ++ks) {
-            uint32_t ak[4], aq[4];
-            frag_a(ak, s.K, SD, m0, ks * 16, lane);
-            frag_a(aq, s.Q, SD, m0, ks * 16, lane);
+        if (live) {
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t ak[4], aq[4];
+                frag_a(ak, s.K, SD, m0, ks * 16, lane);
+                frag_a(aq, s.Q, SD, m0, ks * 16, lane);
 #pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                if (2 * np < ntiles) {
+                for (int np = 0; np < 2; ++np) {
                     uint32_t bk[4];
-                    frag_b_nk(bk, s.K, SD, np * 16, ks * 16, lane);
+                    frag_b_nk(bk, s.K, SD, n0 + np * 16, ks * 16, lane);
                     mma16816(kk[2 * np], ak, bk[0], bk[1]);
                     mma16816(kk[2 * np + 1], ak, bk[2], bk[3]);
                     mma16816(qk[2 * np], aq, bk[0], bk[1]);
@@ -220,86 +266,89 @@ __global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace
             }
         }
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = m0 + g8 + (e >> 1) * 8;
-                const int i = nt * 8 + 2 * tg + (e & 1);
+                const int i = n0 + nt * 8 + 2 * tg + (e & 1);
                 const bool lower = i <= t && t < n;
                 const float dec = lower ? expf(s.g[t] - s.g[i]) : 0.f;
-                s.A[t * FP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
+                A[t * FP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
                 s.P[t * SC + i] = __float2bfloat16_rn(lower ? dec * qk[nt][e] : 0.f);
             }
         }
     }
+    for (int e = tid; e < C * TP; e += PREP_THREADS) T[e] = 0.f;
     __syncthreads();
 
-    // ---- T = (I + A)^{-1}: forward substitution, one thread per column (fp32)
+    // ---- T = (I + A)^{-1}, blocked by 16: diagonal blocks by forward substitution, then
+    //      T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ block row by block row
     if (tid < C) {
-        const int j = tid;
-        for (int t = 0; t <= j; ++t) s.T[t * FP + j] = t == j ? 1.f : 0.f;
-        for (int t = j + 1; t < C; ++t) {
-            float a0 = 0.f, a1 = 0.f;
-            int i = j;
-            for (; i + 1 < t; i += 2) {
-                a0 = fmaf(s.A[t * FP + i], s.T[i * FP + j], a0);
-                a1 = fmaf(s.A[t * FP + i + 1], s.T[(i + 1) * FP + j], a1);
-            }
-            if (i < t) a0 = fmaf(s.A[t * FP + i], s.T[i * FP + j], a0);
-            s.T[t * FP + j] = -(a0 + a1);
+        const int I = tid >> 4, jj = tid & 15, base = I * 16, j = base + jj;
+        T[j * TP + j] = 1.f;
+        for (int t = jj + 1; t < 16; ++t) {
+            float acc = 0.f;
+            for (int i = jj; i < t; ++i) acc = fmaf(A[(base + t) * FP + base + i], T[(base + i) * TP + j], acc);
+            T[(base + t) * TP + j] = -acc;
         }
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += THREADS) {
-        const int t = e / C, i = e % C;
-        const float tv = s.T[t * FP + i];
-        s.T1[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i] * expf(s.g[i]));
-        s.T2[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i]);
+    for (int I = 1; I < 4; ++I) {
+        // X_IJ = sum_{K=J}^{I-1} A_IK T_KJ for J < I   (I blocks of 256 entries)
+        for (int e = tid; e < I * 256; e += PREP_THREADS) {
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int row = I * 16 + r, col = J * 16 + c;
+            float acc = 0.f;
+            for (int kx = J * 16; kx < I * 16; ++kx) acc = fmaf(A[row * FP + kx], T[kx * TP + col], acc);
+            s.X[e] = acc;
+        }
+        __syncthreads();
+        // T_IJ = -T_II X_IJ
+        for (int e = tid; e < I * 256; e += PREP_THREADS) {
+            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int row = I * 16 + r;
+            float acc = 0.f;
+            for (int kx = 0; kx <= r; ++kx) acc = fmaf(T[row * TP + I * 16 + kx], s.X[(J << 8) + (kx << 4) + c], acc);
+            T[row * TP + J * 16 + c] = -acc;
+        }
+        __syncthreads();
+    }
+    // ---- T1 = T diag(b e^g), T2 = T diag(b) in bf16 (over A, which is dead)
+    for (int e = tid; e < C * C; e += PREP_THREADS) {
+        const int t = e >> 6, i = e & 63;
+        const float tv = T[t * TP + i];
+        T1[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i] * s.eg[i]);
+        T2[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i]);
     }
     __syncthreads();
 
-    const int m0 = warp * 16;
-    const int ksteps = warp + 1;              // T1, T2, P are lower triangular
-    // ---- W = T1 K, Up = T2 V  (kept in smem as bf16)
+    // ---- W = T1 K, Up = T2 V (lower-triangular T: k-steps 0 .. rb)
+    const int nc0 = ch * 64;
     {
-        float acc[16][4];
-        gemm_rows_kn<16>(acc, s.T1, SC, s.K, SD, m0, ksteps, lane);
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = nt * 8 + 2 * tg;
-            st_pair(&s.W[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
-            st_pair(&s.W[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
-        }
-        gemm_rows_kn<16>(acc, s.T2, SC, s.V, SD, m0, ksteps, lane);
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = nt * 8 + 2 * tg;
-            st_pair(&s.U[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
-            st_pair(&s.U[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
-        }
+        float w[8][4], u[8][4];
+        gemm_rows_kn<8>(w, T1, SC, s.K, SD, m0, nc0, rb + 1, lane);
+        gemm_rows_kn<8>(u, T2, SC, s.V, SD, m0, nc0, rb + 1, lane);
+        __syncthreads();                                   // T, T1, T2 and V are dead now
+        store_acc_bf16<8>(W, SD, w, m0, nc0, lane);
+        store_acc_bf16<8>(s.V, SD, u, m0, nc0, lane);
     }
     __syncthreads();
-    // ---- Op = P Up (into the V buffer), Qt = e^g Q - P W (in place over Q)
+    // ---- Op = P Up (into R1), Qt = diag(e^g) Q - P W (in place over Q)
     {
-        float acc[16][4];
-        gemm_rows_kn<16>(acc, s.P, SC, s.U, SD, m0, ksteps, lane);
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = nt * 8 + 2 * tg;
-            st_pair(&s.V[(m0 + g8) * SD + c], acc[nt][0], acc[nt][1]);
-            st_pair(&s.V[(m0 + g8 + 8) * SD + c], acc[nt][2], acc[nt][3]);
-        }
-        gemm_rows_kn<16>(acc, s.P, SC, s.W, SD, m0, ksteps, lane);
+        float op[8][4], pw[8][4];
+        gemm_rows_kn<8>(op, s.P, SC, s.V, SD, m0, nc0, rb + 1, lane);
+        gemm_rows_kn<8>(pw, s.P, SC, W, SD, m0, nc0, rb + 1, lane);
+        store_acc_bf16<8>(Op, SD, op, m0, nc0, lane);
         const int ta = m0 + g8, tb = ta + 8;
-        const float ea = ta < n ? expf(s.g[ta]) : 0.f, eb = tb < n ? expf(s.g[tb]) : 0.f;
+        const float ea = s.eg[ta], eb = s.eg[tb];          // zero for rows >= n
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = nt * 8 + 2 * tg;
+        for (int nt = 0; nt < 8; ++nt) {
+            const int c = nc0 + nt * 8 + 2 * tg;
             __nv_bfloat16 *qa = &s.Q[ta * SD + c], *qb = &s.Q[tb * SD + c];
             const float qa0 = __bfloat162float(qa[0]), qa1 = __bfloat162float(qa[1]);
             const float qb0 = __bfloat162float(qb[0]), qb1 = __bfloat162float(qb[1]);
-            st_pair(qa, ta < n ? ea * qa0 - acc[nt][0] : 0.f, ta < n ? ea * qa1 - acc[nt][1] : 0.f);
-            st_pair(qb, tb < n ? eb * qb0 - acc[nt][2] : 0.f, tb < n ? eb * qb1 - acc[nt][3] : 0.f);
+            st_pair(qa, ta < n ? ea * qa0 - pw[nt][0] : 0.f, ta < n ? ea * qa1 - pw[nt][1] : 0.f);
+            st_pair(qb, tb < n ? eb * qb0 - pw[nt][2] : 0.f, tb < n ? eb * qb1 - pw[nt][3] : 0.f);
         }
     }
     __syncthreads();
@@ -311,15 +360,14 @@ __global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace
     uint4 *oO = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Op + base);
     uint4 *oQ = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Qt + base);
     uint4 *oK = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Kt + base);
-    const float gn = s.g[n - 1];
-    for (int e = tid; e < C * (D / 8); e += THREADS) {
+    for (int e = tid; e < C * (D / 8); e += PREP_THREADS) {
         const int t = e / (D / 8), c8 = e % (D / 8);
         const int so = t * SD + c8 * 8;
-        oW[e] = *reinterpret_cast<const uint4 *>(&s.W[so]);
-        oU[e] = *reinterpret_cast<const uint4 *>(&s.U[so]);
-        oO[e] = *reinterpret_cast<const uint4 *>(&s.V[so]);
+        oW[e] = *reinterpret_cast<const uint4 *>(&W[so]);
+        oU[e] = *reinterpret_cast<const uint4 *>(&s.V[so]);
+        oO[e] = *reinterpret_cast<const uint4 *>(&Op[so]);
         oQ[e] = *reinterpret_cast<const uint4 *>(&s.Q[so]);
-        const float dk = t < n ? expf(gn - s.g[t]) : 0.f;
+        const float dk = s.ek[t];
         uint4 kv = *reinterpret_cast<const uint4 *>(&s.K[so]);
         __nv_bfloat162 *k2 = reinterpret_cast<__nv_bfloat162 *>(&kv);
 #pragma unroll
@@ -329,7 +377,7 @@ __global__ void __launch_bounds__(THREADS) gdn_prep_bf16(GdnArgs p, GdnWorkspace
         }
         oK[e] = kv;
     }
-    if (tid == 0) ws.gam[(long)bh * nch + chunk] = expf(gn);
+    if (tid == 0) ws.gam[(long)bh * nch + chunk] = expf(s.g[n - 1]);
 }
 
 // -----------------------------------------------------------------------------------------
@@ -339,8 +387,9 @@ struct StateBuf {
     __nv_bfloat16 W[C * SD], Q[C * SD], K[C * SD];   // W, Qt, Kt of one chunk
     __nv_bfloat16 U[C * SR], O[C * SR];              // this CTA's 16 columns of Up, Op
 };
+constexpr int NSTAGE = 3;          // chunk operand buffers of the state pass
 struct StateSmem {
-    StateBuf buf[2];
+    StateBuf buf[NSTAGE];
     __nv_bfloat16 Sb[RB * SD];                       // state slice as bf16 [i][j]
     __nv_bfloat16 Ut[RB * SC];                       // U^T slice [i][t]
     __nv_bfloat16 Os[C * SR];                        // output staging [t][i]
@@ -394,13 +443,17 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
                 s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
             }
 
-    load_chunk(s.buf[0], ws, bh, nch, 0, i0, tid);
-    cp_async_commit();
+    // prefetch NSTAGE-1 chunks ahead; one cp.async group per chunk (empty groups past the end)
+    for (int c = 0; c < NSTAGE - 1; ++c) {
+        if (c < nch) load_chunk(s.buf[c], ws, bh, nch, c, i0, tid);
+        cp_async_commit();
+    }
     for (long c = 0; c < nch; ++c) {
-        StateBuf &cur = s.buf[c & 1];
-        cp_async_wait<0>();
-        __syncthreads();                       // chunk c landed; Sb holds the incoming state
-        if (c + 1 < nch) load_chunk(s.buf[(c + 1) & 1], ws, bh, nch, c + 1, i0, tid);
+        StateBuf &cur = s.buf[c % NSTAGE];
+        cp_async_wait<NSTAGE - 2>();           // the group of chunk c has landed
+        __syncthreads();                       // ... for every thread; Sb holds the incoming state
+        if (c + NSTAGE - 1 < nch)
+            load_chunk(s.buf[(c + NSTAGE - 1) % NSTAGE], ws, bh, nch, c + NSTAGE - 1, i0, tid);
         cp_async_commit();
         const float gam = ws.gam[(long)bh * nch + c];
 
@@ -509,7 +562,7 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     const long nch = gdn_num_chunks(g.L, C);
     if (nch > 0x7fffffffL) return cudaErrorNotSupported;
     GdnWorkspace ws = gdn_workspace_carve(g.ws, (long)g.B * g.Hg, g.L, D, C, true);
-    const size_t smem_prep = sizeof(PrepSmem) + 128;
+    const size_t smem_prep = sizeof(PrepSmem) + 128;   // about 99 KB: two CTAs per SM
     const size_t smem_state = sizeof(StateSmem) + 128;
     cudaError_t e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_prep);
@@ -517,7 +570,7 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), THREADS, smem_prep, s>>>(g, ws);
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), PREP_THREADS, smem_prep, s>>>(g, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     gdn_state_bf16<<<dim3(D / RB, (unsigned)(g.B * g.Hg)), THREADS, smem_state, s>>>(g, ws);
     return cudaGetLastError();
