@@ -9,15 +9,21 @@
 // per-element mask (row frame vs. key frame, ragged frame end) removes what a row must not
 // see.
 //
-// One CTA = one 128-row query tile of one head; 6 warps:
-//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring (128B swizzle)
-//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers,
-//               O += P_j V_j into the TMEM O accumulator (tcgen05.mma kind::f16)
-//   warps 2..5  softmax: one thread per query row; reads S from TMEM, updates the running
-//               max (rescaling O in TMEM only when the max grows by more than 2^8), writes
-//               P (bf16) to shared memory for the PV product, and finally normalises O.
-// Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in the
-// device error word, every role stops, and the TMEM allocation is released.
+// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 12 warps
+// in three warpgroups (softmax 0, softmax 1, and one holding the TMA and MMA warps):
+//   warp 8      TMA producer: Q (both sub-tiles) once, then K and V tiles into a 2-stage ring
+//               (128B swizzle); the sub-tiles share every K/V tile
+//   warp 9      TMEM owner and MMA issuer (tcgen05.mma kind::f16): S_q = Q_q K_j^T into TMEM,
+//               O_q += P_q V_j with P_q read from TMEM (written there by the softmax over the
+//               first 64 columns of S_q) and V_j an MN-major shared-memory operand; order
+//               S_0(j) S_1(j) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ... so the tensor pipe works
+//               on one sub-tile while the other sub-tile's softmax runs
+//   warps 0..3  softmax of sub-tile 0, warps 4..7 softmax of sub-tile 1: one thread per query
+//               row; S from TMEM, running max (O rescaled in TMEM only when the max grows by
+//               more than 2^8), P (bf16) back to TMEM, final normalisation of O.
+// A key tile that no row of a sub-tile may see is skipped for that sub-tile (no MMA, no
+// softmax). Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in
+// the device error word, every role stops, and the TMEM allocation is released.
 #include "hlta_internal.cuh"
 
 #include <cuda.h>
@@ -28,33 +34,35 @@
 namespace hlta {
 namespace {
 
-constexpr int BM = 128;                 // query rows per tile
+constexpr int BM = 128;                 // query rows per sub-tile
+constexpr int QT = 2;                   // query sub-tiles per CTA
 constexpr int BN = 128;                 // keys per tile
 constexpr int D = 128;                  // head dim
 constexpr int NS = 2;                   // K/V ring stages
-constexpr int THREADS = 192;
+constexpr int THREADS = 384;           // 3 warpgroups: softmax 0, softmax 1, {TMA, MMA, 2 idle}
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr uint32_t HALF = 16384;        // one [128 rows][64 cols] bf16 half tile
 constexpr uint32_t TILE = 2 * HALF;     // [128][128] bf16
-constexpr uint32_t TMEM_COLS = 512;     // S0 @0, S1 @128, O @256
-constexpr uint32_t TM_S = 0, TM_O = 256;
+constexpr uint32_t TMEM_COLS = 512;     // S_0 @0, S_1 @128, O_0 @256, O_1 @384
+__host__ __device__ constexpr uint32_t TM_S(int q) { return (uint32_t)q * 128u; }
+__host__ __device__ constexpr uint32_t TM_O(int q) { return 256u + (uint32_t)q * 128u; }
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t SM_Q = 0;
-constexpr uint32_t SM_K0 = TILE;                        // K[s] = SM_K0 + s * 2 * TILE
-constexpr uint32_t SM_P = TILE + NS * 2 * TILE;
-constexpr uint32_t SM_BAR = SM_P + TILE;
+__host__ __device__ constexpr uint32_t SM_Q(int q) { return (uint32_t)q * TILE; }
+__host__ __device__ constexpr uint32_t SM_K(int st) { return QT * TILE + (uint32_t)st * 2 * TILE; }
+__host__ __device__ constexpr uint32_t SM_V(int st) { return SM_K(st) + TILE; }
+constexpr uint32_t SM_BAR = SM_K(NS);
 // barriers (8 bytes each)
 enum {
     B_QFULL = 0,
-    B_KFULL = 1,                // + s
+    B_KFULL = 1,                // + stage
     B_VFULL = B_KFULL + NS,
     B_KEMPTY = B_VFULL + NS,
     B_VEMPTY = B_KEMPTY + NS,
-    B_SFULL = B_VEMPTY + NS,    // + buffer (2)
-    B_SFREE = B_SFULL + 2,
-    B_PFULL = B_SFREE + 2,
-    B_PVDONE = B_PFULL + 1,
-    NBARS = B_PVDONE + 1
+    B_SFULL = B_VEMPTY + NS,    // + sub-tile
+    B_PFULL = B_SFULL + QT,
+    B_PVDONE = B_PFULL + QT,
+    NBARS = B_PVDONE + QT
 };
 constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
 constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
@@ -161,6 +169,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
+// Same with the A operand read from tensor memory (M lanes x K bf16 packed in pairs per column)
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version bit.
 // lbo / sbo in bytes: K-major operands use sbo = 1024 (8 rows of 128 B) and an unused lbo;
 // MN-major operands use lbo = distance between 64-element column blocks, sbo = 1024.
@@ -231,6 +251,32 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[128])
         : "memory");
 }
 
+// 64 consecutive fp32 columns, load and wait in one statement
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&x)[64])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, "
+        "[%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : TMEM_REGS32(x), TMEM_REGS32((x + 32))
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&x)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(x[0]), "r"(x[1]), "r"(x[2]), "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7]),
+        "r"(x[8]), "r"(x[9]), "r"(x[10]), "r"(x[11]), "r"(x[12]), "r"(x[13]), "r"(x[14]), "r"(x[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&x)[32])
 {
     asm volatile(
@@ -259,14 +305,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 // ---------------------------------------------------------------------------------------
 // key-tile walk shared by every role (all roles must visit the same sequence)
 // ---------------------------------------------------------------------------------------
+// frame fk is a key frame of some query frame in [fa, fb]
+__device__ __forceinline__ bool frame_needed(int fk, int fa, int fb, int w, int r)
+{
+    const int i0 = fa > fk ? (fa - fk + r - 1) / r : 0;
+    return i0 < w && fk + r * i0 <= fb;
+}
+
 struct Walk {
     int fa, fb, w, r, tpf;
-    // frame fk is a key frame of some query frame in [fa, fb]
-    __device__ __forceinline__ bool needed(int fk) const
-    {
-        int i0 = fa > fk ? (fa - fk + r - 1) / r : 0;
-        return i0 < w && fk + r * i0 <= fb;
-    }
+    __device__ __forceinline__ bool needed(int fk) const { return frame_needed(fk, fa, fb, w, r); }
     // advance (fk, jt) to the next tile; false when done
     __device__ __forceinline__ bool next(int &fk, int &jt) const
     {
@@ -301,37 +349,49 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
     const int b = bh / p.Hbr, h = bh % p.Hbr;
-    const long l0 = (long)blockIdx.x * BM;
+    const long l0 = (long)blockIdx.x * (QT * BM);
     const long q_head = (long)(b * p.q_Htot + p.q_h0 + h) * p.q_rows;
     const long kv_head = (long)(b * p.kv_Htot + p.kv_h0 + h) * p.kv_rows;
-    const int nrows = (int)min((long)BM, p.q_rows - l0);
+    // frame ranges of the two sub-tiles (sub-tile 1 may be empty in the last CTA of a head)
+    int sfa[QT], sfb[QT];
+    bool svalid[QT];
+#pragma unroll
+    for (int q = 0; q < QT; ++q) {
+        const long r0 = l0 + q * BM;
+        svalid[q] = r0 < p.q_rows;
+        const long r1 = min(r0 + BM, p.q_rows) - 1;
+        sfa[q] = p.fq0 + (int)(r0 / p.N);
+        sfb[q] = svalid[q] ? p.fq0 + (int)(r1 / p.N) : sfa[q];
+    }
     Walk wk;
-    wk.fa = p.fq0 + (int)(l0 / p.N);
-    wk.fb = p.fq0 + (int)((l0 + nrows - 1) / p.N);
+    wk.fa = sfa[0];
+    wk.fb = svalid[1] ? sfb[1] : sfb[0];
     wk.w = p.w;
     wk.r = p.r;
     wk.tpf = (p.N + BN - 1) / BN;
     const int fstart = max(0, wk.fa - p.r * (p.w - 1));
+    auto active = [&](int q, int fk) {
+        return svalid[q] && frame_needed(fk, sfa[q], sfb[q], p.w, p.r);
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(B_QFULL), 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(BAR(B_KFULL + s), 1);
-            mbar_init(BAR(B_VFULL + s), 1);
-            mbar_init(BAR(B_KEMPTY + s), 1);
-            mbar_init(BAR(B_VEMPTY + s), 1);
+        for (int st = 0; st < NS; ++st) {
+            mbar_init(BAR(B_KFULL + st), 1);
+            mbar_init(BAR(B_VFULL + st), 1);
+            mbar_init(BAR(B_KEMPTY + st), 1);
+            mbar_init(BAR(B_VEMPTY + st), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(BAR(B_SFULL + i), 1);
-            mbar_init(BAR(B_SFREE + i), 128);
+        for (int q = 0; q < QT; ++q) {
+            mbar_init(BAR(B_SFULL + q), 1);
+            mbar_init(BAR(B_PFULL + q), 128);
+            mbar_init(BAR(B_PVDONE + q), 1);
         }
-        mbar_init(BAR(B_PFULL), 128);
-        mbar_init(BAR(B_PVDONE), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == WARP_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(TMEM_COLS)
@@ -343,120 +403,143 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == WARP_TMA) {
         // ------------------------------- TMA producer -----------------------------------
         if (lane == 0) {
-            const int qrow = (int)(q_head + l0);
-            mbar_expect_tx(BAR(B_QFULL), TILE);
-            tma_load_2d(sbase + SM_Q, &tq, 0, qrow, BAR(B_QFULL));
-            tma_load_2d(sbase + SM_Q + HALF, &tq, 64, qrow, BAR(B_QFULL));
+            mbar_expect_tx(BAR(B_QFULL), QT * TILE);
+            for (int q = 0; q < QT; ++q) {
+                const int qrow = (int)(q_head + l0 + q * BM);
+                tma_load_2d(sbase + SM_Q(q), &tq, 0, qrow, BAR(B_QFULL));
+                tma_load_2d(sbase + SM_Q(q) + HALF, &tq, 64, qrow, BAR(B_QFULL));
+            }
             int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
             while (wk.next(fk, jt)) {
-                const int s = j % NS;
+                const int st = j % NS;
                 const uint32_t ph = (uint32_t)((j / NS) + 1) & 1u;
                 const int krow = (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
-                const uint32_t kdst = sbase + SM_K0 + (uint32_t)s * 2 * TILE;
-                const uint32_t vdst = kdst + TILE;
-                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, p.err)) break;
-                mbar_expect_tx(BAR(B_KFULL + s), TILE);
-                tma_load_2d(kdst, &tk, 0, krow, BAR(B_KFULL + s));
-                tma_load_2d(kdst + HALF, &tk, 64, krow, BAR(B_KFULL + s));
-                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, p.err)) break;
-                mbar_expect_tx(BAR(B_VFULL + s), TILE);
-                tma_load_2d(vdst, &tv, 0, krow, BAR(B_VFULL + s));
-                tma_load_2d(vdst + HALF, &tv, 64, krow, BAR(B_VFULL + s));
+                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + st), ph, abort_flag, p.err)) break;
+                mbar_expect_tx(BAR(B_KFULL + st), TILE);
+                tma_load_2d(sbase + SM_K(st), &tk, 0, krow, BAR(B_KFULL + st));
+                tma_load_2d(sbase + SM_K(st) + HALF, &tk, 64, krow, BAR(B_KFULL + st));
+                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + st), ph, abort_flag, p.err)) break;
+                mbar_expect_tx(BAR(B_VFULL + st), TILE);
+                tma_load_2d(sbase + SM_V(st), &tv, 0, krow, BAR(B_VFULL + st));
+                tma_load_2d(sbase + SM_V(st) + HALF, &tv, 64, krow, BAR(B_VFULL + st));
                 ++j;
             }
             if (*abort_flag) {
                 // let this CTA's copies in flight land before the CTA may exit
                 const long long t0 = clock64();
-                for (int s = 0; s < NS; ++s) {
-                    for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj) {
-                        if (jj % NS != s) continue;
-                        const uint32_t ph = (uint32_t)(jj / NS) & 1u;
-                        while (!mbar_try(BAR(B_KFULL + s), ph) && clock64() - t0 < (1LL << 31)) {}
-                        while (!mbar_try(BAR(B_VFULL + s), ph) && clock64() - t0 < (1LL << 31)) {}
-                    }
+                for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj) {
+                    const int st = jj % NS;
+                    const uint32_t ph = (uint32_t)(jj / NS) & 1u;
+                    while (!mbar_try(BAR(B_KFULL + st), ph) && clock64() - t0 < (1LL << 31)) {}
+                    while (!mbar_try(BAR(B_VFULL + st), ph) && clock64() - t0 < (1LL << 31)) {}
                 }
                 while (!mbar_try(BAR(B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == WARP_MMA) {
         // ------------------------------- MMA issuer -------------------------------------
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
-            constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P K-major, V MN-major
+            constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P (TMEM), V MN-major
+            int n_s[QT] = {0, 0}, n_pv[QT] = {0, 0};
             bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err);
-            auto issue_pv = [&](int t) -> bool {
-                const int s = t % NS;
-                if (!mbar_wait(BAR(B_PFULL), (uint32_t)t & 1u, abort_flag, p.err)) return false;
-                if (!mbar_wait(BAR(B_VFULL + s), (uint32_t)(t / NS) & 1u, abort_flag, p.err)) return false;
+            // S_q = Q_q K^T; first waits for the previous PV of this sub-tile, which reads P_q
+            // from the same TMEM columns
+            auto issue_s = [&](int q, int st) -> bool {
+                if (n_pv[q] > 0 && !mbar_wait(BAR(B_PVDONE + q), (uint32_t)(n_pv[q] - 1) & 1u, abort_flag, p.err))
+                    return false;
                 fence_after_sync();
-                const uint32_t vaddr = sbase + SM_K0 + (uint32_t)s * 2 * TILE + TILE;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(sbase + SM_P + (kk >> 2) * HALF + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(vaddr + kk * 2048, HALF, 1024);
-                    umma_bf16(tmem + TM_O, ad, bd, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(BAR(B_VEMPTY + s));
-                umma_commit(BAR(B_PVDONE));
-                return true;
-            };
-            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
-            while (ok && wk.next(fk, jt)) {
-                const int s = j % NS, sb = j & 1;
-                if (!mbar_wait(BAR(B_KFULL + s), (uint32_t)(j / NS) & 1u, abort_flag, p.err)) { ok = false; break; }
-                if (j >= 2 && !mbar_wait(BAR(B_SFREE + sb), (uint32_t)((j / 2) + 1) & 1u, abort_flag, p.err)) { ok = false; break; }
-                fence_after_sync();
-                const uint32_t kaddr = sbase + SM_K0 + (uint32_t)s * 2 * TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-                    umma_bf16(tmem + TM_S + (uint32_t)sb * BN, sw128_desc(sbase + SM_Q + off, 16, 1024),
-                              sw128_desc(kaddr + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                    umma_bf16(tmem + TM_S(q), sw128_desc(sbase + SM_Q(q) + off, 16, 1024),
+                              sw128_desc(sbase + SM_K(st) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(BAR(B_KEMPTY + s));
-                umma_commit(BAR(B_SFULL + sb));
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+                umma_commit(BAR(B_SFULL + q));
+                ++n_s[q];
+                return true;
+            };
+            // O_q += P_q V, P_q from TMEM (bf16 pairs in the first 64 columns of S_q)
+            auto issue_pv = [&](int q, int st) -> bool {
+                if (!mbar_wait(BAR(B_PFULL + q), (uint32_t)n_pv[q] & 1u, abort_flag, p.err)) return false;
+                fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_bf16_ts(tmem + TM_O(q), tmem + TM_S(q) + kk * 8,
+                                 sw128_desc(sbase + SM_V(st) + kk * 2048, HALF, 1024), IDESC_O,
+                                 (n_pv[q] > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(BAR(B_PVDONE + q));
+                ++n_pv[q];
+                return true;
+            };
+            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
+            bool have = ok && wk.next(fk, jt);
+            if (have) {
+                ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag, p.err);
+                for (int q = 0; q < QT && ok; ++q)
+                    if (active(q, fk)) ok = issue_s(q, 0);
+                if (ok) umma_commit(BAR(B_KEMPTY + 0));
+            }
+            while (ok && have) {
+                const int st = j % NS, fk_cur = fk;
+                int fk_n = fk, jt_n = jt;
+                const bool have_n = wk.next(fk_n, jt_n);
+                const int stn = (j + 1) % NS;
+                if (!mbar_wait(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u, abort_flag, p.err)) { ok = false; break; }
+                bool k_ready = false;                   // K of the next tile, waited for once
+                for (int q = 0; q < QT && ok; ++q) {
+                    if (active(q, fk_cur)) ok = issue_pv(q, st);
+                    if (ok && have_n && active(q, fk_n)) {
+                        if (!k_ready)
+                            ok = k_ready = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err);
+                        if (ok) ok = issue_s(q, stn);
+                    }
+                }
+                if (!ok) break;
+                if (have_n) umma_commit(BAR(B_KEMPTY + stn));
+                umma_commit(BAR(B_VEMPTY + st));
+                fk = fk_n;
+                jt = jt_n;
+                have = have_n;
                 ++j;
             }
-            if (ok && j >= 1) issue_pv(j - 1);
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------- softmax ----------------------------------------
-        const int quad = warp & 3;                       // TMEM lane quadrant of this warp
+        const int q = warp >> 2;                        // sub-tile of this warpgroup
+        const int quad = warp & 3;                      // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
-        const long lrow = l0 + row;
+        const long lrow = l0 + q * BM + row;
         const bool row_valid = lrow < p.q_rows;
         const int fq = p.fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-        uint8_t *prow = smem + SM_P + row * 128;
-        const int sw = row & 7;
         float m = -INFINITY, lsum = 0.f;
         bool ok = true;
-        int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
+        int fk = fstart - 1, jt = wk.tpf - 1, k = 0;
         while (wk.next(fk, jt)) {
-            const int sb = j & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + sb), (uint32_t)(j / 2) & 1u, abort_flag, p.err))) { ok = false; break; }
+            if (!active(q, fk)) continue;               // warp-uniform
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err))) { ok = false; break; }
             fence_after_sync();
-            uint32_t sr[128];
-            tmem_ld128(tlane + TM_S + (uint32_t)sb * BN, sr);
-            fence_before_sync();
-            mbar_arrive(BAR(B_SFREE + sb));
-
             const int nv = min(BN, p.N - jt * BN);
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
             const bool full = rok && nv == BN;
-            // row max of this tile (four independent chains)
+            // pass 1: row max over the tile (two 64-column loads, four independent chains)
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (full) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
-            } else if (rok) {
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t sr[64];
+                tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
+                if (full) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
+                    for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+                } else if (rok) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        mx[i & 3] = fmaxf(mx[i & 3], hf * 64 + i < nv ? __uint_as_float(sr[i]) : -INFINITY);
+                }
             }
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
@@ -464,82 +547,73 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const bool need = rok && mnew > m + 8.f;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // exponentials into registers before waiting for the previous PV product
-            uint32_t pk[64];
+            // pass 2: exponentials of 32 keys at a time; their bf16 pairs (key 2i in the low
+            // half) go to P columns 16c..16c+15, which overlay S columns already read
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
-            if (full) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse));
-                    ps[i & 3] += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
-                }
-            } else {
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sr[32], pk[16];
+                tmem_ld32(tlane + TM_S(q) + c * 32, sr);
+                if (full) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    float p0 = 0.f, p1 = 0.f;
-                    if (rok) {
-                        p0 = 2 * i < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
-                        p1 = 2 * i + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse));
+                        ps[i & 3] += p0 + p1;
+                        pk[i] = pack_bf16(p0, p1);
                     }
-                    ps[i & 3] += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = c * 32 + 2 * i;
+                        float p0 = 0.f, p1 = 0.f;
+                        if (rok) {
+                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
+                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
+                        }
+                        ps[i & 3] += p0 + p1;
+                        pk[i] = pack_bf16(p0, p1);
+                    }
                 }
+                tmem_st16(tlane + TM_S(q) + c * 16, pk);
             }
-            // the P buffer and O belong to the previous tile's PV product until it completes
-            if (j >= 1) {
-                if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (uint32_t)(j - 1) & 1u, abort_flag, p.err))) { ok = false; break; }
-                fence_after_sync();
-                // the O rescale is warp-collective TMEM traffic: the whole warp takes it together
-                if (__any_sync(0xffffffffu, need && m != -INFINITY)) {
+            // the previous PV of this sub-tile completed before S_q was written, so O is free;
+            // its rescale is warp-collective TMEM traffic and the whole warp takes it together
+            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t orow[32];
-                        tmem_ld32(tlane + TM_O + c * 32, orow);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t orow[32];
+                    tmem_ld32(tlane + TM_O(q) + c * 32, orow);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-                        tmem_st32(tlane + TM_O + c * 32, orow);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i)
+                        orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    tmem_st32(tlane + TM_O(q) + c * 32, orow);
                 }
             }
             lsum = lsum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
             m = muse;
-            // 128 keys = 16 chunks of 16 B; the chunk index within each 64-key half is
-            // XOR-swizzled with the row (128-byte swizzle, as the MMA descriptor expects)
-#pragma unroll
-            for (int chunk = 0; chunk < 16; ++chunk) {
-                const int half = chunk >> 3, cc = chunk & 7;
-                uint8_t *dst = prow + half * HALF + ((cc ^ sw) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(dst)),
-                             "r"(pk[4 * chunk]), "r"(pk[4 * chunk + 1]), "r"(pk[4 * chunk + 2]),
-                             "r"(pk[4 * chunk + 3])
-                             : "memory");
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_wait_st();
             fence_before_sync();
-            mbar_arrive(BAR(B_PFULL));
-            ++j;
+            mbar_arrive(BAR(B_PFULL + q));
+            ++k;
         }
-        if (ok && j >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (uint32_t)(j - 1) & 1u, abort_flag, p.err))) {
+        if (ok && k >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err))) {
             fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
             __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(tlane + TM_O + c * 32, ov);
+                tmem_ld32(tlane + TM_O(q) + c * 32, ov);
                 if (row_valid) {
-                    uint32_t pk[16];
+                    uint32_t pk2[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        pk[i] = pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+                        pk2[i] = pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
                     uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        dst[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+                        dst[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
                 }
             }
         }
@@ -548,7 +622,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (warp == 1) {
+    if (warp == WARP_MMA) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
@@ -597,7 +671,7 @@ cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     const long q_total = (long)a.B * a.q_Htot * a.q_rows;
     const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
-    if (q_total + BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
+    if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
     if ((e = make_map(&mq, a.q, q_total)) != cudaSuccess) return e;
     if ((e = make_map(&mk, a.k, kv_total)) != cudaSuccess) return e;
@@ -612,7 +686,7 @@ cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
     e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.q_rows + BM - 1) / BM), (unsigned)(a.B * a.Hbr));
+    dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
     attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }

@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
 struct StateBuf {
     __nv_bfloat16 W[C * SD], Q[C * SD], K[C * SD];   // W, Qt, Kt of one chunk
     __nv_bfloat16 U[C * SR], O[C * SR];              // this CTA's 16 columns of Up, Op
+    alignas(16) float gam[4];                        // gam of the chunk (element 0)
 };
 constexpr int NSTAGE = 3;          // chunk operand buffers of the state pass
 struct StateSmem {
@@ -416,6 +417,10 @@ __device__ __forceinline__ void load_chunk(StateBuf &bf, const GdnWorkspace &ws,
         cp_async16(&bf.U[t * SR + hlf * 8], U + (long)t * D + i0 + hlf * 8);
         cp_async16(&bf.O[t * SR + hlf * 8], O + (long)t * D + i0 + hlf * 8);
     }
+    if (tid == 0)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&bf.gam[0])),
+                     "l"(ws.gam + (long)bh * nch + c)
+                     : "memory");
 }
 
 __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspace ws)
@@ -455,7 +460,7 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
         if (c + NSTAGE - 1 < nch)
             load_chunk(s.buf[(c + NSTAGE - 1) % NSTAGE], ws, bh, nch, c + NSTAGE - 1, i0, tid);
         cp_async_commit();
-        const float gam = ws.gam[(long)bh * nch + c];
+        const float gam = cur.gam[0];
 
         // GEMM 1: rows [W; Qt] (warps 0-1: W rows, warps 2-3: Qt rows) times S^T
         {
