@@ -25,14 +25,14 @@
 // softmax). Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in
 // the device error word, every role stops, and the TMEM allocation is released.
 #include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <math.h>
-#include <mutex>
 
 namespace hlta {
 namespace {
+
+using namespace ptx;
 
 constexpr int BM = 128;                 // query rows per sub-tile
 constexpr int QT = 2;                   // query sub-tiles per CTA
@@ -81,68 +81,6 @@ struct TcParams {
 // ---------------------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait: gives up after ~2^32 SM cycles (about two seconds), or at once when another
-// role already gave up; records the expiry in the device error word.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned int *err)
-{
-    if (mbar_try(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > (1LL << 32)) {
-            *abort_flag = 1;
-            atomicOr(err, (unsigned)DEVERR_ATTN_WAIT);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
-                                            uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void fence_before_sync()
 {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -417,11 +355,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const int st = j % NS;
                 const uint32_t ph = (uint32_t)((j / NS) + 1) & 1u;
                 const int krow = (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
-                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + st), ph, abort_flag, p.err)) break;
+                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + st), ph, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
                 mbar_expect_tx(BAR(B_KFULL + st), TILE);
                 tma_load_2d(sbase + SM_K(st), &tk, 0, krow, BAR(B_KFULL + st));
                 tma_load_2d(sbase + SM_K(st) + HALF, &tk, 64, krow, BAR(B_KFULL + st));
-                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + st), ph, abort_flag, p.err)) break;
+                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + st), ph, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
                 mbar_expect_tx(BAR(B_VFULL + st), TILE);
                 tma_load_2d(sbase + SM_V(st), &tv, 0, krow, BAR(B_VFULL + st));
                 tma_load_2d(sbase + SM_V(st) + HALF, &tv, 64, krow, BAR(B_VFULL + st));
@@ -445,11 +383,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
             constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P (TMEM), V MN-major
             int n_s[QT] = {0, 0}, n_pv[QT] = {0, 0};
-            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err);
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err, DEVERR_ATTN_WAIT);
             // S_q = Q_q K^T; first waits for the previous PV of this sub-tile, which reads P_q
             // from the same TMEM columns
             auto issue_s = [&](int q, int st) -> bool {
-                if (n_pv[q] > 0 && !mbar_wait(BAR(B_PVDONE + q), (uint32_t)(n_pv[q] - 1) & 1u, abort_flag, p.err))
+                if (n_pv[q] > 0 && !mbar_wait(BAR(B_PVDONE + q), (uint32_t)(n_pv[q] - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))
                     return false;
                 fence_after_sync();
 #pragma unroll
@@ -464,7 +402,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             };
             // O_q += P_q V, P_q from TMEM (bf16 pairs in the first 64 columns of S_q)
             auto issue_pv = [&](int q, int st) -> bool {
-                if (!mbar_wait(BAR(B_PFULL + q), (uint32_t)n_pv[q] & 1u, abort_flag, p.err)) return false;
+                if (!mbar_wait(BAR(B_PFULL + q), (uint32_t)n_pv[q] & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) return false;
                 fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
@@ -478,7 +416,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
             bool have = ok && wk.next(fk, jt);
             if (have) {
-                ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag, p.err);
+                ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag, p.err, DEVERR_ATTN_WAIT);
                 for (int q = 0; q < QT && ok; ++q)
                     if (active(q, fk)) ok = issue_s(q, 0);
                 if (ok) umma_commit(BAR(B_KEMPTY + 0));
@@ -488,15 +426,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 int fk_n = fk, jt_n = jt;
                 const bool have_n = wk.next(fk_n, jt_n);
                 const int stn = (j + 1) % NS;
-                if (!mbar_wait(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u, abort_flag, p.err)) { ok = false; break; }
-                bool k_ready = false;                   // K of the next tile, waited for once
-                for (int q = 0; q < QT && ok; ++q) {
+                if (!mbar_wait(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
+                // both PV products first, so the second is queued on the tensor pipe before
+                // the issuer blocks on the first one's completion (S_q of the next tile
+                // overwrites the TMEM columns P_q is read from)
+                for (int q = 0; q < QT && ok; ++q)
                     if (active(q, fk_cur)) ok = issue_pv(q, st);
-                    if (ok && have_n && active(q, fk_n)) {
-                        if (!k_ready)
-                            ok = k_ready = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err);
-                        if (ok) ok = issue_s(q, stn);
-                    }
+                if (ok && have_n) {
+                    ok = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT);
+                    for (int q = 0; q < QT && ok; ++q)
+                        if (active(q, fk_n)) ok = issue_s(q, stn);
                 }
                 if (!ok) break;
                 if (have_n) umma_commit(BAR(B_KEMPTY + stn));
@@ -521,25 +460,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         int fk = fstart - 1, jt = wk.tpf - 1, k = 0;
         while (wk.next(fk, jt)) {
             if (!active(q, fk)) continue;               // warp-uniform
-            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
             const int nv = min(BN, p.N - jt * BN);
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
             const bool full = rok && nv == BN;
-            // pass 1: row max over the tile (two 64-column loads, four independent chains)
+            // the whole row of S in one load (one TMEM round trip per tile)
+            uint32_t sr[128];
+            tmem_ld128(tlane + TM_S(q), sr);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (full) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sr[64];
-                tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
-                if (full) {
+                for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+            } else if (rok) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
-                } else if (rok) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        mx[i & 3] = fmaxf(mx[i & 3], hf * 64 + i < nv ? __uint_as_float(sr[i]) : -INFINITY);
-                }
+                for (int i = 0; i < 128; ++i)
+                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
             }
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
@@ -547,18 +483,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const bool need = rok && mnew > m + 8.f;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // pass 2: exponentials of 32 keys at a time; their bf16 pairs (key 2i in the low
-            // half) go to P columns 16c..16c+15, which overlay S columns already read
+            // exponentials 32 keys at a time; their bf16 pairs (key 2i in the low half) go to
+            // P columns 16c..16c+15, over S columns this thread has already read
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32], pk[16];
-                tmem_ld32(tlane + TM_S(q) + c * 32, sr);
+                uint32_t pk[16];
                 if (full) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse));
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), p.sl2, -muse));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), p.sl2, -muse));
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
                     }
@@ -568,8 +503,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         const int col = c * 32 + 2 * i;
                         float p0 = 0.f, p1 = 0.f;
                         if (rok) {
-                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
-                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
+                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
+                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
                         }
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
@@ -597,7 +532,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             mbar_arrive(BAR(B_PFULL + q));
             ++k;
         }
-        if (ok && k >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err))) {
+        if (ok && k >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) {
             fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
             __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
@@ -632,50 +567,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-cudaError_t get_encoder()
-{
-    std::call_once(g_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
-    });
-    return g_encode ? cudaSuccess : cudaErrorNotSupported;
-}
-
-// 2-D view [rows][128] bf16 of a row-major tensor; box = 128 rows x 64 columns, 128B swizzle
-cudaError_t make_map(CUtensorMap *map, const void *base, long rows)
-{
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)BM};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 }  // namespace
 
 cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
 {
     if (a.d != D) return cudaErrorNotSupported;
-    cudaError_t e = get_encoder();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     const long q_total = (long)a.B * a.q_Htot * a.q_rows;
     const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
     if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
-    if ((e = make_map(&mq, a.q, q_total)) != cudaSuccess) return e;
-    if ((e = make_map(&mk, a.k, kv_total)) != cudaSuccess) return e;
-    if ((e = make_map(&mv, a.v, kv_total)) != cudaSuccess) return e;
+    // [rows][128] bf16 views, boxes of 128 rows x 64 columns, 128-byte swizzle
+    if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
     TcParams p;
     p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
     p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(PREP_THREADS) gdn_prep_f32(GdnArgs p, GdnWorks
         Qo[e] = ok ? expf(g[t]) * Qc[t * dp + c] - pw : 0.f;
         Ko[e] = ok ? expf(gn - g[t]) * Kc[t * dp + c] : 0.f;
     }
-    if (tid == 0) ws.gam[(long)bh * nch + chunk] = expf(gn);
+    if (tid == 0) ws.gam[((long)bh * nch + chunk) * 4] = expf(gn);
 }
 
 __global__ void __launch_bounds__(STATE_THREADS) gdn_state_f32(GdnArgs p, GdnWorkspace ws)
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(STATE_THREADS) gdn_state_f32(GdnArgs p, GdnWor
         const float *W = (const float *)ws.W + base, *Up = (const float *)ws.Up + base;
         const float *Op = (const float *)ws.Op + base, *Q = (const float *)ws.Qt + base;
         const float *K = (const float *)ws.Kt + base;
-        const float gam = ws.gam[(long)bh * nch + c];
+        const float gam = ws.gam[((long)bh * nch + c) * 4];
         __syncthreads();
         for (int e = tid; e < C * d; e += STATE_THREADS) {
             Wc[e] = W[e];

@@ -11,17 +11,20 @@
 // Only decays e^{g_t-g_i} with t >= i are formed, so nothing overflows.
 //
 // Two kernels:
-//   prep   one CTA per (chunk, head), every chunk in parallel: KK^T, QK^T, the forward
-//          substitution for T (fp32), then W, Up, Op, Qt on mma.sync bf16 tensor cores;
-//          writes W, Up, Op, Qt, Kt (bf16) and gam (fp32) to the workspace.
+//   prep   one CTA per (chunk, head), every chunk in parallel: Q, K, V of the chunk arrive
+//          by TMA as 128B-swizzled boxes; KK^T, QK^T, the blocked inversion for T (fp32),
+//          then W, Up, Op, Qt on mma.sync bf16 tensor cores; writes W, Up, Op, Qt, Kt (bf16)
+//          and gam (fp32) to the workspace.
 //   state  serial over the chunks of a head; the 128 state rows are split over 8 CTAs of
 //          16 rows (rows of S evolve independently). The state slice lives in registers as
 //          the accumulator fragments of the S update; each chunk does two dependent small
-//          GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync, with the next chunk's operands
-//          prefetched by cp.async.
+//          GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync. The chunk operands stream in by TMA
+//          (swizzled W/Qt/Kt boxes, this CTA's 16 columns of Up/Op, gam) through a 3-stage
+//          mbarrier ring, two chunks ahead; waits are bounded (DEVERR_GDN_WAIT).
 // The serial chain is latency-bound (two dependent 64x16x128-class products per chunk), so
 // it uses register-resident warp MMAs rather than a TMEM round trip per dependent step.
 #include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
 
 #include <math.h>
 
@@ -37,10 +40,8 @@ constexpr int THREADS = 128;
 constexpr int RB = 16;            // state rows per CTA in the state pass
 constexpr int SR = RB + 8;        // padded stride of [64][16] slices
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
+using ptx::smem_u32;
+using ptx::sw128_off;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
 {
@@ -75,14 +76,6 @@ __device__ __forceinline__ void frag_a(uint32_t (&r)[4], const __nv_bfloat16 *ba
     ldsm_x4(r, smem_u32(base + (m0 + (q & 1) * 8 + rr) * ld + k0 + (q >> 1) * 8));
 }
 
-// A fragment (16x16, rows m, cols k) taken from a [K][M] row-major tile (transposed load)
-__device__ __forceinline__ void frag_a_t(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
-                                         int m0, int k0, int lane)
-{
-    const int q = lane >> 3, rr = lane & 7;
-    ldsm_x4_t(r, smem_u32(base + (k0 + (q >> 1) * 8 + rr) * ld + m0 + (q & 1) * 8));
-}
-
 // B fragments of two adjacent n-tiles (k16 x n16) from a [N][K] row-major tile:
 // r[0], r[1] = n-tile n0, r[2], r[3] = n-tile n0 + 8
 __device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
@@ -91,11 +84,25 @@ __device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 
     ldsm_x4(r, smem_u32(base + (n0 + (lane >> 4) * 8 + (lane & 7)) * ld + k0 + ((lane >> 3) & 1) * 8));
 }
 
-// B fragments of two adjacent n-tiles from a [K][N] row-major tile (transposed load)
-__device__ __forceinline__ void frag_b_kn(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
-                                          int k0, int n0, int lane)
+// The same four loaders on a [64][128] bf16 tile in the 128B-swizzled two-half layout
+// (byte offsets from ptx::sw128_off); every ldmatrix row address is one 16-byte chunk.
+__device__ __forceinline__ void frag_a_sw(uint32_t (&r)[4], const uint8_t *tile, int m0, int k0, int lane)
 {
-    ldsm_x4_t(r, smem_u32(base + (k0 + ((lane >> 3) & 1) * 8 + (lane & 7)) * ld + n0 + (lane >> 4) * 8));
+    const int q = lane >> 3, rr = lane & 7;
+    ldsm_x4(r, smem_u32(tile + sw128_off(m0 + (q & 1) * 8 + rr, k0 + (q >> 1) * 8, C)));
+}
+__device__ __forceinline__ void frag_a_t_sw(uint32_t (&r)[4], const uint8_t *tile, int m0, int k0, int lane)
+{
+    const int q = lane >> 3, rr = lane & 7;
+    ldsm_x4_t(r, smem_u32(tile + sw128_off(k0 + (q >> 1) * 8 + rr, m0 + (q & 1) * 8, C)));
+}
+__device__ __forceinline__ void frag_b_nk_sw(uint32_t (&r)[4], const uint8_t *tile, int n0, int k0, int lane)
+{
+    ldsm_x4(r, smem_u32(tile + sw128_off(n0 + (lane >> 4) * 8 + (lane & 7), k0 + ((lane >> 3) & 1) * 8, C)));
+}
+__device__ __forceinline__ void frag_b_kn_sw(uint32_t (&r)[4], const uint8_t *tile, int k0, int n0, int lane)
+{
+    ldsm_x4_t(r, smem_u32(tile + sw128_off(k0 + ((lane >> 3) & 1) * 8 + (lane & 7), n0 + (lane >> 4) * 8, C)));
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
@@ -104,49 +111,40 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ void st_pair(__nv_bfloat16 *p, float lo, float hi)
-{
-    *reinterpret_cast<uint32_t *>(p) = pack2(lo, hi);
-}
-
-__device__ __forceinline__ void cp_async16(void *dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // -----------------------------------------------------------------------------------------
 // prep
 // -----------------------------------------------------------------------------------------
 constexpr int PREP_THREADS = 256;
-constexpr int TP = C + 4;         // fp32 stride of T (17408 bytes = one [64][136] bf16 tile)
+constexpr int TP = C + 4;                  // fp32 row stride of T
+constexpr uint32_t SWT = C * D * 2;        // one swizzled [64][128] bf16 tile: 16 KB
 
-// Shared memory of the prep kernel (about 99 KB, two CTAs per SM). Regions are reused once
-// their contents are dead:
-//   R1: A (fp32 [64][65]) -> T1, T2 (bf16 [64][72] each) -> Op (bf16 [64][136])
-//   R2: T (fp32 [64][68]) -> W (bf16 [64][136])
-//   V:  V -> Up
-//   Q:  Q -> Qt
+// Shared memory of the prep kernel (about 97 KB: two CTAs per SM). Q, K, V arrive by TMA as
+// swizzled tiles; regions are reused once their contents are dead:
+//   R1: A (fp32 [64][65]) -> T1, T2 (bf16 [64][72] each) -> Op (swizzled tile)
+//   R2: T (fp32 [64][68]) -> W (swizzled tile)
+//   V:  V -> Up          Q:  Q -> Qt (in place)
 struct PrepSmem {
-    __nv_bfloat16 Q[C * SD], K[C * SD], V[C * SD];
-    __nv_bfloat16 P[C * SC];
+    alignas(1024) uint8_t Q[SWT];
+    alignas(1024) uint8_t K[SWT];
+    alignas(1024) uint8_t V[SWT];
+    alignas(1024) uint8_t R2[C * TP * 4];
     alignas(16) uint8_t R1[2 * C * SC * 2];
-    alignas(16) uint8_t R2[C * SD * 2];
+    __nv_bfloat16 P[C * SC];
     float X[3 * 256];             // off-diagonal block products of the blocked inversion
     float g[C], eg[C], ek[C], bb[C];
+    alignas(8) uint64_t bar;
+    int abort_flag;
 };
 static_assert(sizeof(float) * C * (C + 1) <= 2 * C * SC * 2, "A must fit in R1");
-static_assert(sizeof(float) * C * TP <= C * SD * 2, "T must fit in R2");
-static_assert(C * SD * 2 <= 2 * C * SC * 2 + 1024, "Op must fit in R1");
+static_assert(SWT <= 2 * C * SC * 2, "Op must fit in R1");
+static_assert(SWT <= C * TP * 4, "W must fit in R2");
 
-// One warp's 16 rows x (NT*8) columns of X = Am ([64][lda] row-major) * Bm ([K][N] row-major,
-// transposed fragment loads), k-steps 0 .. ksteps-1, columns n0 ...
+// One warp's 16 rows x (NT*8) columns of X = Am ([64][lda] row-major, padded) times a
+// swizzled [K][N] tile, k-steps 0 .. ksteps-1, columns n0 ...
 template <int NT>
 __device__ __forceinline__ void gemm_rows_kn(float (&acc)[NT][4], const __nv_bfloat16 *Am, int lda,
-                                             const __nv_bfloat16 *Bm, int ldb, int m0, int n0,
-                                             int ksteps, int lane)
+                                             const uint8_t *Bt, int m0, int n0, int ksteps, int lane)
 {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -157,36 +155,42 @@ __device__ __forceinline__ void gemm_rows_kn(float (&acc)[NT][4], const __nv_bfl
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
             uint32_t b[4];
-            frag_b_kn(b, Bm, ldb, kk * 16, n0 + np * 16, lane);
+            frag_b_kn_sw(b, Bt, kk * 16, n0 + np * 16, lane);
             mma16816(acc[2 * np], a, b[0], b[1]);
             mma16816(acc[2 * np + 1], a, b[2], b[3]);
         }
     }
 }
 
+// accumulator fragment -> swizzled bf16 tile
 template <int NT>
-__device__ __forceinline__ void store_acc_bf16(__nv_bfloat16 *dst, int ld, const float (&acc)[NT][4],
-                                               int m0, int n0, int lane)
+__device__ __forceinline__ void store_acc_sw(uint8_t *tile, const float (&acc)[NT][4], int m0, int n0,
+                                             int lane)
 {
     const int g8 = lane >> 2, tg = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int c = n0 + nt * 8 + 2 * tg;
-        st_pair(&dst[(m0 + g8) * ld + c], acc[nt][0], acc[nt][1]);
-        st_pair(&dst[(m0 + g8 + 8) * ld + c], acc[nt][2], acc[nt][3]);
+        *reinterpret_cast<uint32_t *>(tile + sw128_off(m0 + g8, c, C)) = pack2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<uint32_t *>(tile + sw128_off(m0 + g8 + 8, c, C)) = pack2(acc[nt][2], acc[nt][3]);
     }
 }
 
-__global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnWorkspace ws)
+struct PrepMaps {
+    CUtensorMap q, k, v;          // [B*Htot*L][128] bf16, boxes 64 rows x 64 columns, swizzled
+};
+
+__global__ void __launch_bounds__(PREP_THREADS, 2)
+gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
 {
     extern __shared__ uint8_t smem_raw[];
-    PrepSmem &s = *reinterpret_cast<PrepSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    PrepSmem &s = *reinterpret_cast<PrepSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     float *A = reinterpret_cast<float *>(s.R1);            // [64][65]
     __nv_bfloat16 *T1 = reinterpret_cast<__nv_bfloat16 *>(s.R1);
     __nv_bfloat16 *T2 = T1 + C * SC;
-    __nv_bfloat16 *Op = reinterpret_cast<__nv_bfloat16 *>(s.R1);
+    uint8_t *Op = s.R1;
     float *T = reinterpret_cast<float *>(s.R2);            // [64][68]
-    __nv_bfloat16 *W = reinterpret_cast<__nv_bfloat16 *>(s.R2);
+    uint8_t *W = s.R2;
 
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
@@ -194,28 +198,26 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
     const long t0 = (long)chunk * C;
     const int n = (int)min((long)C, p.L - t0);
     const long head = (long)(b * p.Htot + p.h0 + h) * p.L;
-    const uint4 *gq = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.q + (head + t0) * D);
-    const uint4 *gk = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.k + (head + t0) * D);
-    const uint4 *gv = reinterpret_cast<const uint4 *>((const __nv_bfloat16 *)p.v + (head + t0) * D);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g8 = lane >> 2, tg = lane & 3;
     const int rb = warp & 3, ch = warp >> 2;               // 16-row block, column half
     const int m0 = rb * 16;
+    const uint32_t bar = smem_u32(&s.bar);
 
-    // ---- load the chunk (rows >= n are zero) and the gates
-    for (int e = tid; e < C * (D / 8); e += PREP_THREADS) {
-        const int t = e / (D / 8), c8 = e % (D / 8);
-        uint4 zq = make_uint4(0, 0, 0, 0), zk = zq, zv = zq;
-        if (t < n) {
-            zq = gq[(long)t * (D / 8) + c8];
-            zk = gk[(long)t * (D / 8) + c8];
-            zv = gv[(long)t * (D / 8) + c8];
+    // ---- Q, K, V of the chunk by TMA (two 64-column boxes each)
+    if (tid == 0) {
+        s.abort_flag = 0;
+        ptx::mbar_init(bar, 1);
+        ptx::mbar_init_fence();
+        ptx::mbar_expect_tx(bar, 3 * SWT);
+        const int row = (int)(head + t0);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::tma_load_2d(smem_u32(s.Q + hf * (SWT / 2)), &maps.q, hf * 64, row, bar);
+            ptx::tma_load_2d(smem_u32(s.K + hf * (SWT / 2)), &maps.k, hf * 64, row, bar);
+            ptx::tma_load_2d(smem_u32(s.V + hf * (SWT / 2)), &maps.v, hf * 64, row, bar);
         }
-        *reinterpret_cast<uint4 *>(&s.Q[t * SD + c8 * 8]) = zq;
-        *reinterpret_cast<uint4 *>(&s.K[t * SD + c8 * 8]) = zk;
-        *reinterpret_cast<uint4 *>(&s.V[t * SD + c8 * 8]) = zv;
     }
-    if (warp == 0) {
+    if (warp == 1) {
         // inclusive prefix sum of log a over 64 entries: two per lane, then a warp scan
         const int t = 2 * lane;
         const float l0 = t < n ? logf(p.a[(long)bh * p.L + t0 + t]) : 0.f;
@@ -226,17 +228,38 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
             const float y = __shfl_up_sync(0xffffffffu, x, off);
             if (lane >= off) x += y;
         }
-        const float excl = x - pair;
-        s.g[t] = excl + l0;
+        s.g[t] = x - pair + l0;
         s.g[t + 1] = x;
         s.bb[t] = t < n ? p.b[(long)bh * p.L + t0 + t] : 0.f;
         s.bb[t + 1] = t + 1 < n ? p.b[(long)bh * p.L + t0 + t + 1] : 0.f;
     }
-    __syncthreads();
+    __syncthreads();                                       // barrier initialised, g, bb ready
     if (tid < C) {
         const float gn = s.g[n - 1];
         s.eg[tid] = tid < n ? expf(s.g[tid]) : 0.f;
         s.ek[tid] = tid < n ? expf(gn - s.g[tid]) : 0.f;
+    }
+    for (int e = tid; e < C * TP; e += PREP_THREADS) T[e] = 0.f;
+    const bool landed = ptx::mbar_wait(bar, 0, (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
+    if (!__syncthreads_and(landed)) {
+        // a bounded wait expired: give the three copies a last bounded chance to land
+        if (tid == 0) {
+            const long long t0 = clock64();
+            while (!ptx::mbar_try(bar, 0) && clock64() - t0 < (1LL << 31)) {}
+        }
+        return;
+    }
+    // a ragged last chunk: the box rows past the chunk belong to the next head (or are past
+    // the tensor); zero them so no stray value reaches a product
+    if (n < C) {
+        for (int e = tid; e < (C - n) * 16; e += PREP_THREADS) {
+            const int t = n + (e >> 4), cc = e & 15;
+            const uint32_t off = (cc >> 3) * (SWT / 2) + t * 128 + (cc & 7) * 16;
+            *reinterpret_cast<uint4 *>(s.Q + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(s.K + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(s.V + off) = make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
     }
 
     // ---- KK^T and QK^T: this warp's 16 rows, 32 columns; columns above the diagonal block
@@ -252,12 +275,12 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
         if (live) {
             for (int ks = 0; ks < D / 16; ++ks) {
                 uint32_t ak[4], aq[4];
-                frag_a(ak, s.K, SD, m0, ks * 16, lane);
-                frag_a(aq, s.Q, SD, m0, ks * 16, lane);
+                frag_a_sw(ak, s.K, m0, ks * 16, lane);
+                frag_a_sw(aq, s.Q, m0, ks * 16, lane);
 #pragma unroll
                 for (int np = 0; np < 2; ++np) {
                     uint32_t bk[4];
-                    frag_b_nk(bk, s.K, SD, n0 + np * 16, ks * 16, lane);
+                    frag_b_nk_sw(bk, s.K, n0 + np * 16, ks * 16, lane);
                     mma16816(kk[2 * np], ak, bk[0], bk[1]);
                     mma16816(kk[2 * np + 1], ak, bk[2], bk[3]);
                     mma16816(qk[2 * np], aq, bk[0], bk[1]);
@@ -278,7 +301,6 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
             }
         }
     }
-    for (int e = tid; e < C * TP; e += PREP_THREADS) T[e] = 0.f;
     __syncthreads();
 
     // ---- T = (I + A)^{-1}, blocked by 16: diagonal blocks by forward substitution, then
@@ -294,7 +316,6 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
     }
     __syncthreads();
     for (int I = 1; I < 4; ++I) {
-        // X_IJ = sum_{K=J}^{I-1} A_IK T_KJ for J < I   (I blocks of 256 entries)
         for (int e = tid; e < I * 256; e += PREP_THREADS) {
             const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
             const int row = I * 16 + r, col = J * 16 + c;
@@ -303,7 +324,6 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
             s.X[e] = acc;
         }
         __syncthreads();
-        // T_IJ = -T_II X_IJ
         for (int e = tid; e < I * 256; e += PREP_THREADS) {
             const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
             const int row = I * 16 + r;
@@ -326,34 +346,35 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
     const int nc0 = ch * 64;
     {
         float w[8][4], u[8][4];
-        gemm_rows_kn<8>(w, T1, SC, s.K, SD, m0, nc0, rb + 1, lane);
-        gemm_rows_kn<8>(u, T2, SC, s.V, SD, m0, nc0, rb + 1, lane);
+        gemm_rows_kn<8>(w, T1, SC, s.K, m0, nc0, rb + 1, lane);
+        gemm_rows_kn<8>(u, T2, SC, s.V, m0, nc0, rb + 1, lane);
         __syncthreads();                                   // T, T1, T2 and V are dead now
-        store_acc_bf16<8>(W, SD, w, m0, nc0, lane);
-        store_acc_bf16<8>(s.V, SD, u, m0, nc0, lane);
+        store_acc_sw<8>(W, w, m0, nc0, lane);
+        store_acc_sw<8>(s.V, u, m0, nc0, lane);
     }
     __syncthreads();
     // ---- Op = P Up (into R1), Qt = diag(e^g) Q - P W (in place over Q)
     {
         float op[8][4], pw[8][4];
-        gemm_rows_kn<8>(op, s.P, SC, s.V, SD, m0, nc0, rb + 1, lane);
-        gemm_rows_kn<8>(pw, s.P, SC, W, SD, m0, nc0, rb + 1, lane);
-        store_acc_bf16<8>(Op, SD, op, m0, nc0, lane);
+        gemm_rows_kn<8>(op, s.P, SC, s.V, m0, nc0, rb + 1, lane);
+        gemm_rows_kn<8>(pw, s.P, SC, W, m0, nc0, rb + 1, lane);
+        store_acc_sw<8>(Op, op, m0, nc0, lane);
         const int ta = m0 + g8, tb = ta + 8;
         const float ea = s.eg[ta], eb = s.eg[tb];          // zero for rows >= n
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
             const int c = nc0 + nt * 8 + 2 * tg;
-            __nv_bfloat16 *qa = &s.Q[ta * SD + c], *qb = &s.Q[tb * SD + c];
-            const float qa0 = __bfloat162float(qa[0]), qa1 = __bfloat162float(qa[1]);
-            const float qb0 = __bfloat162float(qb[0]), qb1 = __bfloat162float(qb[1]);
-            st_pair(qa, ta < n ? ea * qa0 - pw[nt][0] : 0.f, ta < n ? ea * qa1 - pw[nt][1] : 0.f);
-            st_pair(qb, tb < n ? eb * qb0 - pw[nt][2] : 0.f, tb < n ? eb * qb1 - pw[nt][3] : 0.f);
+            uint32_t *qa = reinterpret_cast<uint32_t *>(s.Q + sw128_off(ta, c, C));
+            uint32_t *qb = reinterpret_cast<uint32_t *>(s.Q + sw128_off(tb, c, C));
+            const float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(qa));
+            const float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(qb));
+            *qa = pack2(ta < n ? ea * fa.x - pw[nt][0] : 0.f, ta < n ? ea * fa.y - pw[nt][1] : 0.f);
+            *qb = pack2(tb < n ? eb * fb.x - pw[nt][2] : 0.f, tb < n ? eb * fb.y - pw[nt][3] : 0.f);
         }
     }
     __syncthreads();
 
-    // ---- write W, Up, Op, Qt, Kt and gam
+    // ---- write W, Up, Op, Qt, Kt (row-major [64][128] per chunk) and gam
     const long base = ((long)bh * nch + chunk) * C * D;
     uint4 *oW = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.W + base);
     uint4 *oU = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Up + base);
@@ -361,14 +382,14 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
     uint4 *oQ = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Qt + base);
     uint4 *oK = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Kt + base);
     for (int e = tid; e < C * (D / 8); e += PREP_THREADS) {
-        const int t = e / (D / 8), c8 = e % (D / 8);
-        const int so = t * SD + c8 * 8;
-        oW[e] = *reinterpret_cast<const uint4 *>(&W[so]);
-        oU[e] = *reinterpret_cast<const uint4 *>(&s.V[so]);
-        oO[e] = *reinterpret_cast<const uint4 *>(&Op[so]);
-        oQ[e] = *reinterpret_cast<const uint4 *>(&s.Q[so]);
+        const int t = e >> 4, c8 = e & 15;
+        const uint32_t so = sw128_off(t, c8 * 8, C);
+        oW[e] = *reinterpret_cast<const uint4 *>(W + so);
+        oU[e] = *reinterpret_cast<const uint4 *>(s.V + so);
+        oO[e] = *reinterpret_cast<const uint4 *>(Op + so);
+        oQ[e] = *reinterpret_cast<const uint4 *>(s.Q + so);
         const float dk = s.ek[t];
-        uint4 kv = *reinterpret_cast<const uint4 *>(&s.K[so]);
+        uint4 kv = *reinterpret_cast<const uint4 *>(s.K + so);
         __nv_bfloat162 *k2 = reinterpret_cast<__nv_bfloat162 *>(&kv);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -377,56 +398,60 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) gdn_prep_bf16(GdnArgs p, GdnW
         }
         oK[e] = kv;
     }
-    if (tid == 0) ws.gam[(long)bh * nch + chunk] = expf(s.g[n - 1]);
+    if (tid < 4) ws.gam[((long)bh * nch + chunk) * 4 + tid] = tid == 0 ? expf(s.g[n - 1]) : 0.f;
 }
 
 // -----------------------------------------------------------------------------------------
 // state pass
 // -----------------------------------------------------------------------------------------
+constexpr int NSTAGE = 3;                  // chunk operand buffers of the state pass
+constexpr uint32_t SLICE = C * RB * 2;     // this CTA's 16 columns of Up or Op: 2 KB
+constexpr uint32_t STAGE_TX = 3 * SWT + 2 * SLICE + 16;
+
 struct StateBuf {
-    __nv_bfloat16 W[C * SD], Q[C * SD], K[C * SD];   // W, Qt, Kt of one chunk
-    __nv_bfloat16 U[C * SR], O[C * SR];              // this CTA's 16 columns of Up, Op
-    alignas(16) float gam[4];                        // gam of the chunk (element 0)
+    alignas(1024) uint8_t W[SWT];
+    alignas(1024) uint8_t Q[SWT];          // Qt
+    alignas(1024) uint8_t K[SWT];          // Kt
+    alignas(128) __nv_bfloat16 U[C * RB];  // Up[:, i0:i0+16], row-major [64][16]
+    alignas(128) __nv_bfloat16 O[C * RB];  // Op[:, i0:i0+16]
+    alignas(16) float gam[4];              // gam of the chunk (element 0)
 };
-constexpr int NSTAGE = 3;          // chunk operand buffers of the state pass
 struct StateSmem {
     StateBuf buf[NSTAGE];
-    __nv_bfloat16 Sb[RB * SD];                       // state slice as bf16 [i][j]
-    __nv_bfloat16 Ut[RB * SC];                       // U^T slice [i][t]
-    __nv_bfloat16 Os[C * SR];                        // output staging [t][i]
-    float gam[2];
+    __nv_bfloat16 Sb[RB * SD];             // state slice as bf16 [i][j]
+    __nv_bfloat16 Ut[RB * SC];             // U^T slice [i][t]
+    __nv_bfloat16 Os[C * SR];              // output staging [t][i]
+    alignas(8) uint64_t full[NSTAGE];
+    int abort_flag;
 };
 
-__device__ __forceinline__ void load_chunk(StateBuf &bf, const GdnWorkspace &ws, int bh, long nch,
-                                           long c, int i0, int tid)
+struct StateMaps {
+    CUtensorMap W, Q, K;                   // workspace [BHg*nch*64][128]: 64x64 swizzled boxes
+    CUtensorMap U, O;                      // workspace [BHg*nch*64][128]: 64 rows x 16 columns
+};
+
+__device__ __forceinline__ void issue_chunk(StateSmem &s, const StateMaps &maps, const GdnWorkspace &ws,
+                                            int bh, long nch, long c, int i0)
 {
-    const long base = ((long)bh * nch + c) * C * D;
-    const __nv_bfloat16 *W = (const __nv_bfloat16 *)ws.W + base;
-    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)ws.Qt + base;
-    const __nv_bfloat16 *K = (const __nv_bfloat16 *)ws.Kt + base;
-    const __nv_bfloat16 *U = (const __nv_bfloat16 *)ws.Up + base;
-    const __nv_bfloat16 *O = (const __nv_bfloat16 *)ws.Op + base;
-    for (int e = tid; e < C * (D / 8); e += THREADS) {
-        const int t = e / (D / 8), c8 = e % (D / 8);
-        cp_async16(&bf.W[t * SD + c8 * 8], W + (long)t * D + c8 * 8);
-        cp_async16(&bf.Q[t * SD + c8 * 8], Q + (long)t * D + c8 * 8);
-        cp_async16(&bf.K[t * SD + c8 * 8], K + (long)t * D + c8 * 8);
+    StateBuf &bf = s.buf[c % NSTAGE];
+    const uint32_t bar = smem_u32(&s.full[c % NSTAGE]);
+    const int row = (int)(((long)bh * nch + c) * C);
+    ptx::mbar_expect_tx(bar, STAGE_TX);
+    for (int hf = 0; hf < 2; ++hf) {
+        ptx::tma_load_2d(smem_u32(bf.W + hf * (SWT / 2)), &maps.W, hf * 64, row, bar);
+        ptx::tma_load_2d(smem_u32(bf.Q + hf * (SWT / 2)), &maps.Q, hf * 64, row, bar);
+        ptx::tma_load_2d(smem_u32(bf.K + hf * (SWT / 2)), &maps.K, hf * 64, row, bar);
     }
-    for (int e = tid; e < C * 2; e += THREADS) {
-        const int t = e >> 1, hlf = e & 1;
-        cp_async16(&bf.U[t * SR + hlf * 8], U + (long)t * D + i0 + hlf * 8);
-        cp_async16(&bf.O[t * SR + hlf * 8], O + (long)t * D + i0 + hlf * 8);
-    }
-    if (tid == 0)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&bf.gam[0])),
-                     "l"(ws.gam + (long)bh * nch + c)
-                     : "memory");
+    ptx::tma_load_2d(smem_u32(bf.U), &maps.U, i0, row, bar);
+    ptx::tma_load_2d(smem_u32(bf.O), &maps.O, i0, row, bar);
+    ptx::bulk_load(smem_u32(bf.gam), ws.gam + ((long)bh * nch + c) * 4, 16, bar);
 }
 
-__global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspace ws)
+__global__ void __launch_bounds__(THREADS)
+gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace ws)
 {
     extern __shared__ uint8_t smem_raw[];
-    StateSmem &s = *reinterpret_cast<StateSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    StateSmem &s = *reinterpret_cast<StateSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int i0 = blockIdx.x * RB, bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long nch = gdn_num_chunks(p.L, C);
@@ -434,6 +459,11 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
     const int g8 = lane >> 2, tg = lane & 3;
     __nv_bfloat16 *o = (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D;
 
+    if (tid == 0) {
+        s.abort_flag = 0;
+        for (int st = 0; st < NSTAGE; ++st) ptx::mbar_init(smem_u32(&s.full[st]), 1);
+        ptx::mbar_init_fence();
+    }
     // state fragments: this warp owns key columns j in [32w, 32w+32) of S^T = D[m=j][n=i]
     float st[2][2][4];
 #pragma unroll
@@ -447,24 +477,25 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
                 st[mt][nt][e] = p.S0 ? p.S0[((long)bh * D + i0 + i) * D + j] : 0.f;
                 s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
             }
+    __syncthreads();
+    if (tid == 0)
+        for (long c = 0; c < NSTAGE - 1 && c < nch; ++c) issue_chunk(s, maps, ws, bh, nch, c, i0);
 
-    // prefetch NSTAGE-1 chunks ahead; one cp.async group per chunk (empty groups past the end)
-    for (int c = 0; c < NSTAGE - 1; ++c) {
-        if (c < nch) load_chunk(s.buf[c], ws, bh, nch, c, i0, tid);
-        cp_async_commit();
-    }
+    bool ok = true;
+    long c_fail = 0;
     for (long c = 0; c < nch; ++c) {
         StateBuf &cur = s.buf[c % NSTAGE];
-        cp_async_wait<NSTAGE - 2>();           // the group of chunk c has landed
-        __syncthreads();                       // ... for every thread; Sb holds the incoming state
-        if (c + NSTAGE - 1 < nch)
-            load_chunk(s.buf[(c + NSTAGE - 1) % NSTAGE], ws, bh, nch, c + NSTAGE - 1, i0, tid);
-        cp_async_commit();
+        const bool landed = ptx::mbar_wait(smem_u32(&s.full[c % NSTAGE]), (uint32_t)(c / NSTAGE) & 1u,
+                                           (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
+        // chunk c has landed for every thread, and Sb holds the incoming state
+        if (!__syncthreads_and(landed)) { ok = false; c_fail = c; break; }
+        // the stage of chunk c-1 is free again (every thread passed the barrier above)
+        if (tid == 0 && c + NSTAGE - 1 < nch) issue_chunk(s, maps, ws, bh, nch, c + NSTAGE - 1, i0);
         const float gam = cur.gam[0];
 
         // GEMM 1: rows [W; Qt] (warps 0-1: W rows, warps 2-3: Qt rows) times S^T
         {
-            const __nv_bfloat16 *Am = warp < 2 ? cur.W : cur.Q;
+            const uint8_t *Am = warp < 2 ? cur.W : cur.Q;
             const int mb = (warp & 1) * 32;
             float acc[2][2][4];
 #pragma unroll
@@ -480,7 +511,7 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                     uint32_t a[4];
-                    frag_a(a, Am, SD, mb + mt * 16, ks * 16, lane);
+                    frag_a_sw(a, Am, mb + mt * 16, ks * 16, lane);
                     mma16816(acc[mt][0], a, bsf[0], bsf[1]);
                     mma16816(acc[mt][1], a, bsf[2], bsf[3]);
                 }
@@ -494,10 +525,10 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
                         const int t = mb + mt * 16 + g8 + (e >> 1) * 8;
                         const int i = nt * 8 + 2 * tg + (e & 1);
                         if (warp < 2) {
-                            const float u = __bfloat162float(cur.U[t * SR + i]) - acc[mt][nt][e];
+                            const float u = __bfloat162float(cur.U[t * RB + i]) - acc[mt][nt][e];
                             s.Ut[i * SC + t] = __float2bfloat16_rn(u);
                         } else {
-                            const float ov = __bfloat162float(cur.O[t * SR + i]) + acc[mt][nt][e];
+                            const float ov = __bfloat162float(cur.O[t * RB + i]) + acc[mt][nt][e];
                             s.Os[t * SR + i] = __float2bfloat16_rn(ov);
                         }
                     }
@@ -526,7 +557,7 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 uint32_t a[4];
-                frag_a_t(a, cur.K, SD, warp * 32 + mt * 16, ks * 16, lane);
+                frag_a_t_sw(a, cur.K, warp * 32 + mt * 16, ks * 16, lane);
                 mma16816(st[mt][0], a, bu[0], bu[1]);
                 mma16816(st[mt][1], a, bu[2], bu[3]);
             }
@@ -544,7 +575,18 @@ __global__ void __launch_bounds__(THREADS) gdn_state_bf16(GdnArgs p, GdnWorkspac
                     s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
                 }
     }
-    cp_async_wait<0>();
+    if (!ok) {
+        // a bounded wait expired: let the copies this CTA issued and never consumed land
+        // before it exits (chunks c .. issued-1, each on its own stage and phase)
+        if (tid == 0) {
+            const long long t0 = clock64();
+            for (long cc = c_fail; cc < c_fail + NSTAGE - 1 && cc < nch; ++cc) {
+                const uint32_t bar = smem_u32(&s.full[cc % NSTAGE]);
+                while (!ptx::mbar_try(bar, (uint32_t)(cc / NSTAGE) & 1u) && clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+        return;
+    }
     if (p.S_out) {
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
@@ -565,19 +607,32 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
 {
     if (g.d != D) return cudaErrorNotSupported;
     const long nch = gdn_num_chunks(g.L, C);
-    if (nch > 0x7fffffffL) return cudaErrorNotSupported;
-    GdnWorkspace ws = gdn_workspace_carve(g.ws, (long)g.B * g.Hg, g.L, D, C, true);
-    const size_t smem_prep = sizeof(PrepSmem) + 128;   // about 99 KB: two CTAs per SM
-    const size_t smem_state = sizeof(StateSmem) + 128;
-    cudaError_t e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_prep);
+    const long BH = (long)g.B * g.Hg;
+    const long in_rows = (long)g.B * g.Htot * g.L;
+    const long ws_rows = BH * nch * C;
+    if (nch > 0x7fffffffL || in_rows + C >= (1L << 31) || ws_rows >= (1L << 31))
+        return cudaErrorNotSupported;
+    GdnWorkspace ws = gdn_workspace_carve(g.ws, BH, g.L, D, C, true);
+    cudaError_t e;
+    PrepMaps pm;
+    if ((e = make_tmap_2d_bf16(&pm.q, g.q, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&pm.k, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&pm.v, g.v, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    StateMaps sm;
+    if ((e = make_tmap_2d_bf16(&sm.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows, D, RB, C, false)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows, D, RB, C, false)) != cudaSuccess) return e;
+    const size_t smem_prep = sizeof(PrepSmem) + 1024;
+    const size_t smem_state = sizeof(StateSmem) + 1024;
+    e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_state);
+    e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
     if (e != cudaSuccess) return e;
-    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), PREP_THREADS, smem_prep, s>>>(g, ws);
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / RB, (unsigned)(g.B * g.Hg)), THREADS, smem_state, s>>>(g, ws);
+    gdn_state_bf16<<<dim3(D / RB, (unsigned)BH), THREADS, smem_state, s>>>(sm, g, ws);
     return cudaGetLastError();
 }
 

@@ -169,7 +169,7 @@ size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
     const size_t el = bf16 ? 2 : 4;
     const size_t nch = (size_t)gdn_num_chunks(L, C);
     const size_t arr = ((size_t)BH * nch * C * d * el + 255) & ~(size_t)255;
-    return 5 * arr + (((size_t)BH * nch * sizeof(float) + 255) & ~(size_t)255);
+    return 5 * arr + (((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255);
 }
 
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16)

@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -47,8 +48,8 @@ struct GdnArgs {
 // Chunk workspace (per GDN head, per chunk of C tokens; elements of type E):
 //   W  = T diag(b e^g) K,   Up = T diag(b) V,   Op = P Up,
 //   Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K        each [C][d]
-//   gam = e^{g_C}                                             one float per chunk
-// laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks].
+//   gam = e^{g_C}                               one float per chunk, in a 16-byte slot
+// laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks][4].
 struct GdnWorkspace {
     void *W, *Up, *Op, *Qt, *Kt;
     float *gam;
@@ -57,6 +58,11 @@ struct GdnWorkspace {
 __host__ __device__ inline long gdn_num_chunks(long L, int C) { return (L + C - 1) / C; }
 size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16);
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16);
+
+// 2-D TMA tensor map over a row-major [rows][cols] bf16 tensor with a box of
+// box_rows x box_cols, 128-byte swizzle or none.
+cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                              uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 
 // Launchers. Return cudaGetLastError() of their launches.
 cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);

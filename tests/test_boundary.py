@@ -63,11 +63,11 @@ def test_bad_shapes_rejected_on_host(lib):
 
 def test_workspace_sizes(lib):
     import linear_video_world_b200 as h
-    # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16 plus one float per chunk
+    # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16 plus a 16-byte slot per chunk
     n = h.hlta_gdn_workspace_bytes(1, 8, 32760, 128, 64, h.HLTA_BF16)
     nch = (32760 + 63) // 64
     arr = 8 * nch * 64 * 128 * 2
-    assert n == 5 * arr + ((8 * nch * 4 + 255) // 256) * 256
+    assert n == 5 * arr + ((8 * nch * 16 + 255) // 256) * 256
     assert h.hlta_hybrid_workspace_bytes(1, 8, 21, 1560, 128, 64, h.HLTA_BF16) == n
     assert h.hlta_gdn_workspace_bytes(1, 1, 10, 64, 64, h.HLTA_FP32) > 5 * 64 * 64 * 4 - 1
 
