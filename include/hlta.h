@@ -113,6 +113,31 @@ hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v,
                                void *workspace, size_t ws_bytes,
                                hlta_dtype dt, void *stream);
 
+/*
+ * hlta_gdn_chunk_fwd for callers that cannot allocate device memory (no counterpart on the
+ * pages: an interface addition of this library). Some callers may not allocate: code embedded
+ * in a host application that owns the device-memory budget and passes in only inputs and
+ * outputs, or a latency-critical loop that must never enter the allocator. This entry point
+ * takes no workspace; its scratch is a fixed array of HLTA_STATIC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that uses the library keeps reserved until the process exits.
+ * It calls no allocator (no cudaMalloc / cudaFree, no allocating library routine).
+ * Arguments and results are those of hlta_gdn_chunk_fwd (same kernels). Problems whose
+ * hlta_gdn_workspace_bytes() exceeds HLTA_STATIC_SCRATCH_BYTES are rejected with
+ * HLTA_ERR_INVALID_ARG before anything is enqueued.
+ * The first call on a device looks up the scratch's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture on that device.
+ * Every call on a device shares the one scratch array, and the array keeps the last call's
+ * contents (nothing in it needs to start at zero). Calls whose GPU work overlaps in time (on
+ * different streams, or from different host threads without ordering) race on the scratch and
+ * give wrong results; order them on one stream.
+ */
+#define HLTA_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+hlta_status hlta_gdn_chunk_fwd_static(const void *q, const void *k, const void *v,
+                                      const float *a, const float *b, void *o,
+                                      const float *S0, float *S_out,
+                                      int B, int H, long L, int d, int chunk,
+                                      hlta_dtype dt, void *stream);
+
 /* Workspace size in bytes for hlta_hybrid_fwd. */
 size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk,
                                    hlta_dtype dt);

@@ -42,6 +42,7 @@ def _load() -> ctypes.CDLL:
         "hlta_dswa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, F, I, P]),
         "hlta_gdn_workspace_bytes": (Z, [I, I, L, I, I, I]),
         "hlta_gdn_chunk_fwd": (I, [P, P, P, P, P, P, P, P, I, I, L, I, I, P, Z, I, P]),
+        "hlta_gdn_chunk_fwd_static": (I, [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P]),
         "hlta_hybrid_workspace_bytes": (Z, [I, I, I, I, I, I, I]),
         "hlta_hybrid_fwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F,
                                 P, Z, I, P]),
@@ -123,6 +124,18 @@ def hlta_gdn_chunk_fwd(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, workspace
     _check(_lib.hlta_gdn_chunk_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(o), _p(S0), _p(S_out),
                                    B, H, L, d, chunk, _p(workspace), workspace.numel() * workspace.element_size(),
                                    _dt(q), _stream(stream)))
+
+
+HLTA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def hlta_gdn_chunk_fwd_static(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, stream=None):
+    """hlta_gdn_chunk_fwd without a workspace argument: the library's built-in scratch is used
+    (for callers that may not allocate device memory; see include/hlta.h)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (a, "a"), (b, "b"), (o, "o")):
+        _need(t, n)
+    _check(_lib.hlta_gdn_chunk_fwd_static(_p(q), _p(k), _p(v), _p(a), _p(b), _p(o), _p(S0),
+                                          _p(S_out), B, H, L, d, chunk, _dt(q), _stream(stream)))
 
 
 def hlta_hybrid_workspace_bytes(B, Hg, T, N, d, chunk=64, dt=HLTA_BF16) -> int:

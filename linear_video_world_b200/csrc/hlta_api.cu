@@ -184,6 +184,15 @@ GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool
     return w;
 }
 
+int record_error_impl(int st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_msg, sizeof t_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
 unsigned int *device_error_word()
 {
     DeviceCtx *c;

@@ -59,6 +59,10 @@ __host__ __device__ inline long gdn_num_chunks(long L, int C) { return (L + C - 
 size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16);
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16);
 
+// Records the thread-local message returned by hlta_last_error() and returns `st`.
+int record_error_impl(int st, const char *fmt, ...);
+#define record_error(st, ...) ((hlta_status)::hlta::record_error_impl((int)(st), __VA_ARGS__))
+
 // 2-D TMA tensor map over a row-major [rows][cols] bf16 tensor with a box of
 // box_rows x box_cols, 128-byte swizzle or none.
 cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
