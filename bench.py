@@ -151,7 +151,7 @@ def oracle_sample(x, wl, rows: int, seed: int):
     import oracle
     g = torch.Generator().manual_seed(seed)
     pos = torch.randint(0, wl.L, (rows,), generator=g).numpy()
-    q, k, v = (x[n][0] for n in "qkv")          # [H, L, d], batch 0
+    q, k, v = (x[n][0] for n in "qkv")          # [H, L, d] float32 numpy, batch 0
     Hs, Hd, Hg = wl.Hs, wl.Hd, wl.Hg
     t0 = time.perf_counter()
     if Hs:
@@ -167,15 +167,25 @@ def oracle_sample(x, wl, rows: int, seed: int):
     return rows, time.perf_counter() - t0
 
 
+def host_f32(x):
+    """The sampled inputs as float32 numpy arrays (bf16 values are exact in float32), converted
+    once so that the timed oracle calls do not pay for the conversion."""
+    import numpy as np
+    return {n: np.ascontiguousarray(x[n].float().numpy()) for n in "qkvab"}
+
+
 def calibrated_rows(x, wl, seconds: float, seed: int) -> int:
     n0 = 16
     _, t = oracle_sample(x, wl, n0, seed)
-    return max(n0, int(n0 * seconds / max(t, 1e-3)))
+    n1 = max(n0, int(n0 * min(seconds, 2.0) / max(t, 1e-3)))
+    _, t1 = oracle_sample(x, wl, n1, seed + 1)
+    return max(n0, int(n1 * seconds / max(t1, 1e-3)))
 
 
 def cpu_baseline(x, wl, seconds: float):
     import oracle
     oracle.build()
+    x = host_f32(x)
     rows = calibrated_rows(x, wl, seconds, seed=123)
     tokens, sec = oracle_sample(x, wl, rows, seed=124)
     return {"value": tokens * wl.B / sec, "unit": "tokens/s", "cores": oracle.num_threads(),
@@ -189,7 +199,7 @@ def run_reference(args, wl):
     import hlta_inputs as hi
     import oracle
     oracle.build()
-    x = hi.make_inputs(wl, seed=0)
+    x = host_f32(hi.make_inputs(wl, seed=0))
     budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))   # CPU seconds per step
     rows = calibrated_rows(x, wl, max(0.5, budget), seed=7)
     for i in range(args.warmup):
