@@ -169,26 +169,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&x)[32])
         : "memory");
 }
 
-// 128 consecutive fp32 columns of this thread's TMEM lane, one instruction plus its wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&x)[128])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
-        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
-        "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-        "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
-        "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
-        "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
-        "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
-        "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, "
-        "[%128];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : TMEM_REGS32(x), TMEM_REGS32((x + 32)), TMEM_REGS32((x + 64)), TMEM_REGS32((x + 96))
-        : "r"(taddr)
-        : "memory");
-}
-
 // 64 consecutive fp32 columns, load and wait in one statement
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&x)[64])
 {
@@ -232,6 +212,22 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA pipe, for a share of the softmax exponentials (the MUFU unit computes the
+// rest). Range reduction x = n + f with n = round(x) by the 1.5*2^23 rounding trick (t's low
+// mantissa bits hold n, and bits(t) << 23 = n << 23), f in [-1/2, 1/2]; 2^f by a cubic with
+// p(0) = 1 whose coefficients minimise the maximum relative error on [-1/2, 1/2] (fitted for
+// this kernel by linear programming; max relative error 1.0e-4, twenty times below the bf16
+// rounding P goes through); 2^n added to the exponent field. Valid for x in [-125, 126];
+// smaller x is clamped (the result, ~2^-125, is then negligible next to the row maximum's 1).
+__device__ __forceinline__ float exp2_fma(float x)
+{
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float pf = fmaf(fmaf(fmaf(0.055008937f, f, 0.24221095f), f, 0.6932829f), f, 1.f);
+    return __int_as_float(__float_as_int(pf) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
@@ -382,14 +378,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
             constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P (TMEM), V MN-major
-            int n_s[QT] = {0, 0}, n_pv[QT] = {0, 0};
+            int n_pv[QT] = {0, 0};
             bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err, DEVERR_ATTN_WAIT);
-            // S_q = Q_q K^T; first waits for the previous PV of this sub-tile, which reads P_q
-            // from the same TMEM columns
+            // S_q = Q_q K^T. It overwrites the TMEM columns the previous PV of this sub-tile
+            // reads P_q from; tcgen05.mma operations issued by one thread execute in issue
+            // order, so it is issued right behind that PV without waiting for it.
             auto issue_s = [&](int q, int st) -> bool {
-                if (n_pv[q] > 0 && !mbar_wait(BAR(B_PVDONE + q), (uint32_t)(n_pv[q] - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))
-                    return false;
-                fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
@@ -397,7 +391,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                               sw128_desc(sbase + SM_K(st) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(BAR(B_SFULL + q));
-                ++n_s[q];
                 return true;
             };
             // O_q += P_q V, P_q from TMEM (bf16 pairs in the first 64 columns of S_q)
@@ -427,15 +420,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const bool have_n = wk.next(fk_n, jt_n);
                 const int stn = (j + 1) % NS;
                 if (!mbar_wait(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
-                // both PV products first, so the second is queued on the tensor pipe before
-                // the issuer blocks on the first one's completion (S_q of the next tile
-                // overwrites the TMEM columns P_q is read from)
-                for (int q = 0; q < QT && ok; ++q)
+                bool k_ready = false;                   // K of the next tile, waited for once
+                for (int q = 0; q < QT && ok; ++q) {
                     if (active(q, fk_cur)) ok = issue_pv(q, st);
-                if (ok && have_n) {
-                    ok = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT);
-                    for (int q = 0; q < QT && ok; ++q)
-                        if (active(q, fk_n)) ok = issue_s(q, stn);
+                    if (ok && have_n && active(q, fk_n)) {
+                        if (!k_ready)
+                            ok = k_ready = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT);
+                        if (ok) ok = issue_s(q, stn);
+                    }
                 }
                 if (!ok) break;
                 if (have_n) umma_commit(BAR(B_KEMPTY + stn));
@@ -465,17 +457,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const int nv = min(BN, p.N - jt * BN);
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
             const bool full = rok && nv == BN;
-            // the whole row of S in one load (one TMEM round trip per tile)
-            uint32_t sr[128];
-            tmem_ld128(tlane + TM_S(q), sr);
+            // pass 1: row max over the tile (two 64-column loads, four independent chains)
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (full) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
-            } else if (rok) {
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t sr[64];
+                tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
+                if (full) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
-                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
+                    for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+                } else if (rok) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        mx[i & 3] = fmaxf(mx[i & 3], hf * 64 + i < nv ? __uint_as_float(sr[i]) : -INFINITY);
+                }
             }
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
@@ -483,17 +478,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const bool need = rok && mnew > m + 8.f;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // exponentials 32 keys at a time; their bf16 pairs (key 2i in the low half) go to
-            // P columns 16c..16c+15, over S columns this thread has already read
+            // pass 2: exponentials of 32 keys at a time; their bf16 pairs (key 2i in the low
+            // half) go to P columns 16c..16c+15, which overlay S columns already read
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16];
+                uint32_t sr[32], pk[16];
+                tmem_ld32(tlane + TM_S(q) + c * 32, sr);
                 if (full) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), p.sl2, -muse));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), p.sl2, -muse));
+                        // one exponential in four on the FMA pipe, three on the MUFU unit
+                        const float x0 = fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse);
+                        const float x1 = fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse);
+                        const float p0 = ex2(x0);
+                        const float p1 = (i & 1) ? exp2_fma(x1) : ex2(x1);
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
                     }
@@ -503,8 +502,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         const int col = c * 32 + 2 * i;
                         float p0 = 0.f, p1 = 0.f;
                         if (rok) {
-                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
-                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
+                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
+                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
                         }
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
@@ -512,7 +511,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 }
                 tmem_st16(tlane + TM_S(q) + c * 16, pk);
             }
-            // the previous PV of this sub-tile completed before S_q was written, so O is free;
+            // S_FULL completes only when every MMA issued before it has, so the previous PV of
+            // this sub-tile is done (O is free, P_q may be overwritten);
             // its rescale is warp-collective TMEM traffic and the whole warp takes it together
             if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
 #pragma unroll
