@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stream", action="store_true",
+                    help="skip the streaming-step measurement (detail.stream)")
     return ap.parse_args()
 
 
@@ -64,6 +66,74 @@ def work(wl):
     pd = window_pairs(wl.T, wl.N, wl.w_dswa, wl.r) * wl.B * wl.Hd
     gdn_bytes = wl.B * wl.Hg * wl.L * (4 * wl.d * 2 + 2 * 4)
     return {"swa_flop": 4 * wl.d * ps, "dswa_flop": 4 * wl.d * pd, "gdn_bytes": gdn_bytes}
+
+
+class Replicas:
+    """The N > 1 plumbing: one independent replica per rank (no exchange on the data path);
+    barriers bracket the timed region and the device-timed duration is reduced as the max
+    over ranks. Works with any torch.distributed backend (NCCL on GPUs, gloo in CPU tests)."""
+
+    def __init__(self, world: int, device):
+        self.world, self.device = world, device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def allmax(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], device=self.device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def job_value(self, units_per_rank: int, ms_max: float) -> float:
+        """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+        return units_per_rank * self.world / (ms_max / 1e3)
+
+
+def stream_step_flop(wl, f: int) -> int:
+    """Algorithmic softmax FLOP of one streaming step at frame f (4*d per valid pair)."""
+    taps_s = sum(1 for i in range(wl.w_swa) if f - i >= 0)
+    taps_d = sum(1 for i in range(wl.w_dswa) if f - wl.r * i >= 0)
+    return 4 * wl.d * wl.B * wl.N * wl.N * (taps_s * wl.Hs + taps_d * wl.Hd)
+
+
+def measure_stream(h, torch, dev, warm: int = 24, steps: int = 40) -> dict:
+    """Steady-state step time of the streaming cache on the 8-rollout 480P stream workload.
+
+    The first `warm` steps fill the rings (every tap frame exists from frame r*(w-1) on);
+    `steps` further steps are timed with CUDA events. Inputs: 4 seeded frames, cycled."""
+    import hlta_inputs as hi
+    sw = hi.WORKLOADS["stream_480p"]
+    x = hi.make_inputs(sw, seed=7, frames=4)
+    fr = []
+    for i in range(4):
+        sl = slice(i * sw.N, (i + 1) * sw.N)
+        fr.append({n: x[n][:, :, sl].contiguous().to(dev) for n in "qkvab"})
+    o = torch.empty_like(fr[0]["q"])
+    st = h.Stream(sw.B, sw.Hs, sw.Hd, sw.Hg, sw.N, sw.d, sw.w_swa, sw.w_dswa, sw.r, sw.chunk)
+    for i in range(warm):
+        f = fr[i % 4]
+        st.step(f["q"], f["k"], f["v"], f["a"], f["b"], out=o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        f = fr[i % 4]
+        st.step(f["q"], f["k"], f["v"], f["a"], f["b"], out=o)
+    e1.record()
+    torch.cuda.synchronize()
+    st.close()
+    ms = e0.elapsed_time(e1) / steps
+    flop = stream_step_flop(sw, warm + steps)
+    return {"workload": f"{sw.name}: B={sw.B} new frame N={sw.N} heads {sw.Hs}/{sw.Hd}/{sw.Hg} "
+                        f"SWA w={sw.w_swa} DSWA w={sw.w_dswa} r={sw.r}; steady state (frame >= {warm})",
+            "ms_per_step": ms, "tokens_per_s": sw.B * sw.N / (ms / 1e3),
+            "softmax_tflops": flop / (ms / 1e3) / 1e12, "launches_per_step": 8}
 
 
 def peaks():
@@ -175,11 +245,12 @@ def host_f32(x):
 
 
 def calibrated_rows(x, wl, seconds: float, seed: int) -> int:
-    n0 = 16
+    """Sample size (tokens) whose oracle time is about `seconds`, at most the whole clip."""
+    n0 = min(16, wl.L)
     _, t = oracle_sample(x, wl, n0, seed)
-    n1 = max(n0, int(n0 * min(seconds, 2.0) / max(t, 1e-3)))
+    n1 = min(wl.L, max(n0, int(n0 * min(seconds, 2.0) / max(t, 1e-3))))
     _, t1 = oracle_sample(x, wl, n1, seed + 1)
-    return max(n0, int(n1 * seconds / max(t1, 1e-3)))
+    return min(wl.L, max(n0, int(n1 * seconds / max(t1, 1e-3))))
 
 
 def cpu_baseline(x, wl, seconds: float):
@@ -261,16 +332,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def allmax(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    rep = Replicas(world, dev)
+    barrier, allmax = rep.barrier, rep.allmax
 
     x = hi.make_inputs(wl, seed=rank)
     q, k, v, a, b = (x[n].to(dev) for n in "qkvab")
@@ -318,7 +381,7 @@ def main():
     gdn_ms = statistics.mean(p[3].elapsed_time(p[4]) for p in prof)
     assert h.hlta_device_status() == 0
     tokens = wl.B * wl.L
-    value = tokens * world / (ms / 1e3)
+    value = rep.job_value(tokens, ms)
 
     # ---- end to end through the C ABI with host buffers -----------------------------------
     pin = {n: x[n].pin_memory() for n in "qkvab"}
@@ -348,6 +411,30 @@ def main():
     h2d = sum(pin[n].numel() * pin[n].element_size() for n in "qkvab")
     d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
 
+    # ---- the two softmax launches alone (no GDN branch sharing the SMs) --------------------
+    hs, hd = slice(0, wl.Hs), slice(wl.Hs, wl.Hs + wl.Hd)
+    sub = {n: (x_[:, hs].contiguous(), x_[:, hd].contiguous()) for n, x_ in (("q", q), ("k", k), ("v", v))}
+    o_s, o_d = torch.empty_like(sub["q"][0]), torch.empty_like(sub["q"][1])
+
+    def attn_only():
+        h.hlta_swa_fwd(sub["q"][0], sub["k"][0], sub["v"][0], o_s, wl.B, wl.Hs, wl.T, wl.N, wl.d,
+                       wl.w_swa, 0.0)
+        h.hlta_dswa_fwd(sub["q"][1], sub["k"][1], sub["v"][1], o_d, wl.B, wl.Hd, wl.T, wl.N, wl.d,
+                        wl.w_dswa, wl.r, 0.0)
+
+    for _ in range(3):
+        attn_only()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(K):
+        attn_only()
+    a1.record()
+    torch.cuda.synchronize()
+    attn_alone_ms = a0.elapsed_time(a1) / K
+    del sub, o_s, o_d
+    stream_detail = None if args.no_stream else measure_stream(h, torch, dev)
+
     # ---- roofline of the dominant kernel (windowed attention, both launches) --------------
     wk = work(wl)
     pk, pk_kind = peaks()
@@ -368,16 +455,24 @@ def main():
         "dswa_tflops": wk["dswa_flop"] / (dswa_ms / 1e3) / 1e12,
         "gdn_gbs": gdn_gbs, "gdn_hbm_frac": gdn_gbs / hbm,
         "hbm_peak_gbs": hbm, "hbm_peak_kind": pk_kind,
-        "note": "GDN runs on a second stream concurrently with SWA/DSWA; its HBM fraction "
-                "uses the algorithmic q/k/v/o + gate bytes of the 8 GDN heads",
+        "attn_alone_ms": attn_alone_ms,
+        "attn_alone_tflops": attn_flop / (attn_alone_ms / 1e3) / 1e12,
+        "attn_alone_frac": attn_flop / (attn_alone_ms / 1e3) / 1e12 / float(pk.get("bf16_tflops")),
+        "note": "GDN runs on a second stream concurrently with SWA/DSWA, so swa_ms/dswa_ms (and "
+                "the roofline) include sharing the SMs with it; attn_alone_* times the two "
+                "softmax launches by themselves against the burst bf16 peak. The GDN HBM "
+                "fraction uses the algorithmic q/k/v/o + gate bytes of the GDN heads",
     }
+    if stream_detail is not None:
+        stream_detail["softmax_frac"] = stream_detail["softmax_tflops"] / peak
+        detail["stream"] = stream_detail
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, per-rank seed)",
         "config": config_of(wl), "clocks": clocks,
-        "e2e": {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": rep.job_value(tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 4 * K, "roofline": roofline, "detail": detail,
     }

@@ -9,18 +9,20 @@
 // per-element mask (row frame vs. key frame, ragged frame end) removes what a row must not
 // see.
 //
-// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 12 warps
-// in three warpgroups (softmax 0, softmax 1, and one holding the TMA and MMA warps):
-//   warp 8      TMA producer: Q (both sub-tiles) once, then K and V tiles into a 2-stage ring
-//               (128B swizzle); the sub-tiles share every K/V tile
-//   warp 9      TMEM owner and MMA issuer (tcgen05.mma kind::f16): S_q = Q_q K_j^T into TMEM,
-//               O_q += P_q V_j with P_q read from TMEM (written there by the softmax over the
-//               first 64 columns of S_q) and V_j an MN-major shared-memory operand; order
-//               S_0(j) S_1(j) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ... so the tensor pipe works
-//               on one sub-tile while the other sub-tile's softmax runs
-//   warps 0..3  softmax of sub-tile 0, warps 4..7 softmax of sub-tile 1: one thread per query
-//               row; S from TMEM, running max (O rescaled in TMEM only when the max grows by
-//               more than 2^8), P (bf16) back to TMEM, final normalisation of O.
+// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 18 warps:
+//   warps 0..7    softmax of sub-tile 0, warps 8..15 softmax of sub-tile 1: each query row is
+//                 shared by two threads (same TMEM lane, warps w and w+4), one per 64-key half
+//                 of every S tile; they agree on the row max through shared memory once per
+//                 tile and keep partial row sums until the end
+//   warp 16       TMA producer: Q (both sub-tiles) once, then K and V tiles into a 2-stage
+//                 ring (128B swizzle); the sub-tiles share every K/V tile
+//   warp 17       TMEM owner and MMA issuer (tcgen05.mma kind::f16): S_q = Q_q K_j^T into TMEM,
+//                 O_q += P_q V_j with P_q read from TMEM (written there by the softmax over the
+//                 first 64 columns of S_q) and V_j an MN-major shared-memory operand; order
+//                 S_0(j) S_1(j) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...; same-thread tcgen05.mma
+//                 execute in issue order, so the next S follows the PV that reads P directly
+// The running max lives per row (O rescaled in TMEM only when it grows by more than 2^8), P is
+// bf16 in TMEM, and the final normalisation combines the two partial row sums.
 // A key tile that no row of a sub-tile may see is skipped for that sub-tile (no MMA, no
 // softmax). Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in
 // the device error word, every role stops, and the TMEM allocation is released.
@@ -39,8 +41,9 @@ constexpr int QT = 2;                   // query sub-tiles per CTA
 constexpr int BN = 128;                 // keys per tile
 constexpr int D = 128;                  // head dim
 constexpr int NS = 2;                   // K/V ring stages
-constexpr int THREADS = 384;           // 3 warpgroups: softmax 0, softmax 1, {TMA, MMA, 2 idle}
-constexpr int WARP_TMA = 8, WARP_MMA = 9;
+constexpr int THREADS = 576;           // 16 softmax warps, TMA warp, MMA warp
+constexpr int WARP_TMA = 16, WARP_MMA = 17;
+constexpr int SOFTMAX_THREADS = 256;   // per sub-tile: 128 rows x 2 column halves
 constexpr uint32_t HALF = 16384;        // one [128 rows][64 cols] bf16 half tile
 constexpr uint32_t TILE = 2 * HALF;     // [128][128] bf16
 constexpr uint32_t TMEM_COLS = 512;     // S_0 @0, S_1 @128, O_0 @256, O_1 @384
@@ -66,7 +69,9 @@ enum {
 };
 constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
 constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
-constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
+// row-max exchange between the two column halves: [sub-tile][tile parity][half][row] floats
+constexpr uint32_t SM_XCH = (SM_ABORT + 4 + 15) & ~15u;
+constexpr uint32_t SM_TOTAL = SM_XCH + QT * 2 * 2 * BM * 4;
 constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;          // slack for the 1024-byte alignment
 
 struct TcParams {
@@ -214,22 +219,6 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// 2^x on the FMA pipe, for a share of the softmax exponentials (the MUFU unit computes the
-// rest). Range reduction x = n + f with n = round(x) by the 1.5*2^23 rounding trick (t's low
-// mantissa bits hold n, and bits(t) << 23 = n << 23), f in [-1/2, 1/2]; 2^f by a cubic with
-// p(0) = 1 whose coefficients minimise the maximum relative error on [-1/2, 1/2] (fitted for
-// this kernel by linear programming; max relative error 1.0e-4, twenty times below the bf16
-// rounding P goes through); 2^n added to the exponent field. Valid for x in [-125, 126];
-// smaller x is clamped (the result, ~2^-125, is then negligible next to the row maximum's 1).
-__device__ __forceinline__ float exp2_fma(float x)
-{
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float pf = fmaf(fmaf(fmaf(0.055008937f, f, 0.24221095f), f, 0.6932829f), f, 1.f);
-    return __int_as_float(__float_as_int(pf) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -318,7 +307,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
         for (int q = 0; q < QT; ++q) {
             mbar_init(BAR(B_SFULL + q), 1);
-            mbar_init(BAR(B_PFULL + q), 128);
+            mbar_init(BAR(B_PFULL + q), SOFTMAX_THREADS);
             mbar_init(BAR(B_PVDONE + q), 1);
         }
         *abort_flag = 0;
@@ -438,61 +427,82 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 ++j;
             }
         }
-    } else if (warp < 8) {
+    } else if (warp < 16) {
         // ------------------------------- softmax ----------------------------------------
-        const int q = warp >> 2;                        // sub-tile of this warpgroup
+        const int q = warp >> 3;                        // sub-tile of this warp
+        const int hf = (warp >> 2) & 1;                 // 64-key half of every S tile
         const int quad = warp & 3;                      // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
         const long lrow = l0 + q * BM + row;
         const bool row_valid = lrow < p.q_rows;
         const int fq = p.fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-        float m = -INFINITY, lsum = 0.f;
+        float *xch = (float *)(smem + SM_XCH) + q * (2 * 2 * BM);   // [parity][half][row]
+        auto pair_sync = [&]() {                        // the 256 threads of this sub-tile
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(SOFTMAX_THREADS) : "memory");
+        };
+        // a barrier over the sub-tile's 256 threads that is true only if `v` is true for all:
+        // a bounded wait that expired makes every thread of the sub-tile leave the loop at
+        // the same tile, so the pairing barriers below stay matched
+        auto pair_all = [&](bool v) -> bool {
+            uint32_t r;
+            asm volatile(
+                "{\n\t.reg .pred pi, po;\n\t"
+                "setp.ne.u32 pi, %1, 0;\n\t"
+                "bar.red.and.pred po, %2, %3, pi;\n\t"
+                "selp.u32 %0, 1, 0, po;\n\t}"
+                : "=r"(r)
+                : "r"((uint32_t)v), "r"(1 + q), "r"(SOFTMAX_THREADS)
+                : "memory");
+            return r != 0;
+        };
+        float m = -INFINITY, lsum = 0.f;                // lsum: this half's partial row sum
         bool ok = true;
         int fk = fstart - 1, jt = wk.tpf - 1, k = 0;
         while (wk.next(fk, jt)) {
-            if (!active(q, fk)) continue;               // warp-uniform
-            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+            if (!active(q, fk)) continue;               // uniform over the sub-tile
+            if (!pair_all(mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
             const int nv = min(BN, p.N - jt * BN);
+            const int nvh = min(64, max(0, nv - hf * 64));            // valid keys of this half
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
-            const bool full = rok && nv == BN;
-            // pass 1: row max over the tile (two 64-column loads, four independent chains)
+            const bool full = rok && nvh == 64;
+            // this half of the S row in one TMEM round trip
+            uint32_t sr[64];
+            tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (full) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sr[64];
-                tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
-                if (full) {
+                for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+            } else if (rok) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
-                } else if (rok) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        mx[i & 3] = fmaxf(mx[i & 3], hf * 64 + i < nv ? __uint_as_float(sr[i]) : -INFINITY);
-                }
+                for (int i = 0; i < 64; ++i)
+                    mx[i & 3] = fmaxf(mx[i & 3], i < nvh ? __uint_as_float(sr[i]) : -INFINITY);
             }
-            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            // agree on the row max with the other half (double-buffered by tile parity: a
+            // slot is rewritten two tiles later, after the partner passed the next barrier)
+            float *slot = xch + (k & 1) * (2 * BM);
+            slot[hf * BM + row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            pair_sync();                                // both halves also finished reading S
+            const float mt = fmaxf(slot[row], slot[BM + row]);
             const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
             // grow the reference max only when it rose by more than 2^8 (lazy rescale)
             const bool need = rok && mnew > m + 8.f;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // pass 2: exponentials of 32 keys at a time; their bf16 pairs (key 2i in the low
-            // half) go to P columns 16c..16c+15, which overlay S columns already read
+            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) go to P
+            // columns 32*hf + 16c .. +15 of S_q (S columns both halves have read). `full` and
+            // `rok` differ between lanes whose rows straddle a frame boundary, so only the
+            // arithmetic branches on them; every tcgen05.ld / st stays warp-uniform.
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32], pk[16];
-                tmem_ld32(tlane + TM_S(q) + c * 32, sr);
+            for (int c = 0; c < 2; ++c) {
+                uint32_t pk[16];
                 if (full) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        // one exponential in four on the FMA pipe, three on the MUFU unit
-                        const float x0 = fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse);
-                        const float x1 = fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse);
-                        const float p0 = ex2(x0);
-                        const float p1 = (i & 1) ? exp2_fma(x1) : ex2(x1);
+                        const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), p.sl2, -muse));
+                        const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), p.sl2, -muse));
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
                     }
@@ -502,27 +512,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         const int col = c * 32 + 2 * i;
                         float p0 = 0.f, p1 = 0.f;
                         if (rok) {
-                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[2 * i]), p.sl2, -muse)) : 0.f;
-                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[2 * i + 1]), p.sl2, -muse)) : 0.f;
+                            p0 = col < nvh ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
+                            p1 = col + 1 < nvh ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
                         }
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
                     }
                 }
-                tmem_st16(tlane + TM_S(q) + c * 16, pk);
+                __syncwarp();                           // reconverge before .sync.aligned
+                tmem_st16(tlane + TM_S(q) + hf * 32 + c * 16, pk);
             }
-            // S_FULL completes only when every MMA issued before it has, so the previous PV of
-            // this sub-tile is done (O is free, P_q may be overwritten);
-            // its rescale is warp-collective TMEM traffic and the whole warp takes it together
+            // S_FULL completes only when every MMA issued before it has, so the previous PV
+            // of this sub-tile is done: this half's columns of O may be rescaled (warp-wide
+            // TMEM traffic, so the warp takes the branch together)
             if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     uint32_t orow[32];
-                    tmem_ld32(tlane + TM_O(q) + c * 32, orow);
+                    tmem_ld32(tlane + TM_O(q) + hf * 64 + c * 32, orow);
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-                    tmem_st32(tlane + TM_O(q) + c * 32, orow);
+                    tmem_st32(tlane + TM_O(q) + hf * 64 + c * 32, orow);
                 }
             }
             lsum = lsum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
@@ -532,14 +543,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             mbar_arrive(BAR(B_PFULL + q));
             ++k;
         }
-        if (ok && k >= 1 && __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) {
+        // final: both halves combine their partial sums and normalise their 64 columns of O
+        const bool fin = ok && k >= 1 &&
+                         __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT));
+        float *sums = xch + (k & 1) * (2 * BM);         // a slot no one reads any more
+        sums[hf * BM + row] = lsum;
+        pair_sync();
+        if (fin) {
             fence_after_sync();
-            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
+            const float tot = sums[row] + sums[BM + row];
+            const float inv = tot > 0.f ? 1.f / tot : 0.f;
+            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D + hf * 64;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(tlane + TM_O(q) + c * 32, ov);
+                __syncwarp();
+                tmem_ld32(tlane + TM_O(q) + hf * 64 + c * 32, ov);
                 if (row_valid) {
                     uint32_t pk2[16];
 #pragma unroll

@@ -3,7 +3,8 @@
 // Chunk algebra (derived from S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T; the
 // chunkwise split is the "parallel within a block, recurrent across blocks" form of the
 // llm-atlas long-context explainer, sections 06 and 09). For a chunk of n <= 64 tokens with
-// incoming state S0 and g_t = sum_{s<=t} log a_s within the chunk:
+// incoming state S0 and g_t = sum_{s<=t} log a_s within the chunk (the kernels carry g in
+// log2 units, so e^{g_t - g_i} is a single 2^x):
 //   A_ti = b_t e^{g_t-g_i} k_t.k_i (i < t),    T = (I + A)^{-1}          (UT transform)
 //   W  = T diag(b e^g) K,  Up = T diag(b) V,   P_ti = e^{g_t-g_i} q_t.k_i (i <= t)
 //   Op = P Up,  Qt = diag(e^g) Q - P W,  Kt = diag(e^{g_n-g}) K,  gam = e^{g_n}
@@ -15,12 +16,13 @@
 //          by TMA as 128B-swizzled boxes; KK^T, QK^T, the blocked inversion for T (fp32),
 //          then W, Up, Op, Qt on mma.sync bf16 tensor cores; writes W, Up, Op, Qt, Kt (bf16)
 //          and gam (fp32) to the workspace.
-//   state  serial over the chunks of a head; the 128 state rows are split over 8 CTAs of
-//          16 rows (rows of S evolve independently). The state slice lives in registers as
-//          the accumulator fragments of the S update; each chunk does two dependent small
-//          GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync. The chunk operands stream in by TMA
-//          (swizzled W/Qt/Kt boxes, this CTA's 16 columns of Up/Op, gam) through a 3-stage
-//          mbarrier ring, two chunks ahead; waits are bounded (DEVERR_GDN_WAIT).
+//   state  serial over the chunks of a head; the 128 state rows are split into 16-row blocks
+//          (rows of S evolve independently), four blocks per CTA, two CTAs per head. A
+//          block's state lives in registers as the accumulator fragments of the S update;
+//          each chunk does two dependent small GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync.
+//          The chunk operands (swizzled W/Qt/Kt boxes, the CTA's 64 columns of Up/Op, gam)
+//          stream in by TMA through a 3-stage mbarrier ring shared by the four blocks, two
+//          chunks ahead; waits are bounded (DEVERR_GDN_WAIT).
 // The serial chain is latency-bound (two dependent 64x16x128-class products per chunk), so
 // it uses register-resident warp MMAs rather than a TMEM round trip per dependent step.
 #include "hlta_internal.cuh"
@@ -38,7 +40,6 @@ constexpr int SC = C + 8;         // padded smem row stride of [.][64] bf16 tile
 constexpr int FP = C + 1;         // fp32 [64][65] tiles
 constexpr int THREADS = 128;
 constexpr int RB = 16;            // state rows per CTA in the state pass
-constexpr int SR = RB + 8;        // padded stride of [64][16] slices
 
 using ptx::smem_u32;
 using ptx::sw128_off;
@@ -103,6 +104,19 @@ __device__ __forceinline__ void frag_b_nk_sw(uint32_t (&r)[4], const uint8_t *ti
 __device__ __forceinline__ void frag_b_kn_sw(uint32_t (&r)[4], const uint8_t *tile, int k0, int n0, int lane)
 {
     ldsm_x4_t(r, smem_u32(tile + sw128_off(k0 + ((lane >> 3) & 1) * 8 + (lane & 7), n0 + (lane >> 4) * 8, C)));
+}
+
+__device__ __forceinline__ float fast_lg2(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
@@ -218,10 +232,11 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
         }
     }
     if (warp == 1) {
-        // inclusive prefix sum of log a over 64 entries: two per lane, then a warp scan
+        // inclusive prefix sum of log2 a over 64 entries (decays are then 2^(g_t - g_i), one
+        // ex2 each): two per lane, then a warp scan
         const int t = 2 * lane;
-        const float l0 = t < n ? logf(p.a[(long)bh * p.L + t0 + t]) : 0.f;
-        const float l1 = t + 1 < n ? logf(p.a[(long)bh * p.L + t0 + t + 1]) : 0.f;
+        const float l0 = t < n ? fast_lg2(p.a[(long)bh * p.L + t0 + t]) : 0.f;
+        const float l1 = t + 1 < n ? fast_lg2(p.a[(long)bh * p.L + t0 + t + 1]) : 0.f;
         float pair = l0 + l1, x = pair;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -236,8 +251,8 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
     __syncthreads();                                       // barrier initialised, g, bb ready
     if (tid < C) {
         const float gn = s.g[n - 1];
-        s.eg[tid] = tid < n ? expf(s.g[tid]) : 0.f;
-        s.ek[tid] = tid < n ? expf(gn - s.g[tid]) : 0.f;
+        s.eg[tid] = tid < n ? fast_ex2(s.g[tid]) : 0.f;
+        s.ek[tid] = tid < n ? fast_ex2(gn - s.g[tid]) : 0.f;
     }
     for (int e = tid; e < C * TP; e += PREP_THREADS) T[e] = 0.f;
     const bool landed = ptx::mbar_wait(bar, 0, (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
@@ -295,7 +310,7 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
                 const int t = m0 + g8 + (e >> 1) * 8;
                 const int i = n0 + nt * 8 + 2 * tg + (e & 1);
                 const bool lower = i <= t && t < n;
-                const float dec = lower ? expf(s.g[t] - s.g[i]) : 0.f;
+                const float dec = lower ? fast_ex2(s.g[t] - s.g[i]) : 0.f;
                 A[t * FP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
                 s.P[t * SC + i] = __float2bfloat16_rn(lower ? dec * qk[nt][e] : 0.f);
             }
@@ -398,40 +413,47 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
         }
         oK[e] = kv;
     }
-    if (tid < 4) ws.gam[((long)bh * nch + chunk) * 4 + tid] = tid == 0 ? expf(s.g[n - 1]) : 0.f;
+    if (tid < 4) ws.gam[((long)bh * nch + chunk) * 4 + tid] = tid == 0 ? fast_ex2(s.g[n - 1]) : 0.f;
 }
 
 // -----------------------------------------------------------------------------------------
 // state pass
 // -----------------------------------------------------------------------------------------
+// Two CTAs per head; each CTA holds four 16-row blocks of the state (one group of four warps
+// per block) that share one ring of chunk operands, so a head occupies two SMs.
 constexpr int NSTAGE = 3;                  // chunk operand buffers of the state pass
-constexpr uint32_t SLICE = C * RB * 2;     // this CTA's 16 columns of Up or Op: 2 KB
+constexpr int GROUPS = 4;                  // 16-row blocks per CTA
+constexpr int STATE_THREADS = GROUPS * THREADS;
+constexpr int CW = GROUPS * RB;            // state rows (= Up/Op columns) per CTA: 64
+constexpr uint32_t SLICE = C * CW * 2;     // the CTA's 64 columns of Up or Op: 8 KB
 constexpr uint32_t STAGE_TX = 3 * SWT + 2 * SLICE + 16;
 
 struct StateBuf {
     alignas(1024) uint8_t W[SWT];
     alignas(1024) uint8_t Q[SWT];          // Qt
     alignas(1024) uint8_t K[SWT];          // Kt
-    alignas(128) __nv_bfloat16 U[C * RB];  // Up[:, i0:i0+16], row-major [64][16]
-    alignas(128) __nv_bfloat16 O[C * RB];  // Op[:, i0:i0+16]
+    alignas(128) __nv_bfloat16 U[C * CW];  // Up[:, c0:c0+64], row-major [64][64]
+    alignas(128) __nv_bfloat16 O[C * CW];  // Op[:, c0:c0+64]
     alignas(16) float gam[4];              // gam of the chunk (element 0)
+};
+struct StateGroup {
+    __nv_bfloat16 Sb[RB * SD];             // state slice as bf16 [i][j]
+    __nv_bfloat16 Ut[RB * SC];             // U^T slice [i][t]
 };
 struct StateSmem {
     StateBuf buf[NSTAGE];
-    __nv_bfloat16 Sb[RB * SD];             // state slice as bf16 [i][j]
-    __nv_bfloat16 Ut[RB * SC];             // U^T slice [i][t]
-    __nv_bfloat16 Os[C * SR];              // output staging [t][i]
+    StateGroup grp[GROUPS];
     alignas(8) uint64_t full[NSTAGE];
     int abort_flag;
 };
 
 struct StateMaps {
     CUtensorMap W, Q, K;                   // workspace [BHg*nch*64][128]: 64x64 swizzled boxes
-    CUtensorMap U, O;                      // workspace [BHg*nch*64][128]: 64 rows x 16 columns
+    CUtensorMap U, O;                      // workspace [BHg*nch*64][128]: 64 rows x 64 columns
 };
 
 __device__ __forceinline__ void issue_chunk(StateSmem &s, const StateMaps &maps, const GdnWorkspace &ws,
-                                            int bh, long nch, long c, int i0)
+                                            int bh, long nch, long c, int c0)
 {
     StateBuf &bf = s.buf[c % NSTAGE];
     const uint32_t bar = smem_u32(&s.full[c % NSTAGE]);
@@ -442,21 +464,30 @@ __device__ __forceinline__ void issue_chunk(StateSmem &s, const StateMaps &maps,
         ptx::tma_load_2d(smem_u32(bf.Q + hf * (SWT / 2)), &maps.Q, hf * 64, row, bar);
         ptx::tma_load_2d(smem_u32(bf.K + hf * (SWT / 2)), &maps.K, hf * 64, row, bar);
     }
-    ptx::tma_load_2d(smem_u32(bf.U), &maps.U, i0, row, bar);
-    ptx::tma_load_2d(smem_u32(bf.O), &maps.O, i0, row, bar);
+    ptx::tma_load_2d(smem_u32(bf.U), &maps.U, c0, row, bar);
+    ptx::tma_load_2d(smem_u32(bf.O), &maps.O, c0, row, bar);
     ptx::bulk_load(smem_u32(bf.gam), ws.gam + ((long)bh * nch + c) * 4, 16, bar);
 }
 
-__global__ void __launch_bounds__(THREADS)
+__device__ __forceinline__ void group_sync(int g)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(THREADS) : "memory");
+}
+
+__global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace ws)
 {
     extern __shared__ uint8_t smem_raw[];
     StateSmem &s = *reinterpret_cast<StateSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int i0 = blockIdx.x * RB, bh = blockIdx.y;
+    const int bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long nch = gdn_num_chunks(p.L, C);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int g = tid / THREADS, warp = (tid / 32) % 4;    // row-block group, warp in group
     const int g8 = lane >> 2, tg = lane & 3;
+    const int c0 = blockIdx.x * CW;                        // first state row of this CTA
+    const int i0 = c0 + g * RB;                            // first state row of this group
+    StateGroup &sg = s.grp[g];
     __nv_bfloat16 *o = (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D;
 
     if (tid == 0) {
@@ -475,11 +506,11 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
                 const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
                 const int i = nt * 8 + 2 * tg + (e & 1);
                 st[mt][nt][e] = p.S0 ? p.S0[((long)bh * D + i0 + i) * D + j] : 0.f;
-                s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
+                sg.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
             }
     __syncthreads();
     if (tid == 0)
-        for (long c = 0; c < NSTAGE - 1 && c < nch; ++c) issue_chunk(s, maps, ws, bh, nch, c, i0);
+        for (long c = 0; c < NSTAGE - 1 && c < nch; ++c) issue_chunk(s, maps, ws, bh, nch, c, c0);
 
     bool ok = true;
     long c_fail = 0;
@@ -487,13 +518,14 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
         StateBuf &cur = s.buf[c % NSTAGE];
         const bool landed = ptx::mbar_wait(smem_u32(&s.full[c % NSTAGE]), (uint32_t)(c / NSTAGE) & 1u,
                                            (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
-        // chunk c has landed for every thread, and Sb holds the incoming state
+        // chunk c has landed for every thread; every group's Sb holds its incoming state
         if (!__syncthreads_and(landed)) { ok = false; c_fail = c; break; }
         // the stage of chunk c-1 is free again (every thread passed the barrier above)
-        if (tid == 0 && c + NSTAGE - 1 < nch) issue_chunk(s, maps, ws, bh, nch, c + NSTAGE - 1, i0);
+        if (tid == 0 && c + NSTAGE - 1 < nch) issue_chunk(s, maps, ws, bh, nch, c + NSTAGE - 1, c0);
         const float gam = cur.gam[0];
+        const long t0 = c * C;
 
-        // GEMM 1: rows [W; Qt] (warps 0-1: W rows, warps 2-3: Qt rows) times S^T
+        // GEMM 1: rows [W; Qt] (warps 0-1 of the group: W rows, warps 2-3: Qt rows) times S^T
         {
             const uint8_t *Am = warp < 2 ? cur.W : cur.Q;
             const int mb = (warp & 1) * 32;
@@ -507,7 +539,7 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
                 uint32_t bsf[4];
-                frag_b_nk(bsf, s.Sb, SD, 0, ks * 16, lane);
+                frag_b_nk(bsf, sg.Sb, SD, 0, ks * 16, lane);
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                     uint32_t a[4];
@@ -521,28 +553,24 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int t = mb + mt * 16 + g8 + (e >> 1) * 8;
-                        const int i = nt * 8 + 2 * tg + (e & 1);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int t = mb + mt * 16 + g8 + hh * 8;
+                        const int i = nt * 8 + 2 * tg;
+                        const float a0 = acc[mt][nt][2 * hh], a1 = acc[mt][nt][2 * hh + 1];
                         if (warp < 2) {
-                            const float u = __bfloat162float(cur.U[t * RB + i]) - acc[mt][nt][e];
-                            s.Ut[i * SC + t] = __float2bfloat16_rn(u);
-                        } else {
-                            const float ov = __bfloat162float(cur.O[t * RB + i]) + acc[mt][nt][e];
-                            s.Os[t * SR + i] = __float2bfloat16_rn(ov);
+                            const float u0 = __bfloat162float(cur.U[t * CW + g * RB + i]) - a0;
+                            const float u1 = __bfloat162float(cur.U[t * CW + g * RB + i + 1]) - a1;
+                            sg.Ut[i * SC + t] = __float2bfloat16_rn(u0);
+                            sg.Ut[(i + 1) * SC + t] = __float2bfloat16_rn(u1);
+                        } else if (t0 + t < p.L) {
+                            const float v0 = __bfloat162float(cur.O[t * CW + g * RB + i]) + a0;
+                            const float v1 = __bfloat162float(cur.O[t * CW + g * RB + i + 1]) + a1;
+                            *reinterpret_cast<uint32_t *>(o + (t0 + t) * D + i0 + i) = pack2(v0, v1);
                         }
                     }
         }
-        __syncthreads();                       // Ut and Os complete
+        group_sync(g);                         // this group's Ut is complete
 
-        // outputs of this chunk: 64 rows x 16 columns
-        {
-            const long t0 = c * C;
-            const int t = tid >> 1, hlf = tid & 1;
-            if (t0 + t < p.L)
-                *reinterpret_cast<uint4 *>(o + (t0 + t) * D + i0 + hlf * 8) =
-                    *reinterpret_cast<const uint4 *>(&s.Os[t * SR + hlf * 8]);
-        }
         // GEMM 2: S^T <- gam S^T + Kt^T U   (D[m=j][n=i] = sum_t Kt[t][j] U[t][i])
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
@@ -553,7 +581,7 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks) {
             uint32_t bu[4];
-            frag_b_nk(bu, s.Ut, SC, 0, ks * 16, lane);
+            frag_b_nk(bu, sg.Ut, SC, 0, ks * 16, lane);
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 uint32_t a[4];
@@ -572,17 +600,17 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
                 for (int e = 0; e < 4; ++e) {
                     const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
                     const int i = nt * 8 + 2 * tg + (e & 1);
-                    s.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
+                    sg.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
                 }
     }
     if (!ok) {
         // a bounded wait expired: let the copies this CTA issued and never consumed land
         // before it exits (chunks c .. issued-1, each on its own stage and phase)
         if (tid == 0) {
-            const long long t0 = clock64();
+            const long long tw = clock64();
             for (long cc = c_fail; cc < c_fail + NSTAGE - 1 && cc < nch; ++cc) {
                 const uint32_t bar = smem_u32(&s.full[cc % NSTAGE]);
-                while (!ptx::mbar_try(bar, (uint32_t)(cc / NSTAGE) & 1u) && clock64() - t0 < (1LL << 31)) {}
+                while (!ptx::mbar_try(bar, (uint32_t)(cc / NSTAGE) & 1u) && clock64() - tw < (1LL << 31)) {}
             }
         }
         return;
@@ -622,8 +650,8 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     if ((e = make_tmap_2d_bf16(&sm.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&sm.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&sm.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows, D, RB, C, false)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows, D, RB, C, false)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows, D, CW, C, false)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows, D, CW, C, false)) != cudaSuccess) return e;
     const size_t smem_prep = sizeof(PrepSmem) + 1024;
     const size_t smem_state = sizeof(StateSmem) + 1024;
     e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep);
@@ -632,7 +660,7 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     if (e != cudaSuccess) return e;
     gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / RB, (unsigned)BH), THREADS, smem_state, s>>>(sm, g, ws);
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
     return cudaGetLastError();
 }
 

@@ -65,8 +65,15 @@ hlta_status device_ctx(DeviceCtx **out)
     if (!c.ready) {
         if ((e = cudaGetSymbolAddress((void **)&c.err, g_device_error)) != cudaSuccess)
             return cuda_fail(e, "cudaGetSymbolAddress(error word)");
-        if ((e = cudaStreamCreateWithFlags(&c.aux, cudaStreamNonBlocking)) != cudaSuccess)
-            return cuda_fail(e, "cudaStreamCreate");
+        // The GDN branch (a short parallel prep, then a long serial chain on a few SMs) runs
+        // on this stream at the highest priority: its CTAs are dispatched ahead of the
+        // softmax branches' whenever SMs free up, so the serial chain starts right after its
+        // prep and the softmax kernels fill the remaining SMs around it.
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetStreamPriorityRange");
+        if ((e = cudaStreamCreateWithPriority(&c.aux, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithPriority");
         if ((e = cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming)) != cudaSuccess)
             return cuda_fail(e, "cudaEventCreate");
         if ((e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming)) != cudaSuccess)
@@ -312,23 +319,27 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const f
         prof_record(3, ctx->aux);
         st = run_gdn(g, dt, ctx->aux);
         prof_record(4, ctx->aux);
-        // join even on failure so `s` never runs ahead of work that was enqueued
         cudaEventRecord(ctx->join, ctx->aux);
-        cudaStreamWaitEvent(s, ctx->join, 0);
-        if (st != HLTA_OK) return st;
+        if (st != HLTA_OK) {
+            cudaStreamWaitEvent(s, ctx->join, 0);   // `s` never runs ahead of enqueued work
+            return st;
+        }
     }
+    // the softmax branches run on `s` while the GDN branch runs on the auxiliary stream
     prof_record(0, s);
     if (Hs) {
         AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
-        if ((st = run_attn(a1, dt, s)) != HLTA_OK) return st;
+        st = run_attn(a1, dt, s);
     }
     prof_record(1, s);
-    if (Hd) {
+    if (Hd && st == HLTA_OK) {
         AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
-        if ((st = run_attn(a2, dt, s)) != HLTA_OK) return st;
+        st = run_attn(a2, dt, s);
     }
     prof_record(2, s);
-    return HLTA_OK;
+    // join: work enqueued on `s` after this call sees the GDN outputs too
+    if (Hg) cudaStreamWaitEvent(s, ctx->join, 0);
+    return st;
 }
 
 hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N, int d,
@@ -399,8 +410,10 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
     const int H = c->Hs + c->Hd + c->Hg;
     const int f = c->frames;
     const size_t el = c->dt == HLTA_BF16 ? 2 : 4;
+    // the fork/join events are shared per device: hold them until the join is enqueued
+    std::unique_lock<std::mutex> lk(g_fork_mu, std::defer_lock);
     if (c->Hg) {
-        std::lock_guard<std::mutex> lk(g_fork_mu);
+        lk.lock();
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         GdnArgs g;
@@ -410,8 +423,10 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         g.err = ctx->err;
         st = run_gdn(g, c->dt, ctx->aux);
         cudaEventRecord(ctx->join, ctx->aux);
-        cudaStreamWaitEvent(s, ctx->join, 0);
-        if (st != HLTA_OK) return st;
+        if (st != HLTA_OK) {
+            cudaStreamWaitEvent(s, ctx->join, 0);
+            return st;
+        }
     }
     struct Branch { int h0, Hbr, slots, w, r; void *rk, *rv; } br[2] = {
         {0, c->Hs, c->slots_s, c->w_swa, 1, c->ks, c->vs},
@@ -419,10 +434,11 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
     for (const Branch &x : br) {
         if (!x.Hbr) continue;
         const int slot = f % x.slots;
-        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rk, x.slots, slot, s)) != cudaSuccess)
-            return cuda_fail(e, "ring append");
-        if ((e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rv, x.slots, slot, s)) != cudaSuccess)
-            return cuda_fail(e, "ring append");
+        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rk, x.slots, slot, s)) != cudaSuccess ||
+            (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rv, x.slots, slot, s)) != cudaSuccess) {
+            st = cuda_fail(e, "ring append");
+            break;
+        }
         AttnArgs a;
         a.q = q_new; a.k = x.rk; a.v = x.rv; a.o = o_new;
         a.B = c->B; a.Hbr = x.Hbr;
@@ -430,8 +446,11 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
         a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.scale = c->scale;
         a.err = ctx->err;
-        if ((st = run_attn(a, c->dt, s)) != HLTA_OK) return st;
+        if ((st = run_attn(a, c->dt, s)) != HLTA_OK) break;
     }
+    // join the GDN branch after the softmax branches were enqueued, so the two overlap
+    if (c->Hg) cudaStreamWaitEvent(s, ctx->join, 0);
+    if (st != HLTA_OK) return st;
     c->frames = f + 1;
     return HLTA_OK;
 }
