@@ -5,27 +5,33 @@
 // explainer, section 03 "Flash Attention": the score matrix never leaves the chip and the
 // result equals the full softmax). The key set of a query tile is the union of the key
 // frames of its rows' frames (sliding window: frames f-w+1..f; dilated: f, f-r, ...,
-// f-r(w-1); Kairos abstract, item (2)); each key frame is walked in 128-token tiles and a
+// f-r(w-1); Kairos abstract, item (2)); each key frame is walked in 64-token tiles and a
 // per-element mask (row frame vs. key frame, ragged frame end) removes what a row must not
 // see.
 //
-// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 18 warps:
-//   warps 0..7    softmax of sub-tile 0, warps 8..15 softmax of sub-tile 1: each query row is
-//                 shared by two threads (same TMEM lane, warps w and w+4), one per 64-key half
-//                 of every S tile; they agree on the row max through shared memory once per
-//                 tile and keep partial row sums until the end
-//   warp 16       TMA producer: Q (both sub-tiles) once, then K and V tiles into a 2-stage
-//                 ring (128B swizzle); the sub-tiles share every K/V tile
-//   warp 17       TMEM owner and MMA issuer (tcgen05.mma kind::f16): S_q = Q_q K_j^T into TMEM,
-//                 O_q += P_q V_j with P_q read from TMEM (written there by the softmax over the
-//                 first 64 columns of S_q) and V_j an MN-major shared-memory operand; order
-//                 S_0(j) S_1(j) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...; same-thread tcgen05.mma
-//                 execute in issue order, so the next S follows the PV that reads P directly
-// The running max lives per row (O rescaled in TMEM only when it grows by more than 2^8), P is
-// bf16 in TMEM, and the final normalisation combines the two partial row sums.
-// A key tile that no row of a sub-tile may see is skipped for that sub-tile (no MMA, no
-// softmax). Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT in
-// the device error word, every role stops, and the TMEM allocation is released.
+// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 11 warps:
+//   warps 0..3   softmax of sub-tile 0, warps 4..7 softmax of sub-tile 1, one thread per
+//                query row (the warp's TMEM lane quadrant)
+//   warp 8       TMA producer: Q (both sub-tiles) once, then 64-key K and V tiles into two
+//                4-stage rings (128B swizzle), K two tiles ahead of V; the sub-tiles share
+//                every K/V tile, and a stage is refilled once both sub-tiles released it
+//   warps 9, 10  MMA issuers (tcgen05.mma kind::f16) of sub-tile 0 and 1; warp 9 owns the
+//                TMEM allocation. One thread issues products at a limited rate (tens of
+//                cycles each), so each sub-tile has its own issuing thread.
+// Tensor memory: per sub-tile two S buffers of 64 columns and O (128 columns), 512 in all.
+// S being double-buffered is what keeps the tensor pipe and the softmax apart: the MMA warp
+// issues S_q for the sub-tile's next tile into the other buffer while the softmax works on the
+// current one, so the softmax of consecutive tiles runs back to back. Per tile and sub-tile:
+//   softmax: S_q[b] -> registers (one 64-column load), row max, P = 2^(s*scale*log2e - m) as
+//            bf16 pairs written over the first 32 columns of S_q[b], P_FULL
+//   MMA:     O_q += P_q[b] V_j (P read from tensor memory, V an MN-major smem operand),
+//            then S_q for the tile two ahead into the same buffer (tcgen05.mma operations of
+//            one thread execute in issue order, so the overwrite of P needs no wait)
+// The running max lives per row (O rescaled in TMEM only when it grows by more than 2^8,
+// after the previous P V of the sub-tile has completed). A key tile that no row of a
+// sub-tile may see is skipped for that sub-tile. Every mbarrier wait is bounded; on expiry
+// the kernel records DEVERR_ATTN_WAIT in the device error word, every role stops, and the
+// TMEM allocation is released.
 #include "hlta_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -38,40 +44,42 @@ using namespace ptx;
 
 constexpr int BM = 128;                 // query rows per sub-tile
 constexpr int QT = 2;                   // query sub-tiles per CTA
-constexpr int BN = 128;                 // keys per tile
+constexpr int BN = 64;                  // keys per tile
 constexpr int D = 128;                  // head dim
-constexpr int NS = 2;                   // K/V ring stages
-constexpr int THREADS = 576;           // 16 softmax warps, TMA warp, MMA warp
-constexpr int WARP_TMA = 16, WARP_MMA = 17;
-constexpr int SOFTMAX_THREADS = 256;   // per sub-tile: 128 rows x 2 column halves
-constexpr uint32_t HALF = 16384;        // one [128 rows][64 cols] bf16 half tile
-constexpr uint32_t TILE = 2 * HALF;     // [128][128] bf16
-constexpr uint32_t TMEM_COLS = 512;     // S_0 @0, S_1 @128, O_0 @256, O_1 @384
-__host__ __device__ constexpr uint32_t TM_S(int q) { return (uint32_t)q * 128u; }
+constexpr int NS = 4;                   // stages of each of the K and V rings
+constexpr int LOOKAHEAD = 2;            // S is issued up to two tiles ahead of P V
+constexpr int THREADS = 352;            // 8 softmax warps, TMA warp, two MMA warps
+constexpr int WARP_TMA = 8, WARP_MMA = 9;   // MMA warps 9 (sub-tile 0, owns TMEM) and 10 (sub-tile 1)
+constexpr int SOFTMAX_THREADS = 128;    // per sub-tile: one thread per query row
+constexpr uint32_t QHALF = BM * 128;    // [128 rows][64 cols] bf16: 16 KB
+constexpr uint32_t QTILE = 2 * QHALF;   // [128][128]
+constexpr uint32_t KHALF = BN * 128;    // [64 rows][64 cols] bf16: 8 KB
+constexpr uint32_t KTILE = 2 * KHALF;   // [64][128]
+constexpr uint32_t TMEM_COLS = 512;     // S_0[0] @0, S_0[1] @64, S_1[0] @128, S_1[1] @192, O_0 @256, O_1 @384
+__host__ __device__ constexpr uint32_t TM_S(int q, int b) { return (uint32_t)q * 128u + (uint32_t)b * 64u; }
 __host__ __device__ constexpr uint32_t TM_O(int q) { return 256u + (uint32_t)q * 128u; }
 
 // shared memory map (offsets from a 1024-byte aligned base)
-__host__ __device__ constexpr uint32_t SM_Q(int q) { return (uint32_t)q * TILE; }
-__host__ __device__ constexpr uint32_t SM_K(int st) { return QT * TILE + (uint32_t)st * 2 * TILE; }
-__host__ __device__ constexpr uint32_t SM_V(int st) { return SM_K(st) + TILE; }
-constexpr uint32_t SM_BAR = SM_K(NS);
+__host__ __device__ constexpr uint32_t SM_Q(int q) { return (uint32_t)q * QTILE; }
+__host__ __device__ constexpr uint32_t SM_K(int st) { return QT * QTILE + (uint32_t)st * KTILE; }
+__host__ __device__ constexpr uint32_t SM_V(int st) { return QT * QTILE + (uint32_t)(NS + st) * KTILE; }
+constexpr uint32_t SM_BAR = QT * QTILE + 2 * NS * KTILE;
 // barriers (8 bytes each)
 enum {
     B_QFULL = 0,
     B_KFULL = 1,                // + stage
-    B_VFULL = B_KFULL + NS,
-    B_KEMPTY = B_VFULL + NS,
-    B_VEMPTY = B_KEMPTY + NS,
-    B_SFULL = B_VEMPTY + NS,    // + sub-tile
-    B_PFULL = B_SFULL + QT,
-    B_PVDONE = B_PFULL + QT,
-    NBARS = B_PVDONE + QT
+    B_VFULL = B_KFULL + NS,     // + stage
+    B_EMPTY = B_VFULL + NS,     // + stage: K and V of the stage consumed by both MMA warps
+    B_SFULL = B_EMPTY + NS,     // + 2 * sub-tile + buffer
+    B_PFULL = B_SFULL + 2 * QT, // + 2 * sub-tile + buffer (per buffer: the softmax may finish
+                                //   the next tile before the MMA warp consumed this one)
+    B_PVDONE = B_PFULL + 2 * QT, // + sub-tile
+    B_ODONE = B_PVDONE + QT,    // + sub-tile: every product of the sub-tile has completed
+    NBARS = B_ODONE + QT
 };
 constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
 constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
-// row-max exchange between the two column halves: [sub-tile][tile parity][half][row] floats
-constexpr uint32_t SM_XCH = (SM_ABORT + 4 + 15) & ~15u;
-constexpr uint32_t SM_TOTAL = SM_XCH + QT * 2 * 2 * BM * 4;
+constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
 constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;          // slack for the 1024-byte alignment
 
 struct TcParams {
@@ -219,6 +227,33 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+
+// packed fp32 pairs (sm_100 f32x2 instructions): half the issue slots of two scalar ops
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "add.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -235,21 +270,59 @@ __device__ __forceinline__ bool frame_needed(int fk, int fa, int fb, int w, int 
     return i0 < w && fk + r * i0 <= fb;
 }
 
+// The key-tile walk of a CTA: every 64-key tile of every frame some row of the CTA needs,
+// frame by frame. A position carries the frame's sub-tile mask (bit q: sub-tile q needs the
+// frame), computed once per frame, so stepping through the tiles of a frame costs an
+// increment and a compare: the MMA warp's issue loop is serial code on one thread, and every
+// instruction it spends between products is time the tensor pipe may run dry.
 struct Walk {
-    int fa, fb, w, r, tpf;
-    __device__ __forceinline__ bool needed(int fk) const { return frame_needed(fk, fa, fb, w, r); }
-    // advance (fk, jt) to the next tile; false when done
-    __device__ __forceinline__ bool next(int &fk, int &jt) const
+    int fa0, fb0, fa1, fb1, fb, w, r, tpf;
+    bool valid1;
+    __device__ __forceinline__ int mask_of(int fk) const
     {
-        if (++jt < tpf) return true;
-        for (++fk; fk <= fb; ++fk)
-            if (needed(fk)) {
-                jt = 0;
-                return true;
-            }
-        return false;
+        return (frame_needed(fk, fa0, fb0, w, r) ? 1 : 0) |
+               (valid1 && frame_needed(fk, fa1, fb1, w, r) ? 2 : 0);
     }
 };
+struct Pos {
+    int fk, jt, mask, j;        // frame, tile in the frame, sub-tile mask, global tile index
+    bool valid;
+};
+__device__ __forceinline__ Pos walk_start(const Walk &wk, int fstart)
+{
+    Pos c;
+    c.fk = fstart - 1;
+    c.jt = wk.tpf - 1;
+    c.mask = 0;
+    c.j = -1;
+    c.valid = true;
+    return c;
+}
+// the next tile of the walk (any sub-tile); false when done
+__device__ __forceinline__ bool walk_step(const Walk &wk, Pos &c)
+{
+    ++c.j;
+    if (++c.jt < wk.tpf) return true;
+    for (++c.fk; c.fk <= wk.fb; ++c.fk) {
+        const int m = wk.mask_of(c.fk);
+        if (m) {
+            c.mask = m;
+            c.jt = 0;
+            return true;
+        }
+    }
+    return c.valid = false;
+}
+// the next tile of the walk whose frame sub-tile `want` (a mask bit) needs; false when done
+__device__ __forceinline__ bool walk_next(const Walk &wk, Pos &c, int want)
+{
+    while (walk_step(wk, c)) {
+        if (c.mask & want) return true;
+        c.j += wk.tpf - 1 - c.jt;   // skip the rest of a frame this sub-tile does not need
+        c.jt = wk.tpf - 1;
+    }
+    return false;
+}
 
 __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
 {
@@ -275,26 +348,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     const long l0 = (long)blockIdx.x * (QT * BM);
     const long q_head = (long)(b * p.q_Htot + p.q_h0 + h) * p.q_rows;
     const long kv_head = (long)(b * p.kv_Htot + p.kv_h0 + h) * p.kv_rows;
-    // frame ranges of the two sub-tiles (sub-tile 1 may be empty in the last CTA of a head)
-    int sfa[QT], sfb[QT];
-    bool svalid[QT];
-#pragma unroll
-    for (int q = 0; q < QT; ++q) {
-        const long r0 = l0 + q * BM;
-        svalid[q] = r0 < p.q_rows;
-        const long r1 = min(r0 + BM, p.q_rows) - 1;
-        sfa[q] = p.fq0 + (int)(r0 / p.N);
-        sfb[q] = svalid[q] ? p.fq0 + (int)(r1 / p.N) : sfa[q];
-    }
+    // frame ranges of the two sub-tiles (sub-tile 1 may be empty in the last CTA of a head);
+    // scalars, not arrays indexed by the sub-tile, so nothing lands in local memory
+    const long r1_0 = min(l0 + BM, p.q_rows) - 1;
+    const int fa0 = p.fq0 + (int)(l0 / p.N), fb0 = p.fq0 + (int)(r1_0 / p.N);
+    const bool valid1 = l0 + BM < p.q_rows;
+    const int fa1 = valid1 ? p.fq0 + (int)((l0 + BM) / p.N) : fa0;
+    const int fb1 = valid1 ? p.fq0 + (int)((min(l0 + 2 * BM, p.q_rows) - 1) / p.N) : fa1;
     Walk wk;
-    wk.fa = sfa[0];
-    wk.fb = svalid[1] ? sfb[1] : sfb[0];
+    wk.fa0 = fa0;
+    wk.fb0 = fb0;
+    wk.fa1 = fa1;
+    wk.fb1 = fb1;
+    wk.valid1 = valid1;
+    wk.fb = valid1 ? fb1 : fb0;
     wk.w = p.w;
     wk.r = p.r;
     wk.tpf = (p.N + BN - 1) / BN;
-    const int fstart = max(0, wk.fa - p.r * (p.w - 1));
-    auto active = [&](int q, int fk) {
-        return svalid[q] && frame_needed(fk, sfa[q], sfb[q], p.w, p.r);
+    const int fstart = max(0, fa0 - p.r * (p.w - 1));
+    // row of the K/V tensor maps where tile (fk, jt) starts
+    auto kv_row = [&](int fk, int jt) {
+        return (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
     };
 
     if (threadIdx.x == 0) {
@@ -302,13 +376,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         for (int st = 0; st < NS; ++st) {
             mbar_init(BAR(B_KFULL + st), 1);
             mbar_init(BAR(B_VFULL + st), 1);
-            mbar_init(BAR(B_KEMPTY + st), 1);
-            mbar_init(BAR(B_VEMPTY + st), 1);
+            mbar_init(BAR(B_EMPTY + st), 2);
         }
         for (int q = 0; q < QT; ++q) {
-            mbar_init(BAR(B_SFULL + q), 1);
-            mbar_init(BAR(B_PFULL + q), SOFTMAX_THREADS);
+            mbar_init(BAR(B_SFULL + 2 * q), 1);
+            mbar_init(BAR(B_SFULL + 2 * q + 1), 1);
+            mbar_init(BAR(B_PFULL + 2 * q), SOFTMAX_THREADS);
+            mbar_init(BAR(B_PFULL + 2 * q + 1), SOFTMAX_THREADS);
             mbar_init(BAR(B_PVDONE + q), 1);
+            mbar_init(BAR(B_ODONE + q), 1);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -328,183 +404,202 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 
     if (warp == WARP_TMA) {
         // ------------------------------- TMA producer -----------------------------------
+        // step s loads K(s) and V(s - LOOKAHEAD): the MMA warp consumes K up to LOOKAHEAD
+        // tiles ahead of V
         if (lane == 0) {
-            mbar_expect_tx(BAR(B_QFULL), QT * TILE);
+            mbar_expect_tx(BAR(B_QFULL), QT * QTILE);
             for (int q = 0; q < QT; ++q) {
                 const int qrow = (int)(q_head + l0 + q * BM);
                 tma_load_2d(sbase + SM_Q(q), &tq, 0, qrow, BAR(B_QFULL));
-                tma_load_2d(sbase + SM_Q(q) + HALF, &tq, 64, qrow, BAR(B_QFULL));
+                tma_load_2d(sbase + SM_Q(q) + QHALF, &tq, 64, qrow, BAR(B_QFULL));
             }
-            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
-            while (wk.next(fk, jt)) {
-                const int st = j % NS;
-                const uint32_t ph = (uint32_t)((j / NS) + 1) & 1u;
-                const int krow = (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
-                if (j >= NS && !mbar_wait(BAR(B_KEMPTY + st), ph, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
-                mbar_expect_tx(BAR(B_KFULL + st), TILE);
-                tma_load_2d(sbase + SM_K(st), &tk, 0, krow, BAR(B_KFULL + st));
-                tma_load_2d(sbase + SM_K(st) + HALF, &tk, 64, krow, BAR(B_KFULL + st));
-                if (j >= NS && !mbar_wait(BAR(B_VEMPTY + st), ph, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
-                mbar_expect_tx(BAR(B_VFULL + st), TILE);
-                tma_load_2d(sbase + SM_V(st), &tv, 0, krow, BAR(B_VFULL + st));
-                tma_load_2d(sbase + SM_V(st) + HALF, &tv, 64, krow, BAR(B_VFULL + st));
-                ++j;
+            Pos kp = walk_start(wk, fstart), vp = kp;
+            int nk = 0, nv = 0;                     // K and V tiles issued
+            bool more_k = true, more_v = true, ok = true;
+            while (ok && (more_k || more_v)) {
+                if (more_k && (more_k = walk_step(wk, kp))) {
+                    const int st = nk % NS;
+                    if (nk >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((nk / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
+                    mbar_expect_tx(BAR(B_KFULL + st), KTILE);
+                    const int row = kv_row(kp.fk, kp.jt);
+                    tma_load_2d(sbase + SM_K(st), &tk, 0, row, BAR(B_KFULL + st));
+                    tma_load_2d(sbase + SM_K(st) + KHALF, &tk, 64, row, BAR(B_KFULL + st));
+                    ++nk;
+                }
+                if (nv < nk - LOOKAHEAD || (!more_k && nv < nk)) {
+                    more_v = walk_step(wk, vp);
+                    const int st = nv % NS;
+                    // the same release as K of this tile: complete already (the stage's next
+                    // release needs this V, so the phase cannot have moved on)
+                    if (nv >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((nv / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
+                    mbar_expect_tx(BAR(B_VFULL + st), KTILE);
+                    const int row = kv_row(vp.fk, vp.jt);
+                    tma_load_2d(sbase + SM_V(st), &tv, 0, row, BAR(B_VFULL + st));
+                    tma_load_2d(sbase + SM_V(st) + KHALF, &tv, 64, row, BAR(B_VFULL + st));
+                    ++nv;
+                } else if (!more_k) {
+                    more_v = false;
+                }
             }
             if (*abort_flag) {
                 // let this CTA's copies in flight land before the CTA may exit
                 const long long t0 = clock64();
-                for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj) {
-                    const int st = jj % NS;
-                    const uint32_t ph = (uint32_t)(jj / NS) & 1u;
-                    while (!mbar_try(BAR(B_KFULL + st), ph) && clock64() - t0 < (1LL << 31)) {}
-                    while (!mbar_try(BAR(B_VFULL + st), ph) && clock64() - t0 < (1LL << 31)) {}
-                }
+                for (int jj = nk - 1; jj >= 0 && jj >= nk - NS; --jj)
+                    while (!mbar_try(BAR(B_KFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
+                for (int jj = nv - 1; jj >= 0 && jj >= nv - NS; --jj)
+                    while (!mbar_try(BAR(B_VFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
                 while (!mbar_try(BAR(B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
             }
         }
-    } else if (warp == WARP_MMA) {
-        // ------------------------------- MMA issuer -------------------------------------
+    } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
+        // ------------------------------- MMA issuers ------------------------------------
+        // One warp per sub-tile: a single thread issues tcgen05.mma at a limited rate, so the
+        // two sub-tiles' products come from two threads. Each walks every tile of the CTA
+        // (the release of a K/V stage needs both) and works on its sub-tile's tiles.
         if (lane == 0) {
+            const int q = warp - WARP_MMA;
+            const int want = 1 << q;
             constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
             constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P (TMEM), V MN-major
-            int n_pv[QT] = {0, 0};
-            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, p.err, DEVERR_ATTN_WAIT);
-            // S_q = Q_q K^T. It overwrites the TMEM columns the previous PV of this sub-tile
-            // reads P_q from; tcgen05.mma operations issued by one thread execute in issue
-            // order, so it is issued right behind that PV without waiting for it.
-            auto issue_s = [&](int q, int st) -> bool {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-                    umma_bf16(tmem + TM_S(q), sw128_desc(sbase + SM_Q(q) + off, 16, 1024),
-                              sw128_desc(sbase + SM_K(st) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(BAR(B_SFULL + q));
-                return true;
+            // Shared-memory descriptors built once; each product only adds a compile-time
+            // offset (and the ring stage's) to the 14-bit start-address field.
+            const uint64_t dq = sw128_desc(sbase + SM_Q(q), 16, 1024);
+            const uint64_t dk0 = sw128_desc(sbase + SM_K(0), 16, 1024);
+            const uint64_t dv0 = sw128_desc(sbase + SM_V(0), KHALF, 1024);
+            const uint32_t s_tm = tmem + TM_S(q, 0), o_tm = tmem + TM_O(q);
+            // waits that find their phase complete cost one try_wait, no call
+            auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+                return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
             };
-            // O_q += P_q V, P_q from TMEM (bf16 pairs in the first 64 columns of S_q)
-            auto issue_pv = [&](int q, int st) -> bool {
-                if (!mbar_wait(BAR(B_PFULL + q), (uint32_t)n_pv[q] & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) return false;
-                fence_after_sync();
+            int ns = 0, npv = 0;                    // S and P V products issued
+            Pos c = walk_start(wk, fstart);         // the next tile whose S is not issued yet
+            walk_next(wk, c, want);
+            // S = Q K^T for cursor tiles up to global index jmax while an S buffer is free
+            // (at most two S ahead of P V; K of a tile more than LOOKAHEAD ahead of the walk
+            // may wait on a stage this warp has not released yet)
+            auto topup = [&](int jmax) -> bool {
+                while (c.valid && c.j <= jmax && ns - npv < 2) {
+                    const int st = c.j & (NS - 1);
+                    if (!wait_bar(BAR(B_KFULL + st), (uint32_t)(c.j / NS) & 1u)) return false;
+                    const int bf = ns & 1;
+                    const uint64_t dk = dk0 + (uint64_t)((st * KTILE) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_bf16_ts(tmem + TM_O(q), tmem + TM_S(q) + kk * 8,
-                                 sw128_desc(sbase + SM_V(st) + kk * 2048, HALF, 1024), IDESC_O,
-                                 (n_pv[q] > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(BAR(B_PVDONE + q));
-                ++n_pv[q];
-                return true;
-            };
-            int fk = fstart - 1, jt = wk.tpf - 1, j = 0;
-            bool have = ok && wk.next(fk, jt);
-            if (have) {
-                ok = mbar_wait(BAR(B_KFULL + 0), 0, abort_flag, p.err, DEVERR_ATTN_WAIT);
-                for (int q = 0; q < QT && ok; ++q)
-                    if (active(q, fk)) ok = issue_s(q, 0);
-                if (ok) umma_commit(BAR(B_KEMPTY + 0));
-            }
-            while (ok && have) {
-                const int st = j % NS, fk_cur = fk;
-                int fk_n = fk, jt_n = jt;
-                const bool have_n = wk.next(fk_n, jt_n);
-                const int stn = (j + 1) % NS;
-                if (!mbar_wait(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
-                bool k_ready = false;                   // K of the next tile, waited for once
-                for (int q = 0; q < QT && ok; ++q) {
-                    if (active(q, fk_cur)) ok = issue_pv(q, st);
-                    if (ok && have_n && active(q, fk_n)) {
-                        if (!k_ready)
-                            ok = k_ready = mbar_wait(BAR(B_KFULL + stn), (uint32_t)((j + 1) / NS) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT);
-                        if (ok) ok = issue_s(q, stn);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t qoff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                        const uint32_t koff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                        umma_bf16(s_tm + bf * 64, dq + qoff, dk + koff, IDESC_S, kk > 0 ? 1u : 0u);
                     }
+                    umma_commit(BAR(B_SFULL + 2 * q + bf));
+                    ++ns;
+                    walk_next(wk, c, want);
                 }
+                return true;
+            };
+            bool ok = wait_bar(BAR(B_QFULL), 0);
+            Pos t = walk_start(wk, fstart);
+            while (ok && walk_step(wk, t)) {
+                const int j = t.j, st = j & (NS - 1);
+                ok = topup(j + LOOKAHEAD) && wait_bar(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u);
                 if (!ok) break;
-                if (have_n) umma_commit(BAR(B_KEMPTY + stn));
-                umma_commit(BAR(B_VEMPTY + st));
-                fk = fk_n;
-                jt = jt_n;
-                have = have_n;
-                ++j;
+                if (t.mask & want) {
+                    // O += P V with P in the first 32 columns of the S buffer
+                    const int bf = npv & 1;
+                    if (!(ok = wait_bar(BAR(B_PFULL + 2 * q + bf), (uint32_t)(npv >> 1) & 1u))) break;
+                    fence_after_sync();
+                    const uint64_t dv = dv0 + (uint64_t)((st * KTILE) >> 4);
+                    const uint32_t acc0 = npv > 0 ? 1u : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        umma_bf16_ts(o_tm, s_tm + bf * 64 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                                     kk > 0 ? 1u : acc0);
+                    umma_commit(BAR(B_PVDONE + q));
+                    ++npv;
+                    // the buffer P V just read takes the S two tiles ahead (issue order)
+                    if (!(ok = topup(j + LOOKAHEAD))) break;
+                    // K_j (read by an S issued earlier) and V_j are consumed once these complete
+                    umma_commit(BAR(B_EMPTY + st));
+                } else {
+                    // a tile only the other sub-tile needs: V_j has landed, so this stage's
+                    // previous release is complete and the arrival belongs to this tile
+                    mbar_arrive(BAR(B_EMPTY + st));
+                }
             }
+            if (ok) umma_commit(BAR(B_ODONE + q));
         }
-    } else if (warp < 16) {
+    } else {
         // ------------------------------- softmax ----------------------------------------
-        const int q = warp >> 3;                        // sub-tile of this warp
-        const int hf = (warp >> 2) & 1;                 // 64-key half of every S tile
+        const int q = warp >> 2;                        // sub-tile of this warp
         const int quad = warp & 3;                      // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
         const long lrow = l0 + q * BM + row;
         const bool row_valid = lrow < p.q_rows;
         const int fq = p.fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-        float *xch = (float *)(smem + SM_XCH) + q * (2 * 2 * BM);   // [parity][half][row]
-        auto pair_sync = [&]() {                        // the 256 threads of this sub-tile
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(SOFTMAX_THREADS) : "memory");
-        };
-        // a barrier over the sub-tile's 256 threads that is true only if `v` is true for all:
-        // a bounded wait that expired makes every thread of the sub-tile leave the loop at
-        // the same tile, so the pairing barriers below stay matched
-        auto pair_all = [&](bool v) -> bool {
-            uint32_t r;
-            asm volatile(
-                "{\n\t.reg .pred pi, po;\n\t"
-                "setp.ne.u32 pi, %1, 0;\n\t"
-                "bar.red.and.pred po, %2, %3, pi;\n\t"
-                "selp.u32 %0, 1, 0, po;\n\t}"
-                : "=r"(r)
-                : "r"((uint32_t)v), "r"(1 + q), "r"(SOFTMAX_THREADS)
-                : "memory");
-            return r != 0;
-        };
-        float m = -INFINITY, lsum = 0.f;                // lsum: this half's partial row sum
+        float m = -INFINITY, lsum = 0.f;
         bool ok = true;
-        int fk = fstart - 1, jt = wk.tpf - 1, k = 0;
-        while (wk.next(fk, jt)) {
-            if (!active(q, fk)) continue;               // uniform over the sub-tile
-            if (!pair_all(mbar_wait(BAR(B_SFULL + q), (uint32_t)k & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+        int k = 0;
+        Pos c = walk_start(wk, fstart);
+        while (walk_next(wk, c, 1 << q)) {              // this sub-tile's tiles (uniform per warp)
+            const int fk = c.fk, jt = c.jt;
+            const int bf = k & 1;
+            const uint32_t sbar = BAR(B_SFULL + 2 * q + bf), spar = (uint32_t)(k >> 1) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
             const int nv = min(BN, p.N - jt * BN);
-            const int nvh = min(64, max(0, nv - hf * 64));            // valid keys of this half
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
-            const bool full = rok && nvh == 64;
-            // this half of the S row in one TMEM round trip
+            const bool full = rok && nv == BN;
             uint32_t sr[64];
-            tmem_ld64(tlane + TM_S(q) + hf * 64, sr);
+            tmem_ld64(tlane + TM_S(q, bf), sr);
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             if (full) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(sr[i]));
+                for (int i = 0; i < 32; ++i)
+                    mx[i & 3] = fmax3(mx[i & 3], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
             } else if (rok) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    mx[i & 3] = fmaxf(mx[i & 3], i < nvh ? __uint_as_float(sr[i]) : -INFINITY);
+                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
             }
-            // agree on the row max with the other half (double-buffered by tile parity: a
-            // slot is rewritten two tiles later, after the partner passed the next barrier)
-            float *slot = xch + (k & 1) * (2 * BM);
-            slot[hf * BM + row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            pair_sync();                                // both halves also finished reading S
-            const float mt = fmaxf(slot[row], slot[BM + row]);
+            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
             // grow the reference max only when it rose by more than 2^8 (lazy rescale)
             const bool need = rok && mnew > m + 8.f;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) go to P
-            // columns 32*hf + 16c .. +15 of S_q (S columns both halves have read). `full` and
-            // `rok` differ between lanes whose rows straddle a frame boundary, so only the
-            // arithmetic branches on them; every tcgen05.ld / st stays warp-uniform.
+            // rescale O (warp-wide TMEM traffic, so the warp takes the branch together) once
+            // the previous P V of this sub-tile, which accumulates into O, has completed. The
+            // one before it has: S of this tile was issued behind it and has completed, so
+            // the phase awaited here is the current or the next one, never older.
+            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+                fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t orow[32];
+                    tmem_ld32(tlane + TM_O(q) + c * 32, orow);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    tmem_st32(tlane + TM_O(q) + c * 32, orow);
+                }
+            }
+            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) go to the
+            // first 32 columns of the S buffer. `full` and `rok` differ between lanes whose
+            // rows straddle a frame boundary, so only the arithmetic branches on them; every
+            // tcgen05.ld / st stays warp-uniform.
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            const float2 sl2x2 = make_float2(p.sl2, p.sl2), nm2 = make_float2(-muse, -muse);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t pk[16];
                 if (full) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i]), p.sl2, -muse));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[c * 32 + 2 * i + 1]), p.sl2, -muse));
-                        ps[i & 3] += p0 + p1;
-                        pk[i] = pack_bf16(p0, p1);
+                        const float2 x = ffma2(make_float2(__uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1])), sl2x2, nm2);
+                        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                        ps2[i & 1] = fadd2(ps2[i & 1], pp);
+                        pk[i] = pack_bf16(pp.x, pp.y);
                     }
                 } else {
 #pragma unroll
@@ -512,53 +607,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         const int col = c * 32 + 2 * i;
                         float p0 = 0.f, p1 = 0.f;
                         if (rok) {
-                            p0 = col < nvh ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
-                            p1 = col + 1 < nvh ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
+                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
+                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
                         }
                         ps[i & 3] += p0 + p1;
                         pk[i] = pack_bf16(p0, p1);
                     }
                 }
                 __syncwarp();                           // reconverge before .sync.aligned
-                tmem_st16(tlane + TM_S(q) + hf * 32 + c * 16, pk);
+                tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
             }
-            // S_FULL completes only when every MMA issued before it has, so the previous PV
-            // of this sub-tile is done: this half's columns of O may be rescaled (warp-wide
-            // TMEM traffic, so the warp takes the branch together)
-            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t orow[32];
-                    tmem_ld32(tlane + TM_O(q) + hf * 64 + c * 32, orow);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-                    tmem_st32(tlane + TM_O(q) + hf * 64 + c * 32, orow);
-                }
-            }
-            lsum = lsum * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+            lsum = lsum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y)));
             m = muse;
             tmem_wait_st();
             fence_before_sync();
-            mbar_arrive(BAR(B_PFULL + q));
+            mbar_arrive(BAR(B_PFULL + 2 * q + bf));
             ++k;
         }
-        // final: both halves combine their partial sums and normalise their 64 columns of O
+        // final: once every product of the sub-tile has completed (a one-phase barrier its MMA
+        // warp commits after its last issue; the last two P V of this sub-tile may both still
+        // run, so a parity wait on P_V_DONE would be ambiguous), normalise O and store it
         const bool fin = ok && k >= 1 &&
-                         __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT));
-        float *sums = xch + (k & 1) * (2 * BM);         // a slot no one reads any more
-        sums[hf * BM + row] = lsum;
-        pair_sync();
+                         __all_sync(0xffffffffu, mbar_wait(BAR(B_ODONE + q), 0u, abort_flag, p.err, DEVERR_ATTN_WAIT));
         if (fin) {
             fence_after_sync();
-            const float tot = sums[row] + sums[BM + row];
-            const float inv = tot > 0.f ? 1.f / tot : 0.f;
-            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D + hf * 64;
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
                 __syncwarp();
-                tmem_ld32(tlane + TM_O(q) + hf * 64 + c * 32, ov);
+                tmem_ld32(tlane + TM_O(q) + c * 32, ov);
                 if (row_valid) {
                     uint32_t pk2[16];
 #pragma unroll
@@ -596,7 +675,7 @@ cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
     const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
     if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
-    // [rows][128] bf16 views, boxes of 128 rows x 64 columns, 128-byte swizzle
+    // [rows][128] bf16 views, boxes of 64 columns (128 rows for Q, 64 for K and V), 128-byte swizzle
     if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
