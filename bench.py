@@ -136,6 +136,35 @@ def measure_stream(h, torch, dev, warm: int = 24, steps: int = 40) -> dict:
             "softmax_tflops": flop / (ms / 1e3) / 1e12, "launches_per_step": 8}
 
 
+def measure_raw(h, torch, dev, wl, hi, steps: int) -> dict:
+    """The hybrid step with the GDN prologue fused (raw q, k and gate inputs x, y for the GDN
+    heads): same workload, timed like the main step (inputs resident, back to back)."""
+    raw = hi.make_raw_inputs(wl, seed=11)
+    q, k, v, x, y = (raw[n].to(dev) for n in ("q", "k", "v", "x", "y"))
+    o = torch.empty_like(q)
+    S = torch.empty((wl.B, wl.Hg, wl.d, wl.d), device=dev, dtype=torch.float32)
+    ws = torch.empty(h.hlta_hybrid_workspace_bytes(wl.B, wl.Hg, wl.T, wl.N, wl.d, wl.chunk),
+                     device=dev, dtype=torch.uint8)
+
+    def step():
+        h.hlta_hybrid_fwd_raw(q, k, v, x, y, wl.decay, o, None, S, wl.B, wl.Hs, wl.Hd, wl.Hg,
+                              wl.T, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r, wl.chunk, 0.0, ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms_per_step": ms, "tokens_per_s": wl.B * wl.L / (ms / 1e3),
+            "note": "hlta_hybrid_fwd_raw: the GDN heads' unit-norm q/k and gate activations "
+                    "computed inside the chunk preparation"}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -434,6 +463,7 @@ def main():
     attn_alone_ms = a0.elapsed_time(a1) / K
     del sub, o_s, o_d
     stream_detail = None if args.no_stream else measure_stream(h, torch, dev)
+    raw_detail = None if args.no_stream else measure_raw(h, torch, dev, wl, hi, K)
 
     # ---- roofline of the dominant kernel (windowed attention, both launches) --------------
     wk = work(wl)
@@ -466,6 +496,8 @@ def main():
     if stream_detail is not None:
         stream_detail["softmax_frac"] = stream_detail["softmax_tflops"] / peak
         detail["stream"] = stream_detail
+    if raw_detail is not None:
+        detail["raw_prologue"] = raw_detail
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,

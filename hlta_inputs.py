@@ -113,6 +113,33 @@ def make_inputs(wl: Workload, seed: int = 0, frames: int | None = None) -> dict:
             "a": a.contiguous(), "b": b.contiguous()}
 
 
+def make_raw_inputs(wl: Workload, seed: int = 0, frames: int | None = None) -> dict:
+    """Host tensors for the raw-input entry points (the GDN prologue done by the operator).
+
+    q, k, v: [B, H, L, d] as in ``make_inputs`` before any preprocessing, except that the
+    GDN heads' q and k carry a seeded per-token scale (log-normal, sigma 1) so their norms
+    vary; x, y: [B, Hg, L] float32 raw gate inputs (the same draws ``make_inputs`` turns into
+    a and b). bf16 workloads are rounded once after generation.
+    """
+    T = wl.T if frames is None else int(frames)
+    L = T * wl.N
+    shape = (wl.B, wl.H, L, wl.d)
+    q = _randn(shape, seed)
+    k = _randn(shape, seed + 1)
+    v = _randn(shape, seed + 2)
+    x = _randn((wl.B, wl.Hg, L), seed + 3)
+    y = _randn((wl.B, wl.Hg, L), seed + 4)
+    g0 = wl.Hs + wl.Hd
+    if wl.Hg:
+        sc = torch.exp(_randn((2, wl.B, wl.Hg, L, 1), seed + 5))
+        q[:, g0:] *= sc[0]
+        k[:, g0:] *= sc[1]
+    if wl.dtype == "bf16":
+        q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    return {"q": q.contiguous(), "k": k.contiguous(), "v": v.contiguous(),
+            "x": x.contiguous(), "y": y.contiguous()}
+
+
 def random_state(B: int, Hg: int, d: int, seed: int, scale: float = 1.0) -> torch.Tensor:
     """A seeded fp32 initial GDN state [B, Hg, d, d] (rows: value dim, cols: key dim)."""
     return (_randn((B, Hg, d, d), seed) * scale).contiguous()

@@ -114,6 +114,26 @@ hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v,
                                hlta_dtype dt, void *stream);
 
 /*
+ * hlta_gdn_chunk_fwd with the GDN heads' prologue fused into the chunk preparation, for
+ * callers holding raw projections. The delta rule contracts only for unit keys and gates in
+ * range (researchpapers.dev summary, Theorem 2: ||I - b k k^T|| <= 1 for ||k|| = 1, b in
+ * [0, 1]); here the library establishes that itself: q and k of every token are scaled to
+ * unit L2 norm (a zero vector stays zero), and the gates are
+ *   a = exp(-c * softplus(x)) in (0, 1],   b = sigmoid(y) in (0, 1),
+ * so the result equals hlta_gdn_chunk_fwd on (q/|q|, k/|k|, v, a, b) up to rounding.
+ * q, k: raw [B, H, L, d] (type `dt`); x, y: [B, H, L] float32 device; c: finite, >= 0 (the
+ * decay strength; c = 0 gives a = 1). The normalised q, k never reach device memory:
+ * the preparation normalises its staged copy and rounds it to `dt` once. Other arguments
+ * and errors as hlta_gdn_chunk_fwd; an invalid c is HLTA_ERR_INVALID_ARG.
+ */
+hlta_status hlta_gdn_chunk_fwd_raw(const void *q, const void *k, const void *v,
+                                   const float *x, const float *y, float c, void *o,
+                                   const float *S0, float *S_out,
+                                   int B, int H, long L, int d, int chunk,
+                                   void *workspace, size_t ws_bytes,
+                                   hlta_dtype dt, void *stream);
+
+/*
  * hlta_gdn_chunk_fwd for callers that cannot allocate device memory (no counterpart on the
  * pages: an interface addition of this library). Some callers may not allocate: code embedded
  * in a host application that owns the device-memory budget and passes in only inputs and
@@ -159,6 +179,19 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v,
                             int w_swa, int w_dswa, int r, int chunk, float scale,
                             void *workspace, size_t ws_bytes,
                             hlta_dtype dt, void *stream);
+
+/*
+ * hlta_hybrid_fwd with raw GDN inputs: the GDN heads' q, k are scaled to unit L2 norm per
+ * token and their gates computed from x, y as in hlta_gdn_chunk_fwd_raw (x, y: [B, Hg, T*N]
+ * float32; c >= 0). The softmax heads are unchanged (their q, k are used as given).
+ */
+hlta_status hlta_hybrid_fwd_raw(const void *q, const void *k, const void *v,
+                                const float *x, const float *y, float c, void *o,
+                                const float *S0, float *S_out,
+                                int B, int Hs, int Hd, int Hg, int T, int N, int d,
+                                int w_swa, int w_dswa, int r, int chunk, float scale,
+                                void *workspace, size_t ws_bytes,
+                                hlta_dtype dt, void *stream);
 
 /*
  * Streaming rollout (zhichai.net blog, section 2.3: the "streaming token" design generates

@@ -42,10 +42,13 @@ def _load() -> ctypes.CDLL:
         "hlta_dswa_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, F, I, P]),
         "hlta_gdn_workspace_bytes": (Z, [I, I, L, I, I, I]),
         "hlta_gdn_chunk_fwd": (I, [P, P, P, P, P, P, P, P, I, I, L, I, I, P, Z, I, P]),
+        "hlta_gdn_chunk_fwd_raw": (I, [P, P, P, P, P, F, P, P, P, I, I, L, I, I, P, Z, I, P]),
         "hlta_gdn_chunk_fwd_static": (I, [P, P, P, P, P, P, P, P, I, I, L, I, I, I, P]),
         "hlta_hybrid_workspace_bytes": (Z, [I, I, I, I, I, I, I]),
         "hlta_hybrid_fwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F,
                                 P, Z, I, P]),
+        "hlta_hybrid_fwd_raw": (I, [P, P, P, P, P, F, P, P, P, I, I, I, I, I, I, I, I, I, I, I,
+                                    F, P, Z, I, P]),
         "hlta_stream_create": (I, [ctypes.POINTER(P), I, I, I, I, I, I, I, I, I, I, F, I, P]),
         "hlta_stream_step": (I, [P, P, P, P, P, P, P, P]),
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
@@ -126,6 +129,16 @@ def hlta_gdn_chunk_fwd(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, workspace
                                    _dt(q), _stream(stream)))
 
 
+def hlta_gdn_chunk_fwd_raw(q, k, v, x, y, c, o, S0, S_out, B, H, L, d, chunk, workspace,
+                           stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (x, "x"), (y, "y"), (o, "o"), (workspace, "workspace")):
+        _need(t, n)
+    _check(_lib.hlta_gdn_chunk_fwd_raw(_p(q), _p(k), _p(v), _p(x), _p(y), float(c), _p(o), _p(S0),
+                                       _p(S_out), B, H, L, d, chunk, _p(workspace),
+                                       workspace.numel() * workspace.element_size(), _dt(q),
+                                       _stream(stream)))
+
+
 HLTA_STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
@@ -150,6 +163,16 @@ def hlta_hybrid_fwd(q, k, v, a, b, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa, 
     _check(_lib.hlta_hybrid_fwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(o), _p(S0), _p(S_out),
                                 B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa, r, chunk, float(scale),
                                 ws_ptr, ws_bytes, _dt(q), _stream(stream)))
+
+
+def hlta_hybrid_fwd_raw(q, k, v, x, y, c, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa,
+                        r, chunk, scale, workspace, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, n)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (_p(workspace), workspace.numel() * workspace.element_size())
+    _check(_lib.hlta_hybrid_fwd_raw(_p(q), _p(k), _p(v), _p(x), _p(y), float(c), _p(o), _p(S0),
+                                    _p(S_out), B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa, r, chunk,
+                                    float(scale), ws_ptr, ws_bytes, _dt(q), _stream(stream)))
 
 
 def hlta_device_status(stream=None) -> int:
@@ -199,6 +222,35 @@ def gdn(q, k, v, a, b, S0=None, chunk=64, out=None, S_out=None, workspace=None, 
     if workspace is None:
         workspace = _workspace(hlta_gdn_workspace_bytes(B, H, L, d, chunk, _dt(q)), q.device)
     hlta_gdn_chunk_fwd(q, k, v, a, b, o, S0, S_out, B, H, L, d, chunk, workspace, stream)
+    return o, S_out
+
+
+def gdn_raw(q, k, v, x, y, c, S0=None, chunk=64, out=None, S_out=None, workspace=None,
+            stream=None):
+    """GDN heads from raw q, k and raw gate inputs x, y (see hlta_gdn_chunk_fwd_raw)."""
+    import torch
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    if S_out is None:
+        S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(hlta_gdn_workspace_bytes(B, H, L, d, chunk, _dt(q)), q.device)
+    hlta_gdn_chunk_fwd_raw(q, k, v, x, y, c, o, S0, S_out, B, H, L, d, chunk, workspace, stream)
+    return o, S_out
+
+
+def hybrid_raw(q, k, v, x, y, c, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, S0=None, chunk=64,
+               scale=0.0, out=None, S_out=None, workspace=None, stream=None):
+    """The hybrid operator with raw GDN inputs (see hlta_hybrid_fwd_raw)."""
+    import torch
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    if Hg and S_out is None:
+        S_out = torch.empty((B, Hg, d, d), dtype=torch.float32, device=q.device)
+    if Hg and workspace is None:
+        workspace = _workspace(hlta_hybrid_workspace_bytes(B, Hg, T, N, d, chunk, _dt(q)), q.device)
+    hlta_hybrid_fwd_raw(q, k, v, x, y, c, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa, w_dswa,
+                        r, chunk, scale, workspace, stream)
     return o, S_out
 
 

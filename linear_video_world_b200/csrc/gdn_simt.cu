@@ -63,14 +63,27 @@ __global__ void __launch_bounds__(PREP_THREADS) gdn_prep_f32(GdnArgs p, GdnWorks
         VW[t * dp + c] = ok ? v[(long)t * d + c] : 0.f;
     }
     if (tid == 0) {
+        // log of the decay gate: log a, or with raw inputs -c softplus(x); the write
+        // strength b, or sigmoid(y)
         float acc = 0.f;
         for (int t = 0; t < C; ++t) {
-            if (t < n) acc += logf(ag[t]);
+            if (t < n) acc += p.raw ? -p.raw_c * (ag[t] > 20.f ? ag[t] : log1pf(expf(ag[t]))) : logf(ag[t]);
             g[t] = acc;
-            bb[t] = t < n ? bg[t] : 0.f;
+            bb[t] = t < n ? (p.raw ? 1.f / (1.f + expf(-bg[t])) : bg[t]) : 0.f;
         }
     }
     __syncthreads();
+    // raw inputs: q and k of every token scaled to unit L2 norm (rows of zeros stay zero)
+    if (p.raw) {
+        if (tid < 2 * C) {
+            float *row = (tid < C ? Qc : Kc) + (tid & (C - 1)) * dp;
+            float ss = 0.f;
+            for (int c = 0; c < d; ++c) ss = fmaf(row[c], row[c], ss);
+            const float sc = ss > 0.f ? 1.f / sqrtf(ss) : 0.f;
+            for (int c = 0; c < d; ++c) row[c] *= sc;
+        }
+        __syncthreads();
+    }
 
     // A (strictly lower) and P (lower, diagonal included)
     for (int e = tid; e < C * C; e += PREP_THREADS) {

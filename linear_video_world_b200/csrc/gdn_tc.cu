@@ -119,6 +119,21 @@ __device__ __forceinline__ float fast_ex2(float x)
     return y;
 }
 
+// log2 of the decay gate a of a token: from a itself, or with raw inputs from x as
+// log2 exp(-c softplus(x)) = -c softplus(x) / ln 2 (softplus(x) = log(1 + e^x), taken as x
+// itself where e^-x is below float resolution)
+__device__ __forceinline__ float log2_gate(const GdnArgs &p, float v)
+{
+    if (!p.raw) return fast_lg2(v);
+    const float sp = v > 20.f ? v : log1pf(__expf(v));
+    return -p.raw_c * sp * 1.4426950408889634f;
+}
+// the write strength b of a token: b itself, or with raw inputs sigmoid(y)
+__device__ __forceinline__ float beta_gate(const GdnArgs &p, float v)
+{
+    return p.raw ? 1.f / (1.f + __expf(-v)) : v;
+}
+
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -235,8 +250,8 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
         // inclusive prefix sum of log2 a over 64 entries (decays are then 2^(g_t - g_i), one
         // ex2 each): two per lane, then a warp scan
         const int t = 2 * lane;
-        const float l0 = t < n ? fast_lg2(p.a[(long)bh * p.L + t0 + t]) : 0.f;
-        const float l1 = t + 1 < n ? fast_lg2(p.a[(long)bh * p.L + t0 + t + 1]) : 0.f;
+        const float l0 = t < n ? log2_gate(p, p.a[(long)bh * p.L + t0 + t]) : 0.f;
+        const float l1 = t + 1 < n ? log2_gate(p, p.a[(long)bh * p.L + t0 + t + 1]) : 0.f;
         float pair = l0 + l1, x = pair;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -245,8 +260,8 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
         }
         s.g[t] = x - pair + l0;
         s.g[t + 1] = x;
-        s.bb[t] = t < n ? p.b[(long)bh * p.L + t0 + t] : 0.f;
-        s.bb[t + 1] = t + 1 < n ? p.b[(long)bh * p.L + t0 + t + 1] : 0.f;
+        s.bb[t] = t < n ? beta_gate(p, p.b[(long)bh * p.L + t0 + t]) : 0.f;
+        s.bb[t + 1] = t + 1 < n ? beta_gate(p, p.b[(long)bh * p.L + t0 + t + 1]) : 0.f;
     }
     __syncthreads();                                       // barrier initialised, g, bb ready
     if (tid < C) {
@@ -273,6 +288,39 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
             *reinterpret_cast<uint4 *>(s.Q + off) = make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(s.K + off) = make_uint4(0, 0, 0, 0);
             *reinterpret_cast<uint4 *>(s.V + off) = make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+    }
+    // raw inputs: scale the staged q and k of every token to unit L2 norm (two threads per
+    // row, 64 columns each; rows of zeros stay zero)
+    if (p.raw) {
+        const int row = tid >> 1, half = tid & 1;          // rows 0..63: Q, 64..127: K
+        uint8_t *tile = row < C ? s.Q : s.K;
+        const int t = row & (C - 1);
+        float ss = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(tile + sw128_off(t, (half * 8 + c8) * 8, C));
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+            }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        const float sc = ss > 0.f ? rsqrtf(ss) : 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+            uint4 *pu = reinterpret_cast<uint4 *>(tile + sw128_off(t, (half * 8 + c8) * 8, C));
+            uint4 u = *pu;
+            __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                h2[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+            }
+            *pu = u;
         }
         __syncthreads();
     }

@@ -169,6 +169,12 @@ hlta_status check_gdn_common(const void *q, const void *k, const void *v, const 
     return HLTA_OK;
 }
 
+hlta_status check_raw_c(float c)
+{
+    if (!(c >= 0.f) || !(c <= 1e30f)) return fail(HLTA_ERR_INVALID_ARG, "decay constant c must be finite and >= 0 (got %g)", (double)c);
+    return HLTA_OK;
+}
+
 }  // namespace
 
 size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
@@ -251,12 +257,14 @@ size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dty
     return gdn_workspace_bytes((long)B * H, L, d, chunk, dt == HLTA_BF16);
 }
 
-hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *a,
-                               const float *b, void *o, const float *S0, float *S_out, int B,
-                               int H, long L, int d, int chunk, void *workspace,
-                               size_t ws_bytes, hlta_dtype dt, void *stream)
+namespace {
+hlta_status gdn_fwd_impl(const void *q, const void *k, const void *v, const float *a,
+                         const float *b, int raw, float raw_c, void *o, const float *S0,
+                         float *S_out, int B, int H, long L, int d, int chunk, void *workspace,
+                         size_t ws_bytes, hlta_dtype dt, void *stream)
 {
     hlta_status st = check_gdn_common(q, k, v, a, b, o, S0, S_out, d, chunk, dt);
+    if (st == HLTA_OK && raw) st = check_raw_c(raw_c);
     if (st != HLTA_OK) return st;
     if (B < 0 || H < 0 || L < 1 || L > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld", B, H, L);
     size_t need = gdn_workspace_bytes((long)B * H, L, d, chunk, dt == HLTA_BF16);
@@ -265,11 +273,30 @@ hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v, cons
     if (((uintptr_t)workspace & 255u) != 0) return fail(HLTA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     DeviceCtx *ctx;
     if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
-    GdnArgs g;
-    g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o;
+    GdnArgs g = {};
+    g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o; g.raw = raw; g.raw_c = raw_c;
     g.B = B; g.Hg = H; g.Htot = H; g.h0 = 0; g.L = L; g.d = d; g.chunk = chunk;
     g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
     return run_gdn(g, dt, (cudaStream_t)stream);
+}
+}  // namespace
+
+hlta_status hlta_gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *a,
+                               const float *b, void *o, const float *S0, float *S_out, int B,
+                               int H, long L, int d, int chunk, void *workspace,
+                               size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    return gdn_fwd_impl(q, k, v, a, b, 0, 0.f, o, S0, S_out, B, H, L, d, chunk, workspace,
+                        ws_bytes, dt, stream);
+}
+
+hlta_status hlta_gdn_chunk_fwd_raw(const void *q, const void *k, const void *v, const float *x,
+                                   const float *y, float c, void *o, const float *S0,
+                                   float *S_out, int B, int H, long L, int d, int chunk,
+                                   void *workspace, size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    return gdn_fwd_impl(q, k, v, x, y, 1, c, o, S0, S_out, B, H, L, d, chunk, workspace,
+                        ws_bytes, dt, stream);
 }
 
 size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk, hlta_dtype dt)
@@ -278,11 +305,12 @@ size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk
     return gdn_workspace_bytes((long)B * Hg, (long)T * N, d, chunk, dt == HLTA_BF16);
 }
 
-hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const float *a,
-                            const float *b, void *o, const float *S0, float *S_out, int B,
-                            int Hs, int Hd, int Hg, int T, int N, int d, int w_swa,
-                            int w_dswa, int r, int chunk, float scale, void *workspace,
-                            size_t ws_bytes, hlta_dtype dt, void *stream)
+namespace {
+hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const float *a,
+                            const float *b, int raw, float raw_c, void *o, const float *S0,
+                            float *S_out, int B, int Hs, int Hd, int Hg, int T, int N, int d,
+                            int w_swa, int w_dswa, int r, int chunk, float scale,
+                            void *workspace, size_t ws_bytes, hlta_dtype dt, void *stream)
 {
     hlta_status st;
     if (B < 0 || Hs < 0 || Hd < 0 || Hg < 0 || T < 1 || N < 1)
@@ -298,6 +326,7 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const f
     const long L = (long)T * N;
     if (Hg) {
         if ((st = check_gdn_common(q, k, v, a, b, o, S0, S_out, d, chunk, dt)) != HLTA_OK) return st;
+        if (raw && (st = check_raw_c(raw_c)) != HLTA_OK) return st;
         size_t need = gdn_workspace_bytes((long)B * Hg, L, d, chunk, dt == HLTA_BF16);
         if (!workspace || ws_bytes < need)
             return fail(HLTA_ERR_INVALID_ARG, "workspace too small: need %zu bytes, got %zu", need, ws_bytes);
@@ -312,8 +341,8 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const f
     if (Hg) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
-        GdnArgs g;
-        g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o;
+        GdnArgs g = {};
+        g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o; g.raw = raw; g.raw_c = raw_c;
         g.B = B; g.Hg = Hg; g.Htot = H; g.h0 = Hs + Hd; g.L = L; g.d = d; g.chunk = chunk;
         g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
         prof_record(3, ctx->aux);
@@ -340,6 +369,27 @@ hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const f
     // join: work enqueued on `s` after this call sees the GDN outputs too
     if (Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     return st;
+}
+}  // namespace
+
+hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v, const float *a,
+                            const float *b, void *o, const float *S0, float *S_out, int B,
+                            int Hs, int Hd, int Hg, int T, int N, int d, int w_swa,
+                            int w_dswa, int r, int chunk, float scale, void *workspace,
+                            size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    return hybrid_fwd_impl(q, k, v, a, b, 0, 0.f, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa,
+                           w_dswa, r, chunk, scale, workspace, ws_bytes, dt, stream);
+}
+
+hlta_status hlta_hybrid_fwd_raw(const void *q, const void *k, const void *v, const float *x,
+                                const float *y, float c, void *o, const float *S0, float *S_out,
+                                int B, int Hs, int Hd, int Hg, int T, int N, int d, int w_swa,
+                                int w_dswa, int r, int chunk, float scale, void *workspace,
+                                size_t ws_bytes, hlta_dtype dt, void *stream)
+{
+    return hybrid_fwd_impl(q, k, v, x, y, 1, c, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, w_swa,
+                           w_dswa, r, chunk, scale, workspace, ws_bytes, dt, stream);
 }
 
 hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N, int d,
@@ -416,7 +466,7 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         lk.lock();
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
-        GdnArgs g;
+        GdnArgs g = {};
         g.q = q_new; g.k = k_new; g.v = v_new; g.a = a_new; g.b = b_new; g.o = o_new;
         g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = c->N; g.d = c->d;
         g.chunk = c->chunk; g.S0 = c->S; g.S_out = c->S; g.ws = c->ws; g.ws_bytes = c->ws_bytes;

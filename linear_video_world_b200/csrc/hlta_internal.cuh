@@ -33,7 +33,10 @@ struct AttnArgs {
 // Gates a, b: [B][Hg][L]. State: [B][Hg][d][d] (S[i][j], i value index, j key index).
 struct GdnArgs {
     const void *q, *k, *v;
-    const float *a, *b;
+    const float *a, *b;         // gates; with `raw` the raw gate inputs x, y instead
+    int raw;                    // 1: q, k raw (scaled to unit L2 norm per token inside the
+                                //    chunk preparation), a = exp(-raw_c softplus(x)), b = sigmoid(y)
+    float raw_c;
     void *o;
     int B, Hg, Htot, h0;
     long L;

@@ -50,7 +50,8 @@ def _load():
         lib.oracle_swa.argtypes = [f32, f32, f32, f64, L_, I_, I_, I_, I_, D_, i64, L_]
         lib.oracle_dswa.argtypes = [f32, f32, f32, f64, L_, I_, I_, I_, I_, I_, D_, i64, L_]
         lib.oracle_gdn.argtypes = [f32, f32, f32, f32, f32, f64, f64, f64, f64, L_, L_, I_]
-        for fn in (lib.oracle_swa, lib.oracle_dswa, lib.oracle_gdn):
+        lib.oracle_gdn_raw.argtypes = [f32, f32, f32, f32, f32, D_, f64, f64, f64, L_, L_, I_]
+        for fn in (lib.oracle_swa, lib.oracle_dswa, lib.oracle_gdn, lib.oracle_gdn_raw):
             fn.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -145,11 +146,37 @@ def gdn(q, k, v, a, b, S0=None, history: bool = False):
     return (o, S_out, hist) if history else (o, S_out)
 
 
+def gdn_raw(q, k, v, x, y, c: float, S0=None):
+    """GDN heads from raw inputs: q, k scaled to unit L2 norm per token, gates
+    a = exp(-c softplus(x)), b = sigmoid(y), then the recurrence (all fp64).
+    q,k,v: [..., L, d]; x,y: [..., L]. Returns (o, S_final)."""
+    qf, kf, vf, xf, yf = _f32(q), _f32(k), _f32(v), _f32(x), _f32(y)
+    d = qf.shape[-1]
+    L = qf.shape[-2]
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    S0d = None
+    if S0 is not None:
+        if hasattr(S0, "detach"):
+            S0 = S0.detach().cpu().double().numpy()
+        S0d = np.ascontiguousarray(np.asarray(S0, dtype=np.float64)).reshape(BH, d, d)
+    o = np.empty(qf.shape, dtype=np.float64)
+    S_out = np.empty(lead + (d, d), dtype=np.float64)
+    rc = _load().oracle_gdn_raw(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                                _ptr(vf, ctypes.c_float), _ptr(xf, ctypes.c_float),
+                                _ptr(yf, ctypes.c_float), float(c), _ptr(S0d, ctypes.c_double),
+                                _ptr(o, ctypes.c_double), _ptr(S_out, ctypes.c_double), BH, L, d)
+    if rc != 0:
+        raise RuntimeError(f"oracle gdn_raw failed ({rc})")
+    return o, S_out
+
+
 def hybrid(q, k, v, a, b, Hs: int, Hd: int, Hg: int, T: int, N: int,
-           w_swa: int, w_dswa: int, r: int, S0=None, scale=None):
+           w_swa: int, w_dswa: int, r: int, S0=None, scale=None, raw=None):
     """All three branches on their head groups of [B, H, L, d]; concat on the head axis.
 
-    Returns (o [B,H,L,d] float64, S_final [B,Hg,d,d] float64)."""
+    With ``raw`` = c the GDN heads take raw inputs: ``a``, ``b`` are then x, y and the GDN
+    branch is ``gdn_raw(..., c=raw)``. Returns (o [B,H,L,d] float64, S_final [B,Hg,d,d])."""
     qf, kf, vf = _f32(q), _f32(k), _f32(v)
     B, H, L, d = qf.shape
     assert H == Hs + Hd + Hg
@@ -162,7 +189,10 @@ def hybrid(q, k, v, a, b, Hs: int, Hd: int, Hg: int, T: int, N: int,
     S_fin = np.zeros((B, Hg, d, d))
     if Hg:
         s = slice(Hs + Hd, H)
-        og, S_fin = gdn(qf[:, s], kf[:, s], vf[:, s], a, b, S0)
+        if raw is None:
+            og, S_fin = gdn(qf[:, s], kf[:, s], vf[:, s], a, b, S0)
+        else:
+            og, S_fin = gdn_raw(qf[:, s], kf[:, s], vf[:, s], a, b, raw, S0)
         o[:, s] = og
     return o, S_fin
 

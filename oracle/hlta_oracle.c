@@ -211,6 +211,81 @@ int oracle_gdn(const float *q, const float *k, const float *v, const float *a,
     return err;
 }
 
+/*
+ * GDN heads from raw inputs: the prologue upstream of the recurrence, then the recurrence.
+ * The delta rule's erase step is a contraction only for unit keys (researchpapers.dev
+ * summary, Theorem 2: ||I - b k k^T|| <= 1 needs ||k|| = 1 and b in [0, 1]), so the raw q and
+ * k of a token are scaled to unit L2 norm (a zero vector stays zero); the gates are
+ *     a_t = exp(-c * softplus(x_t)) in (0, 1],   b_t = sigmoid(y_t) in (0, 1),
+ * softplus(x) = log(1 + e^x) evaluated without overflow. Everything in double precision;
+ * the recurrence is the one of oracle_gdn, repeated here on the double inputs.
+ */
+int oracle_gdn_raw(const float *q, const float *k, const float *v, const float *x,
+                   const float *y, double c, const double *S0, double *o, double *S_out,
+                   long BH, long L, int d)
+{
+    if (BH <= 0 || L < 0 || d <= 0) return 1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)d * d);
+        double *Sk = (double *)malloc(sizeof(double) * (size_t)d);
+        double *qn = (double *)malloc(sizeof(double) * (size_t)d);
+        double *kn = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!S || !Sk || !qn || !kn) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                if (S0) memcpy(S, S0 + bh * d * d, sizeof(double) * (size_t)d * d);
+                else memset(S, 0, sizeof(double) * (size_t)d * d);
+                for (long t = 0; t < L; ++t) {
+                    const float *kt = k + (bh * L + t) * d;
+                    const float *vt = v + (bh * L + t) * d;
+                    const float *qt = q + (bh * L + t) * d;
+                    double qq = 0.0, kk = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        qq += (double)qt[j] * (double)qt[j];
+                        kk += (double)kt[j] * (double)kt[j];
+                    }
+                    const double qs = qq > 0.0 ? 1.0 / sqrt(qq) : 0.0;
+                    const double ks = kk > 0.0 ? 1.0 / sqrt(kk) : 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        qn[j] = (double)qt[j] * qs;
+                        kn[j] = (double)kt[j] * ks;
+                    }
+                    const double xt = x[bh * L + t], yt = y[bh * L + t];
+                    const double sp = xt > 0.0 ? xt + log1p(exp(-xt)) : log1p(exp(xt));
+                    const double at = exp(-c * sp);
+                    const double bt = 1.0 / (1.0 + exp(-yt));
+                    for (int i = 0; i < d; ++i) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += S[(long)i * d + j] * kn[j];
+                        Sk[i] = s;
+                    }
+                    for (int i = 0; i < d; ++i)
+                        for (int j = 0; j < d; ++j)
+                            S[(long)i * d + j] = at * (S[(long)i * d + j] - bt * Sk[i] * kn[j])
+                                                 + bt * (double)vt[i] * kn[j];
+                    double *ot = o + (bh * L + t) * d;
+                    for (int i = 0; i < d; ++i) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += S[(long)i * d + j] * qn[j];
+                        ot[i] = s;
+                    }
+                }
+                if (S_out) memcpy(S_out + bh * d * d, S, sizeof(double) * (size_t)d * d);
+            }
+        }
+        free(S);
+        free(Sk);
+        free(qn);
+        free(kn);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

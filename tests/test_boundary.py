@@ -61,6 +61,20 @@ def test_bad_shapes_rejected_on_host(lib):
     assert b"workspace" in lib.hlta_last_error()
 
 
+def test_raw_entry_points_validate_decay_constant_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    for c in (-0.5, float("nan"), float("inf")):
+        assert lib.hlta_gdn_chunk_fwd_raw(p, p, p, p, p, c, p, None, None, 1, 1, 100, 128, 64, p,
+                                          1 << 30, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+        assert b"decay" in lib.hlta_last_error()
+        assert lib.hlta_hybrid_fwd_raw(p, p, p, p, p, c, p, None, None, 1, 1, 1, 1, 2, 16, 128, 2,
+                                       2, 2, 64, 0.0, p, 1 << 30, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+    # null gate inputs are rejected like null gates
+    assert lib.hlta_gdn_chunk_fwd_raw(p, p, p, None, p, 1.0, p, None, None, 1, 1, 100, 128, 64, p,
+                                      1 << 30, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(lib):
     import linear_video_world_b200 as h
     # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16 plus a 16-byte slot per chunk

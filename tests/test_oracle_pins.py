@@ -339,3 +339,94 @@ def test_hybrid_head_groups_in_order(orc):
     og, Sg = orc.gdn(q[:, 2:], k[:, 2:], v[:, 2:], x["a"], x["b"])
     np.testing.assert_array_equal(o[:, 2:], og)
     np.testing.assert_array_equal(S, Sg)
+
+
+# --------------------------------------------------------------------------------------
+# GDN prologue (raw inputs): unit-norm q, k; a = exp(-c softplus(x)), b = sigmoid(y)
+# --------------------------------------------------------------------------------------
+
+def test_gdn_raw_is_scale_invariant_in_q_and_k(orc):
+    """Only the direction of q and k matters: per-token positive scales (powers of two, exact
+    in float32) leave every output and the final state unchanged."""
+    r = _rng(21)
+    L, d = 40, 16
+    q, k, v = (r.standard_normal((2, L, d)).astype(np.float32) for _ in range(3))
+    x, y = (r.standard_normal((2, L)).astype(np.float32) for _ in range(2))
+    sq = np.exp2(r.integers(-6, 7, size=(2, L, 1))).astype(np.float32)
+    sk = np.exp2(r.integers(-6, 7, size=(2, L, 1))).astype(np.float32)
+    o1, S1 = orc.gdn_raw(q, k, v, x, y, 0.7)
+    o2, S2 = orc.gdn_raw(q * sq, k * sk, v, x, y, 0.7)
+    np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S2, S1, rtol=0, atol=1e-12)
+    # and q, k are not used as given: doubling only k changes nothing, doubling v does
+    o3, _ = orc.gdn_raw(q, k, 2 * v, x, y, 0.7)
+    np.testing.assert_allclose(o3, 2 * o1, rtol=1e-12, atol=1e-12)
+
+
+def test_gdn_raw_equals_gdn_through_inverse_gates(orc):
+    """Gates given through the inverses of the activations (x = log(e^s - 1) so that
+    softplus(x) = s = -log(a)/c; y = log(b / (1 - b))) and unit q, k: the raw path must
+    reproduce the pinned recurrence."""
+    r = _rng(22)
+    L, d, c = 30, 12, 0.6
+    q, k, v = (r.standard_normal((1, L, d)) for _ in range(3))
+    q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    a = r.uniform(0.5, 0.99, size=(1, L))
+    b = r.uniform(0.05, 0.95, size=(1, L))
+    s = -np.log(a) / c
+    x = np.log(np.expm1(s))
+    y = np.log(b / (1 - b))
+    o_raw, S_raw = orc.gdn_raw(q.astype(np.float32), k.astype(np.float32), v.astype(np.float32),
+                               x.astype(np.float32), y.astype(np.float32), c)
+    # the reference gets the same float32-rounded values, gates recomputed from the rounded x, y
+    xr, yr = x.astype(np.float32).astype(np.float64), y.astype(np.float32).astype(np.float64)
+    a_r = np.exp(-c * np.log1p(np.exp(xr)))
+    b_r = 1 / (1 + np.exp(-yr))
+    o_ref, S_ref = orc.gdn(q.astype(np.float32), k.astype(np.float32), v.astype(np.float32),
+                           a_r.astype(np.float32), b_r.astype(np.float32))
+    np.testing.assert_allclose(o_raw, o_ref, rtol=0, atol=2e-6)
+    np.testing.assert_allclose(S_raw, S_ref, rtol=0, atol=2e-6)
+
+
+def test_gdn_raw_neutral_gate_inputs_closed_form(orc):
+    """x = 0 gives softplus(0) = ln 2, so a = 2^-c; y = -200 gives b = 0 to double precision:
+    no writes, pure decay, o_t = 2^(-c (t+1)) S0 q_t / |q_t|."""
+    r = _rng(23)
+    L, d, c = 9, 6, 1.5
+    q, k, v = (r.standard_normal((1, L, d)).astype(np.float32) for _ in range(3))
+    S0 = r.standard_normal((1, d, d))
+    x = np.zeros((1, L), np.float32)
+    y = np.full((1, L), -200.0, np.float32)
+    o, S = orc.gdn_raw(q, k, v, x, y, c, S0=S0)
+    qn = q[0].astype(np.float64) / np.linalg.norm(q[0].astype(np.float64), axis=-1, keepdims=True)
+    for t in range(L):
+        np.testing.assert_allclose(o[0, t], 2.0 ** (-c * (t + 1)) * S0[0] @ qn[t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S[0], 2.0 ** (-c * L) * S0[0], rtol=1e-12, atol=1e-13)
+
+
+def test_gdn_raw_zero_token_stays_zero(orc):
+    """A token whose q and k are zero reads nothing and erases/writes along no direction:
+    its output is zero and the state only decays."""
+    r = _rng(24)
+    L, d = 5, 8
+    q, k, v = (r.standard_normal((1, L, d)).astype(np.float32) for _ in range(3))
+    q[0, 2] = 0
+    k[0, 2] = 0
+    x, y = (r.standard_normal((1, L)).astype(np.float32) for _ in range(2))
+    o, _ = orc.gdn_raw(q, k, v, x, y, 1.0)
+    assert np.all(o[0, 2] == 0)
+    assert np.all(np.isfinite(o))
+
+
+def test_hybrid_raw_routes_gdn_heads_through_the_prologue(orc):
+    import hlta_inputs as hi
+    wl = hi.WORKLOADS["tiny_fp32"]
+    x = hi.make_raw_inputs(wl, seed=4)
+    q, k, v = (x[n].numpy() for n in ("q", "k", "v"))
+    o, S = orc.hybrid(q, k, v, x["x"], x["y"], 1, 1, 1, wl.T, wl.N, wl.w_swa, wl.w_dswa, wl.r,
+                      raw=wl.decay)
+    og, Sg = orc.gdn_raw(q[:, 2:], k[:, 2:], v[:, 2:], x["x"], x["y"], wl.decay)
+    np.testing.assert_array_equal(o[:, 2:], og)
+    np.testing.assert_array_equal(S, Sg)
+    np.testing.assert_array_equal(o[:, 0], orc.swa(q[:, 0], k[:, 0], v[:, 0], wl.T, wl.N, wl.w_swa))
