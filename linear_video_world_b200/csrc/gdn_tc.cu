@@ -37,7 +37,7 @@ constexpr int C = 64;             // chunk length
 constexpr int D = 128;            // head dim
 constexpr int SD = D + 8;         // padded smem row stride (elements) of [.][128] bf16 tiles
 constexpr int SC = C + 8;         // padded smem row stride of [.][64] bf16 tiles
-constexpr int FP = C + 1;         // fp32 [64][65] tiles
+constexpr int AP = C + 4;         // fp32 row stride of A: 16-byte aligned rows
 constexpr int THREADS = 128;
 constexpr int RB = 16;            // state rows per CTA in the state pass
 
@@ -145,29 +145,27 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 // prep
 // -----------------------------------------------------------------------------------------
 constexpr int PREP_THREADS = 256;
-constexpr int TP = C + 4;                  // fp32 row stride of T
 constexpr uint32_t SWT = C * D * 2;        // one swizzled [64][128] bf16 tile: 16 KB
 
-// Shared memory of the prep kernel (about 97 KB: two CTAs per SM). Q, K, V arrive by TMA as
+// Shared memory of the prep kernel (about 92 KB: two CTAs per SM). Q, K, V arrive by TMA as
 // swizzled tiles; regions are reused once their contents are dead:
-//   R1: A (fp32 [64][65]) -> T1, T2 (bf16 [64][72] each) -> Op (swizzled tile)
-//   R2: T (fp32 [64][68]) -> W (swizzled tile)
+//   R1: A (fp32 [64][68]) -> T1, T2 (bf16 [64][72] each) -> Op (swizzled tile)
+//   R2: W (swizzled tile)
 //   V:  V -> Up          Q:  Q -> Qt (in place)
+// T = (I + A)^{-1} itself never reaches shared memory: its columns live in registers.
 struct PrepSmem {
     alignas(1024) uint8_t Q[SWT];
     alignas(1024) uint8_t K[SWT];
     alignas(1024) uint8_t V[SWT];
-    alignas(1024) uint8_t R2[C * TP * 4];
+    alignas(1024) uint8_t R2[SWT];
     alignas(16) uint8_t R1[2 * C * SC * 2];
     __nv_bfloat16 P[C * SC];
-    float X[3 * 256];             // off-diagonal block products of the blocked inversion
     float g[C], eg[C], ek[C], bb[C];
     alignas(8) uint64_t bar;
     int abort_flag;
 };
-static_assert(sizeof(float) * C * (C + 1) <= 2 * C * SC * 2, "A must fit in R1");
+static_assert(sizeof(float) * C * AP <= 2 * C * SC * 2, "A must fit in R1");
 static_assert(SWT <= 2 * C * SC * 2, "Op must fit in R1");
-static_assert(SWT <= C * TP * 4, "W must fit in R2");
 
 // One warp's 16 rows x (NT*8) columns of X = Am ([64][lda] row-major, padded) times a
 // swizzled [K][N] tile, k-steps 0 .. ksteps-1, columns n0 ...
@@ -214,11 +212,10 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
 {
     extern __shared__ uint8_t smem_raw[];
     PrepSmem &s = *reinterpret_cast<PrepSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    float *A = reinterpret_cast<float *>(s.R1);            // [64][65]
+    float *A = reinterpret_cast<float *>(s.R1);            // [64][68]
     __nv_bfloat16 *T1 = reinterpret_cast<__nv_bfloat16 *>(s.R1);
     __nv_bfloat16 *T2 = T1 + C * SC;
     uint8_t *Op = s.R1;
-    float *T = reinterpret_cast<float *>(s.R2);            // [64][68]
     uint8_t *W = s.R2;
 
     const int chunk = blockIdx.x, bh = blockIdx.y;
@@ -269,7 +266,6 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
         s.eg[tid] = tid < n ? fast_ex2(s.g[tid]) : 0.f;
         s.ek[tid] = tid < n ? fast_ex2(gn - s.g[tid]) : 0.f;
     }
-    for (int e = tid; e < C * TP; e += PREP_THREADS) T[e] = 0.f;
     const bool landed = ptx::mbar_wait(bar, 0, (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
     if (!__syncthreads_and(landed)) {
         // a bounded wait expired: give the three copies a last bounded chance to land
@@ -359,51 +355,52 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
                 const int i = n0 + nt * 8 + 2 * tg + (e & 1);
                 const bool lower = i <= t && t < n;
                 const float dec = lower ? fast_ex2(s.g[t] - s.g[i]) : 0.f;
-                A[t * FP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
+                A[t * AP + i] = (i < t && t < n) ? s.bb[t] * dec * kk[nt][e] : 0.f;
                 s.P[t * SC + i] = __float2bfloat16_rn(lower ? dec * qk[nt][e] : 0.f);
             }
         }
     }
     __syncthreads();
 
-    // ---- T = (I + A)^{-1}, blocked by 16: diagonal blocks by forward substitution, then
-    //      T_IJ = -T_II * sum_{K=J}^{I-1} A_IK T_KJ block row by block row
-    if (tid < C) {
-        const int I = tid >> 4, jj = tid & 15, base = I * 16, j = base + jj;
-        T[j * TP + j] = 1.f;
-        for (int t = jj + 1; t < 16; ++t) {
-            float acc = 0.f;
-            for (int i = jj; i < t; ++i) acc = fmaf(A[(base + t) * FP + base + i], T[(base + i) * TP + j], acc);
-            T[(base + t) * TP + j] = -acc;
+    // ---- T = (I + A)^{-1} (A strictly lower triangular, so T is unit lower triangular) by
+    //      forward substitution, one column per thread held in registers:
+    //      T_tj = -sum_{i<t} A_ti T_ij (T_tj = 0 above the diagonal, 1 on it), the row of A
+    //      read as float4 broadcasts and summed in four partial sums. Then T1 = T diag(b e^g)
+    //      and T2 = T diag(b) in bf16, written over A once every column is done.
+    {
+        float tc[C];
+        if (tid < C) {
+            const int j = tid;
+#pragma unroll
+            for (int t = 0; t < C; ++t) {
+                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                const float4 *ar = reinterpret_cast<const float4 *>(A + t * AP);
+#pragma unroll
+                for (int i4 = 0; i4 < t / 4; ++i4) {
+                    const float4 av = ar[i4];
+                    a0 = fmaf(av.x, tc[4 * i4], a0);
+                    a1 = fmaf(av.y, tc[4 * i4 + 1], a1);
+                    a2 = fmaf(av.z, tc[4 * i4 + 2], a2);
+                    a3 = fmaf(av.w, tc[4 * i4 + 3], a3);
+                }
+#pragma unroll
+                for (int i = (t / 4) * 4; i < t; ++i) a0 = fmaf(A[t * AP + i], tc[i], a0);
+                const float acc = (a0 + a1) + (a2 + a3);
+                tc[t] = t < j ? 0.f : (t == j ? 1.f : -acc);
+            }
         }
-    }
-    __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < I * 256; e += PREP_THREADS) {
-            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            const int row = I * 16 + r, col = J * 16 + c;
-            float acc = 0.f;
-            for (int kx = J * 16; kx < I * 16; ++kx) acc = fmaf(A[row * FP + kx], T[kx * TP + col], acc);
-            s.X[e] = acc;
+        __syncthreads();                                   // every column done: A is dead
+        if (tid < C) {
+            const int j = tid;
+            const float s1 = s.bb[j] * s.eg[j], s2 = s.bb[j];
+#pragma unroll
+            for (int t = 0; t < C; ++t) {
+                T1[t * SC + j] = __float2bfloat16_rn(tc[t] * s1);
+                T2[t * SC + j] = __float2bfloat16_rn(tc[t] * s2);
+            }
         }
         __syncthreads();
-        for (int e = tid; e < I * 256; e += PREP_THREADS) {
-            const int J = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            const int row = I * 16 + r;
-            float acc = 0.f;
-            for (int kx = 0; kx <= r; ++kx) acc = fmaf(T[row * TP + I * 16 + kx], s.X[(J << 8) + (kx << 4) + c], acc);
-            T[row * TP + J * 16 + c] = -acc;
-        }
-        __syncthreads();
     }
-    // ---- T1 = T diag(b e^g), T2 = T diag(b) in bf16 (over A, which is dead)
-    for (int e = tid; e < C * C; e += PREP_THREADS) {
-        const int t = e >> 6, i = e & 63;
-        const float tv = T[t * TP + i];
-        T1[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i] * s.eg[i]);
-        T2[t * SC + i] = __float2bfloat16_rn(tv * s.bb[i]);
-    }
-    __syncthreads();
 
     // ---- W = T1 K, Up = T2 V (lower-triangular T: k-steps 0 .. rb)
     const int nc0 = ch * 64;
