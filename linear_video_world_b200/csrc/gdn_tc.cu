@@ -13,16 +13,18 @@
 //
 // Two kernels:
 //   prep   one CTA per (chunk, head), every chunk in parallel: Q, K, V of the chunk arrive
-//          by TMA as 128B-swizzled boxes; KK^T, QK^T, the blocked inversion for T (fp32),
-//          then W, Up, Op, Qt on mma.sync bf16 tensor cores; writes W, Up, Op, Qt, Kt (bf16)
-//          and gam (fp32) to the workspace.
+//          by TMA as 128B-swizzled boxes; KK^T, QK^T, T by forward substitution (fp32, one
+//          column per thread in registers), then W, Up, Op, Qt on mma.sync bf16 tensor cores;
+//          writes W, Qt, Kt, and Up, Op transposed (bf16), and gam (fp32) to the workspace.
 //   state  serial over the chunks of a head; the 128 state rows are split into 16-row blocks
-//          (rows of S evolve independently), four blocks per CTA, two CTAs per head. A
-//          block's state lives in registers as the accumulator fragments of the S update;
-//          each chunk does two dependent small GEMMs ([W;Qt] S^T, then U^T Kt) on mma.sync.
-//          The chunk operands (swizzled W/Qt/Kt boxes, the CTA's 64 columns of Up/Op, gam)
-//          stream in by TMA through a 3-stage mbarrier ring shared by the four blocks, two
-//          chunks ahead; waits are bounded (DEVERR_GDN_WAIT).
+//          (rows of S evolve independently), one warp per block, four per CTA, two CTAs per
+//          head. A warp keeps its rows of S in registers over all key columns, in the layout
+//          of m16n8k16 accumulator tiles, which is also the A-operand layout of the next
+//          product: per chunk S [Qt; W]^T, then S <- gam S + U Kt with U taken straight from
+//          the first product's accumulators, without a round trip through shared memory.
+//          A producer warp streams the chunk operands in by TMA through a 3-stage ring
+//          (stage release counted over the four state warps); waits are bounded
+//          (DEVERR_GDN_WAIT).
 // The serial chain is latency-bound (two dependent 64x16x128-class products per chunk), so
 // it uses register-resident warp MMAs rather than a TMEM round trip per dependent step.
 #include "hlta_internal.cuh"
@@ -35,11 +37,8 @@ namespace {
 
 constexpr int C = 64;             // chunk length
 constexpr int D = 128;            // head dim
-constexpr int SD = D + 8;         // padded smem row stride (elements) of [.][128] bf16 tiles
 constexpr int SC = C + 8;         // padded smem row stride of [.][64] bf16 tiles
 constexpr int AP = C + 4;         // fp32 row stride of A: 16-byte aligned rows
-constexpr int THREADS = 128;
-constexpr int RB = 16;            // state rows per CTA in the state pass
 
 using ptx::smem_u32;
 using ptx::sw128_off;
@@ -77,25 +76,12 @@ __device__ __forceinline__ void frag_a(uint32_t (&r)[4], const __nv_bfloat16 *ba
     ldsm_x4(r, smem_u32(base + (m0 + (q & 1) * 8 + rr) * ld + k0 + (q >> 1) * 8));
 }
 
-// B fragments of two adjacent n-tiles (k16 x n16) from a [N][K] row-major tile:
-// r[0], r[1] = n-tile n0, r[2], r[3] = n-tile n0 + 8
-__device__ __forceinline__ void frag_b_nk(uint32_t (&r)[4], const __nv_bfloat16 *base, int ld,
-                                          int n0, int k0, int lane)
-{
-    ldsm_x4(r, smem_u32(base + (n0 + (lane >> 4) * 8 + (lane & 7)) * ld + k0 + ((lane >> 3) & 1) * 8));
-}
-
-// The same four loaders on a [64][128] bf16 tile in the 128B-swizzled two-half layout
+// Fragment loaders on a [64][128] bf16 tile in the 128B-swizzled two-half layout
 // (byte offsets from ptx::sw128_off); every ldmatrix row address is one 16-byte chunk.
 __device__ __forceinline__ void frag_a_sw(uint32_t (&r)[4], const uint8_t *tile, int m0, int k0, int lane)
 {
     const int q = lane >> 3, rr = lane & 7;
     ldsm_x4(r, smem_u32(tile + sw128_off(m0 + (q & 1) * 8 + rr, k0 + (q >> 1) * 8, C)));
-}
-__device__ __forceinline__ void frag_a_t_sw(uint32_t (&r)[4], const uint8_t *tile, int m0, int k0, int lane)
-{
-    const int q = lane >> 3, rr = lane & 7;
-    ldsm_x4_t(r, smem_u32(tile + sw128_off(k0 + (q >> 1) * 8 + rr, m0 + (q & 1) * 8, C)));
 }
 __device__ __forceinline__ void frag_b_nk_sw(uint32_t (&r)[4], const uint8_t *tile, int n0, int k0, int lane)
 {
@@ -434,19 +420,37 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
     }
     __syncthreads();
 
-    // ---- write W, Up, Op, Qt, Kt (row-major [64][128] per chunk) and gam
+    // ---- write W, Qt, Kt (row-major [64 t][128] per chunk), Up and Op transposed
+    //      ([128 i][64 t] per chunk: the state pass reads them in its accumulator layout, state
+    //      row i by token t) and gam
     const long base = ((long)bh * nch + chunk) * C * D;
     uint4 *oW = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.W + base);
     uint4 *oU = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Up + base);
     uint4 *oO = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Op + base);
     uint4 *oQ = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Qt + base);
     uint4 *oK = reinterpret_cast<uint4 *>((__nv_bfloat16 *)ws.Kt + base);
+    for (int e = tid; e < D * (C / 8); e += PREP_THREADS) {
+        // lanes run over the state row i (consecutive 2-byte columns of the staged tiles),
+        // each gathering 8 consecutive tokens
+        const int i = e & (D - 1), t8 = e >> 7;
+        uint32_t up[4], op[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int t = t8 * 8 + 2 * u;
+            const uint16_t u0 = *reinterpret_cast<const uint16_t *>(s.V + sw128_off(t, i, C));
+            const uint16_t u1 = *reinterpret_cast<const uint16_t *>(s.V + sw128_off(t + 1, i, C));
+            const uint16_t o0 = *reinterpret_cast<const uint16_t *>(Op + sw128_off(t, i, C));
+            const uint16_t o1 = *reinterpret_cast<const uint16_t *>(Op + sw128_off(t + 1, i, C));
+            up[u] = (uint32_t)u0 | ((uint32_t)u1 << 16);
+            op[u] = (uint32_t)o0 | ((uint32_t)o1 << 16);
+        }
+        oU[i * (C / 8) + t8] = make_uint4(up[0], up[1], up[2], up[3]);
+        oO[i * (C / 8) + t8] = make_uint4(op[0], op[1], op[2], op[3]);
+    }
     for (int e = tid; e < C * (D / 8); e += PREP_THREADS) {
         const int t = e >> 4, c8 = e & 15;
         const uint32_t so = sw128_off(t, c8 * 8, C);
         oW[e] = *reinterpret_cast<const uint4 *>(W + so);
-        oU[e] = *reinterpret_cast<const uint4 *>(s.V + so);
-        oO[e] = *reinterpret_cast<const uint4 *>(Op + so);
         oQ[e] = *reinterpret_cast<const uint4 *>(s.Q + so);
         const float dk = s.ek[t];
         uint4 kv = *reinterpret_cast<const uint4 *>(s.K + so);
@@ -464,37 +468,44 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
 // -----------------------------------------------------------------------------------------
 // state pass
 // -----------------------------------------------------------------------------------------
-// Two CTAs per head; each CTA holds four 16-row blocks of the state (one group of four warps
-// per block) that share one ring of chunk operands, so a head occupies two SMs.
+// Two CTAs per head, four warps each; a warp owns 16 rows i of the state S (rows evolve
+// independently) and keeps them in registers as m16n8k16 accumulator tiles over all 128 key
+// columns j. Per chunk, with U, O, D laid out state row by token:
+//   D = S [W; Qt]^T   (A operand: S itself, repacked to bf16 pairs; B: the W and Qt tiles)
+//   O = Op^T + D_Qt,  U = Up^T - D_W
+//   S <- gam S + U Kt  (A operand: U, repacked straight from D's accumulator tiles; B: Kt)
+// An m16n8 accumulator tile holds rows (g, g+8) and column pairs (2t, 2t+1) of each lane,
+// which is exactly the A fragment of the next m16n8k16 product over those columns, so
+// neither S nor U goes through shared memory. The chunk operands (swizzled W, Qt, Kt tiles,
+// the CTA's 64 rows of Up^T and Op^T, gam) stream in by TMA through a 3-stage mbarrier ring,
+// two chunks ahead; outputs leave through a double-buffered shared staging tile.
 constexpr int NSTAGE = 3;                  // chunk operand buffers of the state pass
-constexpr int GROUPS = 4;                  // 16-row blocks per CTA
-constexpr int STATE_THREADS = GROUPS * THREADS;
-constexpr int CW = GROUPS * RB;            // state rows (= Up/Op columns) per CTA: 64
-constexpr uint32_t SLICE = C * CW * 2;     // the CTA's 64 columns of Up or Op: 8 KB
+constexpr int SWARPS = 4;                  // state warps per CTA, 16 state rows each
+constexpr int STATE_THREADS = (SWARPS + 1) * 32;   // plus one TMA producer warp
+constexpr int CW = SWARPS * 16;            // state rows per CTA: 64
+constexpr uint32_t SLICE = CW * C * 2;     // the CTA's rows of Up^T or Op^T: [64 i][64 t], 8 KB
 constexpr uint32_t STAGE_TX = 3 * SWT + 2 * SLICE + 16;
+constexpr int OSI = 16 + 8;                // staging row stride of a warp's [64 t][16 i] outputs
 
 struct StateBuf {
-    alignas(1024) uint8_t W[SWT];
+    alignas(1024) uint8_t W[SWT];          // W  [64 t][128 j], two 128B-swizzled halves
     alignas(1024) uint8_t Q[SWT];          // Qt
     alignas(1024) uint8_t K[SWT];          // Kt
-    alignas(128) __nv_bfloat16 U[C * CW];  // Up[:, c0:c0+64], row-major [64][64]
-    alignas(128) __nv_bfloat16 O[C * CW];  // Op[:, c0:c0+64]
+    alignas(1024) uint8_t U[SLICE];        // Up^T rows of this CTA [64 i][64 t], 128B swizzle
+    alignas(1024) uint8_t O[SLICE];        // Op^T rows of this CTA
     alignas(16) float gam[4];              // gam of the chunk (element 0)
-};
-struct StateGroup {
-    __nv_bfloat16 Sb[RB * SD];             // state slice as bf16 [i][j]
-    __nv_bfloat16 Ut[RB * SC];             // U^T slice [i][t]
 };
 struct StateSmem {
     StateBuf buf[NSTAGE];
-    StateGroup grp[GROUPS];
+    alignas(16) __nv_bfloat16 Ost[SWARPS][C * OSI];   // per warp: its outputs of a chunk, [t][i]
     alignas(8) uint64_t full[NSTAGE];
+    alignas(8) uint64_t empty[NSTAGE];     // every warp is done with the stage (count SWARPS)
     int abort_flag;
 };
 
 struct StateMaps {
-    CUtensorMap W, Q, K;                   // workspace [BHg*nch*64][128]: 64x64 swizzled boxes
-    CUtensorMap U, O;                      // workspace [BHg*nch*64][128]: 64 rows x 64 columns
+    CUtensorMap W, Q, K;                   // [BHg*nch*64][128]: 64x64 swizzled boxes
+    CUtensorMap U, O;                      // [BHg*nch*128][64]: 64x64 swizzled boxes
 };
 
 __device__ __forceinline__ void issue_chunk(StateSmem &s, const StateMaps &maps, const GdnWorkspace &ws,
@@ -502,21 +513,60 @@ __device__ __forceinline__ void issue_chunk(StateSmem &s, const StateMaps &maps,
 {
     StateBuf &bf = s.buf[c % NSTAGE];
     const uint32_t bar = smem_u32(&s.full[c % NSTAGE]);
-    const int row = (int)(((long)bh * nch + c) * C);
     ptx::mbar_expect_tx(bar, STAGE_TX);
+    const int row = (int)(((long)bh * nch + c) * C);
     for (int hf = 0; hf < 2; ++hf) {
         ptx::tma_load_2d(smem_u32(bf.W + hf * (SWT / 2)), &maps.W, hf * 64, row, bar);
         ptx::tma_load_2d(smem_u32(bf.Q + hf * (SWT / 2)), &maps.Q, hf * 64, row, bar);
         ptx::tma_load_2d(smem_u32(bf.K + hf * (SWT / 2)), &maps.K, hf * 64, row, bar);
     }
-    ptx::tma_load_2d(smem_u32(bf.U), &maps.U, c0, row, bar);
-    ptx::tma_load_2d(smem_u32(bf.O), &maps.O, c0, row, bar);
+    const int trow = (int)(((long)bh * nch + c) * D + c0);
+    ptx::tma_load_2d(smem_u32(bf.U), &maps.U, 0, trow, bar);
+    ptx::tma_load_2d(smem_u32(bf.O), &maps.O, 0, trow, bar);
     ptx::bulk_load(smem_u32(bf.gam), ws.gam + ((long)bh * nch + c) * 4, 16, bar);
 }
 
-__device__ __forceinline__ void group_sync(int g)
+__device__ __forceinline__ uint32_t pack_acc(float lo, float hi)
 {
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(THREADS) : "memory");
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// four 8x8 bf16 matrices from the accumulator-fragment layout (lane: row lane/4, column pair
+// lane%4) stored transposed; lanes 8k..8k+7 give the 16-byte row addresses of matrix k
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
+                 ::"r"(addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
+}
+
+// DQ[nt] = S Qt^T and DW[nt] = S W^T (nt < 8: tokens 8nt..8nt+7) for this warp's 16 rows, in
+// one pass over the key columns: each A fragment of S is packed to bf16 once for both
+__device__ __forceinline__ void state_times_tiles(float (&dq)[8][4], float (&dw)[8][4], const float (&st)[16][4],
+                                                  const uint8_t *qt, const uint8_t *wt, int lane)
+{
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[nt][e] = dw[nt][e] = 0.f;
+#pragma unroll
+    for (int kb = 0; kb < D / 16; ++kb) {
+        uint32_t a[4];
+        a[0] = pack_acc(st[2 * kb][0], st[2 * kb][1]);
+        a[1] = pack_acc(st[2 * kb][2], st[2 * kb][3]);
+        a[2] = pack_acc(st[2 * kb + 1][0], st[2 * kb + 1][1]);
+        a[3] = pack_acc(st[2 * kb + 1][2], st[2 * kb + 1][3]);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+            uint32_t bq[4], bw[4];
+            frag_b_nk_sw(bq, qt, np * 16, kb * 16, lane);     // tile rows = tokens (n), cols = j (k)
+            frag_b_nk_sw(bw, wt, np * 16, kb * 16, lane);
+            mma16816(dq[2 * np], a, bq[0], bq[1]);
+            mma16816(dq[2 * np + 1], a, bq[2], bq[3]);
+            mma16816(dw[2 * np], a, bw[0], bw[1]);
+            mma16816(dw[2 * np + 1], a, bw[2], bw[3]);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(STATE_THREADS, 1)
@@ -527,151 +577,146 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
     const int bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long nch = gdn_num_chunks(p.L, C);
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int g = tid / THREADS, warp = (tid / 32) % 4;    // row-block group, warp in group
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g8 = lane >> 2, tg = lane & 3;
     const int c0 = blockIdx.x * CW;                        // first state row of this CTA
-    const int i0 = c0 + g * RB;                            // first state row of this group
-    StateGroup &sg = s.grp[g];
+    const int r0 = warp * 16;                              // first row of this warp in the CTA
     __nv_bfloat16 *o = (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D;
 
     if (tid == 0) {
+        for (int i = 0; i < NSTAGE; ++i) {
+            ptx::mbar_init(smem_u32(&s.full[i]), 1);
+            ptx::mbar_init(smem_u32(&s.empty[i]), SWARPS);
+        }
         s.abort_flag = 0;
-        for (int st = 0; st < NSTAGE; ++st) ptx::mbar_init(smem_u32(&s.full[st]), 1);
         ptx::mbar_init_fence();
     }
-    // state fragments: this warp owns key columns j in [32w, 32w+32) of S^T = D[m=j][n=i]
-    float st[2][2][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
-                const int i = nt * 8 + 2 * tg + (e & 1);
-                st[mt][nt][e] = p.S0 ? p.S0[((long)bh * D + i0 + i) * D + j] : 0.f;
-                sg.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
-            }
-    __syncthreads();
-    if (tid == 0)
-        for (long c = 0; c < NSTAGE - 1 && c < nch; ++c) issue_chunk(s, maps, ws, bh, nch, c, c0);
-
-    bool ok = true;
-    long c_fail = 0;
-    for (long c = 0; c < nch; ++c) {
-        StateBuf &cur = s.buf[c % NSTAGE];
-        const bool landed = ptx::mbar_wait(smem_u32(&s.full[c % NSTAGE]), (uint32_t)(c / NSTAGE) & 1u,
-                                           (volatile int *)&s.abort_flag, p.err, DEVERR_GDN_WAIT);
-        // chunk c has landed for every thread; every group's Sb holds its incoming state
-        if (!__syncthreads_and(landed)) { ok = false; c_fail = c; break; }
-        // the stage of chunk c-1 is free again (every thread passed the barrier above)
-        if (tid == 0 && c + NSTAGE - 1 < nch) issue_chunk(s, maps, ws, bh, nch, c + NSTAGE - 1, c0);
-        const float gam = cur.gam[0];
-        const long t0 = c * C;
-
-        // GEMM 1: rows [W; Qt] (warps 0-1 of the group: W rows, warps 2-3: Qt rows) times S^T
-        {
-            const uint8_t *Am = warp < 2 ? cur.W : cur.Q;
-            const int mb = (warp & 1) * 32;
-            float acc[2][2][4];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t bsf[4];
-                frag_b_nk(bsf, sg.Sb, SD, 0, ks * 16, lane);
-#pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    uint32_t a[4];
-                    frag_a_sw(a, Am, mb + mt * 16, ks * 16, lane);
-                    mma16816(acc[mt][0], a, bsf[0], bsf[1]);
-                    mma16816(acc[mt][1], a, bsf[2], bsf[3]);
+    volatile int *abort_flag = (volatile int *)&s.abort_flag;
+    if (warp == SWARPS) {
+        // ------------------------------ TMA producer --------------------------------------
+        // chunk c goes into stage c % NSTAGE once every state warp released chunk c - NSTAGE
+        __syncthreads();
+        if (lane == 0) {
+            long c = 0;
+            for (; c < nch; ++c) {
+                if (c >= NSTAGE) {
+                    const uint32_t eb = smem_u32(&s.empty[c % NSTAGE]);
+                    const uint32_t ep = (uint32_t)((c - NSTAGE) / NSTAGE) & 1u;
+                    if (!(ptx::mbar_try(eb, ep) || ptx::mbar_wait(eb, ep, abort_flag, p.err, DEVERR_GDN_WAIT))) break;
                 }
+                issue_chunk(s, maps, ws, bh, nch, c, c0);
             }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int t = mb + mt * 16 + g8 + hh * 8;
-                        const int i = nt * 8 + 2 * tg;
-                        const float a0 = acc[mt][nt][2 * hh], a1 = acc[mt][nt][2 * hh + 1];
-                        if (warp < 2) {
-                            const float u0 = __bfloat162float(cur.U[t * CW + g * RB + i]) - a0;
-                            const float u1 = __bfloat162float(cur.U[t * CW + g * RB + i + 1]) - a1;
-                            sg.Ut[i * SC + t] = __float2bfloat16_rn(u0);
-                            sg.Ut[(i + 1) * SC + t] = __float2bfloat16_rn(u1);
-                        } else if (t0 + t < p.L) {
-                            const float v0 = __bfloat162float(cur.O[t * CW + g * RB + i]) + a0;
-                            const float v1 = __bfloat162float(cur.O[t * CW + g * RB + i + 1]) + a1;
-                            *reinterpret_cast<uint32_t *>(o + (t0 + t) * D + i0 + i) = pack2(v0, v1);
-                        }
-                    }
-        }
-        group_sync(g);                         // this group's Ut is complete
-
-        // GEMM 2: S^T <- gam S^T + Kt^T U   (D[m=j][n=i] = sum_t Kt[t][j] U[t][i])
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) st[mt][nt][e] *= gam;
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) {
-            uint32_t bu[4];
-            frag_b_nk(bu, sg.Ut, SC, 0, ks * 16, lane);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                uint32_t a[4];
-                frag_a_t_sw(a, cur.K, warp * 32 + mt * 16, ks * 16, lane);
-                mma16816(st[mt][0], a, bu[0], bu[1]);
-                mma16816(st[mt][1], a, bu[2], bu[3]);
-            }
-        }
-        // bf16 copy of the new state for the next chunk's GEMM 1 (made visible by the
-        // barrier at the top of the loop)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
-                    const int i = nt * 8 + 2 * tg + (e & 1);
-                    sg.Sb[i * SD + j] = __float2bfloat16_rn(st[mt][nt][e]);
+            if (*abort_flag) {
+                // a bounded wait expired somewhere: let the copies this CTA issued land before
+                // it exits (the last NSTAGE chunks issued, each on its own stage and phase)
+                const long long tw = clock64();
+                for (long cc = c - 1; cc >= 0 && cc >= c - NSTAGE; --cc) {
+                    const uint32_t bar = smem_u32(&s.full[cc % NSTAGE]);
+                    while (!ptx::mbar_try(bar, (uint32_t)(cc / NSTAGE) & 1u) && clock64() - tw < (1LL << 31)) {}
                 }
-    }
-    if (!ok) {
-        // a bounded wait expired: let the copies this CTA issued and never consumed land
-        // before it exits (chunks c .. issued-1, each on its own stage and phase)
-        if (tid == 0) {
-            const long long tw = clock64();
-            for (long cc = c_fail; cc < c_fail + NSTAGE - 1 && cc < nch; ++cc) {
-                const uint32_t bar = smem_u32(&s.full[cc % NSTAGE]);
-                while (!ptx::mbar_try(bar, (uint32_t)(cc / NSTAGE) & 1u) && clock64() - tw < (1LL << 31)) {}
             }
         }
         return;
     }
-    if (p.S_out) {
+    // the state rows of this warp: st[nt] holds (i = g8, g8 + 8) x (j = 8 nt + 2 tg, +1)
+    float st[16][4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+    for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+        for (int e = 0; e < 4; ++e) {
+            const int i = c0 + r0 + g8 + (e >> 1) * 8;
+            const int j = nt * 8 + 2 * tg + (e & 1);
+            st[nt][e] = p.S0 ? p.S0[((long)bh * D + i) * D + j] : 0.f;
+        }
+    __syncthreads();
+
+    // this warp's outputs of a chunk: staged transposed ([t][i], stmatrix) and written out as
+    // 32-byte runs of its 16 state rows per token
+    __nv_bfloat16 *stage = s.Ost[warp];
+    const uint32_t stage_a = smem_u32(stage);
+
+    for (long c = 0; c < nch; ++c) {
+        StateBuf &cur = s.buf[c % NSTAGE];
+        const uint32_t fb = smem_u32(&s.full[c % NSTAGE]), fp = (uint32_t)(c / NSTAGE) & 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_try(fb, fp) || ptx::mbar_wait(fb, fp, abort_flag, p.err, DEVERR_GDN_WAIT)))
+            return;                                        // the producer waits for its copies
+        const float gam = cur.gam[0];
+        const long t0 = c * C;
+        float dq[8][4], dw[8][4];
+        state_times_tiles(dq, dw, st, cur.Q, cur.W, lane);
+        // O = Op^T + S Qt^T (old S)
+        {
+            uint32_t ov[8][2];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = warp * 32 + mt * 16 + g8 + (e >> 1) * 8;
-                    const int i = nt * 8 + 2 * tg + (e & 1);
-                    p.S_out[((long)bh * D + i0 + i) * D + j] = st[mt][nt][e];
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int il = r0 + g8 + hh * 8, t = nt * 8 + 2 * tg;
+                    const float2 of = __bfloat1622float2(
+                        *reinterpret_cast<const __nv_bfloat162 *>(cur.O + ptx::sw128_off(il, t, CW)));
+                    ov[nt][hh] = pack_acc(of.x + dq[nt][2 * hh], of.y + dq[nt][2 * hh + 1]);
                 }
+            __syncwarp();                                  // the previous chunk's run reads are done
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                // matrices (rows i 0-7 | 8-15) x (tokens 16np .. +7 | +8 .. +15)
+                const int k = lane >> 3, r = lane & 7;
+                const int t = np * 16 + (k >> 1) * 8 + r, ib = (k & 1) * 8;
+                stsm_x4_t(stage_a + (uint32_t)(t * OSI + ib) * 2u, ov[2 * np][0], ov[2 * np][1],
+                          ov[2 * np + 1][0], ov[2 * np + 1][1]);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int t = u * 32 + lane;
+                if (t0 + t < p.L) {
+                    const uint4 *srow = reinterpret_cast<const uint4 *>(stage + t * OSI);
+                    uint4 *drow = reinterpret_cast<uint4 *>(o + (t0 + t) * D + c0 + r0);
+                    drow[0] = srow[0];
+                    drow[1] = srow[1];
+                }
+            }
+        }
+        // U = Up^T - S W^T, as the A fragments of the update product
+        uint32_t ua[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int il = r0 + g8 + hh * 8, t = nt * 8 + 2 * tg;
+                const float2 uf = __bfloat1622float2(
+                    *reinterpret_cast<const __nv_bfloat162 *>(cur.U + ptx::sw128_off(il, t, CW)));
+                ua[nt >> 1][(nt & 1) * 2 + hh] = pack_acc(uf.x - dw[nt][2 * hh], uf.y - dw[nt][2 * hh + 1]);
+            }
+        // S <- gam S + U Kt
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st[nt][e] *= gam;
+#pragma unroll
+        for (int kb = 0; kb < C / 16; ++kb) {
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bk[4];
+                frag_b_kn_sw(bk, cur.K, kb * 16, np * 16, lane);      // Kt rows = tokens (k), cols = j (n)
+                mma16816(st[2 * np], ua[kb], bk[0], bk[1]);
+                mma16816(st[2 * np + 1], ua[kb], bk[2], bk[3]);
+            }
+        }
+        // this warp no longer reads the stage (its shared loads have completed: their values
+        // fed the products above)
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(smem_u32(&s.empty[c % NSTAGE]));
     }
+    if (p.S_out)
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = c0 + r0 + g8 + (e >> 1) * 8;
+                const int j = nt * 8 + 2 * tg + (e & 1);
+                p.S_out[((long)bh * D + i) * D + j] = st[nt][e];
+            }
 }
 
 }  // namespace
@@ -695,8 +740,9 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     if ((e = make_tmap_2d_bf16(&sm.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&sm.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&sm.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows, D, CW, C, false)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows, D, CW, C, false)) != cudaSuccess) return e;
+    // Up^T and Op^T: [BHg*nch*128][64] views, boxes of 64 state rows x 64 tokens, swizzled
+    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
     const size_t smem_prep = sizeof(PrepSmem) + 1024;
     const size_t smem_state = sizeof(StateSmem) + 1024;
     e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep);

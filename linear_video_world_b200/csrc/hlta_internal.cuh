@@ -52,7 +52,8 @@ struct GdnArgs {
 //   W  = T diag(b e^g) K,   Up = T diag(b) V,   Op = P Up,
 //   Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K        each [C][d]
 //   gam = e^{g_C}                               one float per chunk, in a 16-byte slot
-// laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks][4].
+// laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks][4]; the bf16
+// path stores Up and Op of a chunk transposed, [d][C] (state row by token).
 struct GdnWorkspace {
     void *W, *Up, *Op, *Qt, *Kt;
     float *gam;
