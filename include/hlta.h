@@ -168,9 +168,10 @@ size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk
  * (each branch writes its own head range of o, in place).
  * q, k, v, o: [B, H, T*N, d] with H = Hs + Hd + Hg; a, b: [B, Hg, T*N] float32.
  * S0 / S_out: [B, Hg, d, d] float32 or NULL (as hlta_gdn_chunk_fwd).
- * The GDN branch runs on a library-owned second stream ordered after `stream` by events,
- * so it overlaps the softmax branches; the call still completes, in stream order, on
- * `stream` (later work on `stream` sees every output).
+ * The GDN branch runs on a library-owned stream of the highest priority and the DSWA branch
+ * (when SWA heads are present too) on a second library-owned stream, both ordered after
+ * `stream` by an event, so the branches overlap; the call still completes, in stream order,
+ * on `stream` (later work on `stream` sees every output).
  */
 hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v,
                             const float *a, const float *b, void *o,
@@ -225,10 +226,11 @@ hlta_status hlta_stream_destroy(hlta_stream_t c);
 /*
  * Profiling hook for hlta_hybrid_fwd (measurement, not needed for results). `events` is NULL
  * (off) or an array of 5 cudaEvent_t created by the caller on the current device. While set,
- * each hlta_hybrid_fwd call records events[0] before its SWA kernel, events[1] between the
- * SWA and DSWA kernels and events[2] after the DSWA kernel (all on the caller's stream),
- * events[3] before and events[4] after the GDN kernels (on the GDN stream). The array is
- * copied; the setting is process-wide and stays until changed.
+ * each hlta_hybrid_fwd call records events[0] where the branches fork (on the caller's stream,
+ * before any branch kernel), events[1] after the SWA kernel (caller's stream), events[2] after
+ * the DSWA kernel (on the stream it ran on), events[3] before and events[4] after the GDN
+ * kernels (on the GDN stream). The array is copied; the setting is process-wide and stays
+ * until changed.
  */
 hlta_status hlta_set_profile_events(void *const *events);
 

@@ -39,8 +39,9 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 struct DeviceCtx {
     bool ready = false;
     unsigned int *err = nullptr;
-    cudaStream_t aux = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaStream_t aux = nullptr;     // GDN branch (highest priority)
+    cudaStream_t aux2 = nullptr;    // DSWA branch of the hybrid (default priority)
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
 };
 constexpr int kMaxDevices = 64;
 DeviceCtx g_ctx[kMaxDevices];
@@ -77,6 +78,12 @@ hlta_status device_ctx(DeviceCtx **out)
         if ((e = cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming)) != cudaSuccess)
             return cuda_fail(e, "cudaEventCreate");
         if ((e = cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventCreate");
+        // the hybrid's DSWA launch runs beside its SWA launch, so neither waits for the
+        // other's last wave of CTAs
+        if ((e = cudaStreamCreateWithPriority(&c.aux2, cudaStreamNonBlocking, least)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithPriority");
+        if ((e = cudaEventCreateWithFlags(&c.join2, cudaEventDisableTiming)) != cudaSuccess)
             return cuda_fail(e, "cudaEventCreate");
         c.ready = true;
     }
@@ -337,9 +344,15 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     std::lock_guard<std::mutex> lk(g_fork_mu);
-    // GDN heads on the auxiliary stream, ordered after everything already on `s`
-    if (Hg) {
+    // the branches other than SWA run on library streams ordered after everything already
+    // on `s` (one fork event), and `s` waits for them at the end
+    const bool split_d = Hd && Hs;
+    if (Hg || split_d) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    prof_record(0, s);
+    // GDN heads on the high-priority auxiliary stream
+    if (Hg) {
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         GdnArgs g = {};
         g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o; g.raw = raw; g.raw_c = raw_c;
@@ -354,19 +367,25 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
             return st;
         }
     }
-    // the softmax branches run on `s` while the GDN branch runs on the auxiliary stream
-    prof_record(0, s);
-    if (Hs) {
+    // DSWA on the second library stream (beside SWA) when both softmax branches are present
+    if (Hd) {
+        cudaStream_t sd = split_d ? ctx->aux2 : s;
+        if (split_d && (e = cudaStreamWaitEvent(sd, ctx->fork, 0)) != cudaSuccess)
+            st = cuda_fail(e, "cudaStreamWaitEvent");
+        if (st == HLTA_OK) {
+            AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
+            st = run_attn(a2, dt, sd);
+        }
+        prof_record(2, sd);
+        if (split_d) cudaEventRecord(ctx->join2, sd);
+    }
+    if (Hs && st == HLTA_OK) {
         AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
         st = run_attn(a1, dt, s);
     }
     prof_record(1, s);
-    if (Hd && st == HLTA_OK) {
-        AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
-        st = run_attn(a2, dt, s);
-    }
-    prof_record(2, s);
-    // join: work enqueued on `s` after this call sees the GDN outputs too
+    // join: work enqueued on `s` after this call sees every branch's outputs
+    if (split_d) cudaStreamWaitEvent(s, ctx->join2, 0);
     if (Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     return st;
 }
@@ -460,11 +479,16 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
     const int H = c->Hs + c->Hd + c->Hg;
     const int f = c->frames;
     const size_t el = c->dt == HLTA_BF16 ? 2 : 4;
-    // the fork/join events are shared per device: hold them until the join is enqueued
+    // the fork/join events are shared per device: hold them until the joins are enqueued.
+    // GDN runs on the high-priority library stream, the DSWA branch (ring append and
+    // attention) on the second library stream when SWA heads are present too
     std::unique_lock<std::mutex> lk(g_fork_mu, std::defer_lock);
-    if (c->Hg) {
+    const bool split_d = c->Hd && c->Hs;
+    if (c->Hg || split_d) {
         lk.lock();
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    if (c->Hg) {
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         GdnArgs g = {};
         g.q = q_new; g.k = k_new; g.v = v_new; g.a = a_new; g.b = b_new; g.o = o_new;
@@ -481,8 +505,14 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
     struct Branch { int h0, Hbr, slots, w, r; void *rk, *rv; } br[2] = {
         {0, c->Hs, c->slots_s, c->w_swa, 1, c->ks, c->vs},
         {c->Hs, c->Hd, c->slots_d, c->w_dswa, c->r, c->kd, c->vd}};
-    for (const Branch &x : br) {
+    if (split_d && (e = cudaStreamWaitEvent(ctx->aux2, ctx->fork, 0)) != cudaSuccess) {
+        cudaStreamWaitEvent(s, ctx->join, 0);
+        return cuda_fail(e, "cudaStreamWaitEvent");
+    }
+    for (int bi = 1; bi >= 0; --bi) {                  // DSWA first: it goes to its own stream
+        const Branch &x = br[bi];
         if (!x.Hbr) continue;
+        cudaStream_t s = (bi == 1 && split_d) ? ctx->aux2 : (cudaStream_t)stream;
         const int slot = f % x.slots;
         if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rk, x.slots, slot, s)) != cudaSuccess ||
             (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rv, x.slots, slot, s)) != cudaSuccess) {
@@ -498,7 +528,11 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         a.err = ctx->err;
         if ((st = run_attn(a, c->dt, s)) != HLTA_OK) break;
     }
-    // join the GDN branch after the softmax branches were enqueued, so the two overlap
+    // join the other branches after the softmax launches were enqueued, so they overlap
+    if (split_d) {
+        cudaEventRecord(ctx->join2, ctx->aux2);
+        cudaStreamWaitEvent(s, ctx->join2, 0);
+    }
     if (c->Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     if (st != HLTA_OK) return st;
     c->frames = f + 1;
