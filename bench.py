@@ -130,10 +130,30 @@ def measure_stream(h, torch, dev, warm: int = 24, steps: int = 40) -> dict:
     st.close()
     ms = e0.elapsed_time(e1) / steps
     flop = stream_step_flop(sw, warm + steps)
+    # the same rollout advanced 4 frames per call (hlta_stream_step_frames)
+    F = 4
+    big = {n: x[n].to(dev) for n in "qkvab"}          # [B, H, 4N, d], [B, Hg, 4N]
+    o4 = torch.empty_like(big["q"])
+    st4 = h.Stream(sw.B, sw.Hs, sw.Hd, sw.Hg, sw.N, sw.d, sw.w_swa, sw.w_dswa, sw.r, sw.chunk,
+                   max_step_frames=F)
+    for _ in range(warm // F):
+        st4.step_frames(big["q"], big["k"], big["v"], big["a"], big["b"], F, out=o4)
+    torch.cuda.synchronize()
+    e0.record()
+    calls = steps // F
+    for _ in range(calls):
+        st4.step_frames(big["q"], big["k"], big["v"], big["a"], big["b"], F, out=o4)
+    e1.record()
+    torch.cuda.synchronize()
+    st4.close()
+    ms4 = e0.elapsed_time(e1) / (calls * F)
     return {"workload": f"{sw.name}: B={sw.B} new frame N={sw.N} heads {sw.Hs}/{sw.Hd}/{sw.Hg} "
                         f"SWA w={sw.w_swa} DSWA w={sw.w_dswa} r={sw.r}; steady state (frame >= {warm})",
             "ms_per_step": ms, "tokens_per_s": sw.B * sw.N / (ms / 1e3),
-            "softmax_tflops": flop / (ms / 1e3) / 1e12, "launches_per_step": 8}
+            "softmax_tflops": flop / (ms / 1e3) / 1e12, "launches_per_step": 8,
+            "four_frames_per_call": {"ms_per_frame": ms4, "tokens_per_s": sw.B * sw.N / (ms4 / 1e3),
+                                     "note": "hlta_stream_step_frames with 4 frames per rollout "
+                                             "per call, same rollout and steady state"}}
 
 
 def measure_raw(h, torch, dev, wl, hi, steps: int) -> dict:

@@ -210,11 +210,29 @@ hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg
                                int d, int w_swa, int w_dswa, int r, int chunk, float scale,
                                hlta_dtype dt, const float *S0);
 
+/* hlta_stream_create for steps that append up to max_step_frames frames per rollout at once
+ * (hlta_stream_step_frames): the rings keep w_swa - 1 (SWA) and r*(w_dswa-1) (DSWA) earlier
+ * frames plus max_step_frames new ones, and the GDN workspace covers max_step_frames * N
+ * tokens. max_step_frames in [1, 4096]; hlta_stream_create is this call with 1. */
+hlta_status hlta_stream_create_ex(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N,
+                                  int d, int w_swa, int w_dswa, int r, int chunk, float scale,
+                                  int max_step_frames, hlta_dtype dt, const float *S0);
+
 /* One step. q_new, k_new, v_new, o_new: [B, H, N, d] device; a_new, b_new: [B, Hg, N]
  * float32 device. Appends the new K/V to the rings, advances the frame counter. */
 hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_new,
                              const void *v_new, const float *a_new, const float *b_new,
                              void *o_new, void *stream);
+
+/* F frames per rollout in one step (a rollout of F frames whose inputs are all known, e.g. the
+ * conditioning frames): q, k, v, o: [B, H, F*N, d] device; a, b: [B, Hg, F*N] float32. The
+ * result equals F successive hlta_stream_step calls on the frame slices (up to rounding): the
+ * new frames attend to each other exactly as to cached ones (block-causal windows), and the
+ * GDN state advances over the F*N tokens. 1 <= F <= the cache's max_step_frames, else
+ * HLTA_ERR_INVALID_ARG. */
+hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q, const void *k,
+                                    const void *v, const float *a, const float *b, void *o,
+                                    int F, void *stream);
 
 /* Device pointer to the carried GDN state [B, Hg, d, d] (owned by the cache) and the
  * number of frames appended so far. */

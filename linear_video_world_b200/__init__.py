@@ -50,7 +50,9 @@ def _load() -> ctypes.CDLL:
         "hlta_hybrid_fwd_raw": (I, [P, P, P, P, P, F, P, P, P, I, I, I, I, I, I, I, I, I, I, I,
                                     F, P, Z, I, P]),
         "hlta_stream_create": (I, [ctypes.POINTER(P), I, I, I, I, I, I, I, I, I, I, F, I, P]),
+        "hlta_stream_create_ex": (I, [ctypes.POINTER(P), I, I, I, I, I, I, I, I, I, I, F, I, I, P]),
         "hlta_stream_step": (I, [P, P, P, P, P, P, P, P]),
+        "hlta_stream_step_frames": (I, [P, P, P, P, P, P, P, I, P]),
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
@@ -272,12 +274,13 @@ class Stream:
     """Streaming cache (hlta_stream_create / _step / _state / _destroy)."""
 
     def __init__(self, B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk=64, scale=0.0,
-                 dtype=None, S0=None):
+                 dtype=None, S0=None, max_step_frames=1):
         import torch
         dt = HLTA_BF16 if dtype in (None, torch.bfloat16) else HLTA_FP32
         self._h = ctypes.c_void_p()
-        _check(_lib.hlta_stream_create(ctypes.byref(self._h), B, Hs, Hd, Hg, N, d, w_swa,
-                                       w_dswa, r, chunk, float(scale), dt, _p(S0)))
+        _check(_lib.hlta_stream_create_ex(ctypes.byref(self._h), B, Hs, Hd, Hg, N, d, w_swa,
+                                          w_dswa, r, chunk, float(scale), int(max_step_frames),
+                                          dt, _p(S0)))
         self.B, self.H, self.Hg, self.N, self.d = B, Hs + Hd + Hg, Hg, N, d
 
     def step(self, q, k, v, a, b, out=None, stream=None):
@@ -285,6 +288,14 @@ class Stream:
         o = torch.empty_like(q) if out is None else out
         _check(_lib.hlta_stream_step(self._h, _p(q), _p(k), _p(v), _p(a), _p(b), _p(o),
                                      _stream(stream)))
+        return o
+
+    def step_frames(self, q, k, v, a, b, frames, out=None, stream=None):
+        """Append `frames` frames per rollout at once (inputs [B, H, frames*N, d])."""
+        import torch
+        o = torch.empty_like(q) if out is None else out
+        _check(_lib.hlta_stream_step_frames(self._h, _p(q), _p(k), _p(v), _p(a), _p(b), _p(o),
+                                            int(frames), _stream(stream)))
         return o
 
     def state(self):

@@ -231,10 +231,12 @@ struct hlta_stream {
     int B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk;
     float scale;
     hlta_dtype dt;
-    int slots_s, slots_d;     // ring slots: SWA w_swa frames, DSWA r*(w_dswa-1)+1 frames
+    int max_frames;           // frames one step may append
+    int slots_s, slots_d;     // ring slots: SWA w_swa-1, DSWA r*(w_dswa-1) earlier frames plus
+                              // max_frames new ones
     void *ks, *vs, *kd, *vd;  // rings [B][Hs][slots_s][N][d], [B][Hd][slots_d][N][d]
     float *S;                 // [B][Hg][d][d]
-    void *ws;                 // GDN workspace for N tokens
+    void *ws;                 // GDN workspace for max_frames * N tokens
     size_t ws_bytes;
     int frames;
 };
@@ -415,10 +417,19 @@ hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg
                                int w_swa, int w_dswa, int r, int chunk, float scale,
                                hlta_dtype dt, const float *S0)
 {
+    return hlta_stream_create_ex(out, B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk, scale, 1, dt, S0);
+}
+
+hlta_status hlta_stream_create_ex(hlta_stream_t *out, int B, int Hs, int Hd, int Hg, int N, int d,
+                                  int w_swa, int w_dswa, int r, int chunk, float scale,
+                                  int max_step_frames, hlta_dtype dt, const float *S0)
+{
     hlta_status st;
     if (!out) return fail(HLTA_ERR_INVALID_ARG, "null output handle");
     *out = nullptr;
     if (B < 1 || Hs < 0 || Hd < 0 || Hg < 0 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape");
+    if (max_step_frames < 1 || max_step_frames > 4096 || (long)max_step_frames * N > (1L << 30))
+        return fail(HLTA_ERR_INVALID_ARG, "max_step_frames must be in [1, 4096] (got %d)", max_step_frames);
     if ((st = check_dtype_d(dt, d)) != HLTA_OK) return st;
     if (Hs && (st = check_window(w_swa, 1)) != HLTA_OK) return st;
     if (Hd && (st = check_window(w_dswa, r)) != HLTA_OK) return st;
@@ -432,12 +443,13 @@ hlta_status hlta_stream_create(hlta_stream_t *out, int B, int Hs, int Hd, int Hg
     c->B = B; c->Hs = Hs; c->Hd = Hd; c->Hg = Hg; c->N = N; c->d = d;
     c->w_swa = w_swa; c->w_dswa = w_dswa; c->r = r; c->chunk = chunk; c->dt = dt;
     c->scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
-    c->slots_s = Hs ? w_swa : 0;
-    c->slots_d = Hd ? r * (w_dswa - 1) + 1 : 0;
+    c->max_frames = max_step_frames;
+    c->slots_s = Hs ? w_swa - 1 + max_step_frames : 0;
+    c->slots_d = Hd ? r * (w_dswa - 1) + max_step_frames : 0;
     const size_t el = dt == HLTA_BF16 ? 2 : 4;
     const size_t frame = (size_t)N * d * el;
     size_t bs = (size_t)B * Hs * c->slots_s * frame, bd = (size_t)B * Hd * c->slots_d * frame;
-    c->ws_bytes = Hg ? gdn_workspace_bytes((long)B * Hg, N, d, chunk, dt == HLTA_BF16) : 0;
+    c->ws_bytes = Hg ? gdn_workspace_bytes((long)B * Hg, (long)max_step_frames * N, d, chunk, dt == HLTA_BF16) : 0;
     cudaError_t e = cudaSuccess;
     if (bs && e == cudaSuccess) e = cudaMalloc(&c->ks, bs);
     if (bs && e == cudaSuccess) e = cudaMalloc(&c->vs, bs);
@@ -462,7 +474,16 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
                              const void *v_new, const float *a_new, const float *b_new,
                              void *o_new, void *stream)
 {
+    return hlta_stream_step_frames(c, q_new, k_new, v_new, a_new, b_new, o_new, 1, stream);
+}
+
+hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const void *k_new,
+                                    const void *v_new, const float *a_new, const float *b_new,
+                                    void *o_new, int F, void *stream)
+{
     if (!c) return fail(HLTA_ERR_INVALID_ARG, "null cache");
+    if (F < 1 || F > c->max_frames)
+        return fail(HLTA_ERR_INVALID_ARG, "frames per step must be in [1, %d] (got %d)", c->max_frames, F);
     if (!q_new || !k_new || !v_new || !o_new) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
     if (c->Hg && (!a_new || !b_new)) return fail(HLTA_ERR_INVALID_ARG, "null gate pointer");
     if (!aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(o_new) ||
@@ -492,7 +513,7 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         GdnArgs g = {};
         g.q = q_new; g.k = k_new; g.v = v_new; g.a = a_new; g.b = b_new; g.o = o_new;
-        g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = c->N; g.d = c->d;
+        g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = (long)F * c->N; g.d = c->d;
         g.chunk = c->chunk; g.S0 = c->S; g.S_out = c->S; g.ws = c->ws; g.ws_bytes = c->ws_bytes;
         g.err = ctx->err;
         st = run_gdn(g, c->dt, ctx->aux);
@@ -513,16 +534,15 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
         const Branch &x = br[bi];
         if (!x.Hbr) continue;
         cudaStream_t s = (bi == 1 && split_d) ? ctx->aux2 : (cudaStream_t)stream;
-        const int slot = f % x.slots;
-        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rk, x.slots, slot, s)) != cudaSuccess ||
-            (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, x.rv, x.slots, slot, s)) != cudaSuccess) {
+        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rk, x.slots, f, s)) != cudaSuccess ||
+            (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rv, x.slots, f, s)) != cudaSuccess) {
             st = cuda_fail(e, "ring append");
             break;
         }
         AttnArgs a;
         a.q = q_new; a.k = x.rk; a.v = x.rv; a.o = o_new;
         a.B = c->B; a.Hbr = x.Hbr;
-        a.q_Htot = H; a.q_h0 = x.h0; a.q_rows = c->N;
+        a.q_Htot = H; a.q_h0 = x.h0; a.q_rows = (long)F * c->N;
         a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
         a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.scale = c->scale;
         a.err = ctx->err;
@@ -535,7 +555,7 @@ hlta_status hlta_stream_step(hlta_stream_t c, const void *q_new, const void *k_n
     }
     if (c->Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     if (st != HLTA_OK) return st;
-    c->frames = f + 1;
+    c->frames = f + F;
     return HLTA_OK;
 }
 

@@ -77,9 +77,8 @@ cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
-cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N,
-                               int d, size_t elem, void *ring, int slots, int slot,
-                               cudaStream_t s);
+cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,
+                               size_t elem, int F, void *ring, int slots, int f0, cudaStream_t s);
 
 // Device error word: kernels OR a code into it when a bounded wait expires.
 enum : unsigned int {

@@ -75,6 +75,16 @@ def test_raw_entry_points_validate_decay_constant_on_host(lib):
                                       1 << 30, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
 
 
+def test_stream_create_ex_validates_frames_per_step(lib):
+    import linear_video_world_b200 as h
+    out = ctypes.c_void_p()
+    for m in (0, -1, 5000):
+        assert lib.hlta_stream_create_ex(ctypes.byref(out), 1, 1, 1, 1, 16, 128, 3, 4, 6, 64, 0.0,
+                                         m, h.HLTA_BF16, None) == h.HLTA_ERR_INVALID_ARG
+        assert not out.value
+    assert lib.hlta_stream_step_frames(None, None, None, None, None, None, None, 1, None) == h.HLTA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(lib):
     import linear_video_world_b200 as h
     # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16 plus a 16-byte slot per chunk

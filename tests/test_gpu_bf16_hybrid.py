@@ -112,3 +112,43 @@ def test_stream_steps_equal_hybrid_bf16(h, orc):
     assert maxabs(o, o_ref) <= TOL
     assert maxabs(st.state_tensor(), S_ref) <= TOL
     st.close()
+
+
+@pytest.mark.parametrize("groups", [(3, 1, 4, 2, 4), (1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1), (4, 4, 4, 2)])
+def test_stream_multi_frame_steps_equal_hybrid_bf16(h, orc, groups):
+    """Steps appending several frames per rollout at once (ragged group sizes, up to the
+    cache's maximum) reproduce the hybrid operator on the concatenated clip."""
+    wl = hi.Workload("t", B=2, Hs=1, Hd=1, Hg=1, d=128, T=sum(groups), N=130, w_swa=3, w_dswa=4,
+                     r=2, chunk=64, dtype="bf16", decay=1.0)
+    x = hi.make_inputs(wl, seed=19)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    st = h.Stream(wl.B, wl.Hs, wl.Hd, wl.Hg, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r,
+                  max_step_frames=max(groups))
+    outs, f0 = [], 0
+    for g in groups:
+        s = slice(f0 * wl.N, (f0 + g) * wl.N)
+        outs.append(st.step_frames(q[:, :, s].contiguous(), k[:, :, s].contiguous(),
+                                   v[:, :, s].contiguous(), a[:, :, s].contiguous(),
+                                   b[:, :, s].contiguous(), g))
+        f0 += g
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    assert st.state()[1] == wl.T
+    o = torch.cat(outs, dim=2)
+    o_ref, S_ref = orc.hybrid(x["q"], x["k"], x["v"], x["a"], x["b"], wl.Hs, wl.Hd, wl.Hg,
+                              wl.T, wl.N, wl.w_swa, wl.w_dswa, wl.r)
+    assert maxabs(o, o_ref) <= TOL
+    assert maxabs(st.state_tensor(), S_ref) <= TOL
+    st.close()
+
+
+def test_stream_step_frames_rejects_too_many_frames(h):
+    wl = hi.Workload("t", B=1, Hs=1, Hd=1, Hg=1, d=128, T=3, N=64, w_swa=2, w_dswa=2, r=1,
+                     chunk=64, dtype="bf16", decay=1.0)
+    x = hi.make_inputs(wl, seed=2)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    st = h.Stream(wl.B, wl.Hs, wl.Hd, wl.Hg, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r, max_step_frames=2)
+    with pytest.raises(h.HltaError):
+        st.step_frames(q, k, v, a, b, 3)
+    assert st.state()[1] == 0                  # nothing was appended
+    st.close()
