@@ -54,6 +54,15 @@ def _load():
         for fn in (lib.oracle_swa, lib.oracle_dswa, lib.oracle_gdn, lib.oracle_gdn_raw):
             fn.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
+        u8 = ctypes.POINTER(ctypes.c_ubyte)
+        lib.oracle_e4m3_decode.argtypes = [I_]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_int
+        lib.oracle_fp8_quantize_rows.argtypes = [f32, f32, L_, L_, I_, L_, I_, u8, f32]
+        lib.oracle_fp8_quantize_channels.argtypes = [f32, L_, L_, I_, u8, f32]
+        for fn in (lib.oracle_fp8_quantize_rows, lib.oracle_fp8_quantize_channels):
+            fn.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -195,6 +204,84 @@ def hybrid(q, k, v, a, b, Hs: int, Hd: int, Hg: int, T: int, N: int,
             og, S_fin = gdn_raw(qf[:, s], kf[:, s], vf[:, s], a, b, raw, S0)
         o[:, s] = og
     return o, S_fin
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of one E4M3 code (OCP 8-bit floating point, E4M3 encoding)."""
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def e4m3_encode(y: float) -> int:
+    """Nearest E4M3 code to the float32 value y (ties to even, saturating at +-448)."""
+    return int(_load().oracle_e4m3_encode(float(np.float32(y))))
+
+
+def e4m3_values() -> np.ndarray:
+    """float64 value of each of the 256 codes (NaN for 0x7F and 0xFF)."""
+    return np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def fp8_quantize_rows(x, frame_rows: int, block_rows: int, shift=None):
+    """Row-block E4M3 quantisation of x [..., L, d]: blocks of block_rows rows inside frames
+    of frame_rows rows. Returns (codes uint8 [..., L, d], scales float32 [..., nf, nb])."""
+    xf = _f32(x)
+    L, d = xf.shape[-2], xf.shape[-1]
+    lead = xf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    nf = -(-L // frame_rows)
+    nb = -(-frame_rows // block_rows)
+    sh = None if shift is None else _f32(shift).reshape(BH, d)
+    x8 = np.empty(xf.shape, dtype=np.uint8)
+    sc = np.empty(lead + (nf, nb), dtype=np.float32)
+    rc = _load().oracle_fp8_quantize_rows(_ptr(xf, ctypes.c_float), _ptr(sh, ctypes.c_float), BH,
+                                          L, d, frame_rows, block_rows,
+                                          _ptr(x8, ctypes.c_ubyte), _ptr(sc, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle fp8_quantize_rows failed ({rc})")
+    return x8, sc
+
+
+def fp8_quantize_channels(x):
+    """Per-channel E4M3 quantisation of x [..., L, d] (one scale per head and channel).
+    Returns (codes uint8 [..., L, d], scales float32 [..., d])."""
+    xf = _f32(x)
+    L, d = xf.shape[-2], xf.shape[-1]
+    lead = xf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    x8 = np.empty(xf.shape, dtype=np.uint8)
+    sc = np.empty(lead + (d,), dtype=np.float32)
+    rc = _load().oracle_fp8_quantize_channels(_ptr(xf, ctypes.c_float), BH, L, d,
+                                              _ptr(x8, ctypes.c_ubyte), _ptr(sc, ctypes.c_float))
+    if rc != 0:
+        raise RuntimeError(f"oracle fp8_quantize_channels failed ({rc})")
+    return x8, sc
+
+
+def fp8_dequantize_rows(x8, scales, frame_rows: int, block_rows: int) -> np.ndarray:
+    """decode(code) * scale of the code's row block, float64 [..., L, d]."""
+    x8 = np.asarray(x8)
+    L = x8.shape[-2]
+    l = np.arange(L)
+    f, j = l // frame_rows, (l % frame_rows) // block_rows
+    s = np.asarray(scales, dtype=np.float64)[..., f, j]          # [..., L]
+    return e4m3_values()[x8] * s[..., None]
+
+
+def fp8_dequantize_channels(x8, scales) -> np.ndarray:
+    """decode(code) * scale of the code's channel, float64 [..., L, d]."""
+    return e4m3_values()[np.asarray(x8)] * np.asarray(scales, dtype=np.float64)[..., None, :]
+
+
+def window_fp8(q8, qs, k8, ks, v8, vs, T: int, N: int, w: int, r: int, scale=None, rows=None):
+    """Windowed attention (SWA when r == 1, DSWA otherwise) of E4M3 inputs: the plain
+    attention of the dequantised tensors. Q blocks: 128 rows of the head; K blocks: 64-row
+    runs inside each frame; V: one scale per channel. (The dequantised values are passed to
+    the attention as float32, a relative rounding of 2^-24.)"""
+    L = T * N
+    q = fp8_dequantize_rows(q8, qs, L, 128)
+    k = fp8_dequantize_rows(k8, ks, N, 64)
+    v = fp8_dequantize_channels(v8, vs)
+    return _window(q, k, v, T, N, w, r, r > 1, scale, rows)
 
 
 def hybrid_rows(q, k, v, a, b, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, rows, scale=None):

@@ -286,6 +286,131 @@ int oracle_gdn_raw(const float *q, const float *k, const float *v, const float *
     return err;
 }
 
+/*
+ * FP8 attention inputs. The related-papers analysis (zhaifeiyue.github.io, row C1 and the
+ * paragraphs on deployment quantisation) says the deployed model quantises attention to FP8
+ * but gives no method. The format used here is the OCP 8-bit floating point E4M3 encoding
+ * (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ * subnormals m/8 * 2^-6; S.1111.111 is NaN; no infinities; largest finite value 448).
+ *
+ * Quantisation with one fp32 scale per block of rows (or per channel): amax is the largest
+ * magnitude in the block, every element x becomes the E4M3 code nearest to x * (448/amax)
+ * (ties to the even code, magnitudes beyond 448 saturate to 448), and the stored scale is
+ * amax/448, so that x ~ decode(code) * scale. The three fp32 operations (448/amax, the
+ * product, amax/448) are single IEEE roundings, in this order, on both sides of a parity
+ * test: the codes are then integers both sides must agree on bit for bit.
+ */
+double oracle_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* The non-negative finite E4M3 values, codes 0x00 .. 0x7E, increasing with the code. */
+static void e4m3_table(double *tab)
+{
+    for (int c = 0; c < 0x7F; ++c) tab[c] = oracle_e4m3_decode(c);
+}
+
+/* Nearest code by exhaustive search over the 127 non-negative finite values; of two equally
+ * near values (always neighbours) the even code wins; the sign bit is the sign of y. */
+static int e4m3_encode_tab(const double *tab, float y)
+{
+    if (isnan(y)) return 0x7F;
+    int sign = signbit(y) ? 0x80 : 0;
+    if (isinf(y)) return sign | 0x7E;
+    double a = fabs((double)y), bd = INFINITY;
+    int best = 0;
+    for (int c = 0; c < 0x7F; ++c) {
+        double dd = fabs(tab[c] - a);
+        if (dd < bd || (dd == bd && (c & 1) == 0)) {
+            bd = dd;
+            best = c;
+        }
+    }
+    return sign | best;
+}
+
+int oracle_e4m3_encode(float y)
+{
+    double tab[0x7F];
+    e4m3_table(tab);
+    return e4m3_encode_tab(tab, y);
+}
+
+/* One block: rows r0 .. r0+nr-1 of a [L][d] head (optionally minus a per-channel shift),
+ * columns c0 .. c0+nc-1 (a single channel when nc == 1 and the block runs down a column). */
+static float quantize_block(const double *tab, const float *x, const float *shift, long r0,
+                            long nr, int d, int c0, int nc, unsigned char *x8)
+{
+    float amax = 0.0f;
+    for (long r = r0; r < r0 + nr; ++r)
+        for (int c = c0; c < c0 + nc; ++c) {
+            float v = x[r * d + c];
+            if (shift) v = v - shift[c];
+            float a = fabsf(v);
+            if (a > amax) amax = a;
+        }
+    float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+    for (long r = r0; r < r0 + nr; ++r)
+        for (int c = c0; c < c0 + nc; ++c) {
+            float v = x[r * d + c];
+            if (shift) v = v - shift[c];
+            float y = v * inv;
+            x8[r * d + c] = (unsigned char)e4m3_encode_tab(tab, y);
+        }
+    return amax / 448.0f;
+}
+
+/*
+ * Row-block quantisation. x: [BH][L][d] float32; shift: [BH][d] or NULL (subtracted from
+ * every row first, in fp32). Each head is cut into frames of frame_rows rows (the last frame
+ * may be short) and each frame into runs of block_rows rows (the last run of a frame may be
+ * short); a block never spans two frames. Output codes x8: [BH][L][d]; scales:
+ * [BH][nframes][nb], nframes = ceil(L / frame_rows), nb = ceil(frame_rows / block_rows).
+ */
+int oracle_fp8_quantize_rows(const float *x, const float *shift, long BH, long L, int d,
+                             long frame_rows, int block_rows, unsigned char *x8, float *scale)
+{
+    if (BH < 0 || L < 0 || d < 1 || frame_rows < 1 || block_rows < 1) return 1;
+    double tab[0x7F];
+    e4m3_table(tab);
+    long nf = (L + frame_rows - 1) / frame_rows, nb = (frame_rows + block_rows - 1) / block_rows;
+#pragma omp parallel for collapse(2) schedule(dynamic, 4)
+    for (long bh = 0; bh < BH; ++bh)
+        for (long f = 0; f < nf; ++f) {
+            long fr0 = f * frame_rows, fr1 = fr0 + frame_rows < L ? fr0 + frame_rows : L;
+            for (long j = 0; j < nb; ++j) {
+                long r0 = fr0 + j * block_rows;
+                long nr = r0 >= fr1 ? 0 : (r0 + block_rows < fr1 ? block_rows : fr1 - r0);
+                scale[(bh * nf + f) * nb + j] =
+                    nr > 0 ? quantize_block(tab, x + bh * L * d, shift ? shift + bh * d : NULL,
+                                            r0, nr, d, 0, d, x8 + bh * L * d)
+                           : 0.0f;
+            }
+        }
+    return 0;
+}
+
+/*
+ * Per-channel quantisation: one scale per (head, channel) over all L rows of the head.
+ * x: [BH][L][d] float32 -> x8: [BH][L][d] codes, scale: [BH][d].
+ */
+int oracle_fp8_quantize_channels(const float *x, long BH, long L, int d, unsigned char *x8,
+                                 float *scale)
+{
+    if (BH < 0 || L < 0 || d < 1) return 1;
+    double tab[0x7F];
+    e4m3_table(tab);
+#pragma omp parallel for collapse(2)
+    for (long bh = 0; bh < BH; ++bh)
+        for (int c = 0; c < d; ++c)
+            scale[bh * d + c] = quantize_block(tab, x + bh * L * d, NULL, 0, L, d, c, 1, x8 + bh * L * d);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
