@@ -88,6 +88,56 @@ hlta_status hlta_dswa_fwd(const void *q, const void *k, const void *v, void *o,
                           hlta_dtype dt, void *stream);
 
 /*
+ * FP8 (E4M3) window attention: the related-papers analysis (zhaifeiyue.github.io, row C1 and
+ * the paragraphs on deployment quantisation) reports that the deployed model quantises
+ * attention to FP8 without giving the method; this is one. Codes are OCP 8-bit floating
+ * point E4M3 (bias 7, largest finite 448) with fp32 scales, x ~ code * scale:
+ *   queries: one scale per 128-row block of each head's T*N rows,
+ *   keys:    one scale per 64-row run of each frame (ceil(N/64) runs per frame; the last run
+ *            of a frame is short when N % 64 != 0),
+ *   values:  one scale per channel of each head.
+ * hlta_fp8_quantize_rows / hlta_fp8_quantize_channels produce these from bf16 tensors.
+ *
+ * Row-block quantisation of x [B, H, L, d] bf16 (device), d = 128: each head is cut into
+ * frames of frame_rows rows (the last one may be short), each frame into runs of block_rows
+ * rows (1 <= block_rows <= 128; the last run of a frame may be short). Per block:
+ * amax = max |x - shift| (fp32), codes = E4M3 round-to-nearest-even, saturating, of
+ * (x - shift) * (448 / amax), scale = amax / 448 (0 and all-zero codes for amax = 0); each of
+ * the fp32 operations is one IEEE rounding. shift: [B, H, d] float32 subtracted from every
+ * row first (e.g. the per-channel mean of K, which leaves softmax attention unchanged), or
+ * NULL. x8: [B, H, L, d] bytes; scales: [B, H, ceil(L/frame_rows), ceil(frame_rows/block_rows)]
+ * float32. For the attention: q with frame_rows = T*N, block_rows = 128; k with
+ * frame_rows = N, block_rows = 64. All pointers device, 16-byte aligned, caller-owned;
+ * enqueued on `stream`. Bad shapes or pointers: HLTA_ERR_INVALID_ARG / HLTA_ERR_UNSUPPORTED.
+ */
+hlta_status hlta_fp8_quantize_rows(const void *x, const float *shift, int B, int H, long L,
+                                   int d, long frame_rows, int block_rows, void *x8,
+                                   float *scales, void *stream);
+
+/*
+ * Per-channel quantisation of x [B, H, L, d] bf16 (device), d = 128: per (head, channel)
+ * amax over the L rows, codes and scale as above. x8: [B, H, L, d] bytes; scales: [B, H, d]
+ * float32 (also used as scratch while the maxima are gathered). Enqueues four operations on
+ * `stream`.
+ */
+hlta_status hlta_fp8_quantize_channels(const void *x, int B, int H, long L, int d, void *x8,
+                                       float *scales, void *stream);
+
+/*
+ * Window attention of E4M3 inputs (SWA for r = 1, DSWA otherwise; windows as hlta_dswa_fwd).
+ * q8, k8, v8: [B, H, T*N, d] E4M3 codes (device, d = 128); q_scales [B, H, ceil(T*N/128)],
+ * k_scales [B, H, T, ceil(N/64)], v_scales [B, H, d] float32 as produced above; o:
+ * [B, H, T*N, d] bf16. The result approximates the attention of the dequantised inputs:
+ * both products run on E4M3 tensor-core operands with fp32 accumulation, and the softmax
+ * weights are rounded to E4M3 (relative error <= 2^-4 each) before they multiply V.
+ * scale <= 0 selects 1/sqrt(d). Errors as hlta_swa_fwd.
+ */
+hlta_status hlta_window_fp8_fwd(const void *q8, const float *q_scales, const void *k8,
+                                const float *k_scales, const void *v8, const float *v_scales,
+                                void *o, int B, int H, int T, int N, int d, int w, int r,
+                                float scale, void *stream);
+
+/*
  * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens.
  */
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt);

@@ -32,6 +32,15 @@
 // sub-tile may see is skipped for that sub-tile. Every mbarrier wait is bounded; on expiry
 // the kernel records DEVERR_ATTN_WAIT in the device error word, every role stops, and the
 // TMEM allocation is released.
+//
+// E4M3 variant (template flag F8): q, k, v arrive as OCP E4M3 codes with fp32 scales: one per
+// 128-row block of the head's query rows, one per 64-key tile of each key frame (the tiles
+// the walk visits), one per value channel. Both products run as tcgen05.mma kind::f8f6f4
+// (32 keys or head channels per instruction instead of 16): S from the codes, the softmax
+// scales each tile's scores by sl2 * s_q * s_k (one multiply it already does), P is written
+// as E4M3 codes (four per TMEM column) and the channel scales of V multiply the normalised
+// output. P = 2^(x - m + 4) with the running max grown once it rose by more than 2^4, so P
+// stays in [0, 256] (E4M3 reaches 448) and keeps normal precision down to 2^-6 of the max.
 #include "hlta_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -55,6 +64,10 @@ constexpr uint32_t QHALF = BM * 128;    // [128 rows][64 cols] bf16: 16 KB
 constexpr uint32_t QTILE = 2 * QHALF;   // [128][128]
 constexpr uint32_t KHALF = BN * 128;    // [64 rows][64 cols] bf16: 8 KB
 constexpr uint32_t KTILE = 2 * KHALF;   // [64][128]
+// bytes of one Q sub-tile and of one K or V tile as loaded: an E4M3 row is one 128-byte
+// swizzle row, a bf16 row two 64-column halves. The shared-memory slots are sized for bf16.
+template <bool F8> constexpr uint32_t q_bytes() { return F8 ? (uint32_t)BM * 128u : QTILE; }
+template <bool F8> constexpr uint32_t kv_bytes() { return F8 ? (uint32_t)BN * 128u : KTILE; }
 constexpr uint32_t TMEM_COLS = 512;     // S_0[0] @0, S_0[1] @64, S_1[0] @128, S_1[1] @192, O_0 @256, O_1 @384
 __host__ __device__ constexpr uint32_t TM_S(int q, int b) { return (uint32_t)q * 128u + (uint32_t)b * 64u; }
 __host__ __device__ constexpr uint32_t TM_O(int q) { return 256u + (uint32_t)q * 128u; }
@@ -87,6 +100,8 @@ struct TcParams {
     long q_rows, kv_rows;
     int N, w, r, fq0;
     float sl2;                  // softmax scale * log2(e)
+    const float *qs, *ks, *vs;  // E4M3 scales: [heads][nqb], [heads][nkb], [heads][128]
+    int nqb, nkb;               // per head: query blocks of 128 rows, key tiles (slot * tpf + tile)
     __nv_bfloat16 *o;
     unsigned int *err;
 };
@@ -132,6 +147,28 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
+// kind::f8f6f4 forms (both operands E4M3 here; 32 elements of K per instruction)
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version bit.
 // lbo / sbo in bytes: K-major operands use sbo = 1024 (8 rows of 128 B) and an unused lbo;
 // MN-major operands use lbo = distance between 64-element column blocks, sbo = 1024.
@@ -151,6 +188,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
            ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f8f6f4: E4M3 A and B (format code 0), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 #define TMEM_REGS32(x)                                                                      \
@@ -208,6 +252,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&x)[16
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&x)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(x[0]), "r"(x[1]), "r"(x[2]), "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&x)[32])
 {
     asm volatile(
@@ -258,6 +310,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// four E4M3 codes in one word, p0 in the lowest byte (the K order of a TMEM A operand);
+// round to nearest even, saturating at 448
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
+    return r;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -330,6 +396,7 @@ __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
     return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, const TcParams p)
@@ -407,11 +474,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         // step s loads K(s) and V(s - LOOKAHEAD): the MMA warp consumes K up to LOOKAHEAD
         // tiles ahead of V
         if (lane == 0) {
-            mbar_expect_tx(BAR(B_QFULL), QT * QTILE);
+            mbar_expect_tx(BAR(B_QFULL), QT * q_bytes<F8>());
             for (int q = 0; q < QT; ++q) {
                 const int qrow = (int)(q_head + l0 + q * BM);
                 tma_load_2d(sbase + SM_Q(q), &tq, 0, qrow, BAR(B_QFULL));
-                tma_load_2d(sbase + SM_Q(q) + QHALF, &tq, 64, qrow, BAR(B_QFULL));
+                if (!F8) tma_load_2d(sbase + SM_Q(q) + QHALF, &tq, 64, qrow, BAR(B_QFULL));
             }
             Pos kp = walk_start(wk, fstart), vp = kp;
             int nk = 0, nv = 0;                     // K and V tiles issued
@@ -420,10 +487,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 if (more_k && (more_k = walk_step(wk, kp))) {
                     const int st = nk % NS;
                     if (nk >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((nk / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
-                    mbar_expect_tx(BAR(B_KFULL + st), KTILE);
+                    mbar_expect_tx(BAR(B_KFULL + st), kv_bytes<F8>());
                     const int row = kv_row(kp.fk, kp.jt);
                     tma_load_2d(sbase + SM_K(st), &tk, 0, row, BAR(B_KFULL + st));
-                    tma_load_2d(sbase + SM_K(st) + KHALF, &tk, 64, row, BAR(B_KFULL + st));
+                    if (!F8) tma_load_2d(sbase + SM_K(st) + KHALF, &tk, 64, row, BAR(B_KFULL + st));
                     ++nk;
                 }
                 if (nv < nk - LOOKAHEAD || (!more_k && nv < nk)) {
@@ -432,10 +499,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     // the same release as K of this tile: complete already (the stage's next
                     // release needs this V, so the phase cannot have moved on)
                     if (nv >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((nv / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) { ok = false; break; }
-                    mbar_expect_tx(BAR(B_VFULL + st), KTILE);
+                    mbar_expect_tx(BAR(B_VFULL + st), kv_bytes<F8>());
                     const int row = kv_row(vp.fk, vp.jt);
                     tma_load_2d(sbase + SM_V(st), &tv, 0, row, BAR(B_VFULL + st));
-                    tma_load_2d(sbase + SM_V(st) + KHALF, &tv, 64, row, BAR(B_VFULL + st));
+                    if (!F8) tma_load_2d(sbase + SM_V(st) + KHALF, &tv, 64, row, BAR(B_VFULL + st));
                     ++nv;
                 } else if (!more_k) {
                     more_v = false;
@@ -459,8 +526,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         if (lane == 0) {
             const int q = warp - WARP_MMA;
             const int want = 1 << q;
-            constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, false, false);   // Q, K K-major
-            constexpr uint32_t IDESC_O = idesc_bf16(BM, D, false, true);     // P (TMEM), V MN-major
+            // Q, K K-major; P (TMEM), V MN-major
+            constexpr uint32_t IDESC_S = F8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t IDESC_O = F8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
             // Shared-memory descriptors built once; each product only adds a compile-time
             // offset (and the ring stage's) to the 14-bit start-address field.
             const uint64_t dq = sw128_desc(sbase + SM_Q(q), 16, 1024);
@@ -483,11 +551,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     if (!wait_bar(BAR(B_KFULL + st), (uint32_t)(c.j / NS) & 1u)) return false;
                     const int bf = ns & 1;
                     const uint64_t dk = dk0 + (uint64_t)((st * KTILE) >> 4);
+                    if constexpr (F8) {
+                        // 32 channels (32 bytes of the swizzle row) per instruction
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t qoff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
-                        const uint32_t koff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
-                        umma_bf16(s_tm + bf * 64, dq + qoff, dk + koff, IDESC_S, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            umma_f8(s_tm + bf * 64, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), IDESC_S, kk > 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t qoff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                            const uint32_t koff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                            umma_bf16(s_tm + bf * 64, dq + qoff, dk + koff, IDESC_S, kk > 0 ? 1u : 0u);
+                        }
                     }
                     umma_commit(BAR(B_SFULL + 2 * q + bf));
                     ++ns;
@@ -502,16 +577,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 ok = topup(j + LOOKAHEAD) && wait_bar(BAR(B_VFULL + st), (uint32_t)(j / NS) & 1u);
                 if (!ok) break;
                 if (t.mask & want) {
-                    // O += P V with P in the first 32 columns of the S buffer
+                    // O += P V with P in the first 32 (bf16) or 16 (E4M3) columns of the S buffer
                     const int bf = npv & 1;
                     if (!(ok = wait_bar(BAR(B_PFULL + 2 * q + bf), (uint32_t)(npv >> 1) & 1u))) break;
                     fence_after_sync();
                     const uint64_t dv = dv0 + (uint64_t)((st * KTILE) >> 4);
                     const uint32_t acc0 = npv > 0 ? 1u : 0u;
+                    if constexpr (F8) {
+                        // 32 keys per instruction: 8 TMEM columns of P, 32 V rows of 128 B
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        umma_bf16_ts(o_tm, s_tm + bf * 64 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
-                                     kk > 0 ? 1u : acc0);
+                        for (int kk = 0; kk < BN / 32; ++kk)
+                            umma_f8_ts(o_tm, s_tm + bf * 64 + kk * 8, dv + (uint64_t)((kk * 4096) >> 4), IDESC_O,
+                                       kk > 0 ? 1u : acc0);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < BN / 16; ++kk)
+                            umma_bf16_ts(o_tm, s_tm + bf * 64 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                                         kk > 0 ? 1u : acc0);
+                    }
                     umma_commit(BAR(B_PVDONE + q));
                     ++npv;
                     // the buffer P V just read takes the S two tiles ahead (issue order)
@@ -535,6 +618,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         const bool row_valid = lrow < p.q_rows;
         const int fq = p.fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+        // E4M3: scores carry the Q block's scale (per sub-tile) and the K tile's (per tile);
+        // sub-tile 1 of a head's last CTA may lie past the last query block
+        const int kvh = b * p.kv_Htot + p.kv_h0 + h;
+        const long qblk = l0 / BM + q;
+        const float sl2q = !F8 ? p.sl2
+                         : qblk < p.nqb ? p.sl2 * __ldg(p.qs + (long)(b * p.q_Htot + p.q_h0 + h) * p.nqb + qblk)
+                                        : 0.f;
+        constexpr float LAZY = F8 ? 4.f : 8.f;          // log2 growth of the max before a rescale
+        constexpr float PBIAS = F8 ? 4.f : 0.f;         // P = 2^(x - m + PBIAS)
         float m = -INFINITY, lsum = 0.f;
         bool ok = true;
         int k = 0;
@@ -542,6 +634,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         while (walk_next(wk, c, 1 << q)) {              // this sub-tile's tiles (uniform per warp)
             const int fk = c.fk, jt = c.jt;
             const int bf = k & 1;
+            // the K tile's scale, fetched before the wait so its latency hides behind it
+            const float sl2 = F8 ? sl2q * __ldg(p.ks + (long)kvh * p.nkb + (long)(fk % p.kv_slots) * wk.tpf + jt) : sl2q;
             const uint32_t sbar = BAR(B_SFULL + 2 * q + bf), spar = (uint32_t)(k >> 1) & 1u;
             if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
@@ -561,9 +655,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
             }
             const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            const float mnew = rok ? fmaxf(m, mt * p.sl2) : m;
-            // grow the reference max only when it rose by more than 2^8 (lazy rescale)
-            const bool need = rok && mnew > m + 8.f;
+            const float mnew = rok ? fmaxf(m, mt * sl2) : m;
+            // grow the reference max only when it rose by more than 2^LAZY (lazy rescale)
+            const bool need = rok && mnew > m + LAZY;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
             // rescale O (warp-wide TMEM traffic, so the warp takes the branch together) once
@@ -583,39 +677,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     tmem_st32(tlane + TM_O(q) + c * 32, orow);
                 }
             }
-            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) go to the
-            // first 32 columns of the S buffer. `full` and `rok` differ between lanes whose
-            // rows straddle a frame boundary, so only the arithmetic branches on them; every
-            // tcgen05.ld / st stays warp-uniform.
+            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) or E4M3
+            // quads (key 4i in the low byte) go to the first 32 or 16 columns of the S buffer.
+            // `full` and `rok` differ between lanes whose rows straddle a frame boundary, so
+            // only the arithmetic branches on them; every tcgen05.ld / st stays warp-uniform.
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
             float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            const float2 sl2x2 = make_float2(p.sl2, p.sl2), nm2 = make_float2(-muse, -muse);
+            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(PBIAS - muse, PBIAS - muse);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t pk[16];
-                if (full) {
+                if constexpr (F8) {
+                    uint32_t pk[8];
+                    if (full) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 x = ffma2(make_float2(__uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1])), sl2x2, nm2);
-                        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-                        ps2[i & 1] = fadd2(ps2[i & 1], pp);
-                        pk[i] = pack_bf16(pp.x, pp.y);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c * 32 + 2 * i;
-                        float p0 = 0.f, p1 = 0.f;
-                        if (rok) {
-                            p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -muse)) : 0.f;
-                            p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -muse)) : 0.f;
+                        for (int i = 0; i < 8; ++i) {
+                            const int col = c * 32 + 4 * i;
+                            const float2 xa = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2x2, nm2);
+                            const float2 xb = ffma2(make_float2(__uint_as_float(sr[col + 2]), __uint_as_float(sr[col + 3])), sl2x2, nm2);
+                            const float2 pa = make_float2(ex2(xa.x), ex2(xa.y));
+                            const float2 pb = make_float2(ex2(xb.x), ex2(xb.y));
+                            ps2[0] = fadd2(ps2[0], pa);
+                            ps2[1] = fadd2(ps2[1], pb);
+                            pk[i] = pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
                         }
-                        ps[i & 3] += p0 + p1;
-                        pk[i] = pack_bf16(p0, p1);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float pv[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int col = c * 32 + 4 * i + t;
+                                pv[t] = rok && col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, PBIAS - muse)) : 0.f;
+                            }
+                            ps[i & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+                            pk[i] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+                        }
                     }
+                    __syncwarp();                       // reconverge before .sync.aligned
+                    tmem_st8(tlane + TM_S(q, bf) + c * 8, pk);
+                } else {
+                    uint32_t pk[16];
+                    if (full) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float2 x = ffma2(make_float2(__uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1])), sl2x2, nm2);
+                            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                            ps2[i & 1] = fadd2(ps2[i & 1], pp);
+                            pk[i] = pack_bf16(pp.x, pp.y);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = c * 32 + 2 * i;
+                            float p0 = 0.f, p1 = 0.f;
+                            if (rok) {
+                                p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, -muse)) : 0.f;
+                                p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), sl2, -muse)) : 0.f;
+                            }
+                            ps[i & 3] += p0 + p1;
+                            pk[i] = pack_bf16(p0, p1);
+                        }
+                    }
+                    __syncwarp();                       // reconverge before .sync.aligned
+                    tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
                 }
-                __syncwarp();                           // reconverge before .sync.aligned
-                tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
             }
             lsum = lsum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y)));
             m = muse;
@@ -633,12 +758,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
             __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
+            const float4 *vsc = F8 ? reinterpret_cast<const float4 *>(p.vs + (long)kvh * D) : nullptr;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
                 __syncwarp();
                 tmem_ld32(tlane + TM_O(q) + c * 32, ov);
                 if (row_valid) {
+                    if constexpr (F8) {
+                        // the value channels' scales (the same 32 floats for every lane)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 sv = __ldg(vsc + c * 8 + i);
+                            ov[4 * i] = __float_as_uint(__uint_as_float(ov[4 * i]) * sv.x);
+                            ov[4 * i + 1] = __float_as_uint(__uint_as_float(ov[4 * i + 1]) * sv.y);
+                            ov[4 * i + 2] = __float_as_uint(__uint_as_float(ov[4 * i + 2]) * sv.z);
+                            ov[4 * i + 3] = __float_as_uint(__uint_as_float(ov[4 * i + 3]) * sv.w);
+                        }
+                    }
                     uint32_t pk2[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -665,9 +802,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
-}  // namespace
 
-cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
+template <bool F8>
+cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
 {
     if (a.d != D) return cudaErrorNotSupported;
     cudaError_t e;
@@ -675,23 +812,39 @@ cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s)
     const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
     if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
-    // [rows][128] bf16 views, boxes of 64 columns (128 rows for Q, 64 for K and V), 128-byte swizzle
-    if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    // [rows][128] views with 128-byte swizzle: bf16 in boxes of 64 columns, E4M3 in boxes of
+    // the whole 128-byte row; 128 rows for Q, 64 for K and V
+    if (F8) {
+        if ((e = make_tmap_2d_u8(&mq, a.q, q_total, D, D, BM)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_u8(&mk, a.k, kv_total, D, D, BN)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_u8(&mv, a.v, kv_total, D, D, BN)) != cudaSuccess) return e;
+    } else {
+        if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    }
     TcParams p;
     p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
     p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
     p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0;
     p.sl2 = a.scale * 1.4426950408889634f;
+    p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
+    p.nqb = (int)((a.q_rows + BM - 1) / BM);
+    p.nkb = a.kv_slots * ((a.N + BN - 1) / BN);
     p.o = (__nv_bfloat16 *)a.o;
     p.err = a.err;
-    e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (F8 && (!p.qs || !p.ks || !p.vs)) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(attn_tc_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
-    attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
+    attn_tc_kernel<F8><<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
+
+}  // namespace
+
+cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc<false>(a, s); }
+cudaError_t launch_attn_fp8_tc(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc<true>(a, s); }
 
 }  // namespace hlta

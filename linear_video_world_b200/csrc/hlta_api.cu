@@ -260,6 +260,66 @@ hlta_status hlta_dswa_fwd(const void *q, const void *k, const void *v, void *o, 
     return window_fwd(q, k, v, o, B, H, T, N, d, w, r, scale, dt, stream);
 }
 
+hlta_status hlta_fp8_quantize_rows(const void *x, const float *shift, int B, int H, long L,
+                                   int d, long frame_rows, int block_rows, void *x8,
+                                   float *scales, void *stream)
+{
+    if (!x || !x8 || !scales) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(x) || !aligned16(x8) || !aligned16(scales) || (shift && !aligned16(shift)))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 0 || H < 0 || L < 0) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld", B, H, L);
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "FP8 quantisation supports d = 128 only (got %d)", d);
+    if (frame_rows < 1 || block_rows < 1 || block_rows > 128)
+        return fail(HLTA_ERR_INVALID_ARG, "need frame_rows >= 1 and 1 <= block_rows <= 128 (got %ld, %d)", frame_rows, block_rows);
+    cudaError_t e = launch_fp8_quantize_rows(x, shift, (long)B * H, L, frame_rows, block_rows, x8,
+                                             scales, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "FP8 quantisation: too many blocks");
+    if (e != cudaSuccess) return cuda_fail(e, "FP8 row quantisation launch");
+    return HLTA_OK;
+}
+
+hlta_status hlta_fp8_quantize_channels(const void *x, int B, int H, long L, int d, void *x8,
+                                       float *scales, void *stream)
+{
+    if (!x || !x8 || !scales) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(x) || !aligned16(x8) || !aligned16(scales))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 0 || H < 0 || L < 0) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld", B, H, L);
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "FP8 quantisation supports d = 128 only (got %d)", d);
+    cudaError_t e = launch_fp8_quantize_channels(x, (long)B * H, L, x8, scales, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "FP8 quantisation: too many heads");
+    if (e != cudaSuccess) return cuda_fail(e, "FP8 channel quantisation launch");
+    return HLTA_OK;
+}
+
+hlta_status hlta_window_fp8_fwd(const void *q8, const float *q_scales, const void *k8,
+                                const float *k_scales, const void *v8, const float *v_scales,
+                                void *o, int B, int H, int T, int N, int d, int w, int r,
+                                float scale, void *stream)
+{
+    hlta_status st;
+    if (!q8 || !k8 || !v8 || !o || !q_scales || !k_scales || !v_scales)
+        return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) ||
+        !aligned16(q_scales) || !aligned16(k_scales) || !aligned16(v_scales))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 0 || H < 0 || T < 1 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d T=%d N=%d", B, H, T, N);
+    if ((long)T * N > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "T*N too large");
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "FP8 attention supports d = 128 only (got %d)", d);
+    if ((st = check_window(w, r)) != HLTA_OK) return st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    AttnArgs a = clip_attn_args(q8, k8, v8, o, B, H, 0, H, T, N, d, w, r, scale, ctx->err);
+    a.qs = q_scales;
+    a.ks = k_scales;
+    a.vs = v_scales;
+    if (B * H == 0) return HLTA_OK;
+    cudaError_t e = launch_attn_fp8_tc(a, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "FP8 window attention: unsupported shape");
+    if (e != cudaSuccess) return cuda_fail(e, "FP8 window attention launch");
+    return HLTA_OK;
+}
+
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt)
 {
     if (B < 0 || H < 0 || L < 0 || d < 1 || chunk != 64) return 0;

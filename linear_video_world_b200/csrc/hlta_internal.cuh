@@ -27,6 +27,9 @@ struct AttnArgs {
     int fq0;
     float scale;
     unsigned int *err;   // device error word (bounded waits that expired)
+    // E4M3 inputs only: fp32 scales of the query blocks ([B*q_Htot][ceil(q_rows/128)]), the
+    // key tiles ([B*kv_Htot][kv_slots][ceil(N/64)]) and the value channels ([B*kv_Htot][d])
+    const float *qs = nullptr, *ks = nullptr, *vs = nullptr;
 };
 
 // Gated delta rule over [B][Htot][L][d] tensors, this branch's heads at h0 .. h0 + Hg.
@@ -71,10 +74,20 @@ int record_error_impl(int st, const char *fmt, ...);
 // box_rows x box_cols, 128-byte swizzle or none.
 cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                               uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+// The same over bytes (E4M3 codes), always with the 128-byte swizzle (box_cols <= 128).
+cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                            uint32_t box_cols, uint32_t box_rows);
 
 // Launchers. Return cudaGetLastError() of their launches.
 cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attn_fp8_tc(const AttnArgs &a, cudaStream_t s);
+// E4M3 quantisation (bf16 input, d = 128): row blocks inside frames, and value channels
+cudaError_t launch_fp8_quantize_rows(const void *x, const float *shift, long BH, long L,
+                                     long frame_rows, int block_rows, void *x8, float *scales,
+                                     cudaStream_t s);
+cudaError_t launch_fp8_quantize_channels(const void *x, long BH, long L, void *x8,
+                                         float *scales, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,

@@ -1,4 +1,4 @@
-// Host helper: 2-D TMA tensor maps over row-major [rows][cols] bf16 tensors. The driver's
+// Host helper: 2-D TMA tensor maps over row-major [rows][cols] bf16 or byte tensors. The driver's
 // encoder is fetched once through the runtime's entry-point query (no link-time libcuda).
 #include "hlta_internal.cuh"
 
@@ -13,8 +13,9 @@ std::once_flag g_encode_once;
 
 }  // namespace
 
-cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-                              uint32_t box_cols, uint32_t box_rows, bool swizzle128)
+static cudaError_t encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint32_t elem,
+                             const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                             uint32_t box_rows, bool swizzle128)
 {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
@@ -26,14 +27,28 @@ cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows,
     });
     if (!g_encode) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = g_encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                              uint32_t box_cols, uint32_t box_rows, bool swizzle128)
+{
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, box_cols,
+                     box_rows, swizzle128);
+}
+
+cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                            uint32_t box_cols, uint32_t box_rows)
+{
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, box_cols, box_rows,
+                     true);
 }
 
 }  // namespace hlta
