@@ -185,6 +185,39 @@ def measure_raw(h, torch, dev, wl, hi, steps: int) -> dict:
                     "computed inside the chunk preparation"}
 
 
+def measure_fp8(h, torch, dev, wl, q, k, v, steps: int) -> dict:
+    """The two softmax launches on E4M3 inputs (per-block q/k scales, per-channel v scales):
+    attention alone on resident codes, and the three quantisations plus attention from the
+    bf16 tensors. Same heads, windows and timing as attn_alone_*."""
+    hs, hd = slice(0, wl.Hs), slice(wl.Hs, wl.Hs + wl.Hd)
+    br = [(hs, wl.Hs, wl.w_swa, 1), (hd, wl.Hd, wl.w_dswa, wl.r)]
+    src = [tuple(x_[:, s_].contiguous() for x_ in (q, k, v)) for s_, _, _, _ in br]
+    codes = [h.fp8_quantize_window_inputs(*t, wl.T, wl.N) for t in src]
+    outs = [torch.empty(t[0].shape, dtype=torch.bfloat16, device=dev) for t in src]
+
+    def attn():
+        for (_, _, w, r), c, o in zip(br, codes, outs):
+            h.window_fp8(*c, wl.T, wl.N, w, r, out=o)
+
+    def quant_attn():
+        for (_, _, w, r), t, o in zip(br, src, outs):
+            h.window_fp8(*h.fp8_quantize_window_inputs(*t, wl.T, wl.N), wl.T, wl.N, w, r, out=o)
+
+    res = {}
+    for name, fn in (("attn", attn), ("quantise_and_attn", quant_attn)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = e0.elapsed_time(e1) / steps
+    return res
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -486,6 +519,8 @@ def main():
     del sub, o_s, o_d
     stream_detail = None if args.no_stream else measure_stream(h, torch, dev)
     raw_detail = None if args.no_stream else measure_raw(h, torch, dev, wl, hi, K)
+    fp8_ms = (measure_fp8(h, torch, dev, wl, q, k, v, K)
+              if not args.no_stream and wl.dtype == "bf16" and wl.Hs + wl.Hd > 0 else None)
 
     # ---- roofline of the dominant kernel (windowed attention, both launches) --------------
     wk = work(wl)
@@ -523,6 +558,21 @@ def main():
         detail["stream"] = stream_detail
     if raw_detail is not None:
         detail["raw_prologue"] = raw_detail
+    if fp8_ms is not None:
+        # E4M3 dense peak = the measured bf16 burst peak x 2 (nominal fp8:bf16 ratio 4.5:2.25)
+        fp8_peak = 2.0 * float(pk.get("bf16_tflops"))
+        elems = wl.B * (wl.Hs + wl.Hd) * wl.L * wl.d
+        detail["fp8"] = {
+            "attn_ms": fp8_ms["attn"],
+            "attn_tflops": attn_flop / (fp8_ms["attn"] / 1e3) / 1e12,
+            "attn_frac_of_fp8_peak": attn_flop / (fp8_ms["attn"] / 1e3) / 1e12 / fp8_peak,
+            "fp8_peak_tflops": fp8_peak,
+            "attn_bytes": 5 * elems,
+            "quantise_and_attn_ms": fp8_ms["quantise_and_attn"],
+            "note": "hlta_window_fp8_fwd for the SWA and DSWA heads back to back on resident E4M3 "
+                    "codes (q, k, v 1 byte, o bf16: attn_bytes), then with the three "
+                    "quantisations from bf16 in the timed region; peak = measured bf16 burst x 2",
+        }
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,

@@ -55,6 +55,9 @@ def _load() -> ctypes.CDLL:
         "hlta_stream_step_frames": (I, [P, P, P, P, P, P, P, I, P]),
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
+        "hlta_fp8_quantize_rows": (I, [P, P, I, I, L, I, L, I, P, P, P]),
+        "hlta_fp8_quantize_channels": (I, [P, I, I, L, I, P, P, P]),
+        "hlta_window_fp8_fwd": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
         "hlta_set_profile_events": (I, [ctypes.POINTER(P)]),
     }
@@ -177,6 +180,40 @@ def hlta_hybrid_fwd_raw(q, k, v, x, y, c, o, S0, S_out, B, Hs, Hd, Hg, T, N, d, 
                                     float(scale), ws_ptr, ws_bytes, _dt(q), _stream(stream)))
 
 
+def _need_types(x, x8, scales):
+    import torch
+    if x.dtype != torch.bfloat16 or x8.dtype != torch.uint8 or scales.dtype != torch.float32:
+        raise HltaError(HLTA_ERR_INVALID_ARG, "FP8 quantisation takes bf16 x, uint8 codes and "
+                        "float32 scales")
+
+
+def hlta_fp8_quantize_rows(x, shift, B, H, L, d, frame_rows, block_rows, x8, scales,
+                           stream=None):
+    for t, n in ((x, "x"), (x8, "x8"), (scales, "scales")):
+        _need(t, n)
+    _need_types(x, x8, scales)
+    if shift is not None:
+        _need(shift, "shift")
+    _check(_lib.hlta_fp8_quantize_rows(_p(x), _p(shift), B, H, L, d, frame_rows, block_rows,
+                                       _p(x8), _p(scales), _stream(stream)))
+
+
+def hlta_fp8_quantize_channels(x, B, H, L, d, x8, scales, stream=None):
+    for t, n in ((x, "x"), (x8, "x8"), (scales, "scales")):
+        _need(t, n)
+    _need_types(x, x8, scales)
+    _check(_lib.hlta_fp8_quantize_channels(_p(x), B, H, L, d, _p(x8), _p(scales),
+                                           _stream(stream)))
+
+
+def hlta_window_fp8_fwd(q8, qs, k8, ks, v8, vs, o, B, H, T, N, d, w, r, scale=0.0, stream=None):
+    for t, n in ((q8, "q8"), (qs, "q_scales"), (k8, "k8"), (ks, "k_scales"), (v8, "v8"),
+                 (vs, "v_scales"), (o, "o")):
+        _need(t, n)
+    _check(_lib.hlta_window_fp8_fwd(_p(q8), _p(qs), _p(k8), _p(ks), _p(v8), _p(vs), _p(o), B, H,
+                                    T, N, d, w, r, float(scale), _stream(stream)))
+
+
 def hlta_device_status(stream=None) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
@@ -212,6 +249,47 @@ def dswa(q, k, v, T, N, w, r, scale=0.0, out=None, stream=None):
     B, H, _, d = q.shape
     o = torch.empty_like(q) if out is None else out
     hlta_dswa_fwd(q, k, v, o, B, H, T, N, d, w, r, scale, stream)
+    return o
+
+
+def fp8_quantize_rows(x, frame_rows, block_rows, shift=None, stream=None):
+    """E4M3 codes (uint8, shape of x) and per-block scales [B, H, nframes, nblocks] of a bf16
+    [B, H, L, d] tensor; blocks of block_rows rows inside frames of frame_rows rows."""
+    import torch
+    B, H, L, d = x.shape
+    nf, nb = -(-L // frame_rows), -(-frame_rows // block_rows)
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty((B, H, nf, nb), dtype=torch.float32, device=x.device)
+    hlta_fp8_quantize_rows(x, shift, B, H, L, d, frame_rows, block_rows, x8, sc, stream)
+    return x8, sc
+
+
+def fp8_quantize_channels(x, stream=None):
+    """E4M3 codes and per-channel scales [B, H, d] of a bf16 [B, H, L, d] tensor."""
+    import torch
+    B, H, L, d = x.shape
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty((B, H, d), dtype=torch.float32, device=x.device)
+    hlta_fp8_quantize_channels(x, B, H, L, d, x8, sc, stream)
+    return x8, sc
+
+
+def fp8_quantize_window_inputs(q, k, v, T, N, k_shift=None, stream=None):
+    """The three quantisations the FP8 window attention takes: q in 128-row blocks of the
+    head, k in 64-row runs of each frame (optionally minus a per-channel shift), v per channel.
+    Returns (q8, qs, k8, ks, v8, vs)."""
+    q8, qs = fp8_quantize_rows(q, T * N, 128, None, stream)
+    k8, ks = fp8_quantize_rows(k, N, 64, k_shift, stream)
+    v8, vs = fp8_quantize_channels(v, stream)
+    return q8, qs, k8, ks, v8, vs
+
+
+def window_fp8(q8, qs, k8, ks, v8, vs, T, N, w, r=1, scale=0.0, out=None, stream=None):
+    """FP8 window attention (SWA for r = 1, DSWA otherwise); bf16 output [B, H, T*N, d]."""
+    import torch
+    B, H, L, d = q8.shape
+    o = torch.empty((B, H, L, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
+    hlta_window_fp8_fwd(q8, qs, k8, ks, v8, vs, o, B, H, T, N, d, w, r, scale, stream)
     return o
 
 

@@ -396,10 +396,10 @@ __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
     return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
 }
 
+// The kernel body of both variants; the tensor maps stay in the kernel's parameter space.
 template <bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-               const __grid_constant__ CUtensorMap tv, const TcParams p)
+__device__ __forceinline__ void attn_body(const CUtensorMap &tq, const CUtensorMap &tk,
+                                          const CUtensorMap &tv, const TcParams &p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -644,54 +644,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             const bool full = rok && nv == BN;
             uint32_t sr[64];
             tmem_ld64(tlane + TM_S(q, bf), sr);
-            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (full) {
+            // E4M3 fast path, taken when every row of the warp has a full tile and a reference
+            // max already: the exponentials run against the reference max while the tile max
+            // is taken in the same pass. A tile whose max rose more than 2^LAZY above the
+            // reference (after a row's first tiles, rare) is redone by the general path below,
+            // which grows the reference and rescales O; its P stores overwrite these. (With
+            // E4M3 products the softmax is the longer side of the S -> P -> P V -> S cycle, so
+            // the pass saved shows; the bf16 kernel is bound by the product issue and keeps
+            // the two-pass form, measured no slower.)
+            bool done = false;
+            if (F8 && __all_sync(0xffffffffu, full && m != -INFINITY)) {
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(PBIAS - m, PBIAS - m);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mx[i & 3] = fmax3(mx[i & 3], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
-            } else if (rok) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
-            }
-            const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            const float mnew = rok ? fmaxf(m, mt * sl2) : m;
-            // grow the reference max only when it rose by more than 2^LAZY (lazy rescale)
-            const bool need = rok && mnew > m + LAZY;
-            const float muse = need ? mnew : m;
-            const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-            // rescale O (warp-wide TMEM traffic, so the warp takes the branch together) once
-            // the previous P V of this sub-tile, which accumulates into O, has completed. The
-            // one before it has: S of this tile was issued behind it and has completed, so
-            // the phase awaited here is the current or the next one, never older.
-            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
-                if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
-                fence_after_sync();
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t orow[32];
-                    tmem_ld32(tlane + TM_O(q) + c * 32, orow);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-                    tmem_st32(tlane + TM_O(q) + c * 32, orow);
-                }
-            }
-            // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) or E4M3
-            // quads (key 4i in the low byte) go to the first 32 or 16 columns of the S buffer.
-            // `full` and `rok` differ between lanes whose rows straddle a frame boundary, so
-            // only the arithmetic branches on them; every tcgen05.ld / st stays warp-uniform.
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
-            float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(PBIAS - muse, PBIAS - muse);
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                if constexpr (F8) {
-                    uint32_t pk[8];
-                    if (full) {
+                for (int c = 0; c < 2; ++c) {
+                    if constexpr (F8) {
+                        uint32_t pk[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int col = c * 32 + 4 * i;
+                            mx[i & 1] = fmax3(mx[i & 1], __uint_as_float(sr[col]), __uint_as_float(sr[col + 1]));
+                            mx[2 + (i & 1)] = fmax3(mx[2 + (i & 1)], __uint_as_float(sr[col + 2]), __uint_as_float(sr[col + 3]));
                             const float2 xa = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2x2, nm2);
                             const float2 xb = ffma2(make_float2(__uint_as_float(sr[col + 2]), __uint_as_float(sr[col + 3])), sl2x2, nm2);
                             const float2 pa = make_float2(ex2(xa.x), ex2(xa.y));
@@ -700,50 +674,127 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                             ps2[1] = fadd2(ps2[1], pb);
                             pk[i] = pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
                         }
+                        tmem_st8(tlane + TM_S(q, bf) + c * 8, pk);
                     } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float pv[4];
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const int col = c * 32 + 4 * i + t;
-                                pv[t] = rok && col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, PBIAS - muse)) : 0.f;
-                            }
-                            ps[i & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-                            pk[i] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
-                        }
-                    }
-                    __syncwarp();                       // reconverge before .sync.aligned
-                    tmem_st8(tlane + TM_S(q, bf) + c * 8, pk);
-                } else {
-                    uint32_t pk[16];
-                    if (full) {
+                        uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float2 x = ffma2(make_float2(__uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1])), sl2x2, nm2);
+                            const int col = c * 32 + 2 * i;
+                            mx[i & 3] = fmax3(mx[i & 3], __uint_as_float(sr[col]), __uint_as_float(sr[col + 1]));
+                            const float2 x = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2x2, nm2);
                             const float2 pp = make_float2(ex2(x.x), ex2(x.y));
                             ps2[i & 1] = fadd2(ps2[i & 1], pp);
                             pk[i] = pack_bf16(pp.x, pp.y);
                         }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int col = c * 32 + 2 * i;
-                            float p0 = 0.f, p1 = 0.f;
-                            if (rok) {
-                                p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, -muse)) : 0.f;
-                                p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), sl2, -muse)) : 0.f;
-                            }
-                            ps[i & 3] += p0 + p1;
-                            pk[i] = pack_bf16(p0, p1);
-                        }
+                        tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
                     }
-                    __syncwarp();                       // reconverge before .sync.aligned
-                    tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
                 }
+                const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                done = __all_sync(0xffffffffu, !(mt * sl2 > m + LAZY));
+                if (done) lsum += (ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y);
             }
-            lsum = lsum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y)));
-            m = muse;
+            if (!done) {
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if (full) {
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        mx[i & 3] = fmax3(mx[i & 3], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+                } else if (rok) {
+    #pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        mx[i & 3] = fmaxf(mx[i & 3], i < nv ? __uint_as_float(sr[i]) : -INFINITY);
+                }
+                const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                const float mnew = rok ? fmaxf(m, mt * sl2) : m;
+                // grow the reference max only when it rose by more than 2^LAZY (lazy rescale)
+                const bool need = rok && mnew > m + LAZY;
+                const float muse = need ? mnew : m;
+                const float alpha = (need && m != -INFINITY) ? ex2(m - mnew) : 1.f;
+                // rescale O (warp-wide TMEM traffic, so the warp takes the branch together) once
+                // the previous P V of this sub-tile, which accumulates into O, has completed. The
+                // one before it has: S of this tile was issued behind it and has completed, so
+                // the phase awaited here is the current or the next one, never older.
+                if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+                    fence_after_sync();
+    #pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t orow[32];
+                        tmem_ld32(tlane + TM_O(q) + c * 32, orow);
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                        tmem_st32(tlane + TM_O(q) + c * 32, orow);
+                    }
+                }
+                // exponentials 32 keys at a time; bf16 pairs (key 2i in the low half) or E4M3
+                // quads (key 4i in the low byte) go to the first 32 or 16 columns of the S buffer.
+                // `full` and `rok` differ between lanes whose rows straddle a frame boundary, so
+                // only the arithmetic branches on them; every tcgen05.ld / st stays warp-uniform.
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(PBIAS - muse, PBIAS - muse);
+    #pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    if constexpr (F8) {
+                        uint32_t pk[8];
+                        if (full) {
+    #pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int col = c * 32 + 4 * i;
+                                const float2 xa = ffma2(make_float2(__uint_as_float(sr[col]), __uint_as_float(sr[col + 1])), sl2x2, nm2);
+                                const float2 xb = ffma2(make_float2(__uint_as_float(sr[col + 2]), __uint_as_float(sr[col + 3])), sl2x2, nm2);
+                                const float2 pa = make_float2(ex2(xa.x), ex2(xa.y));
+                                const float2 pb = make_float2(ex2(xb.x), ex2(xb.y));
+                                ps2[0] = fadd2(ps2[0], pa);
+                                ps2[1] = fadd2(ps2[1], pb);
+                                pk[i] = pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
+                            }
+                        } else {
+    #pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float pv[4];
+    #pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const int col = c * 32 + 4 * i + t;
+                                    pv[t] = rok && col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, PBIAS - muse)) : 0.f;
+                                }
+                                ps[i & 3] += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+                                pk[i] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+                            }
+                        }
+                        __syncwarp();                       // reconverge before .sync.aligned
+                        tmem_st8(tlane + TM_S(q, bf) + c * 8, pk);
+                    } else {
+                        uint32_t pk[16];
+                        if (full) {
+    #pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float2 x = ffma2(make_float2(__uint_as_float(sr[c * 32 + 2 * i]), __uint_as_float(sr[c * 32 + 2 * i + 1])), sl2x2, nm2);
+                                const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                                ps2[i & 1] = fadd2(ps2[i & 1], pp);
+                                pk[i] = pack_bf16(pp.x, pp.y);
+                            }
+                        } else {
+    #pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int col = c * 32 + 2 * i;
+                                float p0 = 0.f, p1 = 0.f;
+                                if (rok) {
+                                    p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), sl2, -muse)) : 0.f;
+                                    p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), sl2, -muse)) : 0.f;
+                                }
+                                ps[i & 3] += p0 + p1;
+                                pk[i] = pack_bf16(p0, p1);
+                            }
+                        }
+                        __syncwarp();                       // reconverge before .sync.aligned
+                        tmem_st16(tlane + TM_S(q, bf) + c * 16, pk);
+                    }
+                }
+                lsum = lsum * alpha + (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y)));
+                m = muse;
+            }
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PFULL + 2 * q + bf));
@@ -799,6 +850,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     }
 }
 
+__global__ void __launch_bounds__(THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+               const __grid_constant__ CUtensorMap tv, const TcParams p)
+{
+    attn_body<false>(tq, tk, tv, p);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+attn_fp8_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const TcParams p)
+{
+    attn_body<true>(tq, tk, tv, p);
+}
+
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
@@ -834,11 +899,11 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     p.o = (__nv_bfloat16 *)a.o;
     p.err = a.err;
     if (F8 && (!p.qs || !p.ks || !p.vs)) return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(attn_tc_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES);
+    auto kern = F8 ? attn_fp8_kernel : attn_tc_kernel;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
-    attn_tc_kernel<F8><<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
+    kern<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
     return cudaGetLastError();
 }
 

@@ -104,3 +104,28 @@ def test_stream_create_validates_before_allocating(lib):
     assert lib.hlta_stream_create(ctypes.byref(out), 1, 1, 1, 1, 16, 128, 3, 4, 6, 32, 0.0,
                                   h.HLTA_BF16, None) == h.HLTA_ERR_UNSUPPORTED
     assert out.value is None
+
+
+def test_fp8_entry_points_validate_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(264)
+    q = lib.hlta_fp8_quantize_rows
+    assert q(None, None, 1, 1, 100, 128, 100, 64, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert q(p, None, 1, 1, 100, 64, 100, 64, p, p, None) == h.HLTA_ERR_UNSUPPORTED
+    assert q(p, None, 1, 1, 100, 128, 100, 0, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert q(p, None, 1, 1, 100, 128, 100, 129, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert q(p, None, 1, 1, 100, 128, 0, 64, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert q(p, odd, 1, 1, 100, 128, 100, 64, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert q(p, None, -1, 1, 100, 128, 100, 64, p, p, None) == h.HLTA_ERR_INVALID_ARG
+    c = lib.hlta_fp8_quantize_channels
+    assert c(p, 1, 1, 100, 128, None, p, None) == h.HLTA_ERR_INVALID_ARG
+    assert c(p, 1, 1, 100, 96, p, p, None) == h.HLTA_ERR_UNSUPPORTED
+    assert c(p, 1, 1, 100, 128, p, odd, None) == h.HLTA_ERR_INVALID_ARG
+    a = lib.hlta_window_fp8_fwd
+    assert a(p, p, p, p, p, None, p, 1, 1, 2, 16, 128, 2, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    assert a(p, p, p, p, p, p, p, 1, 1, 2, 16, 64, 2, 1, 0.0, None) == h.HLTA_ERR_UNSUPPORTED
+    assert a(p, p, p, p, p, p, p, 1, 1, 0, 16, 128, 2, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    assert a(p, p, p, p, p, p, p, 1, 1, 2, 16, 128, 0, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    assert a(p, p, p, p, p, p, p, 1, 1, 2, 16, 128, 2, 0, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    assert a(p, odd, p, p, p, p, p, 1, 1, 2, 16, 128, 2, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
