@@ -569,8 +569,10 @@ def main():
             "fp8_peak_tflops": fp8_peak,
             "attn_bytes": 5 * elems,
             "quantise_and_attn_ms": fp8_ms["quantise_and_attn"],
+            "attn_traffic": (tr["fp8_swa_bytes"] + tr["fp8_dswa_bytes"]) if tr and "fp8_swa_bytes" in tr else None,
             "note": "hlta_window_fp8_fwd for the SWA and DSWA heads back to back on resident E4M3 "
-                    "codes (q, k, v 1 byte, o bf16: attn_bytes), then with the three "
+                    "codes (q, k, v 1 byte, o bf16: attn_bytes; attn_traffic: DRAM bytes of the two "
+                    "launches from the committed ncu summary), then with the three "
                     "quantisations from bf16 in the timed region; peak = measured bf16 burst x 2",
         }
 

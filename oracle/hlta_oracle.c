@@ -32,7 +32,9 @@
  *
  * Parity status: every function here is pinned by tests that do not re-type its
  * formula (brute-force full attention, closed forms, contraction and retrieval
- * invariants); see tests/test_oracle_pins.py.
+ * invariants; for the E4M3 codec and quantisers, PyTorch's float8_e4m3fn conversion,
+ * the round-to-nearest reconstruction bound and lossless cases); see
+ * tests/test_oracle_pins.py and tests/test_oracle_fp8_pins.py.
  */
 #include <math.h>
 #include <stdlib.h>
