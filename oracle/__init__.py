@@ -63,6 +63,9 @@ def _load():
         lib.oracle_fp8_quantize_channels.argtypes = [f32, L_, L_, I_, u8, f32]
         for fn in (lib.oracle_fp8_quantize_rows, lib.oracle_fp8_quantize_channels):
             fn.restype = ctypes.c_int
+        lib.oracle_window_bwd.argtypes = [f32, f32, f32, f32, f64, f64, f64, L_, I_, I_, I_, I_,
+                                          I_, D_]
+        lib.oracle_window_bwd.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -204,6 +207,26 @@ def hybrid(q, k, v, a, b, Hs: int, Hd: int, Hg: int, T: int, N: int,
             og, S_fin = gdn_raw(qf[:, s], kf[:, s], vf[:, s], a, b, raw, S0)
         o[:, s] = og
     return o, S_fin
+
+
+def window_bwd(q, k, v, dO, T: int, N: int, w: int, r: int = 1, scale=None):
+    """Gradients (dq, dk, dv) of the windowed attention (SWA for r == 1, DSWA otherwise) for
+    the upstream gradient dO, float64 [..., L, d] each."""
+    qf, kf, vf, gf = _f32(q), _f32(k), _f32(v), _f32(dO)
+    d = qf.shape[-1]
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    assert qf.shape[-2] == T * N, "q must hold T*N rows"
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = [np.empty(qf.shape, dtype=np.float64) for _ in range(3)]
+    rc = _load().oracle_window_bwd(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                                   _ptr(vf, ctypes.c_float), _ptr(gf, ctypes.c_float),
+                                   *(_ptr(o, ctypes.c_double) for o in out), BH, T, N, d, w, r,
+                                   float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle window_bwd failed ({rc})")
+    return tuple(out)
 
 
 def e4m3_decode(code: int) -> float:

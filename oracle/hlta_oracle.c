@@ -413,6 +413,94 @@ int oracle_fp8_quantize_channels(const float *x, long BH, long L, int d, unsigne
     return 0;
 }
 
+/*
+ * Backward pass of the windowed attention (training: the backbone is trained from scratch,
+ * related-papers analysis row E). Reverse-mode derivative of o_i = sum_j p_ij v_j,
+ * p_ij = softmax_j(scale q_i . k_j) over the keys of row i's window frames, for a given
+ * upstream gradient dO, written out per query row:
+ *   dP_ij = dO_i . v_j,  D_i = sum_j p_ij dP_ij,  dS_ij = p_ij (dP_ij - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j += scale dS_ij q_i,  dv_j += p_ij dO_i.
+ * q, k, v, dO: [BH][L][d] float32; dq, dk, dv: [BH][L][d] double (overwritten).
+ * Heads run in parallel; the rows of a head run in order (dk, dv accumulate).
+ */
+static int window_backward(const float *q, const float *k, const float *v, const float *dO,
+                           double *dq, double *dk, double *dv, long BH, int T, int N, int d,
+                           int w, int r, int dilated, double scale)
+{
+    if (BH <= 0 || T <= 0 || N <= 0 || d <= 0 || w <= 0 || r <= 0) return 1;
+    long L = (long)T * N;
+    int err = 0;
+    for (long i = 0; i < BH * L * d; ++i) dq[i] = dk[i] = dv[i] = 0.0;
+#pragma omp parallel
+    {
+        int *frames = (int *)malloc(sizeof(int) * (size_t)w);
+        double *pz = (double *)malloc(sizeof(double) * (size_t)w * (size_t)N);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)w * (size_t)N);
+        if (!frames || !pz || !dp) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                const float *Q = q + bh * L * d, *K = k + bh * L * d, *V = v + bh * L * d;
+                const float *G = dO + bh * L * d;
+                double *DQ = dq + bh * L * d, *DK = dk + bh * L * d, *DV = dv + bh * L * d;
+                for (long l = 0; l < L; ++l) {
+                    int f = (int)(l / N);
+                    int nf = dilated ? dswa_key_frames(f, w, r, frames) : swa_key_frames(f, w, frames);
+                    int nk = nf * N;
+                    double m = -INFINITY;
+                    for (int i = 0; i < nf; ++i)
+                        for (int n = 0; n < N; ++n) {
+                            long kr = (long)frames[i] * N + n;
+                            double s = 0.0;
+                            for (int c = 0; c < d; ++c) s += (double)Q[l * d + c] * (double)K[kr * d + c];
+                            s *= scale;
+                            pz[(long)i * N + n] = s;
+                            if (s > m) m = s;
+                        }
+                    double den = 0.0;
+                    for (int j = 0; j < nk; ++j) {
+                        pz[j] = exp(pz[j] - m);
+                        den += pz[j];
+                    }
+                    double Dsum = 0.0;
+                    for (int i = 0; i < nf; ++i)
+                        for (int n = 0; n < N; ++n) {
+                            long j = (long)i * N + n, kr = (long)frames[i] * N + n;
+                            pz[j] /= den;
+                            double g = 0.0;
+                            for (int c = 0; c < d; ++c) g += (double)G[l * d + c] * (double)V[kr * d + c];
+                            dp[j] = g;
+                            Dsum += pz[j] * g;
+                        }
+                    for (int i = 0; i < nf; ++i)
+                        for (int n = 0; n < N; ++n) {
+                            long j = (long)i * N + n, kr = (long)frames[i] * N + n;
+                            double ds = pz[j] * (dp[j] - Dsum);
+                            for (int c = 0; c < d; ++c) {
+                                DQ[l * d + c] += scale * ds * (double)K[kr * d + c];
+                                DK[kr * d + c] += scale * ds * (double)Q[l * d + c];
+                                DV[kr * d + c] += pz[j] * (double)G[l * d + c];
+                            }
+                        }
+                }
+            }
+        }
+        free(frames);
+        free(pz);
+        free(dp);
+    }
+    return err;
+}
+
+int oracle_window_bwd(const float *q, const float *k, const float *v, const float *dO,
+                      double *dq, double *dk, double *dv, long BH, int T, int N, int d, int w,
+                      int r, double scale)
+{
+    return window_backward(q, k, v, dO, dq, dk, dv, BH, T, N, d, w, r, r > 1, scale);
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
