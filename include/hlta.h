@@ -138,6 +138,35 @@ hlta_status hlta_window_fp8_fwd(const void *q8, const float *q_scales, const voi
                                 float scale, void *stream);
 
 /*
+ * Training pair of the windowed attention (the backbone is trained from scratch: related-papers
+ * analysis, row E). hlta_window_fwd_lse is hlta_dswa_fwd (bf16, d = 128; r = 1 gives SWA) that
+ * also writes lse [B, H, T*N] float32 (device): the natural log-sum-exp of each query row's
+ * scaled scores over its window keys, the softmax normaliser the backward pass reuses.
+ */
+hlta_status hlta_window_fwd_lse(const void *q, const void *k, const void *v, void *o,
+                                float *lse, int B, int H, int T, int N, int d, int w, int r,
+                                float scale, void *stream);
+
+/* Workspace bytes of hlta_window_bwd: one float per query row (B*H*T*N*4, 256-byte rounded). */
+size_t hlta_window_bwd_workspace_bytes(int B, int H, int T, int N);
+
+/*
+ * Backward pass of the windowed attention: the reverse-mode derivative of o = softmax(scale
+ * q k^T over the window) v for the upstream gradient dO:
+ *   D_i = dO_i . o_i,  p_ij = exp(scale q_i.k_j - lse_i),  dS_ij = p_ij (dO_i.v_j - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,  dv_j = sum_i p_ij dO_i.
+ * q, k, v, o, dO, dq, dk, dv: [B, H, T*N, d] bf16 device (d = 128); o and lse as written by
+ * hlta_window_fwd_lse with the same q, k, v, w, r, scale. dq, dk, dv are overwritten.
+ * workspace: device scratch of at least hlta_window_bwd_workspace_bytes(...), caller-owned,
+ * 16-byte aligned. Enqueued on `stream` (three launches). Errors as hlta_swa_fwd, plus
+ * HLTA_ERR_INVALID_ARG for a short workspace.
+ */
+hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const void *o,
+                            const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                            int B, int H, int T, int N, int d, int w, int r, float scale,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens.
  */
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt);

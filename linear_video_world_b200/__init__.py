@@ -58,6 +58,9 @@ def _load() -> ctypes.CDLL:
         "hlta_fp8_quantize_rows": (I, [P, P, I, I, L, I, L, I, P, P, P]),
         "hlta_fp8_quantize_channels": (I, [P, I, I, L, I, P, P, P]),
         "hlta_window_fp8_fwd": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
+        "hlta_window_fwd_lse": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
+        "hlta_window_bwd_workspace_bytes": (Z, [I, I, I, I]),
+        "hlta_window_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
         "hlta_set_profile_events": (I, [ctypes.POINTER(P)]),
     }
@@ -214,6 +217,27 @@ def hlta_window_fp8_fwd(q8, qs, k8, ks, v8, vs, o, B, H, T, N, d, w, r, scale=0.
                                     T, N, d, w, r, float(scale), _stream(stream)))
 
 
+def hlta_window_fwd_lse(q, k, v, o, lse, B, H, T, N, d, w, r, scale=0.0, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse")):
+        _need(t, n)
+    _check(_lib.hlta_window_fwd_lse(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, T, N, d, w, r,
+                                    float(scale), _stream(stream)))
+
+
+def hlta_window_bwd_workspace_bytes(B, H, T, N) -> int:
+    return int(_lib.hlta_window_bwd_workspace_bytes(B, H, T, N))
+
+
+def hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale, workspace,
+                    stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dO, "dO"), (dq, "dq"),
+                 (dk, "dk"), (dv, "dv"), (workspace, "workspace")):
+        _need(t, n)
+    _check(_lib.hlta_window_bwd(_p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(dq), _p(dk),
+                                _p(dv), B, H, T, N, d, w, r, float(scale), _p(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def hlta_device_status(stream=None) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
@@ -291,6 +315,28 @@ def window_fp8(q8, qs, k8, ks, v8, vs, T, N, w, r=1, scale=0.0, out=None, stream
     o = torch.empty((B, H, L, d), dtype=torch.bfloat16, device=q8.device) if out is None else out
     hlta_window_fp8_fwd(q8, qs, k8, ks, v8, vs, o, B, H, T, N, d, w, r, scale, stream)
     return o
+
+
+def window_fwd_lse(q, k, v, T, N, w, r=1, scale=0.0, out=None, lse=None, stream=None):
+    """Window attention forward that also returns the per-row log-sum-exp (for the backward)."""
+    import torch
+    B, H, L, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    ls = torch.empty((B, H, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    hlta_window_fwd_lse(q, k, v, o, ls, B, H, T, N, d, w, r, scale, stream)
+    return o, ls
+
+
+def window_bwd(q, k, v, o, lse, dO, T, N, w, r=1, scale=0.0, grads=None, workspace=None,
+               stream=None):
+    """Gradients (dq, dk, dv) of the window attention for the upstream gradient dO."""
+    import torch
+    B, H, L, d = q.shape
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q) for _ in range(3))
+    ws = workspace if workspace is not None else _workspace(
+        hlta_window_bwd_workspace_bytes(B, H, T, N), q.device)
+    hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale, ws, stream)
+    return dq, dk, dv
 
 
 def gdn(q, k, v, a, b, S0=None, chunk=64, out=None, S_out=None, workspace=None, stream=None):

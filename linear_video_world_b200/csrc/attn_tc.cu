@@ -102,6 +102,7 @@ struct TcParams {
     float sl2;                  // softmax scale * log2(e)
     const float *qs, *ks, *vs;  // E4M3 scales: [heads][nqb], [heads][nkb], [heads][128]
     int nqb, nkb;               // per head: query blocks of 128 rows, key tiles (slot * tpf + tile)
+    float *lse;                 // per query row log-sum-exp (natural log) of its scores, or null
     __nv_bfloat16 *o;
     unsigned int *err;
 };
@@ -808,6 +809,9 @@ __device__ __forceinline__ void attn_body(const CUtensorMap &tq, const CUtensorM
         if (fin) {
             fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            // the softmax normaliser for the backward pass: scores s, P = 2^(s sl2 - m) / lsum,
+            // so log sum exp(s scale) = (m + log2(lsum)) ln 2 (the bf16 kernel only: PBIAS = 0)
+            if (!F8 && p.lse && row_valid) p.lse[q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
             __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
             const float4 *vsc = F8 ? reinterpret_cast<const float4 *>(p.vs + (long)kvh * D) : nullptr;
 #pragma unroll
@@ -894,6 +898,7 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0;
     p.sl2 = a.scale * 1.4426950408889634f;
     p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
+    p.lse = a.lse;
     p.nqb = (int)((a.q_rows + BM - 1) / BM);
     p.nkb = a.kv_slots * ((a.N + BN - 1) / BN);
     p.o = (__nv_bfloat16 *)a.o;

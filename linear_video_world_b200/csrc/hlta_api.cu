@@ -320,6 +320,63 @@ hlta_status hlta_window_fp8_fwd(const void *q8, const float *q_scales, const voi
     return HLTA_OK;
 }
 
+hlta_status hlta_window_fwd_lse(const void *q, const void *k, const void *v, void *o,
+                                float *lse, int B, int H, int T, int N, int d, int w, int r,
+                                float scale, void *stream)
+{
+    hlta_status st;
+    if (!lse || !aligned16(lse)) return fail(HLTA_ERR_INVALID_ARG, "lse must be a 16-byte aligned device pointer");
+    if (!q || !k || !v || !o) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 0 || H < 0 || T < 1 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d T=%d N=%d", B, H, T, N);
+    if ((long)T * N > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "T*N too large");
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "training attention supports bf16, d = 128 only (got %d)", d);
+    if ((st = check_window(w, r)) != HLTA_OK) return st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    AttnArgs a = clip_attn_args(q, k, v, o, B, H, 0, H, T, N, d, w, r, scale, ctx->err);
+    a.lse = lse;
+    return run_attn(a, HLTA_BF16, (cudaStream_t)stream);
+}
+
+size_t hlta_window_bwd_workspace_bytes(int B, int H, int T, int N)
+{
+    if (B < 0 || H < 0 || T < 0 || N < 0) return 0;
+    return (((size_t)B * H * T * N * sizeof(float)) + 255) & ~(size_t)255;
+}
+
+hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const void *o,
+                            const float *lse, const void *dO, void *dq, void *dk, void *dv,
+                            int B, int H, int T, int N, int d, int w, int r, float scale,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
+    hlta_status st;
+    const void *ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, workspace};
+    for (const void *p : ptrs) {
+        if (!p) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+        if (!aligned16(p)) return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    }
+    if (B < 0 || H < 0 || T < 1 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d T=%d N=%d", B, H, T, N);
+    if ((long)T * N > (1L << 30)) return fail(HLTA_ERR_INVALID_ARG, "T*N too large");
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "attention backward supports bf16, d = 128 only (got %d)", d);
+    if ((st = check_window(w, r)) != HLTA_OK) return st;
+    if (workspace_bytes < hlta_window_bwd_workspace_bytes(B, H, T, N))
+        return fail(HLTA_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)", workspace_bytes,
+                    hlta_window_bwd_workspace_bytes(B, H, T, N));
+    if (B * H == 0) return HLTA_OK;
+    AttnBwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO; a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.Dws = (float *)workspace;
+    a.BH = B * H; a.T = T; a.N = N; a.w = w; a.r = r;
+    a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+    cudaError_t e = launch_attn_bwd(a, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "attention backward: unsupported shape");
+    if (e != cudaSuccess) return cuda_fail(e, "attention backward launch");
+    return HLTA_OK;
+}
+
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt)
 {
     if (B < 0 || H < 0 || L < 0 || d < 1 || chunk != 64) return 0;

@@ -30,6 +30,9 @@ struct AttnArgs {
     // E4M3 inputs only: fp32 scales of the query blocks ([B*q_Htot][ceil(q_rows/128)]), the
     // key tiles ([B*kv_Htot][kv_slots][ceil(N/64)]) and the value channels ([B*kv_Htot][d])
     const float *qs = nullptr, *ks = nullptr, *vs = nullptr;
+    // bf16 kernel only: per query row log-sum-exp (natural log) of the scaled scores
+    // ([B*q_Htot][q_rows] float32), written when non-null
+    float *lse = nullptr;
 };
 
 // Gated delta rule over [B][Htot][L][d] tensors, this branch's heads at h0 .. h0 + Hg.
@@ -88,6 +91,17 @@ cudaError_t launch_fp8_quantize_rows(const void *x, const float *shift, long BH,
                                      cudaStream_t s);
 cudaError_t launch_fp8_quantize_channels(const void *x, long BH, long L, void *x8,
                                          float *scales, cudaStream_t s);
+// Window attention backward (bf16, d = 128): D = rowsum(dO o O) into `Dws` ([BH][L] fp32),
+// then dq (query-tile major) and dk, dv (key-tile major).
+struct AttnBwdArgs {
+    const void *q, *k, *v, *o, *dO;
+    const float *lse;
+    void *dq, *dk, *dv;
+    float *Dws;
+    int BH, T, N, w, r;
+    float scale;
+};
+cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,

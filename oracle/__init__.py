@@ -66,6 +66,8 @@ def _load():
         lib.oracle_window_bwd.argtypes = [f32, f32, f32, f32, f64, f64, f64, L_, I_, I_, I_, I_,
                                           I_, D_]
         lib.oracle_window_bwd.restype = ctypes.c_int
+        lib.oracle_window_lse.argtypes = [f32, f32, f64, L_, I_, I_, I_, I_, I_, D_]
+        lib.oracle_window_lse.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -227,6 +229,22 @@ def window_bwd(q, k, v, dO, T: int, N: int, w: int, r: int = 1, scale=None):
     if rc != 0:
         raise RuntimeError(f"oracle window_bwd failed ({rc})")
     return tuple(out)
+
+
+def window_lse(q, k, T: int, N: int, w: int, r: int = 1, scale=None) -> np.ndarray:
+    """Natural log-sum-exp of each query row's scaled scores over its window keys, [..., L]."""
+    qf, kf = _f32(q), _f32(k)
+    d = qf.shape[-1]
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    out = np.empty(qf.shape[:-1], dtype=np.float64)
+    rc = _load().oracle_window_lse(_ptr(qf, ctypes.c_float), _ptr(kf, ctypes.c_float),
+                                   _ptr(out, ctypes.c_double), BH, T, N, d, w, r, float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle window_lse failed ({rc})")
+    return out
 
 
 def e4m3_decode(code: int) -> float:

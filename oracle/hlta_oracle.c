@@ -501,6 +501,49 @@ int oracle_window_bwd(const float *q, const float *k, const float *v, const floa
     return window_backward(q, k, v, dO, dq, dk, dv, BH, T, N, d, w, r, r > 1, scale);
 }
 
+/* Log-sum-exp of each query row's scaled scores over its window keys (natural log): the
+ * softmax normaliser the backward pass reuses. q, k: [BH][L][d] float32; lse: [BH][L]. */
+int oracle_window_lse(const float *q, const float *k, double *lse, long BH, int T, int N, int d,
+                      int w, int r, double scale)
+{
+    if (BH <= 0 || T <= 0 || N <= 0 || d <= 0 || w <= 0 || r <= 0) return 1;
+    long L = (long)T * N;
+    int err = 0;
+#pragma omp parallel
+    {
+        int *frames = (int *)malloc(sizeof(int) * (size_t)w);
+        double *z = (double *)malloc(sizeof(double) * (size_t)w * (size_t)N);
+        if (!frames || !z) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long it = 0; it < BH * L; ++it) {
+                long bh = it / L, l = it % L;
+                int f = (int)(l / N);
+                int nf = r > 1 ? dswa_key_frames(f, w, r, frames) : swa_key_frames(f, w, frames);
+                const float *K = k + bh * L * d;
+                double m = -INFINITY;
+                for (int i = 0; i < nf; ++i)
+                    for (int n = 0; n < N; ++n) {
+                        const float *krow = K + ((long)frames[i] * N + n) * d;
+                        double s = 0.0;
+                        for (int c = 0; c < d; ++c) s += (double)q[it * d + c] * (double)krow[c];
+                        s *= scale;
+                        z[(long)i * N + n] = s;
+                        if (s > m) m = s;
+                    }
+                double den = 0.0;
+                for (int j = 0; j < nf * N; ++j) den += exp(z[j] - m);
+                lse[it] = m + log(den);
+            }
+        }
+        free(frames);
+        free(z);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

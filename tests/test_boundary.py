@@ -129,3 +129,25 @@ def test_fp8_entry_points_validate_on_host(lib):
     assert a(p, p, p, p, p, p, p, 1, 1, 2, 16, 128, 0, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
     assert a(p, p, p, p, p, p, p, 1, 1, 2, 16, 128, 2, 0, 0.0, None) == h.HLTA_ERR_INVALID_ARG
     assert a(p, odd, p, p, p, p, p, 1, 1, 2, 16, 128, 2, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+
+
+def test_attention_backward_entry_points_validate_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    f = lib.hlta_window_fwd_lse
+    assert f(p, p, p, p, None, 1, 1, 2, 16, 128, 2, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    assert f(p, p, p, p, p, 1, 1, 2, 16, 64, 2, 1, 0.0, None) == h.HLTA_ERR_UNSUPPORTED
+    assert f(p, p, p, p, p, 1, 1, 2, 16, 128, 0, 1, 0.0, None) == h.HLTA_ERR_INVALID_ARG
+    ws = lib.hlta_window_bwd_workspace_bytes(2, 3, 4, 100)
+    assert ws == (2 * 3 * 4 * 100 * 4 + 255) // 256 * 256
+    b = lib.hlta_window_bwd
+    args = [p] * 9 + [2, 3, 4, 100, 128, 2, 1, 0.0, p, ws, None]
+    bad = list(args); bad[4] = None
+    assert b(*bad) == h.HLTA_ERR_INVALID_ARG
+    bad = list(args); bad[18] = ws - 1
+    assert b(*bad) == h.HLTA_ERR_INVALID_ARG
+    assert b"workspace" in lib.hlta_last_error()
+    bad = list(args); bad[13] = 96
+    assert b(*bad) == h.HLTA_ERR_UNSUPPORTED
+    bad = list(args); bad[7] = ctypes.c_void_p(264)
+    assert b(*bad) == h.HLTA_ERR_INVALID_ARG

@@ -52,3 +52,17 @@ def test_window_bwd_invariants(orc):
     dq, dk, dv = orc.window_bwd(q, k, v, g, T, N, w, r)
     assert np.abs(dk.sum(axis=1)).max() < 1e-12
     assert np.abs(dv.sum(axis=1) - g.astype(np.float64).sum(axis=1)).max() < 1e-12
+
+
+@pytest.mark.parametrize("T,N,d,w,r", [(3, 4, 6, 2, 1), (7, 3, 5, 3, 2)])
+def test_window_lse_matches_dense_logsumexp(orc, T, N, d, w, r):
+    rng = np.random.default_rng(3 + r)
+    q, k = (rng.standard_normal((2, T * N, d)).astype(np.float32) for _ in range(2))
+    got = orc.window_lse(q, k, T, N, w, r)
+    allowed = _allowed(T, N, w, r)
+    for b in range(2):
+        s = (q[b].astype(np.float64) @ k[b].astype(np.float64).T) / math.sqrt(d)
+        s = np.where(allowed, s, -np.inf)
+        m = s.max(axis=1)
+        ref = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        assert np.abs(got[b] - ref).max() < 1e-12
