@@ -68,6 +68,9 @@ def _load():
         lib.oracle_window_bwd.restype = ctypes.c_int
         lib.oracle_window_lse.argtypes = [f32, f32, f64, L_, I_, I_, I_, I_, I_, D_]
         lib.oracle_window_lse.restype = ctypes.c_int
+        lib.oracle_gdn_bwd.argtypes = [f32, f32, f32, f32, f32, f64, f32, f64, f64, f64, f64, f64,
+                                       f64, f64, L_, L_, I_]
+        lib.oracle_gdn_bwd.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -158,6 +161,37 @@ def gdn(q, k, v, a, b, S0=None, history: bool = False):
     if rc != 0:
         raise RuntimeError(f"oracle gdn failed ({rc})")
     return (o, S_out, hist) if history else (o, S_out)
+
+
+def gdn_bwd(q, k, v, a, b, dO, S0=None, dS_final=None):
+    """Gradients of the gated delta rule for the upstream gradients dO (of every output) and
+    dS_final (of the final state, or None for zero). Returns (dq, dk, dv, da, db, dS0), float64:
+    dq, dk, dv [..., L, d]; da, db [..., L]; dS0 [..., d, d]."""
+    qf, kf, vf, af, bf, gf = _f32(q), _f32(k), _f32(v), _f32(a), _f32(b), _f32(dO)
+    d = qf.shape[-1]
+    L = qf.shape[-2]
+    lead = qf.shape[:-2]
+    BH = int(np.prod(lead)) if lead else 1
+
+    def dmat(x):
+        if x is None:
+            return None
+        if hasattr(x, "detach"):
+            x = x.detach().cpu().double().numpy()
+        return np.ascontiguousarray(np.asarray(x, dtype=np.float64)).reshape(BH, d, d)
+
+    S0d, dSd = dmat(S0), dmat(dS_final)
+    dq, dk, dv = (np.empty(qf.shape, dtype=np.float64) for _ in range(3))
+    da, db = (np.empty(qf.shape[:-1], dtype=np.float64) for _ in range(2))
+    dS0 = np.empty(lead + (d, d), dtype=np.float64)
+    rc = _load().oracle_gdn_bwd(*(_ptr(x, ctypes.c_float) for x in (qf, kf, vf, af, bf)),
+                                _ptr(S0d, ctypes.c_double), _ptr(gf, ctypes.c_float),
+                                _ptr(dSd, ctypes.c_double),
+                                *(_ptr(x, ctypes.c_double) for x in (dq, dk, dv, da, db, dS0)),
+                                BH, L, d)
+    if rc != 0:
+        raise RuntimeError(f"oracle gdn_bwd failed ({rc})")
+    return dq, dk, dv, da, db, dS0
 
 
 def gdn_raw(q, k, v, x, y, c: float, S0=None):

@@ -544,6 +544,107 @@ int oracle_window_lse(const float *q, const float *k, double *lse, long BH, int 
     return err;
 }
 
+/*
+ * Backward pass of the gated delta rule: reverse-mode derivative of the token recurrence of
+ * oracle_gdn (S_t = a_t S_{t-1} (I - b_t k_t k_t^T) + b_t v_t k_t^T, o_t = S_t q_t) for the
+ * upstream gradients dO (of every o_t) and dSL (of the final state, or NULL for zero). With
+ * G the gradient of the current state, walking t = L-1 .. 0:
+ *   G += dO_t q_t^T;  dq_t = S_t^T dO_t;  sk = S_{t-1} k_t;  gk = G k_t;
+ *   dv_t = b_t gk;  db_t = gk . (v_t - a_t sk);  da_t = <G, S_{t-1}> - b_t gk . sk;
+ *   dk_t = -a_t b_t (S_{t-1}^T gk + G^T sk) + b_t G^T v_t;  G <- a_t (G - b_t gk k_t^T)
+ * and dS0 = G at the end. The forward states are recomputed and kept per head.
+ * Inputs as oracle_gdn; dq, dk, dv: [BH][L][d], da, db: [BH][L], dS0: [BH][d][d] (or NULL).
+ */
+int oracle_gdn_bwd(const float *q, const float *k, const float *v, const float *a,
+                   const float *b, const double *S0, const float *dO, const double *dSL,
+                   double *dq, double *dk, double *dv, double *da, double *db, double *dS0,
+                   long BH, long L, int d)
+{
+    if (BH <= 0 || L < 0 || d <= 0) return 1;
+    int err = 0;
+    const size_t dd = (size_t)d * d;
+#pragma omp parallel
+    {
+        double *hist = (double *)malloc(sizeof(double) * dd * (size_t)(L + 1));
+        double *G = (double *)malloc(sizeof(double) * dd);
+        double *sk = (double *)malloc(sizeof(double) * (size_t)d);
+        double *gk = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!hist || !G || !sk || !gk) {
+#pragma omp atomic write
+            err = 2;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (long bh = 0; bh < BH; ++bh) {
+                /* forward: hist[t + 1] = S_t, hist[0] = S0 */
+                if (S0) memcpy(hist, S0 + bh * dd, sizeof(double) * dd);
+                else memset(hist, 0, sizeof(double) * dd);
+                for (long t = 0; t < L; ++t) {
+                    const float *kt = k + (bh * L + t) * d, *vt = v + (bh * L + t) * d;
+                    double at = a[bh * L + t], bt = b[bh * L + t];
+                    const double *Sp = hist + (size_t)t * dd;
+                    double *Sn = hist + (size_t)(t + 1) * dd;
+                    for (int i = 0; i < d; ++i) {
+                        double s = 0.0;
+                        for (int j = 0; j < d; ++j) s += Sp[(long)i * d + j] * (double)kt[j];
+                        for (int j = 0; j < d; ++j)
+                            Sn[(long)i * d + j] = at * (Sp[(long)i * d + j] - bt * s * (double)kt[j])
+                                                  + bt * (double)vt[i] * (double)kt[j];
+                    }
+                }
+                /* backward */
+                if (dSL) memcpy(G, dSL + bh * dd, sizeof(double) * dd);
+                else memset(G, 0, sizeof(double) * dd);
+                for (long t = L - 1; t >= 0; --t) {
+                    const long tt = bh * L + t;
+                    const float *kt = k + tt * d, *vt = v + tt * d, *qt = q + tt * d;
+                    const float *gt = dO + tt * d;
+                    double at = a[tt], bt = b[tt];
+                    const double *Sp = hist + (size_t)t * dd, *St = hist + (size_t)(t + 1) * dd;
+                    for (int i = 0; i < d; ++i)
+                        for (int j = 0; j < d; ++j) G[(long)i * d + j] += (double)gt[i] * (double)qt[j];
+                    for (int j = 0; j < d; ++j) {
+                        double s = 0.0;
+                        for (int i = 0; i < d; ++i) s += St[(long)i * d + j] * (double)gt[i];
+                        dq[tt * d + j] = s;
+                    }
+                    double gs = 0.0, gksk = 0.0, dbt = 0.0;
+                    for (int i = 0; i < d; ++i) {
+                        double s1 = 0.0, s2 = 0.0;
+                        for (int j = 0; j < d; ++j) {
+                            s1 += Sp[(long)i * d + j] * (double)kt[j];
+                            s2 += G[(long)i * d + j] * (double)kt[j];
+                            gs += G[(long)i * d + j] * Sp[(long)i * d + j];
+                        }
+                        sk[i] = s1;
+                        gk[i] = s2;
+                        gksk += s2 * s1;
+                        dbt += s2 * ((double)vt[i] - at * s1);
+                        dv[tt * d + i] = bt * s2;
+                    }
+                    db[tt] = dbt;
+                    da[tt] = gs - bt * gksk;
+                    for (int j = 0; j < d; ++j) {
+                        double s = 0.0;
+                        for (int i = 0; i < d; ++i)
+                            s += -at * bt * (Sp[(long)i * d + j] * gk[i] + G[(long)i * d + j] * sk[i])
+                                 + bt * G[(long)i * d + j] * (double)vt[i];
+                        dk[tt * d + j] = s;
+                    }
+                    for (int i = 0; i < d; ++i)
+                        for (int j = 0; j < d; ++j)
+                            G[(long)i * d + j] = at * (G[(long)i * d + j] - bt * gk[i] * (double)kt[j]);
+                }
+                if (dS0) memcpy(dS0 + bh * dd, G, sizeof(double) * dd);
+            }
+        }
+        free(hist);
+        free(G);
+        free(sk);
+        free(gk);
+    }
+    return err;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP
