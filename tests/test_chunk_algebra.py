@@ -75,3 +75,104 @@ def test_chunk_form_strong_decay_no_overflow(orc):
     o, S = chunk_form(*(x.astype(np.float64) for x in (q, k, v, a, b)), np.zeros((d, d)), 64)
     assert np.all(np.isfinite(o))
     np.testing.assert_allclose(o, o_ref[0], rtol=1e-9, atol=1e-12)
+
+
+# --------------------------------------------------------------------------------------
+# Backward pass in chunk form
+# --------------------------------------------------------------------------------------
+# Reverse-mode derivative of the chunk form above, term by term (derived here from it; the
+# kernels implement the same algebra). Per chunk, with R = diag(b)(V - diag(e^g) K S0^T)
+# (so U = T R), Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K and dS_C the gradient of the
+# chunk's end state:
+#   across chunks (serial, last to first): dS0 = dS_C (gamma I - Kt^T W) + dO^T Qt
+#   within a chunk (parallel):
+#     dU = P^T dO + Kt dS_C^T,  dR = T^T dU,  dA = -(dR U^T) on s < t,  dP = dO U^T on s <= t
+#     dQ = diag(e^g) dO S0 + (dP o Gam) K
+#     dK = (dP o Gam)^T Q + diag(e^{g_C - g}) U dS_C + M K + M^T K - diag(b e^g) dR S0,
+#          M = dA o (b_t e^{g_t - g_s})
+#     dV = diag(b) dR
+#     db = rowsum(dA o Gam o K K^T) + rowsum(dR o (V - diag(e^g) K S0^T))
+#     dg = rowsum - colsum of (dP o P) and of (dA o A) + e^g o rowsum(dO o Q S0^T)
+#          - b e^g o rowsum(dR o K S0^T) - e^{g_C - g} o rowsum(U o K dS_C^T)
+#          + [last token] (gamma <dS_C, S0> + sum_s e^{g_C - g_s} u_s^T dS_C k_s)
+#     d(log a) = reverse running sum of dg inside the chunk;  da = d(log a) / a
+
+def chunk_backward(q, k, v, a, b, S0, dO, dSL, C):
+    L, d = q.shape
+    S = S0.copy()
+    chunks = []
+    for c0 in range(0, L, C):
+        sl = slice(c0, min(L, c0 + C))
+        Q, K, V, G = q[sl], k[sl], v[sl], dO[sl]
+        bb = b[sl]
+        g = np.cumsum(np.log(a[sl]))
+        n = g.size
+        diff = g[:, None] - g[None, :]
+        low = np.tril(np.ones((n, n)), -1)
+        inc = np.tril(np.ones((n, n)))
+        E_low = low * np.exp(np.where(low > 0, diff, 0))
+        Gam = inc * np.exp(np.where(inc > 0, diff, 0))
+        A = bb[:, None] * E_low * (K @ K.T)
+        Tm = np.linalg.solve(np.eye(n) + A, np.eye(n))
+        W = Tm @ ((bb * np.exp(g))[:, None] * K)
+        Up = Tm @ (bb[:, None] * V)
+        P = Gam * (Q @ K.T)
+        Qt = np.exp(g)[:, None] * Q - P @ W
+        Kt = np.exp(g[-1] - g)[:, None] * K
+        chunks.append(dict(sl=sl, Q=Q, K=K, V=V, G=G, b=bb, a=a[sl], g=g, E_low=E_low, Gam=Gam,
+                           A=A, T=Tm, W=W, Up=Up, P=P, Qt=Qt, Kt=Kt, S0=S.copy()))
+        U = Up - W @ S.T
+        S = np.exp(g[-1]) * S + U.T @ Kt
+    dS = np.zeros((d, d)) if dSL is None else dSL.copy()
+    for ch in reversed(chunks):
+        ch["dSC"] = dS.copy()
+        dS = dS @ (np.exp(ch["g"][-1]) * np.eye(d) - ch["Kt"].T @ ch["W"]) + ch["G"].T @ ch["Qt"]
+    dS0 = dS
+    dq, dk, dv = (np.zeros((L, d)) for _ in range(3))
+    da, db = np.zeros(L), np.zeros(L)
+    for ch in chunks:
+        Q, K, V, G, bb, g, S0c, dSC = (ch[x] for x in ("Q", "K", "V", "G", "b", "g", "S0", "dSC"))
+        U = ch["Up"] - ch["W"] @ S0c.T
+        dU = ch["P"].T @ G + ch["Kt"] @ dSC.T
+        dR = ch["T"].T @ dU
+        inc = ch["Gam"] > 0
+        low = ch["E_low"] > 0
+        dP = np.where(inc, G @ U.T, 0.0)
+        dA = np.where(low, -(dR @ U.T), 0.0)
+        eg = np.exp(g)
+        dQc = eg[:, None] * (G @ S0c) + (dP * ch["Gam"]) @ K
+        M = dA * bb[:, None] * ch["E_low"]
+        KS = K @ S0c.T
+        dKc = (dP * ch["Gam"]).T @ Q + np.exp(g[-1] - g)[:, None] * (U @ dSC) + M @ K + M.T @ K \
+            - (bb * eg)[:, None] * (dR @ S0c)
+        dVc = bb[:, None] * dR
+        dbc = (dA * ch["E_low"] * (K @ K.T)).sum(1) + (dR * (V - eg[:, None] * KS)).sum(1)
+        PP, AA = dP * ch["P"], dA * ch["A"]
+        dg = PP.sum(1) - PP.sum(0) + AA.sum(1) - AA.sum(0) + eg * (G * (Q @ S0c.T)).sum(1) \
+            - bb * eg * (dR * KS).sum(1) - np.exp(g[-1] - g) * (U * (K @ dSC.T)).sum(1)
+        dg[-1] += np.exp(g[-1]) * np.sum(dSC * S0c) + np.sum(np.exp(g[-1] - g) * (U * (K @ dSC.T)).sum(1))
+        dlog = np.cumsum(dg[::-1])[::-1]
+        sl = ch["sl"]
+        dq[sl], dk[sl], dv[sl], db[sl], da[sl] = dQc, dKc, dVc, dbc, dlog / ch["a"]
+    return dq, dk, dv, da, db, dS0
+
+
+@pytest.mark.parametrize("C", [1, 5, 16, 64])
+def test_chunk_backward_equals_recurrence_backward(orc, C):
+    rng = np.random.default_rng(40 + C)
+    L, d = 150, 16
+    q = rng.standard_normal((L, d)); q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k = rng.standard_normal((L, d)); k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((L, d))
+    a = np.exp(-np.log1p(np.exp(rng.standard_normal(L))))
+    b = 1 / (1 + np.exp(-rng.standard_normal(L)))
+    dO = rng.standard_normal((L, d))
+    q, k, v, a, b, dO = (x.astype(np.float32) for x in (q, k, v, a, b, dO))
+    S0 = rng.standard_normal((d, d))
+    dSL = rng.standard_normal((d, d))
+    ref = orc.gdn_bwd(q[None], k[None], v[None], a[None], b[None], dO[None], S0=S0[None],
+                      dS_final=dSL[None])
+    got = chunk_backward(*(x.astype(np.float64) for x in (q, k, v, a, b)), S0,
+                         dO.astype(np.float64), dSL, C)
+    for x, r in zip(got, ref):
+        np.testing.assert_allclose(x, r[0], rtol=1e-8, atol=1e-9)
