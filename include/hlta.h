@@ -166,6 +166,30 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
                             int B, int H, int T, int N, int d, int w, int r, float scale,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Workspace bytes of hlta_gdn_chunk_bwd (chunk = 64, d = 128): about 0.8 MB per 64-token
+ * chunk of every (batch, head); 0 for unsupported arguments. */
+size_t hlta_gdn_bwd_workspace_bytes(int B, int H, long L, int d, int chunk);
+
+/*
+ * Backward pass of the gated delta rule (training: related-papers analysis, row E): the
+ * reverse-mode derivative of hlta_gdn_chunk_fwd's recurrence for the upstream gradients dO of
+ * every output and dS_final of the final state (NULL for zero). Computed in chunk form with
+ * the chunk start states recomputed from S0 (NULL for zero): a forward pass over the chunks
+ * storing each start state, a backward pass over the chunks carrying the state gradient
+ * (dS_start = dS_end (gamma I - Kt^T W) + dO^T Qt with the forward's chunk products), and the
+ * gradients of every chunk in parallel; fp32 arithmetic throughout.
+ * q, k, v, dO, dq, dk, dv: [B, H, L, d] device, element type `dt` (d = 128); a, b, da, db:
+ * [B, H, L] float32 (a > 0); S0, dS_final, dS0: [B, H, d, d] float32 (dS0 NULL to skip).
+ * workspace: device scratch of at least hlta_gdn_bwd_workspace_bytes(...), caller-owned, 16-byte
+ * aligned. Enqueued on `stream` (four launches). Errors as hlta_gdn_chunk_fwd.
+ */
+hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *a,
+                               const float *b, const float *S0, const void *dO,
+                               const float *dS_final, void *dq, void *dk, void *dv, float *da,
+                               float *db, float *dS0, int B, int H, long L, int d, int chunk,
+                               void *workspace, size_t workspace_bytes, hlta_dtype dt,
+                               void *stream);
+
 /*
  * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens.
  */

@@ -61,6 +61,9 @@ def _load() -> ctypes.CDLL:
         "hlta_window_fwd_lse": (I, [P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
         "hlta_window_bwd_workspace_bytes": (Z, [I, I, I, I]),
         "hlta_window_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]),
+        "hlta_gdn_bwd_workspace_bytes": (Z, [I, I, L, I, I]),
+        "hlta_gdn_chunk_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, L, I, I, P, Z, I,
+                                   P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
         "hlta_set_profile_events": (I, [ctypes.POINTER(P)]),
     }
@@ -238,6 +241,25 @@ def hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale,
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def hlta_gdn_bwd_workspace_bytes(B, H, L, d=128, chunk=64) -> int:
+    return int(_lib.hlta_gdn_bwd_workspace_bytes(B, H, L, d, chunk))
+
+
+def hlta_gdn_chunk_bwd(q, k, v, a, b, S0, dO, dS_final, dq, dk, dv, da, db, dS0, B, H, L, d,
+                       chunk, workspace, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (a, "a"), (b, "b"), (dO, "dO"), (dq, "dq"),
+                 (dk, "dk"), (dv, "dv"), (da, "da"), (db, "db"), (workspace, "workspace")):
+        _need(t, n)
+    for t, n in ((S0, "S0"), (dS_final, "dS_final"), (dS0, "dS0")):
+        if t is not None:
+            _need(t, n)
+    _check(_lib.hlta_gdn_chunk_bwd(_p(q), _p(k), _p(v), _p(a), _p(b), _p(S0), _p(dO),
+                                   _p(dS_final), _p(dq), _p(dk), _p(dv), _p(da), _p(db), _p(dS0),
+                                   B, H, L, d, chunk, _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _dt(q),
+                                   _stream(stream)))
+
+
 def hlta_device_status(stream=None) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
@@ -337,6 +359,20 @@ def window_bwd(q, k, v, o, lse, dO, T, N, w, r=1, scale=0.0, grads=None, workspa
         hlta_window_bwd_workspace_bytes(B, H, T, N), q.device)
     hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale, ws, stream)
     return dq, dk, dv
+
+
+def gdn_bwd(q, k, v, a, b, dO, S0=None, dS_final=None, chunk=64, workspace=None, stream=None):
+    """Gradients (dq, dk, dv, da, db, dS0) of the gated delta rule."""
+    import torch
+    B, H, L, d = q.shape
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    da, db = (torch.empty((B, H, L), dtype=torch.float32, device=q.device) for _ in range(2))
+    dS0 = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    ws = workspace if workspace is not None else _workspace(
+        hlta_gdn_bwd_workspace_bytes(B, H, L, d, chunk), q.device)
+    hlta_gdn_chunk_bwd(q, k, v, a, b, S0, dO, dS_final, dq, dk, dv, da, db, dS0, B, H, L, d,
+                       chunk, ws, stream)
+    return dq, dk, dv, da, db, dS0
 
 
 def gdn(q, k, v, a, b, S0=None, chunk=64, out=None, S_out=None, workspace=None, stream=None):

@@ -1,0 +1,556 @@
+// Backward pass of the gated delta rule in chunk form, fp32 arithmetic on the CUDA cores
+// (bf16 or fp32 inputs and gradients; d = 128, chunks of 64 tokens).
+//
+// The derivative of the chunk form of the forward pass, term by term. Per chunk, with start
+// state S0, end-state gradient dS_C, g the running sum of log a, R = diag(b)(V - diag(e^g) K S0^T),
+// U = T R, Qt = diag(e^g) Q - P W and Kt = diag(e^{g_C - g}) K as in the forward:
+//   across chunks, last to first:  dS0 = dS_C (gamma I - Kt^T W) + dO^T Qt
+//   inside a chunk:  dU = P^T dO + Kt dS_C^T,  dR = T^T dU,  dP = dO U^T (s <= t),
+//                    dA = -dR U^T (s < t),  M = dA o b_t e^{g_t - g_s}
+//     dQ = diag(e^g) dO S0 + (dP o Gam) K
+//     dK = (dP o Gam)^T Q + diag(e^{g_C - g}) U dS_C + M K + M^T K - diag(b e^g) dR S0
+//     dV = diag(b) dR
+//     db = rowsum(dA o e^{g_t - g_s} o K K^T) + rowsum(dR o (V - diag(e^g) K S0^T))
+//     dg = rowsum - colsum of (dP o P) and (dA o A) + e^g o rowsum(Q o dO S0)
+//          - b e^g o rowsum(dR o K S0^T) - e^{g_C - g} o rowsum(U o K dS_C^T)
+//          + on the last token: gamma <dS_C, S0> + sum_s e^{g_C - g_s} rowsum(U o K dS_C^T)_s
+//     d(log a) = reverse running sum of dg inside the chunk,  da = d(log a) / a
+// (Gam: e^{g_t - g_s} on s <= t; only such decays, with non-positive exponents, are formed.)
+//
+// Four launches: prep (every chunk in parallel: inputs to fp32, the chunk's A, T, P, W, Up,
+// Qt, Kt), the forward state pass storing each chunk's start state, the backward state pass
+// storing each chunk's end-state gradient (both serial over chunks, parallel over rows of the
+// state), and the gradient kernel (every chunk in parallel). Products go through one block
+// GEMM routine on fp32 operands in the workspace (a chunk's working set stays in L2).
+#include "hlta_internal.cuh"
+
+#include <math.h>
+
+namespace hlta {
+namespace {
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int THREADS = 256;
+constexpr int R = 8;                // state rows per CTA in the state passes
+constexpr int CD = C * D, CC = C * C, DD = D * D;
+constexpr int DS = D + 4;           // staged row stride: 16-byte rows, no bank conflicts
+constexpr int CDS = C * DS;
+
+// per chunk-head scratch (floats)
+enum : long {
+    O_Q = 0, O_K = O_Q + CD, O_V = O_K + CD, O_G = O_V + CD, O_W = O_G + CD, O_UP = O_W + CD,
+    O_QT = O_UP + CD, O_KT = O_QT + CD, O_U = O_KT + CD, O_DU = O_U + CD, O_DR = O_DU + CD,
+    O_DS = O_DR + CD, O_RS = O_DS + CD, O_UD = O_RS + CD, O_KS = O_UD + CD, O_KD = O_KS + CD,
+    O_DQ = O_KD + CD, O_DK = O_DQ + CD,
+    O_T = O_DK + CD, O_P = O_T + CC, O_A = O_P + CC, O_KK = O_A + CC, O_DP = O_KK + CC,
+    O_DA = O_DP + CC,
+    O_S0 = O_DA + CC, O_DSC = O_S0 + DD,
+    O_VEC = O_DSC + DD,                 // g, b, a, b e^g, dg (C each), gamma and n
+    CHUNK_FLOATS = O_VEC + 6 * C
+};
+
+struct BwdP {
+    const void *q, *k, *v, *dO;
+    const float *a, *b, *S0, *dSL;
+    void *dq, *dk, *dv;
+    float *da, *db, *dS0;
+    float *ws;
+    long L;
+    int BH, nch;
+};
+
+template <typename E> __device__ __forceinline__ float ldf(const E *p, long i);
+template <> __device__ __forceinline__ float ldf<float>(const float *p, long i) { return p[i]; }
+template <> __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, long i) { return __bfloat162float(p[i]); }
+template <typename E> __device__ __forceinline__ void stf(E *p, long i, float x);
+template <> __device__ __forceinline__ void stf<float>(float *p, long i, float x) { p[i] = x; }
+template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p, long i, float x) { p[i] = __float2bfloat16(x); }
+
+// O[M][N] = alpha * sum_k opA(m, k) s(k) opB(k, n) + beta * O[m][n]; opA(m, k) = A[m][k] or,
+// transposed, A[k][m] (leading dimension lda); opB likewise; s an optional per-k scale.
+// M, N multiples of 64 and K of 32; 256 threads, each a 4 x 4 block of the 64 x 64 tile.
+// O must not alias A or B. `sm`: 2 * 32 * 65 floats of shared memory.
+__device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
+                      bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *sm)
+{
+    float *As = sm, *Bs = sm + 32 * 65;            // [k][m], [k][n]
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    // element e of a 32 x 64 operand tile; consecutive threads walk the contiguous index
+    auto a_at = [&](int m0, int k0, int e, int &kk, int &mm) -> float {
+        if (tA) { kk = e >> 6; mm = e & 63; return A[(long)(k0 + kk) * lda + m0 + mm]; }
+        kk = e & 31; mm = e >> 5;
+        return A[(long)(m0 + mm) * lda + k0 + kk];
+    };
+    auto b_at = [&](int n0, int k0, int e, int &kb, int &nb) -> float {
+        if (tB) { kb = e & 31; nb = e >> 5; return B[(long)(n0 + nb) * ldb + k0 + kb]; }
+        kb = e >> 6; nb = e & 63;
+        return B[(long)(k0 + kb) * ldb + n0 + nb];
+    };
+    constexpr int PER = 32 * 64 / THREADS;          // elements of each tile per thread
+    for (int m0 = 0; m0 < M; m0 += 64)
+        for (int n0 = 0; n0 < N; n0 += 64) {
+            float acc[4][4] = {};
+            float ra[PER], rb[PER];
+            int dummy0, dummy1;
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {             // loads of the first k-step
+                ra[r] = a_at(m0, 0, threadIdx.x + r * THREADS, dummy0, dummy1);
+                rb[r] = b_at(n0, 0, threadIdx.x + r * THREADS, dummy0, dummy1);
+            }
+            for (int k0 = 0; k0 < K; k0 += 32) {
+                __syncthreads();
+#pragma unroll
+                for (int r = 0; r < PER; ++r) {
+                    const int e = threadIdx.x + r * THREADS;
+                    int kk, mm, kb, nb;
+                    if (tA) { kk = e >> 6; mm = e & 63; } else { kk = e & 31; mm = e >> 5; }
+                    if (tB) { kb = e & 31; nb = e >> 5; } else { kb = e >> 6; nb = e & 63; }
+                    As[kk * 65 + mm] = ra[r];
+                    Bs[kb * 65 + nb] = (s ? s[k0 + kb] : 1.f) * rb[r];
+                }
+                __syncthreads();
+                if (k0 + 32 < K) {                      // next k-step's loads, in flight meanwhile
+#pragma unroll
+                    for (int r = 0; r < PER; ++r) {
+                        ra[r] = a_at(m0, k0 + 32, threadIdx.x + r * THREADS, dummy0, dummy1);
+                        rb[r] = b_at(n0, k0 + 32, threadIdx.x + r * THREADS, dummy0, dummy1);
+                    }
+                }
+#pragma unroll 8
+                for (int kk = 0; kk < 32; ++kk) {
+                    float x[4], y[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        x[i] = As[kk * 65 + ty * 4 + i];
+                        y[i] = Bs[kk * 65 + tx * 4 + i];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(x[i], y[j], acc[i][j]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float *o = O + (long)(m0 + ty * 4 + i) * ldo + n0 + tx * 4 + j;
+                    *o = alpha * acc[i][j] + (beta != 0.f ? beta * *o : 0.f);
+                }
+        }
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------------------------------
+// prep: one CTA per (chunk, head)
+template <typename E>
+__global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
+{
+    __shared__ float sm[2 * 32 * 65];
+    __shared__ float Tt[C][C + 1];
+    float (*At)[C + 1] = reinterpret_cast<float (*)[C + 1]>(sm);   // between GEMMs only
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
+    const long t0 = (long)c * C;
+    const int n = (int)min((long)C, p.L - t0);
+    const long base = ((long)bh * p.L + t0) * D;
+    float *g = w + O_VEC, *bb = g + C, *aa = bb + C, *bg = aa + C;
+    for (int e = tid; e < CD; e += THREADS) {
+        const int t = e / D;
+        const bool ok = t < n;
+        w[O_Q + e] = ok ? ldf((const E *)p.q, base + e) : 0.f;
+        w[O_K + e] = ok ? ldf((const E *)p.k, base + e) : 0.f;
+        w[O_V + e] = ok ? ldf((const E *)p.v, base + e) : 0.f;
+        w[O_G + e] = ok ? ldf((const E *)p.dO, base + e) : 0.f;
+    }
+    if (tid == 0) {
+        float acc = 0.f;
+        for (int t = 0; t < C; ++t) {
+            const bool ok = t < n;
+            if (ok) acc += logf(p.a[(long)bh * p.L + t0 + t]);
+            g[t] = acc;
+            bb[t] = ok ? p.b[(long)bh * p.L + t0 + t] : 0.f;
+            aa[t] = ok ? p.a[(long)bh * p.L + t0 + t] : 1.f;
+            bg[t] = bb[t] * expf(acc);
+        }
+        w[O_VEC + 5 * C] = expf(g[C - 1]);              // gamma = e^{g of the last token}
+        w[O_VEC + 5 * C + 1] = (float)n;
+    }
+    __syncthreads();
+    bgemm(w + O_KK, C, w + O_K, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    bgemm(w + O_P, C, w + O_Q, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    for (int e = tid; e < CC; e += THREADS) {
+        const int t = e / C, s = e % C;
+        const bool inc = s <= t && t < n;
+        const float dec = inc ? expf(g[t] - g[s]) : 0.f;
+        const float av = s < t ? bb[t] * dec * w[O_KK + e] : 0.f;
+        w[O_A + e] = av;
+        At[t][s] = av;
+        w[O_P + e] = dec * w[O_P + e];
+    }
+    __syncthreads();
+    if (tid < C) {                                      // T = (I + A)^{-1}, column tid
+        const int j = tid;
+        for (int t = 0; t < C; ++t) Tt[t][j] = t == j ? 1.f : 0.f;
+        for (int t = j + 1; t < C; ++t) {
+            float s = 0.f;
+            for (int i = j; i < t; ++i) s = fmaf(At[t][i], Tt[i][j], s);
+            Tt[t][j] = -s;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < CC; e += THREADS) w[O_T + e] = Tt[e / C][e % C];
+    __syncthreads();
+    bgemm(w + O_W, D, w + O_T, C, false, w + O_K, D, false, bg, C, D, C, 1.f, 0.f, sm);
+    bgemm(w + O_UP, D, w + O_T, C, false, w + O_V, D, false, bb, C, D, C, 1.f, 0.f, sm);
+    const float gC = g[C - 1];
+    for (int e = tid; e < CD; e += THREADS) {
+        const int t = e / D;
+        w[O_QT + e] = t < n ? expf(g[t]) * w[O_Q + e] : 0.f;
+        w[O_KT + e] = t < n ? expf(gC - g[t]) * w[O_K + e] : 0.f;
+    }
+    bgemm(w + O_QT, D, w + O_P, C, false, w + O_W, D, false, nullptr, C, D, C, -1.f, 1.f, sm);
+}
+
+// ----------------------------------------------------------------------------------------
+// State passes: one CTA per R rows of one head's state, serial over the chunks; each chunk's
+// C x d products are staged in shared memory (coalesced float4 copies) before use.
+// a C x D fp32 array into shared memory rows of DS floats
+__device__ __forceinline__ void stage(float *dst, const float *src, int n)
+{
+    const uint32_t d0 = (uint32_t)__cvta_generic_to_shared(dst);
+    for (int e = threadIdx.x; e < n / 4; e += THREADS) {
+        const int t = e / (D / 4), c4 = e % (D / 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d0 + 4u * (uint32_t)(t * DS + 4 * c4)),
+                     "l"(src + 4 * e)
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void stage_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void stage_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Register-blocked inner products of the state passes (R = 8 rows per CTA):
+//   dot:    thread (token tq, lane quarter q) sums x_i = sum_j X[tq][j] S[i][j] over the
+//           columns j = 4 jj + q for all eight rows (the rows of S at one column are one 32-byte
+//           line of ST, read as two broadcast float4), then the four quarters are added by
+//           shuffles;
+//   update: thread (column j, rows h4 .. h4+3) keeps its four state values in registers and
+//           adds the C rank-one terms, reading the per-row coefficients as broadcast float4.
+static_assert(R == 8, "state passes are written for 8 rows per CTA");
+
+__device__ __forceinline__ void dot8(float (&x)[8], const float *Xrow, const float *ST, int q)
+{
+    const float4 *ST4 = reinterpret_cast<const float4 *>(ST);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+#pragma unroll 8
+    for (int jj = 0; jj < D / 4; ++jj) {
+        const int jx = 4 * jj + q;
+        const float wv = Xrow[jx];
+        const float4 a = ST4[2 * jx], b = ST4[2 * jx + 1];
+        x[0] = fmaf(wv, a.x, x[0]); x[1] = fmaf(wv, a.y, x[1]);
+        x[2] = fmaf(wv, a.z, x[2]); x[3] = fmaf(wv, a.w, x[3]);
+        x[4] = fmaf(wv, b.x, x[4]); x[5] = fmaf(wv, b.y, x[5]);
+        x[6] = fmaf(wv, b.z, x[6]); x[7] = fmaf(wv, b.w, x[7]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[i] += __shfl_xor_sync(0xffffffffu, x[i], 1);
+        x[i] += __shfl_xor_sync(0xffffffffu, x[i], 2);
+    }
+}
+
+// forward: stores every chunk's start state (rows of this CTA)
+__global__ void __launch_bounds__(THREADS) gdn_bwd_fwdstate(BwdP p)
+{
+    extern __shared__ __align__(16) float dsm[];
+    float *buf = dsm;                               // two stages of W, Kt: [2][2][C][DS]
+    float *ST = dsm + 4 * CDS;                      // [D][R] the state, column-major
+    float *Uc = ST + D * R;                         // [C][R] U on this slice
+    float *Ups = Uc + C * R;                        // [C][R] this slice's columns of Up
+    const int i0 = blockIdx.x * R, bh = blockIdx.y, tid = threadIdx.x;
+    const int j = tid & (D - 1), h4 = (tid >> 7) * 4;
+    const int q = tid & 3, tq = tid >> 2;
+    float sv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        sv[r] = p.S0 ? p.S0[((long)bh * D + i0 + h4 + r) * D + j] : 0.f;
+        ST[j * R + h4 + r] = sv[r];
+    }
+    {
+        const float *w0 = p.ws + (long)bh * p.nch * CHUNK_FLOATS;
+        stage(buf, w0 + O_W, CD);
+        stage(buf + CDS, w0 + O_KT, CD);
+        stage_commit();
+    }
+    for (int c = 0; c < p.nch; ++c) {
+        float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
+        const float *Wc = buf + (c & 1) * 2 * CDS, *Kc = Wc + CDS;
+        const float gam = w[O_VEC + 5 * C];
+        __syncthreads();                            // the other stage and Uc are free again
+        if (c + 1 < p.nch) {
+            const float *wn = w + CHUNK_FLOATS;
+            stage(buf + ((c + 1) & 1) * 2 * CDS, wn + O_W, CD);
+            stage(buf + ((c + 1) & 1) * 2 * CDS + CDS, wn + O_KT, CD);
+        }
+        stage_commit();
+#pragma unroll
+        for (int r = 0; r < 4; ++r) w[O_S0 + (long)(i0 + h4 + r) * D + j] = sv[r];
+        for (int e = tid; e < C * R; e += THREADS) Ups[e] = w[O_UP + (e / R) * D + i0 + e % R];
+        stage_wait_prev();
+        __syncthreads();
+        float x[8];                                 // U = Up - W S0^T on this slice
+        dot8(x, Wc + tq * DS, ST, q);
+        if (q == 0)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) Uc[tq * R + i] = Ups[tq * R + i] - x[i];
+        __syncthreads();
+        const float4 *U4 = reinterpret_cast<const float4 *>(Uc);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sv[r] *= gam;   // S = gamma S + U^T Kt
+#pragma unroll 8
+        for (int t = 0; t < C; ++t) {
+            const float kv = Kc[t * DS + j];
+            const float4 u = U4[t * 2 + h4 / 4];
+            sv[0] = fmaf(u.x, kv, sv[0]); sv[1] = fmaf(u.y, kv, sv[1]);
+            sv[2] = fmaf(u.z, kv, sv[2]); sv[3] = fmaf(u.w, kv, sv[3]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) ST[j * R + h4 + r] = sv[r];
+    }
+}
+
+// backward: dS <- dS (gamma I - Kt^T W) + dO^T Qt from the last chunk to the first; stores
+// every chunk's end-state gradient and writes dS0
+__global__ void __launch_bounds__(THREADS) gdn_bwd_bwdstate(BwdP p)
+{
+    extern __shared__ __align__(16) float dsm[];
+    float *buf = dsm;                               // two stages of W, Kt, Qt: [2][3][C][DS]
+    float *ST = dsm + 6 * CDS;                      // [D][R] the state gradient, column-major
+    float *Y = ST + D * R;                          // [C][R] Kt dS^T on this slice
+    float *Gs = Y + C * R;                          // [C][R] this slice's columns of dO
+    const int i0 = blockIdx.x * R, bh = blockIdx.y, tid = threadIdx.x;
+    const int j = tid & (D - 1), h4 = (tid >> 7) * 4;
+    const int q = tid & 3, tq = tid >> 2;
+    float sv[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        sv[r] = p.dSL ? p.dSL[((long)bh * D + i0 + h4 + r) * D + j] : 0.f;
+        ST[j * R + h4 + r] = sv[r];
+    }
+    {
+        const float *wl = p.ws + ((long)bh * p.nch + p.nch - 1) * CHUNK_FLOATS;
+        stage(buf, wl + O_W, CD);
+        stage(buf + CDS, wl + O_KT, CD);
+        stage(buf + 2 * CDS, wl + O_QT, CD);
+        stage_commit();
+    }
+    for (int c = p.nch - 1; c >= 0; --c) {
+        float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
+        const int sl = (p.nch - 1 - c) & 1;
+        const float *Wc = buf + sl * 3 * CDS, *Kc = Wc + CDS, *Qc = Kc + CDS;
+        const float gam = w[O_VEC + 5 * C];
+        __syncthreads();                            // the other stage, Y and Gs are free again
+        if (c > 0) {
+            const float *wn = w - CHUNK_FLOATS;
+            float *nb = buf + (sl ^ 1) * 3 * CDS;
+            stage(nb, wn + O_W, CD);
+            stage(nb + CDS, wn + O_KT, CD);
+            stage(nb + 2 * CDS, wn + O_QT, CD);
+        }
+        stage_commit();
+#pragma unroll
+        for (int r = 0; r < 4; ++r) w[O_DSC + (long)(i0 + h4 + r) * D + j] = sv[r];
+        for (int e = tid; e < C * R; e += THREADS) Gs[e] = w[O_G + (e / R) * D + i0 + e % R];
+        stage_wait_prev();
+        __syncthreads();
+        float x[8];                                 // Y = Kt dS^T on this slice
+        dot8(x, Kc + tq * DS, ST, q);
+        if (q == 0)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) Y[tq * R + i] = x[i];
+        __syncthreads();
+        const float4 *Y4 = reinterpret_cast<const float4 *>(Y), *G4 = reinterpret_cast<const float4 *>(Gs);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sv[r] *= gam;
+#pragma unroll 4
+        for (int t = 0; t < C; ++t) {
+            const float qv = Qc[t * DS + j], wv = Wc[t * DS + j];
+            const float4 gg = G4[t * 2 + h4 / 4], yy = Y4[t * 2 + h4 / 4];
+            sv[0] = fmaf(gg.x, qv, fmaf(-yy.x, wv, sv[0]));
+            sv[1] = fmaf(gg.y, qv, fmaf(-yy.y, wv, sv[1]));
+            sv[2] = fmaf(gg.z, qv, fmaf(-yy.z, wv, sv[2]));
+            sv[3] = fmaf(gg.w, qv, fmaf(-yy.w, wv, sv[3]));
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) ST[j * R + h4 + r] = sv[r];
+    }
+    if (p.dS0)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) p.dS0[((long)bh * D + i0 + h4 + r) * D + j] = sv[r];
+}
+
+// ----------------------------------------------------------------------------------------
+// gradients of one chunk
+template <typename E>
+__global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
+{
+    __shared__ float sm[2 * 32 * 65];
+    __shared__ float red[THREADS / 32];
+    __shared__ float rowv[6][C];
+    const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
+    float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
+    const float *g = w + O_VEC, *bb = g + C, *aa = bb + C;
+    float *dg = w + O_VEC + 4 * C;
+    const float gam = w[O_VEC + 5 * C];
+    const int n = (int)w[O_VEC + 5 * C + 1];
+    const float gC = g[C - 1];
+    const float *S0 = w + O_S0, *dSC = w + O_DSC;
+    // U = Up - W S0^T
+    for (int e = tid; e < CD; e += THREADS) w[O_U + e] = w[O_UP + e];
+    bgemm(w + O_U, D, w + O_W, D, false, S0, D, true, nullptr, C, D, D, -1.f, 1.f, sm);
+    // dU = Kt dS_C^T + P^T dO ;  dR = T^T dU
+    bgemm(w + O_DU, D, w + O_KT, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);
+    bgemm(w + O_DU, D, w + O_P, C, true, w + O_G, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    bgemm(w + O_DR, D, w + O_T, C, true, w + O_DU, D, false, nullptr, C, D, C, 1.f, 0.f, sm);
+    // C x C: dP = dO U^T, dA' = dR U^T
+    bgemm(w + O_DP, C, w + O_G, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    bgemm(w + O_DA, C, w + O_DR, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    // products with the d x d states
+    bgemm(w + O_DS, D, w + O_G, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);     // dO S0
+    bgemm(w + O_RS, D, w + O_DR, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // dR S0
+    bgemm(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // U dS_C
+    bgemm(w + O_KS, D, w + O_K, D, false, S0, D, true, nullptr, C, D, D, 1.f, 0.f, sm);      // K S0^T
+    bgemm(w + O_KD, D, w + O_K, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);     // K dS_C^T
+    // per-row sums over the C x C products (threads 0..63 rows, 64..127 columns) and the
+    // C x d ones (threads 128..191)
+    if (tid < C) {
+        const int t = tid;
+        float pp = 0.f, ap = 0.f, db1 = 0.f;
+        for (int s = 0; s < C; ++s) {
+            const bool inc = s <= t && t < n, low = s < t && t < n;
+            const float dpv = inc ? w[O_DP + t * C + s] : 0.f;
+            const float dav = low ? -w[O_DA + t * C + s] : 0.f;
+            pp += dpv * w[O_P + t * C + s];
+            ap += dav * w[O_A + t * C + s];
+            db1 += low ? dav * expf(g[t] - g[s]) * w[O_KK + t * C + s] : 0.f;
+        }
+        rowv[0][t] = pp;
+        rowv[1][t] = ap;
+        rowv[2][t] = db1;
+    } else if (tid < 2 * C) {
+        const int s = tid - C;
+        float pp = 0.f, ap = 0.f;
+        for (int t = s; t < n; ++t) {
+            pp += w[O_DP + t * C + s] * w[O_P + t * C + s];
+            if (t > s) ap += -w[O_DA + t * C + s] * w[O_A + t * C + s];
+        }
+        rowv[3][s] = pp;
+        rowv[4][s] = ap;
+    } else if (tid < 3 * C) {
+        const int t = tid - 2 * C;
+        const float eg = expf(g[t]);
+        float qds = 0.f, drk = 0.f, ukd = 0.f, drv = 0.f;
+        for (int j = 0; j < D; ++j) {
+            const float ks = w[O_KS + t * D + j], dr = w[O_DR + t * D + j];
+            qds = fmaf(w[O_Q + t * D + j], w[O_DS + t * D + j], qds);
+            drk = fmaf(dr, ks, drk);
+            ukd = fmaf(w[O_U + t * D + j], w[O_KD + t * D + j], ukd);
+            drv = fmaf(dr, w[O_V + t * D + j] - eg * ks, drv);
+        }
+        const bool ok = t < n;
+        dg[t] = ok ? eg * qds - bb[t] * eg * drk - expf(gC - g[t]) * ukd : 0.f;
+        rowv[5][t] = ok ? expf(gC - g[t]) * ukd : 0.f;      // for the last token's term
+        w[O_DU + t] = drv;                                   // (dU is free now) db part 2
+    }
+    // <dS_C, S0>
+    float sd = 0.f;
+    for (int e = tid; e < DD; e += THREADS) sd = fmaf(dSC[e], S0[e], sd);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
+    if ((tid & 31) == 0) red[tid >> 5] = sd;
+    __syncthreads();
+    if (tid == 0) {
+        float tot = 0.f, su = 0.f;
+        for (int i = 0; i < THREADS / 32; ++i) tot += red[i];
+        for (int s = 0; s < n; ++s) su += rowv[5][s];
+        float run = 0.f;
+        for (int t = n - 1; t >= 0; --t) {
+            float v = dg[t] + rowv[0][t] - rowv[3][t] + rowv[1][t] - rowv[4][t];
+            if (t == n - 1) v += gam * tot + su;
+            run += v;
+            const long gi = (long)bh * p.L + (long)c * C + t;
+            p.da[gi] = run / aa[t];
+            p.db[gi] = rowv[2][t] + w[O_DU + t];
+        }
+    }
+    // M = dA o b_t e^{g_t - g_s} (s < t) into O_DA;  dP o Gam into O_DP
+    for (int e = tid; e < CC; e += THREADS) {
+        const int t = e / C, s = e % C;
+        const bool inc = s <= t && t < n, low = s < t && t < n;
+        const float dec = inc ? expf(g[t] - g[s]) : 0.f;
+        w[O_DA + e] = low ? -w[O_DA + e] * bb[t] * dec : 0.f;
+        w[O_DP + e] = inc ? w[O_DP + e] * dec : 0.f;
+    }
+    __syncthreads();
+    // dQ = diag(e^g) dO S0 + (dP o Gam) K
+    for (int e = tid; e < CD; e += THREADS) w[O_DQ + e] = expf(g[e / D]) * w[O_DS + e];
+    bgemm(w + O_DQ, D, w + O_DP, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    // dK = diag(e^{g_C - g}) U dS_C - diag(b e^g) dR S0 + (dP o Gam)^T Q + M K + M^T K
+    for (int e = tid; e < CD; e += THREADS) {
+        const int t = e / D;
+        w[O_DK + e] = t < n ? expf(gC - g[t]) * w[O_UD + e] - bb[t] * expf(g[t]) * w[O_RS + e] : 0.f;
+    }
+    bgemm(w + O_DK, D, w + O_DP, C, true, w + O_Q, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    bgemm(w + O_DK, D, w + O_DA, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    bgemm(w + O_DK, D, w + O_DA, C, true, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    const long base = ((long)bh * p.L + (long)c * C) * D;
+    for (int e = tid; e < n * D; e += THREADS) {
+        stf((E *)p.dq, base + e, w[O_DQ + e]);
+        stf((E *)p.dk, base + e, w[O_DK + e]);
+        stf((E *)p.dv, base + e, bb[e / D] * w[O_DR + e]);
+    }
+}
+
+template <typename E>
+cudaError_t launch_typed(const BwdP &p, cudaStream_t s)
+{
+    const dim3 gc((unsigned)p.nch, (unsigned)p.BH), gs((unsigned)(D / R), (unsigned)p.BH);
+    const int sm_f = (int)sizeof(float) * (4 * CDS + D * R + 2 * C * R);
+    const int sm_b = (int)sizeof(float) * (6 * CDS + D * R + 2 * C * R);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(gdn_bwd_fwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_f)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_bwd_bwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_b)) != cudaSuccess) return e;
+    gdn_bwd_prep<E><<<gc, THREADS, 0, s>>>(p);
+    gdn_bwd_fwdstate<<<gs, THREADS, sm_f, s>>>(p);
+    gdn_bwd_bwdstate<<<gs, THREADS, sm_b, s>>>(p);
+    gdn_bwd_grad<E><<<gc, THREADS, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gdn_bwd_workspace_bytes(long BH, long L)
+{
+    return (size_t)BH * (size_t)gdn_num_chunks(L, C) * (size_t)CHUNK_FLOATS * sizeof(float);
+}
+
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
+{
+    if (a.d != D) return cudaErrorNotSupported;
+    if (a.B * a.H == 0 || a.L == 0) return cudaSuccess;
+    const long nch = gdn_num_chunks(a.L, C);
+    if (nch >= (1L << 31) || (long)a.B * a.H > 65535) return cudaErrorNotSupported;
+    BwdP p;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.dO = a.dO;
+    p.a = a.a; p.b = a.b; p.S0 = a.S0; p.dSL = a.dS_final;
+    p.dq = a.dq; p.dk = a.dk; p.dv = a.dv; p.da = a.da; p.db = a.db; p.dS0 = a.dS0;
+    p.ws = (float *)a.ws;
+    p.L = a.L;
+    p.BH = a.B * a.H;
+    p.nch = (int)nch;
+    return a.bf16 ? launch_typed<__nv_bfloat16>(p, s) : launch_typed<float>(p, s);
+}
+
+}  // namespace hlta

@@ -377,6 +377,53 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
     return HLTA_OK;
 }
 
+size_t hlta_gdn_bwd_workspace_bytes(int B, int H, long L, int d, int chunk)
+{
+    if (B < 0 || H < 0 || L < 0 || d != 128 || chunk != 64) return 0;
+    return gdn_bwd_workspace_bytes((long)B * H, L);
+}
+
+hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *a,
+                               const float *b, const float *S0, const void *dO,
+                               const float *dS_final, void *dq, void *dk, void *dv, float *da,
+                               float *db, float *dS0, int B, int H, long L, int d, int chunk,
+                               void *workspace, size_t workspace_bytes, hlta_dtype dt,
+                               void *stream)
+{
+    const void *req[] = {q, k, v, a, b, dO, dq, dk, dv, da, db, workspace};
+    for (const void *p : req) {
+        if (!p) return fail(HLTA_ERR_INVALID_ARG, "null tensor pointer");
+        if (!aligned16(p)) return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    }
+    const void *opt[] = {S0, dS_final, dS0};
+    for (const void *p : opt)
+        if (p && !aligned16(p)) return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (dt != HLTA_BF16 && dt != HLTA_FP32) return fail(HLTA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (B < 0 || H < 0 || L < 0) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld", B, H, L);
+    if (chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64 (got %d)", chunk);
+    if (d != 128) return fail(HLTA_ERR_UNSUPPORTED, "gated delta rule backward supports d = 128 only (got %d)", d);
+    const size_t need = hlta_gdn_bwd_workspace_bytes(B, H, L, d, chunk);
+    if (workspace_bytes < need)
+        return fail(HLTA_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)", workspace_bytes, need);
+    GdnBwdArgs g;
+    g.q = q; g.k = k; g.v = v; g.dO = dO; g.a = a; g.b = b; g.S0 = S0; g.dS_final = dS_final;
+    g.dq = dq; g.dk = dk; g.dv = dv; g.da = da; g.db = db; g.dS0 = dS0;
+    g.ws = workspace; g.B = B; g.H = H; g.d = d; g.L = L; g.bf16 = dt == HLTA_BF16;
+    if ((long)B * H == 0 || L == 0) {
+        // no tokens: the state gradient passes through unchanged
+        if (dS0 && (long)B * H > 0) {
+            cudaError_t e = dS_final ? cudaMemcpyAsync(dS0, dS_final, (size_t)B * H * d * d * sizeof(float), cudaMemcpyDeviceToDevice, (cudaStream_t)stream)
+                                     : cudaMemsetAsync(dS0, 0, (size_t)B * H * d * d * sizeof(float), (cudaStream_t)stream);
+            if (e != cudaSuccess) return cuda_fail(e, "dS0 copy");
+        }
+        return HLTA_OK;
+    }
+    cudaError_t e = launch_gdn_bwd(g, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "gated delta rule backward: unsupported shape");
+    if (e != cudaSuccess) return cuda_fail(e, "gated delta rule backward launch");
+    return HLTA_OK;
+}
+
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt)
 {
     if (B < 0 || H < 0 || L < 0 || d < 1 || chunk != 64) return 0;

@@ -102,6 +102,21 @@ struct AttnBwdArgs {
     float scale;
 };
 cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s);
+// Gated delta rule backward (chunk form, fp32 arithmetic, d = 128): q, k, v, dO, dq, dk, dv
+// [B][H][L][d] (bf16 when `bf16`, else fp32); a, b, da, db [B][H][L]; S0, dS_final, dS0
+// [B][H][d][d] fp32 (S0 / dS_final null for zero, dS0 null to skip).
+struct GdnBwdArgs {
+    const void *q, *k, *v, *dO;
+    const float *a, *b, *S0, *dS_final;
+    void *dq, *dk, *dv;
+    float *da, *db, *dS0;
+    void *ws;
+    int B, H, d;
+    long L;
+    bool bf16;
+};
+size_t gdn_bwd_workspace_bytes(long BH, long L);
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,

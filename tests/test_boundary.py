@@ -151,3 +151,22 @@ def test_attention_backward_entry_points_validate_on_host(lib):
     assert b(*bad) == h.HLTA_ERR_UNSUPPORTED
     bad = list(args); bad[7] = ctypes.c_void_p(264)
     assert b(*bad) == h.HLTA_ERR_INVALID_ARG
+
+
+def test_gdn_backward_entry_point_validates_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    ws = lib.hlta_gdn_bwd_workspace_bytes(1, 2, 100, 128, 64)
+    assert ws > 0 and lib.hlta_gdn_bwd_workspace_bytes(1, 2, 100, 64, 64) == 0
+    f = lib.hlta_gdn_chunk_bwd
+    args = [p, p, p, p, p, None, p, None, p, p, p, p, p, None, 1, 2, 100, 128, 64, p, ws, h.HLTA_BF16, None]
+    bad = list(args); bad[0] = None
+    assert f(*bad) == h.HLTA_ERR_INVALID_ARG
+    bad = list(args); bad[20] = ws - 1
+    assert f(*bad) == h.HLTA_ERR_INVALID_ARG and b"workspace" in lib.hlta_last_error()
+    bad = list(args); bad[18] = 32
+    assert f(*bad) == h.HLTA_ERR_UNSUPPORTED
+    bad = list(args); bad[17] = 64
+    assert f(*bad) == h.HLTA_ERR_UNSUPPORTED
+    bad = list(args); bad[5] = ctypes.c_void_p(264)
+    assert f(*bad) == h.HLTA_ERR_INVALID_ARG
