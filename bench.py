@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the training-pass measurement (detail.backward)")
     ap.add_argument("--no-stream", action="store_true",
                     help="skip the streaming-step measurement (detail.stream)")
     return ap.parse_args()
@@ -215,6 +217,59 @@ def measure_fp8(h, torch, dev, wl, q, k, v, steps: int) -> dict:
         e1.record()
         torch.cuda.synchronize()
         res[name] = e0.elapsed_time(e1) / steps
+    return res
+
+
+def measure_backward(h, torch, dev, wl, q, k, v, a, b, steps: int) -> dict:
+    """Training pass of the same workload: the softmax branches' forward with log-sum-exp and
+    their backward, and the GDN heads' backward (chunk-start states recomputed inside), each
+    timed back to back over `steps` repetitions with a seeded upstream gradient."""
+    g0 = wl.Hs + wl.Hd
+    gen = torch.Generator(device=dev).manual_seed(99)
+    res = {}
+    br = [(slice(0, wl.Hs), wl.w_swa, 1), (slice(wl.Hs, g0), wl.w_dswa, wl.r)]
+    bf16 = q.dtype == torch.bfloat16          # the softmax training pair is bf16 only
+    src = [tuple(x_[:, s_].contiguous() for x_ in (q, k, v)) for s_, _, _ in br if bf16 and s_.stop > s_.start]
+    cfg = [(w, r) for s_, w, r in br if bf16 and s_.stop > s_.start]
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    if src:
+        outs = [h.window_fwd_lse(*t, wl.T, wl.N, w, r) for t, (w, r) in zip(src, cfg)]
+        dOs = [torch.randn(t[0].shape, device=dev, generator=gen).to(t[0].dtype) for t in src]
+        grads = [tuple(torch.empty_like(t[0]) for _ in range(3)) for t in src]
+        wss = [torch.empty(h.hlta_window_bwd_workspace_bytes(wl.B, t[0].shape[1], wl.T, wl.N),
+                           dtype=torch.uint8, device=dev) for t in src]
+
+        def fwd():
+            for t, (w, r), (o, ls) in zip(src, cfg, outs):
+                h.window_fwd_lse(*t, wl.T, wl.N, w, r, out=o, lse=ls)
+
+        def bwd():
+            for t, (w, r), (o, ls), dO, gr, ws in zip(src, cfg, outs, dOs, grads, wss):
+                h.window_bwd(*t, o, ls, dO, wl.T, wl.N, w, r, grads=gr, workspace=ws)
+
+        res["attn_fwd_lse_ms"] = timed(fwd)
+        res["attn_bwd_ms"] = timed(bwd)
+        del outs, dOs, grads, wss
+    if wl.Hg:
+        qg, kg, vg = (x_[:, g0:].contiguous() for x_ in (q, k, v))
+        dOg = torch.randn(qg.shape, device=dev, generator=gen).to(qg.dtype)
+        wsg = torch.empty(h.hlta_gdn_bwd_workspace_bytes(wl.B, wl.Hg, wl.L), dtype=torch.uint8,
+                          device=dev)
+        res["gdn_bwd_ms"] = timed(lambda: h.gdn_bwd(qg, kg, vg, a, b, dOg, workspace=wsg))
+        res["gdn_bwd_workspace_gb"] = wsg.numel() / 1e9
+        del qg, kg, vg, dOg, wsg
     return res
 
 
@@ -521,6 +576,8 @@ def main():
     raw_detail = None if args.no_stream else measure_raw(h, torch, dev, wl, hi, K)
     fp8_ms = (measure_fp8(h, torch, dev, wl, q, k, v, K)
               if not args.no_stream and wl.dtype == "bf16" and wl.Hs + wl.Hd > 0 else None)
+    bwd_ms = (measure_backward(h, torch, dev, wl, q, k, v, a, b, max(2, min(K, 5)))
+              if not args.no_stream and not args.no_backward and wl.d == 128 else None)
 
     # ---- roofline of the dominant kernel (windowed attention, both launches) --------------
     wk = work(wl)
@@ -558,6 +615,18 @@ def main():
         detail["stream"] = stream_detail
     if raw_detail is not None:
         detail["raw_prologue"] = raw_detail
+    if bwd_ms is not None:
+        bw = dict(bwd_ms)
+        if "attn_bwd_ms" in bw:
+            # five products of 2 d FLOP per valid pair (S, dP, dV, dK, dQ; the kernels
+            # recompute S and dP once more, not counted)
+            bflop = 2.5 * attn_flop
+            bw["attn_bwd_tflops"] = bflop / (bw["attn_bwd_ms"] / 1e3) / 1e12
+            bw["attn_bwd_frac"] = bw["attn_bwd_tflops"] / float(pk.get("bf16_tflops"))
+        bw["note"] = ("training pass: hlta_window_fwd_lse + hlta_window_bwd for the SWA and DSWA "
+                      "heads (mma.sync products), hlta_gdn_chunk_bwd for the GDN heads (fp32 "
+                      "arithmetic, chunk-start states recomputed); frac against the burst bf16 peak")
+        detail["backward"] = bw
     if fp8_ms is not None:
         # E4M3 dense peak = the measured bf16 burst peak x 2 (nominal fp8:bf16 ratio 4.5:2.25)
         fp8_peak = 2.0 * float(pk.get("bf16_tflops"))

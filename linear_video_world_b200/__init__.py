@@ -220,9 +220,16 @@ def hlta_window_fp8_fwd(q8, qs, k8, ks, v8, vs, o, B, H, T, N, d, w, r, scale=0.
                                     T, N, d, w, r, float(scale), _stream(stream)))
 
 
+def _need_bf16(*ts):
+    import torch
+    if any(t.dtype != torch.bfloat16 for t in ts):
+        raise HltaError(HLTA_ERR_INVALID_ARG, "the attention training pair takes bf16 tensors")
+
+
 def hlta_window_fwd_lse(q, k, v, o, lse, B, H, T, N, d, w, r, scale=0.0, stream=None):
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse")):
         _need(t, n)
+    _need_bf16(q, k, v, o)
     _check(_lib.hlta_window_fwd_lse(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, T, N, d, w, r,
                                     float(scale), _stream(stream)))
 
@@ -236,6 +243,7 @@ def hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale,
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (lse, "lse"), (dO, "dO"), (dq, "dq"),
                  (dk, "dk"), (dv, "dv"), (workspace, "workspace")):
         _need(t, n)
+    _need_bf16(q, k, v, o, dO, dq, dk, dv)
     _check(_lib.hlta_window_bwd(_p(q), _p(k), _p(v), _p(o), _p(lse), _p(dO), _p(dq), _p(dk),
                                 _p(dv), B, H, T, N, d, w, r, float(scale), _p(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
