@@ -91,6 +91,14 @@ def test_hybrid_480p_long_sampled(h, orc):
     _hybrid_check(h, orc, hi.WORKLOADS["480p_long"], 64)
 
 
+def test_hybrid_720p_long_geometry_sampled(h, orc):
+    """The 720P long rollout's geometry (T=61 frames of N=3600 tokens, L=219600: ragged 64-key
+    tiles, row indices past 2^17; SWA w=3, DSWA w=4 r=6) on two heads per branch: softmax heads
+    on sampled rows, the GDN heads over the whole 219600-token recurrence."""
+    wl = hi.WORKLOADS["720p_long"].with_(Hs=2, Hd=2, Hg=2)
+    _hybrid_check(h, orc, wl, 48)
+
+
 def test_stream_steps_equal_hybrid_bf16(h, orc):
     """Successive streaming steps from empty caches reproduce the hybrid operator on the
     concatenated clip (frame by frame) and its final state; rings wrap several times."""
