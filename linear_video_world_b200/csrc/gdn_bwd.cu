@@ -36,6 +36,7 @@ constexpr int R = 8;                // state rows per CTA in the state passes
 constexpr int CD = C * D, CC = C * C, DD = D * D;
 constexpr int DS = D + 4;           // staged row stride: 16-byte rows, no bank conflicts
 constexpr int CDS = C * DS;
+constexpr int TS = 68;              // row stride of the block GEMM's staged tiles
 
 // per chunk-head scratch (floats)
 enum : long {
@@ -69,12 +70,13 @@ template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p,
 
 // O[M][N] = alpha * sum_k opA(m, k) s(k) opB(k, n) + beta * O[m][n]; opA(m, k) = A[m][k] or,
 // transposed, A[k][m] (leading dimension lda); opB likewise; s an optional per-k scale.
-// M, N multiples of 64 and K of 32; 256 threads, each a 4 x 4 block of the 64 x 64 tile.
-// O must not alias A or B. `sm`: 2 * 32 * 65 floats of shared memory.
+// M, N multiples of 64 and K of 32; 256 threads, each a 4 x 4 block of the 64 x 64 tile read
+// as two float4 per k (tile rows padded to 68 floats). O must not alias A or B.
+// `sm`: 2 * 32 * 68 floats of shared memory, 16-byte aligned.
 __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
                       bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *sm)
 {
-    float *As = sm, *Bs = sm + 32 * 65;            // [k][m], [k][n]
+    float *As = sm, *Bs = sm + 32 * TS;            // [k][m], [k][n]
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
     // element e of a 32 x 64 operand tile; consecutive threads walk the contiguous index
     auto a_at = [&](int m0, int k0, int e, int &kk, int &mm) -> float {
@@ -106,8 +108,8 @@ __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const
                     int kk, mm, kb, nb;
                     if (tA) { kk = e >> 6; mm = e & 63; } else { kk = e & 31; mm = e >> 5; }
                     if (tB) { kb = e & 31; nb = e >> 5; } else { kb = e >> 6; nb = e & 63; }
-                    As[kk * 65 + mm] = ra[r];
-                    Bs[kb * 65 + nb] = (s ? s[k0 + kb] : 1.f) * rb[r];
+                    As[kk * TS + mm] = ra[r];
+                    Bs[kb * TS + nb] = (s ? s[k0 + kb] : 1.f) * rb[r];
                 }
                 __syncthreads();
                 if (k0 + 32 < K) {                      // next k-step's loads, in flight meanwhile
@@ -119,12 +121,9 @@ __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const
                 }
 #pragma unroll 8
                 for (int kk = 0; kk < 32; ++kk) {
-                    float x[4], y[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        x[i] = As[kk * 65 + ty * 4 + i];
-                        y[i] = Bs[kk * 65 + tx * 4 + i];
-                    }
+                    const float4 xa = *reinterpret_cast<const float4 *>(As + kk * TS + ty * 4);
+                    const float4 yb = *reinterpret_cast<const float4 *>(Bs + kk * TS + tx * 4);
+                    const float x[4] = {xa.x, xa.y, xa.z, xa.w}, y[4] = {yb.x, yb.y, yb.z, yb.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -147,7 +146,7 @@ __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const
 template <typename E>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
 {
-    __shared__ float sm[2 * 32 * 65];
+    __shared__ __align__(16) float sm[2 * 32 * TS];
     __shared__ float Tt[C][C + 1];
     float (*At)[C + 1] = reinterpret_cast<float (*)[C + 1]>(sm);   // between GEMMs only
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
@@ -396,7 +395,7 @@ __global__ void __launch_bounds__(THREADS) gdn_bwd_bwdstate(BwdP p)
 template <typename E>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
 {
-    __shared__ float sm[2 * 32 * 65];
+    __shared__ __align__(16) float sm[2 * 32 * TS];
     __shared__ float red[THREADS / 32];
     __shared__ float rowv[6][C];
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
