@@ -1,0 +1,513 @@
+// Gradients of the windowed attention on the sm_100a tensor cores (bf16, d = 128): dK and dV
+// (one kernel, key-tile major) and dQ (one kernel, query-tile major), with the forward's per-row
+// log-sum-exp to recompute p = exp(s scale - lse) and D = rowsum(dO o O) from the first launch.
+//
+// dK / dV: one CTA per 128-key tile of one key frame g; it walks the 64-row query tiles of every
+// frame that sees g (f = g + r i, i < w, f < T) and keeps dK and dV of its keys in tensor memory.
+// Per query tile j:
+//   S^T  = K Q_j^T,  dP^T = V dO_j^T                   (128 x 64 each; shared-memory operands)
+//   P^T  = exp2(S^T sl2 - lse2_j),  dS^T = P^T o (dP^T - D_j)     (elementwise warps)
+//   dV  += P^T dO_j,  dK += dS^T Q_j                   (P^T and dS^T read from tensor memory)
+// dQ: the same with queries and keys exchanged (one CTA per 128-row query tile of a frame,
+// walking the 64-key tiles of its window; dQ += dS K_j).
+// The roles mirror the forward kernel (attn_tc.cu): the CTA's own 128-row tile takes the place
+// of its query sub-tile, the other side's tiles stream through a TMA ring like its key tiles,
+// P^T / dS are written over the first 32 columns of their fp32 buffers as bf16 pairs, and
+// products of one issuing thread execute in issue order, so S of tile j+1 is issued into the
+// buffers that the accumulating products of tile j-1 read without a wait.
+// Threads: warps 0..3 elementwise (one thread per row of the CTA's tile, the warp's TMEM lane
+// quadrant), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner. Tensor memory: per buffer
+// b (two) S at 128 b and dP at 128 b + 64; accumulators at 256 (dV or dQ) and 384 (dK). Every
+// mbarrier wait is bounded.
+#include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_ptx.cuh"
+
+#include <math.h>
+
+namespace hlta {
+namespace {
+
+using namespace ptx;
+using namespace tc;
+
+constexpr int BK = 128;                 // keys per CTA (the products' M)
+constexpr int BQ = 64;                  // queries per tile (N of S^T, K of the accumulations)
+constexpr int D = 128;
+constexpr int NS = 3;                   // Q / dO ring stages
+constexpr int THREADS = 192;
+constexpr int WARP_TMA = 4, WARP_MMA = 5;
+constexpr uint32_t KHALF = BK * 128;    // [128 rows][64 cols] bf16: 16 KB
+constexpr uint32_t KTILE = 2 * KHALF;
+constexpr uint32_t QHALF = BQ * 128;    // [64 rows][64 cols]: 8 KB
+constexpr uint32_t QTILE = 2 * QHALF;
+constexpr uint32_t SM_K = 0, SM_V = KTILE;
+__host__ __device__ constexpr uint32_t SM_Q(int st) { return 2 * KTILE + (uint32_t)st * 2 * QTILE; }
+__host__ __device__ constexpr uint32_t SM_G(int st) { return SM_Q(st) + QTILE; }
+constexpr uint32_t SM_LD = 2 * KTILE + NS * 2 * QTILE;       // per elementwise warp: lse2[64] | D[64]
+constexpr uint32_t SM_BAR = SM_LD + 4 * 2 * BQ * 4;
+enum { B_KV = 0, B_QFULL = 1, B_EMPTY = B_QFULL + NS, B_SFULL = B_EMPTY + NS, B_PFULL = B_SFULL + 2,
+       B_ODONE = B_PFULL + 2, NBARS = B_ODONE + 1 };
+constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
+constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
+constexpr size_t SMEM_BYTES = SM_ABORT + 4 + 1024;
+constexpr uint32_t TM_ST(int b) { return (uint32_t)b * 128u; }
+constexpr uint32_t TM_DPT(int b) { return (uint32_t)b * 128u + 64u; }
+constexpr uint32_t TM_DV = 256, TM_DK = 384;
+
+struct Params {
+    const float *lse, *Dws;
+    __nv_bfloat16 *dk, *dv;
+    long L;
+    int T, N, w, r, tpk, tpq;   // key tiles (128) and query tiles (64) per frame
+    float sl2, scale;
+    unsigned int *err;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tg,
+                const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    auto BAR = [&](int i) { return sbase + SM_BAR + 8u * (uint32_t)i; };
+    volatile int *abort_flag = (volatile int *)(smem + SM_ABORT);
+    uint32_t *tmem_slot = (uint32_t *)(smem + SM_TMEMSLOT);
+    float *LD = (float *)(smem + SM_LD);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long bh = blockIdx.y;
+    const int g = blockIdx.x / p.tpk, jt = blockIdx.x % p.tpk;
+    const long k0 = (long)g * p.N + (long)jt * BK;
+    const int nv = min(BK, p.N - jt * BK);
+    const long head = bh * p.L;
+    const int nframes = min(p.w, (p.T - 1 - g) / p.r + 1);
+    const int ntiles = nframes * p.tpq;
+    auto qrow0 = [&](int j) { return head + (long)(g + p.r * (j / p.tpq)) * p.N + (long)(j % p.tpq) * BQ; };
+    auto qcount = [&](int j) { return min(BQ, p.N - (j % p.tpq) * BQ); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_KV), 1);
+        for (int st = 0; st < NS; ++st) {
+            mbar_init(BAR(B_QFULL + st), 1);
+            mbar_init(BAR(B_EMPTY + st), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_SFULL + b), 1);
+            mbar_init(BAR(B_PFULL + b), 128);
+        }
+        mbar_init(BAR(B_ODONE), 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == WARP_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == WARP_TMA) {
+        if (lane == 0) {
+            mbar_expect_tx(BAR(B_KV), 2 * KTILE);
+            const int kr = (int)(head + k0);
+            tma_load_2d(sbase + SM_K, &tk, 0, kr, BAR(B_KV));
+            tma_load_2d(sbase + SM_K + KHALF, &tk, 64, kr, BAR(B_KV));
+            tma_load_2d(sbase + SM_V, &tv, 0, kr, BAR(B_KV));
+            tma_load_2d(sbase + SM_V + KHALF, &tv, 64, kr, BAR(B_KV));
+            int j = 0;
+            for (; j < ntiles; ++j) {
+                const int st = j % NS;
+                if (j >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((j / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
+                mbar_expect_tx(BAR(B_QFULL + st), 2 * QTILE);
+                const int qr = (int)qrow0(j);
+                tma_load_2d(sbase + SM_Q(st), &tq, 0, qr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_Q(st) + QHALF, &tq, 64, qr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_G(st), &tg, 0, qr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_G(st) + QHALF, &tg, 64, qr, BAR(B_QFULL + st));
+            }
+            if (*abort_flag) {
+                // let this CTA's copies in flight land before the CTA may exit
+                const long long t0 = clock64();
+                while (!mbar_try(BAR(B_KV), 0) && clock64() - t0 < (1LL << 31)) {}
+                for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj)
+                    while (!mbar_try(BAR(B_QFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(BK, BQ, false, false);   // K / V and Q / dO K-major
+            constexpr uint32_t IDESC_A = idesc_bf16(BK, D, false, true);     // P^T, dS^T from TMEM; dO, Q MN-major
+            const uint64_t dk_ = sw128_desc(sbase + SM_K, 16, 1024);
+            const uint64_t dv_ = sw128_desc(sbase + SM_V, 16, 1024);
+            auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+                return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
+            };
+            // S^T and dP^T of tile j into buffer j & 1
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % NS, b = j & 1;
+                if (!wait_bar(BAR(B_QFULL + st), (uint32_t)(j / NS) & 1u)) return false;
+                fence_after_sync();
+                const uint64_t dq_ = sw128_desc(sbase + SM_Q(st), 16, 1024);
+                const uint64_t dg_ = sw128_desc(sbase + SM_G(st), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + TM_ST(b), dk_ + aoff, dq_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + TM_DPT(b), dv_ + aoff, dg_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(BAR(B_SFULL + b));
+                return true;
+            };
+            bool ok = wait_bar(BAR(B_KV), 0) && issue_s(0);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
+                const int st = j % NS, b = j & 1;
+                if (!(ok = wait_bar(BAR(B_PFULL + b), (uint32_t)(j >> 1) & 1u))) break;
+                fence_after_sync();
+                // dV += P^T dO_j, dK += dS^T Q_j: 64 queries in 4 steps of 16 (8 TMEM columns each)
+                const uint64_t dgm = sw128_desc(sbase + SM_G(st), QHALF, 1024);
+                const uint64_t dqm = sw128_desc(sbase + SM_Q(st), QHALF, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    umma_bf16_ts(tmem + TM_DV, tmem + TM_ST(b) + kk * 8, dgm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    umma_bf16_ts(tmem + TM_DK, tmem + TM_DPT(b) + kk * 8, dqm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(BAR(B_EMPTY + st));
+            }
+            if (ok) umma_commit(BAR(B_ODONE));
+        }
+    } else {
+        // ---------------------------- elementwise: one thread per key row -------------------
+        const int kr = warp * 32 + lane;
+        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        bool ok = true;
+        float *LDw = LD + warp * 2 * BQ;            // this warp's copy (no wait across warps)
+        for (int j = 0; j < ntiles; ++j) {
+            const int b = j & 1;
+            // this tile's lse2 (log2 units) and D per query column; past the frame: +inf and 0
+            {
+                const long q0 = qrow0(j);
+                const int nq = qcount(j);
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = lane + 32 * h;
+                    LDw[c] = c < nq ? p.lse[q0 + c] * 1.4426950408889634f : INFINITY;
+                    LDw[BQ + c] = c < nq ? p.Dws[q0 + c] : 0.f;
+                }
+                __syncwarp();
+            }
+            const uint32_t sbar = BAR(B_SFULL + b), spar = (uint32_t)(j >> 1) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+            fence_after_sync();
+            uint32_t sr[64], dr[64];
+            tmem_ld64(tlane + TM_ST(b), sr);
+            tmem_ld64(tlane + TM_DPT(b), dr);
+            const float4 *L4 = reinterpret_cast<const float4 *>(LDw);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t pk[16], gk[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 l = L4[c * 8 + i], dd = L4[BQ / 4 + c * 8 + i];
+                    const int col = c * 32 + 4 * i;
+                    const float p0 = ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -l.x));
+                    const float p1 = ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -l.y));
+                    const float p2 = ex2(fmaf(__uint_as_float(sr[col + 2]), p.sl2, -l.z));
+                    const float p3 = ex2(fmaf(__uint_as_float(sr[col + 3]), p.sl2, -l.w));
+                    pk[2 * i] = pack_bf16(p0, p1);
+                    pk[2 * i + 1] = pack_bf16(p2, p3);
+                    gk[2 * i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - dd.x), p1 * (__uint_as_float(dr[col + 1]) - dd.y));
+                    gk[2 * i + 1] = pack_bf16(p2 * (__uint_as_float(dr[col + 2]) - dd.z), p3 * (__uint_as_float(dr[col + 3]) - dd.w));
+                }
+                tmem_st16(tlane + TM_ST(b) + c * 16, pk);
+                tmem_st16(tlane + TM_DPT(b) + c * 16, gk);
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PFULL + b));
+        }
+        // epilogue: dK (times the softmax scale) and dV rows of this thread's key
+        const bool fin = ok && __all_sync(0xffffffffu, mbar_wait(BAR(B_ODONE), 0u, abort_flag, p.err, DEVERR_ATTN_WAIT));
+        if (fin) {
+            fence_after_sync();
+            const long row = head + k0 + kr;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                __nv_bfloat16 *dst = (which ? p.dv : p.dk) + row * D;
+                const float mul = which ? 1.f : p.scale;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tlane + (which ? TM_DV : TM_DK) + c * 32, v);
+                    if (kr < nv) {
+                        uint32_t pk2[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk2[i] = pack_bf16(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
+                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            d4[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
+                    }
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    }
+}
+
+// ----------------------------------------------------------------------------------------
+// dQ: one CTA per 128-row query tile of one frame f; walks the 64-key tiles of the frame's
+// window (f - r i, i < w, >= 0). Per key tile j:
+//   S = Q K_j^T,  dP = dO V_j^T,  dS = exp2(S sl2 - lse2) o (dP - D)   (row constants)
+//   dQ += dS K_j                                                      (dS from tensor memory)
+// Same roles and barrier protocol as the dK / dV kernel with queries and keys exchanged.
+__global__ void __launch_bounds__(THREADS, 1)
+attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tg,
+               const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+               const Params p, __nv_bfloat16 *dq)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    auto BAR = [&](int i) { return sbase + SM_BAR + 8u * (uint32_t)i; };
+    volatile int *abort_flag = (volatile int *)(smem + SM_ABORT);
+    uint32_t *tmem_slot = (uint32_t *)(smem + SM_TMEMSLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long bh = blockIdx.y;
+    const int f = blockIdx.x / p.tpk, ut = blockIdx.x % p.tpk;
+    const long q0 = (long)f * p.N + (long)ut * BK;
+    const int nq = min(BK, p.N - ut * BK);
+    const long head = bh * p.L;
+    const int nframes = min(p.w, f / p.r + 1);
+    const int ntiles = nframes * p.tpq;
+    // key frames from the oldest
+    auto krow0 = [&](int j) { return head + (long)(f - p.r * (nframes - 1 - j / p.tpq)) * p.N + (long)(j % p.tpq) * BQ; };
+    auto kcount = [&](int j) { return min(BQ, p.N - (j % p.tpq) * BQ); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_KV), 1);
+        for (int st = 0; st < NS; ++st) {
+            mbar_init(BAR(B_QFULL + st), 1);
+            mbar_init(BAR(B_EMPTY + st), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_SFULL + b), 1);
+            mbar_init(BAR(B_PFULL + b), 128);
+        }
+        mbar_init(BAR(B_ODONE), 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == WARP_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == WARP_TMA) {
+        if (lane == 0) {
+            // the query tile's Q and dO (128 rows) in the slots of K and V of the other kernel
+            mbar_expect_tx(BAR(B_KV), 2 * KTILE);
+            const int qr = (int)(head + q0);
+            tma_load_2d(sbase + SM_K, &tq, 0, qr, BAR(B_KV));
+            tma_load_2d(sbase + SM_K + KHALF, &tq, 64, qr, BAR(B_KV));
+            tma_load_2d(sbase + SM_V, &tg, 0, qr, BAR(B_KV));
+            tma_load_2d(sbase + SM_V + KHALF, &tg, 64, qr, BAR(B_KV));
+            int j = 0;
+            for (; j < ntiles; ++j) {
+                const int st = j % NS;
+                if (j >= NS && !mbar_wait(BAR(B_EMPTY + st), (uint32_t)((j / NS) + 1) & 1u, abort_flag, p.err, DEVERR_ATTN_WAIT)) break;
+                mbar_expect_tx(BAR(B_QFULL + st), 2 * QTILE);
+                const int kr = (int)krow0(j);
+                tma_load_2d(sbase + SM_Q(st), &tk, 0, kr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_Q(st) + QHALF, &tk, 64, kr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_G(st), &tv, 0, kr, BAR(B_QFULL + st));
+                tma_load_2d(sbase + SM_G(st) + QHALF, &tv, 64, kr, BAR(B_QFULL + st));
+            }
+            if (*abort_flag) {
+                const long long t0 = clock64();
+                while (!mbar_try(BAR(B_KV), 0) && clock64() - t0 < (1LL << 31)) {}
+                for (int jj = j - 1; jj >= 0 && jj >= j - NS; --jj)
+                    while (!mbar_try(BAR(B_QFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(BK, BQ, false, false);   // Q / dO and K / V K-major
+            constexpr uint32_t IDESC_A = idesc_bf16(BK, D, false, true);     // dS from TMEM; K MN-major
+            const uint64_t dq_ = sw128_desc(sbase + SM_K, 16, 1024);
+            const uint64_t dg_ = sw128_desc(sbase + SM_V, 16, 1024);
+            auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+                return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
+            };
+            auto issue_s = [&](int j) -> bool {
+                const int st = j % NS, b = j & 1;
+                if (!wait_bar(BAR(B_QFULL + st), (uint32_t)(j / NS) & 1u)) return false;
+                fence_after_sync();
+                const uint64_t dk_ = sw128_desc(sbase + SM_Q(st), 16, 1024);
+                const uint64_t dv_ = sw128_desc(sbase + SM_G(st), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + TM_ST(b), dq_ + aoff, dk_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + TM_DPT(b), dg_ + aoff, dv_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(BAR(B_SFULL + b));
+                return true;
+            };
+            bool ok = wait_bar(BAR(B_KV), 0) && issue_s(0);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
+                const int st = j % NS, b = j & 1;
+                if (!(ok = wait_bar(BAR(B_PFULL + b), (uint32_t)(j >> 1) & 1u))) break;
+                fence_after_sync();
+                // dQ += dS K_j: 64 keys in 4 steps of 16 (8 TMEM columns each), K MN-major
+                const uint64_t dkm = sw128_desc(sbase + SM_Q(st), QHALF, 1024);
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    umma_bf16_ts(tmem + TM_DV, tmem + TM_DPT(b) + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(BAR(B_EMPTY + st));
+            }
+            if (ok) umma_commit(BAR(B_ODONE));
+        }
+    } else {
+        // ---------------------------- elementwise: one thread per query row -----------------
+        const int qrw = warp * 32 + lane;
+        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        const bool rv = qrw < nq;
+        const float lse2 = rv ? p.lse[head + q0 + qrw] * 1.4426950408889634f : INFINITY;
+        const float Dr = rv ? p.Dws[head + q0 + qrw] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            const int b = j & 1;
+            const int nv = kcount(j);
+            const uint32_t sbar = BAR(B_SFULL + b), spar = (uint32_t)(j >> 1) & 1u;
+            if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
+            fence_after_sync();
+            uint32_t sr[64], dr[64];
+            tmem_ld64(tlane + TM_ST(b), sr);
+            tmem_ld64(tlane + TM_DPT(b), dr);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t gk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int col = c * 32 + 2 * i;
+                    const float p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -lse2)) : 0.f;
+                    const float p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -lse2)) : 0.f;
+                    gk[i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - Dr), p1 * (__uint_as_float(dr[col + 1]) - Dr));
+                }
+                tmem_st16(tlane + TM_DPT(b) + c * 16, gk);
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PFULL + b));
+        }
+        const bool fin = ok && __all_sync(0xffffffffu, mbar_wait(BAR(B_ODONE), 0u, abort_flag, p.err, DEVERR_ATTN_WAIT));
+        if (fin) {
+            fence_after_sync();
+            __nv_bfloat16 *dst = dq + (head + q0 + qrw) * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tlane + TM_DV + c * 32, v);
+                if (rv) {
+                    uint32_t pk2[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk2[i] = pack_bf16(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        d4[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd_tc(const AttnBwdArgs &a, cudaStream_t s)
+{
+    const long L = (long)a.T * a.N;
+    const long rows = (long)a.BH * L;
+    if (rows + BK >= (1L << 31)) return cudaErrorNotSupported;
+    CUtensorMap mk, mv, mq, mg;
+    cudaError_t e;
+    if ((e = make_tmap_2d_bf16(&mk, a.k, rows, D, 64, BK, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mv, a.v, rows, D, 64, BK, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mq, a.q, rows, D, 64, BQ, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mg, a.dO, rows, D, 64, BQ, true)) != cudaSuccess) return e;
+    Params p;
+    p.lse = a.lse; p.Dws = a.Dws;
+    p.dk = (__nv_bfloat16 *)a.dk; p.dv = (__nv_bfloat16 *)a.dv;
+    p.L = L; p.T = a.T; p.N = a.N; p.w = a.w; p.r = a.r;
+    p.tpk = (a.N + BK - 1) / BK;
+    p.tpq = (a.N + BQ - 1) / BQ;
+    p.scale = a.scale;
+    p.sl2 = a.scale * 1.4426950408889634f;
+    p.err = device_error_word();
+    if (!p.err) return cudaErrorUnknown;
+    if ((e = cudaFuncSetAttribute(attn_bwd_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess)
+        return e;
+    const dim3 grid((unsigned)((long)a.T * p.tpk), (unsigned)a.BH);
+    attn_bwd_dkv_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mk, mv, mq, mg, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dQ: query tiles of 128 rows (the maps of the other kernel with the boxes exchanged)
+    CUtensorMap mq2, mg2, mk2, mv2;
+    if ((e = make_tmap_2d_bf16(&mq2, a.q, rows, D, 64, BK, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mg2, a.dO, rows, D, 64, BK, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mk2, a.k, rows, D, 64, BQ, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mv2, a.v, rows, D, 64, BQ, true)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess)
+        return e;
+    attn_bwd_dq_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mq2, mg2, mk2, mv2, p, (__nv_bfloat16 *)a.dq);
+    return cudaGetLastError();
+}
+
+}  // namespace hlta

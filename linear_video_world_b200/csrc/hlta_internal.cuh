@@ -102,6 +102,7 @@ struct AttnBwdArgs {
     float scale;
 };
 cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s);
+cudaError_t launch_attn_bwd_tc(const AttnBwdArgs &a, cudaStream_t s);
 // Gated delta rule backward (chunk form, fp32 arithmetic, d = 128): q, k, v, dO, dq, dk, dv
 // [B][H][L][d] (bf16 when `bf16`, else fp32); a, b, da, db [B][H][L]; S0, dS_final, dS0
 // [B][H][d][d] fp32 (S0 / dS_final null for zero, dS0 null to skip).
