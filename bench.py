@@ -624,8 +624,9 @@ def main():
             bw["attn_bwd_tflops"] = bflop / (bw["attn_bwd_ms"] / 1e3) / 1e12
             bw["attn_bwd_frac"] = bw["attn_bwd_tflops"] / float(pk.get("bf16_tflops"))
         bw["note"] = ("training pass: hlta_window_fwd_lse + hlta_window_bwd for the SWA and DSWA "
-                      "heads (mma.sync products), hlta_gdn_chunk_bwd for the GDN heads (fp32 "
-                      "arithmetic, chunk-start states recomputed); frac against the burst bf16 peak")
+                      "heads (tcgen05 dK/dV and dQ kernels), hlta_gdn_chunk_bwd for the GDN heads "
+                      "(fp32 arithmetic, chunk-start states recomputed); frac against the burst "
+                      "bf16 peak")
         detail["backward"] = bw
     if fp8_ms is not None:
         # E4M3 dense peak = the measured bf16 burst peak x 2 (nominal fp8:bf16 ratio 4.5:2.25)
