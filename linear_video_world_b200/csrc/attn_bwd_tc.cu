@@ -14,9 +14,11 @@
 // of its query sub-tile, the other side's tiles stream through a TMA ring like its key tiles,
 // P^T / dS are written over the first 32 columns of their fp32 buffers as bf16 pairs, and
 // products of one issuing thread execute in issue order, so S of tile j+1 is issued into the
-// buffers that the accumulating products of tile j-1 read without a wait.
+// buffers that the same thread's accumulating products of tile j-1 read without a wait (dQ's S
+// buffer, which only the elementwise warps read, is reissued after their arrival).
 // Threads: warps 0..3 elementwise (one thread per row of the CTA's tile, the warp's TMEM lane
-// quadrant), warp 4 TMA producer, warp 5 MMA issuer and TMEM owner. Tensor memory: per buffer
+// quadrant), warp 4 TMA producer, warps 5 and 6 MMA issuers (one thread issues at a limited
+// rate, so the products are split over two; warp 5 owns TMEM). Tensor memory: per buffer
 // b (two) S at 128 b and dP at 128 b + 64; accumulators at 256 (dV or dQ) and 384 (dK). Every
 // mbarrier wait is bounded.
 #include "hlta_internal.cuh"
@@ -35,8 +37,8 @@ constexpr int BK = 128;                 // keys per CTA (the products' M)
 constexpr int BQ = 64;                  // queries per tile (N of S^T, K of the accumulations)
 constexpr int D = 128;
 constexpr int NS = 3;                   // Q / dO ring stages
-constexpr int THREADS = 192;
-constexpr int WARP_TMA = 4, WARP_MMA = 5;
+constexpr int THREADS = 224;
+constexpr int WARP_TMA = 4, WARP_MMA = 5;   // issuers: warp 5 (A, owns TMEM) and warp 6 (B)
 constexpr uint32_t KHALF = BK * 128;    // [128 rows][64 cols] bf16: 16 KB
 constexpr uint32_t KTILE = 2 * KHALF;
 constexpr uint32_t QHALF = BQ * 128;    // [64 rows][64 cols]: 8 KB
@@ -63,6 +65,8 @@ struct Params {
     float sl2, scale;
     unsigned int *err;
 };
+
+constexpr uint32_t ODONE_DKV = 2, ODONE_DQ = 1;
 
 __global__ void __launch_bounds__(THREADS, 1)
 attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -92,13 +96,13 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         mbar_init(BAR(B_KV), 1);
         for (int st = 0; st < NS; ++st) {
             mbar_init(BAR(B_QFULL + st), 1);
-            mbar_init(BAR(B_EMPTY + st), 1);
+            mbar_init(BAR(B_EMPTY + st), 2);            // both issuers' products on the stage
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(B_SFULL + b), 1);
+            mbar_init(BAR(B_SFULL + b), 2);             // S and dP, one from each issuer
             mbar_init(BAR(B_PFULL + b), 128);
         }
-        mbar_init(BAR(B_ODONE), 1);
+        mbar_init(BAR(B_ODONE), ODONE_DKV);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -140,33 +144,28 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                     while (!mbar_try(BAR(B_QFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
             }
         }
-    } else if (warp == WARP_MMA) {
+    } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
+        // Issuer A: S^T = K Q^T and dV += P^T dO (buffer ST); issuer B: dP^T = V dO^T and
+        // dK += dS^T Q (buffer DPT). Each issuer reuses only its own buffers, in issue order.
         if (lane == 0) {
+            const bool A = warp == WARP_MMA;
             constexpr uint32_t IDESC_S = idesc_bf16(BK, BQ, false, false);   // K / V and Q / dO K-major
             constexpr uint32_t IDESC_A = idesc_bf16(BK, D, false, true);     // P^T, dS^T from TMEM; dO, Q MN-major
-            const uint64_t dk_ = sw128_desc(sbase + SM_K, 16, 1024);
-            const uint64_t dv_ = sw128_desc(sbase + SM_V, 16, 1024);
+            const uint64_t da_ = sw128_desc(sbase + (A ? SM_K : SM_V), 16, 1024);
             auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
                 return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
             };
-            // S^T and dP^T of tile j into buffer j & 1
             auto issue_s = [&](int j) -> bool {
                 const int st = j % NS, b = j & 1;
                 if (!wait_bar(BAR(B_QFULL + st), (uint32_t)(j / NS) & 1u)) return false;
                 fence_after_sync();
-                const uint64_t dq_ = sw128_desc(sbase + SM_Q(st), 16, 1024);
-                const uint64_t dg_ = sw128_desc(sbase + SM_G(st), 16, 1024);
+                const uint64_t db_ = sw128_desc(sbase + (A ? SM_Q(st) : SM_G(st)), 16, 1024);
+                const uint32_t dst = tmem + (A ? TM_ST(b) : TM_DPT(b));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
                     const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
-                    umma_bf16(tmem + TM_ST(b), dk_ + aoff, dq_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
-                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
-                    umma_bf16(tmem + TM_DPT(b), dv_ + aoff, dg_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                    umma_bf16(dst, da_ + aoff, db_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(BAR(B_SFULL + b));
                 return true;
@@ -177,16 +176,12 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 const int st = j % NS, b = j & 1;
                 if (!(ok = wait_bar(BAR(B_PFULL + b), (uint32_t)(j >> 1) & 1u))) break;
                 fence_after_sync();
-                // dV += P^T dO_j, dK += dS^T Q_j: 64 queries in 4 steps of 16 (8 TMEM columns each)
-                const uint64_t dgm = sw128_desc(sbase + SM_G(st), QHALF, 1024);
-                const uint64_t dqm = sw128_desc(sbase + SM_Q(st), QHALF, 1024);
+                // dV += P^T dO_j (A) or dK += dS^T Q_j (B): 64 queries in 4 steps of 16
+                const uint64_t dbm = sw128_desc(sbase + (A ? SM_G(st) : SM_Q(st)), QHALF, 1024);
+                const uint32_t acc = tmem + (A ? TM_DV : TM_DK), src = tmem + (A ? TM_ST(b) : TM_DPT(b));
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    umma_bf16_ts(tmem + TM_DV, tmem + TM_ST(b) + kk * 8, dgm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
-                                 (j > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-                for (int kk = 0; kk < BQ / 16; ++kk)
-                    umma_bf16_ts(tmem + TM_DK, tmem + TM_DPT(b) + kk * 8, dqm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                    umma_bf16_ts(acc, src + kk * 8, dbm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
                                  (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(BAR(B_EMPTY + st));
             }
@@ -313,13 +308,13 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         mbar_init(BAR(B_KV), 1);
         for (int st = 0; st < NS; ++st) {
             mbar_init(BAR(B_QFULL + st), 1);
-            mbar_init(BAR(B_EMPTY + st), 1);
+            mbar_init(BAR(B_EMPTY + st), 2);            // both issuers' products on the stage
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(B_SFULL + b), 1);
+            mbar_init(BAR(B_SFULL + b), 2);             // S and dP, one from each issuer
             mbar_init(BAR(B_PFULL + b), 128);
         }
-        mbar_init(BAR(B_ODONE), 1);
+        mbar_init(BAR(B_ODONE), ODONE_DQ);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -361,39 +356,38 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                     while (!mbar_try(BAR(B_QFULL + jj % NS), (uint32_t)(jj / NS) & 1u) && clock64() - t0 < (1LL << 31)) {}
             }
         }
-    } else if (warp == WARP_MMA) {
+    } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
+        // Issuer A: S = Q K^T (buffer ST; it waits until the elementwise warps have read the S
+        // it overwrites); issuer B: dP = dO V^T and dQ += dS K (buffer DPT, reused in issue order).
         if (lane == 0) {
+            const bool A = warp == WARP_MMA;
             constexpr uint32_t IDESC_S = idesc_bf16(BK, BQ, false, false);   // Q / dO and K / V K-major
             constexpr uint32_t IDESC_A = idesc_bf16(BK, D, false, true);     // dS from TMEM; K MN-major
-            const uint64_t dq_ = sw128_desc(sbase + SM_K, 16, 1024);
-            const uint64_t dg_ = sw128_desc(sbase + SM_V, 16, 1024);
+            const uint64_t da_ = sw128_desc(sbase + (A ? SM_K : SM_V), 16, 1024);
             auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
                 return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
             };
             auto issue_s = [&](int j) -> bool {
                 const int st = j % NS, b = j & 1;
                 if (!wait_bar(BAR(B_QFULL + st), (uint32_t)(j / NS) & 1u)) return false;
+                if (A && j >= 2 && !wait_bar(BAR(B_PFULL + b), (uint32_t)((j - 2) >> 1) & 1u)) return false;
                 fence_after_sync();
-                const uint64_t dk_ = sw128_desc(sbase + SM_Q(st), 16, 1024);
-                const uint64_t dv_ = sw128_desc(sbase + SM_G(st), 16, 1024);
+                const uint64_t db_ = sw128_desc(sbase + (A ? SM_Q(st) : SM_G(st)), 16, 1024);
+                const uint32_t dst = tmem + (A ? TM_ST(b) : TM_DPT(b));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
                     const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
-                    umma_bf16(tmem + TM_ST(b), dq_ + aoff, dk_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = ((kk >> 2) * KHALF + (kk & 3) * 32) >> 4;
-                    const uint32_t boff = ((kk >> 2) * QHALF + (kk & 3) * 32) >> 4;
-                    umma_bf16(tmem + TM_DPT(b), dg_ + aoff, dv_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
+                    umma_bf16(dst, da_ + aoff, db_ + boff, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(BAR(B_SFULL + b));
+                if (A) umma_commit(BAR(B_EMPTY + st));   // A reads the stage's K only here
                 return true;
             };
             bool ok = wait_bar(BAR(B_KV), 0) && issue_s(0);
             for (int j = 0; ok && j < ntiles; ++j) {
                 if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
+                if (A) continue;
                 const int st = j % NS, b = j & 1;
                 if (!(ok = wait_bar(BAR(B_PFULL + b), (uint32_t)(j >> 1) & 1u))) break;
                 fence_after_sync();
@@ -405,7 +399,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                                  (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(BAR(B_EMPTY + st));
             }
-            if (ok) umma_commit(BAR(B_ODONE));
+            if (ok && !A) umma_commit(BAR(B_ODONE));
         }
     } else {
         // ---------------------------- elementwise: one thread per query row -----------------
