@@ -12,13 +12,16 @@
 // walking the 64-key tiles of its window; dQ += dS K_j).
 // The roles mirror the forward kernel (attn_tc.cu): the CTA's own 128-row tile takes the place
 // of its query sub-tile, the other side's tiles stream through a TMA ring like its key tiles,
-// P^T / dS are written over the first 32 columns of their fp32 buffers as bf16 pairs, and
+// P^T / dS are written over their fp32 buffers as bf16 pairs (each half of the columns into the
+// first 16 of its own 32 fp32 columns, so the two warps of a lane quadrant never overwrite each
+// other's unread scores), and
 // products of one issuing thread execute in issue order, so S of tile j+1 is issued into the
 // buffers that the same thread's accumulating products of tile j-1 read without a wait (dQ's S
 // buffer, which only the elementwise warps read, is reissued after their arrival).
-// Threads: warps 0..3 elementwise (one thread per row of the CTA's tile, the warp's TMEM lane
-// quadrant), warp 4 TMA producer, warps 5 and 6 MMA issuers (one thread issues at a limited
-// rate, so the products are split over two; warp 5 owns TMEM). Tensor memory: per buffer
+// Threads: warps 0..7 elementwise (one row of the CTA's tile per lane, the warp's TMEM lane
+// quadrant; warps w and w + 4 split the 64 columns), warp 8 TMA producer, warps 9 and 10 MMA
+// issuers (one thread issues at a limited rate, so the products are split over two; warp 9 owns
+// TMEM). Tensor memory: per buffer
 // b (two) S at 128 b and dP at 128 b + 64; accumulators at 256 (dV or dQ) and 384 (dK). Every
 // mbarrier wait is bounded.
 #include "hlta_internal.cuh"
@@ -37,8 +40,9 @@ constexpr int BK = 128;                 // keys per CTA (the products' M)
 constexpr int BQ = 64;                  // queries per tile (N of S^T, K of the accumulations)
 constexpr int D = 128;
 constexpr int NS = 3;                   // Q / dO ring stages
-constexpr int THREADS = 224;
-constexpr int WARP_TMA = 4, WARP_MMA = 5;   // issuers: warp 5 (A, owns TMEM) and warp 6 (B)
+constexpr int THREADS = 352;
+constexpr int WARP_TMA = 8, WARP_MMA = 9;   // issuers: warp 9 (A, owns TMEM) and warp 10 (B)
+constexpr int EW_THREADS = 256;             // elementwise: 8 warps, two per TMEM lane quadrant
 constexpr uint32_t KHALF = BK * 128;    // [128 rows][64 cols] bf16: 16 KB
 constexpr uint32_t KTILE = 2 * KHALF;
 constexpr uint32_t QHALF = BQ * 128;    // [64 rows][64 cols]: 8 KB
@@ -46,8 +50,8 @@ constexpr uint32_t QTILE = 2 * QHALF;
 constexpr uint32_t SM_K = 0, SM_V = KTILE;
 __host__ __device__ constexpr uint32_t SM_Q(int st) { return 2 * KTILE + (uint32_t)st * 2 * QTILE; }
 __host__ __device__ constexpr uint32_t SM_G(int st) { return SM_Q(st) + QTILE; }
-constexpr uint32_t SM_LD = 2 * KTILE + NS * 2 * QTILE;       // per elementwise warp: lse2[64] | D[64]
-constexpr uint32_t SM_BAR = SM_LD + 4 * 2 * BQ * 4;
+constexpr uint32_t SM_LD = 2 * KTILE + NS * 2 * QTILE;       // per elementwise warp: lse2[32] | D[32]
+constexpr uint32_t SM_BAR = SM_LD + 8 * 64 * 4;
 enum { B_KV = 0, B_QFULL = 1, B_EMPTY = B_QFULL + NS, B_SFULL = B_EMPTY + NS, B_PFULL = B_SFULL + 2,
        B_ODONE = B_PFULL + 2, NBARS = B_ODONE + 1 };
 constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
@@ -100,7 +104,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_SFULL + b), 2);             // S and dP, one from each issuer
-            mbar_init(BAR(B_PFULL + b), 128);
+            mbar_init(BAR(B_PFULL + b), EW_THREADS);
         }
         mbar_init(BAR(B_ODONE), ODONE_DKV);
         *abort_flag = 0;
@@ -181,64 +185,62 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 const uint32_t acc = tmem + (A ? TM_DV : TM_DK), src = tmem + (A ? TM_ST(b) : TM_DPT(b));
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    umma_bf16_ts(acc, src + kk * 8, dbm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                    umma_bf16_ts(acc, src + (kk >> 1) * 32 + (kk & 1) * 8, dbm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
                                  (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(BAR(B_EMPTY + st));
             }
             if (ok) umma_commit(BAR(B_ODONE));
         }
     } else {
-        // ---------------------------- elementwise: one thread per key row -------------------
-        const int kr = warp * 32 + lane;
-        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        // ----------- elementwise: one key row per lane, query columns split over two warps ----
+        // Warps q4 and q4 + 4 share TMEM lanes 32 q4 ..; warp half h takes query columns
+        // 32 h .. 32 h + 31 and writes its bf16 pairs over the first 16 of its own 32 fp32
+        // columns (columns 0..15 and 32..47), which the accumulating products read as A.
+        const int q4 = warp & 3, h = warp >> 2;
+        const int kr = q4 * 32 + lane;
+        const uint32_t tlane = tmem + ((uint32_t)(q4 * 32) << 16);
         bool ok = true;
-        float *LDw = LD + warp * 2 * BQ;            // this warp's copy (no wait across warps)
+        float *LDw = LD + warp * 64;                // this warp's lse2 | D (no wait across warps)
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
-            // this tile's lse2 (log2 units) and D per query column; past the frame: +inf and 0
+            // this tile's lse2 (log2 units) and D of the warp's columns; past the frame: +inf, 0
             {
                 const long q0 = qrow0(j);
                 const int nq = qcount(j);
+                const int c = 32 * h + lane;
                 __syncwarp();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = lane + 32 * h;
-                    LDw[c] = c < nq ? p.lse[q0 + c] * 1.4426950408889634f : INFINITY;
-                    LDw[BQ + c] = c < nq ? p.Dws[q0 + c] : 0.f;
-                }
+                LDw[lane] = c < nq ? p.lse[q0 + c] * 1.4426950408889634f : INFINITY;
+                LDw[32 + lane] = c < nq ? p.Dws[q0 + c] : 0.f;
                 __syncwarp();
             }
             const uint32_t sbar = BAR(B_SFULL + b), spar = (uint32_t)(j >> 1) & 1u;
             if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
-            uint32_t sr[64], dr[64];
-            tmem_ld64(tlane + TM_ST(b), sr);
-            tmem_ld64(tlane + TM_DPT(b), dr);
+            uint32_t sr[32], dr[32];
+            tmem_ld32(tlane + TM_ST(b) + 32 * h, sr);
+            tmem_ld32(tlane + TM_DPT(b) + 32 * h, dr);
             const float4 *L4 = reinterpret_cast<const float4 *>(LDw);
+            uint32_t pk[16], gk[16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t pk[16], gk[16];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 l = L4[c * 8 + i], dd = L4[BQ / 4 + c * 8 + i];
-                    const int col = c * 32 + 4 * i;
-                    const float p0 = ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -l.x));
-                    const float p1 = ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -l.y));
-                    const float p2 = ex2(fmaf(__uint_as_float(sr[col + 2]), p.sl2, -l.z));
-                    const float p3 = ex2(fmaf(__uint_as_float(sr[col + 3]), p.sl2, -l.w));
-                    pk[2 * i] = pack_bf16(p0, p1);
-                    pk[2 * i + 1] = pack_bf16(p2, p3);
-                    gk[2 * i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - dd.x), p1 * (__uint_as_float(dr[col + 1]) - dd.y));
-                    gk[2 * i + 1] = pack_bf16(p2 * (__uint_as_float(dr[col + 2]) - dd.z), p3 * (__uint_as_float(dr[col + 3]) - dd.w));
-                }
-                tmem_st16(tlane + TM_ST(b) + c * 16, pk);
-                tmem_st16(tlane + TM_DPT(b) + c * 16, gk);
+            for (int i = 0; i < 8; ++i) {
+                const float4 l = L4[i], dd = L4[8 + i];
+                const int col = 4 * i;
+                const float p0 = ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -l.x));
+                const float p1 = ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -l.y));
+                const float p2 = ex2(fmaf(__uint_as_float(sr[col + 2]), p.sl2, -l.z));
+                const float p3 = ex2(fmaf(__uint_as_float(sr[col + 3]), p.sl2, -l.w));
+                pk[2 * i] = pack_bf16(p0, p1);
+                pk[2 * i + 1] = pack_bf16(p2, p3);
+                gk[2 * i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - dd.x), p1 * (__uint_as_float(dr[col + 1]) - dd.y));
+                gk[2 * i + 1] = pack_bf16(p2 * (__uint_as_float(dr[col + 2]) - dd.z), p3 * (__uint_as_float(dr[col + 3]) - dd.w));
             }
+            tmem_st16(tlane + TM_ST(b) + 32 * h, pk);
+            tmem_st16(tlane + TM_DPT(b) + 32 * h, gk);
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PFULL + b));
         }
-        // epilogue: dK (times the softmax scale) and dV rows of this thread's key
+        // epilogue: dK (times the softmax scale) and dV of this thread's key, columns 64 h ..
         const bool fin = ok && __all_sync(0xffffffffu, mbar_wait(BAR(B_ODONE), 0u, abort_flag, p.err, DEVERR_ATTN_WAIT));
         if (fin) {
             fence_after_sync();
@@ -248,7 +250,7 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 __nv_bfloat16 *dst = (which ? p.dv : p.dk) + row * D;
                 const float mul = which ? 1.f : p.scale;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 2 * h; c < 2 * h + 2; ++c) {
                     uint32_t v[32];
                     tmem_ld32(tlane + (which ? TM_DV : TM_DK) + c * 32, v);
                     if (kr < nv) {
@@ -258,8 +260,8 @@ attn_bwd_dkv_tc(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                             pk2[i] = pack_bf16(__uint_as_float(v[2 * i]) * mul, __uint_as_float(v[2 * i + 1]) * mul);
                         uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            d4[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
+                        for (int q4_ = 0; q4_ < 4; ++q4_)
+                            d4[q4_] = make_uint4(pk2[4 * q4_], pk2[4 * q4_ + 1], pk2[4 * q4_ + 2], pk2[4 * q4_ + 3]);
                     }
                 }
             }
@@ -312,7 +314,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_SFULL + b), 2);             // S and dP, one from each issuer
-            mbar_init(BAR(B_PFULL + b), 128);
+            mbar_init(BAR(B_PFULL + b), EW_THREADS);
         }
         mbar_init(BAR(B_ODONE), ODONE_DQ);
         *abort_flag = 0;
@@ -395,41 +397,39 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                 const uint64_t dkm = sw128_desc(sbase + SM_Q(st), QHALF, 1024);
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    umma_bf16_ts(tmem + TM_DV, tmem + TM_DPT(b) + kk * 8, dkm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
+                    umma_bf16_ts(tmem + TM_DV, tmem + TM_DPT(b) + (kk >> 1) * 32 + (kk & 1) * 8, dkm + (uint64_t)((kk * 2048) >> 4), IDESC_A,
                                  (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(BAR(B_EMPTY + st));
             }
             if (ok && !A) umma_commit(BAR(B_ODONE));
         }
     } else {
-        // ---------------------------- elementwise: one thread per query row -----------------
-        const int qrw = warp * 32 + lane;
-        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        // ----------- elementwise: one query row per lane, key columns split over two warps ----
+        const int q4 = warp & 3, h = warp >> 2;
+        const int qrw = q4 * 32 + lane;
+        const uint32_t tlane = tmem + ((uint32_t)(q4 * 32) << 16);
         const bool rv = qrw < nq;
         const float lse2 = rv ? p.lse[head + q0 + qrw] * 1.4426950408889634f : INFINITY;
         const float Dr = rv ? p.Dws[head + q0 + qrw] : 0.f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
             const int b = j & 1;
-            const int nv = kcount(j);
+            const int nv = kcount(j) - 32 * h;      // valid key columns of this warp's half
             const uint32_t sbar = BAR(B_SFULL + b), spar = (uint32_t)(j >> 1) & 1u;
             if (!__all_sync(0xffffffffu, mbar_try(sbar, spar) || mbar_wait(sbar, spar, abort_flag, p.err, DEVERR_ATTN_WAIT))) { ok = false; break; }
             fence_after_sync();
-            uint32_t sr[64], dr[64];
-            tmem_ld64(tlane + TM_ST(b), sr);
-            tmem_ld64(tlane + TM_DPT(b), dr);
+            uint32_t sr[32], dr[32];
+            tmem_ld32(tlane + TM_ST(b) + 32 * h, sr);
+            tmem_ld32(tlane + TM_DPT(b) + 32 * h, dr);
+            uint32_t gk[16];
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t gk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int col = c * 32 + 2 * i;
-                    const float p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -lse2)) : 0.f;
-                    const float p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -lse2)) : 0.f;
-                    gk[i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - Dr), p1 * (__uint_as_float(dr[col + 1]) - Dr));
-                }
-                tmem_st16(tlane + TM_DPT(b) + c * 16, gk);
+            for (int i = 0; i < 16; ++i) {
+                const int col = 2 * i;
+                const float p0 = col < nv ? ex2(fmaf(__uint_as_float(sr[col]), p.sl2, -lse2)) : 0.f;
+                const float p1 = col + 1 < nv ? ex2(fmaf(__uint_as_float(sr[col + 1]), p.sl2, -lse2)) : 0.f;
+                gk[i] = pack_bf16(p0 * (__uint_as_float(dr[col]) - Dr), p1 * (__uint_as_float(dr[col + 1]) - Dr));
             }
+            tmem_st16(tlane + TM_DPT(b) + 32 * h, gk);
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PFULL + b));
@@ -439,7 +439,7 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
             fence_after_sync();
             __nv_bfloat16 *dst = dq + (head + q0 + qrw) * D;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tlane + TM_DV + c * 32, v);
                 if (rv) {
@@ -449,8 +449,8 @@ attn_bwd_dq_tc(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
                         pk2[i] = pack_bf16(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
                     uint4 *d4 = reinterpret_cast<uint4 *>(dst + c * 32);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        d4[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
+                    for (int q4_ = 0; q4_ < 4; ++q4_)
+                        d4[q4_] = make_uint4(pk2[4 * q4_], pk2[4 * q4_ + 1], pk2[4 * q4_ + 2], pk2[4 * q4_ + 3]);
                 }
             }
         }
