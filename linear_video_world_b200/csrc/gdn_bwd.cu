@@ -141,6 +141,111 @@ __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const
     __syncthreads();
 }
 
+// The same product on the tensor cores (mma.sync m16n8k16, fp32 accumulation) with A and B
+// rounded to bf16 as they are staged: the bf16 path's block GEMM. Eight warps, each a 16 x 32
+// piece of the 64 x 64 tile; k-steps of 32 staged as [64 rows][32] bf16 with 80-byte rows
+// (conflict-free ldmatrix). M, N multiples of 64, K of 32; same operand conventions as bgemm.
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int TR = 40;              // staged row stride in bf16 elements (80 bytes)
+
+__device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
+                         bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *smf)
+{
+    __nv_bfloat16 *As = reinterpret_cast<__nv_bfloat16 *>(smf), *Bs = As + 64 * TR;  // [m][k], [n][k]
+    const uint32_t sA = (uint32_t)__cvta_generic_to_shared(As), sB = (uint32_t)__cvta_generic_to_shared(Bs);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wm = warp & 3, wn = warp >> 2, g = lane >> 2, t = lane & 3;
+    constexpr int PER = 32 * 64 / THREADS;
+    auto ld_a = [&](int m0, int k0, int e) -> float {
+        int kk, mm;
+        if (tA) { kk = e >> 6; mm = e & 63; return A[(long)(k0 + kk) * lda + m0 + mm]; }
+        kk = e & 31; mm = e >> 5;
+        return A[(long)(m0 + mm) * lda + k0 + kk];
+    };
+    auto ld_b = [&](int n0, int k0, int e) -> float {
+        int kb, nb;
+        if (tB) { kb = e & 31; nb = e >> 5; return B[(long)(n0 + nb) * ldb + k0 + kb]; }
+        kb = e >> 6; nb = e & 63;
+        return B[(long)(k0 + kb) * ldb + n0 + nb];
+    };
+    for (int m0 = 0; m0 < M; m0 += 64)
+        for (int n0 = 0; n0 < N; n0 += 64) {
+            float acc[4][4] = {};
+            float ra[PER], rb[PER];
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                ra[r] = ld_a(m0, 0, threadIdx.x + r * THREADS);
+                rb[r] = ld_b(n0, 0, threadIdx.x + r * THREADS);
+            }
+            for (int k0 = 0; k0 < K; k0 += 32) {
+                __syncthreads();
+#pragma unroll
+                for (int r = 0; r < PER; ++r) {
+                    const int e = threadIdx.x + r * THREADS;
+                    int kk, mm, kb, nb;
+                    if (tA) { kk = e >> 6; mm = e & 63; } else { kk = e & 31; mm = e >> 5; }
+                    if (tB) { kb = e & 31; nb = e >> 5; } else { kb = e >> 6; nb = e & 63; }
+                    As[mm * TR + kk] = __float2bfloat16(ra[r]);
+                    Bs[nb * TR + kb] = __float2bfloat16((s ? s[k0 + kb] : 1.f) * rb[r]);
+                }
+                __syncthreads();
+                if (k0 + 32 < K) {
+#pragma unroll
+                    for (int r = 0; r < PER; ++r) {
+                        ra[r] = ld_a(m0, k0 + 32, threadIdx.x + r * THREADS);
+                        rb[r] = ld_b(n0, k0 + 32, threadIdx.x + r * THREADS);
+                    }
+                }
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t a0, a1, a2, a3;
+                    ldsm4(sA + 2u * (uint32_t)((16 * wm + (lane & 15)) * TR + ks * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
+                    const int mid = lane >> 3;
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t b0, b1, b2, b3;
+                        const int nrow = 32 * wn + 16 * np + 8 * (mid >> 1) + (lane & 7);
+                        ldsm4(sB + 2u * (uint32_t)(nrow * TR + ks * 16 + 8 * (mid & 1)), b0, b1, b2, b3);
+                        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+                        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float *o = O + (long)(m0 + 16 * wm + g + 8 * (e >> 1)) * ldo + n0 + 32 * wn + 8 * nt + 2 * t + (e & 1);
+                    *o = alpha * acc[nt][e] + (beta != 0.f ? beta * *o : 0.f);
+                }
+        }
+    __syncthreads();
+}
+
+// the element type's block GEMM: tensor cores for bf16 tensors, fp32 CUDA cores for fp32
+template <typename E>
+__device__ __forceinline__ void gemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
+                                     bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *sm)
+{
+    if constexpr (sizeof(E) == 2) bgemm_tc(O, ldo, A, lda, tA, B, ldb, tB, s, M, N, K, alpha, beta, sm);
+    else bgemm(O, ldo, A, lda, tA, B, ldb, tB, s, M, N, K, alpha, beta, sm);
+}
+
 // ----------------------------------------------------------------------------------------
 // prep: one CTA per (chunk, head)
 template <typename E>
@@ -177,8 +282,8 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
         w[O_VEC + 5 * C + 1] = (float)n;
     }
     __syncthreads();
-    bgemm(w + O_KK, C, w + O_K, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
-    bgemm(w + O_P, C, w + O_Q, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    gemm<E>(w + O_KK, C, w + O_K, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    gemm<E>(w + O_P, C, w + O_Q, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
     for (int e = tid; e < CC; e += THREADS) {
         const int t = e / C, s = e % C;
         const bool inc = s <= t && t < n;
@@ -201,15 +306,15 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
     __syncthreads();
     for (int e = tid; e < CC; e += THREADS) w[O_T + e] = Tt[e / C][e % C];
     __syncthreads();
-    bgemm(w + O_W, D, w + O_T, C, false, w + O_K, D, false, bg, C, D, C, 1.f, 0.f, sm);
-    bgemm(w + O_UP, D, w + O_T, C, false, w + O_V, D, false, bb, C, D, C, 1.f, 0.f, sm);
+    gemm<E>(w + O_W, D, w + O_T, C, false, w + O_K, D, false, bg, C, D, C, 1.f, 0.f, sm);
+    gemm<E>(w + O_UP, D, w + O_T, C, false, w + O_V, D, false, bb, C, D, C, 1.f, 0.f, sm);
     const float gC = g[C - 1];
     for (int e = tid; e < CD; e += THREADS) {
         const int t = e / D;
         w[O_QT + e] = t < n ? expf(g[t]) * w[O_Q + e] : 0.f;
         w[O_KT + e] = t < n ? expf(gC - g[t]) * w[O_K + e] : 0.f;
     }
-    bgemm(w + O_QT, D, w + O_P, C, false, w + O_W, D, false, nullptr, C, D, C, -1.f, 1.f, sm);
+    gemm<E>(w + O_QT, D, w + O_P, C, false, w + O_W, D, false, nullptr, C, D, C, -1.f, 1.f, sm);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -408,20 +513,20 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     const float *S0 = w + O_S0, *dSC = w + O_DSC;
     // U = Up - W S0^T
     for (int e = tid; e < CD; e += THREADS) w[O_U + e] = w[O_UP + e];
-    bgemm(w + O_U, D, w + O_W, D, false, S0, D, true, nullptr, C, D, D, -1.f, 1.f, sm);
+    gemm<E>(w + O_U, D, w + O_W, D, false, S0, D, true, nullptr, C, D, D, -1.f, 1.f, sm);
     // dU = Kt dS_C^T + P^T dO ;  dR = T^T dU
-    bgemm(w + O_DU, D, w + O_KT, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);
-    bgemm(w + O_DU, D, w + O_P, C, true, w + O_G, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
-    bgemm(w + O_DR, D, w + O_T, C, true, w + O_DU, D, false, nullptr, C, D, C, 1.f, 0.f, sm);
+    gemm<E>(w + O_DU, D, w + O_KT, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);
+    gemm<E>(w + O_DU, D, w + O_P, C, true, w + O_G, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    gemm<E>(w + O_DR, D, w + O_T, C, true, w + O_DU, D, false, nullptr, C, D, C, 1.f, 0.f, sm);
     // C x C: dP = dO U^T, dA' = dR U^T
-    bgemm(w + O_DP, C, w + O_G, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
-    bgemm(w + O_DA, C, w + O_DR, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    gemm<E>(w + O_DP, C, w + O_G, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
+    gemm<E>(w + O_DA, C, w + O_DR, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
     // products with the d x d states
-    bgemm(w + O_DS, D, w + O_G, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);     // dO S0
-    bgemm(w + O_RS, D, w + O_DR, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // dR S0
-    bgemm(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // U dS_C
-    bgemm(w + O_KS, D, w + O_K, D, false, S0, D, true, nullptr, C, D, D, 1.f, 0.f, sm);      // K S0^T
-    bgemm(w + O_KD, D, w + O_K, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);     // K dS_C^T
+    gemm<E>(w + O_DS, D, w + O_G, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);     // dO S0
+    gemm<E>(w + O_RS, D, w + O_DR, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // dR S0
+    gemm<E>(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // U dS_C
+    gemm<E>(w + O_KS, D, w + O_K, D, false, S0, D, true, nullptr, C, D, D, 1.f, 0.f, sm);      // K S0^T
+    gemm<E>(w + O_KD, D, w + O_K, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);     // K dS_C^T
     // per-row sums over the C x C products (threads 0..63 rows, 64..127 columns) and the
     // C x d ones (threads 128..191)
     if (tid < C) {
@@ -495,15 +600,15 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     __syncthreads();
     // dQ = diag(e^g) dO S0 + (dP o Gam) K
     for (int e = tid; e < CD; e += THREADS) w[O_DQ + e] = expf(g[e / D]) * w[O_DS + e];
-    bgemm(w + O_DQ, D, w + O_DP, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    gemm<E>(w + O_DQ, D, w + O_DP, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     // dK = diag(e^{g_C - g}) U dS_C - diag(b e^g) dR S0 + (dP o Gam)^T Q + M K + M^T K
     for (int e = tid; e < CD; e += THREADS) {
         const int t = e / D;
         w[O_DK + e] = t < n ? expf(gC - g[t]) * w[O_UD + e] - bb[t] * expf(g[t]) * w[O_RS + e] : 0.f;
     }
-    bgemm(w + O_DK, D, w + O_DP, C, true, w + O_Q, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
-    bgemm(w + O_DK, D, w + O_DA, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
-    bgemm(w + O_DK, D, w + O_DA, C, true, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    gemm<E>(w + O_DK, D, w + O_DP, C, true, w + O_Q, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    gemm<E>(w + O_DK, D, w + O_DA, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
+    gemm<E>(w + O_DK, D, w + O_DA, C, true, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     const long base = ((long)bh * p.L + (long)c * C) * D;
     for (int e = tid; e < n * D; e += THREADS) {
         stf((E *)p.dq, base + e, w[O_DQ + e]);
