@@ -338,8 +338,22 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q, const void *
                                     int F, void *stream);
 
 /* Device pointer to the carried GDN state [B, Hg, d, d] (owned by the cache) and the
- * number of frames appended so far. */
+ * number of frames appended so far by the calls made on the host. */
 hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done);
+
+/*
+ * Replaying steps (the rollout part of deployment: the pages' streaming-token design runs the
+ * same step frame after frame). A step's frame index lives in a device counter owned by the
+ * cache: the ring appends and the attention kernels read it when they run, and every step
+ * ends by advancing it by F in stream order. A step captured into a CUDA graph (stream capture
+ * on `stream`, whose library-internal branch streams join the capture through events) can
+ * therefore be replayed for successive frames, with the new frame's inputs written into the
+ * captured input buffers before each replay; the host-side count of hlta_stream_state then
+ * counts calls, not replays. The cache creates the library's per-device helpers, so no step
+ * needs to do so during a capture. *f_dev receives the counter's device address (an int,
+ * owned by the cache): the number of frames appended so far, replays included.
+ */
+hlta_status hlta_stream_frame_counter(hlta_stream_t c, int **f_dev);
 
 /* Frees the cache. Synchronizes the device first. */
 hlta_status hlta_stream_destroy(hlta_stream_t c);

@@ -55,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "hlta_stream_step_frames": (I, [P, P, P, P, P, P, P, I, P]),
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
+        "hlta_stream_frame_counter": (I, [P, ctypes.POINTER(P)]),
         "hlta_fp8_quantize_rows": (I, [P, P, I, I, L, I, L, I, P, P, P]),
         "hlta_fp8_quantize_channels": (I, [P, I, I, L, I, P, P, P]),
         "hlta_window_fp8_fwd": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
@@ -471,6 +472,13 @@ class Stream:
         ptr, n = ctypes.c_void_p(), ctypes.c_int()
         _check(_lib.hlta_stream_state(self._h, ctypes.byref(ptr), ctypes.byref(n)))
         return ptr.value, n.value
+
+    def frame_counter(self):
+        """Device address of the cache's frame counter (an int advanced by every step, in
+        stream order, replays of a captured step included)."""
+        ptr = ctypes.c_void_p()
+        _check(_lib.hlta_stream_frame_counter(self._h, ctypes.byref(ptr)))
+        return ptr.value
 
     def state_tensor(self):
         """A torch copy of the carried state [B, Hg, d, d] fp32 (ordered on the current stream)."""

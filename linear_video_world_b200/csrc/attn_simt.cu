@@ -58,8 +58,9 @@ __global__ void __launch_bounds__(THREADS) attn_f32_kernel(AttnArgs p)
         Qs[e] = rr < nrows ? q[(l0 + rr) * d + c] : 0.f;
     }
 
-    const int fa = p.fq0 + (int)(l0 / p.N);
-    const int fb = p.fq0 + (int)((l0 + nrows - 1) / p.N);
+    const int fq0 = p.fq0_dev ? *p.fq0_dev : p.fq0;
+    const int fa = fq0 + (int)(l0 / p.N);
+    const int fb = fq0 + (int)((l0 + nrows - 1) / p.N);
     const int span = p.r * (p.w - 1);
 
     // per warp: rows warp*4 .. warp*4+3; per row running max m, sum l, output dims per lane
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(THREADS) attn_f32_kernel(AttnArgs p)
     for (int i = 0; i < 4; ++i) {
         int rr = warp * 4 + i;
         valid[i] = rr < nrows;
-        fq[i] = p.fq0 + (int)((l0 + rr) / p.N);
+        fq[i] = fq0 + (int)((l0 + rr) / p.N);
         m[i] = -INFINITY;
         l[i] = 0.f;
 #pragma unroll

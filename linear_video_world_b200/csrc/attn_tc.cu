@@ -99,6 +99,7 @@ struct TcParams {
     int Hbr, q_Htot, q_h0, kv_Htot, kv_h0, kv_slots;
     long q_rows, kv_rows;
     int N, w, r, fq0;
+    const int *fq0_dev;         // if set, the frame of query row 0 is read here (streaming steps)
     float sl2;                  // softmax scale * log2(e)
     const float *qs, *ks, *vs;  // E4M3 scales: [heads][nqb], [heads][nkb], [heads][128]
     int nqb, nkb;               // per head: query blocks of 128 rows, key tiles (slot * tpf + tile)
@@ -419,10 +420,11 @@ __device__ __forceinline__ void attn_body(const CUtensorMap &tq, const CUtensorM
     // frame ranges of the two sub-tiles (sub-tile 1 may be empty in the last CTA of a head);
     // scalars, not arrays indexed by the sub-tile, so nothing lands in local memory
     const long r1_0 = min(l0 + BM, p.q_rows) - 1;
-    const int fa0 = p.fq0 + (int)(l0 / p.N), fb0 = p.fq0 + (int)(r1_0 / p.N);
+    const int fq0 = p.fq0_dev ? *p.fq0_dev : p.fq0;
+    const int fa0 = fq0 + (int)(l0 / p.N), fb0 = fq0 + (int)(r1_0 / p.N);
     const bool valid1 = l0 + BM < p.q_rows;
-    const int fa1 = valid1 ? p.fq0 + (int)((l0 + BM) / p.N) : fa0;
-    const int fb1 = valid1 ? p.fq0 + (int)((min(l0 + 2 * BM, p.q_rows) - 1) / p.N) : fa1;
+    const int fa1 = valid1 ? fq0 + (int)((l0 + BM) / p.N) : fa0;
+    const int fb1 = valid1 ? fq0 + (int)((min(l0 + 2 * BM, p.q_rows) - 1) / p.N) : fa1;
     Walk wk;
     wk.fa0 = fa0;
     wk.fb0 = fb0;
@@ -617,7 +619,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap &tq, const CUtensorM
         const int row = quad * 32 + lane;
         const long lrow = l0 + q * BM + row;
         const bool row_valid = lrow < p.q_rows;
-        const int fq = p.fq0 + (int)(lrow / p.N);
+        const int fq = fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
         // E4M3: scores carry the Q block's scale (per sub-tile) and the K tile's (per tile);
         // sub-tile 1 of a head's last CTA may lie past the last query block
@@ -895,7 +897,7 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     TcParams p;
     p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
     p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
-    p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0;
+    p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0; p.fq0_dev = a.fq0_dev;
     p.sl2 = a.scale * 1.4426950408889634f;
     p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
     p.lse = a.lse;

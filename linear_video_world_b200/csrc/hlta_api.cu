@@ -238,7 +238,9 @@ struct hlta_stream {
     float *S;                 // [B][Hg][d][d]
     void *ws;                 // GDN workspace for max_frames * N tokens
     size_t ws_bytes;
-    int frames;
+    int frames;               // steps' frames appended, counted on the host per call
+    int *fdev;                // the same count on the device: the kernels read it and each step
+                              // advances it in stream order, so a captured step can be replayed
 };
 
 extern "C" {
@@ -599,7 +601,7 @@ hlta_status hlta_stream_create_ex(hlta_stream_t *out, int B, int Hs, int Hd, int
     if (Hd && (st = check_window(w_dswa, r)) != HLTA_OK) return st;
     if (Hg && chunk != 64) return fail(HLTA_ERR_UNSUPPORTED, "chunk must be 64");
     if (S0 && !aligned16(S0)) return fail(HLTA_ERR_INVALID_ARG, "S0 must be 16-byte aligned");
-    DeviceCtx *ctx;
+    DeviceCtx *ctx;   // the device helpers (library streams, events) exist before any capture
     if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
     hlta_stream *c = new (std::nothrow) hlta_stream();
     if (!c) return fail(HLTA_ERR_CUDA, "host allocation failed");
@@ -621,6 +623,8 @@ hlta_status hlta_stream_create_ex(hlta_stream_t *out, int B, int Hs, int Hd, int
     if (bd && e == cudaSuccess) e = cudaMalloc(&c->vd, bd);
     if (Hg && e == cudaSuccess) e = cudaMalloc((void **)&c->S, (size_t)B * Hg * d * d * sizeof(float));
     if (Hg && e == cudaSuccess) e = cudaMalloc(&c->ws, c->ws_bytes);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&c->fdev, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(c->fdev, 0, sizeof(int));
     if (e == cudaSuccess && Hg) {
         if (S0) e = cudaMemcpy(c->S, S0, (size_t)B * Hg * d * d * sizeof(float), cudaMemcpyDeviceToDevice);
         else e = cudaMemset(c->S, 0, (size_t)B * Hg * d * d * sizeof(float));
@@ -698,8 +702,8 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         const Branch &x = br[bi];
         if (!x.Hbr) continue;
         cudaStream_t s = (bi == 1 && split_d) ? ctx->aux2 : (cudaStream_t)stream;
-        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rk, x.slots, f, s)) != cudaSuccess ||
-            (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rv, x.slots, f, s)) != cudaSuccess) {
+        if ((e = launch_ring_append(k_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rk, x.slots, f, c->fdev, s)) != cudaSuccess ||
+            (e = launch_ring_append(v_new, c->B, H, x.h0, x.Hbr, c->N, c->d, el, F, x.rv, x.slots, f, c->fdev, s)) != cudaSuccess) {
             st = cuda_fail(e, "ring append");
             break;
         }
@@ -708,7 +712,7 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         a.B = c->B; a.Hbr = x.Hbr;
         a.q_Htot = H; a.q_h0 = x.h0; a.q_rows = (long)F * c->N;
         a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
-        a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.scale = c->scale;
+        a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.fq0_dev = c->fdev; a.scale = c->scale;
         a.err = ctx->err;
         if ((st = run_attn(a, c->dt, s)) != HLTA_OK) break;
     }
@@ -719,7 +723,15 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
     }
     if (c->Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     if (st != HLTA_OK) return st;
+    if ((e = launch_frame_advance(c->fdev, F, s)) != cudaSuccess) return cuda_fail(e, "frame counter");
     c->frames = f + F;
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_frame_counter(hlta_stream_t c, int **f_dev)
+{
+    if (!c || !f_dev) return fail(HLTA_ERR_INVALID_ARG, "null argument");
+    *f_dev = c->fdev;
     return HLTA_OK;
 }
 
@@ -738,7 +750,7 @@ hlta_status hlta_stream_destroy(hlta_stream_t c)
     cudaGetDevice(&prev);
     cudaSetDevice(c->device);
     cudaDeviceSynchronize();
-    void *bufs[] = {c->ks, c->vs, c->kd, c->vd, c->S, c->ws};
+    void *bufs[] = {c->ks, c->vs, c->kd, c->vd, c->S, c->ws, c->fdev};
     for (void *p : bufs)
         if (p) cudaFree(p);
     if (prev >= 0) cudaSetDevice(prev);

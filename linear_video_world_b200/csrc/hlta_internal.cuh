@@ -25,6 +25,7 @@ struct AttnArgs {
     int kv_slots;
     int N, d, w, r;
     int fq0;
+    const int *fq0_dev = nullptr;   // if set, fq0 is read from this device int when the kernel runs
     float scale;
     unsigned int *err;   // device error word (bounded waits that expired)
     // E4M3 inputs only: fp32 scales of the query blocks ([B*q_Htot][ceil(q_rows/128)]), the
@@ -120,8 +121,13 @@ size_t gdn_bwd_workspace_bytes(long BH, long L);
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
+// f0: the first new frame's index, read from f0_dev when that is set (streaming steps keep
+// their frame counter on the device so that a captured step can be replayed)
 cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,
-                               size_t elem, int F, void *ring, int slots, int f0, cudaStream_t s);
+                               size_t elem, int F, void *ring, int slots, int f0,
+                               const int *f0_dev, cudaStream_t s);
+// *f += F on the device (one thread), in stream order
+cudaError_t launch_frame_advance(int *f, int F, cudaStream_t s);
 
 // Device error word: kernels OR a code into it when a bounded wait expires.
 enum : unsigned int {

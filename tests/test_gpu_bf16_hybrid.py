@@ -160,3 +160,56 @@ def test_stream_step_frames_rejects_too_many_frames(h):
         st.step_frames(q, k, v, a, b, 3)
     assert st.state()[1] == 0                  # nothing was appended
     st.close()
+
+
+def _frame_counter(st):
+    ptr = st.frame_counter()
+
+    class _View:
+        __cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (ptr, False),
+                                    "version": 2}
+    return int(torch.as_tensor(_View(), device="cuda").item())
+
+
+def test_stream_step_graph_replay_equals_hybrid_bf16(h, orc):
+    """A step captured once into a CUDA graph and replayed for successive frames (inputs
+    written into the captured buffers before each replay), with eager steps before and after,
+    reproduces the hybrid operator on the concatenated clip: the frame index the ring appends
+    and the attention read comes from the cache's device counter, advanced by every replay."""
+    F = 2
+    wl = hi.Workload("t", B=2, Hs=1, Hd=1, Hg=1, d=128, T=16, N=130, w_swa=3, w_dswa=4, r=2,
+                     chunk=64, dtype="bf16", decay=1.0)
+    x = hi.make_inputs(wl, seed=23)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    st = h.Stream(wl.B, wl.Hs, wl.Hd, wl.Hg, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r,
+                  max_step_frames=F)
+
+    def part(t, f0):
+        return t[:, :, f0 * wl.N:(f0 + F) * wl.N].contiguous()
+
+    outs = [st.step_frames(*(part(t, 0) for t in (q, k, v, a, b)), F)]     # eager, frames 0-1
+    static = [part(t, 0).clone() for t in (q, k, v, a, b)]
+    so = torch.empty_like(static[0])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        st.step_frames(*static, F, out=so)                                  # captured, not run
+    assert _frame_counter(st) == F                                         # capture ran nothing
+    f0 = F
+    while f0 < wl.T - F:                                                   # replays, frames 2-13
+        for buf, t in zip(static, (q, k, v, a, b)):
+            buf.copy_(part(t, f0))
+        g.replay()
+        outs.append(so.clone())
+        f0 += F
+    outs.append(st.step_frames(*(part(t, f0) for t in (q, k, v, a, b)), F))  # eager again
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    assert _frame_counter(st) == wl.T
+    o = torch.cat(outs, dim=2)
+    o_ref, S_ref = orc.hybrid(x["q"], x["k"], x["v"], x["a"], x["b"], wl.Hs, wl.Hd, wl.Hg,
+                              wl.T, wl.N, wl.w_swa, wl.w_dswa, wl.r)
+    assert maxabs(o, o_ref) <= TOL
+    assert maxabs(st.state_tensor(), S_ref) <= TOL
+    del g
+    st.close()
