@@ -633,11 +633,18 @@ cudaError_t launch_typed(const BwdP &p, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// fp32 chunk scratch, then the bf16 forward's chunk products (the bf16 path's state passes
+// run on the tensor cores from those)
+size_t bwd_f32_bytes(long BH, long L)
+{
+    return ((size_t)BH * (size_t)gdn_num_chunks(L, C) * (size_t)CHUNK_FLOATS * sizeof(float) + 255) & ~(size_t)255;
+}
+
 }  // namespace
 
 size_t gdn_bwd_workspace_bytes(long BH, long L)
 {
-    return (size_t)BH * (size_t)gdn_num_chunks(L, C) * (size_t)CHUNK_FLOATS * sizeof(float);
+    return bwd_f32_bytes(BH, L) + gdn_workspace_bytes(BH, L, D, C, true);
 }
 
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
@@ -654,7 +661,24 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
     p.L = a.L;
     p.BH = a.B * a.H;
     p.nch = (int)nch;
-    return a.bf16 ? launch_typed<__nv_bfloat16>(p, s) : launch_typed<float>(p, s);
+    if (!a.bf16) return launch_typed<float>(p, s);
+    // bf16: the state passes on the tensor cores, from the forward's bf16 chunk products
+    cudaError_t e;
+    gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    GdnArgs g = {};
+    g.q = a.q; g.k = a.k; g.v = a.v; g.a = a.a; g.b = a.b;
+    g.o = nullptr;
+    g.B = a.B; g.Hg = a.H; g.Htot = a.H; g.h0 = 0; g.L = a.L; g.d = D; g.chunk = C;
+    g.S0 = a.S0;
+    g.ws = (char *)a.ws + bwd_f32_bytes(p.BH, a.L);
+    g.ws_bytes = gdn_workspace_bytes(p.BH, a.L, D, C, true);
+    g.err = a.err;
+    g.S_chunks = p.ws + O_S0;
+    g.S_chunk_stride = CHUNK_FLOATS;
+    if ((e = launch_gdn_bf16_bwd_states(g, a.dO, a.dS_final, p.ws + O_DSC, a.dS0, s)) != cudaSuccess) return e;
+    gdn_bwd_grad<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace hlta

@@ -569,6 +569,19 @@ __device__ __forceinline__ void state_times_tiles(float (&dq)[8][4], float (&dw)
     }
 }
 
+// a warp's 16 state rows (accumulator tiles over the 128 key columns) to a row-major
+// [128][128] fp32 matrix at `dst` (rows i0 .. i0 + 15)
+__device__ __forceinline__ void store_rows(float *dst, const float (&st)[16][4], int i0, int lane)
+{
+    const int g8 = lane >> 2, tg = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+            *reinterpret_cast<float2 *>(dst + (long)(i0 + g8 + hh * 8) * D + nt * 8 + 2 * tg) =
+                make_float2(st[nt][2 * hh], st[nt][2 * hh + 1]);
+}
+
 __global__ void __launch_bounds__(STATE_THREADS, 1)
 gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace ws)
 {
@@ -636,6 +649,7 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
     const uint32_t stage_a = smem_u32(stage);
 
     for (long c = 0; c < nch; ++c) {
+        if (p.S_chunks) store_rows(p.S_chunks + ((long)bh * nch + c) * p.S_chunk_stride, st, c0 + r0, lane);
         StateBuf &cur = s.buf[c % NSTAGE];
         const uint32_t fb = smem_u32(&s.full[c % NSTAGE]), fp = (uint32_t)(c / NSTAGE) & 1u;
         if (!__all_sync(0xffffffffu, ptx::mbar_try(fb, fp) || ptx::mbar_wait(fb, fp, abort_flag, p.err, DEVERR_GDN_WAIT)))
@@ -644,8 +658,8 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
         const long t0 = c * C;
         float dq[8][4], dw[8][4];
         state_times_tiles(dq, dw, st, cur.Q, cur.W, lane);
-        // O = Op^T + S Qt^T (old S)
-        {
+        // O = Op^T + S Qt^T (old S); skipped when only the chunk states are wanted
+        if (p.o) {
             uint32_t ov[8][2];
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
@@ -719,6 +733,184 @@ gdn_state_bf16(const __grid_constant__ StateMaps maps, GdnArgs p, GdnWorkspace w
             }
 }
 
+// -----------------------------------------------------------------------------------------
+// backward state pass (training)
+// -----------------------------------------------------------------------------------------
+// The state gradient carried from the last chunk to the first. With S_end = gam S + U^T Kt,
+// U = Up - W S^T and O = Op + Qt S^T, the gradient of the chunk's start state S is
+//   dS = gam dS_end - (dS_end Kt^T) W + dO^T Qt.
+// Rows i of dS evolve independently, so the layout is the forward pass's: two CTAs per head,
+// four warps of 16 rows each, kept in registers as accumulator tiles over the key columns j.
+// Per chunk (last to first): X = dS_end Kt^T (A operand: dS_end repacked to bf16; B: Kt),
+// then dS = gam dS_end + [-X | dO^T] [W; Qt] (A operands: -X straight from X's accumulator
+// tiles, dO^T by transposing ldmatrix from the chunk's dO rows; B: W, Qt). Each chunk's
+// end-state gradient is stored before the chunk is processed.
+struct DStateBuf {
+    alignas(1024) uint8_t W[SWT];          // W  [64 t][128 j]
+    alignas(1024) uint8_t Q[SWT];          // Qt
+    alignas(1024) uint8_t K[SWT];          // Kt
+    alignas(1024) uint8_t G[SLICE];        // dO [64 t][64 i] on this CTA's state rows
+    alignas(16) float gam[4];
+};
+struct DStateSmem {
+    DStateBuf buf[NSTAGE];
+    alignas(8) uint64_t full[NSTAGE];
+    alignas(8) uint64_t empty[NSTAGE];     // count SWARPS
+    int abort_flag;
+};
+constexpr uint32_t DSTAGE_TX = 3 * SWT + SLICE + 16;
+
+struct DStateMaps {
+    CUtensorMap W, Q, K;                   // [BHg*nch*64][128]: 64x64 swizzled boxes
+    CUtensorMap G;                         // dO [B*Htot*L][128]: 64x64 swizzled boxes
+};
+
+// A fragment (16 rows x 16 k) of A = B^T from a swizzled tile holding B row-major ([k][m]):
+// four transposed 8x8 matrices (m 0-7 | 8-15) x (k 0-7 | 8-15)
+__device__ __forceinline__ void frag_a_t_sw(uint32_t (&r)[4], const uint8_t *tile, int m0, int k0, int lane)
+{
+    const int q = lane >> 3;
+    ldsm_x4_t(r, smem_u32(tile + sw128_off(k0 + (q >> 1) * 8 + (lane & 7), m0 + (q & 1) * 8, C)));
+}
+
+// the k-th chunk processed (chunk c = nch - 1 - k) into stage k % NSTAGE
+__device__ __forceinline__ void issue_dchunk(DStateSmem &s, const DStateMaps &maps, const GdnWorkspace &ws,
+                                             int bh, long nch, long c, long k, long g_row, int c0)
+{
+    DStateBuf &bf = s.buf[k % NSTAGE];
+    const uint32_t bar = smem_u32(&s.full[k % NSTAGE]);
+    ptx::mbar_expect_tx(bar, DSTAGE_TX);
+    const int row = (int)(((long)bh * nch + c) * C);
+    for (int hf = 0; hf < 2; ++hf) {
+        ptx::tma_load_2d(smem_u32(bf.W + hf * (SWT / 2)), &maps.W, hf * 64, row, bar);
+        ptx::tma_load_2d(smem_u32(bf.Q + hf * (SWT / 2)), &maps.Q, hf * 64, row, bar);
+        ptx::tma_load_2d(smem_u32(bf.K + hf * (SWT / 2)), &maps.K, hf * 64, row, bar);
+    }
+    ptx::tma_load_2d(smem_u32(bf.G), &maps.G, c0, (int)(g_row + c * C), bar);
+    ptx::bulk_load(smem_u32(bf.gam), ws.gam + ((long)bh * nch + c) * 4, 16, bar);
+}
+
+__global__ void __launch_bounds__(STATE_THREADS, 1)
+gdn_dstate_bf16(const __grid_constant__ DStateMaps maps, GdnArgs p, GdnWorkspace ws,
+                const float *dS_final, float *dS_chunks, float *dS0)
+{
+    extern __shared__ uint8_t smem_raw[];
+    DStateSmem &s = *reinterpret_cast<DStateSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int bh = blockIdx.y;
+    const int b = bh / p.Hg, h = bh % p.Hg;
+    const long nch = gdn_num_chunks(p.L, C);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, tg = lane & 3;
+    const int c0 = blockIdx.x * CW;
+    const int r0 = warp * 16;
+
+    if (tid == 0) {
+        for (int i = 0; i < NSTAGE; ++i) {
+            ptx::mbar_init(smem_u32(&s.full[i]), 1);
+            ptx::mbar_init(smem_u32(&s.empty[i]), SWARPS);
+        }
+        s.abort_flag = 0;
+        ptx::mbar_init_fence();
+    }
+    volatile int *abort_flag = (volatile int *)&s.abort_flag;
+    if (warp == SWARPS) {
+        // ------------------------------ TMA producer --------------------------------------
+        __syncthreads();
+        if (lane == 0) {
+            const long g_row = (long)(b * p.Htot + p.h0 + h) * p.L;
+            long k = 0;
+            for (; k < nch; ++k) {
+                if (k >= NSTAGE) {
+                    const uint32_t eb = smem_u32(&s.empty[k % NSTAGE]);
+                    const uint32_t ep = (uint32_t)((k - NSTAGE) / NSTAGE) & 1u;
+                    if (!(ptx::mbar_try(eb, ep) || ptx::mbar_wait(eb, ep, abort_flag, p.err, DEVERR_GDN_WAIT))) break;
+                }
+                issue_dchunk(s, maps, ws, bh, nch, nch - 1 - k, k, g_row, c0);
+            }
+            if (*abort_flag) {
+                const long long tw = clock64();
+                for (long kk = k - 1; kk >= 0 && kk >= k - NSTAGE; --kk) {
+                    const uint32_t bar = smem_u32(&s.full[kk % NSTAGE]);
+                    while (!ptx::mbar_try(bar, (uint32_t)(kk / NSTAGE) & 1u) && clock64() - tw < (1LL << 31)) {}
+                }
+            }
+        }
+        return;
+    }
+    // this warp's rows of the state gradient: ds[nt] holds (i = g8, g8 + 8) x (j = 8 nt + 2 tg, +1)
+    float ds[16][4];
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int i = c0 + r0 + g8 + (e >> 1) * 8;
+            const int j = nt * 8 + 2 * tg + (e & 1);
+            ds[nt][e] = dS_final ? dS_final[((long)bh * D + i) * D + j] : 0.f;
+        }
+    __syncthreads();
+
+    for (long k = 0; k < nch; ++k) {
+        const long c = nch - 1 - k;
+        if (dS_chunks) store_rows(dS_chunks + ((long)bh * nch + c) * p.S_chunk_stride, ds, c0 + r0, lane);
+        DStateBuf &cur = s.buf[k % NSTAGE];
+        const uint32_t fb = smem_u32(&s.full[k % NSTAGE]), fp = (uint32_t)(k / NSTAGE) & 1u;
+        if (!__all_sync(0xffffffffu, ptx::mbar_try(fb, fp) || ptx::mbar_wait(fb, fp, abort_flag, p.err, DEVERR_GDN_WAIT)))
+            return;                                        // the producer waits for its copies
+        const float gam = cur.gam[0];
+        // X = dS_end Kt^T (tokens 8 nt .. 8 nt + 7)
+        float x[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[nt][e] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < D / 16; ++kb) {
+            uint32_t a[4];
+            a[0] = pack_acc(ds[2 * kb][0], ds[2 * kb][1]);
+            a[1] = pack_acc(ds[2 * kb][2], ds[2 * kb][3]);
+            a[2] = pack_acc(ds[2 * kb + 1][0], ds[2 * kb + 1][1]);
+            a[3] = pack_acc(ds[2 * kb + 1][2], ds[2 * kb + 1][3]);
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t bk[4];
+                frag_b_nk_sw(bk, cur.K, np * 16, kb * 16, lane);      // Kt rows = tokens (n), cols = j (k)
+                mma16816(x[2 * np], a, bk[0], bk[1]);
+                mma16816(x[2 * np + 1], a, bk[2], bk[3]);
+            }
+        }
+        // -X as the A fragments of the update product (tokens as k)
+        uint32_t xa[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                xa[nt >> 1][(nt & 1) * 2 + hh] = pack_acc(-x[nt][2 * hh], -x[nt][2 * hh + 1]);
+        // dS = gam dS_end - X W + dO^T Qt
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ds[nt][e] *= gam;
+#pragma unroll
+        for (int kb = 0; kb < C / 16; ++kb) {
+            uint32_t ga[4];
+            frag_a_t_sw(ga, cur.G, r0, kb * 16, lane);                 // dO^T: rows i, k = tokens
+#pragma unroll
+            for (int np = 0; np < 8; ++np) {
+                uint32_t bw[4], bq[4];
+                frag_b_kn_sw(bw, cur.W, kb * 16, np * 16, lane);      // rows = tokens (k), cols = j (n)
+                frag_b_kn_sw(bq, cur.Q, kb * 16, np * 16, lane);
+                mma16816(ds[2 * np], xa[kb], bw[0], bw[1]);
+                mma16816(ds[2 * np + 1], xa[kb], bw[2], bw[3]);
+                mma16816(ds[2 * np], ga, bq[0], bq[1]);
+                mma16816(ds[2 * np + 1], ga, bq[2], bq[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(smem_u32(&s.empty[k % NSTAGE]));
+    }
+    if (dS0) store_rows(dS0 + (long)bh * D * D, ds, c0 + r0, lane);
+}
+
 }  // namespace
 
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
@@ -752,6 +944,47 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,
+                                       float *dS_chunks, float *dS0, cudaStream_t s)
+{
+    if (g.d != D || g.o != nullptr || !g.S_chunks) return cudaErrorNotSupported;
+    const long nch = gdn_num_chunks(g.L, C);
+    const long BH = (long)g.B * g.Hg;
+    const long in_rows = (long)g.B * g.Htot * g.L;
+    const long ws_rows = BH * nch * C;
+    if (nch > 0x7fffffffL || in_rows + C >= (1L << 31) || ws_rows >= (1L << 31))
+        return cudaErrorNotSupported;
+    GdnWorkspace ws = gdn_workspace_carve(g.ws, BH, g.L, D, C, true);
+    cudaError_t e;
+    PrepMaps pm;
+    if ((e = make_tmap_2d_bf16(&pm.q, g.q, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&pm.k, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&pm.v, g.v, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    StateMaps sm;
+    if ((e = make_tmap_2d_bf16(&sm.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
+    DStateMaps dm;
+    dm.W = sm.W;
+    dm.Q = sm.Q;
+    dm.K = sm.K;
+    if ((e = make_tmap_2d_bf16(&dm.G, dO, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    const size_t smem_prep = sizeof(PrepSmem) + 1024;
+    const size_t smem_state = sizeof(StateSmem) + 1024;
+    const size_t smem_dstate = sizeof(DStateSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_dstate_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dstate)) != cudaSuccess) return e;
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gdn_dstate_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_dstate, s>>>(dm, g, ws, dS_final, dS_chunks, dS0);
     return cudaGetLastError();
 }
 

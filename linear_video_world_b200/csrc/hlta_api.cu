@@ -407,7 +407,11 @@ hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, cons
     const size_t need = hlta_gdn_bwd_workspace_bytes(B, H, L, d, chunk);
     if (workspace_bytes < need)
         return fail(HLTA_ERR_INVALID_ARG, "workspace too small (%zu < %zu bytes)", workspace_bytes, need);
+    DeviceCtx *ctx;
+    hlta_status st;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
     GdnBwdArgs g;
+    g.err = ctx->err;
     g.q = q; g.k = k; g.v = v; g.dO = dO; g.a = a; g.b = b; g.S0 = S0; g.dS_final = dS_final;
     g.dq = dq; g.dk = dk; g.dv = dv; g.da = da; g.db = db; g.dS0 = dS0;
     g.ws = workspace; g.B = B; g.H = H; g.d = d; g.L = L; g.bf16 = dt == HLTA_BF16;

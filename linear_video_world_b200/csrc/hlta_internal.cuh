@@ -53,6 +53,10 @@ struct GdnArgs {
     void *ws;
     size_t ws_bytes;
     unsigned int *err;
+    // optional (bf16 state pass): each chunk's start state, [d][d] fp32 at
+    // S_chunks + (bh * nchunks + c) * S_chunk_stride; with o null the outputs are skipped
+    float *S_chunks;
+    long S_chunk_stride;
 };
 
 // Chunk workspace (per GDN head, per chunk of C tokens; elements of type E):
@@ -116,8 +120,16 @@ struct GdnBwdArgs {
     int B, H, d;
     long L;
     bool bf16;
+    unsigned int *err;
 };
 size_t gdn_bwd_workspace_bytes(long BH, long L);
+// The two state passes of the bf16 backward on the tensor cores, from the forward's bf16
+// chunk products (g.ws: a bf16 forward workspace; g.o null): the forward pass storing each
+// chunk's start state (g.S_chunks), and the backward pass over the chunks storing each chunk's
+// end-state gradient at dS_chunks + (bh * nchunks + c) * g.S_chunk_stride and the initial
+// state's gradient in dS0 (null to skip); dS_final null for zero.
+cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,
+                                       float *dS_chunks, float *dS0, cudaStream_t s);
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);

@@ -45,6 +45,9 @@ def _rel(got, ref):
     (2, 1, 700, 0.05, "fp32", 1e-4, True),    # slow decay: long memory
     (1, 2, 150, 1.0, "bf16", 2e-2, True),
     (2, 2, 1000, 0.05, "bf16", 2e-2, True),
+    (1, 1, 1, 1.0, "bf16", 2e-2, True),       # one token
+    (1, 1, 64, 1.0, "bf16", 2e-2, False),     # one full chunk, zero S0 and dS_final
+    (1, 1, 2000, 0.05, "bf16", 2e-2, True),   # 32 chunks: the state passes' rings wrap
 ])
 def test_gdn_bwd(h, orc, B, H, L, decay, dtype, tol, states):
     x = _case(B, H, L, decay, dtype, seed=L + 3)
@@ -53,6 +56,7 @@ def test_gdn_bwd(h, orc, B, H, L, decay, dtype, tol, states):
     got = h.gdn_bwd(*(dev(x[n]) for n in ("q", "k", "v", "a", "b", "dO")),
                     S0=None if S0 is None else dev(S0), dS_final=None if dSL is None else dev(dSL))
     torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
     ref = orc.gdn_bwd(x["q"], x["k"], x["v"], x["a"], x["b"], x["dO"],
                       S0=None if S0 is None else S0.double().numpy(),
                       dS_final=None if dSL is None else dSL.double().numpy())
