@@ -647,7 +647,7 @@ size_t gdn_bwd_workspace_bytes(long BH, long L)
     return bwd_f32_bytes(BH, L) + gdn_workspace_bytes(BH, L, D, C, true);
 }
 
-cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStreams *side)
 {
     if (a.d != D) return cudaErrorNotSupported;
     if (a.B * a.H == 0 || a.L == 0) return cudaSuccess;
@@ -662,10 +662,15 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
     p.BH = a.B * a.H;
     p.nch = (int)nch;
     if (!a.bf16) return launch_typed<float>(p, s);
-    // bf16: the state passes on the tensor cores, from the forward's bf16 chunk products
+    // bf16: the state passes on the tensor cores, from the forward's bf16 chunk products.
+    // With side streams they run there (each a serial chain on a few SMs, dispatched first),
+    // beside the chunk preparation on the caller's stream; the gradient kernel needs both.
     cudaError_t e;
-    gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const cudaStream_t sa = side ? side->a : s, sb = side ? side->b : s;
+    if (side) {
+        if ((e = cudaEventRecord(side->fork, s)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(sa, side->fork, 0)) != cudaSuccess) return e;
+    }
     GdnArgs g = {};
     g.q = a.q; g.k = a.k; g.v = a.v; g.a = a.a; g.b = a.b;
     g.o = nullptr;
@@ -676,7 +681,19 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s)
     g.err = a.err;
     g.S_chunks = p.ws + O_S0;
     g.S_chunk_stride = CHUNK_FLOATS;
-    if ((e = launch_gdn_bf16_bwd_states(g, a.dO, a.dS_final, p.ws + O_DSC, a.dS0, s)) != cudaSuccess) return e;
+    const cudaError_t es = launch_gdn_bf16_bwd_states(g, a.dO, a.dS_final, p.ws + O_DSC, a.dS0, sa, sb,
+                                                      side ? side->mid : nullptr);
+    gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
+    e = cudaGetLastError();
+    if (side) {
+        // join whatever was enqueued on the side streams, also after a failed launch
+        cudaEventRecord(side->join_a, sa);
+        cudaEventRecord(side->join_b, sb);
+        cudaStreamWaitEvent(s, side->join_a, 0);
+        cudaStreamWaitEvent(s, side->join_b, 0);
+    }
+    if (es != cudaSuccess) return es;
+    if (e != cudaSuccess) return e;
     gdn_bwd_grad<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
     return cudaGetLastError();
 }

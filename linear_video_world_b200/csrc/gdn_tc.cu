@@ -948,7 +948,8 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
 }
 
 cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,
-                                       float *dS_chunks, float *dS0, cudaStream_t s)
+                                       float *dS_chunks, float *dS0, cudaStream_t s,
+                                       cudaStream_t s2, cudaEvent_t mid)
 {
     if (g.d != D || g.o != nullptr || !g.S_chunks) return cudaErrorNotSupported;
     const long nch = gdn_num_chunks(g.L, C);
@@ -982,9 +983,14 @@ cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const f
     if ((e = cudaFuncSetAttribute(gdn_dstate_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dstate)) != cudaSuccess) return e;
     gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
+    if (s2 != s) {
+        // the two state passes are independent of each other: side by side
+        if ((e = cudaEventRecord(mid, s)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(s2, mid, 0)) != cudaSuccess) return e;
+    }
+    gdn_dstate_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_dstate, s2>>>(dm, g, ws, dS_final, dS_chunks, dS0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_dstate_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_dstate, s>>>(dm, g, ws, dS_final, dS_chunks, dS0);
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
     return cudaGetLastError();
 }
 

@@ -41,7 +41,8 @@ struct DeviceCtx {
     unsigned int *err = nullptr;
     cudaStream_t aux = nullptr;     // GDN branch (highest priority)
     cudaStream_t aux2 = nullptr;    // DSWA branch of the hybrid (default priority)
-    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr;
+    cudaStream_t aux3 = nullptr;    // second serial pass of the GDN backward (highest priority)
+    cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, mid = nullptr;
 };
 constexpr int kMaxDevices = 64;
 DeviceCtx g_ctx[kMaxDevices];
@@ -84,6 +85,10 @@ hlta_status device_ctx(DeviceCtx **out)
         if ((e = cudaStreamCreateWithPriority(&c.aux2, cudaStreamNonBlocking, least)) != cudaSuccess)
             return cuda_fail(e, "cudaStreamCreateWithPriority");
         if ((e = cudaEventCreateWithFlags(&c.join2, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventCreate");
+        if ((e = cudaStreamCreateWithPriority(&c.aux3, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamCreateWithPriority");
+        if ((e = cudaEventCreateWithFlags(&c.mid, cudaEventDisableTiming)) != cudaSuccess)
             return cuda_fail(e, "cudaEventCreate");
         c.ready = true;
     }
@@ -424,7 +429,13 @@ hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, cons
         }
         return HLTA_OK;
     }
-    cudaError_t e = launch_gdn_bwd(g, (cudaStream_t)stream);
+    // the bf16 path's two serial state passes run on the library's high-priority side
+    // streams, beside the chunk preparation (the per-device events are shared: hold them
+    // until the joins are enqueued)
+    std::unique_lock<std::mutex> lk(g_fork_mu, std::defer_lock);
+    SideStreams side = {ctx->aux, ctx->aux3, ctx->fork, ctx->mid, ctx->join, ctx->join2};
+    if (g.bf16) lk.lock();
+    cudaError_t e = launch_gdn_bwd(g, (cudaStream_t)stream, g.bf16 ? &side : nullptr);
     if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "gated delta rule backward: unsupported shape");
     if (e != cudaSuccess) return cuda_fail(e, "gated delta rule backward launch");
     return HLTA_OK;

@@ -123,14 +123,23 @@ struct GdnBwdArgs {
     unsigned int *err;
 };
 size_t gdn_bwd_workspace_bytes(long BH, long L);
+// Two side streams and four events for running the bf16 backward's serial state passes
+// beside its parallel chunk preparation (null: everything on the caller's stream)
+struct SideStreams {
+    cudaStream_t a, b;
+    cudaEvent_t fork, mid, join_a, join_b;
+};
 // The two state passes of the bf16 backward on the tensor cores, from the forward's bf16
 // chunk products (g.ws: a bf16 forward workspace; g.o null): the forward pass storing each
 // chunk's start state (g.S_chunks), and the backward pass over the chunks storing each chunk's
 // end-state gradient at dS_chunks + (bh * nchunks + c) * g.S_chunk_stride and the initial
 // state's gradient in dS0 (null to skip); dS_final null for zero.
+// The forward preparation and state pass run on `s`, the state-gradient pass on `s2` after
+// the preparation (event `mid`, recorded on `s`; unused when s2 == s).
 cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,
-                                       float *dS_chunks, float *dS0, cudaStream_t s);
-cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s);
+                                       float *dS_chunks, float *dS0, cudaStream_t s,
+                                       cudaStream_t s2, cudaEvent_t mid);
+cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStreams *side);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 // f0: the first new frame's index, read from f0_dev when that is set (streaming steps keep
