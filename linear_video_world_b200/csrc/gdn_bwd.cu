@@ -142,102 +142,145 @@ __device__ void bgemm(float *O, int ldo, const float *A, int lda, bool tA, const
 }
 
 // The same product on the tensor cores (mma.sync m16n8k16, fp32 accumulation) with A and B
-// rounded to bf16 as they are staged: the bf16 path's block GEMM. Eight warps, each a 16 x 32
-// piece of the 64 x 64 tile; k-steps of 32 staged as [64 rows][32] bf16 with 80-byte rows
-// (conflict-free ldmatrix). M, N multiples of 64, K of 32; same operand conventions as bgemm.
-__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1)
+// rounded to bf16 as their fragments are formed: the bf16 path's block GEMM. The fp32 operand
+// tiles of every (64 x 64 output tile, 32-wide k-step) stream into shared memory by cp.async
+// through a three-stage ring that runs across output tiles, so the loads of later steps are
+// in flight while a step computes. Eight warps, each a 16 x 32 piece of the output tile.
+// Staged tiles keep the source layout: [64][32] with 40-float rows when k is the contiguous
+// index, [32][64] with 68-float rows otherwise (both conflict-free for the fragment reads).
+// M, N multiples of 64, K of 32; operand pointers and leading dimensions 16-byte aligned;
+// same conventions as bgemm. `smf`: TC_SMEM_FLOATS floats of shared memory, 16-byte aligned.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void cp_async16(float *dst, const float *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src) : "memory");
 }
 
-constexpr int TR = 40;              // staged row stride in bf16 elements (80 bytes)
+constexpr int TC_NSTG = 3;                  // stages of the operand ring
+constexpr int TC_SK = 40;                   // row stride of [64][32] tiles (floats)
+constexpr int TC_SN = 68;                   // row stride of [32][64] tiles
+constexpr int TC_TILE = 64 * TC_SK;         // floats reserved per operand tile (>= 32 * TC_SN)
+constexpr int TC_SMEM_FLOATS = TC_NSTG * 2 * TC_TILE;
+static_assert(32 * TC_SN <= TC_TILE, "a [32][64] tile must fit the reservation");
 
 __device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
                          bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *smf)
 {
-    __nv_bfloat16 *As = reinterpret_cast<__nv_bfloat16 *>(smf), *Bs = As + 64 * TR;  // [m][k], [n][k]
-    const uint32_t sA = (uint32_t)__cvta_generic_to_shared(As), sB = (uint32_t)__cvta_generic_to_shared(Bs);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wm = warp & 3, wn = warp >> 2, g = lane >> 2, t = lane & 3;
-    constexpr int PER = 32 * 64 / THREADS;
-    auto ld_a = [&](int m0, int k0, int e) -> float {
-        int kk, mm;
-        if (tA) { kk = e >> 6; mm = e & 63; return A[(long)(k0 + kk) * lda + m0 + mm]; }
-        kk = e & 31; mm = e >> 5;
-        return A[(long)(m0 + mm) * lda + k0 + kk];
-    };
-    auto ld_b = [&](int n0, int k0, int e) -> float {
-        int kb, nb;
-        if (tB) { kb = e & 31; nb = e >> 5; return B[(long)(n0 + nb) * ldb + k0 + kb]; }
-        kb = e >> 6; nb = e & 63;
-        return B[(long)(k0 + kb) * ldb + n0 + nb];
-    };
-    for (int m0 = 0; m0 < M; m0 += 64)
-        for (int n0 = 0; n0 < N; n0 += 64) {
-            float acc[4][4] = {};
-            float ra[PER], rb[PER];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wm = warp & 3, wn = warp >> 2, g = lane >> 2, tg = lane & 3;
+    const int nk = K / 32, ntn = N / 64, steps = (M / 64) * ntn * nk;
+    // step st: output tile st / nk, k-step st % nk, into stage st % TC_NSTG (16-byte copies,
+    // two per thread and operand)
+    auto issue = [&](int st) {
+        if (st < steps) {
+            const int tile = st / nk, k0 = (st % nk) * 32;
+            const int m0 = (tile / ntn) * 64, n0 = (tile % ntn) * 64;
+            float *sa = smf + (st % TC_NSTG) * 2 * TC_TILE, *sb = sa + TC_TILE;
 #pragma unroll
-            for (int r = 0; r < PER; ++r) {
-                ra[r] = ld_a(m0, 0, threadIdx.x + r * THREADS);
-                rb[r] = ld_b(n0, 0, threadIdx.x + r * THREADS);
+            for (int r = 0; r < 2; ++r) {
+                const int e = tid + r * THREADS;
+                if (!tA) cp_async16(sa + (e >> 3) * TC_SK + (e & 7) * 4, A + (long)(m0 + (e >> 3)) * lda + k0 + (e & 7) * 4);
+                else     cp_async16(sa + (e >> 4) * TC_SN + (e & 15) * 4, A + (long)(k0 + (e >> 4)) * lda + m0 + (e & 15) * 4);
+                if (tB)  cp_async16(sb + (e >> 3) * TC_SK + (e & 7) * 4, B + (long)(n0 + (e >> 3)) * ldb + k0 + (e & 7) * 4);
+                else     cp_async16(sb + (e >> 4) * TC_SN + (e & 15) * 4, B + (long)(k0 + (e >> 4)) * ldb + n0 + (e & 15) * 4);
             }
-            for (int k0 = 0; k0 < K; k0 += 32) {
-                __syncthreads();
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");   // empty groups past the end keep the count uniform
+    };
+    __syncthreads();                                // the caller's operand stores are visible
 #pragma unroll
-                for (int r = 0; r < PER; ++r) {
-                    const int e = threadIdx.x + r * THREADS;
-                    int kk, mm, kb, nb;
-                    if (tA) { kk = e >> 6; mm = e & 63; } else { kk = e & 31; mm = e >> 5; }
-                    if (tB) { kb = e & 31; nb = e >> 5; } else { kb = e >> 6; nb = e & 63; }
-                    As[mm * TR + kk] = __float2bfloat16(ra[r]);
-                    Bs[nb * TR + kb] = __float2bfloat16((s ? s[k0 + kb] : 1.f) * rb[r]);
-                }
-                __syncthreads();
-                if (k0 + 32 < K) {
+    for (int st = 0; st < TC_NSTG - 1; ++st) issue(st);
+    float acc[4][4] = {};
+    for (int st = 0; st < steps; ++st) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(TC_NSTG - 2) : "memory");
+        __syncthreads();                            // step st landed for all; stage st - 1 is free
+        issue(st + TC_NSTG - 1);
+        const float *sa = smf + (st % TC_NSTG) * 2 * TC_TILE, *sb = sa + TC_TILE;
+        const int k0 = (st % nk) * 32;
 #pragma unroll
-                    for (int r = 0; r < PER; ++r) {
-                        ra[r] = ld_a(m0, k0 + 32, threadIdx.x + r * THREADS);
-                        rb[r] = ld_b(n0, k0 + 32, threadIdx.x + r * THREADS);
-                    }
-                }
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                    uint32_t a0, a1, a2, a3;
-                    ldsm4(sA + 2u * (uint32_t)((16 * wm + (lane & 15)) * TR + ks * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
-                    const int mid = lane >> 3;
-#pragma unroll
-                    for (int np = 0; np < 2; ++np) {
-                        uint32_t b0, b1, b2, b3;
-                        const int nrow = 32 * wn + 16 * np + 8 * (mid >> 1) + (lane & 7);
-                        ldsm4(sB + 2u * (uint32_t)(nrow * TR + ks * 16 + 8 * (mid & 1)), b0, b1, b2, b3);
-                        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-                        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-                    }
-                }
+        for (int ks = 0; ks < 2; ++ks) {
+            const int kb = ks * 16 + 2 * tg;        // this lane's k pairs: kb, kb + 1 and kb + 8, kb + 9
+            const int r0 = 16 * wm + g;
+            uint32_t a[4];
+            if (!tA) {
+                const float2 x0 = *reinterpret_cast<const float2 *>(sa + r0 * TC_SK + kb);
+                const float2 x1 = *reinterpret_cast<const float2 *>(sa + (r0 + 8) * TC_SK + kb);
+                const float2 x2 = *reinterpret_cast<const float2 *>(sa + r0 * TC_SK + kb + 8);
+                const float2 x3 = *reinterpret_cast<const float2 *>(sa + (r0 + 8) * TC_SK + kb + 8);
+                a[0] = pack_bf16x2(x0.x, x0.y);
+                a[1] = pack_bf16x2(x1.x, x1.y);
+                a[2] = pack_bf16x2(x2.x, x2.y);
+                a[3] = pack_bf16x2(x3.x, x3.y);
+            } else {
+                a[0] = pack_bf16x2(sa[kb * TC_SN + r0], sa[(kb + 1) * TC_SN + r0]);
+                a[1] = pack_bf16x2(sa[kb * TC_SN + r0 + 8], sa[(kb + 1) * TC_SN + r0 + 8]);
+                a[2] = pack_bf16x2(sa[(kb + 8) * TC_SN + r0], sa[(kb + 9) * TC_SN + r0]);
+                a[3] = pack_bf16x2(sa[(kb + 8) * TC_SN + r0 + 8], sa[(kb + 9) * TC_SN + r0 + 8]);
             }
+            float s0 = 1.f, s1 = 1.f, s8 = 1.f, s9 = 1.f;
+            if (s) {
+                s0 = s[k0 + kb];
+                s1 = s[k0 + kb + 1];
+                s8 = s[k0 + kb + 8];
+                s9 = s[k0 + kb + 9];
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int cn = 32 * wn + 8 * nt + g;
+                float b0, b1, b8, b9;
+                if (tB) {
+                    const float2 y0 = *reinterpret_cast<const float2 *>(sb + cn * TC_SK + kb);
+                    const float2 y1 = *reinterpret_cast<const float2 *>(sb + cn * TC_SK + kb + 8);
+                    b0 = y0.x; b1 = y0.y; b8 = y1.x; b9 = y1.y;
+                } else {
+                    b0 = sb[kb * TC_SN + cn];
+                    b1 = sb[(kb + 1) * TC_SN + cn];
+                    b8 = sb[(kb + 8) * TC_SN + cn];
+                    b9 = sb[(kb + 9) * TC_SN + cn];
+                }
+                mma_bf16_16816(acc[nt], a, pack_bf16x2(b0 * s0, b1 * s1), pack_bf16x2(b8 * s8, b9 * s9));
+            }
+        }
+        if (st % nk == nk - 1) {                    // the output tile's last k-step
+            const int tile = st / nk;
+            const int m0 = (tile / ntn) * 64, n0 = (tile % ntn) * 64;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float *o = O + (long)(m0 + 16 * wm + g + 8 * (e >> 1)) * ldo + n0 + 32 * wn + 8 * nt + 2 * t + (e & 1);
-                    *o = alpha * acc[nt][e] + (beta != 0.f ? beta * *o : 0.f);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float2 *o = reinterpret_cast<float2 *>(O + (long)(m0 + 16 * wm + g + 8 * hh) * ldo + n0 + 32 * wn + 8 * nt + 2 * tg);
+                    float2 v = make_float2(alpha * acc[nt][2 * hh], alpha * acc[nt][2 * hh + 1]);
+                    if (beta != 0.f) {
+                        const float2 old = *o;
+                        v.x = fmaf(beta, old.x, v.x);
+                        v.y = fmaf(beta, old.y, v.y);
+                    }
+                    *o = v;
+                    acc[nt][2 * hh] = acc[nt][2 * hh + 1] = 0.f;
                 }
         }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 }
 
-// the element type's block GEMM: tensor cores for bf16 tensors, fp32 CUDA cores for fp32
+template <typename E>
+constexpr int gemm_smem_bytes() { return (int)sizeof(float) * (sizeof(E) == 2 ? TC_SMEM_FLOATS : 2 * 32 * TS); }
+static_assert(C * (C + 1) <= 2 * 32 * TS, "the prep kernel's A^T scratch aliases the GEMM staging");
+
 template <typename E>
 __device__ __forceinline__ void gemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
                                      bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *sm)
@@ -251,7 +294,7 @@ __device__ __forceinline__ void gemm(float *O, int ldo, const float *A, int lda,
 template <typename E>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
 {
-    __shared__ __align__(16) float sm[2 * 32 * TS];
+    extern __shared__ __align__(16) float sm[];        // the block GEMM's staging (gemm_smem_bytes)
     __shared__ float Tt[C][C + 1];
     float (*At)[C + 1] = reinterpret_cast<float (*)[C + 1]>(sm);   // between GEMMs only
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
@@ -500,7 +543,7 @@ __global__ void __launch_bounds__(THREADS) gdn_bwd_bwdstate(BwdP p)
 template <typename E>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
 {
-    __shared__ __align__(16) float sm[2 * 32 * TS];
+    extern __shared__ __align__(16) float sm[];        // the block GEMM's staging (gemm_smem_bytes)
     __shared__ float red[THREADS / 32];
     __shared__ float rowv[6][C];
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
@@ -618,6 +661,14 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
 }
 
 template <typename E>
+cudaError_t set_gemm_smem()
+{
+    cudaError_t e = cudaFuncSetAttribute(gdn_bwd_prep<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<E>());
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gdn_bwd_grad<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes<E>());
+}
+
+template <typename E>
 cudaError_t launch_typed(const BwdP &p, cudaStream_t s)
 {
     const dim3 gc((unsigned)p.nch, (unsigned)p.BH), gs((unsigned)(D / R), (unsigned)p.BH);
@@ -626,10 +677,11 @@ cudaError_t launch_typed(const BwdP &p, cudaStream_t s)
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(gdn_bwd_fwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_f)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_bwd_bwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_b)) != cudaSuccess) return e;
-    gdn_bwd_prep<E><<<gc, THREADS, 0, s>>>(p);
+    if ((e = set_gemm_smem<E>()) != cudaSuccess) return e;
+    gdn_bwd_prep<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p);
     gdn_bwd_fwdstate<<<gs, THREADS, sm_f, s>>>(p);
     gdn_bwd_bwdstate<<<gs, THREADS, sm_b, s>>>(p);
-    gdn_bwd_grad<E><<<gc, THREADS, 0, s>>>(p);
+    gdn_bwd_grad<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p);
     return cudaGetLastError();
 }
 
@@ -683,8 +735,12 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStream
     g.S_chunk_stride = CHUNK_FLOATS;
     const cudaError_t es = launch_gdn_bf16_bwd_states(g, a.dO, a.dS_final, p.ws + O_DSC, a.dS0, sa, sb,
                                                       side ? side->mid : nullptr);
-    gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
-    e = cudaGetLastError();
+    e = set_gemm_smem<__nv_bfloat16>();
+    if (e == cudaSuccess) {
+        gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS,
+                                      gemm_smem_bytes<__nv_bfloat16>(), s>>>(p);
+        e = cudaGetLastError();
+    }
     if (side) {
         // join whatever was enqueued on the side streams, also after a failed launch
         cudaEventRecord(side->join_a, sa);
@@ -694,7 +750,8 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStream
     }
     if (es != cudaSuccess) return es;
     if (e != cudaSuccess) return e;
-    gdn_bwd_grad<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS, 0, s>>>(p);
+    gdn_bwd_grad<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS,
+                                  gemm_smem_bytes<__nv_bfloat16>(), s>>>(p);
     return cudaGetLastError();
 }
 
