@@ -546,6 +546,7 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     extern __shared__ __align__(16) float sm[];        // the block GEMM's staging (gemm_smem_bytes)
     __shared__ float red[THREADS / 32];
     __shared__ float rowv[6][C];
+    __shared__ float colp[THREADS / C][C], cola[THREADS / C][C];
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
     const float *g = w + O_VEC, *bb = g + C, *aa = bb + C;
@@ -570,66 +571,107 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     gemm<E>(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // U dS_C
     gemm<E>(w + O_KS, D, w + O_K, D, false, S0, D, true, nullptr, C, D, D, 1.f, 0.f, sm);      // K S0^T
     gemm<E>(w + O_KD, D, w + O_K, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);     // K dS_C^T
-    // per-row sums over the C x C products (threads 0..63 rows, 64..127 columns) and the
-    // C x d ones (threads 128..191)
-    if (tid < C) {
-        const int t = tid;
+    // per-row sums over the C x C products and the C x d ones: warp w takes rows 8w .. 8w + 7,
+    // its lanes the columns (coalesced), combined by butterfly shuffles
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int rr = 0; rr < C / 8; ++rr) {
+        const int t = warp * (C / 8) + rr;
+        const bool ok = t < n;
         float pp = 0.f, ap = 0.f, db1 = 0.f;
-        for (int s = 0; s < C; ++s) {
-            const bool inc = s <= t && t < n, low = s < t && t < n;
+        for (int s = lane; s < C; s += 32) {
+            const bool inc = s <= t && ok, low = s < t && ok;
             const float dpv = inc ? w[O_DP + t * C + s] : 0.f;
             const float dav = low ? -w[O_DA + t * C + s] : 0.f;
             pp += dpv * w[O_P + t * C + s];
             ap += dav * w[O_A + t * C + s];
             db1 += low ? dav * expf(g[t] - g[s]) * w[O_KK + t * C + s] : 0.f;
         }
-        rowv[0][t] = pp;
-        rowv[1][t] = ap;
-        rowv[2][t] = db1;
-    } else if (tid < 2 * C) {
-        const int s = tid - C;
-        float pp = 0.f, ap = 0.f;
-        for (int t = s; t < n; ++t) {
-            pp += w[O_DP + t * C + s] * w[O_P + t * C + s];
-            if (t > s) ap += -w[O_DA + t * C + s] * w[O_A + t * C + s];
-        }
-        rowv[3][s] = pp;
-        rowv[4][s] = ap;
-    } else if (tid < 3 * C) {
-        const int t = tid - 2 * C;
         const float eg = expf(g[t]);
         float qds = 0.f, drk = 0.f, ukd = 0.f, drv = 0.f;
-        for (int j = 0; j < D; ++j) {
+        for (int j = lane; j < D; j += 32) {
             const float ks = w[O_KS + t * D + j], dr = w[O_DR + t * D + j];
             qds = fmaf(w[O_Q + t * D + j], w[O_DS + t * D + j], qds);
             drk = fmaf(dr, ks, drk);
             ukd = fmaf(w[O_U + t * D + j], w[O_KD + t * D + j], ukd);
             drv = fmaf(dr, w[O_V + t * D + j] - eg * ks, drv);
         }
-        const bool ok = t < n;
-        dg[t] = ok ? eg * qds - bb[t] * eg * drk - expf(gC - g[t]) * ukd : 0.f;
-        rowv[5][t] = ok ? expf(gC - g[t]) * ukd : 0.f;      // for the last token's term
-        w[O_DU + t] = drv;                                   // (dU is free now) db part 2
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            pp += __shfl_xor_sync(0xffffffffu, pp, o);
+            ap += __shfl_xor_sync(0xffffffffu, ap, o);
+            db1 += __shfl_xor_sync(0xffffffffu, db1, o);
+            qds += __shfl_xor_sync(0xffffffffu, qds, o);
+            drk += __shfl_xor_sync(0xffffffffu, drk, o);
+            ukd += __shfl_xor_sync(0xffffffffu, ukd, o);
+            drv += __shfl_xor_sync(0xffffffffu, drv, o);
+        }
+        if (lane == 0) {
+            rowv[0][t] = pp;
+            rowv[1][t] = ap;
+            rowv[2][t] = db1;
+            dg[t] = ok ? eg * qds - bb[t] * eg * drk - expf(gC - g[t]) * ukd : 0.f;
+            rowv[5][t] = ok ? expf(gC - g[t]) * ukd : 0.f;  // for the last token's term
+            w[O_DU + t] = drv;                               // (dU is free now) db part 2
+        }
+    }
+    // column sums of the same C x C products: column s = tid % C, rows t = tid / C + 4i
+    {
+        const int sc = tid & (C - 1), q4 = tid >> 6;
+        float pp = 0.f, ap = 0.f;
+        for (int t = q4; t < n; t += THREADS / C) {
+            if (t < sc) continue;
+            pp += w[O_DP + t * C + sc] * w[O_P + t * C + sc];
+            if (t > sc) ap += -w[O_DA + t * C + sc] * w[O_A + t * C + sc];
+        }
+        colp[q4][sc] = pp;
+        cola[q4][sc] = ap;
     }
     // <dS_C, S0>
     float sd = 0.f;
     for (int e = tid; e < DD; e += THREADS) sd = fmaf(dSC[e], S0[e], sd);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
-    if ((tid & 31) == 0) red[tid >> 5] = sd;
+    if (lane == 0) red[warp] = sd;
     __syncthreads();
-    if (tid == 0) {
-        float tot = 0.f, su = 0.f;
+    if (warp == 0) {
+        // d(log a)_t = sum over t' >= t (t' < n) of v_t': a reverse running sum, two tokens a lane
+        float tot = 0.f;
+#pragma unroll
         for (int i = 0; i < THREADS / 32; ++i) tot += red[i];
-        for (int s = 0; s < n; ++s) su += rowv[5][s];
-        float run = 0.f;
-        for (int t = n - 1; t >= 0; --t) {
-            float v = dg[t] + rowv[0][t] - rowv[3][t] + rowv[1][t] - rowv[4][t];
-            if (t == n - 1) v += gam * tot + su;
-            run += v;
-            const long gi = (long)bh * p.L + (long)c * C + t;
-            p.da[gi] = run / aa[t];
-            p.db[gi] = rowv[2][t] + w[O_DU + t];
+        float su = (lane < n ? rowv[5][lane] : 0.f) + (lane + 32 < n ? rowv[5][lane + 32] : 0.f);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) su += __shfl_xor_sync(0xffffffffu, su, o);
+        float v[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int t = lane + 32 * hh;
+            float cs = 0.f, ca = 0.f;
+#pragma unroll
+            for (int i = 0; i < THREADS / C; ++i) {
+                cs += colp[i][t];
+                ca += cola[i][t];
+            }
+            float x = dg[t] + rowv[0][t] - cs + rowv[1][t] - ca;
+            if (t == n - 1) x += gam * tot + su;
+            v[hh] = t < n ? x : 0.f;
+        }
+        // suffix sums: the upper half within itself, the lower half plus the upper total
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, v[hh], o);
+                if (lane + o < 32) v[hh] += y;
+            }
+        v[0] += __shfl_sync(0xffffffffu, v[1], 0);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int t = lane + 32 * hh;
+            if (t < n) {
+                const long gi = (long)bh * p.L + (long)c * C + t;
+                p.da[gi] = v[hh] / aa[t];
+                p.db[gi] = rowv[2][t] + w[O_DU + t];
+            }
         }
     }
     // M = dA o b_t e^{g_t - g_s} (s < t) into O_DA;  dP o Gam into O_DP
