@@ -37,6 +37,7 @@ constexpr int CD = C * D, CC = C * C, DD = D * D;
 constexpr int DS = D + 4;           // staged row stride: 16-byte rows, no bank conflicts
 constexpr int CDS = C * DS;
 constexpr int TS = 68;              // row stride of the block GEMM's staged tiles
+constexpr int AP = C + 4;           // row stride of the prep's A scratch (16-byte rows)
 
 // per chunk-head scratch (floats)
 enum : long {
@@ -279,7 +280,7 @@ __device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, co
 
 template <typename E>
 constexpr int gemm_smem_bytes() { return (int)sizeof(float) * (sizeof(E) == 2 ? TC_SMEM_FLOATS : 2 * 32 * TS); }
-static_assert(C * (C + 1) <= 2 * 32 * TS, "the prep kernel's A^T scratch aliases the GEMM staging");
+static_assert(C * AP <= 2 * 32 * TS, "the prep kernel's A scratch aliases the GEMM staging");
 
 template <typename E>
 __device__ __forceinline__ void gemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
@@ -295,8 +296,7 @@ template <typename E>
 __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
 {
     extern __shared__ __align__(16) float sm[];        // the block GEMM's staging (gemm_smem_bytes)
-    __shared__ float Tt[C][C + 1];
-    float (*At)[C + 1] = reinterpret_cast<float (*)[C + 1]>(sm);   // between GEMMs only
+    float *At = sm;                                     // [C][AP] between GEMMs only
     const int c = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
     float *w = p.ws + ((long)bh * p.nch + c) * CHUNK_FLOATS;
     const long t0 = (long)c * C;
@@ -311,18 +311,32 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
         w[O_V + e] = ok ? ldf((const E *)p.v, base + e) : 0.f;
         w[O_G + e] = ok ? ldf((const E *)p.dO, base + e) : 0.f;
     }
-    if (tid == 0) {
-        float acc = 0.f;
-        for (int t = 0; t < C; ++t) {
-            const bool ok = t < n;
-            if (ok) acc += logf(p.a[(long)bh * p.L + t0 + t]);
-            g[t] = acc;
-            bb[t] = ok ? p.b[(long)bh * p.L + t0 + t] : 0.f;
-            aa[t] = ok ? p.a[(long)bh * p.L + t0 + t] : 1.f;
-            bg[t] = bb[t] * expf(acc);
+    if (tid < 32) {
+        // g_t = running sum of log a over the chunk (tokens past n add nothing): two tokens a
+        // lane, then a warp scan
+        const int lane = tid, t = 2 * lane;
+        const long gi = (long)bh * p.L + t0 + t;
+        const float a0 = t < n ? p.a[gi] : 1.f, a1 = t + 1 < n ? p.a[gi + 1] : 1.f;
+        const float l0 = t < n ? logf(a0) : 0.f, l1 = t + 1 < n ? logf(a1) : 0.f;
+        const float pair = l0 + l1;
+        float x = pair;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
         }
-        w[O_VEC + 5 * C] = expf(g[C - 1]);              // gamma = e^{g of the last token}
-        w[O_VEC + 5 * C + 1] = (float)n;
+        const float gt0 = x - pair + l0, gt1 = x;
+        const float b0 = t < n ? p.b[gi] : 0.f, b1 = t + 1 < n ? p.b[gi + 1] : 0.f;
+        g[t] = gt0;
+        g[t + 1] = gt1;
+        bb[t] = b0;
+        bb[t + 1] = b1;
+        aa[t] = a0;
+        aa[t + 1] = a1;
+        bg[t] = b0 * expf(gt0);
+        bg[t + 1] = b1 * expf(gt1);
+        if (lane == 31) w[O_VEC + 5 * C] = expf(gt1);   // gamma = e^{g of the last token}
+        if (lane == 0) w[O_VEC + 5 * C + 1] = (float)n;
     }
     __syncthreads();
     gemm<E>(w + O_KK, C, w + O_K, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
@@ -333,21 +347,35 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
         const float dec = inc ? expf(g[t] - g[s]) : 0.f;
         const float av = s < t ? bb[t] * dec * w[O_KK + e] : 0.f;
         w[O_A + e] = av;
-        At[t][s] = av;
+        At[t * AP + s] = av;
         w[O_P + e] = dec * w[O_P + e];
     }
     __syncthreads();
-    if (tid < C) {                                      // T = (I + A)^{-1}, column tid
+    if (tid < C) {
+        // T = (I + A)^{-1} by forward substitution, column j = tid in registers:
+        // T_tj = -sum_{i<t} A_ti T_ij (0 above the diagonal, 1 on it); rows of A read as
+        // float4 broadcasts into four partial sums
         const int j = tid;
-        for (int t = 0; t < C; ++t) Tt[t][j] = t == j ? 1.f : 0.f;
-        for (int t = j + 1; t < C; ++t) {
-            float s = 0.f;
-            for (int i = j; i < t; ++i) s = fmaf(At[t][i], Tt[i][j], s);
-            Tt[t][j] = -s;
+        float tc[C];
+#pragma unroll
+        for (int t = 0; t < C; ++t) {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+            const float4 *ar = reinterpret_cast<const float4 *>(At + t * AP);
+#pragma unroll
+            for (int i4 = 0; i4 < t / 4; ++i4) {
+                const float4 av = ar[i4];
+                a0 = fmaf(av.x, tc[4 * i4], a0);
+                a1 = fmaf(av.y, tc[4 * i4 + 1], a1);
+                a2 = fmaf(av.z, tc[4 * i4 + 2], a2);
+                a3 = fmaf(av.w, tc[4 * i4 + 3], a3);
+            }
+#pragma unroll
+            for (int i = (t / 4) * 4; i < t; ++i) a0 = fmaf(At[t * AP + i], tc[i], a0);
+            tc[t] = t < j ? 0.f : (t == j ? 1.f : -((a0 + a1) + (a2 + a3)));
         }
+#pragma unroll
+        for (int t = 0; t < C; ++t) w[O_T + t * C + j] = tc[t];
     }
-    __syncthreads();
-    for (int e = tid; e < CC; e += THREADS) w[O_T + e] = Tt[e / C][e % C];
     __syncthreads();
     gemm<E>(w + O_W, D, w + O_T, C, false, w + O_K, D, false, bg, C, D, C, 1.f, 0.f, sm);
     gemm<E>(w + O_UP, D, w + O_T, C, false, w + O_V, D, false, bb, C, D, C, 1.f, 0.f, sm);
