@@ -648,7 +648,8 @@ def main():
             bw["attn_bwd_frac"] = bw["attn_bwd_tflops"] / float(pk.get("bf16_tflops"))
         bw["note"] = ("training pass: hlta_window_fwd_lse + hlta_window_bwd for the SWA and DSWA "
                       "heads (tcgen05 dK/dV and dQ kernels), hlta_gdn_chunk_bwd for the GDN heads "
-                      "(fp32 arithmetic, chunk-start states recomputed); frac against the burst "
+                      "(state passes on the tensor cores beside the chunk preparation, chunk "
+                      "gradients through the pipelined block GEMM); frac against the burst "
                       "bf16 peak")
         detail["backward"] = bw
     if fp8_ms is not None:

@@ -166,8 +166,9 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
                             int B, int H, int T, int N, int d, int w, int r, float scale,
                             void *workspace, size_t workspace_bytes, void *stream);
 
-/* Workspace bytes of hlta_gdn_chunk_bwd (chunk = 64, d = 128): about 0.8 MB per 64-token
- * chunk of every (batch, head); 0 for unsupported arguments. */
+/* Workspace bytes of hlta_gdn_chunk_bwd (chunk = 64, d = 128): about 0.9 MB per 64-token
+ * chunk of every (batch, head) (fp32 chunk intermediates plus the forward's bf16 chunk
+ * products); 0 for unsupported arguments. */
 size_t hlta_gdn_bwd_workspace_bytes(int B, int H, long L, int d, int chunk);
 
 /*
@@ -177,11 +178,16 @@ size_t hlta_gdn_bwd_workspace_bytes(int B, int H, long L, int d, int chunk);
  * the chunk start states recomputed from S0 (NULL for zero): a forward pass over the chunks
  * storing each start state, a backward pass over the chunks carrying the state gradient
  * (dS_start = dS_end (gamma I - Kt^T W) + dO^T Qt with the forward's chunk products), and the
- * gradients of every chunk in parallel; fp32 arithmetic throughout.
+ * gradients of every chunk in parallel. fp32 tensors: fp32 arithmetic throughout. bf16
+ * tensors: the two passes over the chunks run on the tensor cores from the forward's bf16 chunk
+ * products (state and state gradient carried in fp32), side by side on the library's
+ * high-priority streams (joined back into `stream` before the gradient launch), and the chunk
+ * products take bf16-rounded operands with fp32 accumulation.
  * q, k, v, dO, dq, dk, dv: [B, H, L, d] device, element type `dt` (d = 128); a, b, da, db:
  * [B, H, L] float32 (a > 0); S0, dS_final, dS0: [B, H, d, d] float32 (dS0 NULL to skip).
  * workspace: device scratch of at least hlta_gdn_bwd_workspace_bytes(...), caller-owned, 16-byte
- * aligned. Enqueued on `stream` (four launches). Errors as hlta_gdn_chunk_fwd.
+ * aligned. Enqueued on `stream` (four launches for fp32, five for bf16). Errors as
+ * hlta_gdn_chunk_fwd.
  */
 hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, const float *a,
                                const float *b, const float *S0, const void *dO,
