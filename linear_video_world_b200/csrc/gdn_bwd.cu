@@ -174,29 +174,38 @@ constexpr int TC_NSTG = 3;                  // stages of the operand ring
 constexpr int TC_SK = 40;                   // row stride of [64][32] tiles (floats)
 constexpr int TC_SN = 68;                   // row stride of [32][64] tiles
 constexpr int TC_TILE = 64 * TC_SK;         // floats reserved per operand tile (>= 32 * TC_SN)
-constexpr int TC_SMEM_FLOATS = TC_NSTG * 2 * TC_TILE;
+constexpr int TC_MAXA = 2;                  // products sharing one B operand per pass
+constexpr int TC_SMEM_FLOATS = TC_NSTG * (TC_MAXA + 1) * TC_TILE;
 static_assert(32 * TC_SN <= TC_TILE, "a [32][64] tile must fit the reservation");
 
-__device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
-                         bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *smf)
+// NA products O_a = alpha_a A_a opB + beta_a O_a (a < NA) sharing B, tA, lda, ldo and the shape:
+// each B tile is staged once for all of them
+template <int NA>
+__device__ void bgemm_tc_n(float *const (&O)[NA], int ldo, const float *const (&A)[NA], int lda, bool tA,
+                           const float *B, int ldb, bool tB, const float *s, int M, int N, int K,
+                           const float (&alpha)[NA], const float (&beta)[NA], float *smf)
 {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wm = warp & 3, wn = warp >> 2, g = lane >> 2, tg = lane & 3;
     const int nk = K / 32, ntn = N / 64, steps = (M / 64) * ntn * nk;
+    constexpr int STAGE = (NA + 1) * TC_TILE;
     // step st: output tile st / nk, k-step st % nk, into stage st % TC_NSTG (16-byte copies,
-    // two per thread and operand)
+    // two per thread and operand tile)
     auto issue = [&](int st) {
         if (st < steps) {
             const int tile = st / nk, k0 = (st % nk) * 32;
             const int m0 = (tile / ntn) * 64, n0 = (tile % ntn) * 64;
-            float *sa = smf + (st % TC_NSTG) * 2 * TC_TILE, *sb = sa + TC_TILE;
+            float *sa = smf + (st % TC_NSTG) * STAGE, *sb = sa + NA * TC_TILE;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int e = tid + r * THREADS;
-                if (!tA) cp_async16(sa + (e >> 3) * TC_SK + (e & 7) * 4, A + (long)(m0 + (e >> 3)) * lda + k0 + (e & 7) * 4);
-                else     cp_async16(sa + (e >> 4) * TC_SN + (e & 15) * 4, A + (long)(k0 + (e >> 4)) * lda + m0 + (e & 15) * 4);
-                if (tB)  cp_async16(sb + (e >> 3) * TC_SK + (e & 7) * 4, B + (long)(n0 + (e >> 3)) * ldb + k0 + (e & 7) * 4);
-                else     cp_async16(sb + (e >> 4) * TC_SN + (e & 15) * 4, B + (long)(k0 + (e >> 4)) * ldb + n0 + (e & 15) * 4);
+#pragma unroll
+                for (int ia = 0; ia < NA; ++ia) {
+                    if (!tA) cp_async16(sa + ia * TC_TILE + (e >> 3) * TC_SK + (e & 7) * 4, A[ia] + (long)(m0 + (e >> 3)) * lda + k0 + (e & 7) * 4);
+                    else     cp_async16(sa + ia * TC_TILE + (e >> 4) * TC_SN + (e & 15) * 4, A[ia] + (long)(k0 + (e >> 4)) * lda + m0 + (e & 15) * 4);
+                }
+                if (tB) cp_async16(sb + (e >> 3) * TC_SK + (e & 7) * 4, B + (long)(n0 + (e >> 3)) * ldb + k0 + (e & 7) * 4);
+                else    cp_async16(sb + (e >> 4) * TC_SN + (e & 15) * 4, B + (long)(k0 + (e >> 4)) * ldb + n0 + (e & 15) * 4);
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");   // empty groups past the end keep the count uniform
@@ -204,32 +213,36 @@ __device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, co
     __syncthreads();                                // the caller's operand stores are visible
 #pragma unroll
     for (int st = 0; st < TC_NSTG - 1; ++st) issue(st);
-    float acc[4][4] = {};
+    float acc[NA][4][4] = {};
     for (int st = 0; st < steps; ++st) {
         asm volatile("cp.async.wait_group %0;" ::"n"(TC_NSTG - 2) : "memory");
         __syncthreads();                            // step st landed for all; stage st - 1 is free
         issue(st + TC_NSTG - 1);
-        const float *sa = smf + (st % TC_NSTG) * 2 * TC_TILE, *sb = sa + TC_TILE;
+        const float *sa = smf + (st % TC_NSTG) * STAGE, *sb = sa + NA * TC_TILE;
         const int k0 = (st % nk) * 32;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
             const int kb = ks * 16 + 2 * tg;        // this lane's k pairs: kb, kb + 1 and kb + 8, kb + 9
             const int r0 = 16 * wm + g;
-            uint32_t a[4];
-            if (!tA) {
-                const float2 x0 = *reinterpret_cast<const float2 *>(sa + r0 * TC_SK + kb);
-                const float2 x1 = *reinterpret_cast<const float2 *>(sa + (r0 + 8) * TC_SK + kb);
-                const float2 x2 = *reinterpret_cast<const float2 *>(sa + r0 * TC_SK + kb + 8);
-                const float2 x3 = *reinterpret_cast<const float2 *>(sa + (r0 + 8) * TC_SK + kb + 8);
-                a[0] = pack_bf16x2(x0.x, x0.y);
-                a[1] = pack_bf16x2(x1.x, x1.y);
-                a[2] = pack_bf16x2(x2.x, x2.y);
-                a[3] = pack_bf16x2(x3.x, x3.y);
-            } else {
-                a[0] = pack_bf16x2(sa[kb * TC_SN + r0], sa[(kb + 1) * TC_SN + r0]);
-                a[1] = pack_bf16x2(sa[kb * TC_SN + r0 + 8], sa[(kb + 1) * TC_SN + r0 + 8]);
-                a[2] = pack_bf16x2(sa[(kb + 8) * TC_SN + r0], sa[(kb + 9) * TC_SN + r0]);
-                a[3] = pack_bf16x2(sa[(kb + 8) * TC_SN + r0 + 8], sa[(kb + 9) * TC_SN + r0 + 8]);
+            uint32_t a[NA][4];
+#pragma unroll
+            for (int ia = 0; ia < NA; ++ia) {
+                const float *t = sa + ia * TC_TILE;
+                if (!tA) {
+                    const float2 x0 = *reinterpret_cast<const float2 *>(t + r0 * TC_SK + kb);
+                    const float2 x1 = *reinterpret_cast<const float2 *>(t + (r0 + 8) * TC_SK + kb);
+                    const float2 x2 = *reinterpret_cast<const float2 *>(t + r0 * TC_SK + kb + 8);
+                    const float2 x3 = *reinterpret_cast<const float2 *>(t + (r0 + 8) * TC_SK + kb + 8);
+                    a[ia][0] = pack_bf16x2(x0.x, x0.y);
+                    a[ia][1] = pack_bf16x2(x1.x, x1.y);
+                    a[ia][2] = pack_bf16x2(x2.x, x2.y);
+                    a[ia][3] = pack_bf16x2(x3.x, x3.y);
+                } else {
+                    a[ia][0] = pack_bf16x2(t[kb * TC_SN + r0], t[(kb + 1) * TC_SN + r0]);
+                    a[ia][1] = pack_bf16x2(t[kb * TC_SN + r0 + 8], t[(kb + 1) * TC_SN + r0 + 8]);
+                    a[ia][2] = pack_bf16x2(t[(kb + 8) * TC_SN + r0], t[(kb + 9) * TC_SN + r0]);
+                    a[ia][3] = pack_bf16x2(t[(kb + 8) * TC_SN + r0 + 8], t[(kb + 9) * TC_SN + r0 + 8]);
+                }
             }
             float s0 = 1.f, s1 = 1.f, s8 = 1.f, s9 = 1.f;
             if (s) {
@@ -252,35 +265,65 @@ __device__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, co
                     b8 = sb[(kb + 8) * TC_SN + cn];
                     b9 = sb[(kb + 9) * TC_SN + cn];
                 }
-                mma_bf16_16816(acc[nt], a, pack_bf16x2(b0 * s0, b1 * s1), pack_bf16x2(b8 * s8, b9 * s9));
+                const uint32_t bp0 = pack_bf16x2(b0 * s0, b1 * s1), bp1 = pack_bf16x2(b8 * s8, b9 * s9);
+#pragma unroll
+                for (int ia = 0; ia < NA; ++ia) mma_bf16_16816(acc[ia][nt], a[ia], bp0, bp1);
             }
         }
         if (st % nk == nk - 1) {                    // the output tile's last k-step
             const int tile = st / nk;
             const int m0 = (tile / ntn) * 64, n0 = (tile % ntn) * 64;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int ia = 0; ia < NA; ++ia)
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float2 *o = reinterpret_cast<float2 *>(O + (long)(m0 + 16 * wm + g + 8 * hh) * ldo + n0 + 32 * wn + 8 * nt + 2 * tg);
-                    float2 v = make_float2(alpha * acc[nt][2 * hh], alpha * acc[nt][2 * hh + 1]);
-                    if (beta != 0.f) {
-                        const float2 old = *o;
-                        v.x = fmaf(beta, old.x, v.x);
-                        v.y = fmaf(beta, old.y, v.y);
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float2 *o = reinterpret_cast<float2 *>(O[ia] + (long)(m0 + 16 * wm + g + 8 * hh) * ldo + n0 + 32 * wn + 8 * nt + 2 * tg);
+                        float2 v = make_float2(alpha[ia] * acc[ia][nt][2 * hh], alpha[ia] * acc[ia][nt][2 * hh + 1]);
+                        if (beta[ia] != 0.f) {
+                            const float2 old = *o;
+                            v.x = fmaf(beta[ia], old.x, v.x);
+                            v.y = fmaf(beta[ia], old.y, v.y);
+                        }
+                        *o = v;
+                        acc[ia][nt][2 * hh] = acc[ia][nt][2 * hh + 1] = 0.f;
                     }
-                    *o = v;
-                    acc[nt][2 * hh] = acc[nt][2 * hh + 1] = 0.f;
-                }
         }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
 }
 
+__device__ __forceinline__ void bgemm_tc(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
+                                         bool tB, const float *s, int M, int N, int K, float alpha, float beta, float *smf)
+{
+    float *const o1[1] = {O};
+    const float *const a1[1] = {A};
+    const float al[1] = {alpha}, be[1] = {beta};
+    bgemm_tc_n<1>(o1, ldo, a1, lda, tA, B, ldb, tB, s, M, N, K, al, be, smf);
+}
+
 template <typename E>
 constexpr int gemm_smem_bytes() { return (int)sizeof(float) * (sizeof(E) == 2 ? TC_SMEM_FLOATS : 2 * 32 * TS); }
 static_assert(C * AP <= 2 * 32 * TS, "the prep kernel's A scratch aliases the GEMM staging");
+
+// two products sharing B (and tA, lda, ldo, the shape): B staged once on the tensor-core path
+template <typename E>
+__device__ __forceinline__ void gemm2(float *O1, float *O2, int ldo, const float *A1, const float *A2, int lda,
+                                      bool tA, const float *B, int ldb, bool tB, int M, int N, int K,
+                                      float alpha1, float beta1, float alpha2, float beta2, float *sm)
+{
+    if constexpr (sizeof(E) == 2) {
+        float *const o[2] = {O1, O2};
+        const float *const a[2] = {A1, A2};
+        const float al[2] = {alpha1, alpha2}, be[2] = {beta1, beta2};
+        bgemm_tc_n<2>(o, ldo, a, lda, tA, B, ldb, tB, nullptr, M, N, K, al, be, sm);
+    } else {
+        bgemm(O1, ldo, A1, lda, tA, B, ldb, tB, nullptr, M, N, K, alpha1, beta1, sm);
+        bgemm(O2, ldo, A2, lda, tA, B, ldb, tB, nullptr, M, N, K, alpha2, beta2, sm);
+    }
+}
 
 template <typename E>
 __device__ __forceinline__ void gemm(float *O, int ldo, const float *A, int lda, bool tA, const float *B, int ldb,
@@ -583,22 +626,18 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     const int n = (int)w[O_VEC + 5 * C + 1];
     const float gC = g[C - 1];
     const float *S0 = w + O_S0, *dSC = w + O_DSC;
-    // U = Up - W S0^T
+    // U = Up - W S0^T and K S0^T
     for (int e = tid; e < CD; e += THREADS) w[O_U + e] = w[O_UP + e];
-    gemm<E>(w + O_U, D, w + O_W, D, false, S0, D, true, nullptr, C, D, D, -1.f, 1.f, sm);
-    // dU = Kt dS_C^T + P^T dO ;  dR = T^T dU
-    gemm<E>(w + O_DU, D, w + O_KT, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);
+    gemm2<E>(w + O_U, w + O_KS, D, w + O_W, w + O_K, D, false, S0, D, true, C, D, D, -1.f, 1.f, 1.f, 0.f, sm);
+    // dU = Kt dS_C^T + P^T dO (and K dS_C^T);  dR = T^T dU
+    gemm2<E>(w + O_DU, w + O_KD, D, w + O_KT, w + O_K, D, false, dSC, D, true, C, D, D, 1.f, 0.f, 1.f, 0.f, sm);
     gemm<E>(w + O_DU, D, w + O_P, C, true, w + O_G, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     gemm<E>(w + O_DR, D, w + O_T, C, true, w + O_DU, D, false, nullptr, C, D, C, 1.f, 0.f, sm);
     // C x C: dP = dO U^T, dA' = dR U^T
-    gemm<E>(w + O_DP, C, w + O_G, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
-    gemm<E>(w + O_DA, C, w + O_DR, D, false, w + O_U, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
-    // products with the d x d states
-    gemm<E>(w + O_DS, D, w + O_G, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);     // dO S0
-    gemm<E>(w + O_RS, D, w + O_DR, D, false, S0, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // dR S0
-    gemm<E>(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);    // U dS_C
-    gemm<E>(w + O_KS, D, w + O_K, D, false, S0, D, true, nullptr, C, D, D, 1.f, 0.f, sm);      // K S0^T
-    gemm<E>(w + O_KD, D, w + O_K, D, false, dSC, D, true, nullptr, C, D, D, 1.f, 0.f, sm);     // K dS_C^T
+    gemm2<E>(w + O_DP, w + O_DA, C, w + O_G, w + O_DR, D, false, w + O_U, D, true, C, C, D, 1.f, 0.f, 1.f, 0.f, sm);
+    // products with the d x d states: dO S0, dR S0, U dS_C
+    gemm2<E>(w + O_DS, w + O_RS, D, w + O_G, w + O_DR, D, false, S0, D, false, C, D, D, 1.f, 0.f, 1.f, 0.f, sm);
+    gemm<E>(w + O_UD, D, w + O_U, D, false, dSC, D, false, nullptr, C, D, D, 1.f, 0.f, sm);
     // per-row sums over the C x C products and the C x d ones: warp w takes rows 8w .. 8w + 7,
     // its lanes the columns (coalesced), combined by butterfly shuffles
     const int warp = tid >> 5, lane = tid & 31;
