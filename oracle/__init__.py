@@ -71,6 +71,8 @@ def _load():
         lib.oracle_gdn_bwd.argtypes = [f32, f32, f32, f32, f32, f64, f32, f64, f64, f64, f64, f64,
                                        f64, f64, L_, L_, I_]
         lib.oracle_gdn_bwd.restype = ctypes.c_int
+        lib.oracle_rope.argtypes = [f32, f64, L_, L_, I_, I_, D_, I_, I_]
+        lib.oracle_rope.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -279,6 +281,20 @@ def window_lse(q, k, T: int, N: int, w: int, r: int = 1, scale=None) -> np.ndarr
     if rc != 0:
         raise RuntimeError(f"oracle window_lse failed ({rc})")
     return out
+
+
+def rope(x, N: int, base: float = 10000.0, pos_mode: int = 0, sign: int = 1) -> np.ndarray:
+    """Rotary embedding of x [..., L, d] (see oracle_rope: position l mod N or l), fp64."""
+    xf = _f32(x)
+    shp = xf.shape
+    L, d = shp[-2], shp[-1]
+    BH = int(np.prod(shp[:-2])) if len(shp) > 2 else 1
+    y = np.empty(shp, dtype=np.float64)
+    rc = _load().oracle_rope(_ptr(xf, ctypes.c_float), _ptr(y, ctypes.c_double), BH, L, N, d,
+                             float(base), int(pos_mode), int(sign))
+    if rc:
+        raise ValueError("oracle_rope: bad arguments")
+    return y
 
 
 def e4m3_decode(code: int) -> float:

@@ -33,8 +33,10 @@
  * Parity status: every function here is pinned by tests that do not re-type its
  * formula (brute-force full attention, closed forms, contraction and retrieval
  * invariants; for the E4M3 codec and quantisers, PyTorch's float8_e4m3fn conversion,
- * the round-to-nearest reconstruction bound and lossless cases); see
- * tests/test_oracle_pins.py and tests/test_oracle_fp8_pins.py.
+ * the round-to-nearest reconstruction bound and lossless cases; for the rotary embedding,
+ * the complex-exponential form, the relative-position (Toeplitz) property, norms and the
+ * inverse); see tests/test_oracle_pins.py, tests/test_oracle_fp8_pins.py and
+ * tests/test_oracle_rope_pins.py.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -643,6 +645,36 @@ int oracle_gdn_bwd(const float *q, const float *k, const float *v, const float *
         free(gk);
     }
     return err;
+}
+
+/*
+ * Rotary position embedding (llm-atlas long-context explainer, the position-encoding section:
+ * RoPE turns a position into a rotation of Q and K so that their dot product depends only on
+ * the relative position). Kairos gives RoPE the local position and the linear path the global
+ * one (the related-papers analysis, row B1). Reading used here: 1-D RoPE, the pair
+ * (x_{2i}, x_{2i+1}) of a token at position p rotated by the angle p * base^(-2i/d);
+ * p = l mod N (the token's index inside its frame) for pos_mode 0, p = l for pos_mode 1;
+ * sign = -1 rotates back (the inverse rotation, which is also the map of the gradient).
+ * x, y: [BH][L][d].
+ */
+int oracle_rope(const float *x, double *y, long BH, long L, int N, int d, double base,
+                int pos_mode, int sign)
+{
+    if (d < 2 || d % 2 || (pos_mode == 0 && N < 1) || !(base > 1.0)) return 1;
+    for (long bh = 0; bh < BH; ++bh)
+        for (long l = 0; l < L; ++l) {
+            const double p = pos_mode ? (double)l : (double)(l % N);
+            const float *xr = x + (bh * L + l) * d;
+            double *yr = y + (bh * L + l) * d;
+            for (int i = 0; i < d / 2; ++i) {
+                const double ang = sign * p * pow(base, -2.0 * i / d);
+                const double c = cos(ang), s = sin(ang);
+                const double x0 = xr[2 * i], x1 = xr[2 * i + 1];
+                yr[2 * i] = x0 * c - x1 * s;
+                yr[2 * i + 1] = x0 * s + x1 * c;
+            }
+        }
+    return 0;
 }
 
 int oracle_num_threads(void)
