@@ -205,9 +205,39 @@ def measure_raw(h, torch, dev, wl, hi, steps: int) -> dict:
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
+    # the softmax heads' prologue: rotary embedding of their q and k in place (within-frame
+    # position), alone and in front of the raw step
+    Hsm = wl.Hs + wl.Hd
+
+    def rope():
+        h.rope(q, k, wl.N, heads=(0, Hsm), pos_mode=0)
+
+    for _ in range(3):
+        rope()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        rope()
+    e1.record()
+    torch.cuda.synchronize()
+    rope_ms = e0.elapsed_time(e1) / steps
+    e0.record()
+    for _ in range(steps):
+        rope()
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_rope = e0.elapsed_time(e1) / steps
+    rope_bytes = 2 * 2 * wl.B * Hsm * wl.L * wl.d * q.element_size()   # q and k, read + write
     return {"ms_per_step": ms, "tokens_per_s": wl.B * wl.L / (ms / 1e3),
             "note": "hlta_hybrid_fwd_raw: the GDN heads' unit-norm q/k and gate activations "
-                    "computed inside the chunk preparation"}
+                    "computed inside the chunk preparation",
+            "with_rope": {"ms_per_step": ms_rope, "tokens_per_s": wl.B * wl.L / (ms_rope / 1e3),
+                          "rope_ms": rope_ms, "rope_bytes": rope_bytes,
+                          "rope_gbs": rope_bytes / (rope_ms / 1e3) / 1e9,
+                          "note": "hlta_rope on the softmax heads' q and k (in place, position "
+                                  "inside the frame), then hlta_hybrid_fwd_raw; rope_gbs against "
+                                  "the HBM peak in hbm_peak_gbs"}}
 
 
 def measure_fp8(h, torch, dev, wl, q, k, v, steps: int) -> dict:

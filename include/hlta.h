@@ -166,6 +166,28 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
                             int B, int H, int T, int N, int d, int w, int r, float scale,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Rotary position embedding of the softmax heads' q and k, in place: the prologue of the SWA /
+ * DSWA branches (llm-atlas long-context explainer, position-encoding section: RoPE turns a
+ * position into a rotation of Q and K, so their dot product depends on the relative position;
+ * Kairos gives RoPE the local position and leaves the global one to the linear path,
+ * related-papers analysis row B1). The pair (x_{2i}, x_{2i+1}) of a token at position p turns
+ * by the angle p * base^(-2i/d), clockwise for inverse != 0 (the inverse rotation, which is
+ * also the map of the gradient, so the backward pass calls the same entry point).
+ * p = l mod N, the token's index inside its frame, for pos_mode 0 (the local position; a
+ * streaming step's frame index does not enter); p = l, the index in the sequence, for
+ * pos_mode 1.
+ * q, k: [B, H, L, d] device, element type `dt`, either may be NULL (skipped); heads
+ * [h0, h0 + Hr) are rotated, the others untouched (so the softmax heads of a hybrid tensor
+ * can be rotated in place). d even, 2 <= d <= 128; base > 1 finite (10000 is the usual
+ * value); N >= 1. The angle is reduced in double precision before a single-precision sine and
+ * cosine; the result is rounded to `dt` once. One launch on `stream`. Errors:
+ * HLTA_ERR_INVALID_ARG for bad shapes, ranges, base, pos_mode or misaligned (16-byte)
+ * pointers.
+ */
+hlta_status hlta_rope(void *q, void *k, int B, int H, int h0, int Hr, long L, int N, int d,
+                      float base, int pos_mode, int inverse, hlta_dtype dt, void *stream);
+
 /* Workspace bytes of hlta_gdn_chunk_bwd (chunk = 64, d = 128): about 0.9 MB per 64-token
  * chunk of every (batch, head) (fp32 chunk intermediates plus the forward's bf16 chunk
  * products); 0 for unsupported arguments. */

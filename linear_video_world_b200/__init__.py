@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
         "hlta_stream_frame_counter": (I, [P, ctypes.POINTER(P)]),
+        "hlta_rope": (I, [P, P, I, I, I, I, L, I, I, F, I, I, I, P]),
         "hlta_fp8_quantize_rows": (I, [P, P, I, I, L, I, L, I, P, P, P]),
         "hlta_fp8_quantize_channels": (I, [P, I, I, L, I, P, P, P]),
         "hlta_window_fp8_fwd": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]),
@@ -252,6 +253,25 @@ def hlta_window_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, T, N, d, w, r, scale,
 
 def hlta_gdn_bwd_workspace_bytes(B, H, L, d=128, chunk=64) -> int:
     return int(_lib.hlta_gdn_bwd_workspace_bytes(B, H, L, d, chunk))
+
+
+def hlta_rope(q, k, B, H, h0, Hr, L, N, d, base=10000.0, pos_mode=0, inverse=False,
+              stream=None):
+    for t, n in ((q, "q"), (k, "k")):
+        if t is not None:
+            _need(t, n)
+    ref = q if q is not None else k
+    _check(_lib.hlta_rope(_p(q), _p(k), B, H, h0, Hr, L, N, d, float(base), int(pos_mode),
+                          1 if inverse else 0, _dt(ref), _stream(stream)))
+
+
+def rope(q, k, N, heads=None, base=10000.0, pos_mode=0, inverse=False, stream=None):
+    """Rotate q and k ([B, H, L, d]) in place; `heads` = (h0, Hr) or None for all heads."""
+    ref = q if q is not None else k
+    B, H, L, d = ref.shape
+    h0, Hr = heads if heads is not None else (0, H)
+    hlta_rope(q, k, B, H, h0, Hr, L, N, d, base, pos_mode, inverse, stream)
+    return q, k
 
 
 def hlta_gdn_chunk_bwd(q, k, v, a, b, S0, dO, dS_final, dq, dk, dv, da, db, dS0, B, H, L, d,

@@ -384,6 +384,24 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
     return HLTA_OK;
 }
 
+hlta_status hlta_rope(void *q, void *k, int B, int H, int h0, int Hr, long L, int N, int d,
+                      float base, int pos_mode, int inverse, hlta_dtype dt, void *stream)
+{
+    if (dt != HLTA_BF16 && dt != HLTA_FP32) return fail(HLTA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (B < 0 || H < 0 || L < 0 || N < 1) return fail(HLTA_ERR_INVALID_ARG, "bad shape B=%d H=%d L=%ld N=%d", B, H, L, N);
+    if (d < 2 || d > 128 || d % 2) return fail(HLTA_ERR_INVALID_ARG, "d must be even, 2 <= d <= 128 (got %d)", d);
+    if (h0 < 0 || Hr < 0 || h0 + Hr > H) return fail(HLTA_ERR_INVALID_ARG, "head range [%d, %d) outside [0, %d)", h0, h0 + Hr, H);
+    if (!(base > 1.f) || !(base < 1e30f)) return fail(HLTA_ERR_INVALID_ARG, "base must be finite and > 1 (got %g)", (double)base);
+    if (pos_mode != 0 && pos_mode != 1) return fail(HLTA_ERR_INVALID_ARG, "pos_mode must be 0 or 1 (got %d)", pos_mode);
+    if ((q && !aligned16(q)) || (k && !aligned16(k)))
+        return fail(HLTA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    cudaError_t e = launch_rope(q, k, dt == HLTA_BF16, B, H, h0, Hr, L, N, d, (double)base, pos_mode,
+                                inverse ? -1 : 1, (cudaStream_t)stream);
+    if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "rotary embedding: shape too large");
+    if (e != cudaSuccess) return cuda_fail(e, "rotary embedding launch");
+    return HLTA_OK;
+}
+
 size_t hlta_gdn_bwd_workspace_bytes(int B, int H, long L, int d, int chunk)
 {
     if (B < 0 || H < 0 || L < 0 || d != 128 || chunk != 64) return 0;

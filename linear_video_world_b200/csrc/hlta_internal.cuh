@@ -150,6 +150,11 @@ cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr
 // *f += F on the device (one thread), in stream order
 cudaError_t launch_frame_advance(int *f, int F, cudaStream_t s);
 
+// Rotary embedding of heads [h0, h0 + Hr) of q and k ([B][Htot][L][d], either may be null),
+// in place; sign -1 for the inverse rotation
+cudaError_t launch_rope(void *q, void *k, bool bf16, int B, int Htot, int h0, int Hr, long L,
+                        int N, int d, double base, int pos_mode, int sign, cudaStream_t s);
+
 // Device error word: kernels OR a code into it when a bounded wait expires.
 enum : unsigned int {
     DEVERR_ATTN_WAIT = 1u << 0,

@@ -170,3 +170,24 @@ def test_gdn_backward_entry_point_validates_on_host(lib):
     assert f(*bad) == h.HLTA_ERR_UNSUPPORTED
     bad = list(args); bad[5] = ctypes.c_void_p(264)
     assert f(*bad) == h.HLTA_ERR_INVALID_ARG
+
+
+def test_rope_entry_point_validates_on_host(lib):
+    import linear_video_world_b200 as h
+    p = ctypes.c_void_p(256)
+    F = ctypes.c_float
+    bad = [
+        (p, p, 1, 4, 0, 4, 100, 10, 127, F(1e4), 0, 0, h.HLTA_BF16),    # odd d
+        (p, p, 1, 4, 0, 4, 100, 10, 130, F(1e4), 0, 0, h.HLTA_BF16),    # d > 128
+        (p, p, 1, 4, 2, 3, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16),    # heads past H
+        (p, p, 1, 4, 0, 4, 100, 10, 128, F(1.0), 0, 0, h.HLTA_BF16),    # base <= 1
+        (p, p, 1, 4, 0, 4, 100, 10, 128, F(1e4), 2, 0, h.HLTA_BF16),    # pos_mode
+        (p, p, 1, 4, 0, 4, 100, 0, 128, F(1e4), 0, 0, h.HLTA_BF16),     # N < 1
+        (ctypes.c_void_p(264), p, 1, 4, 0, 4, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16),
+        (p, p, 1, 4, 0, 4, 100, 10, 128, F(1e4), 0, 0, 7),               # dtype
+    ]
+    for args in bad:
+        assert lib.hlta_rope(*args, None) == h.HLTA_ERR_INVALID_ARG, args
+    # nothing to rotate: accepted without touching a device
+    assert lib.hlta_rope(None, None, 1, 4, 0, 4, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16, None) == h.HLTA_OK
+    assert lib.hlta_rope(p, p, 1, 4, 1, 0, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16, None) == h.HLTA_OK
