@@ -13,8 +13,9 @@
 //
 // Two kernels:
 //   prep   one CTA per (chunk, head), every chunk in parallel: Q, K, V of the chunk arrive
-//          by TMA as 128B-swizzled boxes; KK^T, QK^T, T by forward substitution (fp32, one
-//          column per thread in registers), then W, Up, Op, Qt on mma.sync bf16 tensor cores;
+//          by TMA as 128B-swizzled boxes; KK^T, QK^T, T in 32 x 32 blocks (fp32: forward
+//          substitution of the diagonal blocks, a column per thread, then two block products),
+//          then W, Up, Op, Qt on mma.sync bf16 tensor cores;
 //          writes W, Qt, Kt, and Up, Op transposed (bf16), and gam (fp32) to the workspace.
 //   state  serial over the chunks of a head; the 128 state rows are split into 16-row blocks
 //          (rows of S evolve independently), one warp per block, four per CTA, two CTAs per
@@ -135,10 +136,10 @@ constexpr uint32_t SWT = C * D * 2;        // one swizzled [64][128] bf16 tile: 
 
 // Shared memory of the prep kernel (about 92 KB: two CTAs per SM). Q, K, V arrive by TMA as
 // swizzled tiles; regions are reused once their contents are dead:
-//   R1: A (fp32 [64][68]) -> T1, T2 (bf16 [64][72] each) -> Op (swizzled tile)
+//   R1: A (fp32 [64][68]) -> T (in place) -> T1, T2 (bf16 [64][72] each) -> Op (swizzled tile)
 //   R2: W (swizzled tile)
 //   V:  V -> Up          Q:  Q -> Qt (in place)
-// T = (I + A)^{-1} itself never reaches shared memory: its columns live in registers.
+// T = (I + A)^{-1} is formed over A in place (fp32) before T1, T2 replace both.
 struct PrepSmem {
     alignas(1024) uint8_t Q[SWT];
     alignas(1024) uint8_t K[SWT];
@@ -348,41 +349,75 @@ gdn_prep_bf16(const __grid_constant__ PrepMaps maps, GdnArgs p, GdnWorkspace ws)
     }
     __syncthreads();
 
-    // ---- T = (I + A)^{-1} (A strictly lower triangular, so T is unit lower triangular) by
-    //      forward substitution, one column per thread held in registers:
-    //      T_tj = -sum_{i<t} A_ti T_ij (T_tj = 0 above the diagonal, 1 on it), the row of A
-    //      read as float4 broadcasts and summed in four partial sums. Then T1 = T diag(b e^g)
-    //      and T2 = T diag(b) in bf16, written over A once every column is done.
+    // ---- T = (I + A)^{-1} (A strictly lower triangular, so T is unit lower triangular), in
+    //      two levels of 32 x 32 blocks, written over A in place:
+    //        T00 = (I + A00)^-1, T11 = (I + A11)^-1  forward substitution, a column per thread
+    //                                               (T_tj = -sum_{i<t} A_ti T_ij inside a block)
+    //        T10 = -T11 A10 T00                     two 32 x 32 products, four columns a thread
+    //      (T01 = 0 = A01). Then T1 = T diag(b e^g) and T2 = T diag(b) in bf16 over R1.
     {
-        float tc[C];
         if (tid < C) {
-            const int j = tid;
+            const int base = (tid >> 5) * 32, jj = tid & 31;
+            float tc[32];
 #pragma unroll
-            for (int t = 0; t < C; ++t) {
+            for (int t = 0; t < 32; ++t) {
                 float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                const float4 *ar = reinterpret_cast<const float4 *>(A + t * AP);
+                const float *ar = A + (base + t) * AP + base;
+                const float4 *ar4 = reinterpret_cast<const float4 *>(ar);
 #pragma unroll
                 for (int i4 = 0; i4 < t / 4; ++i4) {
-                    const float4 av = ar[i4];
+                    const float4 av = ar4[i4];
                     a0 = fmaf(av.x, tc[4 * i4], a0);
                     a1 = fmaf(av.y, tc[4 * i4 + 1], a1);
                     a2 = fmaf(av.z, tc[4 * i4 + 2], a2);
                     a3 = fmaf(av.w, tc[4 * i4 + 3], a3);
                 }
 #pragma unroll
-                for (int i = (t / 4) * 4; i < t; ++i) a0 = fmaf(A[t * AP + i], tc[i], a0);
-                const float acc = (a0 + a1) + (a2 + a3);
-                tc[t] = t < j ? 0.f : (t == j ? 1.f : -acc);
+                for (int i = (t / 4) * 4; i < t; ++i) a0 = fmaf(ar[i], tc[i], a0);
+                tc[t] = t < jj ? 0.f : (t == jj ? 1.f : -((a0 + a1) + (a2 + a3)));
             }
+            __syncwarp();
+            // every column of this block is in registers once all threads of the block (one
+            // warp) are here: the diagonal block of A is dead
+#pragma unroll
+            for (int t = 0; t < 32; ++t) A[(base + t) * AP + base + jj] = tc[t];
         }
-        __syncthreads();                                   // every column done: A is dead
+        __syncthreads();
+        const int r = tid >> 3, c4 = (tid & 7) * 4;         // a row of the 32 x 32 block, 4 columns
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {                   // Y = A10 T00
+            const float a = A[(32 + r) * AP + kk];
+            const float4 t4 = *reinterpret_cast<const float4 *>(A + kk * AP + c4);
+            y.x = fmaf(a, t4.x, y.x); y.y = fmaf(a, t4.y, y.y);
+            y.z = fmaf(a, t4.z, y.z); y.w = fmaf(a, t4.w, y.w);
+        }
+        __syncthreads();                                    // A10 is read: Y takes its place
+        *reinterpret_cast<float4 *>(A + (32 + r) * AP + c4) = y;
+        __syncthreads();
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int kk = 0; kk < 32; ++kk) {                   // T10 = -T11 Y
+            const float tk = A[(32 + r) * AP + 32 + kk];
+            const float4 y4 = *reinterpret_cast<const float4 *>(A + (32 + kk) * AP + c4);
+            z.x = fmaf(-tk, y4.x, z.x); z.y = fmaf(-tk, y4.y, z.y);
+            z.z = fmaf(-tk, y4.z, z.z); z.w = fmaf(-tk, y4.w, z.w);
+        }
+        __syncthreads();
+        *reinterpret_cast<float4 *>(A + (32 + r) * AP + c4) = z;
+        __syncthreads();
+        float tcol[C];
+        if (tid < C)
+#pragma unroll
+            for (int t = 0; t < C; ++t) tcol[t] = A[t * AP + tid];
+        __syncthreads();                                   // T is in registers: A is dead
         if (tid < C) {
             const int j = tid;
             const float s1 = s.bb[j] * s.eg[j], s2 = s.bb[j];
 #pragma unroll
             for (int t = 0; t < C; ++t) {
-                T1[t * SC + j] = __float2bfloat16_rn(tc[t] * s1);
-                T2[t * SC + j] = __float2bfloat16_rn(tc[t] * s2);
+                T1[t * SC + j] = __float2bfloat16_rn(tcol[t] * s1);
+                T2[t * SC + j] = __float2bfloat16_rn(tcol[t] * s2);
             }
         }
         __syncthreads();
