@@ -65,6 +65,30 @@ struct BwdP {
 template <typename E> __device__ __forceinline__ float ldf(const E *p, long i);
 template <> __device__ __forceinline__ float ldf<float>(const float *p, long i) { return p[i]; }
 template <> __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, long i) { return __bfloat162float(p[i]); }
+// four consecutive elements (i a multiple of 4, the row 16-byte aligned)
+template <typename E> __device__ __forceinline__ float4 ld4(const E *p, long i);
+template <> __device__ __forceinline__ float4 ld4<float>(const float *p, long i) { return *reinterpret_cast<const float4 *>(p + i); }
+template <> __device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16 *p, long i)
+{
+    const uint2 u = *reinterpret_cast<const uint2 *>(p + i);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+template <typename E> __device__ __forceinline__ void st4(E *p, long i, float4 v);
+template <> __device__ __forceinline__ void st4<float>(float *p, long i, float4 v) { *reinterpret_cast<float4 *>(p + i) = v; }
+template <> __device__ __forceinline__ void st4<__nv_bfloat16>(__nv_bfloat16 *p, long i, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p + i) = u;
+}
+__device__ __forceinline__ float4 f4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void f4st(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ float4 scale4(float a, float4 x) { return make_float4(a * x.x, a * x.y, a * x.z, a * x.w); }
+
 template <typename E> __device__ __forceinline__ void stf(E *p, long i, float x);
 template <> __device__ __forceinline__ void stf<float>(float *p, long i, float x) { p[i] = x; }
 template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p, long i, float x) { p[i] = __float2bfloat16(x); }
@@ -346,13 +370,13 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
     const int n = (int)min((long)C, p.L - t0);
     const long base = ((long)bh * p.L + t0) * D;
     float *g = w + O_VEC, *bb = g + C, *aa = bb + C, *bg = aa + C;
-    for (int e = tid; e < CD; e += THREADS) {
-        const int t = e / D;
-        const bool ok = t < n;
-        w[O_Q + e] = ok ? ldf((const E *)p.q, base + e) : 0.f;
-        w[O_K + e] = ok ? ldf((const E *)p.k, base + e) : 0.f;
-        w[O_V + e] = ok ? ldf((const E *)p.v, base + e) : 0.f;
-        w[O_G + e] = ok ? ldf((const E *)p.dO, base + e) : 0.f;
+    for (int e = 4 * tid; e < CD; e += 4 * THREADS) {  // four elements of one token a thread
+        const bool ok = e / D < n;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        f4st(w + O_Q + e, ok ? ld4((const E *)p.q, base + e) : z);
+        f4st(w + O_K + e, ok ? ld4((const E *)p.k, base + e) : z);
+        f4st(w + O_V + e, ok ? ld4((const E *)p.v, base + e) : z);
+        f4st(w + O_G + e, ok ? ld4((const E *)p.dO, base + e) : z);
     }
     if (tid < 32) {
         // g_t = running sum of log a over the chunk (tokens past n add nothing): two tokens a
@@ -423,10 +447,10 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
     gemm<E>(w + O_W, D, w + O_T, C, false, w + O_K, D, false, bg, C, D, C, 1.f, 0.f, sm);
     gemm<E>(w + O_UP, D, w + O_T, C, false, w + O_V, D, false, bb, C, D, C, 1.f, 0.f, sm);
     const float gC = g[C - 1];
-    for (int e = tid; e < CD; e += THREADS) {
+    for (int e = 4 * tid; e < CD; e += 4 * THREADS) {
         const int t = e / D;
-        w[O_QT + e] = t < n ? expf(g[t]) * w[O_Q + e] : 0.f;
-        w[O_KT + e] = t < n ? expf(gC - g[t]) * w[O_K + e] : 0.f;
+        f4st(w + O_QT + e, scale4(t < n ? expf(g[t]) : 0.f, f4(w + O_Q + e)));
+        f4st(w + O_KT + e, scale4(t < n ? expf(gC - g[t]) : 0.f, f4(w + O_K + e)));
     }
     gemm<E>(w + O_QT, D, w + O_P, C, false, w + O_W, D, false, nullptr, C, D, C, -1.f, 1.f, sm);
 }
@@ -627,7 +651,7 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     const float gC = g[C - 1];
     const float *S0 = w + O_S0, *dSC = w + O_DSC;
     // U = Up - W S0^T and K S0^T
-    for (int e = tid; e < CD; e += THREADS) w[O_U + e] = w[O_UP + e];
+    for (int e = 4 * tid; e < CD; e += 4 * THREADS) f4st(w + O_U + e, f4(w + O_UP + e));
     gemm2<E>(w + O_U, w + O_KS, D, w + O_W, w + O_K, D, false, S0, D, true, C, D, D, -1.f, 1.f, 1.f, 0.f, sm);
     // dU = Kt dS_C^T + P^T dO (and K dS_C^T);  dR = T^T dU
     gemm2<E>(w + O_DU, w + O_KD, D, w + O_KT, w + O_K, D, false, dSC, D, true, C, D, D, 1.f, 0.f, 1.f, 0.f, sm);
@@ -751,21 +775,24 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     }
     __syncthreads();
     // dQ = diag(e^g) dO S0 + (dP o Gam) K
-    for (int e = tid; e < CD; e += THREADS) w[O_DQ + e] = expf(g[e / D]) * w[O_DS + e];
+    for (int e = 4 * tid; e < CD; e += 4 * THREADS) f4st(w + O_DQ + e, scale4(expf(g[e / D]), f4(w + O_DS + e)));
     gemm<E>(w + O_DQ, D, w + O_DP, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     // dK = diag(e^{g_C - g}) U dS_C - diag(b e^g) dR S0 + (dP o Gam)^T Q + M K + M^T K
-    for (int e = tid; e < CD; e += THREADS) {
+    for (int e = 4 * tid; e < CD; e += 4 * THREADS) {
         const int t = e / D;
-        w[O_DK + e] = t < n ? expf(gC - g[t]) * w[O_UD + e] - bb[t] * expf(g[t]) * w[O_RS + e] : 0.f;
+        const float cu = t < n ? expf(gC - g[t]) : 0.f, cr = t < n ? -bb[t] * expf(g[t]) : 0.f;
+        const float4 ud = f4(w + O_UD + e), rs = f4(w + O_RS + e);
+        f4st(w + O_DK + e, make_float4(fmaf(cu, ud.x, cr * rs.x), fmaf(cu, ud.y, cr * rs.y),
+                                       fmaf(cu, ud.z, cr * rs.z), fmaf(cu, ud.w, cr * rs.w)));
     }
     gemm<E>(w + O_DK, D, w + O_DP, C, true, w + O_Q, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     gemm<E>(w + O_DK, D, w + O_DA, C, false, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     gemm<E>(w + O_DK, D, w + O_DA, C, true, w + O_K, D, false, nullptr, C, D, C, 1.f, 1.f, sm);
     const long base = ((long)bh * p.L + (long)c * C) * D;
-    for (int e = tid; e < n * D; e += THREADS) {
-        stf((E *)p.dq, base + e, w[O_DQ + e]);
-        stf((E *)p.dk, base + e, w[O_DK + e]);
-        stf((E *)p.dv, base + e, bb[e / D] * w[O_DR + e]);
+    for (int e = 4 * tid; e < n * D; e += 4 * THREADS) {
+        st4((E *)p.dq, base + e, f4(w + O_DQ + e));
+        st4((E *)p.dk, base + e, f4(w + O_DK + e));
+        st4((E *)p.dv, base + e, scale4(bb[e / D], f4(w + O_DR + e)));
     }
 }
 
