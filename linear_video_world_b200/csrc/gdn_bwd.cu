@@ -34,6 +34,7 @@ constexpr int D = 128;
 constexpr int THREADS = 256;
 constexpr int R = 8;                // state rows per CTA in the state passes
 constexpr int CD = C * D, CC = C * C, DD = D * D;
+static_assert(D == 128, "the gradient kernel's row sums take four columns a lane");
 constexpr int DS = D + 4;           // staged row stride: 16-byte rows, no bank conflicts
 constexpr int CDS = C * DS;
 constexpr int TS = 68;              // row stride of the block GEMM's staged tiles
@@ -408,14 +409,24 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_prep(BwdP p)
     __syncthreads();
     gemm<E>(w + O_KK, C, w + O_K, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
     gemm<E>(w + O_P, C, w + O_Q, D, false, w + O_K, D, true, nullptr, C, C, D, 1.f, 0.f, sm);
-    for (int e = tid; e < CC; e += THREADS) {
-        const int t = e / C, s = e % C;
-        const bool inc = s <= t && t < n;
-        const float dec = inc ? expf(g[t] - g[s]) : 0.f;
-        const float av = s < t ? bb[t] * dec * w[O_KK + e] : 0.f;
-        w[O_A + e] = av;
-        At[t * AP + s] = av;
-        w[O_P + e] = dec * w[O_P + e];
+    for (int e = 4 * tid; e < CC; e += 4 * THREADS) {  // columns s .. s + 3 of row t
+        const int t = e / C, s0 = e % C;
+        const float gt = g[t], bt = bb[t];
+        const float4 gs = f4(g + s0), kk = f4(w + O_KK + e), pp = f4(w + O_P + e);
+        const float gsv[4] = {gs.x, gs.y, gs.z, gs.w}, kkv[4] = {kk.x, kk.y, kk.z, kk.w};
+        const float ppv[4] = {pp.x, pp.y, pp.z, pp.w};
+        float av[4], pv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            const float dec = (s <= t && t < n) ? expf(gt - gsv[u]) : 0.f;
+            av[u] = s < t ? bt * dec * kkv[u] : 0.f;
+            pv[u] = dec * ppv[u];
+        }
+        const float4 a4 = make_float4(av[0], av[1], av[2], av[3]);
+        f4st(w + O_A + e, a4);
+        f4st(At + t * AP + s0, a4);
+        f4st(w + O_P + e, make_float4(pv[0], pv[1], pv[2], pv[3]));
     }
     __syncthreads();
     if (tid < C) {
@@ -679,12 +690,17 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
         }
         const float eg = expf(g[t]);
         float qds = 0.f, drk = 0.f, ukd = 0.f, drv = 0.f;
-        for (int j = lane; j < D; j += 32) {
-            const float ks = w[O_KS + t * D + j], dr = w[O_DR + t * D + j];
-            qds = fmaf(w[O_Q + t * D + j], w[O_DS + t * D + j], qds);
-            drk = fmaf(dr, ks, drk);
-            ukd = fmaf(w[O_U + t * D + j], w[O_KD + t * D + j], ukd);
-            drv = fmaf(dr, w[O_V + t * D + j] - eg * ks, drv);
+        {
+            const int j = 4 * lane;                         // D = 128: four columns a lane
+            const float4 ks = f4(w + O_KS + t * D + j), dr = f4(w + O_DR + t * D + j);
+            const float4 qq = f4(w + O_Q + t * D + j), ds = f4(w + O_DS + t * D + j);
+            const float4 uu = f4(w + O_U + t * D + j), kd = f4(w + O_KD + t * D + j);
+            const float4 vv = f4(w + O_V + t * D + j);
+            qds = fmaf(qq.x, ds.x, fmaf(qq.y, ds.y, fmaf(qq.z, ds.z, qq.w * ds.w)));
+            drk = fmaf(dr.x, ks.x, fmaf(dr.y, ks.y, fmaf(dr.z, ks.z, dr.w * ks.w)));
+            ukd = fmaf(uu.x, kd.x, fmaf(uu.y, kd.y, fmaf(uu.z, kd.z, uu.w * kd.w)));
+            drv = fmaf(dr.x, vv.x - eg * ks.x, fmaf(dr.y, vv.y - eg * ks.y,
+                  fmaf(dr.z, vv.z - eg * ks.z, dr.w * (vv.w - eg * ks.w))));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -719,7 +735,10 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
     }
     // <dS_C, S0>
     float sd = 0.f;
-    for (int e = tid; e < DD; e += THREADS) sd = fmaf(dSC[e], S0[e], sd);
+    for (int e = 4 * tid; e < DD; e += 4 * THREADS) {
+        const float4 x = f4(dSC + e), y = f4(S0 + e);
+        sd = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, sd))));
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);
     if (lane == 0) red[warp] = sd;
@@ -766,12 +785,23 @@ __global__ void __launch_bounds__(THREADS, 2) gdn_bwd_grad(BwdP p)
         }
     }
     // M = dA o b_t e^{g_t - g_s} (s < t) into O_DA;  dP o Gam into O_DP
-    for (int e = tid; e < CC; e += THREADS) {
-        const int t = e / C, s = e % C;
-        const bool inc = s <= t && t < n, low = s < t && t < n;
-        const float dec = inc ? expf(g[t] - g[s]) : 0.f;
-        w[O_DA + e] = low ? -w[O_DA + e] * bb[t] * dec : 0.f;
-        w[O_DP + e] = inc ? w[O_DP + e] * dec : 0.f;
+    for (int e = 4 * tid; e < CC; e += 4 * THREADS) {  // columns s .. s + 3 of row t
+        const int t = e / C, s0 = e % C;
+        const float gt = g[t], bt = bb[t];
+        const float4 gs = f4(g + s0), da = f4(w + O_DA + e), dp = f4(w + O_DP + e);
+        const float gsv[4] = {gs.x, gs.y, gs.z, gs.w}, dav[4] = {da.x, da.y, da.z, da.w};
+        const float dpv[4] = {dp.x, dp.y, dp.z, dp.w};
+        float mo[4], po[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = s0 + u;
+            const bool inc = s <= t && t < n, low = s < t && t < n;
+            const float dec = inc ? expf(gt - gsv[u]) : 0.f;
+            mo[u] = low ? -dav[u] * bt * dec : 0.f;
+            po[u] = inc ? dpv[u] * dec : 0.f;
+        }
+        f4st(w + O_DA + e, make_float4(mo[0], mo[1], mo[2], mo[3]));
+        f4st(w + O_DP + e, make_float4(po[0], po[1], po[2], po[3]));
     }
     __syncthreads();
     // dQ = diag(e^g) dO S0 + (dP o Gam) K
