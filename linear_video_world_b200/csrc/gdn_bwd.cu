@@ -1,5 +1,5 @@
-// Backward pass of the gated delta rule in chunk form, fp32 arithmetic on the CUDA cores
-// (bf16 or fp32 inputs and gradients; d = 128, chunks of 64 tokens).
+// Backward pass of the gated delta rule in chunk form (bf16 or fp32 inputs and gradients;
+// d = 128, chunks of 64 tokens; fp32 accumulation throughout).
 //
 // The derivative of the chunk form of the forward pass, term by term. Per chunk, with start
 // state S0, end-state gradient dS_C, g the running sum of log a, R = diag(b)(V - diag(e^g) K S0^T),
@@ -17,11 +17,14 @@
 //     d(log a) = reverse running sum of dg inside the chunk,  da = d(log a) / a
 // (Gam: e^{g_t - g_s} on s <= t; only such decays, with non-positive exponents, are formed.)
 //
-// Four launches: prep (every chunk in parallel: inputs to fp32, the chunk's A, T, P, W, Up,
-// Qt, Kt), the forward state pass storing each chunk's start state, the backward state pass
+// Launches: prep (every chunk in parallel: inputs to fp32, the chunk's A, T, P, W, Up, Qt,
+// Kt), the forward state pass storing each chunk's start state, the backward state pass
 // storing each chunk's end-state gradient (both serial over chunks, parallel over rows of the
-// state), and the gradient kernel (every chunk in parallel). Products go through one block
-// GEMM routine on fp32 operands in the workspace (a chunk's working set stays in L2).
+// state), and the gradient kernel (every chunk in parallel). The per-chunk products go through
+// one block GEMM routine on the fp32 operands in the workspace: on the CUDA cores for fp32
+// tensors, on the tensor cores (mma.sync, operands rounded to bf16, fp32 accumulation) for
+// bf16 ones. With bf16 tensors the two state passes are the tensor-core kernels of gdn_tc.cu
+// (after the forward's chunk preparation), run on side streams beside this file's prep.
 #include "hlta_internal.cuh"
 
 #include <math.h>
@@ -63,9 +66,6 @@ struct BwdP {
     int BH, nch;
 };
 
-template <typename E> __device__ __forceinline__ float ldf(const E *p, long i);
-template <> __device__ __forceinline__ float ldf<float>(const float *p, long i) { return p[i]; }
-template <> __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, long i) { return __bfloat162float(p[i]); }
 // four consecutive elements (i a multiple of 4, the row 16-byte aligned)
 template <typename E> __device__ __forceinline__ float4 ld4(const E *p, long i);
 template <> __device__ __forceinline__ float4 ld4<float>(const float *p, long i) { return *reinterpret_cast<const float4 *>(p + i); }
@@ -90,9 +90,6 @@ __device__ __forceinline__ float4 f4(const float *p) { return *reinterpret_cast<
 __device__ __forceinline__ void f4st(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
 __device__ __forceinline__ float4 scale4(float a, float4 x) { return make_float4(a * x.x, a * x.y, a * x.z, a * x.w); }
 
-template <typename E> __device__ __forceinline__ void stf(E *p, long i, float x);
-template <> __device__ __forceinline__ void stf<float>(float *p, long i, float x) { p[i] = x; }
-template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p, long i, float x) { p[i] = __float2bfloat16(x); }
 
 // O[M][N] = alpha * sum_k opA(m, k) s(k) opB(k, n) + beta * O[m][n]; opA(m, k) = A[m][k] or,
 // transposed, A[k][m] (leading dimension lda); opB likewise; s an optional per-k scale.
