@@ -460,7 +460,9 @@ def hybrid(q, k, v, a, b, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, S0=None, chunk=64,
 
 
 class Stream:
-    """Streaming cache (hlta_stream_create / _step / _state / _destroy)."""
+    """Streaming cache (hlta_stream_create_ex / _step / _step_frames / _state /
+    _frame_counter / _destroy). A step may be captured into a CUDA graph and replayed for the
+    following frames: the frame index lives in a device counter that every step advances."""
 
     def __init__(self, B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk=64, scale=0.0,
                  dtype=None, S0=None, max_step_frames=1):
