@@ -192,7 +192,7 @@ __device__ __forceinline__ void cp_async16(float *dst, const float *src)
                  "l"(src) : "memory");
 }
 
-constexpr int TC_NSTG = 3;                  // stages of the operand ring
+constexpr int TC_NSTG = 3;                  // stages of the operand ring with two A operands
 constexpr int TC_SK = 40;                   // row stride of [64][32] tiles (floats)
 constexpr int TC_SN = 68;                   // row stride of [32][64] tiles
 constexpr int TC_TILE = 64 * TC_SK;         // floats reserved per operand tile (>= 32 * TC_SN)
@@ -211,13 +211,16 @@ __device__ void bgemm_tc_n(float *const (&O)[NA], int ldo, const float *const (&
     const int wm = warp & 3, wn = warp >> 2, g = lane >> 2, tg = lane & 3;
     const int nk = K / 32, ntn = N / 64, steps = (M / 64) * ntn * nk;
     constexpr int STAGE = (NA + 1) * TC_TILE;
-    // step st: output tile st / nk, k-step st % nk, into stage st % TC_NSTG (16-byte copies,
+    // as many stages as the staging area holds: four with one A operand, three with two
+    constexpr int NSTG = TC_SMEM_FLOATS / STAGE;
+    static_assert(NSTG >= 3, "at least three stages");
+    // step st: output tile st / nk, k-step st % nk, into stage st % NSTG (16-byte copies,
     // two per thread and operand tile)
     auto issue = [&](int st) {
         if (st < steps) {
             const int tile = st / nk, k0 = (st % nk) * 32;
             const int m0 = (tile / ntn) * 64, n0 = (tile % ntn) * 64;
-            float *sa = smf + (st % TC_NSTG) * STAGE, *sb = sa + NA * TC_TILE;
+            float *sa = smf + (st % NSTG) * STAGE, *sb = sa + NA * TC_TILE;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int e = tid + r * THREADS;
@@ -234,13 +237,13 @@ __device__ void bgemm_tc_n(float *const (&O)[NA], int ldo, const float *const (&
     };
     __syncthreads();                                // the caller's operand stores are visible
 #pragma unroll
-    for (int st = 0; st < TC_NSTG - 1; ++st) issue(st);
+    for (int st = 0; st < NSTG - 1; ++st) issue(st);
     float acc[NA][4][4] = {};
     for (int st = 0; st < steps; ++st) {
-        asm volatile("cp.async.wait_group %0;" ::"n"(TC_NSTG - 2) : "memory");
+        asm volatile("cp.async.wait_group %0;" ::"n"(NSTG - 2) : "memory");
         __syncthreads();                            // step st landed for all; stage st - 1 is free
-        issue(st + TC_NSTG - 1);
-        const float *sa = smf + (st % TC_NSTG) * STAGE, *sb = sa + NA * TC_TILE;
+        issue(st + NSTG - 1);
+        const float *sa = smf + (st % NSTG) * STAGE, *sb = sa + NA * TC_TILE;
         const int k0 = (st % nk) * 32;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
