@@ -176,3 +176,36 @@ def test_chunk_backward_equals_recurrence_backward(orc, C):
                          dO.astype(np.float64), dSL, C)
     for x, r in zip(got, ref):
         np.testing.assert_allclose(x, r[0], rtol=1e-8, atol=1e-9)
+
+
+def _blocked_unit_lower_inverse(A):
+    """(I + A)^-1 for strictly lower-triangular 64 x 64 A the way the chunk preparation forms
+    it: the two diagonal 32 x 32 blocks by forward substitution, then T10 = -T11 A10 T00."""
+    n = A.shape[0]
+    h = n // 2
+    T = np.zeros_like(A)
+    for base in (0, h):
+        for j in range(h):
+            col = np.zeros(h)
+            for t in range(h):
+                if t < j:
+                    continue
+                col[t] = 1.0 if t == j else -A[base + t, base:base + t] @ col[:t]
+            T[base:base + h, base + j] = col
+    T[h:, :h] = -T[h:, h:] @ (A[h:, :h] @ T[:h, :h])
+    return T
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_blocked_inverse_equals_inverse(seed):
+    rng = np.random.default_rng(seed)
+    n = 64
+    k = rng.standard_normal((n, 128))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    b = rng.uniform(0.0, 1.0, n)
+    g = np.cumsum(np.log(rng.uniform(0.5, 1.0, n)))
+    low = np.tril(np.ones((n, n)), -1)
+    A = low * b[:, None] * np.exp(np.where(low > 0, g[:, None] - g[None, :], 0)) * (k @ k.T)
+    T = _blocked_unit_lower_inverse(A)
+    assert np.allclose(T, np.linalg.inv(np.eye(n) + A), atol=1e-10)
+    assert np.allclose(np.triu(T, 1), 0.0) and np.allclose(np.diag(T), 1.0)
