@@ -177,7 +177,8 @@ hlta_status hlta_window_bwd(const void *q, const void *k, const void *v, const v
  * p = l mod N, the token's index inside its frame, for pos_mode 0 (the local position; a
  * streaming step's frame index does not enter); p = l, the index in the sequence, for
  * pos_mode 1.
- * q, k: [B, H, L, d] device, element type `dt`, either may be NULL (skipped); heads
+ * q, k: [B, H, L, d] device, element type `dt`, either may be NULL (skipped), not overlapping
+ * each other (the same rows passed as both would turn twice); heads
  * [h0, h0 + Hr) are rotated, the others untouched (so the softmax heads of a hybrid tensor
  * can be rotated in place). d even, 2 <= d <= 128; base > 1 finite (10000 is the usual
  * value); N >= 1. The angle is reduced in double precision before a single-precision sine and
