@@ -388,22 +388,51 @@ hlta_status hlta_stream_frame_counter(hlta_stream_t c, int **f_dev);
 hlta_status hlta_stream_destroy(hlta_stream_t c);
 
 /*
- * Profiling hook for hlta_hybrid_fwd (measurement, not needed for results). `events` is NULL
- * (off) or an array of 5 cudaEvent_t created by the caller on the current device. While set,
- * each hlta_hybrid_fwd call records events[0] where the branches fork (on the caller's stream,
- * before any branch kernel), events[1] after the SWA kernel (caller's stream), events[2] after
- * the DSWA kernel (on the stream it ran on), events[3] before and events[4] after the GDN
- * kernels (on the GDN stream). The array is copied; the setting is process-wide and stays
- * until changed.
+ * Profiling hook for hlta_hybrid_fwd(_raw) and the streaming steps (measurement, not needed
+ * for results). `events` is NULL (off) or an array of 5 cudaEvent_t created by the caller on
+ * the current device. While set, each hybrid call or streaming step records events[0] where
+ * the branches fork (on the caller's stream, before any branch kernel), events[1] after the
+ * SWA kernel (caller's stream), events[2] after the DSWA kernel (on the stream it ran on),
+ * events[3] before and events[4] after the GDN kernels (on the GDN stream). The array is
+ * copied; the setting is process-wide and stays until changed.
  */
 hlta_status hlta_set_profile_events(void *const *events);
 
 /*
+ * Measurement hook: the number of kernels this library has enqueued in this process so far
+ * (all devices, all host threads; replays of a captured CUDA graph are not calls and are not
+ * counted). The difference over a region is the number of the library's kernel launches in it.
+ */
+unsigned long long hlta_kernel_launches(void);
+
+/* Bits of the device error word (hlta_device_status): the kernel kind whose bounded wait
+ * expired. */
+#define HLTA_DEVERR_ATTN_WAIT 0x1u  /* a window-attention kernel (forward or backward) */
+#define HLTA_DEVERR_GDN_WAIT 0x2u   /* a gated-delta-rule kernel */
+#define HLTA_DEVERR_SELFTEST 0x4u   /* hlta_wait_expiry_selftest */
+
+/*
  * Synchronizes `stream`, then reads and clears the library's device error word.
- * *code receives the raw word (0: no kernel stopped early). Returns HLTA_ERR_TIMEOUT if a
- * bounded wait expired in any kernel since the last call, HLTA_ERR_CUDA on a CUDA error.
+ * *code receives the raw word (0: no kernel stopped early; otherwise HLTA_DEVERR_* bits).
+ * Returns HLTA_ERR_TIMEOUT if a bounded wait expired in any kernel since the last call,
+ * HLTA_ERR_CUDA on a CUDA error.
  */
 hlta_status hlta_device_status(void *stream, unsigned int *code);
+
+/*
+ * Failure-detection self-test (no counterpart on the pages: it exercises this library's own
+ * bounded-wait protocol). Every pipelined kernel of the library waits on its mbarriers with a
+ * cycle limit, after which it records its HLTA_DEVERR_* bit in the device error word, stops
+ * its roles and returns, so a lost arrival ends in an error status instead of a hung GPU.
+ * This call enqueues on `stream` one single-thread kernel that makes such a wait run out: it
+ * waits on a fresh shared-memory mbarrier that nothing arrives at, through the same bounded
+ * wait, for `cycles` SM clock cycles (1 <= cycles <= 2^32; 2^24 is about 9 ms at 1.9 GHz),
+ * then ORs HLTA_DEVERR_SELFTEST into the word and returns. No copy or tensor-core operation is
+ * in flight, so the context stays usable: the next hlta_device_status() reports
+ * HLTA_ERR_TIMEOUT with that bit and clears it. A `cycles` outside the range is
+ * HLTA_ERR_INVALID_ARG (nothing enqueued).
+ */
+hlta_status hlta_wait_expiry_selftest(unsigned long long cycles, void *stream);
 
 #ifdef __cplusplus
 }

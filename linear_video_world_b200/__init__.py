@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libhlta.so")
 
 HLTA_OK, HLTA_ERR_INVALID_ARG, HLTA_ERR_UNSUPPORTED, HLTA_ERR_CUDA, HLTA_ERR_TIMEOUT = range(5)
 HLTA_BF16, HLTA_FP32 = 0, 1
+HLTA_DEVERR_ATTN_WAIT, HLTA_DEVERR_GDN_WAIT, HLTA_DEVERR_SELFTEST = 0x1, 0x2, 0x4
 _STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "CUDA", 4: "TIMEOUT"}
 
 
@@ -67,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "hlta_gdn_chunk_bwd": (I, [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, L, I, I, P, Z, I,
                                    P]),
         "hlta_device_status": (I, [P, ctypes.POINTER(ctypes.c_uint)]),
+        "hlta_kernel_launches": (ctypes.c_ulonglong, []),
+        "hlta_wait_expiry_selftest": (I, [ctypes.c_ulonglong, P]),
         "hlta_set_profile_events": (I, [ctypes.POINTER(P)]),
     }
     for name, (res, args) in sig.items():
@@ -293,6 +296,22 @@ def hlta_device_status(stream=None) -> int:
     code = ctypes.c_uint(0)
     _check(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
     return int(code.value)
+
+
+def hlta_device_status_code(stream=None):
+    """(status, raw device error word) without raising: hlta_device_status for callers that
+    handle an expired wait themselves."""
+    code = ctypes.c_uint(0)
+    st = int(_lib.hlta_device_status(_stream(stream), ctypes.byref(code)))
+    return st, int(code.value)
+
+
+def hlta_kernel_launches() -> int:
+    return int(_lib.hlta_kernel_launches())
+
+
+def hlta_wait_expiry_selftest(cycles, stream=None):
+    _check(_lib.hlta_wait_expiry_selftest(int(cycles), _stream(stream)))
 
 
 def hlta_set_profile_events(events):

@@ -45,7 +45,7 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs &a, cudaStream_t s)
     if (rows == 0) return cudaSuccess;
     if (a.BH > 65535 || rows >= (1L << 40)) return cudaErrorNotSupported;
     attn_bwd_dot<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const __nv_bfloat16 *)a.o,
-                                                            (const __nv_bfloat16 *)a.dO, a.Dws, rows);
+                                                            (const __nv_bfloat16 *)a.dO, a.Dws, rows), note_launch();
     cudaError_t e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return launch_attn_bwd_tc(a, s);

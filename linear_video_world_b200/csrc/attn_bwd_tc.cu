@@ -490,7 +490,7 @@ cudaError_t launch_attn_bwd_tc(const AttnBwdArgs &a, cudaStream_t s)
     if ((e = cudaFuncSetAttribute(attn_bwd_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess)
         return e;
     const dim3 grid((unsigned)((long)a.T * p.tpk), (unsigned)a.BH);
-    attn_bwd_dkv_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mk, mv, mq, mg, p);
+    attn_bwd_dkv_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mk, mv, mq, mg, p), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // dQ: query tiles of 128 rows (the maps of the other kernel with the boxes exchanged)
     CUtensorMap mq2, mg2, mk2, mv2;
@@ -500,7 +500,7 @@ cudaError_t launch_attn_bwd_tc(const AttnBwdArgs &a, cudaStream_t s)
     if ((e = make_tmap_2d_bf16(&mv2, a.v, rows, D, 64, BQ, true)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(attn_bwd_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES)) != cudaSuccess)
         return e;
-    attn_bwd_dq_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mq2, mg2, mk2, mv2, p, (__nv_bfloat16 *)a.dq);
+    attn_bwd_dq_tc<<<grid, THREADS, SMEM_BYTES, s>>>(mq2, mg2, mk2, mv2, p, (__nv_bfloat16 *)a.dq), note_launch();
     return cudaGetLastError();
 }
 

@@ -139,7 +139,7 @@ cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s)
     size_t smem = sizeof(float) * ((size_t)QB * a.d + (size_t)KT * (a.d + 1) + (size_t)KT * a.d);
     // d <= 128: at most 41 KB, inside the default dynamic shared memory limit
     dim3 grid((unsigned)((a.q_rows + QB - 1) / QB), (unsigned)(a.B * a.Hbr));
-    attn_f32_kernel<<<grid, THREADS, smem, s>>>(a);
+    attn_f32_kernel<<<grid, THREADS, smem, s>>>(a), note_launch();
     return cudaGetLastError();
 }
 

@@ -910,7 +910,7 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t s)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
-    kern<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p);
+    kern<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p), note_launch();
     return cudaGetLastError();
 }
 

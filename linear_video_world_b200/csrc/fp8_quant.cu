@@ -182,7 +182,7 @@ cudaError_t launch_fp8_quantize_rows(const void *x, const float *shift, long BH,
     if (blocks >= (1L << 31) || nf >= (1L << 31) || nb >= (1L << 31)) return cudaErrorNotSupported;
     fp8_rows_kernel<<<(unsigned)blocks, QTHREADS, 0, s>>>((const __nv_bfloat16 *)x, shift, L,
                                                          frame_rows, block_rows, (int)nf, (int)nb,
-                                                         (uint8_t *)x8, scales);
+                                                         (uint8_t *)x8, scales), note_launch();
     return cudaGetLastError();
 }
 
@@ -195,12 +195,12 @@ cudaError_t launch_fp8_quantize_channels(const void *x, long BH, long L, void *x
     if (e != cudaSuccess) return e;
     if (L > 0) {
         const dim3 grid((unsigned)((L + CH_ROWS - 1) / CH_ROWS), (unsigned)BH);
-        fp8_channel_max_kernel<<<grid, QTHREADS, 0, s>>>((const __nv_bfloat16 *)x, L, (unsigned int *)scales);
+        fp8_channel_max_kernel<<<grid, QTHREADS, 0, s>>>((const __nv_bfloat16 *)x, L, (unsigned int *)scales), note_launch();
         fp8_channel_quant_kernel<<<grid, QTHREADS, 0, s>>>((const __nv_bfloat16 *)x, L, (const unsigned int *)scales,
-                                                           (uint8_t *)x8);
+                                                           (uint8_t *)x8), note_launch();
     }
     const long n = BH * D;
-    fp8_channel_scale_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, n);
+    fp8_channel_scale_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, n), note_launch();
     return cudaGetLastError();
 }
 

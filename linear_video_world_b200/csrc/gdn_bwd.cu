@@ -844,10 +844,10 @@ cudaError_t launch_typed(const BwdP &p, cudaStream_t s)
     if ((e = cudaFuncSetAttribute(gdn_bwd_fwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_f)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_bwd_bwdstate, cudaFuncAttributeMaxDynamicSharedMemorySize, sm_b)) != cudaSuccess) return e;
     if ((e = set_gemm_smem<E>()) != cudaSuccess) return e;
-    gdn_bwd_prep<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p);
-    gdn_bwd_fwdstate<<<gs, THREADS, sm_f, s>>>(p);
-    gdn_bwd_bwdstate<<<gs, THREADS, sm_b, s>>>(p);
-    gdn_bwd_grad<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p);
+    gdn_bwd_prep<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p), note_launch();
+    gdn_bwd_fwdstate<<<gs, THREADS, sm_f, s>>>(p), note_launch();
+    gdn_bwd_bwdstate<<<gs, THREADS, sm_b, s>>>(p), note_launch();
+    gdn_bwd_grad<E><<<gc, THREADS, gemm_smem_bytes<E>(), s>>>(p), note_launch();
     return cudaGetLastError();
 }
 
@@ -904,7 +904,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStream
     e = set_gemm_smem<__nv_bfloat16>();
     if (e == cudaSuccess) {
         gdn_bwd_prep<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS,
-                                      gemm_smem_bytes<__nv_bfloat16>(), s>>>(p);
+                                      gemm_smem_bytes<__nv_bfloat16>(), s>>>(p), note_launch();
         e = cudaGetLastError();
     }
     if (side) {
@@ -917,7 +917,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStream
     if (es != cudaSuccess) return es;
     if (e != cudaSuccess) return e;
     gdn_bwd_grad<__nv_bfloat16><<<dim3((unsigned)nch, (unsigned)p.BH), THREADS,
-                                  gemm_smem_bytes<__nv_bfloat16>(), s>>>(p);
+                                  gemm_smem_bytes<__nv_bfloat16>(), s>>>(p), note_launch();
     return cudaGetLastError();
 }
 

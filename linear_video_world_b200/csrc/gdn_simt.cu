@@ -234,11 +234,11 @@ cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s)
     e = cudaFuncSetAttribute(gdn_state_f32, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_state);
     if (e != cudaSuccess) return e;
-    gdn_prep_f32<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), PREP_THREADS, smem_prep, s>>>(g, ws);
+    gdn_prep_f32<<<dim3((unsigned)nch, (unsigned)(g.B * g.Hg)), PREP_THREADS, smem_prep, s>>>(g, ws), note_launch();
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     gdn_state_f32<<<dim3((unsigned)((d + R - 1) / R), (unsigned)(g.B * g.Hg)), STATE_THREADS,
-                    smem_state, s>>>(g, ws);
+                    smem_state, s>>>(g, ws), note_launch();
     return cudaGetLastError();
 }
 

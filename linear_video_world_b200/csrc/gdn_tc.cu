@@ -976,9 +976,9 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
     if (e != cudaSuccess) return e;
-    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws), note_launch();
     return cudaGetLastError();
 }
 
@@ -1016,16 +1016,16 @@ cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const f
     if ((e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_dstate_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dstate)) != cudaSuccess) return e;
-    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws);
+    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (s2 != s) {
         // the two state passes are independent of each other: side by side
         if ((e = cudaEventRecord(mid, s)) != cudaSuccess) return e;
         if ((e = cudaStreamWaitEvent(s2, mid, 0)) != cudaSuccess) return e;
     }
-    gdn_dstate_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_dstate, s2>>>(dm, g, ws, dS_final, dS_chunks, dS0);
+    gdn_dstate_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_dstate, s2>>>(dm, g, ws, dS_final, dS_chunks, dS0), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws);
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws), note_launch();
     return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 #include "hlta.h"
 #include "hlta_internal.cuh"
 
+#include <atomic>
 #include <math.h>
 #include <mutex>
 #include <stdarg.h>
@@ -217,6 +218,12 @@ int record_error_impl(int st, const char *fmt, ...)
     va_end(ap);
     return st;
 }
+
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 unsigned int *device_error_word()
 {
@@ -706,18 +713,21 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
     // attention) on the second library stream when SWA heads are present too
     std::unique_lock<std::mutex> lk(g_fork_mu, std::defer_lock);
     const bool split_d = c->Hd && c->Hs;
+    lk.lock();
     if (c->Hg || split_d) {
-        lk.lock();
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
+    prof_record(0, s);
     if (c->Hg) {
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+        prof_record(3, ctx->aux);
         GdnArgs g = {};
         g.q = q_new; g.k = k_new; g.v = v_new; g.a = a_new; g.b = b_new; g.o = o_new;
         g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = (long)F * c->N; g.d = c->d;
         g.chunk = c->chunk; g.S0 = c->S; g.S_out = c->S; g.ws = c->ws; g.ws_bytes = c->ws_bytes;
         g.err = ctx->err;
         st = run_gdn(g, c->dt, ctx->aux);
+        prof_record(4, ctx->aux);
         cudaEventRecord(ctx->join, ctx->aux);
         if (st != HLTA_OK) {
             cudaStreamWaitEvent(s, ctx->join, 0);
@@ -748,6 +758,7 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.fq0_dev = c->fdev; a.scale = c->scale;
         a.err = ctx->err;
         if ((st = run_attn(a, c->dt, s)) != HLTA_OK) break;
+        prof_record(bi == 1 ? 2 : 1, s);
     }
     // join the other branches after the softmax launches were enqueued, so they overlap
     if (split_d) {
@@ -796,6 +807,20 @@ hlta_status hlta_set_profile_events(void *const *events)
     std::lock_guard<std::mutex> lk(g_fork_mu);
     g_prof_on = events != nullptr;
     for (int i = 0; i < 5; ++i) g_prof[i] = events ? (cudaEvent_t)events[i] : nullptr;
+    return HLTA_OK;
+}
+
+unsigned long long hlta_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+hlta_status hlta_wait_expiry_selftest(unsigned long long cycles, void *stream)
+{
+    if (cycles < 1 || cycles > (1ull << 32))
+        return fail(HLTA_ERR_INVALID_ARG, "cycles must be in [1, 2^32] (got %llu)", cycles);
+    hlta_status st;
+    DeviceCtx *ctx;
+    if ((st = device_ctx(&ctx)) != HLTA_OK) return st;
+    cudaError_t e = launch_wait_selftest(ctx->err, (long long)cycles, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
     return HLTA_OK;
 }
 

@@ -1,6 +1,8 @@
 // Internal declarations shared by the library's translation units (not part of the ABI).
 #pragma once
 
+#include "hlta.h"
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -155,11 +157,23 @@ cudaError_t launch_frame_advance(int *f, int F, cudaStream_t s);
 cudaError_t launch_rope(void *q, void *k, bool bf16, int B, int Htot, int h0, int Hr, long L,
                         int N, int d, double base, int pos_mode, int sign, cudaStream_t s);
 
-// Device error word: kernels OR a code into it when a bounded wait expires.
+// Device error word: kernels OR a code into it when a bounded wait expires (the bits are the
+// HLTA_DEVERR_* values of hlta.h).
 enum : unsigned int {
     DEVERR_ATTN_WAIT = 1u << 0,
     DEVERR_GDN_WAIT = 1u << 1,
+    DEVERR_SELFTEST = 1u << 2,
 };
+static_assert(DEVERR_ATTN_WAIT == HLTA_DEVERR_ATTN_WAIT && DEVERR_GDN_WAIT == HLTA_DEVERR_GDN_WAIT &&
+                  DEVERR_SELFTEST == HLTA_DEVERR_SELFTEST,
+              "device error bits must match hlta.h");
+
+// Counts one kernel launch enqueued by the library (hlta_kernel_launches); every launch site
+// appends it to its launch statement.
+void note_launch();
+
+// The bounded-wait self-test kernel: waits `cycles` on an mbarrier nothing arrives at.
+cudaError_t launch_wait_selftest(unsigned int *err, long long cycles, cudaStream_t s);
 unsigned int *device_error_word();  // device address of the word (current device)
 
 }  // namespace hlta

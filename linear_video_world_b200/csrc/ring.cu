@@ -26,7 +26,7 @@ __global__ void frame_advance_kernel(int *f, int F) { *f += F; }
 
 cudaError_t launch_frame_advance(int *f, int F, cudaStream_t s)
 {
-    frame_advance_kernel<<<1, 1, 0, s>>>(f, F);
+    frame_advance_kernel<<<1, 1, 0, s>>>(f, F), note_launch();
     return cudaGetLastError();
 }
 
@@ -40,7 +40,7 @@ cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr
     const long frame_vec = (long)(bytes / 16);
     const unsigned gx = (unsigned)((frame_vec + 255) / 256 < 64 ? (frame_vec + 255) / 256 : 64);
     ring_append_kernel<<<dim3(gx, (unsigned)(B * Hbr), (unsigned)F), 256, 0, s>>>(
-        (const uint4 *)src, (uint4 *)ring, Htot, h0, Hbr, frame_vec, F, slots, f0, f0_dev);
+        (const uint4 *)src, (uint4 *)ring, Htot, h0, Hbr, frame_vec, F, slots, f0, f0_dev), note_launch();
     return cudaGetLastError();
 }
 

@@ -131,18 +131,18 @@ cudaError_t launch_rope(void *q, void *k, bool bf16, int B, int Htot, int h0, in
         const unsigned bv = (unsigned)((tv + 255) / 256);
         if (bf16)
             rope_kernel_v<__nv_bfloat16><<<bv, 256, 0, s>>>((__nv_bfloat16 *)q, (__nv_bfloat16 *)k, Htot, h0,
-                                                            Hr, L, N, d, lb, pos_mode, sign, tv);
+                                                            Hr, L, N, d, lb, pos_mode, sign, tv), note_launch();
         else
             rope_kernel_v<float><<<bv, 256, 0, s>>>((float *)q, (float *)k, Htot, h0, Hr, L, N, d, lb,
-                                                    pos_mode, sign, tv);
+                                                    pos_mode, sign, tv), note_launch();
         return cudaGetLastError();
     }
     if (bf16)
         rope_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-            (__nv_bfloat16 *)q, (__nv_bfloat16 *)k, Htot, h0, Hr, L, N, d, lb, pos_mode, sign, total);
+            (__nv_bfloat16 *)q, (__nv_bfloat16 *)k, Htot, h0, Hr, L, N, d, lb, pos_mode, sign, total), note_launch();
     else
         rope_kernel<float><<<(unsigned)blocks, 256, 0, s>>>((float *)q, (float *)k, Htot, h0, Hr, L, N,
-                                                            d, lb, pos_mode, sign, total);
+                                                            d, lb, pos_mode, sign, total), note_launch();
     return cudaGetLastError();
 }
 

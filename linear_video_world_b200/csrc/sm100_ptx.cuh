@@ -49,18 +49,19 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase: gives up after ~2^32 SM cycles (about two seconds), or
-// at once when another role of the CTA already gave up (*abort_flag != 0); an expiry sets
-// *abort_flag and ORs `code` into the device error word.
+// Bounded wait on an mbarrier phase: gives up after `limit` SM cycles (default 2^32, about two
+// seconds), or at once when another role of the CTA already gave up (*abort_flag != 0); an
+// expiry sets *abort_flag and ORs `code` into the device error word.
 __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                              unsigned int *err, unsigned int code)
+                                              unsigned int *err, unsigned int code,
+                                              long long limit = 1LL << 32)
 {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > (1LL << 32)) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(err, code);
             return false;

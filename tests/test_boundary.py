@@ -191,3 +191,14 @@ def test_rope_entry_point_validates_on_host(lib):
     # nothing to rotate: accepted without touching a device
     assert lib.hlta_rope(None, None, 1, 4, 0, 4, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16, None) == h.HLTA_OK
     assert lib.hlta_rope(p, p, 1, 4, 1, 0, 100, 10, 128, F(1e4), 0, 0, h.HLTA_BF16, None) == h.HLTA_OK
+
+
+def test_static_scratch_size_matches_header():
+    """The binding's copy of HLTA_STATIC_SCRATCH_BYTES is the value include/hlta.h defines."""
+    import linear_video_world_b200 as h
+    src = open(os.path.join(ROOT, "include", "hlta.h")).read()
+    m = re.search(r"#define\s+HLTA_STATIC_SCRATCH_BYTES\s+\(([^)]*)\)", src)
+    assert m, "HLTA_STATIC_SCRATCH_BYTES not defined in hlta.h"
+    expr = re.sub(r"(\d+)[uUlL]+", r"\1", m.group(1))
+    assert re.fullmatch(r"[\d\s*+()]+", expr), expr
+    assert eval(expr) == h.HLTA_STATIC_SCRATCH_BYTES

@@ -122,6 +122,40 @@ def test_stream_steps_equal_hybrid_bf16(h, orc):
     st.close()
 
 
+def test_stream_steps_streaming_workload_geometry_sampled(h, orc):
+    """The streaming workload's geometry: B=8 rollouts, frames of N=1560 tokens (64-key tiles
+    straddle frames), SWA w=3, DSWA w=4 r=6 (a ring of r(w-1)+1 = 19 frame slots), d=128, one
+    head per branch. 26 single-frame steps from empty caches, so every ring slot is reused and
+    the last eight steps see all DSWA taps. Each step's softmax outputs on sampled rows of
+    every frame, every GDN output and the final state are compared with the oracle's hybrid
+    over the concatenated 26-frame clip."""
+    wl = hi.WORKLOADS["stream_480p"].with_(Hs=1, Hd=1, Hg=1, T=26, streaming=False)
+    assert wl.r * (wl.w_dswa - 1) + 1 == 19
+    x = hi.make_inputs(wl, seed=41)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    st = h.Stream(wl.B, wl.Hs, wl.Hd, wl.Hg, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r)
+    outs = []
+    for f in range(wl.T):
+        s = slice(f * wl.N, (f + 1) * wl.N)
+        outs.append(st.step(q[:, :, s].contiguous(), k[:, :, s].contiguous(),
+                            v[:, :, s].contiguous(), a[:, :, s].contiguous(),
+                            b[:, :, s].contiguous(), out=poison_like(q[:, :, s].contiguous())))
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    o = torch.cat(outs, dim=2)
+    assert torch.isfinite(o).all()
+    rows = hi.sample_rows(wl.L, wl.N, 256, seed=42).numpy()
+    o_s, o_d, o_g, S_ref = orc.hybrid_rows(x["q"], x["k"], x["v"], x["a"], x["b"], wl.Hs,
+                                           wl.Hd, wl.Hg, wl.T, wl.N, wl.w_swa, wl.w_dswa, wl.r,
+                                           rows)
+    ridx = torch.from_numpy(rows).cuda()
+    assert maxabs(o[:, :1, ridx], o_s) <= TOL
+    assert maxabs(o[:, 1:2, ridx], o_d) <= TOL
+    assert maxabs(o[:, 2:], o_g) <= TOL
+    assert maxabs(st.state_tensor(), S_ref) <= TOL
+    st.close()
+
+
 @pytest.mark.parametrize("groups", [(3, 1, 4, 2, 4), (1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1), (4, 4, 4, 2)])
 def test_stream_multi_frame_steps_equal_hybrid_bf16(h, orc, groups):
     """Steps appending several frames per rollout at once (ragged group sizes, up to the

@@ -48,6 +48,8 @@ def _rel(got, ref):
     (1, 1, 1, 1.0, "bf16", 2e-2, True),       # one token
     (1, 1, 64, 1.0, "bf16", 2e-2, False),     # one full chunk, zero S0 and dS_final
     (1, 1, 2000, 0.05, "bf16", 2e-2, True),   # 32 chunks: the state passes' rings wrap
+    (1, 1, 8360, 0.05, "bf16", 2e-2, True),   # 131 chunks (ragged tail), slow decay
+    (1, 2, 8320, 1.0, "bf16", 2e-2, True),    # 130 full chunks per head
 ])
 def test_gdn_bwd(h, orc, B, H, L, decay, dtype, tol, states):
     x = _case(B, H, L, decay, dtype, seed=L + 3)
