@@ -220,7 +220,9 @@ hlta_status hlta_gdn_chunk_bwd(const void *q, const void *k, const void *v, cons
                                void *stream);
 
 /*
- * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens.
+ * Workspace size in bytes needed by hlta_gdn_chunk_fwd for B*H heads of L tokens: the chunk
+ * products of every 64-token chunk, and for bf16 heads long enough to be split into
+ * segments (see hlta_gdn_chunk_fwd) each segment's fp32 state map and start state.
  */
 size_t hlta_gdn_workspace_bytes(int B, int H, long L, int d, int chunk, hlta_dtype dt);
 

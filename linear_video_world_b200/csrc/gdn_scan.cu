@@ -1,0 +1,533 @@
+// Gated delta rule, bf16: the pass over the chunks as a two-level scan on the sm_100a tensor
+// cores (tcgen05.mma with tensor-memory accumulators).
+//
+// The chunk preparation (gdn_tc.cu) leaves per 64-token chunk c of a head the bf16 products
+// W, Qt, Kt ([64 t][128 j]), Up^T, Op^T ([128 i][64 t]) and gam = e^{g_n}. Over a chunk with
+// start state S (S[i][j], i value index, j key index) the recurrence is
+//   U = Up - S W^T,   O = Op + S Qt^T,   S_end = gam S + U Kt,
+// i.e. for every row s of S (with up the matching row of Up^T): s_end = s (gam I - W^T Kt) +
+// up Kt. The rows of S evolve independently and the map over a chunk is affine in S. Over a
+// segment of consecutive chunks the composition is affine too, S_end = S_start A_p + B_p, where
+// A_p is what the chain does to the rows of the identity with Up = 0 and B_p what it does to
+// zero rows with Up. That is the "state passing is a composition of multiplicative
+// transitions" of the llm-atlas long-context explainer (sections 06 and 09: chunkwise =
+// parallel within a block, recurrent across blocks); the scan applies it at two levels:
+//   1. segmap  (every segment but the last, A and B parts in separate CTAs, all in parallel):
+//              the chain over the segment's chunks from I (A part) or 0 (B part), no output;
+//   2. compose (serial over segments, rows split over CTAs, fp32 on the CUDA cores):
+//              S_0 = S0, S_{p+1} = S_p A_p + B_p;
+//   3. replay  (every segment in parallel): the chain from S_p with the outputs O, the last
+//              segment also writing the final state.
+// A head whose chunks fit one segment runs only the replay (from S0).
+//
+// The chain kernel (one CTA per segment, 192 threads):
+//   warps 0-3  chain: thread i holds row i of the state (fp32, registers); per chunk it stores
+//              the row as bf16 pairs into tensor memory (the A operand of S [Qt; W]^T), takes
+//              D_W, forms U = Up - D_W as bf16 pairs (the A operand of U Kt), and while U Kt
+//              runs on the tensor pipe writes its outputs O = Op + D_Q (replay); then it takes
+//              U Kt and updates s <- gam s + (U Kt)_i
+//   warp 4     TMA producer: the chunk operands through a two-stage ring
+//   warp 5     tensor-memory owner and MMA issuer (one thread)
+// Tensor memory (512 columns allocated): S bf16 [0, 64), U bf16 [64, 96), D = [D_Q | D_W] at
+// 128 (replay; D_W alone at 192 in the segment maps), U Kt at 256.
+// Every mbarrier wait is bounded (DEVERR_GDN_WAIT); on expiry every role stops, the producer
+// lets its copies land, and the tensor memory is released.
+#include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_ptx.cuh"
+
+namespace hlta {
+namespace {
+
+constexpr int C = 64;                  // chunk length
+constexpr int D = 128;                 // head dim (state is D x D)
+constexpr int NSTG = 2;                // stages of the operand ring
+constexpr int WARP_TMA = 4, WARP_MMA = 5;
+constexpr int THREADS = 192;
+constexpr int ROWS = 128;              // chain threads = state rows
+
+constexpr uint32_t QW_HALF = 128 * 128;    // [128 t-rows: Qt 0-63, W 64-127][64 j] bf16: 16 KB
+constexpr uint32_t W_OFF = 64 * 128;       // W rows start 8 KB into a half
+constexpr uint32_t KT_HALF = 64 * 128;     // [64 t][64 j] bf16: 8 KB
+constexpr uint32_t SLICE = 128 * 128;      // [128 i][64 t] bf16: 16 KB
+
+// tensor-memory columns
+constexpr uint32_t TM_S = 0, TM_U = 64, TM_D = 128, TM_DL = 256, TM_COLS = 512;
+
+enum Mode { SEGMAP_A = 0, SEGMAP_B = 1, REPLAY = 2 };
+
+struct Stage {
+    alignas(1024) uint8_t QW[2 * QW_HALF];   // per key half: Qt rows 0-63 (replay), W rows 64-127
+    alignas(1024) uint8_t Kt[2 * KT_HALF];   // Kt [64 t][128 j] as two 64-column halves
+    alignas(1024) uint8_t Up[SLICE];         // Up^T [128 i][64 t]
+    alignas(1024) uint8_t Op[SLICE];         // Op^T (replay)
+    alignas(16) float gam[4];
+};
+struct ChainSmem {
+    Stage st[NSTG];
+    alignas(8) uint64_t full[NSTG];
+    alignas(8) uint64_t empty[NSTG];       // MMA commit (+ chain threads done with Op, replay)
+    alignas(8) uint64_t s_ready;           // chain threads stored S (count ROWS)
+    alignas(8) uint64_t u_ready;           // chain threads stored U (count ROWS)
+    alignas(8) uint64_t d_full;            // S [Qt; W]^T complete
+    alignas(8) uint64_t dl_full;           // U Kt complete
+    uint32_t tmem_slot;
+    int abort_flag;
+};
+
+struct ChainMaps {
+    CUtensorMap W, Q, K;                   // [BH*nch*64][128]: 64x64 swizzled boxes
+    CUtensorMap U, O;                      // [BH*nch*128][64]: 64 cols x 128 rows, swizzled
+};
+
+struct ChainArgs {
+    GdnArgs g;
+    GdnWorkspace ws;
+    long nch;
+    int seg, nseg;
+    float *Amap, *Bmap, *Sseg;             // [BH][nseg][D][D] fp32 each
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                         unsigned int *err)
+{
+    return ptx::mbar_try(bar, parity) || ptx::mbar_wait(bar, parity, abort_flag, err, DEVERR_GDN_WAIT);
+}
+
+// element (i, t) of a [128 i][64 t] bf16 tile staged by a 128B-swizzled TMA box: 16-byte chunk
+// t/8 of row i sits at chunk (t/8) ^ (i % 8)
+__device__ __forceinline__ const uint4 *slice_chunk(const uint8_t *tile, int i, int c8)
+{
+    return reinterpret_cast<const uint4 *>(tile + i * 128 + ((c8 ^ (i & 7)) << 4));
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    ChainSmem &s = *reinterpret_cast<ChainSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const GdnArgs &p = a.g;
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / p.Hg, h = bh % p.Hg;
+    const long c_begin = (long)seg * a.seg;
+    const long c_end = min(a.nch, c_begin + a.seg);
+    const int nc = (int)(c_end - c_begin);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int *abort_flag = (volatile int *)&s.abort_flag;
+    const uint32_t FULL0 = ptx::smem_u32(&s.full[0]), EMPTY0 = ptx::smem_u32(&s.empty[0]);
+    const uint32_t S_READY = ptx::smem_u32(&s.s_ready), U_READY = ptx::smem_u32(&s.u_ready);
+    const uint32_t D_FULL = ptx::smem_u32(&s.d_full), DL_FULL = ptx::smem_u32(&s.dl_full);
+
+    if (tid == 0) {
+        for (int i = 0; i < NSTG; ++i) {
+            ptx::mbar_init(FULL0 + 8 * i, 1);
+            ptx::mbar_init(EMPTY0 + 8 * i, MODE == REPLAY ? 1 + ROWS : 1);
+        }
+        ptx::mbar_init(S_READY, ROWS);
+        ptx::mbar_init(U_READY, ROWS);
+        ptx::mbar_init(D_FULL, 1);
+        ptx::mbar_init(DL_FULL, 1);
+        s.abort_flag = 0;
+        ptx::mbar_init_fence();
+    }
+    if (warp == WARP_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         ptx::smem_u32(&s.tmem_slot)),
+                     "r"(TM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s.tmem_slot;
+
+    if (warp == WARP_TMA) {
+        // ------------------------------ TMA producer --------------------------------------
+        if (lane == 0) {
+            constexpr uint32_t TX = (MODE == REPLAY ? 2 * QW_HALF : 2 * KT_HALF) + 2 * KT_HALF +
+                                    (MODE == SEGMAP_A ? 0 : SLICE) + (MODE == REPLAY ? SLICE : 0) + 16;
+            int k = 0;
+            for (; k < nc; ++k) {
+                const int st = k % NSTG;
+                if (k >= NSTG && !wait_bar(EMPTY0 + 8 * st, (uint32_t)((k - NSTG) / NSTG) & 1u, abort_flag, p.err)) break;
+                Stage &sg = s.st[st];
+                const uint32_t full = FULL0 + 8 * st;
+                ptx::mbar_expect_tx(full, TX);
+                const long c = c_begin + k;
+                const int row = (int)(((long)bh * a.nch + c) * C);
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (MODE == REPLAY)
+                        ptx::tma_load_2d(ptx::smem_u32(sg.QW + hf * QW_HALF), &maps.Q, hf * 64, row, full);
+                    ptx::tma_load_2d(ptx::smem_u32(sg.QW + hf * QW_HALF + W_OFF), &maps.W, hf * 64, row, full);
+                    ptx::tma_load_2d(ptx::smem_u32(sg.Kt + hf * KT_HALF), &maps.K, hf * 64, row, full);
+                }
+                const int trow = (int)(((long)bh * a.nch + c) * D);
+                if (MODE != SEGMAP_A) ptx::tma_load_2d(ptx::smem_u32(sg.Up), &maps.U, 0, trow, full);
+                if (MODE == REPLAY) ptx::tma_load_2d(ptx::smem_u32(sg.Op), &maps.O, 0, trow, full);
+                ptx::bulk_load(ptx::smem_u32(sg.gam), a.ws.gam + ((long)bh * a.nch + c) * 4, 16, full);
+            }
+            if (*abort_flag) {
+                // a bounded wait expired somewhere: let the copies this CTA issued land
+                const long long t0 = clock64();
+                for (int kk = k - 1; kk >= 0 && kk >= k - NSTG; --kk)
+                    while (!ptx::mbar_try(FULL0 + 8 * (kk % NSTG), (uint32_t)(kk / NSTG) & 1u) &&
+                           clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+    } else if (warp == WARP_MMA) {
+        // ------------------------------ MMA issuer ----------------------------------------
+        if (lane == 0) {
+            // S [Qt; W]^T: A = S (tensor memory), B = the Qt/W rows, K-major (key j along K);
+            // replay N = 128 tokens (Qt then W), segmap N = 64 (W only, into the D_W half)
+            constexpr int N1 = MODE == REPLAY ? 128 : 64;
+            constexpr uint32_t IDESC1 = tc::idesc_bf16(128, N1, false, false);
+            // U Kt: A = U (tensor memory), B = Kt, MN-major (key j along N)
+            constexpr uint32_t IDESC2 = tc::idesc_bf16(128, 128, false, true);
+            bool ok = true;
+            for (int k = 0; k < nc && ok; ++k) {
+                const int st = k % NSTG;
+                Stage &sg = s.st[st];
+                ok = wait_bar(FULL0 + 8 * st, (uint32_t)(k / NSTG) & 1u, abort_flag, p.err) &&
+                     wait_bar(S_READY, (uint32_t)k & 1u, abort_flag, p.err);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint64_t d1 = tc::sw128_desc(ptx::smem_u32(sg.QW) + (MODE == REPLAY ? 0u : W_OFF), 16, 1024);
+                const uint32_t dcol = tmem + TM_D + (MODE == REPLAY ? 0u : 64u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * QW_HALF + (kk & 3) * 32) >> 4;
+                    tc::umma_bf16_ts(dcol, tmem + TM_S + kk * 8, d1 + off, IDESC1, kk > 0 ? 1u : 0u);
+                }
+                tc::umma_commit(D_FULL);
+                if (!(ok = wait_bar(U_READY, (uint32_t)k & 1u, abort_flag, p.err))) break;
+                tc::fence_after_sync();
+                const uint64_t d2 = tc::sw128_desc(ptx::smem_u32(sg.Kt), KT_HALF, 1024);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::umma_bf16_ts(tmem + TM_DL, tmem + TM_U + kk * 8, d2 + (uint64_t)((kk * 2048) >> 4),
+                                     IDESC2, kk > 0 ? 1u : 0u);
+                tc::umma_commit(DL_FULL);
+                tc::umma_commit(EMPTY0 + 8 * st);
+            }
+        }
+    } else if (warp < 4) {
+        // ------------------------------ chain (state rows) --------------------------------
+        const int i = warp * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        __nv_bfloat16 *o = MODE == REPLAY ? (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D + i : nullptr;
+        float sr[D];
+        if (MODE == SEGMAP_A) {
+#pragma unroll
+            for (int j = 0; j < D; ++j) sr[j] = j == i ? 1.f : 0.f;
+        } else if (MODE == SEGMAP_B) {
+#pragma unroll
+            for (int j = 0; j < D; ++j) sr[j] = 0.f;
+        } else {
+            // segment 0 starts from S0 (or zero) when it is the only one; otherwise every
+            // segment starts from its composed start state
+            const float *src = a.nseg > 1 ? a.Sseg + (((long)bh * a.nseg + seg) * D + i) * D
+                                          : (p.S0 ? p.S0 + ((long)bh * D + i) * D : nullptr);
+            if (src) {
+                const float4 *s4 = reinterpret_cast<const float4 *>(src);
+#pragma unroll
+                for (int j4 = 0; j4 < D / 4; ++j4) {
+                    const float4 v = s4[j4];
+                    sr[4 * j4] = v.x; sr[4 * j4 + 1] = v.y; sr[4 * j4 + 2] = v.z; sr[4 * j4 + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < D; ++j) sr[j] = 0.f;
+            }
+        }
+        bool ok = true;
+        for (int k = 0; k < nc; ++k) {
+            const int st = k % NSTG;
+            const Stage &sg = s.st[st];
+            // the state row as bf16 pairs: A operand of S [Qt; W]^T
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int m = 0; m < 32; ++m) pk[m] = tc::pack_bf16(sr[hf * 64 + 2 * m], sr[hf * 64 + 2 * m + 1]);
+                tc::tmem_st32(tl + TM_S + hf * 32, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            ptx::mbar_arrive(S_READY);
+            // U = Up - S W^T, as bf16 pairs: A operand of U Kt (the stage's gam is read here
+            // too: the stage may be refilled as soon as U is handed over)
+            if (!__all_sync(0xffffffffu, wait_bar(D_FULL, (uint32_t)k & 1u, abort_flag, p.err) &&
+                                             wait_bar(FULL0 + 8 * st, (uint32_t)(k / NSTG) & 1u, abort_flag, p.err))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const float gam = sg.gam[0];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t dw[32];
+                tc::tmem_ld32(tl + TM_D + 64 + hf * 32, dw);
+                uint32_t pk[16];
+                if (MODE == SEGMAP_A) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        pk[m] = tc::pack_bf16(-__uint_as_float(dw[2 * m]), -__uint_as_float(dw[2 * m + 1]));
+                } else {
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const uint4 u = *slice_chunk(sg.Up, i, hf * 4 + c4);
+                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
+                            const int m = c4 * 4 + e;
+                            pk[m] = tc::pack_bf16(f.x - __uint_as_float(dw[2 * m]), f.y - __uint_as_float(dw[2 * m + 1]));
+                        }
+                    }
+                }
+                tc::tmem_st16(tl + TM_U + hf * 16, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            ptx::mbar_arrive(U_READY);
+            if (MODE == REPLAY) {
+                // while U Kt runs: O = Op + S Qt^T of this chunk, row i of every token
+                const long t0 = (c_begin + k) * C;
+                const int n = (int)min((long)C, p.L - t0);
+                __nv_bfloat16 *orow = o + t0 * D;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t dq[32];
+                    tc::tmem_ld32(tl + TM_D + hf * 32, dq);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const uint4 u = *slice_chunk(sg.Op, i, hf * 4 + c4);
+                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
+                            const int t = hf * 32 + c4 * 8 + 2 * e;
+                            if (t < n) orow[(long)t * D] = __float2bfloat16_rn(f.x + __uint_as_float(dq[c4 * 8 + 2 * e]));
+                            if (t + 1 < n) orow[(long)(t + 1) * D] = __float2bfloat16_rn(f.y + __uint_as_float(dq[c4 * 8 + 2 * e + 1]));
+                        }
+                    }
+                }
+                // Op of this stage is read (the MMA commit releases the rest of it)
+                ptx::mbar_arrive(EMPTY0 + 8 * st);
+            }
+            // s <- gam s + (U Kt)_i
+            if (!__all_sync(0xffffffffu, wait_bar(DL_FULL, (uint32_t)k & 1u, abort_flag, p.err))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t dl[32];
+                tc::tmem_ld32(tl + TM_DL + q * 32, dl);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sr[q * 32 + j] = fmaf(gam, sr[q * 32 + j], __uint_as_float(dl[j]));
+            }
+        }
+        if (ok) {
+            float *dst = nullptr;
+            if (MODE == SEGMAP_A) dst = a.Amap + (((long)bh * a.nseg + seg) * D + i) * D;
+            else if (MODE == SEGMAP_B) dst = a.Bmap + (((long)bh * a.nseg + seg) * D + i) * D;
+            else if (seg == a.nseg - 1 && p.S_out) dst = p.S_out + ((long)bh * D + i) * D;
+            if (dst) {
+                float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+                for (int j4 = 0; j4 < D / 4; ++j4)
+                    d4[j4] = make_float4(sr[4 * j4], sr[4 * j4 + 1], sr[4 * j4 + 2], sr[4 * j4 + 3]);
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS)
+                     : "memory");
+    }
+}
+
+// -----------------------------------------------------------------------------------------
+// compose: S_0 = S0, S_{p+1} = S_p A_p + B_p, fp32 on the CUDA cores. Rows of S are
+// independent: a CTA owns CR rows of one head. Each step's A_p (64 KB) and the CTA's rows of
+// B_p arrive by bulk copy into one of two buffers, the next step's while this one computes;
+// a thread owns one key column j of half the rows, two rows per packed f32x2 FMA.
+// -----------------------------------------------------------------------------------------
+constexpr int CR = 8;
+constexpr int COMPOSE_THREADS = 256;
+struct ComposeSmem {
+    float A[2][D * D];
+    float Bm[2][CR * D];
+    alignas(16) float srow[D][CR];         // S_p rows of this CTA, transposed ([k][r])
+    alignas(8) uint64_t bar[2];
+    int abort_flag;
+};
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__global__ void __launch_bounds__(COMPOSE_THREADS, 1)
+gdn_compose(const ChainArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    ComposeSmem &s = *reinterpret_cast<ComposeSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    const GdnArgs &p = a.g;
+    const int bh = blockIdx.y, r0 = blockIdx.x * CR;
+    const int tid = threadIdx.x, j = tid & (D - 1), rh = tid >> 7;   // rows r0 + 4 rh .. + 3
+    volatile int *abort_flag = (volatile int *)&s.abort_flag;
+    const uint32_t bar0 = ptx::smem_u32(&s.bar[0]);
+    constexpr uint32_t TX = D * D * 4 + CR * D * 4;
+    auto issue = [&](int sp) {             // one thread: A_sp and this CTA's rows of B_sp
+        const uint32_t bar = bar0 + 8 * (sp & 1);
+        ptx::mbar_expect_tx(bar, TX);
+        ptx::bulk_load(ptx::smem_u32(s.A[sp & 1]), a.Amap + ((long)bh * a.nseg + sp) * D * D, D * D * 4, bar);
+        ptx::bulk_load(ptx::smem_u32(s.Bm[sp & 1]), a.Bmap + (((long)bh * a.nseg + sp) * D + r0) * D, CR * D * 4, bar);
+    };
+    if (tid == 0) {
+        ptx::mbar_init(bar0, 1);
+        ptx::mbar_init(bar0 + 8, 1);
+        s.abort_flag = 0;
+        ptx::mbar_init_fence();
+        issue(0);                          // the launch has nseg > 1
+    }
+    float cur[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = r0 + 4 * rh + r;
+        cur[r] = p.S0 ? p.S0[((long)bh * D + row) * D + j] : 0.f;
+        a.Sseg[(((long)bh * a.nseg) * D + row) * D + j] = cur[r];
+    }
+    int issued = 1;
+    bool ok = true;
+    for (int sp = 0; sp + 1 < a.nseg; ++sp) {
+        // buffer (sp + 1) & 1 was last read in step sp - 1, which every thread has finished
+        if (tid == 0 && sp + 1 < a.nseg - 1) {
+            issue(sp + 1);
+            issued = sp + 2;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) s.srow[j][4 * rh + r] = cur[r];
+        __syncthreads();
+        ok = ptx::mbar_try(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u) ||
+             ptx::mbar_wait(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u, abort_flag, p.err, DEVERR_GDN_WAIT);
+        if (!__syncthreads_and(ok)) break;
+        const float *A = s.A[sp & 1];
+        float2 acc01 = make_float2(s.Bm[sp & 1][(4 * rh) * D + j], s.Bm[sp & 1][(4 * rh + 1) * D + j]);
+        float2 acc23 = make_float2(s.Bm[sp & 1][(4 * rh + 2) * D + j], s.Bm[sp & 1][(4 * rh + 3) * D + j]);
+#pragma unroll 16
+        for (int k = 0; k < D; ++k) {
+            const float av = A[k * D + j];
+            const float4 sk = *reinterpret_cast<const float4 *>(&s.srow[k][4 * rh]);
+            acc01 = ffma2(make_float2(sk.x, sk.y), make_float2(av, av), acc01);
+            acc23 = ffma2(make_float2(sk.z, sk.w), make_float2(av, av), acc23);
+        }
+        cur[0] = acc01.x; cur[1] = acc01.y; cur[2] = acc23.x; cur[3] = acc23.y;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            a.Sseg[(((long)bh * a.nseg + sp + 1) * D + r0 + 4 * rh + r) * D + j] = cur[r];
+        __syncthreads();                   // srow and this buffer are free again
+    }
+    if (!ok && tid == 0) {
+        // a bounded wait expired: let the copies in flight land before the CTA exits
+        const long long t0 = clock64();
+        for (int sp = issued - 1; sp >= 0 && sp >= issued - 2; --sp)
+            while (!ptx::mbar_try(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u) && clock64() - t0 < (1LL << 31)) {}
+    }
+}
+static_assert(COMPOSE_THREADS == 2 * D && CR == 8, "a compose thread owns one key column of four rows");
+
+}  // namespace
+
+int gdn_scan_segment_len(long BH, long nch)
+{
+    // about 128 replay CTAs in all (one per SM, the rest of the GPU left to the softmax
+    // branches running beside), never segments shorter than 32 chunks: below that the
+    // segment maps and their composition cost more than the shorter chain saves
+    const long per_head = BH >= 128 ? 1 : 128 / BH;
+    const long seg = (nch + per_head - 1) / per_head;
+    return (int)(seg < 32 ? 32 : seg);
+}
+
+int gdn_scan_segments_beside(long BH, long nch, double attn_flop)
+{
+    // Estimates from measurements on the B200 at 480P: the softmax launches run at about
+    // 6e8 FLOP per microsecond; one chunk step of the chain takes about 1.5 us when the
+    // chains of few heads run side by side. The chain is cut into as few segments as keep it
+    // within 70 % of the softmax time (each segment adds a map pass and a composition step).
+    const long seg_lat = gdn_scan_segment_len(BH, nch);
+    const long max_seg = (nch + seg_lat - 1) / seg_lat;
+    const double attn_us = attn_flop / 6.0e8, chunk_us = 1.5;
+    long nseg = 1;
+    while (nseg < max_seg && chunk_us * (double)((nch + nseg - 1) / nseg) > 0.7 * attn_us) ++nseg;
+    return (int)nseg;
+}
+
+size_t gdn_scan_bytes(long BH, long nch)
+{
+    const long seg = gdn_scan_segment_len(BH, nch);
+    const long nseg = (nch + seg - 1) / seg;
+    if (nseg <= 1) return 0;
+    return (size_t)3 * BH * nseg * D * D * sizeof(float);
+}
+
+cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWorkspace &ws, float *scan_ws, cudaStream_t s)
+{
+    const long nch = gdn_num_chunks(g.L, C);
+    const long BH = (long)g.B * g.Hg;
+    const long ws_rows = BH * nch * C;
+    ChainArgs a;
+    a.g = g;
+    a.ws = ws;
+    a.nch = nch;
+    a.seg = gdn_scan_segment_len(BH, nch);
+    a.nseg = (int)((nch + a.seg - 1) / a.seg);
+    if (g.scan_segments > 0 && g.scan_segments < a.nseg) {
+        // fewer, longer segments than the latency-oriented split (the workspace holds more)
+        a.seg = (int)((nch + g.scan_segments - 1) / g.scan_segments);
+        a.nseg = (int)((nch + a.seg - 1) / a.seg);
+    }
+    a.Amap = scan_ws;
+    a.Bmap = scan_ws ? scan_ws + BH * a.nseg * D * D : nullptr;
+    a.Sseg = scan_ws ? scan_ws + 2 * BH * a.nseg * D * D : nullptr;
+    if (a.nseg > 1 && !scan_ws) return cudaErrorInvalidValue;
+    if (BH > 65535) return cudaErrorNotSupported;
+    cudaError_t e;
+    ChainMaps m;
+    if ((e = make_tmap_2d_bf16(&m.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.U, ws.Up, ws_rows * 2, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.O, ws.Op, ws_rows * 2, C, 64, D, true)) != cudaSuccess) return e;
+    const size_t smem = sizeof(ChainSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_A>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<REPLAY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    const size_t csmem = sizeof(ComposeSmem) + 128;
+    if ((e = cudaFuncSetAttribute(gdn_compose, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem)) != cudaSuccess) return e;
+    if (a.nseg > 1) {
+        // the maps of every segment but the last, then their composition
+        const dim3 gm((unsigned)(a.nseg - 1), (unsigned)BH);
+        gdn_chain_bf16<SEGMAP_A><<<gm, THREADS, smem, s>>>(m, a), note_launch();
+        gdn_chain_bf16<SEGMAP_B><<<gm, THREADS, smem, s>>>(m, a), note_launch();
+        gdn_compose<<<dim3(D / CR, (unsigned)BH), COMPOSE_THREADS, csmem, s>>>(a), note_launch();
+    }
+    gdn_chain_bf16<REPLAY><<<dim3((unsigned)a.nseg, (unsigned)BH), THREADS, smem, s>>>(m, a), note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace hlta

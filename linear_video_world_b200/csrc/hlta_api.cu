@@ -195,7 +195,8 @@ size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
     const size_t el = bf16 ? 2 : 4;
     const size_t nch = (size_t)gdn_num_chunks(L, C);
     const size_t arr = ((size_t)BH * nch * C * d * el + 255) & ~(size_t)255;
-    return 5 * arr + (((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255);
+    const size_t gam = ((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255;
+    return 5 * arr + gam + (bf16 && d == 128 ? gdn_scan_bytes(BH, (long)nch) : 0);
 }
 
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16)
@@ -207,6 +208,8 @@ GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool
     GdnWorkspace w;
     w.W = p; w.Up = p + arr; w.Op = p + 2 * arr; w.Qt = p + 3 * arr; w.Kt = p + 4 * arr;
     w.gam = (float *)(p + 5 * arr);
+    const size_t gam = ((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255;
+    w.scan = bf16 && d == 128 && gdn_scan_bytes(BH, (long)nch) ? (float *)(p + 5 * arr + gam) : nullptr;
     return w;
 }
 
@@ -566,6 +569,15 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
         g.q = q; g.k = k; g.v = v; g.a = a; g.b = b; g.o = o; g.raw = raw; g.raw_c = raw_c;
         g.B = B; g.Hg = Hg; g.Htot = H; g.h0 = Hs + Hd; g.L = L; g.d = d; g.chunk = chunk;
         g.S0 = S0; g.S_out = S_out; g.ws = workspace; g.ws_bytes = ws_bytes; g.err = ctx->err;
+        // the GDN branch runs beside the softmax branches: its chain needs to end only within
+        // their time, so it takes as few segments (and SMs) as that allows
+        double pairs = 0.0;
+        for (int f = 0; f < T; ++f) {
+            for (int i = 0; i < w_swa && Hs; ++i) pairs += f - i >= 0 ? (double)Hs : 0.0;
+            for (int i = 0; i < w_dswa && Hd; ++i) pairs += f - (long)r * i >= 0 ? (double)Hd : 0.0;
+        }
+        pairs *= (double)B * N * N;
+        g.scan_segments = gdn_scan_segments_beside((long)B * Hg, gdn_num_chunks(L, chunk), 4.0 * d * pairs);
         prof_record(3, ctx->aux);
         st = run_gdn(g, dt, ctx->aux);
         prof_record(4, ctx->aux);

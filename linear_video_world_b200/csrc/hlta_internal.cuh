@@ -59,6 +59,10 @@ struct GdnArgs {
     // S_chunks + (bh * nchunks + c) * S_chunk_stride; with o null the outputs are skipped
     float *S_chunks;
     long S_chunk_stride;
+    // bf16 pass over the chunks: segments per head of the two-level scan (0: as many as keep
+    // the latency low; 1: one serial chain per head on as few SMs as possible, for a branch
+    // that runs beside other work); at most the count the workspace was sized for
+    int scan_segments;
 };
 
 // Chunk workspace (per GDN head, per chunk of C tokens; elements of type E):
@@ -66,10 +70,12 @@ struct GdnArgs {
 //   Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K        each [C][d]
 //   gam = e^{g_C}                               one float per chunk, in a 16-byte slot
 // laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks][4]; the bf16
-// path stores Up and Op of a chunk transposed, [d][C] (state row by token).
+// path stores Up and Op of a chunk transposed, [d][C] (state row by token), and adds the
+// segment scan's fp32 maps and start states (gdn_scan_bytes) at the end.
 struct GdnWorkspace {
     void *W, *Up, *Op, *Qt, *Kt;
     float *gam;
+    float *scan;               // bf16: the segment scan's maps and start states (or null)
 };
 
 __host__ __device__ inline long gdn_num_chunks(long L, int C) { return (L + C - 1) / C; }
@@ -143,6 +149,16 @@ cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const f
                                        cudaStream_t s2, cudaEvent_t mid);
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStreams *side);
 cudaError_t launch_gdn_f32(const GdnArgs &g, cudaStream_t s);
+// The bf16 pass over the chunks as a two-level segment scan (gdn_scan.cu): segment length in
+// chunks, the fp32 scratch it needs after the chunk workspace (0 for a single segment), and
+// the launches (segment maps, their composition, the replay with outputs) after the prep.
+int gdn_scan_segment_len(long BH, long nch);
+// segments per head for a GDN branch running beside softmax work of `attn_flop` (the fewest
+// whose serial chain still ends within that work's estimated time)
+int gdn_scan_segments_beside(long BH, long nch, double attn_flop);
+size_t gdn_scan_bytes(long BH, long nch);
+cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWorkspace &ws, float *scan_ws,
+                                 cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 // f0: the first new frame's index, read from f0_dev when that is set (streaming steps keep
 // their frame counter on the device so that a captured step can be replayed)
