@@ -862,7 +862,7 @@ size_t bwd_f32_bytes(long BH, long L)
 
 size_t gdn_bwd_workspace_bytes(long BH, long L)
 {
-    return bwd_f32_bytes(BH, L) + gdn_workspace_bytes(BH, L, D, C, true);
+    return bwd_f32_bytes(BH, L) + gdn_rowmajor_bytes(BH, L, D, C, true);
 }
 
 cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStreams *side)
@@ -895,7 +895,7 @@ cudaError_t launch_gdn_bwd(const GdnBwdArgs &a, cudaStream_t s, const SideStream
     g.B = a.B; g.Hg = a.H; g.Htot = a.H; g.h0 = 0; g.L = a.L; g.d = D; g.chunk = C;
     g.S0 = a.S0;
     g.ws = (char *)a.ws + bwd_f32_bytes(p.BH, a.L);
-    g.ws_bytes = gdn_workspace_bytes(p.BH, a.L, D, C, true);
+    g.ws_bytes = gdn_rowmajor_bytes(p.BH, a.L, D, C, true);
     g.err = a.err;
     g.S_chunks = p.ws + O_S0;
     g.S_chunk_stride = CHUNK_FLOATS;

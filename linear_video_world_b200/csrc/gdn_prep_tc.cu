@@ -1,0 +1,484 @@
+// Gated delta rule, bf16 forward: the chunk preparation on the sm_100a tensor cores.
+//
+// Per 64-token chunk of a head (one CTA, 128 threads, two CTAs per SM), with g_t the running
+// sum of log a inside the chunk (carried in log2 units) and the chunk algebra of the
+// llm-atlas long-context explainer's chunkwise form (sections 06 and 09) derived from
+// S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T:
+//   A_ti = b_t e^{g_t-g_i} k_t.k_i (i < t),   T = (I + A)^{-1},   P_ti = e^{g_t-g_i} q_t.k_i (i <= t)
+//   W = T diag(b e^g) K,   Up = T diag(b) V,   Op = P Up,   Qt = diag(e^g) Q - P W.
+// Every product runs as tcgen05.mma (bf16 operands, fp32 in tensor memory), and every output
+// is formed transposed, so that a TMEM lane is a row of the state the later pass keeps:
+//   [K; Q] K^T                  (A: K and Q stacked, K-major; B: K)      -> A, P
+//   W^T = K^T T1^T, Up^T = V^T T2^T  (A: K, V as MN-major operands; B: T1 = T diag(b e^g),
+//                                     T2 = T diag(b), K-major)
+//   Op^T = Up^T P^T, (P W)^T = W^T P^T  (A: the staged Up^T, W^T; B: P)
+//   Qt^T = (diag(e^g) Q)^T - (P W)^T
+// T is formed in fp32 on the CUDA cores: 16 x 16 diagonal blocks by forward substitution, then
+// two levels of T10 = -T11 A10 T00. The four [128][64] outputs are staged in shared memory in
+// the 128-byte swizzle and leave by TMA stores. Per chunk a record of fp32 scalars follows:
+// gam = e^{g_n} and ek_t = e^{g_n - g_t} (times 1/|k_t| for raw inputs): the pass over the
+// chunks reads K itself from the input and applies ek to U instead of storing Kt = diag(ek) K.
+#include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_ptx.cuh"
+
+#include <math.h>
+
+namespace hlta {
+namespace {
+
+constexpr int C = 64;                      // chunk length
+constexpr int D = 128;                     // head dim
+constexpr int THREADS = 128;
+constexpr uint32_t KQ_HALF = 128 * 128;    // per 64-column half: K rows 0-63, Q rows 64-127: 16 KB
+constexpr uint32_t Q_OFF = 64 * 128;       // Q rows start 8 KB into a half
+constexpr uint32_t V_HALF = 64 * 128;      // per 64-column half of V: 8 KB
+constexpr uint32_t SQ = 64 * 128;          // a [64][64] bf16 swizzled tile: 8 KB
+constexpr uint32_t SLICE = 128 * 128;      // a [128][64] bf16 swizzled tile: 16 KB
+constexpr int AP = 68;                     // fp32 row stride of A and T
+constexpr uint32_t TM_D1 = 0, TM_WT = 64, TM_UT = 128, TM_OT = 192, TM_PW = 0, TM_COLS = 256;
+
+struct Smem {
+    alignas(1024) uint8_t KQ[2 * KQ_HALF];   // K, Q by TMA; later Op^T staged over the K rows
+    alignas(1024) uint8_t V[2 * V_HALF];     // V by TMA; later Qt^T staged
+    alignas(1024) uint8_t Wt[SLICE];         // W^T staged (also the A operand of (P W)^T)
+    alignas(1024) uint8_t Ut[SLICE];         // Up^T staged (also the A operand of Op^T)
+    alignas(1024) uint8_t P[SQ];             // P [t][t'] bf16
+    alignas(1024) float A[C * AP];           // A, T in place, then T1 and T2 (bf16 tiles) over it
+    float g[C], eg[C], ek[C], bb[C], ks[C];
+    alignas(8) uint64_t bar_ld, bar_mma;
+    uint32_t tmem_slot;
+    int abort_flag;
+};
+static_assert(2 * SQ <= sizeof(float) * C * AP, "T1 and T2 fit over A");
+
+struct Maps {
+    CUtensorMap q, k, v;                   // inputs [B*Htot*L][128]: 64 cols x 64 rows, swizzled
+    CUtensorMap wt, ut, qt;                // outputs [BH*nch*128][64]: 64 cols x 128 rows, swizzled
+    CUtensorMap ot;                        // Op^T in two boxes of 64 rows
+};
+
+__device__ __forceinline__ float fast_lg2(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2-D tiled TMA store from shared memory (bulk-group completion)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     (uint64_t)map),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// byte offset of row r, 16-byte chunk c of a 128B-swizzled tile of 128-byte rows
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// one thread's 64 fp32 values (a row of a [rows][64] tile) as bf16 into row r of a swizzled tile
+__device__ __forceinline__ void store_row_bf16(uint8_t *tile, int r, const float (&x)[64])
+{
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint4 u;
+        u.x = tc::pack_bf16(x[8 * c], x[8 * c + 1]);
+        u.y = tc::pack_bf16(x[8 * c + 2], x[8 * c + 3]);
+        u.z = tc::pack_bf16(x[8 * c + 4], x[8 * c + 5]);
+        u.w = tc::pack_bf16(x[8 * c + 6], x[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + swz(r, c)) = u;
+    }
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Smem &s = *reinterpret_cast<Smem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / p.Hg, h = bh % p.Hg;
+    const long nch = gdn_num_chunks(p.L, C);
+    const long t0 = (long)chunk * C;
+    const int n = (int)min((long)C, p.L - t0);
+    const long head = (long)(b * p.Htot + p.h0 + h) * p.L;
+    const long rec = (long)bh * nch + chunk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    volatile int *abort_flag = (volatile int *)&s.abort_flag;
+    const uint32_t KQ = ptx::smem_u32(s.KQ), V = ptx::smem_u32(s.V);
+    const uint32_t WT = ptx::smem_u32(s.Wt), UT = ptx::smem_u32(s.Ut), PS = ptx::smem_u32(s.P);
+    const uint32_t T1 = ptx::smem_u32(s.A), T2 = T1 + SQ;
+    const uint32_t BLD = ptx::smem_u32(&s.bar_ld), BMMA = ptx::smem_u32(&s.bar_mma);
+    uint8_t *t1p = reinterpret_cast<uint8_t *>(s.A), *t2p = t1p + SQ;
+
+    if (tid == 0) {
+        ptx::mbar_init(BLD, 1);
+        ptx::mbar_init(BMMA, 1);
+        s.abort_flag = 0;
+        ptx::mbar_init_fence();
+        ptx::mbar_expect_tx(BLD, 2 * KQ_HALF + 2 * V_HALF);
+        const int row = (int)(head + t0);
+        for (int hf = 0; hf < 2; ++hf) {
+            ptx::tma_load_2d(KQ + hf * KQ_HALF, &m.k, hf * 64, row, BLD);
+            ptx::tma_load_2d(KQ + hf * KQ_HALF + Q_OFF, &m.q, hf * 64, row, BLD);
+            ptx::tma_load_2d(V + hf * V_HALF, &m.v, hf * 64, row, BLD);
+        }
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         ptx::smem_u32(&s.tmem_slot)),
+                     "r"(TM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 1) {
+        // running sum of log2 a over the chunk (two tokens a lane, then a warp scan) and the
+        // write strengths; with raw inputs the gates are formed here from x, y
+        const int t = 2 * lane;
+        auto lg = [&](int tt) -> float {
+            if (tt >= n) return 0.f;
+            const float v = p.a[(long)bh * p.L + t0 + tt];
+            if (!p.raw) return fast_lg2(v);
+            const float sp = v > 20.f ? v : log1pf(__expf(v));
+            return -p.raw_c * sp * 1.4426950408889634f;
+        };
+        auto beta = [&](int tt) -> float {
+            if (tt >= n) return 0.f;
+            const float v = p.b[(long)bh * p.L + t0 + tt];
+            return p.raw ? 1.f / (1.f + __expf(-v)) : v;
+        };
+        const float l0 = lg(t), l1 = lg(t + 1);
+        const float pair = l0 + l1;
+        float x = pair;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        s.g[t] = x - pair + l0;
+        s.g[t + 1] = x;
+        s.bb[t] = beta(t);
+        s.bb[t + 1] = beta(t + 1);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s.tmem_slot;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    if (tid < C) {
+        const float gn = s.g[n - 1];
+        s.eg[tid] = tid < n ? fast_ex2(s.g[tid]) : 0.f;
+        s.ek[tid] = tid < n ? fast_ex2(gn - s.g[tid]) : 0.f;
+        s.ks[tid] = 1.f;
+    }
+    bool ok = ptx::mbar_try(BLD, 0) || ptx::mbar_wait(BLD, 0, abort_flag, p.err, DEVERR_GDN_WAIT);
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) {                    // let the copies land before the CTA exits
+            const long long tw = clock64();
+            while (!ptx::mbar_try(BLD, 0) && clock64() - tw < (1LL << 31)) {}
+        }
+        goto done;
+    }
+    // a ragged last chunk: rows past it belong to the next head (or lie past the tensor)
+    if (n < C) {
+        for (int e = tid; e < (C - n) * 8; e += THREADS) {
+            const int t = n + (e >> 3), c = e & 7;
+            for (int hf = 0; hf < 2; ++hf) {
+                *reinterpret_cast<uint4 *>(s.KQ + hf * KQ_HALF + swz(t, c)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(s.KQ + hf * KQ_HALF + Q_OFF + swz(t, c)) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(s.V + hf * V_HALF + swz(t, c)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    // raw inputs: q and k of every token scaled to unit L2 norm in the staged tiles (a row of
+    // zeros stays zero); 1/|k_t| is kept for the pass over the chunks, which reads K itself
+    if (p.raw) {
+        __syncthreads();
+        const int t = tid & (C - 1);
+        const uint32_t base = (tid < C ? 0u : Q_OFF);
+        float ss = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(s.KQ + hf * KQ_HALF + base + swz(t, c));
+                const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+            }
+        const float sc = ss > 0.f ? rsqrtf(ss) : 0.f;
+        if (tid < C) s.ks[t] = sc;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 *pu = reinterpret_cast<uint4 *>(s.KQ + hf * KQ_HALF + base + swz(t, c));
+                uint4 u = *pu;
+                __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    h2[e] = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+                }
+                *pu = u;
+            }
+    }
+    fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---- [K; Q] K^T
+    if (tid == 0) {
+        tc::fence_after_sync();
+        constexpr uint32_t ID = tc::idesc_bf16(128, 64, false, false);
+        const uint64_t da = tc::sw128_desc(KQ, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * KQ_HALF + (kk & 3) * 32) >> 4);
+            tc::umma_bf16(tmem + TM_D1, da + off, da + off, ID, kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(BMMA);
+    }
+    ok = ptx::mbar_try(BMMA, 0) || ptx::mbar_wait(BMMA, 0, abort_flag, p.err, DEVERR_GDN_WAIT);
+    if (!__syncthreads_and(ok)) goto done;
+    tc::fence_after_sync();
+    {
+        // lanes 0-63: row t of A (fp32, shared); lanes 64-127: row t of P (bf16 tile)
+        uint32_t dv[64];
+        tc::tmem_ld64(tl + TM_D1, dv);
+        const int t = tid & (C - 1);
+        const float gt = s.g[t];
+        float x[64];
+        if (tid < C) {
+            const float bt = s.bb[t];
+#pragma unroll
+            for (int i = 0; i < C; ++i)
+                x[i] = (i < t && t < n) ? bt * fast_ex2(gt - s.g[i]) * __uint_as_float(dv[i]) : 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < C / 4; ++i4)
+                *reinterpret_cast<float4 *>(s.A + t * AP + 4 * i4) = make_float4(x[4 * i4], x[4 * i4 + 1], x[4 * i4 + 2], x[4 * i4 + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < C; ++i)
+                x[i] = (i <= t && t < n) ? fast_ex2(gt - s.g[i]) * __uint_as_float(dv[i]) : 0.f;
+            store_row_bf16(s.P, t, x);
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^{-1}, fp32, in place over A (unit lower triangular)
+    // level 1: the four 16 x 16 diagonal blocks, a column per thread (forward substitution)
+    if (tid < C) {
+        const int bb0 = (tid >> 4) * 16, jj = tid & 15;
+        float tcv[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < t; ++i) acc = fmaf(s.A[(bb0 + t) * AP + bb0 + i], tcv[i], acc);
+            tcv[t] = t < jj ? 0.f : (t == jj ? 1.f : -acc);
+        }
+        __syncwarp();                      // the block's 16 columns (one warp) read A's block
+#pragma unroll
+        for (int t = 0; t < 16; ++t) s.A[(bb0 + t) * AP + bb0 + jj] = tcv[t];
+    }
+    __syncthreads();
+    // levels 2 and 3: T10 = -T11 (A10 T00) for the 32 x 32 blocks, then for the whole 64 x 64
+#pragma unroll
+    for (int lvl = 0; lvl < 2; ++lvl) {
+        const int bs = lvl == 0 ? 16 : 32;                     // size of T00, T11, A10
+        const int per = bs * bs / (lvl == 0 ? 64 : 128);       // outputs per thread: 4 or 8
+        const int blk = lvl == 0 ? (tid >> 6) : 0;             // which 32 x 32 block (level 2)
+        const int u = lvl == 0 ? (tid & 63) : tid;
+        const int r = u / (bs / per), c0 = (u % (bs / per)) * per;
+        const int o = blk * 32;                                 // block origin
+        float y[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) y[c] = 0.f;
+        for (int k = 0; k < bs; ++k) {                          // Y = A10 T00
+            const float av = s.A[(o + bs + r) * AP + o + k];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < per) y[c] = fmaf(av, s.A[(o + k) * AP + o + c0 + c], y[c]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (c < per) s.A[(o + bs + r) * AP + o + c0 + c] = y[c];
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) y[c] = 0.f;
+        for (int k = 0; k < bs; ++k) {                          // T10 = -T11 Y
+            const float tv = s.A[(o + bs + r) * AP + o + bs + k];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < per) y[c] = fmaf(-tv, s.A[(o + bs + k) * AP + o + c0 + c], y[c]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            if (c < per) s.A[(o + bs + r) * AP + o + c0 + c] = y[c];
+        __syncthreads();
+    }
+    // T1 = T diag(b e^g) (threads 0-63) and T2 = T diag(b) (threads 64-127), bf16 [t][t'] tiles
+    // over A once every row of T has been read
+    {
+        const int t = tid & (C - 1);
+        float x[64];
+#pragma unroll
+        for (int i4 = 0; i4 < C / 4; ++i4) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(s.A + t * AP + 4 * i4);
+            x[4 * i4] = v4.x; x[4 * i4 + 1] = v4.y; x[4 * i4 + 2] = v4.z; x[4 * i4 + 3] = v4.w;
+        }
+        if (tid < C) {
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] *= s.bb[i] * s.eg[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] *= s.bb[i];
+        }
+        __syncthreads();
+        store_row_bf16(tid < C ? t1p : t2p, t, x);
+    }
+    fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---- W^T = K^T T1^T and Up^T = V^T T2^T (K and V read as MN-major operands)
+    if (tid == 0) {
+        tc::fence_after_sync();
+        constexpr uint32_t ID = tc::idesc_bf16(128, 64, true, false);
+        const uint64_t dk = tc::sw128_desc(KQ, KQ_HALF, 1024), dvv = tc::sw128_desc(V, V_HALF, 1024);
+        const uint64_t d1 = tc::sw128_desc(T1, 16, 1024), d2 = tc::sw128_desc(T2, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc::umma_bf16(tmem + TM_WT, dk + (uint64_t)((kk * 2048) >> 4), d1 + (uint64_t)((kk * 32) >> 4), ID, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc::umma_bf16(tmem + TM_UT, dvv + (uint64_t)((kk * 2048) >> 4), d2 + (uint64_t)((kk * 32) >> 4), ID, kk > 0 ? 1u : 0u);
+        tc::umma_commit(BMMA);
+    }
+    ok = ptx::mbar_try(BMMA, 1) || ptx::mbar_wait(BMMA, 1, abort_flag, p.err, DEVERR_GDN_WAIT);
+    if (!__syncthreads_and(ok)) goto done;
+    tc::fence_after_sync();
+    {
+        uint32_t dv[64];
+        float x[64];
+        tc::tmem_ld64(tl + TM_WT, dv);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
+        store_row_bf16(s.Wt, tid, x);
+        tc::tmem_ld64(tl + TM_UT, dv);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
+        store_row_bf16(s.Ut, tid, x);
+    }
+    fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---- W^T and Up^T leave; Op^T = Up^T P^T and (P W)^T = W^T P^T
+    if (tid == 0) {
+        tc::fence_after_sync();
+        tma_store_2d(&m.wt, WT, 0, (int)(rec * D));
+        tma_store_2d(&m.ut, UT, 0, (int)(rec * D));
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        constexpr uint32_t ID = tc::idesc_bf16(128, 64, false, false);
+        const uint64_t du = tc::sw128_desc(UT, 16, 1024), dw = tc::sw128_desc(WT, 16, 1024);
+        const uint64_t dp = tc::sw128_desc(PS, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc::umma_bf16(tmem + TM_OT, du + (uint64_t)((kk * 32) >> 4), dp + (uint64_t)((kk * 32) >> 4), ID, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < C / 16; ++kk)
+            tc::umma_bf16(tmem + TM_PW, dw + (uint64_t)((kk * 32) >> 4), dp + (uint64_t)((kk * 32) >> 4), ID, kk > 0 ? 1u : 0u);
+        tc::umma_commit(BMMA);
+    }
+    ok = ptx::mbar_try(BMMA, 0) || ptx::mbar_wait(BMMA, 0, abort_flag, p.err, DEVERR_GDN_WAIT);
+    if (!__syncthreads_and(ok)) goto done;
+    tc::fence_after_sync();
+    {
+        uint32_t dv[64];
+        float x[64];
+        // Op^T row i over the dead K rows: rows 0-63 in the first half, 64-127 in the second
+        tc::tmem_ld64(tl + TM_OT, dv);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
+        store_row_bf16(s.KQ + (tid >> 6) * KQ_HALF, tid & 63, x);
+        // Qt^T row j = e^g_t Q[t][j] - (P W)^T[j][t], over the dead V tile
+        tc::tmem_ld64(tl + TM_PW, dv);
+        const int j = tid;
+        const uint8_t *qh = s.KQ + (j >> 6) * KQ_HALF + Q_OFF;
+        const int jc = (j & 63) >> 3, je = j & 7;
+#pragma unroll
+        for (int t = 0; t < C; ++t) {
+            const float qv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(qh + swz(t, jc) + 2 * je));
+            x[t] = fmaf(s.eg[t], qv, -__uint_as_float(dv[t]));
+        }
+        store_row_bf16(s.V, tid, x);
+    }
+    fence_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        tma_store_2d(&m.ot, KQ, 0, (int)(rec * D));
+        tma_store_2d(&m.ot, KQ + KQ_HALF, 0, (int)(rec * D + 64));
+        tma_store_2d(&m.qt, V, 0, (int)(rec * D));
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    // the chunk's scalars: gam = e^{g_n} and ek_t (times 1/|k_t| for raw inputs), 0 past n
+    if (tid < C) ws.scal[rec * GDN_SCAL + 4 + tid] = s.ek[tid] * s.ks[tid];
+    else if (tid < C + 4) ws.scal[rec * GDN_SCAL + (tid - C)] = tid == C ? fast_ex2(s.g[n - 1]) : 0.f;
+
+done:
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gdn_bf16_v2(const GdnArgs &g, cudaStream_t s)
+{
+    if (g.d != D) return cudaErrorNotSupported;
+    const long nch = gdn_num_chunks(g.L, C);
+    const long BH = (long)g.B * g.Hg;
+    const long in_rows = (long)g.B * g.Htot * g.L;
+    const long out_rows = BH * nch * D;
+    if (nch > 0x7fffffffL || in_rows + C >= (1L << 31) || out_rows >= (1L << 31) || BH > 65535)
+        return cudaErrorNotSupported;
+    GdnWs2 ws = gdn_ws2_carve(g.ws, BH, g.L);
+    cudaError_t e;
+    Maps m;
+    if ((e = make_tmap_2d_bf16(&m.q, g.q, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.k, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.v, g.v, in_rows, D, 64, C, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.wt, ws.Wt, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.ut, ws.Ut, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.qt, ws.Qt, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.ot, ws.Ot, out_rows, C, 64, 64, true)) != cudaSuccess) return e;
+    const size_t smem = sizeof(Smem) + 1024;
+    if ((e = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    gdn_prep_tc<<<dim3((unsigned)nch, (unsigned)BH), THREADS, smem, s>>>(m, g, ws), note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_gdn_bf16_scan(g, ws, s);
+}
+
+}  // namespace hlta

@@ -1,10 +1,11 @@
 // Gated delta rule, bf16: the pass over the chunks as a two-level scan on the sm_100a tensor
 // cores (tcgen05.mma with tensor-memory accumulators).
 //
-// The chunk preparation (gdn_tc.cu) leaves per 64-token chunk c of a head the bf16 products
-// W, Qt, Kt ([64 t][128 j]), Up^T, Op^T ([128 i][64 t]) and gam = e^{g_n}. Over a chunk with
-// start state S (S[i][j], i value index, j key index) the recurrence is
-//   U = Up - S W^T,   O = Op + S Qt^T,   S_end = gam S + U Kt,
+// The chunk preparation (gdn_prep_tc.cu) leaves per 64-token chunk c of a head the bf16
+// products W^T, Qt^T ([128 j][64 t]), Up^T, Op^T ([128 i][64 t]), gam = e^{g_n} and
+// ek_t = e^{g_n - g_t}; with Kt = diag(ek) K and a chunk start state S (S[i][j], i value
+// index, j key index) the recurrence is
+//   U = Up - S W^T,   O = Op + S Qt^T,   S_end = gam S + U Kt = gam S + (U diag(ek)) K,
 // i.e. for every row s of S (with up the matching row of Up^T): s_end = s (gam I - W^T Kt) +
 // up Kt. The rows of S evolve independently and the map over a chunk is affine in S. Over a
 // segment of consecutive chunks the composition is affine too, S_end = S_start A_p + B_p, where
@@ -22,10 +23,12 @@
 //
 // The chain kernel (one CTA per segment, 192 threads):
 //   warps 0-3  chain: thread i holds row i of the state (fp32, registers); per chunk it stores
-//              the row as bf16 pairs into tensor memory (the A operand of S [Qt; W]^T), takes
-//              D_W, forms U = Up - D_W as bf16 pairs (the A operand of U Kt), and while U Kt
-//              runs on the tensor pipe writes its outputs O = Op + D_Q (replay); then it takes
-//              U Kt and updates s <- gam s + (U Kt)_i
+//              the row as bf16 pairs into tensor memory (the A operand of S [Qt; W]^T, whose
+//              B operand is [Qt^T | W^T] read MN-major), takes D_W, forms U diag(ek) =
+//              (Up - D_W) diag(ek) as bf16 pairs (the A operand of the product with K, read
+//              from the input, MN-major), and while that runs on the tensor pipe writes its
+//              outputs O = Op + D_Q (replay); then it takes U Kt and updates
+//              s <- gam s + (U Kt)_i
 //   warp 4     TMA producer: the chunk operands through a two-stage ring
 //   warp 5     tensor-memory owner and MMA issuer (one thread)
 // Tensor memory (512 columns allocated): S bf16 [0, 64), U bf16 [64, 96), D = [D_Q | D_W] at
@@ -46,10 +49,9 @@ constexpr int WARP_TMA = 4, WARP_MMA = 5;
 constexpr int THREADS = 192;
 constexpr int ROWS = 128;              // chain threads = state rows
 
-constexpr uint32_t QW_HALF = 128 * 128;    // [128 t-rows: Qt 0-63, W 64-127][64 j] bf16: 16 KB
-constexpr uint32_t W_OFF = 64 * 128;       // W rows start 8 KB into a half
+constexpr uint32_t SLICE = 128 * 128;      // [128 rows][64 t] bf16: 16 KB
+constexpr uint32_t W_OFF = SLICE;          // W^T follows Qt^T in the stage
 constexpr uint32_t KT_HALF = 64 * 128;     // [64 t][64 j] bf16: 8 KB
-constexpr uint32_t SLICE = 128 * 128;      // [128 i][64 t] bf16: 16 KB
 
 // tensor-memory columns
 constexpr uint32_t TM_S = 0, TM_U = 64, TM_D = 128, TM_DL = 256, TM_COLS = 512;
@@ -57,11 +59,11 @@ constexpr uint32_t TM_S = 0, TM_U = 64, TM_D = 128, TM_DL = 256, TM_COLS = 512;
 enum Mode { SEGMAP_A = 0, SEGMAP_B = 1, REPLAY = 2 };
 
 struct Stage {
-    alignas(1024) uint8_t QW[2 * QW_HALF];   // per key half: Qt rows 0-63 (replay), W rows 64-127
-    alignas(1024) uint8_t Kt[2 * KT_HALF];   // Kt [64 t][128 j] as two 64-column halves
+    alignas(1024) uint8_t QW[2 * SLICE];     // Qt^T (replay) then W^T, each [128 j][64 t]
+    alignas(1024) uint8_t Kt[2 * KT_HALF];   // K [64 t][128 j] (the input) as two 64-column halves
     alignas(1024) uint8_t Up[SLICE];         // Up^T [128 i][64 t]
     alignas(1024) uint8_t Op[SLICE];         // Op^T (replay)
-    alignas(16) float gam[4];
+    alignas(16) float scal[GDN_SCAL];        // gam, then ek_t at 4 + t
 };
 struct ChainSmem {
     Stage st[NSTG];
@@ -76,13 +78,13 @@ struct ChainSmem {
 };
 
 struct ChainMaps {
-    CUtensorMap W, Q, K;                   // [BH*nch*64][128]: 64x64 swizzled boxes
-    CUtensorMap U, O;                      // [BH*nch*128][64]: 64 cols x 128 rows, swizzled
+    CUtensorMap W, Q, U, O;                // [BH*nch*128][64]: 64 cols x 128 rows, swizzled
+    CUtensorMap K;                         // the input k [B*Htot*L][128]: 64x64 swizzled boxes
 };
 
 struct ChainArgs {
     GdnArgs g;
-    GdnWorkspace ws;
+    GdnWs2 ws;
     long nch;
     int seg, nseg;
     float *Amap, *Bmap, *Sseg;             // [BH][nseg][D][D] fp32 each
@@ -146,8 +148,10 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     if (warp == WARP_TMA) {
         // ------------------------------ TMA producer --------------------------------------
         if (lane == 0) {
-            constexpr uint32_t TX = (MODE == REPLAY ? 2 * QW_HALF : 2 * KT_HALF) + 2 * KT_HALF +
-                                    (MODE == SEGMAP_A ? 0 : SLICE) + (MODE == REPLAY ? SLICE : 0) + 16;
+            constexpr uint32_t TX = (MODE == REPLAY ? 2 * SLICE : SLICE) + 2 * KT_HALF +
+                                    (MODE == SEGMAP_A ? 0 : SLICE) + (MODE == REPLAY ? SLICE : 0) +
+                                    GDN_SCAL * 4;
+            const long krow0 = (long)(b * p.Htot + p.h0 + h) * p.L;
             int k = 0;
             for (; k < nc; ++k) {
                 const int st = k % NSTG;
@@ -156,17 +160,18 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                 const uint32_t full = FULL0 + 8 * st;
                 ptx::mbar_expect_tx(full, TX);
                 const long c = c_begin + k;
-                const int row = (int)(((long)bh * a.nch + c) * C);
-                for (int hf = 0; hf < 2; ++hf) {
-                    if (MODE == REPLAY)
-                        ptx::tma_load_2d(ptx::smem_u32(sg.QW + hf * QW_HALF), &maps.Q, hf * 64, row, full);
-                    ptx::tma_load_2d(ptx::smem_u32(sg.QW + hf * QW_HALF + W_OFF), &maps.W, hf * 64, row, full);
-                    ptx::tma_load_2d(ptx::smem_u32(sg.Kt + hf * KT_HALF), &maps.K, hf * 64, row, full);
-                }
                 const int trow = (int)(((long)bh * a.nch + c) * D);
+                if (MODE == REPLAY) ptx::tma_load_2d(ptx::smem_u32(sg.QW), &maps.Q, 0, trow, full);
+                ptx::tma_load_2d(ptx::smem_u32(sg.QW + W_OFF), &maps.W, 0, trow, full);
+                // K rows past a ragged last chunk belong to the next head (or are zero-filled
+                // past the tensor): U diag(ek) is zero there, so they add nothing
+                const int krow = (int)(krow0 + c * C);
+                for (int hf = 0; hf < 2; ++hf)
+                    ptx::tma_load_2d(ptx::smem_u32(sg.Kt + hf * KT_HALF), &maps.K, hf * 64, krow, full);
                 if (MODE != SEGMAP_A) ptx::tma_load_2d(ptx::smem_u32(sg.Up), &maps.U, 0, trow, full);
                 if (MODE == REPLAY) ptx::tma_load_2d(ptx::smem_u32(sg.Op), &maps.O, 0, trow, full);
-                ptx::bulk_load(ptx::smem_u32(sg.gam), a.ws.gam + ((long)bh * a.nch + c) * 4, 16, full);
+                ptx::bulk_load(ptx::smem_u32(sg.scal), a.ws.scal + ((long)bh * a.nch + c) * GDN_SCAL,
+                               GDN_SCAL * 4, full);
             }
             if (*abort_flag) {
                 // a bounded wait expired somewhere: let the copies this CTA issued land
@@ -179,10 +184,10 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     } else if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ----------------------------------------
         if (lane == 0) {
-            // S [Qt; W]^T: A = S (tensor memory), B = the Qt/W rows, K-major (key j along K);
+            // S [Qt; W]^T: A = S (tensor memory), B = [Qt^T | W^T], MN-major (token t along N);
             // replay N = 128 tokens (Qt then W), segmap N = 64 (W only, into the D_W half)
             constexpr int N1 = MODE == REPLAY ? 128 : 64;
-            constexpr uint32_t IDESC1 = tc::idesc_bf16(128, N1, false, false);
+            constexpr uint32_t IDESC1 = tc::idesc_bf16(128, N1, false, true);
             // U Kt: A = U (tensor memory), B = Kt, MN-major (key j along N)
             constexpr uint32_t IDESC2 = tc::idesc_bf16(128, 128, false, true);
             bool ok = true;
@@ -193,13 +198,11 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                      wait_bar(S_READY, (uint32_t)k & 1u, abort_flag, p.err);
                 if (!ok) break;
                 tc::fence_after_sync();
-                const uint64_t d1 = tc::sw128_desc(ptx::smem_u32(sg.QW) + (MODE == REPLAY ? 0u : W_OFF), 16, 1024);
+                const uint64_t d1 = tc::sw128_desc(ptx::smem_u32(sg.QW) + (MODE == REPLAY ? 0u : W_OFF), SLICE, 1024);
                 const uint32_t dcol = tmem + TM_D + (MODE == REPLAY ? 0u : 64u);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * QW_HALF + (kk & 3) * 32) >> 4;
-                    tc::umma_bf16_ts(dcol, tmem + TM_S + kk * 8, d1 + off, IDESC1, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::umma_bf16_ts(dcol, tmem + TM_S + kk * 8, d1 + (uint64_t)((kk * 2048) >> 4), IDESC1, kk > 0 ? 1u : 0u);
                 tc::umma_commit(D_FULL);
                 if (!(ok = wait_bar(U_READY, (uint32_t)k & 1u, abort_flag, p.err))) break;
                 tc::fence_after_sync();
@@ -264,16 +267,23 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                 break;
             }
             tc::fence_after_sync();
-            const float gam = sg.gam[0];
+            const float gam = sg.scal[0];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 uint32_t dw[32];
                 tc::tmem_ld32(tl + TM_D + 64 + hf * 32, dw);
+                float ek[32];
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 e4 = *reinterpret_cast<const float4 *>(&sg.scal[4 + hf * 32 + 4 * q4]);
+                    ek[4 * q4] = e4.x; ek[4 * q4 + 1] = e4.y; ek[4 * q4 + 2] = e4.z; ek[4 * q4 + 3] = e4.w;
+                }
                 uint32_t pk[16];
                 if (MODE == SEGMAP_A) {
 #pragma unroll
                     for (int m = 0; m < 16; ++m)
-                        pk[m] = tc::pack_bf16(-__uint_as_float(dw[2 * m]), -__uint_as_float(dw[2 * m + 1]));
+                        pk[m] = tc::pack_bf16(-ek[2 * m] * __uint_as_float(dw[2 * m]),
+                                              -ek[2 * m + 1] * __uint_as_float(dw[2 * m + 1]));
                 } else {
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
@@ -283,7 +293,8 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                         for (int e = 0; e < 4; ++e) {
                             const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
                             const int m = c4 * 4 + e;
-                            pk[m] = tc::pack_bf16(f.x - __uint_as_float(dw[2 * m]), f.y - __uint_as_float(dw[2 * m + 1]));
+                            pk[m] = tc::pack_bf16(ek[2 * m] * (f.x - __uint_as_float(dw[2 * m])),
+                                                  ek[2 * m + 1] * (f.y - __uint_as_float(dw[2 * m + 1])));
                         }
                     }
                 }
@@ -485,11 +496,13 @@ size_t gdn_scan_bytes(long BH, long nch)
     return (size_t)3 * BH * nseg * D * D * sizeof(float);
 }
 
-cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWorkspace &ws, float *scan_ws, cudaStream_t s)
+cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWs2 &ws, cudaStream_t s)
 {
     const long nch = gdn_num_chunks(g.L, C);
     const long BH = (long)g.B * g.Hg;
-    const long ws_rows = BH * nch * C;
+    const long out_rows = BH * nch * D;
+    const long in_rows = (long)g.B * g.Htot * g.L;
+    float *scan_ws = ws.scan;
     ChainArgs a;
     a.g = g;
     a.ws = ws;
@@ -508,11 +521,11 @@ cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWorkspace &ws, float
     if (BH > 65535) return cudaErrorNotSupported;
     cudaError_t e;
     ChainMaps m;
-    if ((e = make_tmap_2d_bf16(&m.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&m.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&m.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&m.U, ws.Up, ws_rows * 2, C, 64, D, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&m.O, ws.Op, ws_rows * 2, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.W, ws.Wt, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.Q, ws.Qt, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.U, ws.Ut, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.O, ws.Ot, out_rows, C, 64, D, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&m.K, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
     const size_t smem = sizeof(ChainSmem) + 1024;
     if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_A>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;

@@ -978,9 +978,8 @@ cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
     if (e != cudaSuccess) return e;
     gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    (void)sm;
-    (void)smem_state;
-    return launch_gdn_bf16_scan(g, ws, ws.scan, s);
+    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws), note_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,

@@ -129,7 +129,7 @@ hlta_status run_attn(const AttnArgs &a, hlta_dtype dt, cudaStream_t s)
 hlta_status run_gdn(const GdnArgs &g, hlta_dtype dt, cudaStream_t s)
 {
     if (g.B * g.Hg == 0) return HLTA_OK;
-    cudaError_t e = dt == HLTA_FP32 ? launch_gdn_f32(g, s) : launch_gdn_bf16(g, s);
+    cudaError_t e = dt == HLTA_FP32 ? launch_gdn_f32(g, s) : launch_gdn_bf16_v2(g, s);
     if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "gated delta rule: unsupported shape");
     if (e != cudaSuccess) return cuda_fail(e, "gated delta rule launch");
     return HLTA_OK;
@@ -190,13 +190,34 @@ hlta_status check_raw_c(float c)
 
 }  // namespace
 
-size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
+size_t gdn_rowmajor_bytes(long BH, long L, int d, int C, bool bf16)
 {
     const size_t el = bf16 ? 2 : 4;
     const size_t nch = (size_t)gdn_num_chunks(L, C);
     const size_t arr = ((size_t)BH * nch * C * d * el + 255) & ~(size_t)255;
-    const size_t gam = ((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255;
-    return 5 * arr + gam + (bf16 && d == 128 ? gdn_scan_bytes(BH, (long)nch) : 0);
+    return 5 * arr + (((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255);
+}
+
+namespace {
+size_t ws2_arr(long BH, long L) { return ((size_t)BH * gdn_num_chunks(L, 64) * 128 * 64 * 2 + 255) & ~(size_t)255; }
+size_t ws2_scal(long BH, long L) { return ((size_t)BH * gdn_num_chunks(L, 64) * GDN_SCAL * 4 + 255) & ~(size_t)255; }
+}  // namespace
+
+size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16)
+{
+    if (!bf16 || d != 128 || C != 64) return gdn_rowmajor_bytes(BH, L, d, C, bf16);
+    return 4 * ws2_arr(BH, L) + ws2_scal(BH, L) + gdn_scan_bytes(BH, gdn_num_chunks(L, 64));
+}
+
+GdnWs2 gdn_ws2_carve(void *base, long BH, long L)
+{
+    char *p = (char *)base;
+    const size_t arr = ws2_arr(BH, L), sc = ws2_scal(BH, L);
+    GdnWs2 w;
+    w.Wt = p; w.Qt = p + arr; w.Ut = p + 2 * arr; w.Ot = p + 3 * arr;
+    w.scal = (float *)(p + 4 * arr);
+    w.scan = gdn_scan_bytes(BH, gdn_num_chunks(L, 64)) ? (float *)(p + 4 * arr + sc) : nullptr;
+    return w;
 }
 
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16)
@@ -208,8 +229,6 @@ GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool
     GdnWorkspace w;
     w.W = p; w.Up = p + arr; w.Op = p + 2 * arr; w.Qt = p + 3 * arr; w.Kt = p + 4 * arr;
     w.gam = (float *)(p + 5 * arr);
-    const size_t gam = ((size_t)BH * nch * 4 * sizeof(float) + 255) & ~(size_t)255;
-    w.scan = bf16 && d == 128 && gdn_scan_bytes(BH, (long)nch) ? (float *)(p + 5 * arr + gam) : nullptr;
     return w;
 }
 

@@ -70,17 +70,32 @@ struct GdnArgs {
 //   Qt = diag(e^g) Q - P W, Kt = diag(e^{g_C - g}) K        each [C][d]
 //   gam = e^{g_C}                               one float per chunk, in a 16-byte slot
 // laid out as five arrays [BHg][nchunks][C][d] followed by gam [BHg][nchunks][4]; the bf16
-// path stores Up and Op of a chunk transposed, [d][C] (state row by token), and adds the
-// segment scan's fp32 maps and start states (gdn_scan_bytes) at the end.
+// path stores Up and Op of a chunk transposed, [d][C] (state row by token).
 struct GdnWorkspace {
     void *W, *Up, *Op, *Qt, *Kt;
     float *gam;
-    float *scan;               // bf16: the segment scan's maps and start states (or null)
 };
 
 __host__ __device__ inline long gdn_num_chunks(long L, int C) { return (L + C - 1) / C; }
-size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16);
+// the layout above (the fp32 path, and the bf16 chunk products the backward pass uses)
+size_t gdn_rowmajor_bytes(long BH, long L, int d, int C, bool bf16);
 GdnWorkspace gdn_workspace_carve(void *base, long BH, long L, int d, int C, bool bf16);
+// workspace of hlta_gdn_chunk_fwd: the layout above for fp32, GdnWs2 for bf16
+size_t gdn_workspace_bytes(long BH, long L, int d, int C, bool bf16);
+
+// Chunk workspace of the bf16 forward (d = 128, C = 64), per chunk of a head, every array
+// [BHg * nchunks][128][64] bf16 (state row, or key index, by token):
+//   Wt = W^T, Qt = Qt^T, Ut = Up^T, Ot = Op^T,
+//   scal: GDN_SCAL floats, gam = e^{g_n} at 0, ek_t = e^{g_n - g_t} (times 1/|k_t| for raw
+//         inputs, 0 past the chunk's end) at 4 + t,
+// then the segment scan's fp32 maps and start states (gdn_scan_bytes).
+constexpr int GDN_SCAL = 68;
+struct GdnWs2 {
+    void *Wt, *Qt, *Ut, *Ot;
+    float *scal;
+    float *scan;
+};
+GdnWs2 gdn_ws2_carve(void *base, long BH, long L);
 
 // Records the thread-local message returned by hlta_last_error() and returns `st`.
 int record_error_impl(int st, const char *fmt, ...);
@@ -157,8 +172,9 @@ int gdn_scan_segment_len(long BH, long nch);
 // whose serial chain still ends within that work's estimated time)
 int gdn_scan_segments_beside(long BH, long nch, double attn_flop);
 size_t gdn_scan_bytes(long BH, long nch);
-cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWorkspace &ws, float *scan_ws,
-                                 cudaStream_t s);
+cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWs2 &ws, cudaStream_t s);
+// the bf16 forward: the tensor-core chunk preparation, then the segment scan
+cudaError_t launch_gdn_bf16_v2(const GdnArgs &g, cudaStream_t s);
 cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 // f0: the first new frame's index, read from f0_dev when that is set (streaming steps keep
 // their frame counter on the device so that a captured step can be replayed)

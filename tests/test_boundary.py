@@ -87,15 +87,16 @@ def test_stream_create_ex_validates_frames_per_step(lib):
 
 def test_workspace_sizes(lib):
     import linear_video_world_b200 as h
-    # 5 arrays of chunk-padded [BH][nchunks][64][d] bf16, a 16-byte slot per chunk, and the
-    # segment scan's three fp32 [BH][nseg][d][d] arrays (512 chunks per head: 16 segments)
+    # bf16: 4 arrays of [BH][nchunks][128][64] bf16 (W^T, Qt^T, Up^T, Op^T), 68 fp32 scalars
+    # per chunk, and the segment scan's three fp32 [BH][nseg][d][d] arrays (512 chunks per
+    # head: 16 segments)
     n = h.hlta_gdn_workspace_bytes(1, 8, 32760, 128, 64, h.HLTA_BF16)
     nch = (32760 + 63) // 64
     arr = 8 * nch * 64 * 128 * 2
-    assert n == 5 * arr + ((8 * nch * 16 + 255) // 256) * 256 + 3 * 8 * 16 * 128 * 128 * 4
+    assert n == 4 * arr + ((8 * nch * 68 * 4 + 255) // 256) * 256 + 3 * 8 * 16 * 128 * 128 * 4
     # a head short enough for one segment needs no scan arrays
     n1 = h.hlta_gdn_workspace_bytes(1, 8, 1560, 128, 64, h.HLTA_BF16)
-    assert n1 == 5 * (8 * 25 * 64 * 128 * 2) + ((8 * 25 * 16 + 255) // 256) * 256
+    assert n1 == 4 * (8 * 25 * 64 * 128 * 2) + ((8 * 25 * 68 * 4 + 255) // 256) * 256
     assert h.hlta_hybrid_workspace_bytes(1, 8, 21, 1560, 128, 64, h.HLTA_BF16) == n
     assert h.hlta_gdn_workspace_bytes(1, 1, 10, 64, 64, h.HLTA_FP32) > 5 * 64 * 64 * 4 - 1
 
