@@ -1,0 +1,535 @@
+// Windowed softmax attention (SWA / DSWA / streaming step), bf16, head dim 128, on the sm_100a
+// tensor cores: 128-key tiles, two query sub-tiles per CTA, S decoupled from P.
+//
+// Exact attention by tiles with a running max and normaliser (llm-atlas long-context
+// explainer, section 03 "Flash Attention"); the key set of a query tile is the union of the
+// key frames of its rows' frames (sliding window: frames f-w+1..f; dilated: f, f-r, ...,
+// f-r(w-1); Kairos abstract, item (2)), walked frame by frame in tiles of up to 128 keys (the
+// last tile of a frame holds N mod 128 keys; its products shrink to match), with a
+// per-element mask (row frame vs. key frame, frame end).
+//
+// Why this shape. At d = 128 a (query, key) pair costs 4 d = 512 tensor FLOP and one
+// exponential, and an SM runs 8192 bf16 FLOP and 16 exponentials per cycle, so the softmax
+// of one tile takes as long as its two products; the products of tile t+1 must run while the
+// softmax works on tile t. Here the scores S live in tensor memory and the probabilities P go
+// to shared memory (the A operand of P V), so S of the next tile is issued as soon as the
+// softmax has read this tile's scores into registers, not after P V: per sub-tile the softmax
+// then runs tile after tile with its next scores already computed. 128-key tiles give every S
+// product N = 128, which halves the products one issuing thread sends per key compared with
+// 64-key tiles (one thread issues a tcgen05.mma in roughly a hundred cycles).
+//
+// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 11 warps:
+//   warps 0-3 / 4-7  softmax of sub-tile 0 / 1, one thread per query row (its TMEM lane)
+//   warp 8           TMA producer: Q once, then K and V tiles of 128 keys through one ring of
+//                    three 32 KB slots, in the order K0, K1, V0, K2, V1, ... (the order the
+//                    MMA warps consume them)
+//   warps 9, 10      MMA issuers of sub-tile 0 / 1 (warp 9 owns the TMEM allocation). Each
+//                    walks every tile in the ring's order: for K of a tile its sub-tile needs,
+//                    S = Q K^T once the softmax freed the S buffer; for V, O += P V once P is in
+//                    shared memory; a slot is released by both warps
+// Tensor memory: per sub-tile S (128 columns) and O (128). Shared memory: Q (64 KB), the ring
+// (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
+// O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
+// denominator use the same stale max). Every mbarrier wait is bounded; on expiry the kernel
+// records DEVERR_ATTN_WAIT, every role stops, and the TMEM allocation is released.
+#include "hlta_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_ptx.cuh"
+
+#include <math.h>
+
+namespace hlta {
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;                 // query rows per sub-tile
+constexpr int QT = 2;                   // query sub-tiles per CTA
+constexpr int BN = 128;                 // keys per tile
+constexpr int D = 128;                  // head dim
+constexpr int NSLOT = 3;                // ring slots (K and V tiles in consumption order)
+constexpr int THREADS = 352;            // 8 softmax warps, TMA warp, two MMA warps
+constexpr int WARP_TMA = 8, WARP_MMA = 9;
+constexpr int SOFTMAX_THREADS = 128;    // per sub-tile
+constexpr uint32_t QHALF = BM * 128;    // [128 rows][64 cols] bf16: 16 KB
+constexpr uint32_t QTILE = 2 * QHALF;
+constexpr uint32_t KHALF = BN * 128;    // [128 keys][64 cols] bf16: 16 KB
+constexpr uint32_t KTILE = 2 * KHALF;
+constexpr uint32_t PHALF = BM * 128;    // P: [128 rows][64 keys] bf16: 16 KB
+constexpr uint32_t PTILE = 2 * PHALF;
+constexpr uint32_t TMEM_COLS = 512;     // S_0 @0, S_1 @128, O_0 @256, O_1 @384
+__host__ __device__ constexpr uint32_t TM_S(int q) { return (uint32_t)q * 128u; }
+__host__ __device__ constexpr uint32_t TM_O(int q) { return 256u + (uint32_t)q * 128u; }
+
+__host__ __device__ constexpr uint32_t SM_Q(int q) { return (uint32_t)q * QTILE; }
+__host__ __device__ constexpr uint32_t SM_SLOT(int i) { return QT * QTILE + (uint32_t)i * KTILE; }
+__host__ __device__ constexpr uint32_t SM_P(int q) { return QT * QTILE + NSLOT * KTILE + (uint32_t)q * PTILE; }
+constexpr uint32_t SM_BAR = QT * QTILE + NSLOT * KTILE + QT * PTILE;
+enum {
+    B_QFULL = 0,
+    B_FULL = 1,                  // + slot
+    B_EMPTY = B_FULL + NSLOT,    // + slot: both MMA warps done with it (count 2)
+    B_SFULL = B_EMPTY + NSLOT,   // + sub-tile
+    B_SFREE = B_SFULL + QT,      // + sub-tile: its softmax read S (count SOFTMAX_THREADS)
+    B_PFULL = B_SFREE + QT,      // + sub-tile: P in shared memory (count SOFTMAX_THREADS)
+    B_PVDONE = B_PFULL + QT,     // + sub-tile
+    B_ODONE = B_PVDONE + QT,     // + sub-tile: every product of the sub-tile has completed
+    NBARS = B_ODONE + QT
+};
+constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
+constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
+constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
+constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+
+struct Params {
+    int Hbr, q_Htot, q_h0, kv_Htot, kv_h0, kv_slots;
+    long q_rows, kv_rows;
+    int N, w, r, fq0;
+    const int *fq0_dev;
+    float sl2;                  // softmax scale * log2(e)
+    float *lse;
+    __nv_bfloat16 *o;
+    unsigned int *err;
+};
+
+// packed fp32 pairs (sm_100 f32x2 instructions)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 pa, pb, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+        "add.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// ---------------------------------------------------------------------------------------
+// key-tile walk shared by every role (all roles visit the same sequence)
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ bool frame_needed(int fk, int fa, int fb, int w, int r)
+{
+    const int i0 = fa > fk ? (fa - fk + r - 1) / r : 0;
+    return i0 < w && fk + r * i0 <= fb;
+}
+struct Walk {
+    int fa0, fb0, fa1, fb1, fb, w, r, tpf;
+    bool valid1;
+    __device__ __forceinline__ int mask_of(int fk) const
+    {
+        return (frame_needed(fk, fa0, fb0, w, r) ? 1 : 0) |
+               (valid1 && frame_needed(fk, fa1, fb1, w, r) ? 2 : 0);
+    }
+};
+struct Pos {
+    int fk, jt, mask, j;        // frame, tile in the frame, sub-tile mask, global tile index
+    bool valid;
+};
+__device__ __forceinline__ Pos walk_start(const Walk &wk, int fstart)
+{
+    Pos c;
+    c.fk = fstart - 1;
+    c.jt = wk.tpf - 1;
+    c.mask = 0;
+    c.j = -1;
+    c.valid = true;
+    return c;
+}
+__device__ __forceinline__ bool walk_step(const Walk &wk, Pos &c)
+{
+    ++c.j;
+    if (++c.jt < wk.tpf) return true;
+    for (++c.fk; c.fk <= wk.fb; ++c.fk) {
+        const int m = wk.mask_of(c.fk);
+        if (m) {
+            c.mask = m;
+            c.jt = 0;
+            return true;
+        }
+    }
+    return c.valid = false;
+}
+__device__ __forceinline__ bool walk_next(const Walk &wk, Pos &c, int want)
+{
+    while (walk_step(wk, c)) {
+        if (c.mask & want) return true;
+        c.j += wk.tpf - 1 - c.jt;
+        c.jt = wk.tpf - 1;
+    }
+    return false;
+}
+__device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
+{
+    const int dist = fq - fk;
+    return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + SM_BAR;
+    auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    volatile int *abort_flag = (volatile int *)(smem + SM_ABORT);
+    uint32_t *tmem_slot = (uint32_t *)(smem + SM_TMEMSLOT);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int b = bh / p.Hbr, h = bh % p.Hbr;
+    const long l0 = (long)blockIdx.x * (QT * BM);
+    const long q_head = (long)(b * p.q_Htot + p.q_h0 + h) * p.q_rows;
+    const long kv_head = (long)(b * p.kv_Htot + p.kv_h0 + h) * p.kv_rows;
+    const long r1_0 = min(l0 + BM, p.q_rows) - 1;
+    const int fq0 = p.fq0_dev ? *p.fq0_dev : p.fq0;
+    const int fa0 = fq0 + (int)(l0 / p.N), fb0 = fq0 + (int)(r1_0 / p.N);
+    const bool valid1 = l0 + BM < p.q_rows;
+    const int fa1 = valid1 ? fq0 + (int)((l0 + BM) / p.N) : fa0;
+    const int fb1 = valid1 ? fq0 + (int)((min(l0 + 2 * BM, p.q_rows) - 1) / p.N) : fa1;
+    Walk wk;
+    wk.fa0 = fa0;
+    wk.fb0 = fb0;
+    wk.fa1 = fa1;
+    wk.fb1 = fb1;
+    wk.valid1 = valid1;
+    wk.fb = valid1 ? fb1 : fb0;
+    wk.w = p.w;
+    wk.r = p.r;
+    wk.tpf = (p.N + BN - 1) / BN;
+    const int fstart = max(0, fa0 - p.r * (p.w - 1));
+    auto kv_row = [&](int fk, int jt) {
+        return (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
+    };
+    auto nkeys = [&](int jt) { return min(BN, p.N - jt * BN); };
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QFULL), 1);
+        for (int i = 0; i < NSLOT; ++i) {
+            mbar_init(BAR(B_FULL + i), 1);
+            mbar_init(BAR(B_EMPTY + i), 2);
+        }
+        for (int q = 0; q < QT; ++q) {
+            mbar_init(BAR(B_SFULL + q), 1);
+            mbar_init(BAR(B_SFREE + q), SOFTMAX_THREADS);
+            mbar_init(BAR(B_PFULL + q), SOFTMAX_THREADS);
+            mbar_init(BAR(B_PVDONE + q), 1);
+            mbar_init(BAR(B_ODONE + q), 1);
+        }
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == WARP_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+        return mbar_try(bar, parity) || mbar_wait(bar, parity, abort_flag, p.err, DEVERR_ATTN_WAIT);
+    };
+    // The ring's items in order: K of tile 0, then K of tile j + 1 and V of tile j for j = 0, 1,
+    // ...; item i sits in slot i % NSLOT. K(j) is item 2j - 1 (j >= 1), V(j) is item 2j + 2
+    // (2j + 1 when tile j + 1 does not exist, i.e. for the last tile).
+
+    if (warp == WARP_TMA) {
+        // ------------------------------- TMA producer -----------------------------------
+        if (lane == 0) {
+            mbar_expect_tx(BAR(B_QFULL), QT * QTILE);
+            for (int q = 0; q < QT; ++q) {
+                const int qrow = (int)(q_head + l0 + q * BM);
+                tma_load_2d(sbase + SM_Q(q), &tq, 0, qrow, BAR(B_QFULL));
+                tma_load_2d(sbase + SM_Q(q) + QHALF, &tq, 64, qrow, BAR(B_QFULL));
+            }
+            int it = 0;                                  // ring items issued
+            bool ok = true;
+            auto load = [&](const CUtensorMap *map, int row) -> bool {
+                const int sl = it % NSLOT;
+                if (it >= NSLOT && !wait_bar(BAR(B_EMPTY + sl), (uint32_t)((it / NSLOT) + 1) & 1u)) return false;
+                mbar_expect_tx(BAR(B_FULL + sl), KTILE);
+                tma_load_2d(sbase + SM_SLOT(sl), map, 0, row, BAR(B_FULL + sl));
+                tma_load_2d(sbase + SM_SLOT(sl) + KHALF, map, 64, row, BAR(B_FULL + sl));
+                ++it;
+                return true;
+            };
+            Pos kp = walk_start(wk, fstart), vp = kp;
+            if (walk_step(wk, kp)) ok = load(&tk, kv_row(kp.fk, kp.jt));
+            while (ok && walk_step(wk, vp)) {
+                if (walk_step(wk, kp) && !(ok = load(&tk, kv_row(kp.fk, kp.jt)))) break;
+                if (!(ok = load(&tv, kv_row(vp.fk, vp.jt)))) break;
+            }
+            if (*abort_flag) {
+                const long long t0 = clock64();
+                for (int ii = it - 1; ii >= 0 && ii >= it - NSLOT; --ii)
+                    while (!mbar_try(BAR(B_FULL + ii % NSLOT), (uint32_t)(ii / NSLOT) & 1u) && clock64() - t0 < (1LL << 31)) {}
+                while (!mbar_try(BAR(B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
+            }
+        }
+    } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
+        // ------------------------------- MMA issuers ------------------------------------
+        if (lane == 0) {
+            const int q = warp - WARP_MMA;
+            const int want = 1 << q;
+            constexpr uint32_t IDESC_S0 = tc::idesc_bf16(BM, 16, false, false) & ~(0x3Fu << 17);
+            constexpr uint32_t IDESC_O = tc::idesc_bf16(BM, D, false, true);
+            const uint64_t dq = tc::sw128_desc(sbase + SM_Q(q), 16, 1024);
+            const uint64_t dsl0 = tc::sw128_desc(sbase + SM_SLOT(0), 16, 1024);        // K-major (K)
+            const uint64_t dvl0 = tc::sw128_desc(sbase + SM_SLOT(0), KHALF, 1024);     // MN-major (V)
+            const uint64_t dp = tc::sw128_desc(sbase + SM_P(q), 16, 1024);
+            const uint32_t s_tm = tmem + TM_S(q), o_tm = tmem + TM_O(q);
+            int it = 0, ns = 0, npv = 0;
+            bool ok = wait_bar(BAR(B_QFULL), 0);
+            // K of tile u (ring item `it`): S = Q K^T once this sub-tile's softmax read the
+            // previous S (N = the tile's keys rounded up to 16), then the slot released
+            auto handle_k = [&](const Pos &u) -> bool {
+                const int sl = it % NSLOT;
+                if (!wait_bar(BAR(B_FULL + sl), (uint32_t)(it / NSLOT) & 1u)) return false;
+                if (u.mask & want) {
+                    if (ns > 0 && !wait_bar(BAR(B_SFREE + q), (uint32_t)(ns - 1) & 1u)) return false;
+                    tc::fence_after_sync();
+                    const int n16 = (nkeys(u.jt) + 15) & ~15;
+                    const uint32_t idesc = IDESC_S0 | ((uint32_t)(n16 >> 3) << 17);
+                    const uint64_t dk = dsl0 + (uint64_t)((sl * KTILE) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t off = (uint64_t)((((kk >> 2) * QHALF + (kk & 3) * 32) >> 4));
+                        const uint64_t koff = (uint64_t)((((kk >> 2) * KHALF + (kk & 3) * 32) >> 4));
+                        tc::umma_bf16(s_tm, dq + off, dk + koff, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    tc::umma_commit(BAR(B_SFULL + q));
+                    tc::umma_commit(BAR(B_EMPTY + sl));
+                    ++ns;
+                } else {
+                    mbar_arrive(BAR(B_EMPTY + sl));
+                }
+                ++it;
+                return true;
+            };
+            // V of tile t: O += P V once P is in shared memory, then the slot released
+            auto handle_v = [&](const Pos &t) -> bool {
+                const int sl = it % NSLOT;
+                if (!wait_bar(BAR(B_FULL + sl), (uint32_t)(it / NSLOT) & 1u)) return false;
+                if (t.mask & want) {
+                    if (!wait_bar(BAR(B_PFULL + q), (uint32_t)npv & 1u)) return false;
+                    tc::fence_after_sync();
+                    const uint64_t dv = dvl0 + (uint64_t)((sl * KTILE) >> 4);
+                    const int ksteps = (nkeys(t.jt) + 15) >> 4;
+                    if (ksteps == BN / 16 && npv > 0) {
+#pragma unroll
+                        for (int kk = 0; kk < BN / 16; ++kk) {
+                            const uint64_t poff = (uint64_t)((((kk >> 2) * PHALF + (kk & 3) * 32) >> 4));
+                            tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O, 1u);
+                        }
+                    } else {
+                        for (int kk = 0; kk < ksteps; ++kk) {
+                            const uint64_t poff = (uint64_t)((((kk >> 2) * PHALF + (kk & 3) * 32) >> 4));
+                            tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
+                                          (npv > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    tc::umma_commit(BAR(B_PVDONE + q));
+                    tc::umma_commit(BAR(B_EMPTY + sl));
+                    ++npv;
+                } else {
+                    mbar_arrive(BAR(B_EMPTY + sl));
+                }
+                ++it;
+                return true;
+            };
+            Pos t = walk_start(wk, fstart);
+            bool have = ok && walk_step(wk, t);
+            if (have) ok = handle_k(t);
+            while (ok && have) {
+                Pos u = t;
+                const bool next = walk_step(wk, u);
+                if (next && !(ok = handle_k(u))) break;   // K(t + 1) before V(t)
+                if (!(ok = handle_v(t))) break;
+                have = next;
+                t = u;
+            }
+            if (ok) tc::umma_commit(BAR(B_ODONE + q));
+        }
+    } else {
+        // ------------------------------- softmax ----------------------------------------
+        const int q = warp >> 2;
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const long lrow = l0 + q * BM + row;
+        const bool row_valid = lrow < p.q_rows;
+        const int fq = fq0 + (int)(lrow / p.N);
+        const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
+        uint8_t *prow = smem + SM_P(q) + row * 128;      // this row in each 64-key half of P
+        const float sl2 = p.sl2;
+        constexpr float LAZY = 8.f;
+        float m = -INFINITY, lsum = 0.f;
+        bool ok = true;
+        int k = 0;
+        Pos c = walk_start(wk, fstart);
+        while (walk_next(wk, c, 1 << q)) {
+            if (!__all_sync(0xffffffffu, wait_bar(BAR(B_SFULL + q), (uint32_t)k & 1u))) { ok = false; break; }
+            tc::fence_after_sync();
+            const int nv = nkeys(c.jt);
+            const bool rok = row_valid && is_tap(fq, c.fk, p.w, p.r);
+            // the tile's scores into registers, then the S buffer is free for the next tile
+            uint32_t sa[64], sb[64];
+            tc::tmem_ld64(tlane + TM_S(q), sa);
+            tc::tmem_ld64(tlane + TM_S(q) + 64, sb);
+            tc::fence_before_sync();
+            mbar_arrive(BAR(B_SFREE + q));
+            // masked keys (past the frame's end, or a frame this row does not attend) become
+            // -inf, so the exponentials below serve full, partial and masked tiles alike (the
+            // warp takes the masking branch together: rok differs between rows only where the
+            // sub-tile straddles a frame)
+            const int lim = rok ? nv : 0;
+            if (__any_sync(0xffffffffu, lim < BN)) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    if (i >= lim) sa[i] = __float_as_uint(-INFINITY);
+                    if (64 + i >= lim) sb[i] = __float_as_uint(-INFINITY);
+                }
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                mx0 = fmax3(mx0, __uint_as_float(sa[2 * i]), __uint_as_float(sa[2 * i + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(sb[2 * i]), __uint_as_float(sb[2 * i + 1]));
+            }
+            const float mt = fmaxf(mx0, mx1);
+            const float mnew = rok ? fmaxf(m, mt * sl2) : m;
+            const bool need = rok && mnew > m + LAZY;
+            const float muse = need ? mnew : m;
+            const float alpha = (need && m != -INFINITY) ? tc::ex2(m - mnew) : 1.f;
+            // P = 2^(s sl2 - m) as bf16 pairs, first into registers: the shared P tile is still
+            // the A operand of the previous tile's P V until that product completes
+            const float negm = muse == -INFINITY ? 0.f : -muse;
+            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(negm, negm);
+            float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            uint32_t pk[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const uint32_t *sv = i < 32 ? sa : sb;
+                const int j = i & 31;
+                const float2 x = ffma2(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sl2x2, nm2);
+                const float2 pp = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                ps2[i & 1] = fadd2(ps2[i & 1], pp);
+                pk[i] = tc::pack_bf16(pp.x, pp.y);
+            }
+            // the previous P V has completed (it read the P tile and accumulated into O)
+            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+            tc::fence_after_sync();
+            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
+                // the running max grew by more than 2^LAZY: rescale O before P V of this tile
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t orow[32];
+                    tc::tmem_ld32(tlane + TM_O(q) + cc * 32, orow);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                    tc::tmem_st32(tlane + TM_O(q) + cc * 32, orow);
+                }
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+            }
+            // this row of the shared P tile (128-byte swizzle: the 16-byte chunk index XORed
+            // with the row mod 8); masked keys give 0
+#pragma unroll
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(prow + half * PHALF + ((ch ^ (row & 7)) << 4)) =
+                        make_uint4(pk[half * 32 + ch * 4], pk[half * 32 + ch * 4 + 1],
+                                   pk[half * 32 + ch * 4 + 2], pk[half * 32 + ch * 4 + 3]);
+            lsum = lsum * alpha + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y));
+            m = muse;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(BAR(B_PFULL + q));
+            ++k;
+        }
+        // final: every product of the sub-tile has completed (a one-phase barrier its MMA warp
+        // commits after its last issue); normalise O and store it
+        const bool fin = ok && k >= 1 &&
+                         __all_sync(0xffffffffu, wait_bar(BAR(B_ODONE + q), 0u));
+        if (fin) {
+            tc::fence_after_sync();
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+            if (p.lse && row_valid) p.lse[q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
+            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t ov[32];
+                __syncwarp();
+                tc::tmem_ld32(tlane + TM_O(q) + cc * 32, ov);
+                if (row_valid) {
+                    uint32_t pk2[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        pk2[i] = tc::pack_bf16(__uint_as_float(ov[2 * i]) * inv, __uint_as_float(ov[2 * i + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[q4] = make_uint4(pk2[4 * q4], pk2[4 * q4 + 1], pk2[4 * q4 + 2], pk2[4 * q4 + 3]);
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == WARP_MMA) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s)
+{
+    if (a.d != D) return cudaErrorNotSupported;
+    cudaError_t e;
+    const long q_total = (long)a.B * a.q_Htot * a.q_rows;
+    const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
+    if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
+    CUtensorMap mq, mk, mv;
+    if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    Params p;
+    p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
+    p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
+    p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0; p.fq0_dev = a.fq0_dev;
+    p.sl2 = a.scale * 1.4426950408889634f;
+    p.lse = a.lse;
+    p.o = (__nv_bfloat16 *)a.o;
+    p.err = a.err;
+    e = cudaFuncSetAttribute(attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
+    attn_tc2_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p), note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace hlta

@@ -120,7 +120,7 @@ hlta_status check_window(int w, int r)
 hlta_status run_attn(const AttnArgs &a, hlta_dtype dt, cudaStream_t s)
 {
     if (a.B * a.Hbr == 0 || a.q_rows == 0) return HLTA_OK;
-    cudaError_t e = dt == HLTA_FP32 ? launch_attn_f32(a, s) : launch_attn_bf16_tc(a, s);
+    cudaError_t e = dt == HLTA_FP32 ? launch_attn_f32(a, s) : launch_attn_bf16_tc2(a, s);
     if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "window attention: unsupported shape");
     if (e != cudaSuccess) return cuda_fail(e, "window attention launch");
     return HLTA_OK;
