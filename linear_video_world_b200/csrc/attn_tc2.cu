@@ -372,6 +372,8 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         }
     } else {
         // ------------------------------- softmax ----------------------------------------
+        // The loop keeps little besides the 128 scores of a row: its own walk over the
+        // sub-tile's key frames (frame, tile), the running max and sum, and 32-bit addresses.
         const int q = warp >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
@@ -379,18 +381,27 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         const bool row_valid = lrow < p.q_rows;
         const int fq = fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-        uint8_t *prow = smem + SM_P(q) + row * 128;      // this row in each 64-key half of P
+        const uint32_t prow = sbase + SM_P(q) + (uint32_t)row * 128u;
+        const uint32_t rx = (uint32_t)(row & 7);
         const float sl2 = p.sl2;
         constexpr float LAZY = 8.f;
+        const int faq = q == 0 ? fa0 : fa1, fbq = q == 0 ? fb0 : fb1;
+        const bool qvalid = q == 0 || valid1;
         float m = -INFINITY, lsum = 0.f;
         bool ok = true;
         int k = 0;
-        Pos c = walk_start(wk, fstart);
-        while (walk_next(wk, c, 1 << q)) {
+        int fk = fstart - 1, jt = wk.tpf - 1;
+        while (qvalid) {
+            // the next tile of this sub-tile: the same frames and order as the MMA warp's walk
+            if (++jt >= wk.tpf) {
+                for (++fk; fk <= fbq && !frame_needed(fk, faq, fbq, p.w, p.r); ++fk) {}
+                if (fk > fbq) break;
+                jt = 0;
+            }
             if (!__all_sync(0xffffffffu, wait_bar(BAR(B_SFULL + q), (uint32_t)k & 1u))) { ok = false; break; }
             tc::fence_after_sync();
-            const int nv = nkeys(c.jt);
-            const bool rok = row_valid && is_tap(fq, c.fk, p.w, p.r);
+            const int nv = nkeys(jt);
+            const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
             // the tile's scores into registers, then the S buffer is free for the next tile
             uint32_t sa[64], sb[64];
             tc::tmem_ld64(tlane + TM_S(q), sa);
@@ -415,8 +426,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 mx0 = fmax3(mx0, __uint_as_float(sa[2 * i]), __uint_as_float(sa[2 * i + 1]));
                 mx1 = fmax3(mx1, __uint_as_float(sb[2 * i]), __uint_as_float(sb[2 * i + 1]));
             }
-            const float mt = fmaxf(mx0, mx1);
-            const float mnew = rok ? fmaxf(m, mt * sl2) : m;
+            const float mnew = rok ? fmaxf(m, fmaxf(mx0, mx1) * sl2) : m;
             const bool need = rok && mnew > m + LAZY;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? tc::ex2(m - mnew) : 1.f;
@@ -457,9 +467,11 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             for (int half = 0; half < 2; ++half)
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4 *>(prow + half * PHALF + ((ch ^ (row & 7)) << 4)) =
-                        make_uint4(pk[half * 32 + ch * 4], pk[half * 32 + ch * 4 + 1],
-                                   pk[half * 32 + ch * 4 + 2], pk[half * 32 + ch * 4 + 3]);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     prow + (uint32_t)half * PHALF + ((((uint32_t)ch) ^ rx) << 4)),
+                                 "r"(pk[half * 32 + ch * 4]), "r"(pk[half * 32 + ch * 4 + 1]),
+                                 "r"(pk[half * 32 + ch * 4 + 2]), "r"(pk[half * 32 + ch * 4 + 3])
+                                 : "memory");
             lsum = lsum * alpha + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y));
             m = muse;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
