@@ -13,8 +13,9 @@
 // zero rows with Up. That is the "state passing is a composition of multiplicative
 // transitions" of the llm-atlas long-context explainer (sections 06 and 09: chunkwise =
 // parallel within a block, recurrent across blocks); the scan applies it at two levels:
-//   1. segmap  (every segment but the last, A and B parts in separate CTAs, all in parallel):
-//              the chain over the segment's chunks from I (A part) or 0 (B part), no output;
+//   1. segmap  (every segment but the last, A and B parts in separate CTAs of one launch, all
+//              in parallel): the chain over the segment's chunks from I (A part) or 0 (B
+//              part), no output;
 //   2. compose (serial over segments, rows split over CTAs, fp32 on the CUDA cores):
 //              S_0 = S0, S_{p+1} = S_p A_p + B_p;
 //   3. replay  (every segment in parallel): the chain from S_p with the outputs O, the last
@@ -56,7 +57,7 @@ constexpr uint32_t KT_HALF = 64 * 128;     // [64 t][64 j] bf16: 8 KB
 // tensor-memory columns
 constexpr uint32_t TM_S = 0, TM_U = 64, TM_D = 128, TM_DL = 256, TM_COLS = 512;
 
-enum Mode { SEGMAP_A = 0, SEGMAP_B = 1, REPLAY = 2 };
+enum Mode { SEGMAP = 0, REPLAY = 2 };
 
 struct Stage {
     alignas(1024) uint8_t QW[2 * SLICE];     // Qt^T (replay) then W^T, each [128 j][64 t]
@@ -111,6 +112,10 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     ChainSmem &s = *reinterpret_cast<ChainSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const GdnArgs &p = a.g;
     const int seg = blockIdx.x, bh = blockIdx.y;
+    // the segment maps: part A (blockIdx.z 0) runs the chain from the identity with Up = 0,
+    // part B (blockIdx.z 1) from zero with Up; both in one launch
+    const bool segA = MODE == SEGMAP && blockIdx.z == 0;
+    const bool segB = MODE == SEGMAP && blockIdx.z == 1;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long c_begin = (long)seg * a.seg;
     const long c_end = min(a.nch, c_begin + a.seg);
@@ -148,9 +153,8 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     if (warp == WARP_TMA) {
         // ------------------------------ TMA producer --------------------------------------
         if (lane == 0) {
-            constexpr uint32_t TX = (MODE == REPLAY ? 2 * SLICE : SLICE) + 2 * KT_HALF +
-                                    (MODE == SEGMAP_A ? 0 : SLICE) + (MODE == REPLAY ? SLICE : 0) +
-                                    GDN_SCAL * 4;
+            const uint32_t TX = (MODE == REPLAY ? 2 * SLICE : SLICE) + 2 * KT_HALF +
+                                (segA ? 0 : SLICE) + (MODE == REPLAY ? SLICE : 0) + GDN_SCAL * 4;
             const long krow0 = (long)(b * p.Htot + p.h0 + h) * p.L;
             int k = 0;
             for (; k < nc; ++k) {
@@ -168,7 +172,7 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                 const int krow = (int)(krow0 + c * C);
                 for (int hf = 0; hf < 2; ++hf)
                     ptx::tma_load_2d(ptx::smem_u32(sg.Kt + hf * KT_HALF), &maps.K, hf * 64, krow, full);
-                if (MODE != SEGMAP_A) ptx::tma_load_2d(ptx::smem_u32(sg.Up), &maps.U, 0, trow, full);
+                if (!segA) ptx::tma_load_2d(ptx::smem_u32(sg.Up), &maps.U, 0, trow, full);
                 if (MODE == REPLAY) ptx::tma_load_2d(ptx::smem_u32(sg.Op), &maps.O, 0, trow, full);
                 ptx::bulk_load(ptx::smem_u32(sg.scal), a.ws.scal + ((long)bh * a.nch + c) * GDN_SCAL,
                                GDN_SCAL * 4, full);
@@ -221,10 +225,10 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
         const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
         __nv_bfloat16 *o = MODE == REPLAY ? (__nv_bfloat16 *)p.o + (long)(b * p.Htot + p.h0 + h) * p.L * D + i : nullptr;
         float sr[D];
-        if (MODE == SEGMAP_A) {
+        if (segA) {
 #pragma unroll
             for (int j = 0; j < D; ++j) sr[j] = j == i ? 1.f : 0.f;
-        } else if (MODE == SEGMAP_B) {
+        } else if (segB) {
 #pragma unroll
             for (int j = 0; j < D; ++j) sr[j] = 0.f;
         } else {
@@ -279,7 +283,7 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
                     ek[4 * q4] = e4.x; ek[4 * q4 + 1] = e4.y; ek[4 * q4 + 2] = e4.z; ek[4 * q4 + 3] = e4.w;
                 }
                 uint32_t pk[16];
-                if (MODE == SEGMAP_A) {
+                if (segA) {
 #pragma unroll
                     for (int m = 0; m < 16; ++m)
                         pk[m] = tc::pack_bf16(-ek[2 * m] * __uint_as_float(dw[2 * m]),
@@ -344,8 +348,8 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
         }
         if (ok) {
             float *dst = nullptr;
-            if (MODE == SEGMAP_A) dst = a.Amap + (((long)bh * a.nseg + seg) * D + i) * D;
-            else if (MODE == SEGMAP_B) dst = a.Bmap + (((long)bh * a.nseg + seg) * D + i) * D;
+            if (segA) dst = a.Amap + (((long)bh * a.nseg + seg) * D + i) * D;
+            else if (segB) dst = a.Bmap + (((long)bh * a.nseg + seg) * D + i) * D;
             else if (seg == a.nseg - 1 && p.S_out) dst = p.S_out + ((long)bh * D + i) * D;
             if (dst) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst);
@@ -477,15 +481,22 @@ int gdn_scan_segment_len(long BH, long nch)
 int gdn_scan_segments_beside(long BH, long nch, double attn_flop)
 {
     // Estimates from measurements on the B200 at 480P: the softmax launches run at about
-    // 6e8 FLOP per microsecond; one chunk step of the chain takes about 1.5 us when the
-    // chains of few heads run side by side. The chain is cut into as few segments as keep it
-    // within 70 % of the softmax time (each segment adds a map pass and a composition step).
+    // 8e8 FLOP per microsecond; one chunk step of the chain takes about 3 us when the chains
+    // of few heads run beside them. One segment is a single pass over the chunks; s > 1
+    // segments are two passes over ceil(nch / s) chunks (the maps, then the replay) plus s
+    // composition steps of a few microseconds. The fewest segments whose chain ends within
+    // the softmax branches' time beside the GDN branch (about 1.15 times their time alone,
+    // measured: they share the SMs with the chunk preparation and the chain) are taken: every
+    // extra segment occupies more SMs the softmax branches could use.
     const long seg_lat = gdn_scan_segment_len(BH, nch);
     const long max_seg = (nch + seg_lat - 1) / seg_lat;
-    const double attn_us = attn_flop / 6.0e8, chunk_us = 1.5;
-    long nseg = 1;
-    while (nseg < max_seg && chunk_us * (double)((nch + nseg - 1) / nseg) > 0.7 * attn_us) ++nseg;
-    return (int)nseg;
+    const double attn_us = 1.15 * attn_flop / 8.0e8, chunk_us = 3.0, compose_us = 5.0;
+    for (long s = 1; s < max_seg; ++s) {
+        const double lat = s == 1 ? chunk_us * (double)nch
+                                  : 2.0 * chunk_us * (double)((nch + s - 1) / s) + compose_us * (double)s;
+        if (lat <= attn_us) return (int)s;
+    }
+    return (int)max_seg;
 }
 
 size_t gdn_scan_bytes(long BH, long nch)
@@ -527,16 +538,14 @@ cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWs2 &ws, cudaStream_
     if ((e = make_tmap_2d_bf16(&m.O, ws.Ot, out_rows, C, 64, D, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&m.K, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
     const size_t smem = sizeof(ChainSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_A>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP_B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_chain_bf16<REPLAY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
     const size_t csmem = sizeof(ComposeSmem) + 128;
     if ((e = cudaFuncSetAttribute(gdn_compose, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem)) != cudaSuccess) return e;
     if (a.nseg > 1) {
         // the maps of every segment but the last, then their composition
-        const dim3 gm((unsigned)(a.nseg - 1), (unsigned)BH);
-        gdn_chain_bf16<SEGMAP_A><<<gm, THREADS, smem, s>>>(m, a), note_launch();
-        gdn_chain_bf16<SEGMAP_B><<<gm, THREADS, smem, s>>>(m, a), note_launch();
+        const dim3 gm((unsigned)(a.nseg - 1), (unsigned)BH, 2);
+        gdn_chain_bf16<SEGMAP><<<gm, THREADS, smem, s>>>(m, a), note_launch();
         gdn_compose<<<dim3(D / CR, (unsigned)BH), COMPOSE_THREADS, csmem, s>>>(a), note_launch();
     }
     gdn_chain_bf16<REPLAY><<<dim3((unsigned)a.nseg, (unsigned)BH), THREADS, smem, s>>>(m, a), note_launch();
