@@ -374,7 +374,7 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
 // compose: S_0 = S0, S_{p+1} = S_p A_p + B_p, fp32 on the CUDA cores. Rows of S are
 // independent: a CTA owns CR rows of one head. Each step's A_p (64 KB) and the CTA's rows of
 // B_p arrive by bulk copy into one of two buffers, the next step's while this one computes;
-// a thread owns one key column j of half the rows, two rows per packed f32x2 FMA.
+// a thread owns one key column j of four of the rows.
 // -----------------------------------------------------------------------------------------
 constexpr int CR = 8;
 constexpr int COMPOSE_THREADS = 256;
@@ -385,16 +385,6 @@ struct ComposeSmem {
     alignas(8) uint64_t bar[2];
     int abort_flag;
 };
-
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
-        "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
 
 __global__ void __launch_bounds__(COMPOSE_THREADS, 1)
 gdn_compose(const ChainArgs a)
@@ -442,16 +432,24 @@ gdn_compose(const ChainArgs a)
              ptx::mbar_wait(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u, abort_flag, p.err, DEVERR_GDN_WAIT);
         if (!__syncthreads_and(ok)) break;
         const float *A = s.A[sp & 1];
-        float2 acc01 = make_float2(s.Bm[sp & 1][(4 * rh) * D + j], s.Bm[sp & 1][(4 * rh + 1) * D + j]);
-        float2 acc23 = make_float2(s.Bm[sp & 1][(4 * rh + 2) * D + j], s.Bm[sp & 1][(4 * rh + 3) * D + j]);
+        // eight independent accumulators (four rows, even and odd k) keep the FMA chains short
+        float acc[2][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            acc[0][r] = s.Bm[sp & 1][(4 * rh + r) * D + j];
+            acc[1][r] = 0.f;
+        }
 #pragma unroll 16
         for (int k = 0; k < D; ++k) {
             const float av = A[k * D + j];
             const float4 sk = *reinterpret_cast<const float4 *>(&s.srow[k][4 * rh]);
-            acc01 = ffma2(make_float2(sk.x, sk.y), make_float2(av, av), acc01);
-            acc23 = ffma2(make_float2(sk.z, sk.w), make_float2(av, av), acc23);
+            acc[k & 1][0] = fmaf(sk.x, av, acc[k & 1][0]);
+            acc[k & 1][1] = fmaf(sk.y, av, acc[k & 1][1]);
+            acc[k & 1][2] = fmaf(sk.z, av, acc[k & 1][2]);
+            acc[k & 1][3] = fmaf(sk.w, av, acc[k & 1][3]);
         }
-        cur[0] = acc01.x; cur[1] = acc01.y; cur[2] = acc23.x; cur[3] = acc23.y;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cur[r] = acc[0][r] + acc[1][r];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
             a.Sseg[(((long)bh * a.nseg + sp + 1) * D + r0 + 4 * rh + r) * D + j] = cur[r];

@@ -1,4 +1,4 @@
-// Host helper: 2-D TMA tensor maps over row-major [rows][cols] bf16 or byte tensors. The driver's
+// Host helper: TMA tensor maps over row-major bf16 or byte tensors. The driver's
 // encoder is fetched once through the runtime's entry-point query (no link-time libcuda).
 #include "hlta_internal.cuh"
 
@@ -11,11 +11,8 @@ namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
-}  // namespace
-
-static cudaError_t encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint32_t elem,
-                             const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                             uint32_t box_rows, bool swizzle128)
+// the driver's tensor-map encoder (looked up once)
+PFN_cuTensorMapEncodeTiled_v12000 encoder()
 {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
@@ -25,7 +22,16 @@ static cudaError_t encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint32_t 
             q == cudaDriverEntryPointSuccess)
             g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
     });
-    if (!g_encode) return cudaErrorNotSupported;
+    return g_encode;
+}
+
+}  // namespace
+
+static cudaError_t encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint32_t elem,
+                             const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                             uint32_t box_rows, bool swizzle128)
+{
+    if (!encoder()) return cudaErrorNotSupported;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
     cuuint32_t box[2] = {box_cols, box_rows};
