@@ -732,8 +732,9 @@ def main():
     # the timed region lasts K steps of ~2 ms (tens of ms): the burst peak applies, not the
     # seconds-long sustained one
     peak = float(pk.get("bf16_tflops"))
-    tr = traffic_record("attn_tc.cu")
-    roofline = {"bound": "tensor", "kernel": "attn_tc_kernel (SWA + DSWA launches, side by side: "
+    tr = traffic_record("attn_tc2.cu")          # the bf16 window attention kernel
+    tr8 = traffic_record("attn_tc.cu")          # its E4M3 variant
+    roofline = {"bound": "tensor", "kernel": "attn_tc2_kernel (SWA + DSWA launches, side by side: "
                                               "the span from their common start to the later end)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"{pk_kind} bf16 dense, burst (the timed region is {total_ms:.0f} ms)",
@@ -794,7 +795,7 @@ def main():
             "fp8_peak_tflops": fp8_peak,
             "attn_bytes": 5 * elems,
             "quantise_and_attn_ms": fp8_ms["quantise_and_attn"],
-            "attn_traffic": (tr["fp8_swa_bytes"] + tr["fp8_dswa_bytes"]) if tr and "fp8_swa_bytes" in tr else None,
+            "attn_traffic": (tr8["fp8_swa_bytes"] + tr8["fp8_dswa_bytes"]) if tr8 and "fp8_swa_bytes" in tr8 else None,
             "note": "hlta_window_fp8_fwd for the SWA and DSWA heads back to back on resident E4M3 "
                     "codes (q, k, v 1 byte, o bf16: attn_bytes; attn_traffic: DRAM bytes of the two "
                     "launches from the committed ncu summary), then with the three "
