@@ -716,6 +716,32 @@ def main():
     torch.cuda.synchronize()
     attn_alone_ms = a0.elapsed_time(a1) / K
     del sub, o_s, o_d
+
+    # ---- the GDN branch alone (its heads by themselves, all SMs to itself) -----------------
+    gdn_alone_ms = None
+    if wl.Hg > 0:
+        hg = slice(wl.Hs + wl.Hd, wl.Hs + wl.Hd + wl.Hg)
+        gq, gk, gv = (x_[:, hg].contiguous() for x_ in (q, k, v))
+        go = torch.empty_like(gq)
+        gS = torch.empty((wl.B, wl.Hg, wl.d, wl.d), device=dev, dtype=torch.float32)
+        gws = torch.empty(h.hlta_gdn_workspace_bytes(wl.B, wl.Hg, wl.L, wl.d, wl.chunk,
+                                                     h.HLTA_BF16 if wl.dtype == "bf16" else h.HLTA_FP32),
+                          device=dev, dtype=torch.uint8)
+
+        def gdn_only():
+            h.hlta_gdn_chunk_fwd(gq, gk, gv, a, b, go, None, gS, wl.B, wl.Hg, wl.L, wl.d, wl.chunk, gws)
+
+        for _ in range(3):
+            gdn_only()
+        torch.cuda.synchronize()
+        a0.record()
+        for _ in range(K):
+            gdn_only()
+        a1.record()
+        torch.cuda.synchronize()
+        assert h.hlta_device_status() == 0
+        gdn_alone_ms = a0.elapsed_time(a1) / K
+        del gq, gk, gv, go, gS, gws
     stream_detail = None if args.no_stream else measure_stream(h, torch, dev)
     raw_detail = None if args.no_stream else measure_raw(h, torch, dev, wl, hi, K)
     fp8_ms = (measure_fp8(h, torch, dev, wl, q, k, v, K)
@@ -750,12 +776,16 @@ def main():
         "attn_alone_ms": attn_alone_ms,
         "attn_alone_tflops": attn_flop / (attn_alone_ms / 1e3) / 1e12,
         "attn_alone_frac": attn_flop / (attn_alone_ms / 1e3) / 1e12 / float(pk.get("bf16_tflops")),
+        "gdn_alone_ms": gdn_alone_ms,
+        "gdn_alone_gbs": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 if gdn_alone_ms else None,
+        "gdn_alone_hbm_frac": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 / hbm if gdn_alone_ms else None,
         "note": "the three branches run side by side (GDN on a high-priority stream, DSWA beside "
                 "SWA); swa_ms and dswa_ms run from their common start, attn_span_ms to the later "
                 "end (the roofline's duration), all while sharing the SMs with the GDN branch; "
                 "attn_alone_* times the two softmax launches back to back by themselves against "
-                "the burst bf16 peak. The GDN HBM fraction uses the algorithmic q/k/v/o + gate "
-                "bytes of the GDN heads",
+                "the burst bf16 peak; gdn_alone_* times hlta_gdn_chunk_fwd on the GDN heads by "
+                "themselves (segment scan over all SMs). The GDN HBM fractions use the "
+                "algorithmic q/k/v/o + gate bytes of the GDN heads",
     }
     if stream_detail is not None:
         stream_detail["softmax_frac"] = stream_detail["softmax_tflops"] / peak
