@@ -1,6 +1,6 @@
 // Gated delta rule, bf16 forward: the chunk preparation on the sm_100a tensor cores.
 //
-// Per 64-token chunk of a head (one CTA, 128 threads, two CTAs per SM), with g_t the running
+// Per 64-token chunk of a head (one CTA, 128 threads, three CTAs per SM), with g_t the running
 // sum of log a inside the chunk (carried in log2 units) and the chunk algebra of the
 // llm-atlas long-context explainer's chunkwise form (sections 06 and 09) derived from
 // S_t = a_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T:
@@ -15,7 +15,9 @@
 //   Qt^T = (diag(e^g) Q)^T - (P W)^T
 // T is formed in fp32 on the CUDA cores: 16 x 16 diagonal blocks by forward substitution, then
 // two levels of T10 = -T11 A10 T00. The four [128][64] outputs are staged in shared memory in
-// the 128-byte swizzle and leave by TMA stores. Per chunk a record of fp32 scalars follows:
+// the 128-byte swizzle over input tiles that are dead by then, and leave by TMA stores, so a CTA
+// needs 74 KB of shared memory and 128 tensor-memory columns: three CTAs share an SM, and one
+// CTA's loads, stores and tensor-core round trips overlap the others' arithmetic. Per chunk a record of fp32 scalars follows:
 // gam = e^{g_n} and ek_t = e^{g_n - g_t} (times 1/|k_t| for raw inputs): the pass over the
 // chunks reads K itself from the input and applies ek to U instead of storing Kt = diag(ek) K.
 #include "hlta_internal.cuh"
@@ -36,21 +38,28 @@ constexpr uint32_t V_HALF = 64 * 128;      // per 64-column half of V: 8 KB
 constexpr uint32_t SQ = 64 * 128;          // a [64][64] bf16 swizzled tile: 8 KB
 constexpr uint32_t SLICE = 128 * 128;      // a [128][64] bf16 swizzled tile: 16 KB
 constexpr int AP = 68;                     // fp32 row stride of A and T
-constexpr uint32_t TM_D1 = 0, TM_WT = 64, TM_UT = 128, TM_OT = 192, TM_PW = 0, TM_COLS = 256;
+// tensor-memory columns: each pair of products reuses the columns the previous pair's results
+// were read from
+constexpr uint32_t TM_D1 = 0, TM_WT = 0, TM_UT = 64, TM_OT = 0, TM_PW = 64, TM_COLS = 128;
 
 struct Smem {
     alignas(1024) uint8_t KQ[2 * KQ_HALF];   // K, Q by TMA; later Op^T staged over the K rows
-    alignas(1024) uint8_t V[2 * V_HALF];     // V by TMA; later Qt^T staged
-    alignas(1024) uint8_t Wt[SLICE];         // W^T staged (also the A operand of (P W)^T)
-    alignas(1024) uint8_t Ut[SLICE];         // Up^T staged (also the A operand of Op^T)
+    alignas(1024) uint8_t V[2 * V_HALF];     // V by TMA; then W^T staged (the A operand of
+                                             // (P W)^T); then Qt^T staged
+    alignas(1024) float A[C * AP];           // A, T in place; then T1 and T2 (bf16 tiles); then
+                                             // Up^T staged (the A operand of Op^T)
     alignas(1024) uint8_t P[SQ];             // P [t][t'] bf16
-    alignas(1024) float A[C * AP];           // A, T in place, then T1 and T2 (bf16 tiles) over it
     float g[C], eg[C], ek[C], bb[C], ks[C];
     alignas(8) uint64_t bar_ld, bar_mma;
     uint32_t tmem_slot;
     int abort_flag;
 };
-static_assert(2 * SQ <= sizeof(float) * C * AP, "T1 and T2 fit over A");
+static_assert(2 * SQ <= sizeof(float) * C * AP && SLICE <= sizeof(float) * C * AP, "T1, T2 and Up^T fit over A");
+static_assert(SLICE == 2 * V_HALF, "W^T and Qt^T fit over V");
+// the bytes a CTA uses (sizeof(Smem) rounds up to the 1024-byte alignment); three CTAs with
+// their 1 KB reserved each fit the SM's 228 KB
+constexpr size_t SMEM_USED = offsetof(Smem, abort_flag) + sizeof(int);
+static_assert(3 * (SMEM_USED + 1024) <= 228 * 1024, "three CTAs per SM");
 
 struct Maps {
     CUtensorMap q, k, v;                   // inputs [B*Htot*L][128]: 64 cols x 64 rows, swizzled
@@ -98,11 +107,18 @@ __device__ __forceinline__ void store_row_bf16(uint8_t *tile, int r, const float
     }
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 3)
 gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
 {
-    extern __shared__ uint8_t smem_raw[];
-    Smem &s = *reinterpret_cast<Smem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    // the launch requests exactly the bytes used (no slack for aligning the base by hand), so
+    // the swizzled tiles rely on the dynamic shared memory starting 1024-byte aligned, as it
+    // does with no static shared memory; a base that is not is reported, never used
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if ((ptx::smem_u32(smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicOr(p.err, DEVERR_GDN_WAIT);
+        return;
+    }
+    Smem &s = *reinterpret_cast<Smem *>(smem_raw);
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / p.Hg, h = bh % p.Hg;
     const long nch = gdn_num_chunks(p.L, C);
@@ -113,8 +129,9 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     volatile int *abort_flag = (volatile int *)&s.abort_flag;
     const uint32_t KQ = ptx::smem_u32(s.KQ), V = ptx::smem_u32(s.V);
-    const uint32_t WT = ptx::smem_u32(s.Wt), UT = ptx::smem_u32(s.Ut), PS = ptx::smem_u32(s.P);
+    const uint32_t PS = ptx::smem_u32(s.P);
     const uint32_t T1 = ptx::smem_u32(s.A), T2 = T1 + SQ;
+    const uint32_t WT = V, UT = T1;          // staged over V and over T1, T2 once W^T, Up^T exist
     const uint32_t BLD = ptx::smem_u32(&s.bar_ld), BMMA = ptx::smem_u32(&s.bar_mma);
     uint8_t *t1p = reinterpret_cast<uint8_t *>(s.A), *t2p = t1p + SQ;
 
@@ -374,14 +391,15 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
     {
         uint32_t dv[64];
         float x[64];
+        // both products have completed: V and T1, T2 are dead
         tc::tmem_ld64(tl + TM_WT, dv);
 #pragma unroll
         for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
-        store_row_bf16(s.Wt, tid, x);
+        store_row_bf16(s.V, tid, x);
         tc::tmem_ld64(tl + TM_UT, dv);
 #pragma unroll
         for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
-        store_row_bf16(s.Ut, tid, x);
+        store_row_bf16(t1p, tid, x);
     }
     fence_async_smem();
     tc::fence_before_sync();
@@ -405,6 +423,8 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
         tc::umma_commit(BMMA);
     }
     ok = ptx::mbar_try(BMMA, 0) || ptx::mbar_wait(BMMA, 0, abort_flag, p.err, DEVERR_GDN_WAIT);
+    // Qt^T goes over W^T below: its store must have read it first
+    if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     if (!__syncthreads_and(ok)) goto done;
     tc::fence_after_sync();
     {
@@ -415,7 +435,7 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
 #pragma unroll
         for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(dv[i]);
         store_row_bf16(s.KQ + (tid >> 6) * KQ_HALF, tid & 63, x);
-        // Qt^T row j = e^g_t Q[t][j] - (P W)^T[j][t], over the dead V tile
+        // Qt^T row j = e^g_t Q[t][j] - (P W)^T[j][t], over W^T (stored and consumed by now)
         tc::tmem_ld64(tl + TM_PW, dv);
         const int j = tid;
         const uint8_t *qh = s.KQ + (j >> 6) * KQ_HALF + Q_OFF;
@@ -473,8 +493,11 @@ cudaError_t launch_gdn_bf16_v2(const GdnArgs &g, cudaStream_t s)
     if ((e = make_tmap_2d_bf16(&m.ut, ws.Ut, out_rows, C, 64, D, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&m.qt, ws.Qt, out_rows, C, 64, D, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&m.ot, ws.Ot, out_rows, C, 64, 64, true)) != cudaSuccess) return e;
-    const size_t smem = sizeof(Smem) + 1024;
+    const size_t smem = SMEM_USED;
     if ((e = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(gdn_prep_tc, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
         return e;
     gdn_prep_tc<<<dim3((unsigned)nch, (unsigned)BH), THREADS, smem, s>>>(m, g, ws), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -28,6 +28,9 @@
 //          (DEVERR_GDN_WAIT).
 // The serial chain is latency-bound (two dependent 64x16x128-class products per chunk), so
 // it uses register-resident warp MMAs rather than a TMEM round trip per dependent step.
+// These kernels serve the backward pass (its recomputed chunk preparation, the chunk start
+// states, and the state-gradient pass built the same way); the forward runs the tcgen05
+// chunk preparation of gdn_prep_tc.cu and the segment scan of gdn_scan.cu.
 #include "hlta_internal.cuh"
 #include "sm100_ptx.cuh"
 
@@ -947,40 +950,6 @@ gdn_dstate_bf16(const __grid_constant__ DStateMaps maps, GdnArgs p, GdnWorkspace
 }
 
 }  // namespace
-
-cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s)
-{
-    if (g.d != D) return cudaErrorNotSupported;
-    const long nch = gdn_num_chunks(g.L, C);
-    const long BH = (long)g.B * g.Hg;
-    const long in_rows = (long)g.B * g.Htot * g.L;
-    const long ws_rows = BH * nch * C;
-    if (nch > 0x7fffffffL || in_rows + C >= (1L << 31) || ws_rows >= (1L << 31))
-        return cudaErrorNotSupported;
-    GdnWorkspace ws = gdn_workspace_carve(g.ws, BH, g.L, D, C, true);
-    cudaError_t e;
-    PrepMaps pm;
-    if ((e = make_tmap_2d_bf16(&pm.q, g.q, in_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&pm.k, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&pm.v, g.v, in_rows, D, 64, C, true)) != cudaSuccess) return e;
-    StateMaps sm;
-    if ((e = make_tmap_2d_bf16(&sm.W, ws.W, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.Q, ws.Qt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.K, ws.Kt, ws_rows, D, 64, C, true)) != cudaSuccess) return e;
-    // Up^T and Op^T: [BHg*nch*128][64] views, boxes of 64 state rows x 64 tokens, swizzled
-    if ((e = make_tmap_2d_bf16(&sm.U, ws.Up, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&sm.O, ws.Op, ws_rows * 2, C, 64, CW, true)) != cudaSuccess) return e;
-    const size_t smem_prep = sizeof(PrepSmem) + 1024;
-    const size_t smem_state = sizeof(StateSmem) + 1024;
-    e = cudaFuncSetAttribute(gdn_prep_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gdn_state_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
-    if (e != cudaSuccess) return e;
-    gdn_prep_bf16<<<dim3((unsigned)nch, (unsigned)BH), PREP_THREADS, smem_prep, s>>>(pm, g, ws), note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gdn_state_bf16<<<dim3(D / CW, (unsigned)BH), STATE_THREADS, smem_state, s>>>(sm, g, ws), note_launch();
-    return cudaGetLastError();
-}
 
 cudaError_t launch_gdn_bf16_bwd_states(const GdnArgs &g, const void *dO, const float *dS_final,
                                        float *dS_chunks, float *dS0, cudaStream_t s,

@@ -111,8 +111,7 @@ cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, u
 
 // Launchers. Return cudaGetLastError() of their launches.
 cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
-cudaError_t launch_attn_bf16_tc(const AttnArgs &a, cudaStream_t s);
-// bf16 window attention with 128-key tiles and alternating sub-tile softmax (attn_tc2.cu)
+// bf16 window attention: 128-key tiles, two query sub-tiles, P staged in shared memory (attn_tc2.cu)
 cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_fp8_tc(const AttnArgs &a, cudaStream_t s);
 // E4M3 quantisation (bf16 input, d = 128): row blocks inside frames, and value channels
@@ -177,7 +176,6 @@ size_t gdn_scan_bytes(long BH, long nch);
 cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWs2 &ws, cudaStream_t s);
 // the bf16 forward: the tensor-core chunk preparation, then the segment scan
 cudaError_t launch_gdn_bf16_v2(const GdnArgs &g, cudaStream_t s);
-cudaError_t launch_gdn_bf16(const GdnArgs &g, cudaStream_t s);
 // f0: the first new frame's index, read from f0_dev when that is set (streaming steps keep
 // their frame counter on the device so that a captured step can be replayed)
 cudaError_t launch_ring_append(const void *src, int B, int Htot, int h0, int Hbr, int N, int d,

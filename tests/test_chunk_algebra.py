@@ -77,6 +77,40 @@ def test_chunk_form_strong_decay_no_overflow(orc):
     np.testing.assert_allclose(o, o_ref[0], rtol=1e-9, atol=1e-12)
 
 
+def test_segment_maps_compose_to_the_recurrence(orc):
+    """The two-level scan the GPU pass over the chunks uses: the map of a run of tokens is
+    affine in the start state (rows of S evolve independently), S_end = S_start A + B, with
+    A = the run from the identity with v = 0 (every write U is linear in v, so Up = 0) and
+    B = the run from zero with v. Composing the maps of consecutive segments serially gives
+    each segment's true start state, and replaying a segment from it gives the recurrence's
+    outputs (llm-atlas long-context explainer, section 09: state passing as composed
+    transitions). Ragged segment lengths, slow decay so the maps stay far from zero."""
+    rng = np.random.default_rng(11)
+    L, d = 230, 12
+    q = rng.standard_normal((L, d)); q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k = rng.standard_normal((L, d)); k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((L, d))
+    a = np.exp(-0.05 * np.log1p(np.exp(rng.standard_normal(L))))
+    b = 1 / (1 + np.exp(-rng.standard_normal(L)))
+    q, k, v, a, b = (x.astype(np.float32) for x in (q, k, v, a, b))
+    S0 = rng.standard_normal((d, d))
+    o_all, S_all = orc.gdn(q[None], k[None], v[None], a[None], b[None], S0[None])
+    cuts = [0, 64, 100, 192, L]
+    S = S0.copy()
+    zero_v = np.zeros_like(v)
+    for s0, s1 in zip(cuts[:-1], cuts[1:]):
+        sl = slice(s0, s1)
+        # replay from the composed start state: the recurrence's outputs on this segment
+        o_seg, _ = orc.gdn(q[None, sl], k[None, sl], v[None, sl], a[None, sl], b[None, sl], S[None])
+        np.testing.assert_allclose(o_seg[0], o_all[0, sl], rtol=1e-9, atol=1e-10)
+        _, Am = orc.gdn(q[None, sl], k[None, sl], zero_v[None, sl], a[None, sl], b[None, sl],
+                        np.eye(d)[None])
+        _, Bm = orc.gdn(q[None, sl], k[None, sl], v[None, sl], a[None, sl], b[None, sl],
+                        np.zeros((1, d, d)))
+        S = S @ Am[0] + Bm[0]
+    np.testing.assert_allclose(S, S_all[0], rtol=1e-9, atol=1e-10)
+
+
 # --------------------------------------------------------------------------------------
 # Backward pass in chunk form
 # --------------------------------------------------------------------------------------

@@ -37,6 +37,24 @@ def test_gdn_bf16_full(h, orc, B, H, L, decay):
     assert maxabs(S, S_ref) <= TOL
 
 
+@pytest.mark.parametrize("B,H,L,decay", [(1, 8, 32760, 1.0), (1, 2, 8360, 0.05)])
+def test_gdn_bf16_segment_scan(h, orc, B, H, L, decay):
+    """Heads long enough for the two-level scan: 480P's 8 heads of 512 chunks (16 segments
+    of 32 chunks: segment maps, their composition and the replay), and 131 chunks in 5
+    segments with a ragged last segment and a ragged last chunk under slow decay (the maps
+    carry the start state far)."""
+    wl = _gdn_wl(B, H, L, decay)
+    x = hi.make_inputs(wl, seed=L + H)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    S0 = hi.random_state(B, H, 128, seed=4, scale=0.1)
+    o, S = h.gdn(q, k, v, a, b, S0=dev(S0), out=poison_like(q))
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    o_ref, S_ref = orc.gdn(x["q"], x["k"], x["v"], x["a"], x["b"], S0.double().numpy())
+    assert maxabs(o, o_ref) <= TOL
+    assert maxabs(S, S_ref) <= TOL
+
+
 def test_gdn_bf16_zero_gate_write_keeps_zero_state(h):
     """b = 0 from a zero state: the memory stays exactly zero (no write ever happens)."""
     wl = _gdn_wl(1, 1, 300)
