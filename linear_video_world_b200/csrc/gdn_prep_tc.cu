@@ -49,7 +49,7 @@ struct Smem {
     alignas(1024) float A[C * AP];           // A, T in place; then T1 and T2 (bf16 tiles); then
                                              // Up^T staged (the A operand of Op^T)
     alignas(1024) uint8_t P[SQ];             // P [t][t'] bf16
-    float g[C], eg[C], ek[C], bb[C], ks[C];
+    alignas(16) float g[C], eg[C], ek[C], bb[C], ks[C], beg[C];   // beg = b e^g
     alignas(8) uint64_t bar_ld, bar_mma;
     uint32_t tmem_slot;
     int abort_flag;
@@ -192,6 +192,7 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
     if (tid < C) {
         const float gn = s.g[n - 1];
         s.eg[tid] = tid < n ? fast_ex2(s.g[tid]) : 0.f;
+        s.beg[tid] = s.bb[tid] * s.eg[tid];
         s.ek[tid] = tid < n ? fast_ex2(gn - s.g[tid]) : 0.f;
         s.ks[tid] = 1.f;
     }
@@ -310,7 +311,10 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
         for (int t = 0; t < 16; ++t) s.A[(bb0 + t) * AP + bb0 + jj] = tcv[t];
     }
     __syncthreads();
-    // levels 2 and 3: T10 = -T11 (A10 T00) for the 32 x 32 blocks, then for the whole 64 x 64
+    // levels 2 and 3: T10 = -T11 (A10 T00) for the 32 x 32 blocks, then for the whole 64 x 64.
+    // Y = A10 T00 goes to the upper right 32 x 32 block of the array (above the diagonal, where
+    // T is zero and no level reads), so each product needs one barrier: T10 may overwrite A10
+    // as soon as every thread has passed the barrier after the first product.
 #pragma unroll
     for (int lvl = 0; lvl < 2; ++lvl) {
         const int bs = lvl == 0 ? 16 : 32;                     // size of T00, T11, A10
@@ -319,50 +323,50 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
         const int u = lvl == 0 ? (tid & 63) : tid;
         const int r = u / (bs / per), c0 = (u % (bs / per)) * per;
         const int o = blk * 32;                                 // block origin
+        float *yb = s.A + (16 * blk) * AP + 32 + 16 * blk;      // Y scratch: rows 0-31, cols 32-63
         float y[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) y[c] = 0.f;
+#pragma unroll
         for (int k = 0; k < bs; ++k) {                          // Y = A10 T00
             const float av = s.A[(o + bs + r) * AP + o + k];
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 if (c < per) y[c] = fmaf(av, s.A[(o + k) * AP + o + c0 + c], y[c]);
         }
-        __syncthreads();
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-            if (c < per) s.A[(o + bs + r) * AP + o + c0 + c] = y[c];
+            if (c < per) yb[r * AP + c0 + c] = y[c];
         __syncthreads();
 #pragma unroll
         for (int c = 0; c < 8; ++c) y[c] = 0.f;
+#pragma unroll
         for (int k = 0; k < bs; ++k) {                          // T10 = -T11 Y
             const float tv = s.A[(o + bs + r) * AP + o + bs + k];
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-                if (c < per) y[c] = fmaf(-tv, s.A[(o + bs + k) * AP + o + c0 + c], y[c]);
+                if (c < per) y[c] = fmaf(-tv, yb[k * AP + c0 + c], y[c]);
         }
-        __syncthreads();
 #pragma unroll
         for (int c = 0; c < 8; ++c)
             if (c < per) s.A[(o + bs + r) * AP + o + c0 + c] = y[c];
         __syncthreads();
     }
     // T1 = T diag(b e^g) (threads 0-63) and T2 = T diag(b) (threads 64-127), bf16 [t][t'] tiles
-    // over A once every row of T has been read
+    // over A once every row of T has been read (rows 0-31 stop at column 32: the Y scratch)
     {
         const int t = tid & (C - 1);
+        const float *fac = tid < C ? s.beg : s.bb;
         float x[64];
 #pragma unroll
         for (int i4 = 0; i4 < C / 4; ++i4) {
             const float4 v4 = *reinterpret_cast<const float4 *>(s.A + t * AP + 4 * i4);
-            x[4 * i4] = v4.x; x[4 * i4 + 1] = v4.y; x[4 * i4 + 2] = v4.z; x[4 * i4 + 3] = v4.w;
-        }
-        if (tid < C) {
-#pragma unroll
-            for (int i = 0; i < C; ++i) x[i] *= s.bb[i] * s.eg[i];
-        } else {
-#pragma unroll
-            for (int i = 0; i < C; ++i) x[i] *= s.bb[i];
+            const float4 f4 = *reinterpret_cast<const float4 *>(fac + 4 * i4);
+            const bool z = i4 >= C / 8 && t < C / 2;
+            x[4 * i4] = z ? 0.f : v4.x * f4.x;
+            x[4 * i4 + 1] = z ? 0.f : v4.y * f4.y;
+            x[4 * i4 + 2] = z ? 0.f : v4.z * f4.z;
+            x[4 * i4 + 3] = z ? 0.f : v4.w * f4.w;
         }
         __syncthreads();
         store_row_bf16(tid < C ? t1p : t2p, t, x);

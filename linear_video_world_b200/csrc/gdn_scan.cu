@@ -51,23 +51,33 @@ constexpr int THREADS = 192;
 constexpr int ROWS = 128;              // chain threads = state rows
 
 constexpr uint32_t SLICE = 128 * 128;      // [128 rows][64 t] bf16: 16 KB
-constexpr uint32_t W_OFF = SLICE;          // W^T follows Qt^T in the stage
 constexpr uint32_t KT_HALF = 64 * 128;     // [64 t][64 j] bf16: 8 KB
-
-// tensor-memory columns
-constexpr uint32_t TM_S = 0, TM_U = 64, TM_D = 128, TM_DL = 256, TM_COLS = 512;
 
 enum Mode { SEGMAP = 0, REPLAY = 2 };
 
-struct Stage {
-    alignas(1024) uint8_t QW[2 * SLICE];     // Qt^T (replay) then W^T, each [128 j][64 t]
+// Tensor-memory columns. Replay: S bf16 [0, 64), U bf16 [64, 96), D = [D_Q | D_W] at 128, U Kt
+// at 256 (512 allocated). Segment maps (no outputs, two CTAs per SM): D_W and U Kt share the
+// columns at 128, since U Kt is issued after the chain threads read D_W and the next D_W after
+// they read U Kt (256 allocated).
+template <int MODE> struct Tm {
+    static constexpr uint32_t S = 0, U = 64;
+    static constexpr uint32_t D1 = 128;                           // target of S [Qt; W]^T
+    static constexpr uint32_t DW = MODE == REPLAY ? 192 : 128;    // D_W
+    static constexpr uint32_t DL = MODE == REPLAY ? 256 : 128;    // U Kt
+    static constexpr uint32_t COLS = MODE == REPLAY ? 512 : 256;
+};
+
+template <int MODE> struct Stage {
+    // replay: Qt^T then W^T; segment maps: W^T alone; each [128 j][64 t]
+    static constexpr uint32_t W_OFF = MODE == REPLAY ? SLICE : 0;
+    alignas(1024) uint8_t QW[(MODE == REPLAY ? 2 : 1) * SLICE];
     alignas(1024) uint8_t Kt[2 * KT_HALF];   // K [64 t][128 j] (the input) as two 64-column halves
     alignas(1024) uint8_t Up[SLICE];         // Up^T [128 i][64 t]
-    alignas(1024) uint8_t Op[SLICE];         // Op^T (replay)
+    alignas(1024) uint8_t Op[MODE == REPLAY ? SLICE : 16];   // Op^T (replay)
     alignas(16) float scal[GDN_SCAL];        // gam, then ek_t at 4 + t
 };
-struct ChainSmem {
-    Stage st[NSTG];
+template <int MODE> struct ChainSmem {
+    Stage<MODE> st[NSTG];
     alignas(8) uint64_t full[NSTG];
     alignas(8) uint64_t empty[NSTG];       // MMA commit (+ chain threads done with Op, replay)
     alignas(8) uint64_t s_ready;           // chain threads stored S (count ROWS)
@@ -88,7 +98,9 @@ struct ChainArgs {
     GdnWs2 ws;
     long nch;
     int seg, nseg;
-    float *Amap, *Bmap, *Sseg;             // [BH][nseg][D][D] fp32 each
+    // [BH][nseg][D][D] fp32 each, every matrix stored transposed ([j][i]: element (i, j) at
+    // j * D + i), so that a warp's 32 rows i read or write one 128-byte line per column j
+    float *Amap, *Bmap, *Sseg;
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag,
@@ -105,11 +117,13 @@ __device__ __forceinline__ const uint4 *slice_chunk(const uint8_t *tile, int i, 
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, MODE == SEGMAP ? 2 : 1)
 gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    ChainSmem &s = *reinterpret_cast<ChainSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    using TM = Tm<MODE>;
+    using Stg = Stage<MODE>;
+    ChainSmem<MODE> &s = *reinterpret_cast<ChainSmem<MODE> *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const GdnArgs &p = a.g;
     const int seg = blockIdx.x, bh = blockIdx.y;
     // the segment maps: part A (blockIdx.z 0) runs the chain from the identity with Up = 0,
@@ -141,7 +155,7 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     if (warp == WARP_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          ptx::smem_u32(&s.tmem_slot)),
-                     "r"(TM_COLS)
+                     "r"(TM::COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -160,13 +174,13 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
             for (; k < nc; ++k) {
                 const int st = k % NSTG;
                 if (k >= NSTG && !wait_bar(EMPTY0 + 8 * st, (uint32_t)((k - NSTG) / NSTG) & 1u, abort_flag, p.err)) break;
-                Stage &sg = s.st[st];
+                Stg &sg = s.st[st];
                 const uint32_t full = FULL0 + 8 * st;
                 ptx::mbar_expect_tx(full, TX);
                 const long c = c_begin + k;
                 const int trow = (int)(((long)bh * a.nch + c) * D);
                 if (MODE == REPLAY) ptx::tma_load_2d(ptx::smem_u32(sg.QW), &maps.Q, 0, trow, full);
-                ptx::tma_load_2d(ptx::smem_u32(sg.QW + W_OFF), &maps.W, 0, trow, full);
+                ptx::tma_load_2d(ptx::smem_u32(sg.QW + Stg::W_OFF), &maps.W, 0, trow, full);
                 // K rows past a ragged last chunk belong to the next head (or are zero-filled
                 // past the tensor): U diag(ek) is zero there, so they add nothing
                 const int krow = (int)(krow0 + c * C);
@@ -197,23 +211,23 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
             bool ok = true;
             for (int k = 0; k < nc && ok; ++k) {
                 const int st = k % NSTG;
-                Stage &sg = s.st[st];
+                Stg &sg = s.st[st];
                 ok = wait_bar(FULL0 + 8 * st, (uint32_t)(k / NSTG) & 1u, abort_flag, p.err) &&
                      wait_bar(S_READY, (uint32_t)k & 1u, abort_flag, p.err);
                 if (!ok) break;
                 tc::fence_after_sync();
-                const uint64_t d1 = tc::sw128_desc(ptx::smem_u32(sg.QW) + (MODE == REPLAY ? 0u : W_OFF), SLICE, 1024);
-                const uint32_t dcol = tmem + TM_D + (MODE == REPLAY ? 0u : 64u);
+                const uint64_t d1 = tc::sw128_desc(ptx::smem_u32(sg.QW), SLICE, 1024);
+                const uint32_t dcol = tmem + (MODE == REPLAY ? TM::D1 : TM::DW);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::umma_bf16_ts(dcol, tmem + TM_S + kk * 8, d1 + (uint64_t)((kk * 2048) >> 4), IDESC1, kk > 0 ? 1u : 0u);
+                    tc::umma_bf16_ts(dcol, tmem + TM::S + kk * 8, d1 + (uint64_t)((kk * 2048) >> 4), IDESC1, kk > 0 ? 1u : 0u);
                 tc::umma_commit(D_FULL);
                 if (!(ok = wait_bar(U_READY, (uint32_t)k & 1u, abort_flag, p.err))) break;
                 tc::fence_after_sync();
                 const uint64_t d2 = tc::sw128_desc(ptx::smem_u32(sg.Kt), KT_HALF, 1024);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::umma_bf16_ts(tmem + TM_DL, tmem + TM_U + kk * 8, d2 + (uint64_t)((kk * 2048) >> 4),
+                    tc::umma_bf16_ts(tmem + TM::DL, tmem + TM::U + kk * 8, d2 + (uint64_t)((kk * 2048) >> 4),
                                      IDESC2, kk > 0 ? 1u : 0u);
                 tc::umma_commit(DL_FULL);
                 tc::umma_commit(EMPTY0 + 8 * st);
@@ -233,10 +247,13 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
             for (int j = 0; j < D; ++j) sr[j] = 0.f;
         } else {
             // segment 0 starts from S0 (or zero) when it is the only one; otherwise every
-            // segment starts from its composed start state
-            const float *src = a.nseg > 1 ? a.Sseg + (((long)bh * a.nseg + seg) * D + i) * D
-                                          : (p.S0 ? p.S0 + ((long)bh * D + i) * D : nullptr);
-            if (src) {
+            // segment starts from its composed start state (stored transposed)
+            const float *src = a.nseg > 1 ? nullptr : (p.S0 ? p.S0 + ((long)bh * D + i) * D : nullptr);
+            if (a.nseg > 1) {
+                const float *st_t = a.Sseg + ((long)bh * a.nseg + seg) * D * D + i;
+#pragma unroll
+                for (int j = 0; j < D; ++j) sr[j] = st_t[(long)j * D];
+            } else if (src) {
                 const float4 *s4 = reinterpret_cast<const float4 *>(src);
 #pragma unroll
                 for (int j4 = 0; j4 < D / 4; ++j4) {
@@ -251,14 +268,14 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
         bool ok = true;
         for (int k = 0; k < nc; ++k) {
             const int st = k % NSTG;
-            const Stage &sg = s.st[st];
+            const Stg &sg = s.st[st];
             // the state row as bf16 pairs: A operand of S [Qt; W]^T
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[32];
+            for (int qt = 0; qt < 4; ++qt) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int m = 0; m < 32; ++m) pk[m] = tc::pack_bf16(sr[hf * 64 + 2 * m], sr[hf * 64 + 2 * m + 1]);
-                tc::tmem_st32(tl + TM_S + hf * 32, pk);
+                for (int m = 0; m < 16; ++m) pk[m] = tc::pack_bf16(sr[qt * 32 + 2 * m], sr[qt * 32 + 2 * m + 1]);
+                tc::tmem_st16(tl + TM::S + qt * 16, pk);
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
@@ -272,37 +289,30 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
             }
             tc::fence_after_sync();
             const float gam = sg.scal[0];
+            // in quarters of 16 tokens, to keep few registers live beside the state row
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t dw[32];
-                tc::tmem_ld32(tl + TM_D + 64 + hf * 32, dw);
-                float ek[32];
+            for (int qt = 0; qt < 4; ++qt) {
+                uint32_t dw[16];
+                tc::tmem_ld16(tl + TM::DW + qt * 16, dw);
+                uint32_t pk[8];
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 e4 = *reinterpret_cast<const float4 *>(&sg.scal[4 + hf * 32 + 4 * q4]);
-                    ek[4 * q4] = e4.x; ek[4 * q4 + 1] = e4.y; ek[4 * q4 + 2] = e4.z; ek[4 * q4 + 3] = e4.w;
-                }
-                uint32_t pk[16];
-                if (segA) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const float4 ea = *reinterpret_cast<const float4 *>(&sg.scal[4 + qt * 16 + c2 * 8]);
+                    const float4 eb = *reinterpret_cast<const float4 *>(&sg.scal[4 + qt * 16 + c2 * 8 + 4]);
+                    const float ek[8] = {ea.x, ea.y, ea.z, ea.w, eb.x, eb.y, eb.z, eb.w};
+                    uint32_t uw[4] = {0u, 0u, 0u, 0u};    // Up = 0 for the A part of the maps
+                    if (!segA) {
+                        const uint4 u = *slice_chunk(sg.Up, i, qt * 2 + c2);
+                        uw[0] = u.x; uw[1] = u.y; uw[2] = u.z; uw[3] = u.w;
+                    }
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        pk[m] = tc::pack_bf16(-ek[2 * m] * __uint_as_float(dw[2 * m]),
-                                              -ek[2 * m + 1] * __uint_as_float(dw[2 * m + 1]));
-                } else {
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const uint4 u = *slice_chunk(sg.Up, i, hf * 4 + c4);
-                        const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
-                            const int m = c4 * 4 + e;
-                            pk[m] = tc::pack_bf16(ek[2 * m] * (f.x - __uint_as_float(dw[2 * m])),
-                                                  ek[2 * m + 1] * (f.y - __uint_as_float(dw[2 * m + 1])));
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&uw[e]));
+                        pk[c2 * 4 + e] = tc::pack_bf16(ek[2 * e] * (f.x - __uint_as_float(dw[c2 * 8 + 2 * e])),
+                                                       ek[2 * e + 1] * (f.y - __uint_as_float(dw[c2 * 8 + 2 * e + 1])));
                     }
                 }
-                tc::tmem_st16(tl + TM_U + hf * 16, pk);
+                tc::tmem_st8(tl + TM::U + qt * 8, pk);
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
@@ -315,7 +325,7 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t dq[32];
-                    tc::tmem_ld32(tl + TM_D + hf * 32, dq);
+                    tc::tmem_ld32(tl + TM::D1 + hf * 32, dq);
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const uint4 u = *slice_chunk(sg.Op, i, hf * 4 + c4);
@@ -339,18 +349,22 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
             }
             tc::fence_after_sync();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t dl[32];
-                tc::tmem_ld32(tl + TM_DL + q * 32, dl);
+            for (int q = 0; q < 8; ++q) {
+                uint32_t dl[16];
+                tc::tmem_ld16(tl + TM::DL + q * 16, dl);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sr[q * 32 + j] = fmaf(gam, sr[q * 32 + j], __uint_as_float(dl[j]));
+                for (int j = 0; j < 16; ++j) sr[q * 16 + j] = fmaf(gam, sr[q * 16 + j], __uint_as_float(dl[j]));
             }
         }
         if (ok) {
             float *dst = nullptr;
-            if (segA) dst = a.Amap + (((long)bh * a.nseg + seg) * D + i) * D;
-            else if (segB) dst = a.Bmap + (((long)bh * a.nseg + seg) * D + i) * D;
-            else if (seg == a.nseg - 1 && p.S_out) dst = p.S_out + ((long)bh * D + i) * D;
+            if (segA || segB) {
+                // the map transposed (A_p^T is then the K-major operand of the composition's
+                // products); consecutive rows i make each store of a warp one 128-byte line
+                float *mt = (segA ? a.Amap : a.Bmap) + ((long)bh * a.nseg + seg) * D * D + i;
+#pragma unroll
+                for (int j = 0; j < D; ++j) mt[(long)j * D] = sr[j];
+            } else if (seg == a.nseg - 1 && p.S_out) dst = p.S_out + ((long)bh * D + i) * D;
             if (dst) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst);
 #pragma unroll
@@ -365,104 +379,184 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
     tc::fence_after_sync();
     if (warp == WARP_MMA) {
         __syncwarp();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM::COLS)
                      : "memory");
     }
 }
 
 // -----------------------------------------------------------------------------------------
-// compose: S_0 = S0, S_{p+1} = S_p A_p + B_p, fp32 on the CUDA cores. Rows of S are
-// independent: a CTA owns CR rows of one head. Each step's A_p (64 KB) and the CTA's rows of
-// B_p arrive by bulk copy into one of two buffers, the next step's while this one computes;
-// a thread owns one key column j of four of the rows.
+// compose: S_0 = S0, S_{p+1} = S_p A_p + B_p on the tensor cores, one CTA per head.
+// S_p stays in tensor memory in fp32 and is the A operand of the next product directly
+// (kind::tf32, A from tensor memory); A_p arrives by TMA as the K-major B operand (the segment
+// maps store it transposed, [j][k]); the accumulator is set to B_p first (tcgen05.st), so the
+// product adds onto it. Two column regions of 128 alternate: S_p in one, S_{p+1} built in the
+// other. Each S_{p+1} is copied out to the start states the replay reads while the next
+// product runs. Warps 0-3: thread i owns row i (TMEM lane i); warp 4: TMEM owner, TMA
+// producer and MMA issuer (one thread).
 // -----------------------------------------------------------------------------------------
-constexpr int CR = 8;
-constexpr int COMPOSE_THREADS = 256;
+constexpr int COMPOSE_THREADS = 160;
+constexpr uint32_t AT_BOX = 128 * 128;           // [128 j][32 k] fp32, 128-byte swizzle: 16 KB
 struct ComposeSmem {
-    float A[2][D * D];
-    float Bm[2][CR * D];
-    alignas(16) float srow[D][CR];         // S_p rows of this CTA, transposed ([k][r])
-    alignas(8) uint64_t bar[2];
+    alignas(1024) uint8_t At[2][4 * AT_BOX];     // A_p^T, K-major (k along the 128-byte rows)
+    alignas(8) uint64_t full[2];                 // A_p^T landed
+    alignas(8) uint64_t empty[2];                // its product completed
+    alignas(8) uint64_t b_ready;                 // B_p stored into the accumulator (count 128)
+    alignas(8) uint64_t d_full;                  // S_{p+1} complete
+    uint32_t tmem_slot;
     int abort_flag;
 };
 
 __global__ void __launch_bounds__(COMPOSE_THREADS, 1)
-gdn_compose(const ChainArgs a)
+gdn_compose_tc(const __grid_constant__ CUtensorMap mat, const ChainArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    ComposeSmem &s = *reinterpret_cast<ComposeSmem *>(((uintptr_t)smem_raw + 127) & ~(uintptr_t)127);
+    ComposeSmem &s = *reinterpret_cast<ComposeSmem *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const GdnArgs &p = a.g;
-    const int bh = blockIdx.y, r0 = blockIdx.x * CR;
-    const int tid = threadIdx.x, j = tid & (D - 1), rh = tid >> 7;   // rows r0 + 4 rh .. + 3
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nmaps = a.nseg - 1;                // the launch has nseg > 1
     volatile int *abort_flag = (volatile int *)&s.abort_flag;
-    const uint32_t bar0 = ptx::smem_u32(&s.bar[0]);
-    constexpr uint32_t TX = D * D * 4 + CR * D * 4;
-    auto issue = [&](int sp) {             // one thread: A_sp and this CTA's rows of B_sp
-        const uint32_t bar = bar0 + 8 * (sp & 1);
-        ptx::mbar_expect_tx(bar, TX);
-        ptx::bulk_load(ptx::smem_u32(s.A[sp & 1]), a.Amap + ((long)bh * a.nseg + sp) * D * D, D * D * 4, bar);
-        ptx::bulk_load(ptx::smem_u32(s.Bm[sp & 1]), a.Bmap + (((long)bh * a.nseg + sp) * D + r0) * D, CR * D * 4, bar);
-    };
+    const uint32_t FULL0 = ptx::smem_u32(&s.full[0]), EMPTY0 = ptx::smem_u32(&s.empty[0]);
+    const uint32_t B_READY = ptx::smem_u32(&s.b_ready), D_FULL = ptx::smem_u32(&s.d_full);
     if (tid == 0) {
-        ptx::mbar_init(bar0, 1);
-        ptx::mbar_init(bar0 + 8, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(FULL0 + 8 * i, 1);
+            ptx::mbar_init(EMPTY0 + 8 * i, 1);
+        }
+        ptx::mbar_init(B_READY, ROWS);
+        ptx::mbar_init(D_FULL, 1);
         s.abort_flag = 0;
         ptx::mbar_init_fence();
-        issue(0);                          // the launch has nseg > 1
     }
-    float cur[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = r0 + 4 * rh + r;
-        cur[r] = p.S0 ? p.S0[((long)bh * D + row) * D + j] : 0.f;
-        a.Sseg[(((long)bh * a.nseg) * D + row) * D + j] = cur[r];
+    if (warp == 4) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         ptx::smem_u32(&s.tmem_slot)),
+                     "r"(256)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    int issued = 1;
-    bool ok = true;
-    for (int sp = 0; sp + 1 < a.nseg; ++sp) {
-        // buffer (sp + 1) & 1 was last read in step sp - 1, which every thread has finished
-        if (tid == 0 && sp + 1 < a.nseg - 1) {
-            issue(sp + 1);
-            issued = sp + 2;
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s.tmem_slot;
+    const long map0 = (long)bh * a.nseg;         // this head's first map / start state
+
+    if (warp == 4) {
+        if (lane == 0) {
+            // A_p^T of map p: rows (map0 + p) * 128 .. of the [BH * nseg * 128][128] view
+            auto load = [&](int mp) {
+                const uint32_t full = FULL0 + 8 * (mp & 1);
+                ptx::mbar_expect_tx(full, 4 * AT_BOX);
+                for (int q = 0; q < 4; ++q)
+                    ptx::tma_load_2d(ptx::smem_u32(s.At[mp & 1]) + q * AT_BOX, &mat, 32 * q,
+                                     (int)((map0 + mp) * D), full);
+            };
+            load(0);
+            if (nmaps > 1) load(1);
+            int issued = nmaps > 1 ? 2 : 1;
+            constexpr uint32_t ID = tc::idesc_tf32(128, 128);
+            bool ok = true;
+            for (int mp = 0; mp < nmaps && ok; ++mp) {
+                const int st = mp & 1;
+                ok = wait_bar(FULL0 + 8 * st, (uint32_t)(mp >> 1) & 1u, abort_flag, p.err) &&
+                     wait_bar(B_READY, (uint32_t)mp & 1u, abort_flag, p.err);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t a_col = tmem + (uint32_t)(mp & 1) * 128u;         // S_p
+                const uint32_t d_col = tmem + (uint32_t)((mp + 1) & 1) * 128u;   // B_p, then S_{p+1}
+                const uint64_t bd = tc::sw128_desc(ptx::smem_u32(s.At[st]), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 8; ++kk)
+                    tc::umma_tf32_ts(d_col, a_col + kk * 8,
+                                     bd + (uint64_t)(((kk >> 2) * AT_BOX + (kk & 3) * 32) >> 4), ID, 1u);
+                tc::umma_commit(D_FULL);
+                tc::umma_commit(EMPTY0 + 8 * st);
+                if (mp + 2 < nmaps) {
+                    // the stage is free once this product completed
+                    if (!(ok = wait_bar(EMPTY0 + 8 * st, (uint32_t)(mp >> 1) & 1u, abort_flag, p.err))) break;
+                    load(mp + 2);
+                    issued = mp + 3;
+                }
+            }
+            if (*abort_flag) {
+                // a bounded wait expired somewhere: let the copies this CTA issued land
+                const long long t0 = clock64();
+                for (int mp = issued - 1; mp >= 0 && mp >= issued - 2; --mp)
+                    while (!ptx::mbar_try(FULL0 + 8 * (mp & 1), (uint32_t)(mp >> 1) & 1u) &&
+                           clock64() - t0 < (1LL << 31)) {}
+            }
         }
+    } else {
+        const int i = tid;                       // row i of S (TMEM lane i)
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        // start states, B maps: transposed, element (i, j) of matrix m at m * D * D + j * D + i
+        float *sseg = a.Sseg + map0 * D * D + i;
+        const float *bmap = a.Bmap + map0 * D * D + i;
+        // S_0: S0 or zero, into the start states and into columns [0, 128)
+        {
+            const float *src = p.S0 ? p.S0 + ((long)bh * D + i) * D : nullptr;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) s.srow[j][4 * rh + r] = cur[r];
-        __syncthreads();
-        ok = ptx::mbar_try(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u) ||
-             ptx::mbar_wait(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u, abort_flag, p.err, DEVERR_GDN_WAIT);
-        if (!__syncthreads_and(ok)) break;
-        const float *A = s.A[sp & 1];
-        // eight independent accumulators (four rows, even and odd k) keep the FMA chains short
-        float acc[2][4];
+            for (int q = 0; q < 8; ++q) {
+                float4 v[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            acc[0][r] = s.Bm[sp & 1][(4 * rh + r) * D + j];
-            acc[1][r] = 0.f;
+                for (int e = 0; e < 4; ++e)
+                    v[e] = src ? reinterpret_cast<const float4 *>(src)[4 * q + e] : make_float4(0.f, 0.f, 0.f, 0.f);
+                uint32_t u[16];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    u[4 * e] = __float_as_uint(v[e].x); u[4 * e + 1] = __float_as_uint(v[e].y);
+                    u[4 * e + 2] = __float_as_uint(v[e].z); u[4 * e + 3] = __float_as_uint(v[e].w);
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sseg[(long)(16 * q + e) * D] = __uint_as_float(u[e]);
+                tc::tmem_st16(tl + q * 16, u);
+            }
         }
-#pragma unroll 16
-        for (int k = 0; k < D; ++k) {
-            const float av = A[k * D + j];
-            const float4 sk = *reinterpret_cast<const float4 *>(&s.srow[k][4 * rh]);
-            acc[k & 1][0] = fmaf(sk.x, av, acc[k & 1][0]);
-            acc[k & 1][1] = fmaf(sk.y, av, acc[k & 1][1]);
-            acc[k & 1][2] = fmaf(sk.z, av, acc[k & 1][2]);
-            acc[k & 1][3] = fmaf(sk.w, av, acc[k & 1][3]);
+        // B_0's row i
+        float bnext[D];
+#pragma unroll
+        for (int j = 0; j < D; ++j) bnext[j] = bmap[(long)j * D];
+        for (int mp = 0; mp < nmaps; ++mp) {
+            // B_p into the accumulator columns (they held S_{p-1}, whose product completed)
+            const uint32_t dcol = tl + (uint32_t)((mp + 1) & 1) * 128u;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uint32_t u[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(bnext[16 * q + e]);
+                tc::tmem_st16(dcol + q * 16, u);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            ptx::mbar_arrive(B_READY);
+            // the next map's row loads while the product runs
+            if (mp + 1 < nmaps) {
+                const float *bn = bmap + (long)(mp + 1) * D * D;
+#pragma unroll
+                for (int j = 0; j < D; ++j) bnext[j] = bn[(long)j * D];
+            }
+            if (!__all_sync(0xffffffffu, wait_bar(D_FULL, (uint32_t)mp & 1u, abort_flag, p.err))) break;
+            tc::fence_after_sync();
+            // S_{p+1} out to the start states (it stays in tensor memory for the next product)
+            float *dst = sseg + (long)(mp + 1) * D * D;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tc::tmem_ld32(dcol + q * 32, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(long)(32 * q + e) * D] = __uint_as_float(v[e]);
+            }
         }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) cur[r] = acc[0][r] + acc[1][r];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-            a.Sseg[(((long)bh * a.nseg + sp + 1) * D + r0 + 4 * rh + r) * D + j] = cur[r];
-        __syncthreads();                   // srow and this buffer are free again
     }
-    if (!ok && tid == 0) {
-        // a bounded wait expired: let the copies in flight land before the CTA exits
-        const long long t0 = clock64();
-        for (int sp = issued - 1; sp >= 0 && sp >= issued - 2; --sp)
-            while (!ptx::mbar_try(bar0 + 8 * (sp & 1), (uint32_t)(sp >> 1) & 1u) && clock64() - t0 < (1LL << 31)) {}
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 4) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256)
+                     : "memory");
     }
 }
-static_assert(COMPOSE_THREADS == 2 * D && CR == 8, "a compose thread owns one key column of four rows");
 
 }  // namespace
 
@@ -535,16 +629,24 @@ cudaError_t launch_gdn_bf16_scan(const GdnArgs &g, const GdnWs2 &ws, cudaStream_
     if ((e = make_tmap_2d_bf16(&m.U, ws.Ut, out_rows, C, 64, D, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&m.O, ws.Ot, out_rows, C, 64, D, true)) != cudaSuccess) return e;
     if ((e = make_tmap_2d_bf16(&m.K, g.k, in_rows, D, 64, C, true)) != cudaSuccess) return e;
-    const size_t smem = sizeof(ChainSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
+    // the segment maps' A parts, transposed: [BH * nseg * 128 j][128 k] fp32, boxes of 32 k
+    CUtensorMap mat;
+    if (a.nseg > 1 &&
+        (e = make_tmap_2d_f32(&mat, a.Amap, (uint64_t)BH * a.nseg * D, D, 32, D, true)) != cudaSuccess)
+        return e;
+    const size_t smem_map = sizeof(ChainSmem<SEGMAP>) + 1024, smem = sizeof(ChainSmem<REPLAY>) + 1024;
+    static_assert(2 * (sizeof(ChainSmem<SEGMAP>) + 2048) <= 228 * 1024, "two segment-map CTAs per SM");
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_map)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(gdn_chain_bf16<SEGMAP>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gdn_chain_bf16<REPLAY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    const size_t csmem = sizeof(ComposeSmem) + 128;
-    if ((e = cudaFuncSetAttribute(gdn_compose, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem)) != cudaSuccess) return e;
+    const size_t csmem = sizeof(ComposeSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(gdn_compose_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem)) != cudaSuccess) return e;
     if (a.nseg > 1) {
         // the maps of every segment but the last, then their composition
         const dim3 gm((unsigned)(a.nseg - 1), (unsigned)BH, 2);
-        gdn_chain_bf16<SEGMAP><<<gm, THREADS, smem, s>>>(m, a), note_launch();
-        gdn_compose<<<dim3(D / CR, (unsigned)BH), COMPOSE_THREADS, csmem, s>>>(a), note_launch();
+        gdn_chain_bf16<SEGMAP><<<gm, THREADS, smem_map, s>>>(m, a), note_launch();
+        gdn_compose_tc<<<(unsigned)BH, COMPOSE_THREADS, csmem, s>>>(mat, a), note_launch();
     }
     gdn_chain_bf16<REPLAY><<<dim3((unsigned)a.nseg, (unsigned)BH), THREADS, smem, s>>>(m, a), note_launch();
     return cudaGetLastError();

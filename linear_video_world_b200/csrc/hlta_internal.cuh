@@ -105,6 +105,9 @@ int record_error_impl(int st, const char *fmt, ...);
 // box_rows x box_cols, 128-byte swizzle or none.
 cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                               uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+// The same over fp32 (box_cols * 4 <= 128 with the swizzle).
+cudaError_t make_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                             uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 // The same over bytes (E4M3 codes), always with the 128-byte swizzle (box_cols <= 128).
 cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                             uint32_t box_cols, uint32_t box_rows);

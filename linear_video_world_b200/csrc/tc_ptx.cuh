@@ -1,8 +1,9 @@
 // tcgen05 wrappers for the tensor-memory kernels other than the forward attention kernel
 // (which keeps its own copies): fences around thread synchronisation, kind::f16 products with
-// A from shared or tensor memory and their commit to an mbarrier, the 128-byte-swizzle shared
-// memory descriptor, the kind::f16 instruction descriptor, tensor-memory loads and stores of
-// 32-bit columns, ex2 and bf16 packing.
+// A from shared or tensor memory and their commit to an mbarrier, kind::tf32 products with A
+// from tensor memory, the 128-byte-swizzle shared memory descriptor, the kind::f16 and
+// kind::tf32 instruction descriptors, tensor-memory loads and stores of 32-bit columns, ex2
+// and bf16 packing.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,6 +50,19 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         : "memory");
 }
 
+// kind::tf32 with the A operand read from tensor memory (M lanes x K fp32 columns, read as
+// tf32) and B from shared memory (fp32 elements read as tf32)
+__device__ __forceinline__ void umma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), sm_100 version bit.
 // lbo / sbo in bytes: K-major operands use sbo = 1024 (8 rows of 128 B) and an unused lbo;
 // MN-major operands use lbo = distance between 64-element column blocks, sbo = 1024.
@@ -68,6 +82,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
            ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::tf32: tf32 A and B (format 2), fp32 accumulator, both
+// operands K-major, M x N tile.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N)
+{
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 #define TC_REGS32(x)                                                                      \
@@ -112,6 +133,28 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&x)[64])
         "tcgen05.wait::ld.sync.aligned;"
         : TC_REGS32(x), TC_REGS32((x + 32))
         : "r"(taddr)
+        : "memory");
+}
+
+// 16 consecutive fp32 columns, load and wait in one statement
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&x)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]),
+          "=r"(x[7]), "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]),
+          "=r"(x[13]), "=r"(x[14]), "=r"(x[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&x)[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(x[0]), "r"(x[1]), "r"(x[2]), "r"(x[3]), "r"(x[4]), "r"(x[5]), "r"(x[6]), "r"(x[7])
         : "memory");
 }
 

@@ -1,4 +1,4 @@
-// Host helper: TMA tensor maps over row-major bf16 or byte tensors. The driver's
+// Host helper: TMA tensor maps over row-major bf16, fp32 or byte tensors. The driver's
 // encoder is fetched once through the runtime's entry-point query (no link-time libcuda).
 #include "hlta_internal.cuh"
 
@@ -47,6 +47,13 @@ cudaError_t make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t rows,
                               uint32_t box_cols, uint32_t box_rows, bool swizzle128)
 {
     return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, box_cols,
+                     box_rows, swizzle128);
+}
+
+cudaError_t make_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                             uint32_t box_cols, uint32_t box_rows, bool swizzle128)
+{
+    return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, box_cols,
                      box_rows, swizzle128);
 }
 
