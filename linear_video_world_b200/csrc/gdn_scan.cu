@@ -573,16 +573,16 @@ int gdn_scan_segment_len(long BH, long nch)
 int gdn_scan_segments_beside(long BH, long nch, double attn_flop)
 {
     // Estimates from measurements on the B200 at 480P: the softmax launches run at about
-    // 8e8 FLOP per microsecond; one chunk step of the chain takes about 3 us when the chains
+    // 8e8 FLOP per microsecond; one chunk step of the chain takes about 2 us when the chains
     // of few heads run beside them. One segment is a single pass over the chunks; s > 1
     // segments are two passes over ceil(nch / s) chunks (the maps, then the replay) plus s
-    // composition steps of a few microseconds. The fewest segments whose chain ends within
+    // composition steps of about 3 us. The fewest segments whose chain ends within
     // the softmax branches' time beside the GDN branch (about 1.15 times their time alone,
     // measured: they share the SMs with the chunk preparation and the chain) are taken: every
     // extra segment occupies more SMs the softmax branches could use.
     const long seg_lat = gdn_scan_segment_len(BH, nch);
     const long max_seg = (nch + seg_lat - 1) / seg_lat;
-    const double attn_us = 1.15 * attn_flop / 8.0e8, chunk_us = 3.0, compose_us = 5.0;
+    const double attn_us = 1.15 * attn_flop / 8.0e8, chunk_us = 2.0, compose_us = 3.0;
     for (long s = 1; s < max_seg; ++s) {
         const double lat = s == 1 ? chunk_us * (double)nch
                                   : 2.0 * chunk_us * (double)((nch + s - 1) / s) + compose_us * (double)s;

@@ -2,9 +2,10 @@
 each owning a share of independent units, with outputs gathered only when asked.
 
 The operator has no exchange step between its units: the rollouts of a streaming cache evolve
-independently (zhichai.net blog, section 2.3: streaming tokens; the pages report rollouts on
-several A800s without describing the split), and so do the heads of the hybrid call (each head
-is one branch over its own q, k, v). So a node shards them with no collective on the data
+independently (zhichai.net blog, section 2.3: streaming tokens), and so do the heads of the
+hybrid call (each head is one branch over its own q, k, v). The researchpapers.dev summary of
+Kairos reports a 480P rollout on four A800s (its results list, inference latency) without
+describing the split. So a node shards them with no collective on the data
 path: every rank runs the library's kernels on its own slice, on its own GPU, from its own
 memory (no peer memory is ever an operand). When the caller wants every output on every rank,
 one all_gather (NCCL over NVLink on GPUs; gloo in the CPU tests) collects the local results,
