@@ -386,6 +386,30 @@ hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done);
  */
 hlta_status hlta_stream_frame_counter(hlta_stream_t c, int **f_dev);
 
+/*
+ * Checkpoint and resume of a streaming cache (a rollout paused and continued later, in this
+ * process or another one). A checkpoint is a flat byte image: a 64-byte header (magic
+ * "HLTC", format version 1, the cache's geometry, scale and element type, the frames a step
+ * may append (which fix the ring slot counts) and the number of frames appended, replays
+ * included) followed by the carried GDN state
+ * [B, Hg, d, d] float32 and the four rings (SWA K, SWA V, DSWA K, DSWA V, in the cache's
+ * layout). A cache resumed from it continues exactly as the saved one would have: the next
+ * steps give bit-identical outputs.
+ *
+ * hlta_stream_checkpoint_bytes: the image size of this cache (0 for a NULL cache).
+ * hlta_stream_save: writes the image to `dst` (host memory, pageable or pinned, at least
+ *   hlta_stream_checkpoint_bytes bytes, owned by the caller) after the work already enqueued
+ *   on `stream` (NULL: the legacy default stream); returns when the image is complete.
+ * hlta_stream_load: replaces the cache's state, rings and frame count with the image in
+ *   `src` (host memory, `bytes` long), in order on `stream`; returns when the copies are done.
+ *   HLTA_ERR_INVALID_ARG for a wrong magic, version or size, or an image of a cache created
+ *   with other arguments (the cache is then left unchanged).
+ * Neither call allocates device memory; both return HLTA_ERR_CUDA if a copy fails.
+ */
+size_t hlta_stream_checkpoint_bytes(hlta_stream_t c);
+hlta_status hlta_stream_save(hlta_stream_t c, void *dst, size_t bytes, void *stream);
+hlta_status hlta_stream_load(hlta_stream_t c, const void *src, size_t bytes, void *stream);
+
 /* Frees the cache. Synchronizes the device first. */
 hlta_status hlta_stream_destroy(hlta_stream_t c);
 

@@ -57,6 +57,9 @@ def _load() -> ctypes.CDLL:
         "hlta_stream_state": (I, [P, ctypes.POINTER(P), ctypes.POINTER(I)]),
         "hlta_stream_destroy": (I, [P]),
         "hlta_stream_frame_counter": (I, [P, ctypes.POINTER(P)]),
+        "hlta_stream_checkpoint_bytes": (Z, [P]),
+        "hlta_stream_save": (I, [P, P, Z, P]),
+        "hlta_stream_load": (I, [P, P, Z, P]),
         "hlta_rope": (I, [P, P, I, I, I, I, L, I, I, F, I, I, I, P]),
         "hlta_fp8_quantize_rows": (I, [P, P, I, I, L, I, L, I, P, P, P]),
         "hlta_fp8_quantize_channels": (I, [P, I, I, L, I, P, P, P]),
@@ -480,7 +483,7 @@ def hybrid(q, k, v, a, b, Hs, Hd, Hg, T, N, w_swa, w_dswa, r, S0=None, chunk=64,
 
 class Stream:
     """Streaming cache (hlta_stream_create_ex / _step / _step_frames / _state /
-    _frame_counter / _destroy). A step may be captured into a CUDA graph and replayed for the
+    _frame_counter / _checkpoint_bytes / _save / _load / _destroy). A step may be captured into a CUDA graph and replayed for the
     following frames: the frame index lives in a device counter that every step advances."""
 
     def __init__(self, B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk=64, scale=0.0,
@@ -520,6 +523,22 @@ class Stream:
         ptr = ctypes.c_void_p()
         _check(_lib.hlta_stream_frame_counter(self._h, ctypes.byref(ptr)))
         return ptr.value
+
+    def checkpoint_bytes(self):
+        return int(_lib.hlta_stream_checkpoint_bytes(self._h))
+
+    def save(self, stream=None):
+        """The cache's checkpoint image (hlta_stream_save) as a uint8 numpy array."""
+        import numpy as np
+        buf = np.empty(self.checkpoint_bytes(), dtype=np.uint8)
+        _check(_lib.hlta_stream_save(self._h, buf.ctypes.data, buf.nbytes, _stream(stream)))
+        return buf
+
+    def load(self, image, stream=None):
+        """Resume from a checkpoint image (hlta_stream_load)."""
+        import numpy as np
+        buf = np.ascontiguousarray(image, dtype=np.uint8)
+        _check(_lib.hlta_stream_load(self._h, buf.ctypes.data, buf.nbytes, _stream(stream)))
 
     def state_tensor(self):
         """A torch copy of the carried state [B, Hg, d, d] fp32 (ordered on the current stream)."""

@@ -249,7 +249,7 @@ void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 unsigned int *device_error_word()
 {
-    DeviceCtx *c;
+    DeviceCtx *c = nullptr;
     return device_ctx(&c) == HLTA_OK ? c->err : nullptr;
 }
 
@@ -815,6 +815,123 @@ hlta_status hlta_stream_state(hlta_stream_t c, float **S_dev, int *frames_done)
     if (!c) return fail(HLTA_ERR_INVALID_ARG, "null cache");
     if (S_dev) *S_dev = c->S;
     if (frames_done) *frames_done = c->frames;
+    return HLTA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// the checkpoint image's header: 64 bytes, then the state and the four rings
+struct CkptHeader {
+    char magic[4];
+    int32_t version;
+    int32_t B, Hs, Hd, Hg, N, d, w_swa, w_dswa, r, chunk, dt, max_frames;
+    int32_t frames;
+    float scale;
+};
+static_assert(sizeof(CkptHeader) == 64, "checkpoint header is 64 bytes");
+constexpr char CKPT_MAGIC[4] = {'H', 'L', 'T', 'C'};
+
+struct CkptPart { void *p; size_t bytes; };
+
+// the device buffers of a cache in image order (absent branches have 0 bytes)
+void ckpt_parts(const hlta_stream *c, CkptPart (&parts)[5])
+{
+    const size_t el = c->dt == HLTA_BF16 ? 2 : 4;
+    const size_t frame = (size_t)c->N * c->d * el;
+    const size_t bs = (size_t)c->B * c->Hs * c->slots_s * frame, bd = (size_t)c->B * c->Hd * c->slots_d * frame;
+    parts[0] = {c->S, c->Hg ? (size_t)c->B * c->Hg * c->d * c->d * sizeof(float) : 0};
+    parts[1] = {c->ks, bs};
+    parts[2] = {c->vs, bs};
+    parts[3] = {c->kd, bd};
+    parts[4] = {c->vd, bd};
+}
+
+CkptHeader ckpt_header(const hlta_stream *c, int frames)
+{
+    CkptHeader h;
+    memcpy(h.magic, CKPT_MAGIC, 4);
+    h.version = 1;
+    h.B = c->B; h.Hs = c->Hs; h.Hd = c->Hd; h.Hg = c->Hg; h.N = c->N; h.d = c->d;
+    h.w_swa = c->w_swa; h.w_dswa = c->w_dswa; h.r = c->r; h.chunk = c->chunk; h.dt = (int32_t)c->dt;
+    h.max_frames = c->max_frames; h.frames = frames; h.scale = c->scale;
+    return h;
+}
+
+hlta_status ckpt_device(const hlta_stream *c)
+{
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (dev != c->device) return fail(HLTA_ERR_INVALID_ARG, "cache lives on device %d, current device is %d", c->device, dev);
+    return HLTA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t hlta_stream_checkpoint_bytes(hlta_stream_t c)
+{
+    if (!c) return 0;
+    CkptPart parts[5];
+    ckpt_parts(c, parts);
+    size_t n = sizeof(CkptHeader);
+    for (const CkptPart &pt : parts) n += pt.bytes;
+    return n;
+}
+
+hlta_status hlta_stream_save(hlta_stream_t c, void *dst, size_t bytes, void *stream)
+{
+    if (!c || !dst) return fail(HLTA_ERR_INVALID_ARG, "null argument");
+    const size_t need = hlta_stream_checkpoint_bytes(c);
+    if (bytes < need) return fail(HLTA_ERR_INVALID_ARG, "checkpoint buffer too small: need %zu bytes, got %zu", need, bytes);
+    hlta_status st;
+    if ((st = ckpt_device(c)) != HLTA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    int frames = 0;
+    cudaError_t e = cudaMemcpyAsync(&frames, c->fdev, sizeof(int), cudaMemcpyDeviceToHost, s);
+    CkptPart parts[5];
+    ckpt_parts(c, parts);
+    size_t off = sizeof(CkptHeader);
+    for (const CkptPart &pt : parts) {
+        if (e == cudaSuccess && pt.bytes) e = cudaMemcpyAsync((char *)dst + off, pt.p, pt.bytes, cudaMemcpyDeviceToHost, s);
+        off += pt.bytes;
+    }
+    const cudaError_t es = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = es;
+    if (e != cudaSuccess) return cuda_fail(e, "checkpoint copy");
+    const CkptHeader h = ckpt_header(c, frames);
+    memcpy(dst, &h, sizeof h);
+    return HLTA_OK;
+}
+
+hlta_status hlta_stream_load(hlta_stream_t c, const void *src, size_t bytes, void *stream)
+{
+    if (!c || !src) return fail(HLTA_ERR_INVALID_ARG, "null argument");
+    const size_t need = hlta_stream_checkpoint_bytes(c);
+    if (bytes != need) return fail(HLTA_ERR_INVALID_ARG, "checkpoint size %zu does not match this cache's %zu bytes", bytes, need);
+    CkptHeader h;
+    memcpy(&h, src, sizeof h);
+    if (memcmp(h.magic, CKPT_MAGIC, 4) != 0 || h.version != 1)
+        return fail(HLTA_ERR_INVALID_ARG, "not a streaming-cache checkpoint (magic or version)");
+    const CkptHeader mine = ckpt_header(c, h.frames);
+    if (memcmp(&h, &mine, sizeof h) != 0 || h.frames < 0)
+        return fail(HLTA_ERR_INVALID_ARG, "checkpoint of a cache created with other arguments");
+    hlta_status st;
+    if ((st = ckpt_device(c)) != HLTA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int frames = h.frames;
+    cudaError_t e = cudaMemcpyAsync(c->fdev, &frames, sizeof(int), cudaMemcpyHostToDevice, s);
+    CkptPart parts[5];
+    ckpt_parts(c, parts);
+    size_t off = sizeof(CkptHeader);
+    for (const CkptPart &pt : parts) {
+        if (e == cudaSuccess && pt.bytes) e = cudaMemcpyAsync(pt.p, (const char *)src + off, pt.bytes, cudaMemcpyHostToDevice, s);
+        off += pt.bytes;
+    }
+    const cudaError_t es = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = es;
+    if (e != cudaSuccess) return cuda_fail(e, "checkpoint copy");
+    c->frames = frames;
     return HLTA_OK;
 }
 

@@ -111,6 +111,15 @@ def test_stream_create_validates_before_allocating(lib):
     assert out.value is None
 
 
+def test_stream_checkpoint_validates_on_host(lib):
+    import linear_video_world_b200 as h
+    buf = ctypes.create_string_buffer(64)
+    assert lib.hlta_stream_checkpoint_bytes(None) == 0
+    assert lib.hlta_stream_save(None, buf, 64, None) == h.HLTA_ERR_INVALID_ARG
+    assert lib.hlta_stream_load(None, buf, 64, None) == h.HLTA_ERR_INVALID_ARG
+    assert b"null" in lib.hlta_last_error()
+
+
 def test_fp8_entry_points_validate_on_host(lib):
     import linear_video_world_b200 as h
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
