@@ -26,7 +26,9 @@
 //   warps 9, 10      MMA issuers of sub-tile 0 / 1 (warp 9 owns the TMEM allocation). Each
 //                    walks every tile in the ring's order: for K of a tile its sub-tile needs,
 //                    S = Q K^T once the softmax freed the S buffer; for V, O += P V once P is in
-//                    shared memory; a slot is released by both warps
+//                    shared memory, committed in two halves of 64 keys so that the softmax can
+//                    store the next tile's first half of P while it forms the second; a slot is
+//                    released by both warps
 // Tensor memory: per sub-tile S (128 columns) and O (128). Shared memory: Q (64 KB), the ring
 // (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
 // O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
@@ -72,9 +74,10 @@ enum {
     B_SFULL = B_EMPTY + NSLOT,   // + sub-tile
     B_SFREE = B_SFULL + QT,      // + sub-tile: its softmax read S (count SOFTMAX_THREADS)
     B_PFULL = B_SFREE + QT,      // + sub-tile: P in shared memory (count SOFTMAX_THREADS)
-    B_PVDONE = B_PFULL + QT,     // + sub-tile
+    B_PVDONE = B_PFULL + QT,     // + sub-tile: P V complete
     B_ODONE = B_PVDONE + QT,     // + sub-tile: every product of the sub-tile has completed
-    NBARS = B_ODONE + QT
+    B_PVA = B_ODONE + QT,        // + sub-tile: the first half of P V (keys 0-63) complete
+    NBARS = B_PVA + QT
 };
 constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
 constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
@@ -112,6 +115,7 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
     float d;
@@ -230,6 +234,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             mbar_init(BAR(B_SFREE + q), SOFTMAX_THREADS);
             mbar_init(BAR(B_PFULL + q), SOFTMAX_THREADS);
             mbar_init(BAR(B_PVDONE + q), 1);
+            mbar_init(BAR(B_PVA + q), 1);
             mbar_init(BAR(B_ODONE + q), 1);
         }
         *abort_flag = 0;
@@ -336,10 +341,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                     const uint64_t dv = dvl0 + (uint64_t)((sl * KTILE) >> 4);
                     const int ksteps = (nkeys(t.jt) + 15) >> 4;
                     if (ksteps == BN / 16 && npv > 0) {
+                        // the first half of P (keys 0-63) is released once its products are
+                        // done, so the softmax can store the next tile's first half early
 #pragma unroll
                         for (int kk = 0; kk < BN / 16; ++kk) {
                             const uint64_t poff = (uint64_t)((((kk >> 2) * PHALF + (kk & 3) * 32) >> 4));
                             tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O, 1u);
+                            if (kk == BN / 32 - 1) tc::umma_commit(BAR(B_PVA + q));
                         }
                     } else {
                         for (int kk = 0; kk < ksteps; ++kk) {
@@ -347,6 +355,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                             tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
                                           (npv > 0 || kk > 0) ? 1u : 0u);
                         }
+                        tc::umma_commit(BAR(B_PVA + q));
                     }
                     tc::umma_commit(BAR(B_PVDONE + q));
                     tc::umma_commit(BAR(B_EMPTY + sl));
@@ -436,11 +445,31 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(negm, negm);
             float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             uint32_t pk[64];
+            auto store_half = [&](int half) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const uint32_t *sv = i < 32 ? sa : sb;
+                for (int ch = 0; ch < 8; ++ch)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     prow + (uint32_t)half * PHALF + ((((uint32_t)ch) ^ rx) << 4)),
+                                 "r"(pk[half * 32 + ch * 4]), "r"(pk[half * 32 + ch * 4 + 1]),
+                                 "r"(pk[half * 32 + ch * 4 + 2]), "r"(pk[half * 32 + ch * 4 + 3])
+                                 : "memory");
+            };
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float2 x = ffma2(make_float2(__uint_as_float(sa[2 * i]), __uint_as_float(sa[2 * i + 1])), sl2x2, nm2);
+                const float2 pp = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                ps2[i & 1] = fadd2(ps2[i & 1], pp);
+                pk[i] = tc::pack_bf16(pp.x, pp.y);
+            }
+            // the first half of the previous P V has completed: this tile's first half of P
+            // may go over it while the second half is formed (unless O needs rescaling first)
+            const bool resc = k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY);
+            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(B_PVA + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+            if (!resc) store_half(0);
+#pragma unroll
+            for (int i = 32; i < 64; ++i) {
                 const int j = i & 31;
-                const float2 x = ffma2(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), sl2x2, nm2);
+                const float2 x = ffma2(make_float2(__uint_as_float(sb[2 * j]), __uint_as_float(sb[2 * j + 1])), sl2x2, nm2);
                 const float2 pp = make_float2(tc::ex2(x.x), tc::ex2(x.y));
                 ps2[i & 1] = fadd2(ps2[i & 1], pp);
                 pk[i] = tc::pack_bf16(pp.x, pp.y);
@@ -448,7 +477,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             // the previous P V has completed (it read the P tile and accumulated into O)
             if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
             tc::fence_after_sync();
-            if (k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY)) {
+            if (resc) {
                 // the running max grew by more than 2^LAZY: rescale O before P V of this tile
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
@@ -463,15 +492,8 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             }
             // this row of the shared P tile (128-byte swizzle: the 16-byte chunk index XORed
             // with the row mod 8); masked keys give 0
-#pragma unroll
-            for (int half = 0; half < 2; ++half)
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                     prow + (uint32_t)half * PHALF + ((((uint32_t)ch) ^ rx) << 4)),
-                                 "r"(pk[half * 32 + ch * 4]), "r"(pk[half * 32 + ch * 4 + 1]),
-                                 "r"(pk[half * 32 + ch * 4 + 2]), "r"(pk[half * 32 + ch * 4 + 3])
-                                 : "memory");
+            if (resc) store_half(0);
+            store_half(1);
             lsum = lsum * alpha + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y));
             m = muse;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
