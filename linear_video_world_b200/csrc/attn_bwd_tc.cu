@@ -10,8 +10,9 @@
 //   dV  += P^T dO_j,  dK += dS^T Q_j                   (P^T and dS^T read from tensor memory)
 // dQ: the same with queries and keys exchanged (one CTA per 128-row query tile of a frame,
 // walking the 64-key tiles of its window; dQ += dS K_j).
-// The roles mirror the forward kernel (attn_tc.cu): the CTA's own 128-row tile takes the place
-// of its query sub-tile, the other side's tiles stream through a TMA ring like its key tiles,
+// The roles follow the first forward design (64-key tiles, P in tensor memory): the CTA's own
+// 128-row tile takes the place of its query sub-tile, the other side's tiles stream through a
+// TMA ring like its key tiles,
 // P^T / dS are written over their fp32 buffers as bf16 pairs (each half of the columns into the
 // first 16 of its own 32 fp32 columns, so the two warps of a lane quadrant never overwrite each
 // other's unread scores), and

@@ -1,5 +1,6 @@
-// Windowed softmax attention (SWA / DSWA / streaming step), bf16, head dim 128, on the sm_100a
-// tensor cores: 128-key tiles, two query sub-tiles per CTA, S decoupled from P.
+// Windowed softmax attention (SWA / DSWA / streaming step), head dim 128, on the sm_100a
+// tensor cores: 128-key tiles, two query sub-tiles per CTA, S decoupled from P. bf16 operands,
+// or E4M3 codes with fp32 scales (template flag F8, below).
 //
 // Exact attention by tiles with a running max and normaliser (llm-atlas long-context
 // explainer, section 03 "Flash Attention"); the key set of a query tile is the union of the
@@ -32,8 +33,20 @@
 // Tensor memory: per sub-tile S (128 columns) and O (128). Shared memory: Q (64 KB), the ring
 // (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
 // O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
-// denominator use the same stale max). Every mbarrier wait is bounded; on expiry the kernel
-// records DEVERR_ATTN_WAIT, every role stops, and the TMEM allocation is released.
+// denominator use the same stale max).
+//
+// E4M3 instantiation (hlta_window_fp8_fwd): q, k, v arrive as OCP E4M3 codes, one 128-byte
+// swizzled row per token, with fp32 scales: one per 128-row block of a head's query rows (one
+// per sub-tile), one per 64-key run of each key frame (two per 128-key tile), one per value
+// channel. Both products run as tcgen05.mma kind::f8f6f4, 32 elements of K per instruction
+// (four products per S and per P V instead of eight); Q, the ring tiles and P take half the
+// bytes, so the ring holds six tiles. The softmax scales each half of a tile's scores by
+// sl2 * s_q * s_k of its run, forms P = 2^(x - m + 4) with the reference max grown once it
+// rose by more than 2^4 (so P stays within [0, 256], inside E4M3's 448), rounds P to E4M3 codes
+// (four a word, key order), and the value channels' scales multiply the normalised output.
+//
+// Every mbarrier wait is bounded; on expiry the kernel records DEVERR_ATTN_WAIT, every role
+// stops, and the TMEM allocation is released.
 #include "hlta_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "tc_ptx.cuh"
@@ -54,36 +67,40 @@ constexpr int THREADS = 352;            // 8 softmax warps, TMA warp, two MMA wa
 constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr int SOFTMAX_THREADS = 128;    // per sub-tile
 constexpr uint32_t QHALF = BM * 128;    // [128 rows][64 cols] bf16: 16 KB
-constexpr uint32_t QTILE = 2 * QHALF;
 constexpr uint32_t KHALF = BN * 128;    // [128 keys][64 cols] bf16: 16 KB
-constexpr uint32_t KTILE = 2 * KHALF;
 constexpr uint32_t PHALF = BM * 128;    // P: [128 rows][64 keys] bf16: 16 KB
-constexpr uint32_t PTILE = 2 * PHALF;
 constexpr uint32_t TMEM_COLS = 512;     // S_0 @0, S_1 @128, O_0 @256, O_1 @384
 __host__ __device__ constexpr uint32_t TM_S(int q) { return (uint32_t)q * 128u; }
 __host__ __device__ constexpr uint32_t TM_O(int q) { return 256u + (uint32_t)q * 128u; }
 
-__host__ __device__ constexpr uint32_t SM_Q(int q) { return (uint32_t)q * QTILE; }
-__host__ __device__ constexpr uint32_t SM_SLOT(int i) { return QT * QTILE + (uint32_t)i * KTILE; }
-__host__ __device__ constexpr uint32_t SM_P(int q) { return QT * QTILE + NSLOT * KTILE + (uint32_t)q * PTILE; }
-constexpr uint32_t SM_BAR = QT * QTILE + NSLOT * KTILE + QT * PTILE;
-enum {
-    B_QFULL = 0,
-    B_FULL = 1,                  // + slot
-    B_EMPTY = B_FULL + NSLOT,    // + slot: both MMA warps done with it (count 2)
-    B_SFULL = B_EMPTY + NSLOT,   // + sub-tile
-    B_SFREE = B_SFULL + QT,      // + sub-tile: its softmax read S (count SOFTMAX_THREADS)
-    B_PFULL = B_SFREE + QT,      // + sub-tile: P in shared memory (count SOFTMAX_THREADS)
-    B_PVDONE = B_PFULL + QT,     // + sub-tile: P V complete
-    B_ODONE = B_PVDONE + QT,     // + sub-tile: every product of the sub-tile has completed
-    B_PVA = B_ODONE + QT,        // + sub-tile: the first half of P V (keys 0-63) complete
-    NBARS = B_PVA + QT
+// Shared-memory layout per element type. bf16: a Q sub-tile, a K or V tile and a P sub-tile
+// are two 128B-swizzled halves of 64 columns (32 KB); E4M3: one swizzled 128-byte row per
+// token or query row (16 KB), and the ring holds twice as many tiles.
+template <bool F8> struct Lay {
+    static constexpr uint32_t QTILE = F8 ? BM * 128u : 2 * QHALF;
+    static constexpr uint32_t KTILE = F8 ? BN * 128u : 2 * KHALF;
+    static constexpr uint32_t PTILE = F8 ? BM * 128u : 2 * PHALF;
+    static constexpr int NSLOT = F8 ? 6 : 3;    // ring slots (K and V tiles in consumption order)
+    static constexpr uint32_t SM_Q(int q) { return (uint32_t)q * QTILE; }
+    static constexpr uint32_t SM_SLOT(int i) { return QT * QTILE + (uint32_t)i * KTILE; }
+    static constexpr uint32_t SM_P(int q) { return QT * QTILE + NSLOT * KTILE + (uint32_t)q * PTILE; }
+    static constexpr uint32_t SM_BAR = QT * QTILE + NSLOT * KTILE + QT * PTILE;
+    static constexpr int B_QFULL = 0;
+    static constexpr int B_FULL = 1;                    // + slot
+    static constexpr int B_EMPTY = B_FULL + NSLOT;      // + slot: both MMA warps done with it (count 2)
+    static constexpr int B_SFULL = B_EMPTY + NSLOT;     // + sub-tile
+    static constexpr int B_SFREE = B_SFULL + QT;        // + sub-tile: its softmax read S (count SOFTMAX_THREADS)
+    static constexpr int B_PFULL = B_SFREE + QT;        // + sub-tile: P in shared memory (count SOFTMAX_THREADS)
+    static constexpr int B_PVDONE = B_PFULL + QT;       // + sub-tile: P V complete
+    static constexpr int B_ODONE = B_PVDONE + QT;       // + sub-tile: every product of the sub-tile has completed
+    static constexpr int B_PVA = B_ODONE + QT;          // + sub-tile: the first half of P V (keys 0-63) complete
+    static constexpr int NBARS = B_PVA + QT;
+    static constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
+    static constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
+    static constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
+    static constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;
+    static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 };
-constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
-constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
-constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
-constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 
 struct Params {
     int Hbr, q_Htot, q_h0, kv_Htot, kv_h0, kv_slots;
@@ -91,6 +108,8 @@ struct Params {
     int N, w, r, fq0;
     const int *fq0_dev;
     float sl2;                  // softmax scale * log2(e)
+    const float *qs, *ks, *vs;  // E4M3 scales: [heads][nqb], [heads][nkb], [heads][128]
+    int nqb, nkb;               // E4M3: query blocks of 128 rows; key runs of 64 (per frame slot)
     float *lse;
     __nv_bfloat16 *o;
     unsigned int *err;
@@ -114,6 +133,37 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
+}
+
+// kind::f8f6f4 product with both operands E4M3 in shared memory (32 elements of K per
+// instruction), and its instruction descriptor (E4M3 = format code 0, fp32 accumulator)
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// four E4M3 codes in one word, p0 in the lowest byte (key order along the row); round to
+// nearest even, saturating at 448
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r)
+        : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
+    return r;
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c)
@@ -183,17 +233,19 @@ __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
     return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
 }
 
+template <bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const Params p)
 {
+    using LY = Lay<F8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + SM_BAR;
+    const uint32_t bar0 = sbase + LY::SM_BAR;
     auto BAR = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    volatile int *abort_flag = (volatile int *)(smem + SM_ABORT);
-    uint32_t *tmem_slot = (uint32_t *)(smem + SM_TMEMSLOT);
+    volatile int *abort_flag = (volatile int *)(smem + LY::SM_ABORT);
+    uint32_t *tmem_slot = (uint32_t *)(smem + LY::SM_TMEMSLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
@@ -224,18 +276,18 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     auto nkeys = [&](int jt) { return min(BN, p.N - jt * BN); };
 
     if (threadIdx.x == 0) {
-        mbar_init(BAR(B_QFULL), 1);
-        for (int i = 0; i < NSLOT; ++i) {
-            mbar_init(BAR(B_FULL + i), 1);
-            mbar_init(BAR(B_EMPTY + i), 2);
+        mbar_init(BAR(LY::B_QFULL), 1);
+        for (int i = 0; i < LY::NSLOT; ++i) {
+            mbar_init(BAR(LY::B_FULL + i), 1);
+            mbar_init(BAR(LY::B_EMPTY + i), 2);
         }
         for (int q = 0; q < QT; ++q) {
-            mbar_init(BAR(B_SFULL + q), 1);
-            mbar_init(BAR(B_SFREE + q), SOFTMAX_THREADS);
-            mbar_init(BAR(B_PFULL + q), SOFTMAX_THREADS);
-            mbar_init(BAR(B_PVDONE + q), 1);
-            mbar_init(BAR(B_PVA + q), 1);
-            mbar_init(BAR(B_ODONE + q), 1);
+            mbar_init(BAR(LY::B_SFULL + q), 1);
+            mbar_init(BAR(LY::B_SFREE + q), SOFTMAX_THREADS);
+            mbar_init(BAR(LY::B_PFULL + q), SOFTMAX_THREADS);
+            mbar_init(BAR(LY::B_PVDONE + q), 1);
+            mbar_init(BAR(LY::B_PVA + q), 1);
+            mbar_init(BAR(LY::B_ODONE + q), 1);
         }
         *abort_flag = 0;
         mbar_init_fence();
@@ -261,20 +313,20 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     if (warp == WARP_TMA) {
         // ------------------------------- TMA producer -----------------------------------
         if (lane == 0) {
-            mbar_expect_tx(BAR(B_QFULL), QT * QTILE);
+            mbar_expect_tx(BAR(LY::B_QFULL), QT * LY::QTILE);
             for (int q = 0; q < QT; ++q) {
                 const int qrow = (int)(q_head + l0 + q * BM);
-                tma_load_2d(sbase + SM_Q(q), &tq, 0, qrow, BAR(B_QFULL));
-                tma_load_2d(sbase + SM_Q(q) + QHALF, &tq, 64, qrow, BAR(B_QFULL));
+                tma_load_2d(sbase + LY::SM_Q(q), &tq, 0, qrow, BAR(LY::B_QFULL));
+                if constexpr (!F8) tma_load_2d(sbase + LY::SM_Q(q) + QHALF, &tq, 64, qrow, BAR(LY::B_QFULL));
             }
             int it = 0;                                  // ring items issued
             bool ok = true;
             auto load = [&](const CUtensorMap *map, int row) -> bool {
-                const int sl = it % NSLOT;
-                if (it >= NSLOT && !wait_bar(BAR(B_EMPTY + sl), (uint32_t)((it / NSLOT) + 1) & 1u)) return false;
-                mbar_expect_tx(BAR(B_FULL + sl), KTILE);
-                tma_load_2d(sbase + SM_SLOT(sl), map, 0, row, BAR(B_FULL + sl));
-                tma_load_2d(sbase + SM_SLOT(sl) + KHALF, map, 64, row, BAR(B_FULL + sl));
+                const int sl = it % LY::NSLOT;
+                if (it >= LY::NSLOT && !wait_bar(BAR(LY::B_EMPTY + sl), (uint32_t)((it / LY::NSLOT) + 1) & 1u)) return false;
+                mbar_expect_tx(BAR(LY::B_FULL + sl), LY::KTILE);
+                tma_load_2d(sbase + LY::SM_SLOT(sl), map, 0, row, BAR(LY::B_FULL + sl));
+                if constexpr (!F8) tma_load_2d(sbase + LY::SM_SLOT(sl) + KHALF, map, 64, row, BAR(LY::B_FULL + sl));
                 ++it;
                 return true;
             };
@@ -286,9 +338,9 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             }
             if (*abort_flag) {
                 const long long t0 = clock64();
-                for (int ii = it - 1; ii >= 0 && ii >= it - NSLOT; --ii)
-                    while (!mbar_try(BAR(B_FULL + ii % NSLOT), (uint32_t)(ii / NSLOT) & 1u) && clock64() - t0 < (1LL << 31)) {}
-                while (!mbar_try(BAR(B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
+                for (int ii = it - 1; ii >= 0 && ii >= it - LY::NSLOT; --ii)
+                    while (!mbar_try(BAR(LY::B_FULL + ii % LY::NSLOT), (uint32_t)(ii / LY::NSLOT) & 1u) && clock64() - t0 < (1LL << 31)) {}
+                while (!mbar_try(BAR(LY::B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
             }
         }
     } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
@@ -296,49 +348,66 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         if (lane == 0) {
             const int q = warp - WARP_MMA;
             const int want = 1 << q;
-            constexpr uint32_t IDESC_S0 = tc::idesc_bf16(BM, 16, false, false) & ~(0x3Fu << 17);
-            constexpr uint32_t IDESC_O = tc::idesc_bf16(BM, D, false, true);
-            const uint64_t dq = tc::sw128_desc(sbase + SM_Q(q), 16, 1024);
-            const uint64_t dsl0 = tc::sw128_desc(sbase + SM_SLOT(0), 16, 1024);        // K-major (K)
-            const uint64_t dvl0 = tc::sw128_desc(sbase + SM_SLOT(0), KHALF, 1024);     // MN-major (V)
-            const uint64_t dp = tc::sw128_desc(sbase + SM_P(q), 16, 1024);
+            constexpr uint32_t IDESC_S0 = (F8 ? idesc_e4m3(BM, 16, false, false) : tc::idesc_bf16(BM, 16, false, false)) & ~(0x3Fu << 17);
+            constexpr uint32_t IDESC_O = F8 ? idesc_e4m3(BM, D, false, true) : tc::idesc_bf16(BM, D, false, true);
+            const uint64_t dq = tc::sw128_desc(sbase + LY::SM_Q(q), 16, 1024);
+            const uint64_t dsl0 = tc::sw128_desc(sbase + LY::SM_SLOT(0), 16, 1024);        // K-major (K)
+            const uint64_t dvl0 = tc::sw128_desc(sbase + LY::SM_SLOT(0), KHALF, 1024);     // MN-major (V)
+            const uint64_t dp = tc::sw128_desc(sbase + LY::SM_P(q), 16, 1024);
             const uint32_t s_tm = tmem + TM_S(q), o_tm = tmem + TM_O(q);
             int it = 0, ns = 0, npv = 0;
-            bool ok = wait_bar(BAR(B_QFULL), 0);
+            bool ok = wait_bar(BAR(LY::B_QFULL), 0);
             // K of tile u (ring item `it`): S = Q K^T once this sub-tile's softmax read the
             // previous S (N = the tile's keys rounded up to 16), then the slot released
             auto handle_k = [&](const Pos &u) -> bool {
-                const int sl = it % NSLOT;
-                if (!wait_bar(BAR(B_FULL + sl), (uint32_t)(it / NSLOT) & 1u)) return false;
+                const int sl = it % LY::NSLOT;
+                if (!wait_bar(BAR(LY::B_FULL + sl), (uint32_t)(it / LY::NSLOT) & 1u)) return false;
                 if (u.mask & want) {
-                    if (ns > 0 && !wait_bar(BAR(B_SFREE + q), (uint32_t)(ns - 1) & 1u)) return false;
+                    if (ns > 0 && !wait_bar(BAR(LY::B_SFREE + q), (uint32_t)(ns - 1) & 1u)) return false;
                     tc::fence_after_sync();
                     const int n16 = (nkeys(u.jt) + 15) & ~15;
                     const uint32_t idesc = IDESC_S0 | ((uint32_t)(n16 >> 3) << 17);
-                    const uint64_t dk = dsl0 + (uint64_t)((sl * KTILE) >> 4);
+                    const uint64_t dk = dsl0 + (uint64_t)((sl * LY::KTILE) >> 4);
+                    if constexpr (F8) {
+                        // 32 channels (32 bytes of the swizzled row) per instruction
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t off = (uint64_t)((((kk >> 2) * QHALF + (kk & 3) * 32) >> 4));
-                        const uint64_t koff = (uint64_t)((((kk >> 2) * KHALF + (kk & 3) * 32) >> 4));
-                        tc::umma_bf16(s_tm, dq + off, dk + koff, idesc, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            umma_f8(s_tm, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idesc, kk > 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t off = (uint64_t)((((kk >> 2) * QHALF + (kk & 3) * 32) >> 4));
+                            const uint64_t koff = (uint64_t)((((kk >> 2) * KHALF + (kk & 3) * 32) >> 4));
+                            tc::umma_bf16(s_tm, dq + off, dk + koff, idesc, kk > 0 ? 1u : 0u);
+                        }
                     }
-                    tc::umma_commit(BAR(B_SFULL + q));
-                    tc::umma_commit(BAR(B_EMPTY + sl));
+                    tc::umma_commit(BAR(LY::B_SFULL + q));
+                    tc::umma_commit(BAR(LY::B_EMPTY + sl));
                     ++ns;
                 } else {
-                    mbar_arrive(BAR(B_EMPTY + sl));
+                    mbar_arrive(BAR(LY::B_EMPTY + sl));
                 }
                 ++it;
                 return true;
             };
             // V of tile t: O += P V once P is in shared memory, then the slot released
             auto handle_v = [&](const Pos &t) -> bool {
-                const int sl = it % NSLOT;
-                if (!wait_bar(BAR(B_FULL + sl), (uint32_t)(it / NSLOT) & 1u)) return false;
+                const int sl = it % LY::NSLOT;
+                if (!wait_bar(BAR(LY::B_FULL + sl), (uint32_t)(it / LY::NSLOT) & 1u)) return false;
                 if (t.mask & want) {
-                    if (!wait_bar(BAR(B_PFULL + q), (uint32_t)npv & 1u)) return false;
+                    if (!wait_bar(BAR(LY::B_PFULL + q), (uint32_t)npv & 1u)) return false;
                     tc::fence_after_sync();
-                    const uint64_t dv = dvl0 + (uint64_t)((sl * KTILE) >> 4);
+                    const uint64_t dv = dvl0 + (uint64_t)((sl * LY::KTILE) >> 4);
+                    if constexpr (F8) {
+                        // 32 keys per instruction: 32 bytes of each P row, 32 V rows of 128 B
+                        const int ksteps = (nkeys(t.jt) + 31) >> 5;
+                        for (int kk = 0; kk < ksteps; ++kk) {
+                            umma_f8(o_tm, dp + (uint64_t)(kk * 2), dv + (uint64_t)((kk * 4096) >> 4), IDESC_O,
+                                    (npv > 0 || kk > 0) ? 1u : 0u);
+                            if (kk == 1 && ksteps == BN / 32) tc::umma_commit(BAR(LY::B_PVA + q));
+                        }
+                        if (ksteps < BN / 32) tc::umma_commit(BAR(LY::B_PVA + q));
+                    } else {
                     const int ksteps = (nkeys(t.jt) + 15) >> 4;
                     if (ksteps == BN / 16 && npv > 0) {
                         // the first half of P (keys 0-63) is released once its products are
@@ -347,7 +416,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         for (int kk = 0; kk < BN / 16; ++kk) {
                             const uint64_t poff = (uint64_t)((((kk >> 2) * PHALF + (kk & 3) * 32) >> 4));
                             tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O, 1u);
-                            if (kk == BN / 32 - 1) tc::umma_commit(BAR(B_PVA + q));
+                            if (kk == BN / 32 - 1) tc::umma_commit(BAR(LY::B_PVA + q));
                         }
                     } else {
                         for (int kk = 0; kk < ksteps; ++kk) {
@@ -355,13 +424,14 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                             tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
                                           (npv > 0 || kk > 0) ? 1u : 0u);
                         }
-                        tc::umma_commit(BAR(B_PVA + q));
+                        tc::umma_commit(BAR(LY::B_PVA + q));
                     }
-                    tc::umma_commit(BAR(B_PVDONE + q));
-                    tc::umma_commit(BAR(B_EMPTY + sl));
+                    }
+                    tc::umma_commit(BAR(LY::B_PVDONE + q));
+                    tc::umma_commit(BAR(LY::B_EMPTY + sl));
                     ++npv;
                 } else {
-                    mbar_arrive(BAR(B_EMPTY + sl));
+                    mbar_arrive(BAR(LY::B_EMPTY + sl));
                 }
                 ++it;
                 return true;
@@ -377,7 +447,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 have = next;
                 t = u;
             }
-            if (ok) tc::umma_commit(BAR(B_ODONE + q));
+            if (ok) tc::umma_commit(BAR(LY::B_ODONE + q));
         }
     } else {
         // ------------------------------- softmax ----------------------------------------
@@ -390,10 +460,20 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         const bool row_valid = lrow < p.q_rows;
         const int fq = fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t prow = sbase + SM_P(q) + (uint32_t)row * 128u;
+        const uint32_t prow = sbase + LY::SM_P(q) + (uint32_t)row * 128u;
         const uint32_t rx = (uint32_t)(row & 7);
-        const float sl2 = p.sl2;
-        constexpr float LAZY = 8.f;
+        // E4M3: the scores carry the Q block's scale (one per sub-tile; sub-tile 1 of a head's
+        // last CTA may lie past the last query block) and each 64-key run's K scale
+        const int kvh = b * p.kv_Htot + p.kv_h0 + h;
+        const int tpf64 = (p.N + 63) / 64;
+        float sl2 = p.sl2;
+        if constexpr (F8) {
+            const long qblk = l0 / BM + q;
+            sl2 = qblk < p.nqb ? p.sl2 * __ldg(p.qs + (long)(b * p.q_Htot + p.q_h0 + h) * p.nqb + qblk) : 0.f;
+        }
+        // log2 growth of the max before a rescale; E4M3: P = 2^(x - m + 4) stays within 2^8
+        constexpr float LAZY = F8 ? 4.f : 8.f;
+        constexpr float PBIAS = F8 ? 4.f : 0.f;
         const int faq = q == 0 ? fa0 : fa1, fbq = q == 0 ? fb0 : fb1;
         const bool qvalid = q == 0 || valid1;
         float m = -INFINITY, lsum = 0.f;
@@ -407,7 +487,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 if (fk > fbq) break;
                 jt = 0;
             }
-            if (!__all_sync(0xffffffffu, wait_bar(BAR(B_SFULL + q), (uint32_t)k & 1u))) { ok = false; break; }
+            float sla = sl2, slb = sl2;          // the scales of keys 0-63 and 64-127
+            if constexpr (F8) {
+                const long kb = (long)kvh * p.nkb + (long)(fk % p.kv_slots) * tpf64 + 2 * jt;
+                sla = sl2 * __ldg(p.ks + kb);
+                slb = 2 * jt + 1 < tpf64 ? sl2 * __ldg(p.ks + kb + 1) : sla;
+            }
+            if (!__all_sync(0xffffffffu, wait_bar(BAR(LY::B_SFULL + q), (uint32_t)k & 1u))) { ok = false; break; }
             tc::fence_after_sync();
             const int nv = nkeys(jt);
             const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
@@ -416,7 +502,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             tc::tmem_ld64(tlane + TM_S(q), sa);
             tc::tmem_ld64(tlane + TM_S(q) + 64, sb);
             tc::fence_before_sync();
-            mbar_arrive(BAR(B_SFREE + q));
+            mbar_arrive(BAR(LY::B_SFREE + q));
             // masked keys (past the frame's end, or a frame this row does not attend) become
             // -inf, so the exponentials below serve full, partial and masked tiles alike (the
             // warp takes the masking branch together: rok differs between rows only where the
@@ -435,16 +521,72 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 mx0 = fmax3(mx0, __uint_as_float(sa[2 * i]), __uint_as_float(sa[2 * i + 1]));
                 mx1 = fmax3(mx1, __uint_as_float(sb[2 * i]), __uint_as_float(sb[2 * i + 1]));
             }
-            const float mnew = rok ? fmaxf(m, fmaxf(mx0, mx1) * sl2) : m;
+            float mt;
+            if constexpr (F8) mt = fmaxf(mx0 * sla, mx1 * slb);
+            else mt = fmaxf(mx0, mx1) * sl2;
+            const float mnew = rok ? fmaxf(m, mt) : m;
             const bool need = rok && mnew > m + LAZY;
             const float muse = need ? mnew : m;
             const float alpha = (need && m != -INFINITY) ? tc::ex2(m - mnew) : 1.f;
             // P = 2^(s sl2 - m) as bf16 pairs, first into registers: the shared P tile is still
             // the A operand of the previous tile's P V until that product completes
-            const float negm = muse == -INFINITY ? 0.f : -muse;
-            const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(negm, negm);
+            const float negm = muse == -INFINITY ? 0.f : PBIAS - muse;
+            const float2 sl2x2 = make_float2(sla, sla), nm2 = make_float2(negm, negm);
             float2 ps2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
             uint32_t pk[64];
+            if constexpr (F8) {
+                // E4M3 codes, four keys a word: keys 0-63 in words 0-15 (the first four 16-byte
+                // chunks of the row), keys 64-127 in words 16-31
+                const float2 slb2 = make_float2(slb, slb);
+                auto store_half8 = [&](int half) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int ch = half * 4 + c;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                         prow + ((((uint32_t)ch) ^ rx) << 4)),
+                                     "r"(pk[ch * 4]), "r"(pk[ch * 4 + 1]), "r"(pk[ch * 4 + 2]), "r"(pk[ch * 4 + 3])
+                                     : "memory");
+                    }
+                };
+                auto quad8 = [&](const uint32_t *sv, int i, float2 scl) {
+                    const float2 xa = ffma2(make_float2(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])), scl, nm2);
+                    const float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])), scl, nm2);
+                    const float2 pa = make_float2(tc::ex2(xa.x), tc::ex2(xa.y));
+                    const float2 pb = make_float2(tc::ex2(xb.x), tc::ex2(xb.y));
+                    ps2[0] = fadd2(ps2[0], pa);
+                    ps2[1] = fadd2(ps2[1], pb);
+                    return pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
+                };
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = quad8(sa, i, sl2x2);
+                const bool resc = k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY);
+                if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(LY::B_PVA + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+                if (!resc) store_half8(0);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[16 + i] = quad8(sb, i, slb2);
+                if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(LY::B_PVDONE + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+                tc::fence_after_sync();
+                if (resc) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t orow[32];
+                        tc::tmem_ld32(tlane + TM_O(q) + cc * 32, orow);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
+                        tc::tmem_st32(tlane + TM_O(q) + cc * 32, orow);
+                    }
+                    tc::tmem_wait_st();
+                    tc::fence_before_sync();
+                    store_half8(0);
+                }
+                store_half8(1);
+                lsum = lsum * alpha + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y));
+                m = muse;
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(BAR(LY::B_PFULL + q));
+                ++k;
+                continue;
+            }
             auto store_half = [&](int half) {
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
@@ -464,7 +606,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             // the first half of the previous P V has completed: this tile's first half of P
             // may go over it while the second half is formed (unless O needs rescaling first)
             const bool resc = k >= 1 && __any_sync(0xffffffffu, need && m != -INFINITY);
-            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(B_PVA + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(LY::B_PVA + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
             if (!resc) store_half(0);
 #pragma unroll
             for (int i = 32; i < 64; ++i) {
@@ -475,7 +617,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 pk[i] = tc::pack_bf16(pp.x, pp.y);
             }
             // the previous P V has completed (it read the P tile and accumulated into O)
-            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(B_PVDONE + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
+            if (k >= 1 && !__all_sync(0xffffffffu, wait_bar(BAR(LY::B_PVDONE + q), (uint32_t)(k - 1) & 1u))) { ok = false; break; }
             tc::fence_after_sync();
             if (resc) {
                 // the running max grew by more than 2^LAZY: rescale O before P V of this tile
@@ -497,24 +639,36 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             lsum = lsum * alpha + ((ps2[0].x + ps2[0].y) + (ps2[1].x + ps2[1].y));
             m = muse;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(BAR(B_PFULL + q));
+            mbar_arrive(BAR(LY::B_PFULL + q));
             ++k;
         }
         // final: every product of the sub-tile has completed (a one-phase barrier its MMA warp
         // commits after its last issue); normalise O and store it
         const bool fin = ok && k >= 1 &&
-                         __all_sync(0xffffffffu, wait_bar(BAR(B_ODONE + q), 0u));
+                         __all_sync(0xffffffffu, wait_bar(BAR(LY::B_ODONE + q), 0u));
         if (fin) {
             tc::fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-            if (p.lse && row_valid) p.lse[q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
+            if (!F8 && p.lse && row_valid) p.lse[q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
             __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
+            const float4 *vsc = F8 ? reinterpret_cast<const float4 *>(p.vs + (long)kvh * D) : nullptr;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ov[32];
                 __syncwarp();
                 tc::tmem_ld32(tlane + TM_O(q) + cc * 32, ov);
                 if (row_valid) {
+                    if constexpr (F8) {
+                        // the value channels' scales (the same 32 floats for every lane)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 sv = __ldg(vsc + cc * 8 + i);
+                            ov[4 * i] = __float_as_uint(__uint_as_float(ov[4 * i]) * sv.x);
+                            ov[4 * i + 1] = __float_as_uint(__uint_as_float(ov[4 * i + 1]) * sv.y);
+                            ov[4 * i + 2] = __float_as_uint(__uint_as_float(ov[4 * i + 2]) * sv.z);
+                            ov[4 * i + 3] = __float_as_uint(__uint_as_float(ov[4 * i + 3]) * sv.w);
+                        }
+                    }
                     uint32_t pk2[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -538,32 +692,48 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     }
 }
 
-}  // namespace
-
-cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s)
+template <bool F8>
+cudaError_t launch_attn_tc2(const AttnArgs &a, cudaStream_t s)
 {
+    using LY = Lay<F8>;
     if (a.d != D) return cudaErrorNotSupported;
     cudaError_t e;
     const long q_total = (long)a.B * a.q_Htot * a.q_rows;
     const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
     if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
     CUtensorMap mq, mk, mv;
-    if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
-    if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    if (F8) {
+        // E4M3 codes: one 128-byte row per token, one box covers the row
+        if ((e = make_tmap_2d_u8(&mq, a.q, q_total, D, D, BM)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_u8(&mk, a.k, kv_total, D, D, BN)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_u8(&mv, a.v, kv_total, D, D, BN)) != cudaSuccess) return e;
+    } else {
+        if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+        if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+    }
     Params p;
     p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
     p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
     p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0; p.fq0_dev = a.fq0_dev;
     p.sl2 = a.scale * 1.4426950408889634f;
+    p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
+    p.nqb = (int)((a.q_rows + BM - 1) / BM);
+    p.nkb = a.kv_slots * ((a.N + 63) / 64);
     p.lse = a.lse;
     p.o = (__nv_bfloat16 *)a.o;
     p.err = a.err;
-    e = cudaFuncSetAttribute(attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (F8 && (!p.qs || !p.ks || !p.vs)) return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(attn_tc2_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
-    attn_tc2_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, p), note_launch();
+    attn_tc2_kernel<F8><<<grid, THREADS, LY::SMEM_BYTES, s>>>(mq, mk, mv, p), note_launch();
     return cudaGetLastError();
 }
+
+}  // namespace
+
+cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<false>(a, s); }
+cudaError_t launch_attn_fp8_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<true>(a, s); }
 
 }  // namespace hlta

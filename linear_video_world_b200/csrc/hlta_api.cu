@@ -350,7 +350,7 @@ hlta_status hlta_window_fp8_fwd(const void *q8, const float *q_scales, const voi
     a.ks = k_scales;
     a.vs = v_scales;
     if (B * H == 0) return HLTA_OK;
-    cudaError_t e = launch_attn_fp8_tc(a, (cudaStream_t)stream);
+    cudaError_t e = launch_attn_fp8_tc2(a, (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "FP8 window attention: unsupported shape");
     if (e != cudaSuccess) return cuda_fail(e, "FP8 window attention launch");
     return HLTA_OK;

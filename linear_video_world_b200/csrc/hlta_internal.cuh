@@ -116,7 +116,8 @@ cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, u
 cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
 // bf16 window attention: 128-key tiles, two query sub-tiles, P staged in shared memory (attn_tc2.cu)
 cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s);
-cudaError_t launch_attn_fp8_tc(const AttnArgs &a, cudaStream_t s);
+// the same two-tile design on E4M3 codes (attn_tc2.cu)
+cudaError_t launch_attn_fp8_tc2(const AttnArgs &a, cudaStream_t s);
 // E4M3 quantisation (bf16 input, d = 128): row blocks inside frames, and value channels
 cudaError_t launch_fp8_quantize_rows(const void *x, const float *shift, long BH, long L,
                                      long frame_rows, int block_rows, void *x8, float *scales,
