@@ -80,6 +80,14 @@ __device__ __forceinline__ float fast_ex2(float x)
     return y;
 }
 
+// fp32 -> tf32 (round to nearest, ties away), as the 32-bit operand of a tf32 product
+__device__ __forceinline__ uint32_t tf32_bits(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
 // 2-D tiled TMA store from shared memory (bulk-group completion)
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1)
 {
@@ -311,46 +319,71 @@ gdn_prep_tc(const __grid_constant__ Maps m, GdnArgs p, GdnWs2 ws)
         for (int t = 0; t < 16; ++t) s.A[(bb0 + t) * AP + bb0 + jj] = tcv[t];
     }
     __syncthreads();
-    // levels 2 and 3: T10 = -T11 (A10 T00) for the 32 x 32 blocks, then for the whole 64 x 64.
-    // Y = A10 T00 goes to the upper right 32 x 32 block of the array (above the diagonal, where
-    // T is zero and no level reads), so each product needs one barrier: T10 may overwrite A10
-    // as soon as every thread has passed the barrier after the first product.
+    // levels 2 and 3: T10 = -T11 (A10 T00) for the 32 x 32 blocks, then for the whole 64 x 64,
+    // as warp-level tf32 tensor-core products (m16n8k8, fp32 accumulation; the operands lose
+    // 13 bits of mantissa, far below the bf16 rounding T1 and T2 get next). Y = A10 T00 goes to
+    // the upper right 32 x 32 block of the array (above the diagonal, where T is zero and no
+    // level reads), so each product needs one barrier: T10 may overwrite A10 as soon as every
+    // thread has passed the barrier after the first product.
+    {
+        const int g = lane >> 2, t4 = lane & 3;
+        // c (rows r0.., cols n0.. of a 16 x 8 tile) += X[xr.., xc..] Y[yr.., yc..] over K
+        auto mma_tile = [&](float (&c)[4], const float *X, int xr, int xc, const float *Y, int yr, int yc, int K) {
 #pragma unroll
-    for (int lvl = 0; lvl < 2; ++lvl) {
-        const int bs = lvl == 0 ? 16 : 32;                     // size of T00, T11, A10
-        const int per = bs * bs / (lvl == 0 ? 64 : 128);       // outputs per thread: 4 or 8
-        const int blk = lvl == 0 ? (tid >> 6) : 0;             // which 32 x 32 block (level 2)
-        const int u = lvl == 0 ? (tid & 63) : tid;
-        const int r = u / (bs / per), c0 = (u % (bs / per)) * per;
-        const int o = blk * 32;                                 // block origin
-        float *yb = s.A + (16 * blk) * AP + 32 + 16 * blk;      // Y scratch: rows 0-31, cols 32-63
-        float y[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) y[c] = 0.f;
-#pragma unroll
-        for (int k = 0; k < bs; ++k) {                          // Y = A10 T00
-            const float av = s.A[(o + bs + r) * AP + o + k];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (c < per) y[c] = fmaf(av, s.A[(o + k) * AP + o + c0 + c], y[c]);
+            for (int k0 = 0; k0 < 32; k0 += 8) {
+                if (k0 >= K) break;
+                const uint32_t a0 = tf32_bits(X[(xr + g) * AP + xc + k0 + t4]);
+                const uint32_t a1 = tf32_bits(X[(xr + g + 8) * AP + xc + k0 + t4]);
+                const uint32_t a2 = tf32_bits(X[(xr + g) * AP + xc + k0 + t4 + 4]);
+                const uint32_t a3 = tf32_bits(X[(xr + g + 8) * AP + xc + k0 + t4 + 4]);
+                const uint32_t b0 = tf32_bits(Y[(yr + k0 + t4) * AP + yc + g]);
+                const uint32_t b1 = tf32_bits(Y[(yr + k0 + t4 + 4) * AP + yc + g]);
+                asm volatile(
+                    "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, "
+                    "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                    : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                    : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+            }
+        };
+        // store a 16 x 8 accumulator tile (times sgn) at rows r0.., cols n0.. of M
+        auto store_tile = [&](const float (&c)[4], float *M, int r0, int n0, float sgn) {
+            M[(r0 + g) * AP + n0 + 2 * t4] = sgn * c[0];
+            M[(r0 + g) * AP + n0 + 2 * t4 + 1] = sgn * c[1];
+            M[(r0 + g + 8) * AP + n0 + 2 * t4] = sgn * c[2];
+            M[(r0 + g + 8) * AP + n0 + 2 * t4 + 1] = sgn * c[3];
+        };
+        // level 2: warp w takes 32 x 32 block w >> 1 (origin o) and 8 columns (w & 1) of its
+        // 16 x 16 products; Y scratch at rows 16 blk.., cols 32 + 16 blk..
+        {
+            const int blk = warp >> 1, o = 32 * blk, n0 = 8 * (warp & 1);
+            float *yb = s.A + (16 * blk) * AP + 32 + 16 * blk;
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile(c, s.A, o + 16, o, s.A, o, o + n0, 16);          // Y = A10 T00
+            store_tile(c, yb, 0, n0, 1.f);
+            __syncthreads();
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile(d, s.A, o + 16, o + 16, yb, 0, n0, 16);          // T10 = -T11 Y
+            store_tile(d, s.A, o + 16, o + n0, -1.f);
+            __syncthreads();
         }
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            if (c < per) yb[r * AP + c0 + c] = y[c];
-        __syncthreads();
-#pragma unroll
-        for (int c = 0; c < 8; ++c) y[c] = 0.f;
-#pragma unroll
-        for (int k = 0; k < bs; ++k) {                          // T10 = -T11 Y
-            const float tv = s.A[(o + bs + r) * AP + o + bs + k];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                if (c < per) y[c] = fmaf(-tv, yb[k * AP + c0 + c], y[c]);
+        // level 3: warp w takes rows 16 (w >> 1).. and columns 16 (w & 1).. of the 32 x 32
+        // products (two 16 x 8 tiles); Y scratch at rows 0-31, cols 32-63
+        {
+            const int m0 = 16 * (warp >> 1), n0 = 16 * (warp & 1);
+            float *yb = s.A + 32;
+            float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile(c0, s.A, 32 + m0, 0, s.A, 0, n0, 32);            // Y = A10 T00
+            mma_tile(c1, s.A, 32 + m0, 0, s.A, 0, n0 + 8, 32);
+            store_tile(c0, yb, m0, n0, 1.f);
+            store_tile(c1, yb, m0, n0 + 8, 1.f);
+            __syncthreads();
+            float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_tile(d0, s.A, 32 + m0, 32, yb, 0, n0, 32);            // T10 = -T11 Y
+            mma_tile(d1, s.A, 32 + m0, 32, yb, 0, n0 + 8, 32);
+            store_tile(d0, s.A, 32 + m0, n0, -1.f);
+            store_tile(d1, s.A, 32 + m0, n0 + 8, -1.f);
+            __syncthreads();
         }
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            if (c < per) s.A[(o + bs + r) * AP + o + c0 + c] = y[c];
-        __syncthreads();
     }
     // T1 = T diag(b e^g) (threads 0-63) and T2 = T diag(b) (threads 64-127), bf16 [t][t'] tiles
     // over A once every row of T has been read (rows 0-31 stop at column 32: the Y scratch)
