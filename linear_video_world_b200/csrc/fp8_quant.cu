@@ -8,7 +8,8 @@
 //
 // Row blocks: each head is cut into frames of frame_rows rows and each frame into runs of
 // block_rows rows (the last run of a frame, and the last frame, may be short): the attention
-// kernel takes Q in 128-row blocks of the whole head and K in the 64-key tiles of each frame.
+// kernel takes Q in 128-row blocks of the whole head and K in 64-key runs of each frame (two
+// runs per 128-key tile).
 // Value channels: one scale per (head, channel) over all rows.
 //
 // HBM-bound: 2 bytes read and 1 byte written per element (the row kernel holds its block in

@@ -110,7 +110,7 @@ def test_hybrid_480p_long_sampled(h, orc):
 
 
 def test_hybrid_720p_long_geometry_sampled(h, orc):
-    """The 720P long rollout's geometry (T=61 frames of N=3600 tokens, L=219600: ragged 64-key
+    """The 720P long rollout's geometry (T=61 frames of N=3600 tokens, L=219600: ragged key
     tiles, row indices past 2^17; SWA w=3, DSWA w=4 r=6) on two heads per branch: softmax heads
     on sampled rows, the GDN heads over the whole 219600-token recurrence."""
     wl = hi.WORKLOADS["720p_long"].with_(Hs=2, Hd=2, Hg=2)
@@ -141,8 +141,8 @@ def test_stream_steps_equal_hybrid_bf16(h, orc):
 
 
 def test_stream_steps_streaming_workload_geometry_sampled(h, orc):
-    """The streaming workload's geometry: B=8 rollouts, frames of N=1560 tokens (64-key tiles
-    straddle frames), SWA w=3, DSWA w=4 r=6 (a ring of r(w-1)+1 = 19 frame slots), d=128, one
+    """The streaming workload's geometry: B=8 rollouts, frames of N=1560 tokens (key tiles
+    end partly filled at every frame), SWA w=3, DSWA w=4 r=6 (a ring of r(w-1)+1 = 19 frame slots), d=128, one
     head per branch. 26 single-frame steps from empty caches, so every ring slot is reused and
     the last eight steps see all DSWA taps. Each step's softmax outputs on sampled rows of
     every frame, every GDN output and the final state are compared with the oracle's hybrid
