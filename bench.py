@@ -602,9 +602,8 @@ def main():
     clocks = clk.stop()
     total_ms = allmax(ev0.elapsed_time(ev1))
     ms = total_ms / K
-    # SWA and DSWA run side by side from the fork (events 0 -> 1 and 0 -> 2)
-    swa_ms = statistics.mean(p[0].elapsed_time(p[1]) for p in prof)
-    dswa_ms = statistics.mean(p[0].elapsed_time(p[2]) for p in prof)
+    # SWA and DSWA heads share one attention launch, from the fork (event 0) to its end
+    # (events 1 and 2)
     attn_span_ms = statistics.mean(max(p[0].elapsed_time(p[1]), p[0].elapsed_time(p[2])) for p in prof)
     gdn_ms = statistics.mean(p[3].elapsed_time(p[4]) for p in prof)
     assert h.hlta_device_status() == 0
@@ -694,16 +693,16 @@ def main():
     h2d = sum(pin[n].numel() * pin[n].element_size() for n in "qkvab")
     d2h = o_host.numel() * o_host.element_size() + S_host.numel() * S_host.element_size()
 
-    # ---- the two softmax launches alone (no GDN branch sharing the SMs) --------------------
-    hs, hd = slice(0, wl.Hs), slice(wl.Hs, wl.Hs + wl.Hd)
-    sub = {n: (x_[:, hs].contiguous(), x_[:, hd].contiguous()) for n, x_ in (("q", q), ("k", k), ("v", v))}
-    o_s, o_d = torch.empty_like(sub["q"][0]), torch.empty_like(sub["q"][1])
+    # ---- the softmax heads alone (no GDN branch sharing the SMs) ---------------------------
+    # the SWA and DSWA heads as a hybrid call without GDN heads: the same single attention
+    # launch the step makes
+    hsd = slice(0, wl.Hs + wl.Hd)
+    sub = {n: x_[:, hsd].contiguous() for n, x_ in (("q", q), ("k", k), ("v", v))}
+    o_sd = torch.empty_like(sub["q"])
 
     def attn_only():
-        h.hlta_swa_fwd(sub["q"][0], sub["k"][0], sub["v"][0], o_s, wl.B, wl.Hs, wl.T, wl.N, wl.d,
-                       wl.w_swa, 0.0)
-        h.hlta_dswa_fwd(sub["q"][1], sub["k"][1], sub["v"][1], o_d, wl.B, wl.Hd, wl.T, wl.N, wl.d,
-                        wl.w_dswa, wl.r, 0.0)
+        h.hlta_hybrid_fwd(sub["q"], sub["k"], sub["v"], None, None, o_sd, None, None, wl.B, wl.Hs,
+                          wl.Hd, 0, wl.T, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r, wl.chunk, 0.0, None)
 
     for _ in range(3):
         attn_only()
@@ -715,7 +714,7 @@ def main():
     a1.record()
     torch.cuda.synchronize()
     attn_alone_ms = a0.elapsed_time(a1) / K
-    del sub, o_s, o_d
+    del sub, o_sd
 
     # ---- the GDN branch alone (its heads by themselves, all SMs to itself) -----------------
     gdn_alone_ms = None
@@ -760,17 +759,16 @@ def main():
     peak = float(pk.get("bf16_tflops"))
     tr = traffic_record("attn_tc2.cu")          # the bf16 window attention kernel
     tr8 = tr                                    # the E4M3 instantiation lives in the same file
-    roofline = {"bound": "tensor", "kernel": "attn_tc2_kernel (SWA + DSWA launches, side by side: "
-                                              "the span from their common start to the later end)",
+    roofline = {"bound": "tensor", "kernel": "attn_tc2_kernel (the SWA and DSWA heads in one persistent "
+                                              "launch, beside the GDN branch: from the step's start to "
+                                              "the launch's end)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"{pk_kind} bf16 dense, burst (the timed region is {total_ms:.0f} ms)",
-                "traffic": (tr["swa_bytes"] + tr["dswa_bytes"]) if tr else None}
+                "traffic": tr.get("hybrid_bytes") if tr else None}
     hbm = float(pk.get("hbm_gbs"))
     gdn_gbs = wk["gdn_bytes"] / (gdn_ms / 1e3) / 1e9
     detail = {
-        "swa_ms": swa_ms, "dswa_ms": dswa_ms, "attn_span_ms": attn_span_ms, "gdn_ms": gdn_ms,
-        "swa_tflops": wk["swa_flop"] / (swa_ms / 1e3) / 1e12,
-        "dswa_tflops": wk["dswa_flop"] / (dswa_ms / 1e3) / 1e12,
+        "attn_span_ms": attn_span_ms, "gdn_ms": gdn_ms,
         "gdn_gbs": gdn_gbs, "gdn_hbm_frac": gdn_gbs / hbm,
         "hbm_peak_gbs": hbm, "hbm_peak_kind": pk_kind,
         "attn_alone_ms": attn_alone_ms,
@@ -779,13 +777,13 @@ def main():
         "gdn_alone_ms": gdn_alone_ms,
         "gdn_alone_gbs": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 if gdn_alone_ms else None,
         "gdn_alone_hbm_frac": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 / hbm if gdn_alone_ms else None,
-        "note": "the three branches run side by side (GDN on a high-priority stream, DSWA beside "
-                "SWA); swa_ms and dswa_ms run from their common start, attn_span_ms to the later "
-                "end (the roofline's duration), all while sharing the SMs with the GDN branch; "
-                "attn_alone_* times the two softmax launches back to back by themselves against "
-                "the burst bf16 peak; gdn_alone_* times hlta_gdn_chunk_fwd on the GDN heads by "
-                "themselves (segment scan over all SMs). The GDN HBM fractions use the "
-                "algorithmic q/k/v/o + gate bytes of the GDN heads",
+        "note": "the GDN branch runs on a high-priority stream beside one persistent attention "
+                "launch over the SWA and DSWA heads, which leaves the GDN chain its SMs; "
+                "attn_span_ms runs from the step's start to the end of that launch (the "
+                "roofline's duration); attn_alone_* times the attention launch by itself "
+                "against the burst bf16 peak; gdn_alone_* times hlta_gdn_chunk_fwd on the GDN "
+                "heads by themselves (segment scan over all SMs). The GDN HBM fractions use "
+                "the algorithmic q/k/v/o + gate bytes of the GDN heads",
     }
     if stream_detail is not None:
         stream_detail["softmax_frac"] = stream_detail["softmax_tflops"] / peak

@@ -302,10 +302,13 @@ size_t hlta_hybrid_workspace_bytes(int B, int Hg, int T, int N, int d, int chunk
  * (each branch writes its own head range of o, in place).
  * q, k, v, o: [B, H, T*N, d] with H = Hs + Hd + Hg; a, b: [B, Hg, T*N] float32.
  * S0 / S_out: [B, Hg, d, d] float32 or NULL (as hlta_gdn_chunk_fwd).
- * The GDN branch runs on a library-owned stream of the highest priority and the DSWA branch
- * (when SWA heads are present too) on a second library-owned stream, both ordered after
- * `stream` by an event, so the branches overlap; the call still completes, in stream order,
- * on `stream` (later work on `stream` sees every output).
+ * The GDN branch runs on a library-owned stream of the highest priority, ordered after
+ * `stream` by an event, so the branches overlap. bf16: the SWA and DSWA heads run as one
+ * persistent attention launch on `stream`, started after the GDN chunk preparation, leaving
+ * the GDN chain its SMs; a second launch of the same kernel queued behind the chain on the GDN
+ * stream takes the units still left. fp32: the DSWA branch runs on a second library-owned
+ * stream beside the SWA branch. The call still completes, in stream order, on `stream` (later
+ * work on `stream` sees every output).
  */
 hlta_status hlta_hybrid_fwd(const void *q, const void *k, const void *v,
                             const float *a, const float *b, void *o,
@@ -418,8 +421,9 @@ hlta_status hlta_stream_destroy(hlta_stream_t c);
  * for results). `events` is NULL (off) or an array of 5 cudaEvent_t created by the caller on
  * the current device. While set, each hybrid call or streaming step records events[0] where
  * the branches fork (on the caller's stream, before any branch kernel), events[1] after the
- * SWA kernel (caller's stream), events[2] after the DSWA kernel (on the stream it ran on),
- * events[3] before and events[4] after the GDN kernels (on the GDN stream). The array is
+ * SWA kernel (caller's stream), events[2] after the DSWA kernel (on the stream it ran on; with
+ * bf16 both follow the one attention launch that serves both branches), events[3] before and
+ * events[4] after the GDN kernels (on the GDN stream). The array is
  * copied; the setting is process-wide and stays until changed.
  */
 hlta_status hlta_set_profile_events(void *const *events);

@@ -19,11 +19,16 @@
 // product N = 128, which halves the products one issuing thread sends per key compared with
 // 64-key tiles (one thread issues a tcgen05.mma in roughly a hundred cycles).
 //
-// One CTA = two 128-row query sub-tiles (256 consecutive query rows) of one head; 11 warps:
+// Persistent: one CTA per SM (at most), each taking units of work from a launch-wide counter
+// until none is left. A unit is two 128-row query sub-tiles (256 consecutive query rows) of
+// one head of one of up to two branches (the hybrid's SWA and DSWA heads share one launch);
+// units go head by head, the latest query rows of a head first (the longest key sets), so the
+// last units handed out are the shortest. 11 warps:
 //   warps 0-3 / 4-7  softmax of sub-tile 0 / 1, one thread per query row (its TMEM lane)
-//   warp 8           TMA producer: Q once, then K and V tiles of 128 keys through one ring of
-//                    three 32 KB slots, in the order K0, K1, V0, K2, V1, ... (the order the
-//                    MMA warps consume them)
+//   warp 8           TMA producer: takes the units and publishes each in shared memory; per
+//                    unit Q, then K and V tiles of 128 keys through one ring of three 32 KB
+//                    slots, in the order K0, K1, V0, K2, V1, ... (the order the MMA warps
+//                    consume them); the ring runs on from one unit to the next
 //   warps 9, 10      MMA issuers of sub-tile 0 / 1 (warp 9 owns the TMEM allocation). Each
 //                    walks every tile in the ring's order: for K of a tile its sub-tile needs,
 //                    S = Q K^T once the softmax freed the S buffer; for V, O += P V once P is in
@@ -34,6 +39,11 @@
 // (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
 // O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
 // denominator use the same stale max).
+// From one unit to the next: the producer loads the next Q once both issuers' last S of the
+// unit completed; an issuer's first P V of a unit (which overwrites O) waits until its softmax
+// read the previous unit's O; S, P and the ring's barriers keep counting across units. A
+// second launch of the same kernel may share the counter (CTAs that start late, on SMs another
+// kernel held); the last CTA to finish resets the counter.
 //
 // E4M3 instantiation (hlta_window_fp8_fwd): q, k, v arrive as OCP E4M3 codes, one 128-byte
 // swizzled row per token, with fp32 scales: one per 128-row block of a head's query rows (one
@@ -52,6 +62,8 @@
 #include "tc_ptx.cuh"
 
 #include <math.h>
+#include <algorithm>
+#include <atomic>
 
 namespace hlta {
 namespace {
@@ -62,10 +74,10 @@ constexpr int BM = 128;                 // query rows per sub-tile
 constexpr int QT = 2;                   // query sub-tiles per CTA
 constexpr int BN = 128;                 // keys per tile
 constexpr int D = 128;                  // head dim
-constexpr int NSLOT = 3;                // ring slots (K and V tiles in consumption order)
 constexpr int THREADS = 352;            // 8 softmax warps, TMA warp, two MMA warps
 constexpr int WARP_TMA = 8, WARP_MMA = 9;
 constexpr int SOFTMAX_THREADS = 128;    // per sub-tile
+constexpr int UNIT_READERS = 2 + 8;     // the two MMA warps and the eight softmax warps
 constexpr uint32_t QHALF = BM * 128;    // [128 rows][64 cols] bf16: 16 KB
 constexpr uint32_t KHALF = BN * 128;    // [128 keys][64 cols] bf16: 16 KB
 constexpr uint32_t PHALF = BM * 128;    // P: [128 rows][64 keys] bf16: 16 KB
@@ -94,22 +106,40 @@ template <bool F8> struct Lay {
     static constexpr int B_PVDONE = B_PFULL + QT;       // + sub-tile: P V complete
     static constexpr int B_ODONE = B_PVDONE + QT;       // + sub-tile: every product of the sub-tile has completed
     static constexpr int B_PVA = B_ODONE + QT;          // + sub-tile: the first half of P V (keys 0-63) complete
-    static constexpr int NBARS = B_PVA + QT;
-    static constexpr uint32_t SM_TMEMSLOT = SM_BAR + 8 * NBARS;
+    static constexpr int B_QFREE = B_PVA + QT;          // both issuers' last S of a unit done (count 2)
+    static constexpr int B_OFREE = B_QFREE + 1;         // + sub-tile: its epilogue read O (count SOFTMAX_THREADS)
+    static constexpr int B_UFULL = B_OFREE + QT;        // + unit slot: the next unit published (count 1)
+    static constexpr int B_UEMPTY = B_UFULL + 2;        // + unit slot: every role read it (count UNIT_READERS)
+    static constexpr int NBARS = B_UEMPTY + 2;
+    static constexpr uint32_t SM_UNIT = SM_BAR + 8 * NBARS;   // two published unit indices
+    static constexpr uint32_t SM_TMEMSLOT = SM_UNIT + 8;
     static constexpr uint32_t SM_ABORT = SM_TMEMSLOT + 4;
     static constexpr uint32_t SM_TOTAL = SM_ABORT + 4;
     static constexpr size_t SMEM_BYTES = SM_TOTAL + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
 };
 
+// One branch of a launch: its heads (queries at q_h0.. of the query tensor, keys and values at
+// kv_h0.. of its own key/value tensors), window and dilation.
+struct BranchP {
+    int Hbr, q_h0, kv_Htot, kv_h0, kv_slots, w, r;
+    int nkb;                    // E4M3: key runs of 64 per head (kv_slots * ceil(N / 64))
+    long kv_rows;
+    const float *ks, *vs;       // E4M3 scales: [heads][nkb], [heads][128]
+};
 struct Params {
-    int Hbr, q_Htot, q_h0, kv_Htot, kv_h0, kv_slots;
-    long q_rows, kv_rows;
-    int N, w, r, fq0;
+    BranchP br[2];
+    int nbr, B, Hsum;           // branches; batch; heads over the branches
+    int q_Htot;
+    long q_rows;
+    int N, fq0;
     const int *fq0_dev;
     float sl2;                  // softmax scale * log2(e)
-    const float *qs, *ks, *vs;  // E4M3 scales: [heads][nqb], [heads][nkb], [heads][128]
-    int nqb, nkb;               // E4M3: query blocks of 128 rows; key runs of 64 (per frame slot)
+    const float *qs;            // E4M3 query scales: [heads][nqb]
+    int nqb;                    // E4M3: query blocks of 128 rows
+    int nqt, nunits;            // query tiles of 256 rows per head; units = nqt * B * Hsum
+    int slot;                   // this launch's work counter (g_attn_sched)
+    int ctas_total;             // CTAs over the launches sharing the counter
     float *lse;
     __nv_bfloat16 *o;
     unsigned int *err;
@@ -218,25 +248,64 @@ __device__ __forceinline__ bool walk_step(const Walk &wk, Pos &c)
     }
     return c.valid = false;
 }
-__device__ __forceinline__ bool walk_next(const Walk &wk, Pos &c, int want)
-{
-    while (walk_step(wk, c)) {
-        if (c.mask & want) return true;
-        c.j += wk.tpf - 1 - c.jt;
-        c.jt = wk.tpf - 1;
-    }
-    return false;
-}
 __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
 {
     const int dist = fq - fk;
     return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
 }
 
+// Work counters of the persistent launches, one pair per launch slot: [0] the next unit to
+// take, [1] the CTAs that finished. The last CTA of a launch to finish puts both back to zero
+// for the slot's next launch.
+constexpr int SCHED_SLOTS = 64;
+__device__ int g_attn_sched[SCHED_SLOTS][2];
+
+// One unit of work: 256 consecutive query rows (two sub-tiles) of one (rollout, head).
+struct Unit {
+    long l0, q_head, kv_head;
+    int bi, qh, kvh;            // branch; query head and key/value head (rollout included)
+    int fa0, fb0, fa1, fb1, fstart;
+    bool valid1;
+    Walk wk;
+};
+__device__ __forceinline__ Unit unit_of(const Params &p, int u, int fq0)
+{
+    Unit c;
+    const int bh = u / p.nqt;
+    const int b = bh / p.Hsum;
+    int h = bh % p.Hsum;
+    c.bi = p.nbr > 1 && h >= p.br[0].Hbr ? 1 : 0;
+    if (c.bi) h -= p.br[0].Hbr;
+    const BranchP &br = p.br[c.bi];
+    c.l0 = (long)(p.nqt - 1 - u % p.nqt) * (QT * BM);
+    c.qh = b * p.q_Htot + br.q_h0 + h;
+    c.kvh = b * br.kv_Htot + br.kv_h0 + h;
+    c.q_head = (long)c.qh * p.q_rows;
+    c.kv_head = (long)c.kvh * br.kv_rows;
+    const long r1_0 = min(c.l0 + BM, p.q_rows) - 1;
+    c.fa0 = fq0 + (int)(c.l0 / p.N);
+    c.fb0 = fq0 + (int)(r1_0 / p.N);
+    c.valid1 = c.l0 + BM < p.q_rows;
+    c.fa1 = c.valid1 ? fq0 + (int)((c.l0 + BM) / p.N) : c.fa0;
+    c.fb1 = c.valid1 ? fq0 + (int)((min(c.l0 + 2 * BM, p.q_rows) - 1) / p.N) : c.fa1;
+    c.wk.fa0 = c.fa0;
+    c.wk.fb0 = c.fb0;
+    c.wk.fa1 = c.fa1;
+    c.wk.fb1 = c.fb1;
+    c.wk.valid1 = c.valid1;
+    c.wk.fb = c.valid1 ? c.fb1 : c.fb0;
+    c.wk.w = br.w;
+    c.wk.r = br.r;
+    c.wk.tpf = (p.N + BN - 1) / BN;
+    c.fstart = max(0, c.fa0 - br.r * (br.w - 1));
+    return c;
+}
+
 template <bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
-attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                const __grid_constant__ CUtensorMap tv, const Params p)
+attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk0,
+                const __grid_constant__ CUtensorMap tv0, const __grid_constant__ CUtensorMap tk1,
+                const __grid_constant__ CUtensorMap tv1, const __grid_constant__ Params p)
 {
     using LY = Lay<F8>;
     extern __shared__ uint8_t smem_raw[];
@@ -248,30 +317,10 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     uint32_t *tmem_slot = (uint32_t *)(smem + LY::SM_TMEMSLOT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y;
-    const int b = bh / p.Hbr, h = bh % p.Hbr;
-    const long l0 = (long)blockIdx.x * (QT * BM);
-    const long q_head = (long)(b * p.q_Htot + p.q_h0 + h) * p.q_rows;
-    const long kv_head = (long)(b * p.kv_Htot + p.kv_h0 + h) * p.kv_rows;
-    const long r1_0 = min(l0 + BM, p.q_rows) - 1;
     const int fq0 = p.fq0_dev ? *p.fq0_dev : p.fq0;
-    const int fa0 = fq0 + (int)(l0 / p.N), fb0 = fq0 + (int)(r1_0 / p.N);
-    const bool valid1 = l0 + BM < p.q_rows;
-    const int fa1 = valid1 ? fq0 + (int)((l0 + BM) / p.N) : fa0;
-    const int fb1 = valid1 ? fq0 + (int)((min(l0 + 2 * BM, p.q_rows) - 1) / p.N) : fa1;
-    Walk wk;
-    wk.fa0 = fa0;
-    wk.fb0 = fb0;
-    wk.fa1 = fa1;
-    wk.fb1 = fb1;
-    wk.valid1 = valid1;
-    wk.fb = valid1 ? fb1 : fb0;
-    wk.w = p.w;
-    wk.r = p.r;
-    wk.tpf = (p.N + BN - 1) / BN;
-    const int fstart = max(0, fa0 - p.r * (p.w - 1));
-    auto kv_row = [&](int fk, int jt) {
-        return (int)(kv_head + (long)(fk % p.kv_slots) * p.N + (long)jt * BN);
+    volatile int *unit_slot = (volatile int *)(smem + LY::SM_UNIT);
+    auto kv_row = [&](const Unit &c, int fk, int jt) {
+        return (int)(c.kv_head + (long)(fk % p.br[c.bi].kv_slots) * p.N + (long)jt * BN);
     };
     auto nkeys = [&](int jt) { return min(BN, p.N - jt * BN); };
 
@@ -288,6 +337,12 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             mbar_init(BAR(LY::B_PVDONE + q), 1);
             mbar_init(BAR(LY::B_PVA + q), 1);
             mbar_init(BAR(LY::B_ODONE + q), 1);
+            mbar_init(BAR(LY::B_OFREE + q), SOFTMAX_THREADS);
+        }
+        mbar_init(BAR(LY::B_QFREE), 2);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(BAR(LY::B_UFULL + i), 1);
+            mbar_init(BAR(LY::B_UEMPTY + i), UNIT_READERS);
         }
         *abort_flag = 0;
         mbar_init_fence();
@@ -312,14 +367,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 
     if (warp == WARP_TMA) {
         // ------------------------------- TMA producer -----------------------------------
+        // Takes the units of this CTA from the launch's work counter and publishes each in a
+        // shared slot (two, used in turn); then loads the unit's Q (once both issuers' last S
+        // of the previous unit completed) and streams its K and V tiles into the ring, which
+        // runs on from one unit to the next.
         if (lane == 0) {
-            mbar_expect_tx(BAR(LY::B_QFULL), QT * LY::QTILE);
-            for (int q = 0; q < QT; ++q) {
-                const int qrow = (int)(q_head + l0 + q * BM);
-                tma_load_2d(sbase + LY::SM_Q(q), &tq, 0, qrow, BAR(LY::B_QFULL));
-                if constexpr (!F8) tma_load_2d(sbase + LY::SM_Q(q) + QHALF, &tq, 64, qrow, BAR(LY::B_QFULL));
-            }
             int it = 0;                                  // ring items issued
+            int nq = 0;                                  // Q loads issued
             bool ok = true;
             auto load = [&](const CUtensorMap *map, int row) -> bool {
                 const int sl = it % LY::NSLOT;
@@ -330,23 +384,45 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 ++it;
                 return true;
             };
-            Pos kp = walk_start(wk, fstart), vp = kp;
-            if (walk_step(wk, kp)) ok = load(&tk, kv_row(kp.fk, kp.jt));
-            while (ok && walk_step(wk, vp)) {
-                if (walk_step(wk, kp) && !(ok = load(&tk, kv_row(kp.fk, kp.jt)))) break;
-                if (!(ok = load(&tv, kv_row(vp.fk, vp.jt)))) break;
+            for (int i = 0; ok; ++i) {
+                const int us = i & 1;
+                if (i >= 2 && !(ok = wait_bar(BAR(LY::B_UEMPTY + us), (uint32_t)((i - 2) >> 1) & 1u))) break;
+                const int u0 = atomicAdd(&g_attn_sched[p.slot][0], 1);
+                const int u = u0 < p.nunits ? u0 : -1;
+                unit_slot[us] = u;
+                mbar_arrive(BAR(LY::B_UFULL + us));
+                if (u < 0) break;
+                const Unit c = unit_of(p, u, fq0);
+                if (i >= 1 && !(ok = wait_bar(BAR(LY::B_QFREE), (uint32_t)(i - 1) & 1u))) break;
+                mbar_expect_tx(BAR(LY::B_QFULL), QT * LY::QTILE);
+                for (int q = 0; q < QT; ++q) {
+                    const int qrow = (int)(c.q_head + c.l0 + q * BM);
+                    tma_load_2d(sbase + LY::SM_Q(q), &tq, 0, qrow, BAR(LY::B_QFULL));
+                    if constexpr (!F8) tma_load_2d(sbase + LY::SM_Q(q) + QHALF, &tq, 64, qrow, BAR(LY::B_QFULL));
+                }
+                ++nq;
+                const CUtensorMap *tk = c.bi ? &tk1 : &tk0, *tv = c.bi ? &tv1 : &tv0;
+                Pos kp = walk_start(c.wk, c.fstart), vp = kp;
+                if (walk_step(c.wk, kp)) ok = load(tk, kv_row(c, kp.fk, kp.jt));
+                while (ok && walk_step(c.wk, vp)) {
+                    if (walk_step(c.wk, kp) && !(ok = load(tk, kv_row(c, kp.fk, kp.jt)))) break;
+                    if (!(ok = load(tv, kv_row(c, vp.fk, vp.jt)))) break;
+                }
             }
             if (*abort_flag) {
+                // a bounded wait expired somewhere: let the copies this CTA issued land
                 const long long t0 = clock64();
                 for (int ii = it - 1; ii >= 0 && ii >= it - LY::NSLOT; --ii)
                     while (!mbar_try(BAR(LY::B_FULL + ii % LY::NSLOT), (uint32_t)(ii / LY::NSLOT) & 1u) && clock64() - t0 < (1LL << 31)) {}
-                while (!mbar_try(BAR(LY::B_QFULL), 0) && clock64() - t0 < (1LL << 31)) {}
+                if (nq > 0)
+                    while (!mbar_try(BAR(LY::B_QFULL), (uint32_t)(nq - 1) & 1u) && clock64() - t0 < (1LL << 31)) {}
             }
         }
     } else if (warp == WARP_MMA || warp == WARP_MMA + 1) {
         // ------------------------------- MMA issuers ------------------------------------
         if (lane == 0) {
             const int q = warp - WARP_MMA;
+            Walk wk;
             const int want = 1 << q;
             constexpr uint32_t IDESC_S0 = (F8 ? idesc_e4m3(BM, 16, false, false) : tc::idesc_bf16(BM, 16, false, false)) & ~(0x3Fu << 17);
             constexpr uint32_t IDESC_O = F8 ? idesc_e4m3(BM, D, false, true) : tc::idesc_bf16(BM, D, false, true);
@@ -356,7 +432,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             const uint64_t dp = tc::sw128_desc(sbase + LY::SM_P(q), 16, 1024);
             const uint32_t s_tm = tmem + TM_S(q), o_tm = tmem + TM_O(q);
             int it = 0, ns = 0, npv = 0;
-            bool ok = wait_bar(BAR(LY::B_QFULL), 0);
+            int npv0 = 0;                   // P V products issued before the current unit
+            bool ok = true;
+            int ui = 0;                     // units taken
+            // the first P V of a unit overwrites O: the previous unit's epilogue must have read it
+            auto ofree = [&]() -> bool {
+                return ui < 1 || wait_bar(BAR(LY::B_OFREE + q), (uint32_t)(ui - 1) & 1u);
+            };
             // K of tile u (ring item `it`): S = Q K^T once this sub-tile's softmax read the
             // previous S (N = the tile's keys rounded up to 16), then the slot released
             auto handle_k = [&](const Pos &u) -> bool {
@@ -396,6 +478,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 if (!wait_bar(BAR(LY::B_FULL + sl), (uint32_t)(it / LY::NSLOT) & 1u)) return false;
                 if (t.mask & want) {
                     if (!wait_bar(BAR(LY::B_PFULL + q), (uint32_t)npv & 1u)) return false;
+                    if (npv == npv0 && !ofree()) return false;
                     tc::fence_after_sync();
                     const uint64_t dv = dvl0 + (uint64_t)((sl * LY::KTILE) >> 4);
                     if constexpr (F8) {
@@ -403,13 +486,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         const int ksteps = (nkeys(t.jt) + 31) >> 5;
                         for (int kk = 0; kk < ksteps; ++kk) {
                             umma_f8(o_tm, dp + (uint64_t)(kk * 2), dv + (uint64_t)((kk * 4096) >> 4), IDESC_O,
-                                    (npv > 0 || kk > 0) ? 1u : 0u);
+                                    (npv > npv0 || kk > 0) ? 1u : 0u);
                             if (kk == 1 && ksteps == BN / 32) tc::umma_commit(BAR(LY::B_PVA + q));
                         }
                         if (ksteps < BN / 32) tc::umma_commit(BAR(LY::B_PVA + q));
                     } else {
                     const int ksteps = (nkeys(t.jt) + 15) >> 4;
-                    if (ksteps == BN / 16 && npv > 0) {
+                    if (ksteps == BN / 16 && npv > npv0) {
                         // the first half of P (keys 0-63) is released once its products are
                         // done, so the softmax can store the next tile's first half early
 #pragma unroll
@@ -422,7 +505,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                         for (int kk = 0; kk < ksteps; ++kk) {
                             const uint64_t poff = (uint64_t)((((kk >> 2) * PHALF + (kk & 3) * 32) >> 4));
                             tc::umma_bf16(o_tm, dp + poff, dv + (uint64_t)((kk * 2048) >> 4), IDESC_O,
-                                          (npv > 0 || kk > 0) ? 1u : 0u);
+                                          (npv > npv0 || kk > 0) ? 1u : 0u);
                         }
                         tc::umma_commit(BAR(LY::B_PVA + q));
                     }
@@ -436,18 +519,37 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 ++it;
                 return true;
             };
-            Pos t = walk_start(wk, fstart);
-            bool have = ok && walk_step(wk, t);
-            if (have) ok = handle_k(t);
-            while (ok && have) {
-                Pos u = t;
-                const bool next = walk_step(wk, u);
-                if (next && !(ok = handle_k(u))) break;   // K(t + 1) before V(t)
-                if (!(ok = handle_v(t))) break;
-                have = next;
-                t = u;
+            for (; ok; ++ui) {
+                const int us = ui & 1;
+                if (!(ok = wait_bar(BAR(LY::B_UFULL + us), (uint32_t)(ui >> 1) & 1u))) break;
+                const int un = unit_slot[us];
+                mbar_arrive(BAR(LY::B_UEMPTY + us));
+                if (un < 0) break;
+                const Unit c = unit_of(p, un, fq0);
+                wk = c.wk;
+                if (!(ok = wait_bar(BAR(LY::B_QFULL), (uint32_t)ui & 1u))) break;
+                tc::fence_after_sync();
+                npv0 = npv;
+                Pos t = walk_start(wk, c.fstart);
+                bool have = walk_step(wk, t);
+                if (have) ok = handle_k(t);
+                else tc::umma_commit(BAR(LY::B_QFREE));       // a unit without tiles
+                while (ok && have) {
+                    Pos u = t;
+                    const bool next = walk_step(wk, u);
+                    if (next) ok = handle_k(u);           // K(t + 1) before V(t)
+                    else tc::umma_commit(BAR(LY::B_QFREE));   // the unit's last S was issued
+                    if (!ok) break;
+                    if (!(ok = handle_v(t))) break;
+                    have = next;
+                    t = u;
+                }
+                if (!ok) break;
+                // a unit without a P V of this sub-tile still waits for the previous epilogue,
+                // so that its completion below never runs two units ahead of the softmax
+                if (npv == npv0 && !(ok = ofree())) break;
+                tc::umma_commit(BAR(LY::B_ODONE + q));
             }
-            if (ok) tc::umma_commit(BAR(LY::B_ODONE + q));
         }
     } else {
         // ------------------------------- softmax ----------------------------------------
@@ -456,47 +558,57 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         const int q = warp >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
-        const long lrow = l0 + q * BM + row;
-        const bool row_valid = lrow < p.q_rows;
-        const int fq = fq0 + (int)(lrow / p.N);
         const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t prow = sbase + LY::SM_P(q) + (uint32_t)row * 128u;
         const uint32_t rx = (uint32_t)(row & 7);
-        // E4M3: the scores carry the Q block's scale (one per sub-tile; sub-tile 1 of a head's
-        // last CTA may lie past the last query block) and each 64-key run's K scale
-        const int kvh = b * p.kv_Htot + p.kv_h0 + h;
         const int tpf64 = (p.N + 63) / 64;
-        float sl2 = p.sl2;
-        if constexpr (F8) {
-            const long qblk = l0 / BM + q;
-            sl2 = qblk < p.nqb ? p.sl2 * __ldg(p.qs + (long)(b * p.q_Htot + p.q_h0 + h) * p.nqb + qblk) : 0.f;
-        }
         // log2 growth of the max before a rescale; E4M3: P = 2^(x - m + 4) stays within 2^8
         constexpr float LAZY = F8 ? 4.f : 8.f;
         constexpr float PBIAS = F8 ? 4.f : 0.f;
-        const int faq = q == 0 ? fa0 : fa1, fbq = q == 0 ? fb0 : fb1;
-        const bool qvalid = q == 0 || valid1;
-        float m = -INFINITY, lsum = 0.f;
         bool ok = true;
-        int k = 0;
-        int fk = fstart - 1, jt = wk.tpf - 1;
+        int k = 0;                      // tiles of this sub-tile over every unit so far
+        for (int ui = 0; ok; ++ui) {
+        const int us = ui & 1;
+        if (!__all_sync(0xffffffffu, wait_bar(BAR(LY::B_UFULL + us), (uint32_t)(ui >> 1) & 1u))) { ok = false; break; }
+        const int un = unit_slot[us];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(LY::B_UEMPTY + us));
+        if (un < 0) break;
+        const Unit c = unit_of(p, un, fq0);
+        const Walk &wk = c.wk;
+        const long lrow = c.l0 + q * BM + row;
+        const bool row_valid = lrow < p.q_rows;
+        const int fq = fq0 + (int)(lrow / p.N);
+        // E4M3: the scores carry the Q block's scale (one per sub-tile; sub-tile 1 of a head's
+        // last unit may lie past the last query block) and each 64-key run's K scale
+        const BranchP &br = p.br[c.bi];
+        float sl2 = p.sl2;
+        if constexpr (F8) {
+            const long qblk = c.l0 / BM + q;
+            sl2 = qblk < p.nqb ? p.sl2 * __ldg(p.qs + (long)c.qh * p.nqb + qblk) : 0.f;
+        }
+        const int faq = q == 0 ? c.fa0 : c.fa1, fbq = q == 0 ? c.fb0 : c.fb1;
+        const bool qvalid = q == 0 || c.valid1;
+        float m = -INFINITY, lsum = 0.f;
+        const int k0 = k;
+        int fk = c.fstart - 1, jt = wk.tpf - 1;
         while (qvalid) {
             // the next tile of this sub-tile: the same frames and order as the MMA warp's walk
             if (++jt >= wk.tpf) {
-                for (++fk; fk <= fbq && !frame_needed(fk, faq, fbq, p.w, p.r); ++fk) {}
+                for (++fk; fk <= fbq && !frame_needed(fk, faq, fbq, wk.w, wk.r); ++fk) {}
                 if (fk > fbq) break;
                 jt = 0;
             }
             float sla = sl2, slb = sl2;          // the scales of keys 0-63 and 64-127
             if constexpr (F8) {
-                const long kb = (long)kvh * p.nkb + (long)(fk % p.kv_slots) * tpf64 + 2 * jt;
-                sla = sl2 * __ldg(p.ks + kb);
-                slb = 2 * jt + 1 < tpf64 ? sl2 * __ldg(p.ks + kb + 1) : sla;
+                const long kb = (long)c.kvh * br.nkb + (long)(fk % br.kv_slots) * tpf64 + 2 * jt;
+                sla = sl2 * __ldg(br.ks + kb);
+                slb = 2 * jt + 1 < tpf64 ? sl2 * __ldg(br.ks + kb + 1) : sla;
             }
             if (!__all_sync(0xffffffffu, wait_bar(BAR(LY::B_SFULL + q), (uint32_t)k & 1u))) { ok = false; break; }
             tc::fence_after_sync();
             const int nv = nkeys(jt);
-            const bool rok = row_valid && is_tap(fq, fk, p.w, p.r);
+            const bool rok = row_valid && is_tap(fq, fk, wk.w, wk.r);
             // the tile's scores into registers, then the S buffer is free for the next tile
             uint32_t sa[64], sb[64];
             tc::tmem_ld64(tlane + TM_S(q), sa);
@@ -642,16 +754,16 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             mbar_arrive(BAR(LY::B_PFULL + q));
             ++k;
         }
-        // final: every product of the sub-tile has completed (a one-phase barrier its MMA warp
-        // commits after its last issue); normalise O and store it
-        const bool fin = ok && k >= 1 &&
-                         __all_sync(0xffffffffu, wait_bar(BAR(LY::B_ODONE + q), 0u));
-        if (fin) {
-            tc::fence_after_sync();
+        if (!ok) break;
+        // the unit's end: every product of the sub-tile has completed (its MMA warp commits
+        // once per unit after its last issue); normalise O and store it, then hand O back
+        if (!__all_sync(0xffffffffu, wait_bar(BAR(LY::B_ODONE + q), (uint32_t)ui & 1u))) { ok = false; break; }
+        tc::fence_after_sync();
+        if (k > k0) {
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-            if (!F8 && p.lse && row_valid) p.lse[q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
-            __nv_bfloat16 *orow = p.o + (q_head + lrow) * D;
-            const float4 *vsc = F8 ? reinterpret_cast<const float4 *>(p.vs + (long)kvh * D) : nullptr;
+            if (!F8 && p.lse && row_valid) p.lse[c.q_head + lrow] = (m + log2f(lsum)) * 0.69314718055994531f;
+            __nv_bfloat16 *orow = p.o + (c.q_head + lrow) * D;
+            const float4 *vsc = F8 ? reinterpret_cast<const float4 *>(br.vs + (long)c.kvh * D) : nullptr;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ov[32];
@@ -680,6 +792,9 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                 }
             }
         }
+        tc::fence_before_sync();
+        mbar_arrive(BAR(LY::B_OFREE + q));
+        }
     }
 
     tc::fence_before_sync();
@@ -690,50 +805,113 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
     }
+    // every path reaches this point once per CTA, after this CTA's last ticket; the last CTA
+    // (of every launch sharing the counter) to arrive leaves the slot at zero for its next use
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(&g_attn_sched[p.slot][1], 1) == p.ctas_total - 1) {
+            atomicExch(&g_attn_sched[p.slot][0], 0);
+            atomicExch(&g_attn_sched[p.slot][1], 0);
+        }
+    }
+}
+
+// Branches sharing one launch share the query and output tensors, the batch, the query rows,
+// frame size, first query frame, scale and error word; their heads, windows and key/value
+// tensors may differ.
+bool same_launch(const AttnArgs &a, const AttnArgs &b)
+{
+    return a.q == b.q && a.o == b.o && a.B == b.B && a.q_Htot == b.q_Htot && a.q_rows == b.q_rows &&
+           a.N == b.N && a.d == b.d && a.fq0 == b.fq0 && a.fq0_dev == b.fq0_dev && a.scale == b.scale &&
+           a.err == b.err && a.qs == b.qs && a.lse == b.lse;
 }
 
 template <bool F8>
-cudaError_t launch_attn_tc2(const AttnArgs &a, cudaStream_t s)
+cudaError_t launch_attn_tc2(const AttnArgs *br, int nbr, int reserve_sms, cudaStream_t s,
+                            cudaStream_t s_fill)
 {
     using LY = Lay<F8>;
-    if (a.d != D) return cudaErrorNotSupported;
     cudaError_t e;
+    if (nbr < 1 || nbr > 2) return cudaErrorInvalidValue;
+    if (nbr == 2 && !same_launch(br[0], br[1])) return cudaErrorInvalidValue;
+    const AttnArgs &a = br[0];
+    if (a.d != D) return cudaErrorNotSupported;
     const long q_total = (long)a.B * a.q_Htot * a.q_rows;
-    const long kv_total = (long)a.B * a.kv_Htot * a.kv_rows;
-    if (q_total + QT * BM >= (1L << 31) || kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
-    CUtensorMap mq, mk, mv;
+    if (q_total + QT * BM >= (1L << 31)) return cudaErrorNotSupported;
+    CUtensorMap mq, mk[2], mv[2];
     if (F8) {
         // E4M3 codes: one 128-byte row per token, one box covers the row
         if ((e = make_tmap_2d_u8(&mq, a.q, q_total, D, D, BM)) != cudaSuccess) return e;
-        if ((e = make_tmap_2d_u8(&mk, a.k, kv_total, D, D, BN)) != cudaSuccess) return e;
-        if ((e = make_tmap_2d_u8(&mv, a.v, kv_total, D, D, BN)) != cudaSuccess) return e;
     } else {
         if ((e = make_tmap_2d_bf16(&mq, a.q, q_total, D, 64, BM, true)) != cudaSuccess) return e;
-        if ((e = make_tmap_2d_bf16(&mk, a.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
-        if ((e = make_tmap_2d_bf16(&mv, a.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
     }
-    Params p;
-    p.Hbr = a.Hbr; p.q_Htot = a.q_Htot; p.q_h0 = a.q_h0; p.kv_Htot = a.kv_Htot; p.kv_h0 = a.kv_h0;
-    p.kv_slots = a.kv_slots; p.q_rows = a.q_rows; p.kv_rows = a.kv_rows;
-    p.N = a.N; p.w = a.w; p.r = a.r; p.fq0 = a.fq0; p.fq0_dev = a.fq0_dev;
+    Params p = {};
+    int Hsum = 0;
+    for (int i = 0; i < nbr; ++i) {
+        const AttnArgs &x = br[i];
+        const long kv_total = (long)x.B * x.kv_Htot * x.kv_rows;
+        if (kv_total + BN >= (1L << 31)) return cudaErrorNotSupported;
+        if (F8) {
+            if ((e = make_tmap_2d_u8(&mk[i], x.k, kv_total, D, D, BN)) != cudaSuccess) return e;
+            if ((e = make_tmap_2d_u8(&mv[i], x.v, kv_total, D, D, BN)) != cudaSuccess) return e;
+            if (!x.qs || !x.ks || !x.vs) return cudaErrorInvalidValue;
+        } else {
+            if ((e = make_tmap_2d_bf16(&mk[i], x.k, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+            if ((e = make_tmap_2d_bf16(&mv[i], x.v, kv_total, D, 64, BN, true)) != cudaSuccess) return e;
+        }
+        BranchP &b = p.br[i];
+        b.Hbr = x.Hbr; b.q_h0 = x.q_h0; b.kv_Htot = x.kv_Htot; b.kv_h0 = x.kv_h0;
+        b.kv_slots = x.kv_slots; b.w = x.w; b.r = x.r;
+        b.nkb = x.kv_slots * ((x.N + 63) / 64);
+        b.kv_rows = x.kv_rows;
+        b.ks = x.ks; b.vs = x.vs;
+        Hsum += x.Hbr;
+    }
+    if (nbr == 1) { mk[1] = mk[0]; mv[1] = mv[0]; }
+    p.nbr = nbr; p.B = a.B; p.Hsum = Hsum;
+    p.q_Htot = a.q_Htot; p.q_rows = a.q_rows;
+    p.N = a.N; p.fq0 = a.fq0; p.fq0_dev = a.fq0_dev;
     p.sl2 = a.scale * 1.4426950408889634f;
-    p.qs = a.qs; p.ks = a.ks; p.vs = a.vs;
+    p.qs = a.qs;
     p.nqb = (int)((a.q_rows + BM - 1) / BM);
-    p.nkb = a.kv_slots * ((a.N + 63) / 64);
     p.lse = a.lse;
     p.o = (__nv_bfloat16 *)a.o;
     p.err = a.err;
-    if (F8 && (!p.qs || !p.ks || !p.vs)) return cudaErrorInvalidValue;
+    // persistent: one CTA per SM at most (less the SMs left to a kernel running beside it),
+    // each taking 256-row units from the slot's counter; with `s_fill`, as many more CTAs as
+    // SMs were left start behind the work on that stream and take units from the same counter
+    const long nqt = (a.q_rows + QT * BM - 1) / (QT * BM);
+    const long nunits = nqt * a.B * Hsum;
+    if (nunits <= 0) return cudaSuccess;
+    if (nunits >= (1L << 30)) return cudaErrorNotSupported;
+    p.nqt = (int)nqt;
+    p.nunits = (int)nunits;
+    static std::atomic<unsigned> next_slot{0};
+    p.slot = (int)(next_slot.fetch_add(1u) % (unsigned)SCHED_SLOTS);
+    int dev = 0, nsm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    nsm = std::max(nsm, 1);
+    const int ctas = std::max(nsm - std::max(reserve_sms, 0), (nsm + 1) / 2);
     e = cudaFuncSetAttribute(attn_tc2_kernel<F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.q_rows + QT * BM - 1) / (QT * BM)), (unsigned)(a.B * a.Hbr));
-    attn_tc2_kernel<F8><<<grid, THREADS, LY::SMEM_BYTES, s>>>(mq, mk, mv, p), note_launch();
+    const int grid = (int)std::min<long>(nunits, ctas);
+    const int fill = s_fill ? (int)std::min<long>(nunits - grid, nsm - ctas) : 0;
+    p.ctas_total = grid + fill;
+    attn_tc2_kernel<F8><<<grid, THREADS, LY::SMEM_BYTES, s>>>(mq, mk[0], mv[0], mk[1], mv[1], p), note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess || fill <= 0) return e;
+    attn_tc2_kernel<F8><<<fill, THREADS, LY::SMEM_BYTES, s_fill>>>(mq, mk[0], mv[0], mk[1], mv[1], p), note_launch();
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<false>(a, s); }
-cudaError_t launch_attn_fp8_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<true>(a, s); }
+cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<false>(&a, 1, 0, s, nullptr); }
+cudaError_t launch_attn_bf16_tc2_multi(const AttnArgs *br, int nbr, int reserve_sms, cudaStream_t s,
+                                       cudaStream_t s_fill)
+{
+    return launch_attn_tc2<false>(br, nbr, reserve_sms, s, s_fill);
+}
+cudaError_t launch_attn_fp8_tc2(const AttnArgs &a, cudaStream_t s) { return launch_attn_tc2<true>(&a, 1, 0, s, nullptr); }
 
 }  // namespace hlta

@@ -538,6 +538,7 @@ cudaError_t launch_gdn_bf16_v2(const GdnArgs &g, cudaStream_t s)
         return e;
     gdn_prep_tc<<<dim3((unsigned)nch, (unsigned)BH), THREADS, smem, s>>>(m, g, ws), note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (g.prep_done && (e = cudaEventRecord(g.prep_done, s)) != cudaSuccess) return e;
     return launch_gdn_bf16_scan(g, ws, s);
 }
 

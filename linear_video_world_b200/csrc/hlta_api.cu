@@ -4,6 +4,7 @@
 #include "hlta.h"
 #include "hlta_internal.cuh"
 
+#include <algorithm>
 #include <atomic>
 #include <math.h>
 #include <mutex>
@@ -44,6 +45,7 @@ struct DeviceCtx {
     cudaStream_t aux2 = nullptr;    // DSWA branch of the hybrid (default priority)
     cudaStream_t aux3 = nullptr;    // second serial pass of the GDN backward (highest priority)
     cudaEvent_t fork = nullptr, join = nullptr, join2 = nullptr, mid = nullptr;
+    cudaEvent_t prep = nullptr;     // the GDN branch's chunk preparation done (bf16)
 };
 constexpr int kMaxDevices = 64;
 DeviceCtx g_ctx[kMaxDevices];
@@ -91,6 +93,8 @@ hlta_status device_ctx(DeviceCtx **out)
             return cuda_fail(e, "cudaStreamCreateWithPriority");
         if ((e = cudaEventCreateWithFlags(&c.mid, cudaEventDisableTiming)) != cudaSuccess)
             return cuda_fail(e, "cudaEventCreate");
+        if ((e = cudaEventCreateWithFlags(&c.prep, cudaEventDisableTiming)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventCreate");
         c.ready = true;
     }
     *out = &c;
@@ -117,13 +121,34 @@ hlta_status check_window(int w, int r)
     return HLTA_OK;
 }
 
-hlta_status run_attn(const AttnArgs &a, hlta_dtype dt, cudaStream_t s)
+hlta_status attn_status(cudaError_t e)
 {
-    if (a.B * a.Hbr == 0 || a.q_rows == 0) return HLTA_OK;
-    cudaError_t e = dt == HLTA_FP32 ? launch_attn_f32(a, s) : launch_attn_bf16_tc2(a, s);
     if (e == cudaErrorNotSupported) return fail(HLTA_ERR_UNSUPPORTED, "window attention: unsupported shape");
     if (e != cudaSuccess) return cuda_fail(e, "window attention launch");
     return HLTA_OK;
+}
+
+// `reserve_sms`: SMs the bf16 kernel (persistent, one CTA per SM) leaves free for the kernels
+// queued on `s_fill` (the GDN branch's chain); as many more of its CTAs start behind them
+hlta_status run_attn(const AttnArgs &a, hlta_dtype dt, cudaStream_t s, int reserve_sms = 0,
+                     cudaStream_t s_fill = nullptr)
+{
+    if (a.B * a.Hbr == 0 || a.q_rows == 0) return HLTA_OK;
+    return attn_status(dt == HLTA_FP32 ? launch_attn_f32(a, s)
+                                       : launch_attn_bf16_tc2_multi(&a, 1, reserve_sms, s, s_fill));
+}
+
+// The SWA and DSWA branches: on bf16 one persistent launch takes both branches' units (no
+// tail between two launches); fp32 launches them one after the other on `s`
+hlta_status run_attn_pair(const AttnArgs &a0, const AttnArgs &a1, hlta_dtype dt, cudaStream_t s,
+                          int reserve_sms, cudaStream_t s_fill)
+{
+    if (dt != HLTA_BF16) {
+        hlta_status st = run_attn(a0, dt, s);
+        return st != HLTA_OK ? st : run_attn(a1, dt, s);
+    }
+    const AttnArgs br[2] = {a0, a1};
+    return attn_status(launch_attn_bf16_tc2_multi(br, 2, reserve_sms, s, s_fill));
 }
 
 hlta_status run_gdn(const GdnArgs &g, hlta_dtype dt, cudaStream_t s)
@@ -574,9 +599,13 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     std::lock_guard<std::mutex> lk(g_fork_mu);
-    // the branches other than SWA run on library streams ordered after everything already
-    // on `s` (one fork event), and `s` waits for them at the end
-    const bool split_d = Hd && Hs;
+    // the GDN branch runs on a library stream ordered after everything already on `s` (one
+    // fork event), and `s` waits for it at the end; bf16 SWA and DSWA heads share one launch,
+    // fp32 runs DSWA on a second library stream beside SWA
+    const bool pair = Hd && Hs && dt == HLTA_BF16;
+    const bool split_d = Hd && Hs && !pair;
+    int reserve = 0;
+    cudaStream_t s_fill = nullptr;  // bf16 with GDN heads: the attention's late CTAs follow the chain
     if (Hg || split_d) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
@@ -597,6 +626,12 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
         }
         pairs *= (double)B * N * N;
         g.scan_segments = gdn_scan_segments_beside((long)B * Hg, gdn_num_chunks(L, chunk), 4.0 * d * pairs);
+        // the chain's kernels take one SM per (head, segment) at most: the softmax launch
+        // leaves those to it
+        reserve = (int)std::min<long>((long)B * Hg * std::max(g.scan_segments, 1), 1L << 20);
+        // the persistent attention launch holds its SMs to the end: it starts after the
+        // preparation (which takes the whole GPU for a short time), beside the chain
+        if (dt == HLTA_BF16) g.prep_done = ctx->prep;
         prof_record(3, ctx->aux);
         st = run_gdn(g, dt, ctx->aux);
         prof_record(4, ctx->aux);
@@ -605,26 +640,39 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
             cudaStreamWaitEvent(s, ctx->join, 0);   // `s` never runs ahead of enqueued work
             return st;
         }
+        if (dt == HLTA_BF16 && (e = cudaStreamWaitEvent(s, ctx->prep, 0)) != cudaSuccess) {
+            cudaStreamWaitEvent(s, ctx->join, 0);
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        }
+        if (dt == HLTA_BF16) s_fill = ctx->aux;
+    }
+    if (pair) {
+        AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
+        AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
+        st = run_attn_pair(a2, a1, dt, s, reserve, s_fill);
+        prof_record(2, s);
     }
     // DSWA on the second library stream (beside SWA) when both softmax branches are present
-    if (Hd) {
+    if (Hd && !pair) {
         cudaStream_t sd = split_d ? ctx->aux2 : s;
         if (split_d && (e = cudaStreamWaitEvent(sd, ctx->fork, 0)) != cudaSuccess)
             st = cuda_fail(e, "cudaStreamWaitEvent");
         if (st == HLTA_OK) {
             AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
-            st = run_attn(a2, dt, sd);
+            st = run_attn(a2, dt, sd, reserve, s_fill);
         }
         prof_record(2, sd);
         if (split_d) cudaEventRecord(ctx->join2, sd);
     }
-    if (Hs && st == HLTA_OK) {
+    if (Hs && !pair && st == HLTA_OK) {
         AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
-        st = run_attn(a1, dt, s);
+        st = run_attn(a1, dt, s, reserve, s_fill);
     }
     prof_record(1, s);
-    // join: work enqueued on `s` after this call sees every branch's outputs
+    // join: work enqueued on `s` after this call sees every branch's outputs (the GDN stream
+    // also carries the attention's late CTAs)
     if (split_d) cudaStreamWaitEvent(s, ctx->join2, 0);
+    if (s_fill) cudaEventRecord(ctx->join, ctx->aux);
     if (Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     return st;
 }
@@ -740,10 +788,14 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
     const int f = c->frames;
     const size_t el = c->dt == HLTA_BF16 ? 2 : 4;
     // the fork/join events are shared per device: hold them until the joins are enqueued.
-    // GDN runs on the high-priority library stream, the DSWA branch (ring append and
-    // attention) on the second library stream when SWA heads are present too
+    // GDN runs on the high-priority library stream; bf16 SWA and DSWA heads share one
+    // attention launch on `s`, fp32 runs the DSWA branch (ring append and attention) on the
+    // second library stream when SWA heads are present too
     std::unique_lock<std::mutex> lk(g_fork_mu, std::defer_lock);
-    const bool split_d = c->Hd && c->Hs;
+    const bool pair = c->Hd && c->Hs && c->dt == HLTA_BF16;
+    const bool split_d = c->Hd && c->Hs && !pair;
+    int reserve = 0;
+    cudaStream_t s_fill = nullptr;  // bf16 with GDN heads: the attention's late CTAs follow the chain
     lk.lock();
     if (c->Hg || split_d) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -757,6 +809,12 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         g.B = c->B; g.Hg = c->Hg; g.Htot = H; g.h0 = c->Hs + c->Hd; g.L = (long)F * c->N; g.d = c->d;
         g.chunk = c->chunk; g.S0 = c->S; g.S_out = c->S; g.ws = c->ws; g.ws_bytes = c->ws_bytes;
         g.err = ctx->err;
+        // the chain takes one SM per (head, segment): the softmax launch leaves those to it
+        const long nch = gdn_num_chunks(g.L, g.chunk), BHg = (long)c->B * c->Hg;
+        const long seg = gdn_scan_segment_len(BHg, nch);
+        reserve = (int)std::min<long>(BHg * ((nch + seg - 1) / seg), 1L << 20);
+        // the persistent attention launch starts after the preparation, beside the chain
+        if (c->dt == HLTA_BF16) g.prep_done = ctx->prep;
         st = run_gdn(g, c->dt, ctx->aux);
         prof_record(4, ctx->aux);
         cudaEventRecord(ctx->join, ctx->aux);
@@ -764,6 +822,11 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
             cudaStreamWaitEvent(s, ctx->join, 0);
             return st;
         }
+        if (c->dt == HLTA_BF16 && (e = cudaStreamWaitEvent(s, ctx->prep, 0)) != cudaSuccess) {
+            cudaStreamWaitEvent(s, ctx->join, 0);
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        }
+        if (c->dt == HLTA_BF16) s_fill = ctx->aux;
     }
     struct Branch { int h0, Hbr, slots, w, r; void *rk, *rv; } br[2] = {
         {0, c->Hs, c->slots_s, c->w_swa, 1, c->ks, c->vs},
@@ -772,6 +835,7 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         cudaStreamWaitEvent(s, ctx->join, 0);
         return cuda_fail(e, "cudaStreamWaitEvent");
     }
+    AttnArgs pa[2];
     for (int bi = 1; bi >= 0; --bi) {                  // DSWA first: it goes to its own stream
         const Branch &x = br[bi];
         if (!x.Hbr) continue;
@@ -788,14 +852,24 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
         a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.fq0_dev = c->fdev; a.scale = c->scale;
         a.err = ctx->err;
-        if ((st = run_attn(a, c->dt, s)) != HLTA_OK) break;
+        if (pair) {
+            pa[1 - bi] = a;                            // launched below, DSWA's units first
+            continue;
+        }
+        if ((st = run_attn(a, c->dt, s, reserve, s_fill)) != HLTA_OK) break;
         prof_record(bi == 1 ? 2 : 1, s);
+    }
+    if (pair && st == HLTA_OK) {
+        st = run_attn_pair(pa[0], pa[1], c->dt, (cudaStream_t)stream, reserve, s_fill);
+        prof_record(2, (cudaStream_t)stream);
+        prof_record(1, (cudaStream_t)stream);
     }
     // join the other branches after the softmax launches were enqueued, so they overlap
     if (split_d) {
         cudaEventRecord(ctx->join2, ctx->aux2);
         cudaStreamWaitEvent(s, ctx->join2, 0);
     }
+    if (s_fill) cudaEventRecord(ctx->join, ctx->aux);
     if (c->Hg) cudaStreamWaitEvent(s, ctx->join, 0);
     if (st != HLTA_OK) return st;
     if ((e = launch_frame_advance(c->fdev, F, s)) != cudaSuccess) return cuda_fail(e, "frame counter");

@@ -63,6 +63,9 @@ struct GdnArgs {
     // the latency low; 1: one serial chain per head on as few SMs as possible, for a branch
     // that runs beside other work); at most the count the workspace was sized for
     int scan_segments;
+    // bf16: when set, recorded on the launch stream after the chunk preparation (work that
+    // holds SMs for long, such as the persistent attention launch, waits for it)
+    cudaEvent_t prep_done = nullptr;
 };
 
 // Chunk workspace (per GDN head, per chunk of C tokens; elements of type E):
@@ -114,8 +117,15 @@ cudaError_t make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t rows, u
 
 // Launchers. Return cudaGetLastError() of their launches.
 cudaError_t launch_attn_f32(const AttnArgs &a, cudaStream_t s);
-// bf16 window attention: 128-key tiles, two query sub-tiles, P staged in shared memory (attn_tc2.cu)
+// bf16 window attention: 128-key tiles, two query sub-tiles, P staged in shared memory; a
+// persistent launch of one CTA per SM (attn_tc2.cu)
 cudaError_t launch_attn_bf16_tc2(const AttnArgs &a, cudaStream_t s);
+// The same over one or two branches in one launch (the branches share q, o, B, q_rows, N, d,
+// fq0, scale and err; cudaErrorInvalidValue otherwise), leaving `reserve_sms` SMs (at most
+// half) to kernels that run beside it on `s_fill`; with `s_fill` set, a second launch of that
+// many CTAs, queued on `s_fill` behind them, takes the remaining units from the same counter
+cudaError_t launch_attn_bf16_tc2_multi(const AttnArgs *br, int nbr, int reserve_sms, cudaStream_t s,
+                                       cudaStream_t s_fill);
 // the same two-tile design on E4M3 codes (attn_tc2.cu)
 cudaError_t launch_attn_fp8_tc2(const AttnArgs &a, cudaStream_t s);
 // E4M3 quantisation (bf16 input, d = 128): row blocks inside frames, and value channels

@@ -84,3 +84,47 @@ def test_480p_softmax_branches_sampled(h, orc):
     got_d = o_d[0].reshape(-1, wl.d)[torch.from_numpy(flat_d).cuda()]
     assert maxabs(got_d, ref_d) <= TOL
     assert torch.isfinite(o_s).all() and torch.isfinite(o_d).all()
+
+
+def test_swa_and_dswa_heads_in_one_launch(h, orc):
+    """SWA and DSWA heads of one tensor as a hybrid call without GDN heads: both branches'
+    units share one persistent launch (B = 2, ragged key tiles, tiles straddling frames)."""
+    B, Hs, Hd, T, N, w_s, w_d, r = 2, 2, 3, 7, 150, 3, 3, 2
+    wl = hi.Workload("t", B=B, Hs=Hs, Hd=Hd, Hg=0, d=128, T=T, N=N, w_swa=w_s, w_dswa=w_d, r=r,
+                     chunk=64, dtype="bf16", decay=1.0)
+    x = hi.make_inputs(wl, seed=5)
+    q, k, v = (dev(x[n]) for n in "qkv")
+    o, _ = h.hybrid(q, k, v, None, None, Hs, Hd, 0, T, N, w_s, w_d, r, out=poison_like(q))
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    sub = {n: (x[n][:, :Hs].contiguous(), x[n][:, Hs:].contiguous()) for n in "qkv"}
+    ref_s = orc.swa(sub["q"][0], sub["k"][0], sub["v"][0], T, N, w_s)
+    ref_d = orc.dswa(sub["q"][1], sub["k"][1], sub["v"][1], T, N, w_d, r)
+    assert maxabs(o[:, :Hs], ref_s) <= TOL
+    assert maxabs(o[:, Hs:], ref_d) <= TOL
+
+
+def test_work_counter_survives_many_launches(h):
+    """More launches than the kernel has work counters, of different unit counts and on two
+    streams: every launch hands out all its units (each output equals the first of its shape,
+    bit for bit), so each counter is back at zero for its next use."""
+    shapes = [(2, 3, 5, 200, 3), (1, 1, 2, 300, 5), (1, 2, 3, 1560, 3)]
+    data, first = [], []
+    for i, (B, H, T, N, w) in enumerate(shapes):
+        x = hi.make_inputs(_wl(B, H, T, N, w, 1), seed=100 + i)
+        q, k, v = (dev(x[n]) for n in "qkv")
+        data.append((q, k, v, T, N, w))
+        first.append(h.swa(q, k, v, T, N, w))
+    side = torch.cuda.Stream()
+    outs = []
+    for it in range(150):
+        q, k, v, T, N, w = data[it % 3]
+        stream = side if it % 5 == 4 else torch.cuda.current_stream()
+        with torch.cuda.stream(stream):
+            outs.append((it % 3, h.swa(q, k, v, T, N, w, out=poison_like(q))))
+        if it % 5 == 4:
+            torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    for j, o in outs:
+        assert torch.equal(o, first[j])
