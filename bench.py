@@ -602,8 +602,8 @@ def main():
     clocks = clk.stop()
     total_ms = allmax(ev0.elapsed_time(ev1))
     ms = total_ms / K
-    # SWA and DSWA heads share one attention launch, from the fork (event 0) to its end
-    # (events 1 and 2)
+    # SWA and DSWA heads share one attention launch: from its start (event 0, after the GDN
+    # preparation it waits for) to the end of its last CTA (events 1 and 2)
     attn_span_ms = statistics.mean(max(p[0].elapsed_time(p[1]), p[0].elapsed_time(p[2])) for p in prof)
     gdn_ms = statistics.mean(p[3].elapsed_time(p[4]) for p in prof)
     assert h.hlta_device_status() == 0
@@ -760,8 +760,8 @@ def main():
     tr = traffic_record("attn_tc2.cu")          # the bf16 window attention kernel
     tr8 = tr                                    # the E4M3 instantiation lives in the same file
     roofline = {"bound": "tensor", "kernel": "attn_tc2_kernel (the SWA and DSWA heads in one persistent "
-                                              "launch, beside the GDN branch: from the step's start to "
-                                              "the launch's end)",
+                                              "launch beside the GDN chain: from its start, after the "
+                                              "GDN preparation, to the end of its last CTA)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_kind": f"{pk_kind} bf16 dense, burst (the timed region is {total_ms:.0f} ms)",
                 "traffic": tr.get("hybrid_bytes") if tr else None}
@@ -778,9 +778,9 @@ def main():
         "gdn_alone_gbs": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 if gdn_alone_ms else None,
         "gdn_alone_hbm_frac": wk["gdn_bytes"] / (gdn_alone_ms / 1e3) / 1e9 / hbm if gdn_alone_ms else None,
         "note": "the GDN branch runs on a high-priority stream beside one persistent attention "
-                "launch over the SWA and DSWA heads, which leaves the GDN chain its SMs; "
-                "attn_span_ms runs from the step's start to the end of that launch (the "
-                "roofline's duration); attn_alone_* times the attention launch by itself "
+                "launch over the SWA and DSWA heads, which starts after the GDN preparation and "
+                "leaves the GDN chain its SMs; attn_span_ms runs from that launch's start to the "
+                "end of its last CTA (the roofline's duration); attn_alone_* times the attention launch by itself "
                 "against the burst bf16 peak; gdn_alone_* times hlta_gdn_chunk_fwd on the GDN "
                 "heads by themselves (segment scan over all SMs). The GDN HBM fractions use "
                 "the algorithmic q/k/v/o + gate bytes of the GDN heads",

@@ -420,10 +420,12 @@ hlta_status hlta_stream_destroy(hlta_stream_t c);
  * Profiling hook for hlta_hybrid_fwd(_raw) and the streaming steps (measurement, not needed
  * for results). `events` is NULL (off) or an array of 5 cudaEvent_t created by the caller on
  * the current device. While set, each hybrid call or streaming step records events[0] where
- * the branches fork (on the caller's stream, before any branch kernel), events[1] after the
- * SWA kernel (caller's stream), events[2] after the DSWA kernel (on the stream it ran on; with
- * bf16 both follow the one attention launch that serves both branches), events[3] before and
- * events[4] after the GDN kernels (on the GDN stream). The array is
+ * the softmax branches start (on the caller's stream, before their first kernel; with bf16 GDN
+ * heads, after the wait for the GDN chunk preparation), events[1] after the SWA kernel
+ * (caller's stream), events[2] after the DSWA kernel (on the stream it ran on; with bf16 both
+ * branches share one attention launch, and events[2] follows its late CTAs on the GDN stream
+ * when there are any), events[3] before and events[4] after the GDN kernels (on the GDN
+ * stream). The array is
  * copied; the setting is process-wide and stays until changed.
  */
 hlta_status hlta_set_profile_events(void *const *events);

@@ -609,7 +609,6 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
     if (Hg || split_d) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
-    prof_record(0, s);
     // GDN heads on the high-priority auxiliary stream
     if (Hg) {
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
@@ -646,11 +645,12 @@ hlta_status hybrid_fwd_impl(const void *q, const void *k, const void *v, const f
         }
         if (dt == HLTA_BF16) s_fill = ctx->aux;
     }
+    prof_record(0, s);      // the softmax branches start here (bf16: after the preparation)
     if (pair) {
         AttnArgs a1 = clip_attn_args(q, k, v, o, B, H, 0, Hs, T, N, d, w_swa, 1, scale, ctx->err);
         AttnArgs a2 = clip_attn_args(q, k, v, o, B, H, Hs, Hd, T, N, d, w_dswa, r, scale, ctx->err);
         st = run_attn_pair(a2, a1, dt, s, reserve, s_fill);
-        prof_record(2, s);
+        prof_record(2, s_fill ? s_fill : s);        // after the late CTAs, if any
     }
     // DSWA on the second library stream (beside SWA) when both softmax branches are present
     if (Hd && !pair) {
@@ -800,7 +800,6 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
     if (c->Hg || split_d) {
         if ((e = cudaEventRecord(ctx->fork, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
-    prof_record(0, s);
     if (c->Hg) {
         if ((e = cudaStreamWaitEvent(ctx->aux, ctx->fork, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
         prof_record(3, ctx->aux);
@@ -822,12 +821,21 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
             cudaStreamWaitEvent(s, ctx->join, 0);
             return st;
         }
-        if (c->dt == HLTA_BF16 && (e = cudaStreamWaitEvent(s, ctx->prep, 0)) != cudaSuccess) {
-            cudaStreamWaitEvent(s, ctx->join, 0);
-            return cuda_fail(e, "cudaStreamWaitEvent");
-        }
         if (c->dt == HLTA_BF16) s_fill = ctx->aux;
     }
+    // the ring appends run beside the preparation; the attention waits for it (bf16 with GDN
+    // heads). events[0] marks where the attention starts.
+    bool started = false;
+    auto attn_start = [&](cudaStream_t sa) -> hlta_status {
+        if (started) return HLTA_OK;
+        started = true;
+        if (s_fill) {
+            cudaError_t e2 = cudaStreamWaitEvent(sa, ctx->prep, 0);
+            if (e2 != cudaSuccess) return cuda_fail(e2, "cudaStreamWaitEvent");
+        }
+        prof_record(0, sa);
+        return HLTA_OK;
+    };
     struct Branch { int h0, Hbr, slots, w, r; void *rk, *rv; } br[2] = {
         {0, c->Hs, c->slots_s, c->w_swa, 1, c->ks, c->vs},
         {c->Hs, c->Hd, c->slots_d, c->w_dswa, c->r, c->kd, c->vd}};
@@ -856,12 +864,12 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
             pa[1 - bi] = a;                            // launched below, DSWA's units first
             continue;
         }
-        if ((st = run_attn(a, c->dt, s, reserve, s_fill)) != HLTA_OK) break;
+        if ((st = attn_start(s)) != HLTA_OK || (st = run_attn(a, c->dt, s, reserve, s_fill)) != HLTA_OK) break;
         prof_record(bi == 1 ? 2 : 1, s);
     }
-    if (pair && st == HLTA_OK) {
+    if (pair && st == HLTA_OK && (st = attn_start((cudaStream_t)stream)) == HLTA_OK) {
         st = run_attn_pair(pa[0], pa[1], c->dt, (cudaStream_t)stream, reserve, s_fill);
-        prof_record(2, (cudaStream_t)stream);
+        prof_record(2, s_fill ? s_fill : (cudaStream_t)stream);     // after the late CTAs, if any
         prof_record(1, (cudaStream_t)stream);
     }
     // join the other branches after the softmax launches were enqueued, so they overlap
