@@ -27,6 +27,11 @@
  * `stream` is a cudaStream_t (NULL: the legacy default stream). Calls are asynchronous:
  * they validate arguments on the host, enqueue kernels on `stream` and return; they never
  * synchronize the stream.
+ * Concurrency: the bf16 and E4M3 window attention kernels are persistent (one CTA per SM,
+ * taking work from a counter in device memory). Outside the streaming cache, whose steps use
+ * the cache's own counter, the library takes the next of 64 counters per device for each
+ * launch, so at most 64 such launches may be in flight at once. That includes replays of
+ * captured CUDA graphs, whose launches keep the counter they were captured with.
  * Softmax scale: `scale <= 0` selects 1/sqrt(d).
  *
  * Errors: every call returns hlta_status. Argument errors are detected before any launch

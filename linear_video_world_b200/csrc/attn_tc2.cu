@@ -138,7 +138,7 @@ struct Params {
     const float *qs;            // E4M3 query scales: [heads][nqb]
     int nqb;                    // E4M3: query blocks of 128 rows
     int nqt, nunits;            // query tiles of 256 rows per head; units = nqt * B * Hsum
-    int slot;                   // this launch's work counter (g_attn_sched)
+    int *sched;                 // this launch's work counter: [0] next unit, [1] CTAs finished
     int ctas_total;             // CTAs over the launches sharing the counter
     float *lse;
     __nv_bfloat16 *o;
@@ -254,9 +254,10 @@ __device__ __forceinline__ bool is_tap(int fq, int fk, int w, int r)
     return dist >= 0 && dist <= r * (w - 1) && (dist % r) == 0;
 }
 
-// Work counters of the persistent launches, one pair per launch slot: [0] the next unit to
-// take, [1] the CTAs that finished. The last CTA of a launch to finish puts both back to zero
-// for the slot's next launch.
+// Work counters of the persistent launches whose caller passes none, one pair per launch slot,
+// used in turn: [0] the next unit to take, [1] the CTAs that finished. The last CTA of a launch
+// to finish puts both back to zero for the counter's next launch, so a slot serves any launch
+// that starts after the one SCHED_SLOTS launches earlier has finished.
 constexpr int SCHED_SLOTS = 64;
 __device__ int g_attn_sched[SCHED_SLOTS][2];
 
@@ -387,7 +388,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             for (int i = 0; ok; ++i) {
                 const int us = i & 1;
                 if (i >= 2 && !(ok = wait_bar(BAR(LY::B_UEMPTY + us), (uint32_t)((i - 2) >> 1) & 1u))) break;
-                const int u0 = atomicAdd(&g_attn_sched[p.slot][0], 1);
+                const int u0 = atomicAdd(&p.sched[0], 1);
                 const int u = u0 < p.nunits ? u0 : -1;
                 unit_slot[us] = u;
                 mbar_arrive(BAR(LY::B_UFULL + us));
@@ -809,9 +810,9 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     // (of every launch sharing the counter) to arrive leaves the slot at zero for its next use
     if (threadIdx.x == 0) {
         __threadfence();
-        if (atomicAdd(&g_attn_sched[p.slot][1], 1) == p.ctas_total - 1) {
-            atomicExch(&g_attn_sched[p.slot][0], 0);
-            atomicExch(&g_attn_sched[p.slot][1], 0);
+        if (atomicAdd(&p.sched[1], 1) == p.ctas_total - 1) {
+            atomicExch(&p.sched[0], 0);
+            atomicExch(&p.sched[1], 0);
         }
     }
 }
@@ -823,7 +824,7 @@ bool same_launch(const AttnArgs &a, const AttnArgs &b)
 {
     return a.q == b.q && a.o == b.o && a.B == b.B && a.q_Htot == b.q_Htot && a.q_rows == b.q_rows &&
            a.N == b.N && a.d == b.d && a.fq0 == b.fq0 && a.fq0_dev == b.fq0_dev && a.scale == b.scale &&
-           a.err == b.err && a.qs == b.qs && a.lse == b.lse;
+           a.err == b.err && a.qs == b.qs && a.lse == b.lse && a.sched == b.sched;
 }
 
 template <bool F8>
@@ -886,10 +887,16 @@ cudaError_t launch_attn_tc2(const AttnArgs *br, int nbr, int reserve_sms, cudaSt
     if (nunits >= (1L << 30)) return cudaErrorNotSupported;
     p.nqt = (int)nqt;
     p.nunits = (int)nunits;
-    static std::atomic<unsigned> next_slot{0};
-    p.slot = (int)(next_slot.fetch_add(1u) % (unsigned)SCHED_SLOTS);
     int dev = 0, nsm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (a.sched) {
+        p.sched = a.sched;
+    } else {
+        static std::atomic<unsigned> next_slot{0};
+        int *base = nullptr;
+        if ((e = cudaGetSymbolAddress((void **)&base, g_attn_sched)) != cudaSuccess) return e;
+        p.sched = base + 2 * (int)(next_slot.fetch_add(1u) % (unsigned)SCHED_SLOTS);
+    }
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     nsm = std::max(nsm, 1);
     const int ctas = std::max(nsm - std::max(reserve_sms, 0), (nsm + 1) / 2);

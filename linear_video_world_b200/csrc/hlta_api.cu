@@ -299,7 +299,9 @@ struct hlta_stream {
     size_t ws_bytes;
     int frames;               // steps' frames appended, counted on the host per call
     int *fdev;                // the same count on the device: the kernels read it and each step
-                              // advances it in stream order, so a captured step can be replayed
+                              // advances it in stream order, so a captured step can be replayed;
+                              // fdev[2..3] are the cache's own work counter of its attention
+                              // launch (a captured step then shares no counter with other work)
 };
 
 extern "C" {
@@ -742,8 +744,8 @@ hlta_status hlta_stream_create_ex(hlta_stream_t *out, int B, int Hs, int Hd, int
     if (bd && e == cudaSuccess) e = cudaMalloc(&c->vd, bd);
     if (Hg && e == cudaSuccess) e = cudaMalloc((void **)&c->S, (size_t)B * Hg * d * d * sizeof(float));
     if (Hg && e == cudaSuccess) e = cudaMalloc(&c->ws, c->ws_bytes);
-    if (e == cudaSuccess) e = cudaMalloc((void **)&c->fdev, sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(c->fdev, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMalloc((void **)&c->fdev, 4 * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(c->fdev, 0, 4 * sizeof(int));
     if (e == cudaSuccess && Hg) {
         if (S0) e = cudaMemcpy(c->S, S0, (size_t)B * Hg * d * d * sizeof(float), cudaMemcpyDeviceToDevice);
         else e = cudaMemset(c->S, 0, (size_t)B * Hg * d * d * sizeof(float));
@@ -860,6 +862,7 @@ hlta_status hlta_stream_step_frames(hlta_stream_t c, const void *q_new, const vo
         a.kv_Htot = x.Hbr; a.kv_h0 = 0; a.kv_rows = (long)x.slots * c->N; a.kv_slots = x.slots;
         a.N = c->N; a.d = c->d; a.w = x.w; a.r = x.r; a.fq0 = f; a.fq0_dev = c->fdev; a.scale = c->scale;
         a.err = ctx->err;
+        a.sched = c->fdev + 2;
         if (pair) {
             pa[1 - bi] = a;                            // launched below, DSWA's units first
             continue;

@@ -36,6 +36,9 @@ struct AttnArgs {
     // bf16 kernel only: per query row log-sum-exp (natural log) of the scaled scores
     // ([B*q_Htot][q_rows] float32), written when non-null
     float *lse = nullptr;
+    // bf16 / E4M3 kernel: the launch's work counter (two device ints, zero between launches,
+    // used by one launch at a time), or null for one of the library's 64 shared counters
+    int *sched = nullptr;
 };
 
 // Gated delta rule over [B][Htot][L][d] tensors, this branch's heads at h0 .. h0 + Hg.

@@ -320,3 +320,55 @@ def test_hybrid_and_gdn_backward_graph_replay(h):
     for got, ref in zip(replay1, snapshot()):
         assert torch.equal(got, ref)
     del g
+
+
+def test_stream_graph_replay_beside_other_attention(h, orc):
+    """Replays of a captured streaming step run while 70 other window attention launches run
+    on a second stream each time. Those launches cycle through the library's 64 shared work
+    counters; the step's persistent attention uses the cache's own counter, so no launch takes
+    another's units: the replayed frames reproduce the hybrid operator and every side launch
+    reproduces its eager result bit for bit."""
+    wl = hi.Workload("t", B=2, Hs=1, Hd=1, Hg=1, d=128, T=7, N=130, w_swa=3, w_dswa=4, r=2,
+                     chunk=64, dtype="bf16", decay=1.0)
+    x = hi.make_inputs(wl, seed=41)
+    q, k, v, a, b = (dev(x[n]) for n in "qkvab")
+    side_wl = hi.Workload("s", B=1, Hs=0, Hd=2, Hg=0, d=128, T=3, N=300, w_swa=2, w_dswa=2, r=1,
+                          chunk=64, dtype="bf16", decay=1.0)
+    xs = hi.make_inputs(side_wl, seed=42)
+    sq, sk, sv = (dev(xs[n]) for n in "qkv")
+    side_ref = h.swa(sq, sk, sv, side_wl.T, side_wl.N, 2)
+    st = h.Stream(wl.B, wl.Hs, wl.Hd, wl.Hg, wl.N, wl.d, wl.w_swa, wl.w_dswa, wl.r)
+
+    def frame(t, f):
+        return t[:, :, f * wl.N:(f + 1) * wl.N].contiguous()
+
+    outs = [st.step(*(frame(t, 0) for t in (q, k, v, a, b)))]
+    static = [frame(t, 0).clone() for t in (q, k, v, a, b)]
+    so = torch.empty_like(static[0])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        st.step(*static, out=so)
+    side = torch.cuda.Stream()
+    side_outs = []
+    for f in range(1, wl.T):
+        for buf, t in zip(static, (q, k, v, a, b)):
+            buf.copy_(frame(t, f))
+        side.wait_stream(torch.cuda.current_stream())
+        g.replay()
+        with torch.cuda.stream(side):
+            for _ in range(70):
+                side_outs.append(h.swa(sq, sk, sv, side_wl.T, side_wl.N, 2, out=poison_like(sq)))
+        outs.append(so.clone())
+        torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert h.hlta_device_status() == 0
+    for o_side in side_outs:
+        assert torch.equal(o_side, side_ref)
+    o = torch.cat(outs, dim=2)
+    o_ref, S_ref = orc.hybrid(x["q"], x["k"], x["v"], x["a"], x["b"], wl.Hs, wl.Hd, wl.Hg,
+                              wl.T, wl.N, wl.w_swa, wl.w_dswa, wl.r)
+    assert maxabs(o, o_ref) <= TOL
+    assert maxabs(st.state_tensor(), S_ref) <= TOL
+    del g
+    st.close()
