@@ -38,7 +38,9 @@
 // Tensor memory: per sub-tile S (128 columns) and O (128). Shared memory: Q (64 KB), the ring
 // (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
 // O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
-// denominator use the same stale max).
+// denominator use the same stale max). In bf16 one pair in four of a tile's exponentials runs on
+// the FMA pipe (a range-reduced cubic) instead of the exponential unit, which the remaining
+// three keep busy: the unit and the issue slots are then closer to balanced.
 // From one unit to the next: the producer loads the next Q once both issuers' last S of the
 // unit completed; an issuer's first P V of a unit (which overwrites O) waits until its softmax
 // read the previous unit's O; S, P and the ring's barriers keep counting across units. A
@@ -194,6 +196,29 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, fl
         : "=r"(r)
         : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
     return r;
+}
+
+
+// 2^x for a pair of values on the FMA pipe instead of the exponential unit (Cody-Waite range
+// reduction and a polynomial): x + 1.5 * 2^23 rounds x to the nearest integer n in the low
+// mantissa bits, f = x - n lies in [-1/2, 1/2], 2^f is a cubic fitted for minimum relative
+// error on that interval (7.5e-5, below bf16's rounding of P), and n is added to the result's
+// exponent bits. x is clamped below at -125 (masked -inf included) so the exponent stays normal.
+constexpr float EXP2_C0 = 0.9999280571937561f, EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.2426111400127411f, EXP2_C3 = 0.0551716573536396f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x)
+{
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    constexpr float SH = 12582912.f;                            // 1.5 * 2^23
+    const float2 t = fadd2(x, make_float2(SH, SH));
+    const float2 n = fadd2(t, make_float2(-SH, -SH));
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+    float2 q = ffma2(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+    q = ffma2(q, f, make_float2(EXP2_C1, EXP2_C1));
+    q = ffma2(q, f, make_float2(EXP2_C0, EXP2_C0));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c)
@@ -710,9 +735,12 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                  : "memory");
             };
 #pragma unroll
+            // one pair in four on the FMA pipe (it floors 2^x at 2^-125, a masked key's -inf
+            // included: negligible beside the row sum, which is at least 1 once the row has met
+            // a key it attends)
             for (int i = 0; i < 32; ++i) {
                 const float2 x = ffma2(make_float2(__uint_as_float(sa[2 * i]), __uint_as_float(sa[2 * i + 1])), sl2x2, nm2);
-                const float2 pp = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                const float2 pp = ((i & 3) == 3) ? exp2_fma2(x) : make_float2(tc::ex2(x.x), tc::ex2(x.y));
                 ps2[i & 1] = fadd2(ps2[i & 1], pp);
                 pk[i] = tc::pack_bf16(pp.x, pp.y);
             }
@@ -725,7 +753,7 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             for (int i = 32; i < 64; ++i) {
                 const int j = i & 31;
                 const float2 x = ffma2(make_float2(__uint_as_float(sb[2 * j]), __uint_as_float(sb[2 * j + 1])), sl2x2, nm2);
-                const float2 pp = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                const float2 pp = ((i & 3) == 3) ? exp2_fma2(x) : make_float2(tc::ex2(x.x), tc::ex2(x.y));
                 ps2[i & 1] = fadd2(ps2[i & 1], pp);
                 pk[i] = tc::pack_bf16(pp.x, pp.y);
             }
