@@ -38,9 +38,9 @@
 // Tensor memory: per sub-tile S (128 columns) and O (128). Shared memory: Q (64 KB), the ring
 // (96 KB), P per sub-tile ([128 rows][128 keys] bf16, 128-byte swizzle, 64 KB).
 // O is rescaled in TMEM only when a row's max grows by more than 2^8 (exact: numerator and
-// denominator use the same stale max). In bf16 one pair in four of a tile's exponentials runs on
-// the FMA pipe (a range-reduced cubic) instead of the exponential unit, which the remaining
-// three keep busy: the unit and the issue slots are then closer to balanced.
+// denominator use the same stale max). One pair in four of a tile's exponentials runs on the
+// FMA pipe (a range-reduced cubic) instead of the exponential unit, which the remaining three
+// keep busy: the unit and the issue slots are then closer to balanced.
 // From one unit to the next: the producer loads the next Q once both issuers' last S of the
 // unit completed; an issuer's first P V of a unit (which overwrites O) waits until its softmax
 // read the previous unit's O; S, P and the ring's barriers keep counting across units. A
@@ -686,11 +686,13 @@ attn_tc2_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
                                      : "memory");
                     }
                 };
+                // the second pair of every other quad on the FMA pipe (one pair in four; its
+                // floor of 2^-125 rounds to an E4M3 zero)
                 auto quad8 = [&](const uint32_t *sv, int i, float2 scl) {
                     const float2 xa = ffma2(make_float2(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1])), scl, nm2);
                     const float2 xb = ffma2(make_float2(__uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3])), scl, nm2);
                     const float2 pa = make_float2(tc::ex2(xa.x), tc::ex2(xa.y));
-                    const float2 pb = make_float2(tc::ex2(xb.x), tc::ex2(xb.y));
+                    const float2 pb = (i & 1) ? exp2_fma2(xb) : make_float2(tc::ex2(xb.x), tc::ex2(xb.y));
                     ps2[0] = fadd2(ps2[0], pa);
                     ps2[1] = fadd2(ps2[1], pb);
                     return pack_e4m3x4(pa.x, pa.y, pb.x, pb.y);
