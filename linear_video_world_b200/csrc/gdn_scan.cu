@@ -390,8 +390,8 @@ gdn_chain_bf16(const __grid_constant__ ChainMaps maps, const ChainArgs a)
 // (kind::tf32, A from tensor memory); A_p arrives by TMA as the K-major B operand (the segment
 // maps store it transposed, [j][k]); the accumulator is set to B_p first (tcgen05.st), so the
 // product adds onto it. Two column regions of 128 alternate: S_p in one, S_{p+1} built in the
-// other. B_p is written as soon as the previous product completed; S_p is copied out to the
-// start states the replay reads while its product runs. Warps 0-3: thread i owns row i (TMEM lane i); warp 4: TMEM owner, TMA
+// other. Each S_{p+1} is copied out to the start states the replay reads while the next
+// product runs. Warps 0-3: thread i owns row i (TMEM lane i); warp 4: TMEM owner, TMA
 // producer and MMA issuer (one thread).
 // -----------------------------------------------------------------------------------------
 constexpr int COMPOSE_THREADS = 160;
@@ -517,8 +517,7 @@ gdn_compose_tc(const __grid_constant__ CUtensorMap mat, const ChainArgs a)
 #pragma unroll
         for (int j = 0; j < D; ++j) bnext[j] = bmap[(long)j * D];
         for (int mp = 0; mp < nmaps; ++mp) {
-            // B_p into the accumulator columns (they held S_{p-1}, whose product completed):
-            // the product can start as soon as they are written
+            // B_p into the accumulator columns (they held S_{p-1}, whose product completed)
             const uint32_t dcol = tl + (uint32_t)((mp + 1) & 1) * 128u;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -530,19 +529,7 @@ gdn_compose_tc(const __grid_constant__ CUtensorMap mat, const ChainArgs a)
             tc::tmem_wait_st();
             tc::fence_before_sync();
             ptx::mbar_arrive(B_READY);
-            // while the product runs: S_p out to the start states (it is the product's A
-            // operand, read by both), and the next map's row in
-            if (mp >= 1) {
-                const uint32_t scol = tl + (uint32_t)(mp & 1) * 128u;
-                float *dst = sseg + (long)mp * D * D;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(scol + q * 32, v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) dst[(long)(32 * q + e) * D] = __uint_as_float(v[e]);
-                }
-            }
+            // the next map's row loads while the product runs
             if (mp + 1 < nmaps) {
                 const float *bn = bmap + (long)(mp + 1) * D * D;
 #pragma unroll
@@ -550,17 +537,14 @@ gdn_compose_tc(const __grid_constant__ CUtensorMap mat, const ChainArgs a)
             }
             if (!__all_sync(0xffffffffu, wait_bar(D_FULL, (uint32_t)mp & 1u, abort_flag, p.err))) break;
             tc::fence_after_sync();
-            if (mp + 1 == nmaps) {
-                // the last start state, S_{nmaps}
-                const uint32_t scol = tl + (uint32_t)((mp + 1) & 1) * 128u;
-                float *dst = sseg + (long)(mp + 1) * D * D;
+            // S_{p+1} out to the start states (it stays in tensor memory for the next product)
+            float *dst = sseg + (long)(mp + 1) * D * D;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(scol + q * 32, v);
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                tc::tmem_ld32(dcol + q * 32, v);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) dst[(long)(32 * q + e) * D] = __uint_as_float(v[e]);
-                }
+                for (int e = 0; e < 32; ++e) dst[(long)(32 * q + e) * D] = __uint_as_float(v[e]);
             }
         }
     }
