@@ -285,3 +285,50 @@ def test_model_detects_a_planted_protocol_error():
             found = "S overwritten" in str(e) or "phase" in str(e)
             break
     assert found
+
+
+def test_work_counter_shared_by_two_launches():
+    """The persistent launches' work counter: CTAs take units by an atomic ticket until the
+    tickets run past the units, then count themselves finished; the last of all CTAs (of the
+    main launch and of the late CTAs queued behind another kernel, which may start at any
+    time) puts both words back to zero. Every unit is processed exactly once, and the next
+    launch on the counter finds it at zero."""
+    rnd = random.Random(7)
+    counter = [0, 0]
+    for trial in range(300):
+        nunits = rnd.randint(1, 60)
+        grid = rnd.randint(1, 20)
+        late = rnd.randint(0, 8)
+        total = grid + late
+        done = []
+
+        def cta():
+            while True:
+                t = counter[0]
+                counter[0] += 1                     # atomicAdd(&sched[0], 1)
+                yield
+                if t >= nunits:
+                    break
+                done.append(t)
+                for _ in range(rnd.randint(0, 3)):
+                    yield                           # the unit's work
+            last = counter[1] == total - 1          # atomicAdd(&sched[1], 1) == total - 1
+            counter[1] += 1
+            if last:
+                counter[0] = counter[1] = 0
+            yield
+
+        started = [cta() for _ in range(grid)]
+        pending = [cta() for _ in range(late)]
+        alive = list(started)
+        while alive or pending:
+            if pending and (not alive or rnd.random() < 0.1):
+                alive.append(pending.pop())         # a late CTA starts
+                continue
+            a = rnd.choice(alive)
+            try:
+                next(a)
+            except StopIteration:
+                alive.remove(a)
+        assert sorted(done) == list(range(nunits)), trial
+        assert counter == [0, 0], trial
