@@ -19,6 +19,8 @@ it, Q only after the unit's last S completed.
 """
 import random
 
+import pytest
+
 NSLOT = 3
 
 
@@ -58,7 +60,7 @@ class Bar:
         return self.done > phase
 
 
-def simulate(units, seed):
+def simulate(units, seed, NSLOT=NSLOT):
     rnd = random.Random(seed)
     U = len(units)
     items = []                                  # (unit, kind, tile) in ring order
@@ -247,7 +249,8 @@ def simulate(units, seed):
     return False
 
 
-def test_protocol_has_no_deadlock_no_parity_alias_and_no_hazard():
+@pytest.mark.parametrize("nslot", [3, 6])      # the bf16 ring and the E4M3 ring
+def test_protocol_has_no_deadlock_no_parity_alias_and_no_hazard(nslot):
     cases = 0
     for (N, w, r) in [(1560, 3, 1), (1560, 3, 4), (1560, 4, 6), (130, 3, 1), (130, 4, 2),
                       (100, 2, 2), (1, 3, 2), (16, 2, 2), (200, 3, 2), (256, 2, 1)]:
@@ -258,7 +261,7 @@ def test_protocol_has_no_deadlock_no_parity_alias_and_no_hazard():
                 rnd = random.Random(1000 * T + seed)
                 n = rnd.randint(1, min(5, len(walks)))
                 units = [walks[rnd.randrange(len(walks))] for _ in range(n)]
-                assert simulate(units, seed), (N, w, r, T, seed)
+                assert simulate(units, seed, nslot), (N, w, r, T, seed)
                 cases += 1
     assert cases == 240
 
